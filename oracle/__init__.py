@@ -1,0 +1,296 @@
+"""fp64 CPU oracle for Kwai Summary Attention (KSA) -- test infrastructure.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it and
+shares no code with it.  The arithmetic lives in ``ksa_oracle.c`` (plain C,
+fp64); this module only compiles that file, marshals numpy arrays and strings
+together the per-sequence calls of a packed (varlen) batch.
+
+Citations are to "Kwai Summary Attention Technical Report": the augmented
+sequence is section 2.2.1 Eq. (1); visibility is section 2.2.1 (summary rule)
+and section 2.2.2 Eqs. (2)-(3); the attention is Eq. (10); the decode cache is
+section 2.3.1 with Figure 4.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ksa_oracle.c")
+_SO = os.path.join(_HERE, "libksa_oracle.so")
+
+_lib = None
+
+_d = ctypes.POINTER(ctypes.c_double)
+_i64 = ctypes.POINTER(ctypes.c_int64)
+_u8 = ctypes.POINTER(ctypes.c_uint8)
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+
+
+def build(force: bool = False) -> str:
+    """Compile ksa_oracle.c into libksa_oracle.so (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", _SO + ".tmp", _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_SO + ".tmp", _SO)
+    return _SO
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_SO)
+        L.oracle_rope.argtypes = [_I64, _I, _I, _d, _i64, ctypes.c_double, _d]
+        L.oracle_visible.argtypes = [_I64, _I, _I, _I, _I64, _I, _I64]
+        L.oracle_visible.restype = _I
+        L.oracle_aug_len.argtypes = [_I64, _I]
+        L.oracle_aug_len.restype = _I64
+        L.oracle_dense_mask.argtypes = [_I64, _I, _I, _u8]
+        L.oracle_count_pairs.argtypes = [_I64, _I, _I]
+        L.oracle_count_pairs.restype = _I64
+        L.oracle_ksa_attention.argtypes = [_I64, _I, _I, _I, _I, _I, ctypes.c_double,
+                                           _d, _d, _d, _d, _d, _d,
+                                           _I64, _i64, _I64, _i64, _d, _d, _d, _d]
+        L.oracle_cache_slots.argtypes = [_I, _I, _I64]
+        L.oracle_cache_slots.restype = _I64
+        L.oracle_cache_new.argtypes = [_I, _I, _I, _I, _I64]
+        L.oracle_cache_new.restype = ctypes.c_void_p
+        L.oracle_cache_free.argtypes = [ctypes.c_void_p]
+        for nm in ("oracle_cache_k", "oracle_cache_v"):
+            getattr(L, nm).argtypes = [ctypes.c_void_p]
+            getattr(L, nm).restype = _d
+        for nm in ("oracle_cache_n_text", "oracle_cache_m"):
+            getattr(L, nm).argtypes = [ctypes.c_void_p]
+            getattr(L, nm).restype = _I64
+        L.oracle_cache_append_text.argtypes = [ctypes.c_void_p, _d, _d]
+        L.oracle_cache_append_text.restype = _I
+        L.oracle_cache_append_summary.argtypes = [ctypes.c_void_p, _d, _d]
+        L.oracle_cache_append_summary.restype = _I
+        L.oracle_cache_slice.argtypes = [ctypes.c_void_p, _I, _i64, _i64]
+        L.oracle_cache_decode.argtypes = [ctypes.c_void_p, _I, _I, ctypes.c_double, _d, _d, _d]
+        L.oracle_decode_image.argtypes = [_I, _I, _I, _I, _I64, _I64, _I64, _I, _d, _d,
+                                          _I, ctypes.c_double, _d, _d, _d]
+        _lib = L
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a: np.ndarray):
+    if a is None:
+        return None
+    if a.dtype == np.float64:
+        return a.ctypes.data_as(_d)
+    if a.dtype == np.int64:
+        return a.ctypes.data_as(_i64)
+    if a.dtype == np.uint8:
+        return a.ctypes.data_as(_u8)
+    raise TypeError(a.dtype)
+
+
+# --------------------------------------------------------------------------
+# RoPE and positions
+# --------------------------------------------------------------------------
+def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
+    """Rotate-half RoPE in fp64.  x: [rows, heads, d]; pos: [rows]."""
+    x = _f64(x)
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    out = np.empty_like(x)
+    lib().oracle_rope(x.shape[0], x.shape[1], x.shape[2], _p(x), _p(pos), float(theta), _p(out))
+    return out
+
+
+def text_positions(n: int) -> np.ndarray:
+    """Text token t_i of a sequence has position id i (its local index)."""
+    return np.arange(n, dtype=np.int64)
+
+
+def summary_positions(n: int, k: int) -> np.ndarray:
+    """Summary s_j takes the position id of its chunk's last text token, jk+k-1
+    (section 2.2.1, second bullet after Eq. (1))."""
+    m = n // k
+    return np.arange(m, dtype=np.int64) * k + (k - 1)
+
+
+# --------------------------------------------------------------------------
+# Visibility
+# --------------------------------------------------------------------------
+def visible(n: int, k: int, C: int, q_kind: int, q_idx: int, key_kind: int, key_idx: int) -> bool:
+    return bool(lib().oracle_visible(n, k, C, q_kind, q_idx, key_kind, key_idx))
+
+
+def dense_mask(n: int, k: int, C: int) -> np.ndarray:
+    """[L, L] uint8 mask over the augmented sequence of Eq. (1)."""
+    L = int(lib().oracle_aug_len(n, k))
+    out = np.zeros((L, L), dtype=np.uint8)
+    lib().oracle_dense_mask(n, k, C, _p(out))
+    return out
+
+
+# --------------------------------------------------------------------------
+# Prefill attention
+# --------------------------------------------------------------------------
+def ksa_attention(n, k, C, qt, kt, vt, qs, ks, vs, scale=None, tq_idx=None, sq_idx=None):
+    """KSA attention of one sequence on already-RoPE'd fp64 inputs.
+
+    qt [n, Hq, d], kt/vt [n, Hkv, d], qs [m, Hq, d], ks/vs [m, Hkv, d].
+    Returns (ot, lse_t, os, lse_s) for the requested text / summary rows.
+    """
+    qt, kt, vt, qs, ks, vs = (_f64(a) for a in (qt, kt, vt, qs, ks, vs))
+    Hq, d = qt.shape[1], qt.shape[2]
+    Hkv = kt.shape[1]
+    m = n // k
+    assert qs.shape[0] == m and ks.shape[0] == m
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    tq = None if tq_idx is None else np.ascontiguousarray(tq_idx, dtype=np.int64)
+    sq = None if sq_idx is None else np.ascontiguousarray(sq_idx, dtype=np.int64)
+    ntq = n if tq is None else len(tq)
+    nsq = m if sq is None else len(sq)
+    ot = np.zeros((ntq, Hq, d))
+    lt = np.zeros((ntq, Hq))
+    os_ = np.zeros((nsq, Hq, d))
+    ls = np.zeros((nsq, Hq))
+    # empty arrays still need a valid pointer
+    qs_ = qs if m > 0 else np.zeros((1, Hq, d))
+    ks_ = ks if m > 0 else np.zeros((1, Hkv, d))
+    vs_ = vs if m > 0 else np.zeros((1, Hkv, d))
+    lib().oracle_ksa_attention(n, k, C, Hq, Hkv, d, float(scale),
+                               _p(qt), _p(kt), _p(vt), _p(qs_), _p(ks_), _p(vs_),
+                               ntq, _p(tq), nsq, _p(sq),
+                               _p(ot) if ntq else None, _p(lt) if ntq else None,
+                               _p(os_) if nsq else None, _p(ls) if nsq else None)
+    return ot, lt, os_, ls
+
+
+@dataclass
+class SeqResult:
+    text_o: np.ndarray      # [n_rows, Hq, d]
+    text_lse: np.ndarray    # [n_rows, Hq]
+    sum_o: np.ndarray       # [m_rows, Hq, d]
+    sum_lse: np.ndarray     # [m_rows, Hq]
+    text_rows: np.ndarray   # which text indices were computed
+    sum_rows: np.ndarray    # which summary indices were computed
+
+
+def ksa_prefill(seqlens, k, C, qt, kt, vt, qs, ks, vs, theta, scale=None,
+                text_rows=None, sum_rows=None):
+    """The whole prefill path for a packed batch, from un-rotated inputs.
+
+    qt/kt/vt: [sum(n_b), H, d] text tensors packed by sequence;
+    qs/ks/vs: [sum(floor(n_b/k)), H, d] summary tensors packed the same way.
+    RoPE (theta; 0 disables it) is applied per sequence with text position i
+    and summary position jk+k-1, then Eq. (10) under the KSA mask.
+    text_rows / sum_rows: optional per-sequence index arrays to compute.
+    Returns one SeqResult per sequence.
+    """
+    out = []
+    t0 = s0 = 0
+    for b, n in enumerate(seqlens):
+        m = n // k
+        sl_t = slice(t0, t0 + n)
+        sl_s = slice(s0, s0 + m)
+        q1, k1, v1 = _f64(qt[sl_t]), _f64(kt[sl_t]), _f64(vt[sl_t])
+        q2, k2, v2 = _f64(qs[sl_s]), _f64(ks[sl_s]), _f64(vs[sl_s])
+        if theta and theta > 0:
+            pt, ps = text_positions(n), summary_positions(n, k)
+            q1, k1 = rope(q1, pt, theta), rope(k1, pt, theta)
+            if m:
+                q2, k2 = rope(q2, ps, theta), rope(k2, ps, theta)
+        tr = None if text_rows is None else text_rows[b]
+        sr = None if sum_rows is None else sum_rows[b]
+        ot, lt, os_, ls = ksa_attention(n, k, C, q1, k1, v1, q2, k2, v2, scale, tr, sr)
+        out.append(SeqResult(ot, lt, os_, ls,
+                             np.arange(n) if tr is None else np.asarray(tr),
+                             np.arange(m) if sr is None else np.asarray(sr)))
+        t0 += n
+        s0 += m
+    return out
+
+
+# --------------------------------------------------------------------------
+# Decode cache model
+# --------------------------------------------------------------------------
+TEXT, SUMMARY = 0, 1
+
+
+def cache_slots(k: int, C: int, cap: int) -> int:
+    return int(lib().oracle_cache_slots(k, C, cap))
+
+
+class Cache:
+    """One sequence's decode cache under the documented slot map."""
+
+    def __init__(self, k: int, C: int, Hkv: int, d: int, cap: int):
+        self.k, self.C, self.Hkv, self.d, self.cap = k, C, Hkv, d, cap
+        self.S = cache_slots(k, C, cap)
+        self._h = lib().oracle_cache_new(k, C, Hkv, d, cap)
+
+    def __del__(self):
+        if getattr(self, "_h", None):
+            lib().oracle_cache_free(self._h)
+            self._h = None
+
+    @property
+    def n_text(self) -> int:
+        return int(lib().oracle_cache_n_text(self._h))
+
+    @property
+    def m(self) -> int:
+        return int(lib().oracle_cache_m(self._h))
+
+    def K(self) -> np.ndarray:
+        p = lib().oracle_cache_k(self._h)
+        return np.ctypeslib.as_array(p, shape=(self.S, self.Hkv, self.d)).copy()
+
+    def V(self) -> np.ndarray:
+        p = lib().oracle_cache_v(self._h)
+        return np.ctypeslib.as_array(p, shape=(self.S, self.Hkv, self.d)).copy()
+
+    def append_text(self, k_row, v_row) -> int:
+        k_row, v_row = _f64(k_row), _f64(v_row)
+        return int(lib().oracle_cache_append_text(self._h, _p(k_row), _p(v_row)))
+
+    def append_summary(self, k_row, v_row) -> int:
+        k_row, v_row = _f64(k_row), _f64(v_row)
+        return int(lib().oracle_cache_append_summary(self._h, _p(k_row), _p(v_row)))
+
+    def slice(self, kind: int):
+        lo = ctypes.c_int64(0)
+        hi = ctypes.c_int64(0)
+        lib().oracle_cache_slice(self._h, kind, ctypes.byref(lo), ctypes.byref(hi))
+        return int(lo.value), int(hi.value)
+
+    def decode(self, kind: int, q, scale=None):
+        q = _f64(q)
+        Hq = q.shape[0]
+        if scale is None:
+            scale = 1.0 / np.sqrt(self.d)
+        o = np.zeros((Hq, self.d))
+        lse = np.zeros(Hq)
+        lib().oracle_cache_decode(self._h, kind, Hq, float(scale), _p(q), _p(o), _p(lse))
+        return o, lse
+
+
+def decode_image(k, C, cap, n_text, m, kind, K, V, q, scale=None):
+    """Decode against a cache image K/V [S, Hkv, d] (fp64) in the slot map."""
+    K, V, q = _f64(K), _f64(V), _f64(q)
+    S, Hkv, d = K.shape
+    assert S == cache_slots(k, C, cap)
+    Hq = q.shape[0]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.zeros((Hq, d))
+    lse = np.zeros(Hq)
+    lib().oracle_decode_image(k, C, Hkv, d, cap, n_text, m, kind, _p(K), _p(V),
+                              Hq, float(scale), _p(q), _p(o), _p(lse))
+    return o, lse

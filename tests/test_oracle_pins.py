@@ -1,0 +1,331 @@
+"""Pins for the fp64 oracle: each test checks it against something other than
+itself -- a hand-written golden mask, closed forms, a library routine on a
+case where KSA reduces to it, or a second mechanism (the decode cache) that
+the report says encodes the same visibility rule.
+
+Citations: "Kwai Summary Attention Technical Report" (sections 2.2.1, 2.2.2,
+2.3.1, Eqs. (1)-(3), (9), (10), Figures 3 and 4, Tables 1 and 3).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+# ---------------------------------------------------------------------------
+# Visibility
+# ---------------------------------------------------------------------------
+def test_fig3_toy_mask_matches_hand_written_golden():
+    """Figure 3's toy (k=4, C=1, 16 text tokens): the predicate's dense mask
+    equals the mask written out by hand from the rules of sections 2.2.1-2.2.2."""
+    rows = []
+    with open(os.path.join(GOLDEN, "fig3_toy_mask_k4_C1.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            bits = line.split()[0]
+            rows.append([int(ch) for ch in bits])
+    golden = np.array(rows, dtype=np.uint8)
+    assert golden.shape == (20, 20)
+    np.testing.assert_array_equal(oracle.dense_mask(16, 4, 1), golden)
+
+
+def _closed_form_pairs(n, k, C):
+    """Per-head visible pairs summed chunk by chunk: a text row at offset r of
+    chunk c sees min(c, C)*k + r + 1 window keys and max(0, c - C) summaries;
+    each complete chunk's summary sees k + 1 keys."""
+    tot = 0
+    nchunks = (n + k - 1) // k
+    for c in range(nchunks):
+        rows = min(k, n - c * k)
+        tot += rows * min(c, C) * k + rows * (rows + 1) // 2 + rows * max(0, c - C)
+    return tot + (n // k) * (k + 1)
+
+
+@pytest.mark.parametrize("n,k,C,expect", [
+    (256, 8, 2, 8824),            # the small prefill case (2 q / 1 kv heads, d 64)
+    (32768, 8, 8, 69109792),      # the Qwen3-4B-shaped prefill case
+])
+def test_pair_counts_closed_form(n, k, C, expect):
+    assert _closed_form_pairs(n, k, C) == expect
+    assert lib_count(n, k, C) == expect
+
+
+def lib_count(n, k, C):
+    return int(oracle.lib().oracle_count_pairs(n, k, C))
+
+
+def test_pair_counts_varlen_closed_form():
+    lens = (131072, 65536, 16384, 4000)
+    assert sum(lib_count(n, 8, 16) for n in lens) == 1385339220
+    lens = (131072, 65536, 16384, 4003)
+    assert sum(lib_count(n, 8, 16) for n in lens) == sum(_closed_form_pairs(n, 8, 16) for n in lens)
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("C", [0, 1, 2, 100])
+def test_mask_sum_equals_enumerated_keys(k, C):
+    """Brute force over every (query, key) pair of the augmented sequence
+    agrees with the key-set enumeration the attention uses, for all n <= 40."""
+    for n in range(0, 41):
+        mask = oracle.dense_mask(n, k, C)
+        assert int(mask.sum()) == lib_count(n, k, C) == _closed_form_pairs(n, k, C)
+
+
+def test_mask_structure_properties():
+    """Properties the report states in words: a summary sees exactly its own
+    chunk (k text) and itself; no text token sees an in-window summary; every
+    past chunk is either fully visible as text or visible via its summary
+    (section 2.2.2, 'clean partition' under Figure 4)."""
+    for k, C in [(4, 1), (3, 2), (8, 0), (2, 5)]:
+        n = 7 * k + (k // 2)
+        m = n // k
+        for i in range(n):
+            c = i // k
+            for cc in range(c):  # every fully past chunk
+                text_vis = [oracle.visible(n, k, C, 0, i, 0, p) for p in range(cc * k, cc * k + k)]
+                sum_vis = oracle.visible(n, k, C, 0, i, 1, cc)
+                assert all(text_vis) != sum_vis or (all(text_vis) and not sum_vis)
+                assert all(text_vis) or not any(text_vis)  # never a partial chunk
+                assert all(text_vis) ^ sum_vis               # exactly one route
+            # nothing of the future
+            for p in range(i + 1, n):
+                assert not oracle.visible(n, k, C, 0, i, 0, p)
+            for j in range(c, m):
+                assert not oracle.visible(n, k, C, 0, i, 1, j)
+        for j in range(m):
+            seen = [p for p in range(n) if oracle.visible(n, k, C, 1, j, 0, p)]
+            assert seen == list(range(j * k, j * k + k))
+            assert [jj for jj in range(m) if oracle.visible(n, k, C, 1, j, 1, jj)] == [j]
+
+
+# ---------------------------------------------------------------------------
+# Attention values
+# ---------------------------------------------------------------------------
+def _sdpa(q, k, v, causal, scale):
+    """torch fp64 SDPA on [H, L, d] (GQA already expanded)."""
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(k)[None], torch.from_numpy(v)[None],
+        is_causal=causal, scale=scale)[0].numpy()
+
+
+@pytest.mark.parametrize("n,k,Hq,Hkv,d", [(37, 4, 4, 2, 16), (64, 8, 2, 1, 32), (21, 1, 3, 3, 8)])
+def test_text_rows_reduce_to_causal_attention(n, k, Hq, Hkv, d):
+    """With C >= n/k no chunk ever leaves the window, so Eq. (3) has no
+    summaries and the text rows are causal full attention over the text
+    (the teacher of Eq. (9) with a causal mask)."""
+    rng = np.random.default_rng(1)
+    m = n // k
+    qt, kt, vt = _rand(rng, n, Hq, d), _rand(rng, n, Hkv, d), _rand(rng, n, Hkv, d)
+    qs, ks, vs = _rand(rng, m, Hq, d), _rand(rng, m, Hkv, d), _rand(rng, m, Hkv, d)
+    scale = 1 / math.sqrt(d)
+    ot, lt, _, _ = oracle.ksa_attention(n, k, n // k + 1, qt, kt, vt, qs, ks, vs)
+    G = Hq // Hkv
+    ref = _sdpa(qt.transpose(1, 0, 2), np.repeat(kt, G, 1).transpose(1, 0, 2),
+                np.repeat(vt, G, 1).transpose(1, 0, 2), True, scale).transpose(1, 0, 2)
+    np.testing.assert_allclose(ot, ref, rtol=0, atol=1e-12)
+    # LSE: log-sum-exp of the causal scores
+    s = np.einsum("ihd,jhd->hij", qt, np.repeat(kt, G, 1)) * scale
+    s = np.where(np.tril(np.ones((n, n), bool))[None], s, -np.inf)
+    np.testing.assert_allclose(lt, torch.logsumexp(torch.from_numpy(s), -1).numpy().T, atol=1e-12)
+
+
+def test_summary_rows_are_softmax_over_own_chunk():
+    """s_j attends to t_{jk}..t_{jk+k-1} and s_j (k+1 keys): plain SDPA on
+    that slice (section 2.2.1 summary rule, with the self key of Figure 4c)."""
+    rng = np.random.default_rng(2)
+    n, k, C, Hq, Hkv, d = 43, 5, 1, 4, 2, 16
+    m = n // k
+    qt, kt, vt = _rand(rng, n, Hq, d), _rand(rng, n, Hkv, d), _rand(rng, n, Hkv, d)
+    qs, ks, vs = _rand(rng, m, Hq, d), _rand(rng, m, Hkv, d), _rand(rng, m, Hkv, d)
+    _, _, os_, ls = oracle.ksa_attention(n, k, C, qt, kt, vt, qs, ks, vs)
+    G = Hq // Hkv
+    for j in range(m):
+        keys = np.concatenate([kt[j * k:(j + 1) * k], ks[j:j + 1]], 0)
+        vals = np.concatenate([vt[j * k:(j + 1) * k], vs[j:j + 1]], 0)
+        keys, vals = np.repeat(keys, G, 1), np.repeat(vals, G, 1)
+        ref = _sdpa(qs[j][:, None], keys.transpose(1, 0, 2), vals.transpose(1, 0, 2), False,
+                    1 / math.sqrt(d))[:, 0]
+        np.testing.assert_allclose(os_[j], ref, atol=1e-12)
+
+
+@pytest.mark.parametrize("k,C", [(4, 1), (3, 2), (1, 0), (8, 0), (2, 3)])
+def test_one_hot_values_reveal_the_visible_set(k, C):
+    """With q = 0 the softmax is uniform over the visible keys, and with a
+    one-hot value per key the output is 1/count exactly on the keys the
+    dense predicate marks.  Pins the enumeration in the attention against
+    the brute-force mask, both directions."""
+    n = 6 * k + (k - 1 if k > 1 else 0)
+    m = n // k
+    L = n + m
+    mask = oracle.dense_mask(n, k, C)
+    d = L
+    # one-hot V: key with augmented index a carries e_a
+    text_aug = np.array([i + i // k for i in range(n)])
+    sum_aug = np.array([j * (k + 1) + k for j in range(m)])
+    vt = np.zeros((n, 1, d)); vt[np.arange(n), 0, text_aug] = 1
+    vs = np.zeros((m, 1, d)); vs[np.arange(m), 0, sum_aug] = 1
+    z_t, z_s = np.zeros((n, 1, d)), np.zeros((m, 1, d))
+    ot, lt, os_, ls = oracle.ksa_attention(n, k, C, z_t, z_t, vt, z_s, z_s, vs)
+    for i in range(n):
+        row = mask[text_aug[i]]
+        np.testing.assert_allclose(ot[i, 0], row / row.sum(), atol=1e-15)
+        assert abs(lt[i, 0] - math.log(row.sum())) < 1e-12
+    for j in range(m):
+        row = mask[sum_aug[j]]
+        np.testing.assert_allclose(os_[j, 0], row / row.sum(), atol=1e-15)
+        assert abs(ls[j, 0] - math.log(k + 1)) < 1e-12
+
+
+def test_single_visible_key_returns_its_value():
+    """t_0 sees only itself: its output is v_0 whatever q and k are."""
+    rng = np.random.default_rng(3)
+    n, k, C, d = 9, 4, 1, 8
+    qt, kt, vt = _rand(rng, n, 1, d), _rand(rng, n, 1, d), _rand(rng, n, 1, d)
+    m = n // k
+    qs, ks, vs = _rand(rng, m, 1, d), _rand(rng, m, 1, d), _rand(rng, m, 1, d)
+    ot, lt, _, _ = oracle.ksa_attention(n, k, C, qt, kt, vt, qs, ks, vs)
+    np.testing.assert_allclose(ot[0, 0], vt[0, 0], atol=1e-15)
+    assert abs(lt[0, 0] - qt[0, 0] @ kt[0, 0] / math.sqrt(d)) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# RoPE
+# ---------------------------------------------------------------------------
+def test_rope_identity_at_position_zero_and_norm_preserving():
+    rng = np.random.default_rng(4)
+    x = _rand(rng, 5, 3, 16)
+    out0 = oracle.rope(x, np.zeros(5, np.int64), 1e6)
+    np.testing.assert_array_equal(out0, x)
+    out = oracle.rope(x, np.array([1, 7, 100, 4095, 1 << 20]), 1e6)
+    h = 8
+    np.testing.assert_allclose(out[..., :h] ** 2 + out[..., h:] ** 2,
+                               x[..., :h] ** 2 + x[..., h:] ** 2, rtol=1e-13)
+
+
+def test_rope_frequency_schedule_closed_form():
+    """theta = 1e6 (Table 3), d = 128: pair r turns by pos * theta^(-2r/d).
+    Pair 0 turns by pos radians; pair d/4 = 32 turns by pos * 1e-3 radians,
+    so position 1000 turns it by exactly 1 radian; rotate-half pairs element
+    r with element r + d/2."""
+    d = 128
+    x = np.zeros((1, 1, d))
+    x[0, 0, 0] = 1.0
+    x[0, 0, 32] = 1.0
+    out = oracle.rope(x, np.array([1000]), 1e6)[0, 0]
+    assert abs(out[0] - math.cos(1000.0)) < 1e-12 and abs(out[64] - math.sin(1000.0)) < 1e-12
+    assert abs(out[32] - math.cos(1.0)) < 1e-12 and abs(out[96] - math.sin(1.0)) < 1e-12
+    assert np.count_nonzero(np.abs(out) > 1e-15) == 4
+
+
+def test_rope_scores_depend_only_on_relative_position():
+    rng = np.random.default_rng(5)
+    d = 32
+    q, k = _rand(rng, 1, 1, d), _rand(rng, 1, 1, d)
+    def score(pq, pk):
+        return float(oracle.rope(q, np.array([pq]), 1e6)[0, 0] @ oracle.rope(k, np.array([pk]), 1e6)[0, 0])
+    assert abs(score(10, 3) - score(1010, 1003)) < 1e-10
+    assert abs(score(70000, 5) - score(69995, 0)) < 1e-9
+
+
+def test_summary_position_is_last_text_position_of_its_chunk():
+    assert list(oracle.summary_positions(19, 4)) == [3, 7, 11, 15]
+    assert list(oracle.summary_positions(8, 8)) == [7]
+
+
+# ---------------------------------------------------------------------------
+# Decode cache model (section 2.3.1, Figure 4)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("k,C", [(4, 2), (3, 1), (8, 0), (2, 4), (1, 3)])
+def test_cache_decode_equals_prefill_rows(k, C):
+    """Decode step t over the single contiguous slice equals row t of the
+    masked prefill (Eq. (3) enumeration) -- two different mechanisms that the
+    report says encode the same rule ('the cache layout itself inherently
+    encodes the visibility rule').  Covers ring wrap-around (m > C) and the
+    summary steps."""
+    rng = np.random.default_rng(10 + k * 7 + C)
+    Hq, Hkv, d = 4, 2, 8
+    n = 11 * k + (k // 2)
+    m = n // k
+    qt, kt, vt = _rand(rng, n, Hq, d), _rand(rng, n, Hkv, d), _rand(rng, n, Hkv, d)
+    qs, ks, vs = _rand(rng, m, Hq, d), _rand(rng, m, Hkv, d), _rand(rng, m, Hkv, d)
+    ot, lt, os_, ls = oracle.ksa_attention(n, k, C, qt, kt, vt, qs, ks, vs)
+    cache = oracle.Cache(k, C, Hkv, d, cap=m)
+    for i in range(n):
+        assert cache.append_text(kt[i], vt[i]) == 0
+        lo, hi = cache.slice(oracle.TEXT)
+        assert 0 <= lo < hi <= cache.S
+        o, l = cache.decode(oracle.TEXT, qt[i])
+        np.testing.assert_allclose(o, ot[i], atol=1e-12)
+        np.testing.assert_allclose(l, lt[i], atol=1e-12)
+        if (i + 1) % k == 0:
+            j = (i + 1) // k - 1
+            assert cache.append_text(kt[i], vt[i]) == -1      # chunk full: summary first
+            assert cache.append_summary(ks[j], vs[j]) == 0
+            o, l = cache.decode(oracle.SUMMARY, qs[j])
+            np.testing.assert_allclose(o, os_[j], atol=1e-12)
+            np.testing.assert_allclose(l, ls[j], atol=1e-12)
+    assert cache.n_text == n and cache.m == m
+
+
+def test_cache_slot_map_contents():
+    """The documented slot map, checked slot by slot after a run that wraps
+    the ring: scratch = newest summary, summaries in order from slot
+    1+k+C*k, ring block c % C holds chunk c (block copy, reversed order),
+    current chunk right-aligned against the ring."""
+    k, C, Hkv, d = 3, 2, 1, 2
+    n = 5 * k + 2
+    m = n // k
+    tok = np.arange(n, dtype=np.float64)
+    cache = oracle.Cache(k, C, Hkv, d, cap=m + 1)
+    for i in range(n):
+        cache.append_text(np.full((Hkv, d), tok[i]), np.full((Hkv, d), -tok[i]))
+        if (i + 1) % k == 0:
+            j = (i + 1) // k - 1
+            cache.append_summary(np.full((Hkv, d), 1000.0 + j), np.full((Hkv, d), -1000.0 - j))
+    K = cache.K()[:, 0, 0]
+    assert K[0] == 1000 + (m - 1)
+    for j in range(m):
+        assert K[1 + k + C * k + j] == 1000 + j
+    for c in range(m - C, m):
+        b = c % C
+        for r in range(k):
+            assert K[1 + k + b * k + (k - 1 - r)] == c * k + r
+    f = n - m * k
+    for r in range(f):
+        assert K[k - r] == m * k + r
+    lo, hi = cache.slice(oracle.TEXT)
+    assert (lo, hi) == (k - f + 1, 1 + k + C * k + (m - C))
+
+
+def test_cache_capacity_and_order_errors():
+    cache = oracle.Cache(2, 1, 1, 2, cap=1)
+    row = np.ones((1, 2))
+    assert cache.append_summary(row, row) == -1  # chunk not complete
+    cache.append_text(row, row); cache.append_text(row, row)
+    assert cache.append_summary(row, row) == 0
+    cache.append_text(row, row); cache.append_text(row, row)
+    assert cache.append_summary(row, row) == -3  # buffer full
+
+
+def test_table1_cache_ratios():
+    """Table 1: with k = 8 the KSA cache grows at 1/k of full attention; with
+    GQA (g = 8 of h = 128 heads) that is 1/k * g/h = 0.78125% of MHA.  The
+    cache's slot count per sequence is 1 + k + C*k + n/k, so the ratio tends
+    to 1/k as n grows."""
+    k, C = 8, 8
+    n = 1 << 24
+    slots = oracle.cache_slots(k, C, n // k)
+    assert abs(slots / n - 1 / k) < 1e-4
+    h, g = 128, 8
+    assert abs(slots * g / (n * h) - 0.0078125) < 1e-6

@@ -1,0 +1,383 @@
+"""Benchmark of the KSA hot path on B200.
+
+One step = one pass of the whole path over synthetic inputs already in HBM:
+  prefill  (Qwen3-4B layer shape: 1 x 32768 text tokens, 32 q / 8 kv heads,
+           d 128, k 8, w 8, N(0,1)*0.5 bf16, RoPE theta 1e6, fp32 LSE):
+           ksa_interleave_rope + ksa_prefill_fwd;
+  decode   (64 sequences x 131072 prior text tokens: 16384 summaries, full
+           64-token ring, open-chunk fill uniform 0..7; 32 q / 8 kv heads,
+           d 128, k 8, w 8): ksa_cache_append (TEXT) + ksa_decode.
+Reported: prefill TFLOP/s on useful (visible) pairs over the ksa_prefill_fwd
+time (`value`), decode GB/s over the bytes of the KV slices read, each as a
+fraction of the measured B200 peak.  Inputs exceed L2 (126 MB) on both legs.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ksa|reference]
+For N > 1 launch with torchrun: each rank runs its own replica (independent
+batches, no collective: weak scaling), timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+# workloads
+PF = dict(seqlens=[32768], k=8, w=8, Hq=32, Hkv=8, d=128, scale=0.5, seed=1, theta=1e6)
+DC = dict(B=64, m=16384, k=8, w=8, Hq=32, Hkv=8, d=128, seed=3, theta=1e6)
+
+
+def useful_pairs(seqlens, k, w):
+    """Visible (query, key) pairs per head (closed form of Eqs. (2)-(3))."""
+    tot = 0
+    for n in seqlens:
+        i = np.arange(n, dtype=np.int64)
+        c = i // k
+        m = n // k
+        tot += int(((i - np.maximum(c - w, 0) * k + 1) + np.clip(c - w, 0, m)).sum()) + m * (k + 1)
+    return tot
+
+
+def text_pairs(seqlens, k, w):
+    return useful_pairs(seqlens, k, w) - sum((n // k) * (k + 1) for n in seqlens)
+
+
+def decode_slice_rows(m, k, w, fills):
+    """Cache rows one TEXT step reads per (sequence, kv head): open chunk
+    (f+1) + ring min(m,w)*k + far summaries max(0, m-w)."""
+    return np.asarray(fills) + 1 + min(m, w) * k + max(0, m - w)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait()
+            self.f.close()
+
+    def summary(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    import torch.distributed as dist
+    if n_gpus > 1 or "RANK" in os.environ:
+        local = int(os.environ.get("LOCAL_RANK", 0))
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+        return dist.get_rank(), dist.get_world_size(), local
+    torch.cuda.set_device(0)
+    return 0, 1, 0
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# oracle arm (CPU)
+# ---------------------------------------------------------------------------
+def oracle_sample(sample_rows: int, seed: int = 1):
+    """Time the fp64 oracle on a bounded, deterministic sample of the prefill
+    workload's text rows (all 32 heads each) and return (TFLOP/s, cores, rows)."""
+    import oracle
+    import torch
+    from kv_cache_compression_ksa_b200.inputs import prefill_inputs
+    n, k, w = PF["seqlens"][0], PF["k"], PF["w"]
+    x = prefill_inputs(PF["seqlens"], k, PF["Hq"], PF["Hkv"], PF["d"], seed=PF["seed"], scale=PF["scale"])
+    f64 = lambda t: t.double().numpy()
+    rows = np.linspace(0, n - 1, sample_rows).astype(np.int64)
+    qt, kt, vt, qs, ks, vs = (f64(t) for t in (x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum, x.v_sum))
+    pt, ps = oracle.text_positions(n), oracle.summary_positions(n, k)
+    qt, kt = oracle.rope(qt, pt, PF["theta"]), oracle.rope(kt, pt, PF["theta"])
+    qs, ks = oracle.rope(qs, ps, PF["theta"]), oracle.rope(ks, ps, PF["theta"])
+    t0 = time.perf_counter()
+    oracle.ksa_attention(n, k, w, qt, kt, vt, qs, ks, vs, tq_idx=rows, sq_idx=np.zeros(0, np.int64))
+    dt = time.perf_counter() - t0
+    c = rows // k
+    keys = (rows - np.maximum(c - w, 0) * k + 1) + np.clip(c - w, 0, n // k)
+    flops = float(keys.sum()) * PF["Hq"] * 4 * PF["d"]
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return flops / dt / 1e12, cores, len(rows), dt
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    t_total = 0.0
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, cores, nrows, dt = oracle_sample(512)
+        if i >= args.warmup:
+            vals.append(v)
+            t_total += dt
+    v = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": "KSA prefill TFLOP/s (useful pairs)", "value": v, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_total / max(args.steps, 1) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill 1x32768 text tokens, 32q/8kv heads, d128, k8, w8 (sampled rows)"},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{nrows} evenly spaced text rows x 32 heads of the 32768-token prefill"},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------------------
+# KSA arm (GPU)
+# ---------------------------------------------------------------------------
+def run_ksa(args, rank, world, local):
+    import torch
+    from kv_cache_compression_ksa_b200 import _lib as L
+    from kv_cache_compression_ksa_b200 import api, build
+    from kv_cache_compression_ksa_b200.inputs import fill_normal_, prefill_inputs, uniform_ints
+
+    if rank == 0:
+        build.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    hbm_peak, tc_peak, tc_sus, peak_src = load_peaks()
+
+    # ---- prefill inputs (HBM resident) ----
+    sl, k, w, Hq, Hkv, d = PF["seqlens"], PF["k"], PF["w"], PF["Hq"], PF["Hkv"], PF["d"]
+    x = prefill_inputs(sl, k, Hq, Hkv, d, seed=PF["seed"] + 100 * rank, scale=PF["scale"], device=dev)
+    p = L.make_params(k, w, Hq, Hkv, d, 0.0, PF["theta"])
+    nt, ns = sum(sl), sum(n // k for n in sl)
+    rows = L.ksa_aug_rows(p, sl)
+    qa = torch.empty(rows, Hq, d, dtype=torch.bfloat16, device=dev)
+    ka = torch.empty(rows, Hkv, d, dtype=torch.bfloat16, device=dev)
+    va = torch.empty(rows, Hkv, d, dtype=torch.bfloat16, device=dev)
+    oa = torch.empty(rows, Hq, d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(rows, Hq, dtype=torch.float32, device=dev)
+    ws = torch.empty(L.ksa_prefill_workspace_size(p, len(sl), nt), dtype=torch.uint8, device=dev)
+    pf_flops = useful_pairs(sl, k, w) * Hq * 4 * d
+    pf_text_flops = text_pairs(sl, k, w) * Hq * 4 * d
+
+    # ---- decode cache (HBM resident) ----
+    B, m = DC["B"], DC["m"]
+    pd = L.make_params(DC["k"], DC["w"], DC["Hq"], DC["Hkv"], DC["d"], 0.0, DC["theta"])
+    cache = api.DecodeCache(pd, B, cap=m + 64, device=dev)
+    fill_normal_(cache.k, 1000 + rank)
+    fill_normal_(cache.v, 2000 + rank)
+    fills = uniform_ints(B, 0, DC["k"] - 1, seed=DC["seed"]).numpy()
+    state0 = torch.zeros(B, 4, dtype=torch.int32)
+    state0[:, 0] = torch.as_tensor(m * DC["k"] + fills, dtype=torch.int32)
+    state0[:, 1] = m
+    state0 = state0.to(dev)
+    gen = torch.Generator(device=dev).manual_seed(5 + rank)
+    kn = torch.randn(B, DC["Hkv"], DC["d"], generator=gen, device=dev).to(torch.bfloat16)
+    vn = torch.randn(B, DC["Hkv"], DC["d"], generator=gen, device=dev).to(torch.bfloat16)
+    qd = torch.randn(B, DC["Hq"], DC["d"], generator=gen, device=dev).to(torch.bfloat16)
+    kind = torch.zeros(B, dtype=torch.int8, device=dev)
+    max_text = m * DC["k"] + DC["k"]
+    dws = cache.workspace(max_text)
+    od = torch.empty(B, DC["Hq"], DC["d"], dtype=torch.bfloat16, device=dev)
+    lsed = torch.empty(B, DC["Hq"], dtype=torch.float32, device=dev)
+    slice_rows = decode_slice_rows(m, DC["k"], DC["w"], fills)
+    dec_bytes = float(slice_rows.sum()) * DC["Hkv"] * DC["d"] * 2 * 2  # K and V, bf16
+
+    st = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+
+    def step(times):
+        cache.state.copy_(state0)  # same step every iteration (one TEXT append + decode)
+        ev[0].record(st)
+        L.ksa_interleave_rope(p, x.cu_seqlens, nt, ns, rows, x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum,
+                              x.v_sum, qa, ka, va, ws)
+        ev[1].record(st)
+        L.ksa_prefill_fwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, ws)
+        ev[2].record(st)
+        L.ksa_cache_append(pd, cache.desc, kind, kn, vn)
+        ev[3].record(st)
+        L.ksa_decode(pd, cache.desc, kind, qd, od, lsed, max_text, dws)
+        ev[4].record(st)
+        if times is not None:
+            torch.cuda.synchronize()
+            times.append([ev[i].elapsed_time(ev[i + 1]) for i in range(4)])
+
+    for _ in range(args.warmup):
+        step(None)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    times = []
+    with ClockSampler(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(st)
+        for _ in range(args.steps):
+            step(times)
+        t_end.record(st)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = t_start.elapsed_time(t_end)
+    tarr = np.asarray(times)  # [steps, 4] ms: rope, prefill, append, decode
+    rope_ms, pf_ms, app_ms, dec_ms = (float(np.mean(tarr[:, i])) for i in range(4))
+    pf_ms_max = max_over_ranks(pf_ms, world)
+    dec_ms_max = max_over_ranks(dec_ms, world)
+    step_ms = max_over_ranks(float(np.sum(tarr, axis=1).mean()), world)
+
+    value = world * pf_flops / (pf_ms_max * 1e-3) / 1e12
+    dec_gbs = world * dec_bytes / (dec_ms_max * 1e-3) / 1e9
+    kern_tflops = pf_text_flops / (pf_ms * 1e-3) / 1e12
+
+    # ---- e2e through the public API: pinned host inputs -> device -> result ----
+    host = [t.cpu().pin_memory() for t in (x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum, x.v_sum)]
+    cu_h = x.cu_seqlens.cpu().pin_memory()
+    out_h = torch.empty(rows, Hq, d, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host) + cu_h.numel() * 4
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        dv = [t.to(dev, non_blocking=True) for t in host]
+        cu_d = cu_h.to(dev, non_blocking=True)
+        out = api.prefill(p, sl, cu_d, *dv, want_lse=False)
+        out_h.copy_(out.o_aug, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    e2e_val = world * pf_flops / (e2e_ms * 1e-3) / 1e12
+
+    clocks = clk.summary()
+    if rank == 0:
+        line = {
+            "metric": "KSA prefill TFLOP/s (useful pairs) & decode KV GB/s",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": "prefill 1x32768 text tokens (Qwen3-4B layer: 32q/8kv heads, d128), k8, w8, "
+                            "N(0,1)*0.5 bf16, RoPE 1e6, fp32 LSE; + decode 64 seqs x 131072 prior tokens",
+                "global_batch": world, "seq_len": sl[0], "parallelism": f"replicas x{world}",
+                "l2": "inputs larger than L2 (prefill q_aug 302 MB; decode slice 4.3 GB)",
+                "useful_prefill_tflop": pf_flops / 1e12, "decode_slice_gb": dec_bytes / 1e9,
+            },
+            "prefill": {"ms": pf_ms, "rope_interleave_ms": rope_ms, "tflops": value / world,
+                        "frac_of_bf16_peak": (value / world) / tc_peak},
+            "decode": {"ms": dec_ms, "append_ms": app_ms, "gbs": dec_gbs / world,
+                       "frac_of_hbm_peak": (dec_gbs / world) / hbm_peak, "batch": B, "summaries": m},
+            "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                         "frac": kern_tflops / tc_peak, "traffic": None,
+                         "kernel": "prefill_kernel<128> (text rows; time of the ksa_prefill_fwd call)",
+                         "peak_source": f"{peak_src} burst bf16", "peak_sustained": tc_sus},
+            "roofline_decode": {"bound": "hbm", "achieved": dec_gbs / world, "peak": hbm_peak, "unit": "GB/s",
+                                "frac": (dec_gbs / world) / hbm_peak, "traffic": None,
+                                "kernel": "decode_split_kernel<128,4> + combine (time of ksa_decode)"},
+            "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h), "ms": e2e_ms},
+            "gpu_launches": args.steps * 8,
+            "clocks": clocks,
+            "timed_region_ms": total_ms,
+        }
+        if world == 1:
+            v, cores, nrows, dt = oracle_sample(args.cpu_rows)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                    "sample": f"{nrows} evenly spaced text rows x 32 heads of the "
+                                              f"32768-token prefill ({dt:.1f} s)"}
+        print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ksa", choices=["ksa", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=2048)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", 0))
+        world = int(os.environ.get("WORLD_SIZE", 1))
+        run_reference(args, rank, world)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ksa(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,202 @@
+/*
+ * ksa.h -- C ABI of the B200 (sm_100a) Kwai Summary Attention hot path.
+ *
+ * What is computed ("Kwai Summary Attention Technical Report"):
+ *   - the augmented sequence: after every k text tokens comes one summary
+ *     token s_j (section 2.2.1, Eq. (1));
+ *   - a summary token attends to the k text tokens of its own chunk and to
+ *     itself; its RoPE position is that of its chunk's last text token
+ *     (section 2.2.1, rules after Eq. (1); Figure 4c for the self key);
+ *   - a text token t_i attends causally to the text of chunks
+ *     floor(i/k)-w .. floor(i/k) (Sliding Chunk Attention, Eq. (2)) and to
+ *     the summaries s_0 .. s_{floor(i/k)-w-1} of the chunks that have left
+ *     that window (Eq. (3)); in-window summaries are not attended
+ *     (section 2.2.2);
+ *   - softmax(Q K^T * scale + M_KSA) V with scale = 1/sqrt(d) (Eq. (10));
+ *   - decode reads one contiguous slice of a cache made of a scratch slot,
+ *     the current chunk (filled right to left), a ring of w sliding chunks
+ *     and an append-only summary buffer (section 2.3.1, Figure 4 (a)-(e)).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *     contiguous; "bf16" is IEEE bfloat16 (2 bytes).  Base pointers must be
+ *     16-byte aligned.
+ *   - The library allocates no device or host memory and never synchronises
+ *     the stream inside a compute call; all work is enqueued on `stream`
+ *     (cudaStream_t passed as void*, NULL = legacy default stream).
+ *   - Errors found on the host (bad sizes, null pointers, small workspace,
+ *     unsupported shapes) are returned before anything is launched.  Errors
+ *     found on the device (inconsistent cu_seqlens, cache order violations,
+ *     a full summary buffer, a pipeline wait that ran out) never trap: the
+ *     kernel records a KSA_ERR_* code in a device error word and skips the
+ *     affected work.  ksa_get_device_error() reads and clears such a word.
+ *   - Supported: head_dim 64 or 128; num_q_heads % num_kv_heads == 0;
+ *     k >= 1; w >= 0; (num_q_heads/num_kv_heads) * k <= 128 for prefill.
+ */
+#ifndef KSA_H
+#define KSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KSA_API __attribute__((visibility("default")))
+#else
+#define KSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Shape and method parameters shared by all calls. */
+typedef struct ksa_params {
+    int32_t k;            /* chunk size: text tokens per chunk (>= 1)           */
+    int32_t w;            /* sliding chunk number C of Eqs. (2)-(3) (>= 0)      */
+    int32_t num_q_heads;  /* Hq                                                 */
+    int32_t num_kv_heads; /* Hkv; q head h reads kv head h / (Hq/Hkv)           */
+    int32_t head_dim;     /* d: 64 or 128                                       */
+    float scale;          /* softmax scale; 0 selects 1/sqrt(d) (Eq. (10))      */
+    double rope_theta;    /* RoPE base (Table 3 uses 1e6); <= 0 disables RoPE   */
+} ksa_params;
+
+/* Status codes. */
+enum {
+    KSA_OK = 0,
+    KSA_ERR_INVALID = -1,     /* bad argument (null pointer, negative size ...)  */
+    KSA_ERR_UNSUPPORTED = -2, /* valid but not implemented (e.g. head_dim 96)   */
+    KSA_ERR_CAPACITY = -3,    /* summary buffer full / output too small          */
+    KSA_ERR_CUDA = -4,        /* a CUDA runtime or driver call failed            */
+    KSA_ERR_TIMEOUT = -5,     /* a bounded device-side wait gave up              */
+    KSA_ERR_WORKSPACE = -6,   /* workspace smaller than the *_workspace_size()   */
+    KSA_ERR_STATE = -7        /* decode-cache order violated (see ksa_cache_append) */
+};
+
+/* Per-sequence step kinds for the decode calls. */
+enum { KSA_TEXT = 0, KSA_SUMMARY = 1, KSA_SKIP = 2 };
+
+/* ------------------------------------------------------------------------
+ * Augmented layout (prefill).
+ *
+ * Each sequence b (n_b text tokens, cu_seqlens[b+1]-cu_seqlens[b]) owns
+ * nc_b = ceil(n_b / k) whole chunks of k+1 rows, in the order of Eq. (1):
+ * rows k*... t_{jk} .. t_{jk+k-1}, s_j.  Sequence b starts at row
+ * (k+1) * sum_{b'<b} nc_{b'}.  A trailing partial chunk (n_b % k != 0) has
+ * no summary (the report assumes k | n); its unused text rows and its
+ * summary row are padding, written as zeros by ksa_interleave_rope and left
+ * unspecified in the attention output.  Total rows = ksa_aug_rows().
+ * Summary inputs are packed per sequence: sequence b contributes
+ * floor(n_b / k) summary rows.
+ * ------------------------------------------------------------------------ */
+
+/* Rows of the augmented layout for host-side sequence lengths
+ * seqlens_host[0 .. batch-1].  Returns -1 on invalid input. */
+KSA_API int64_t ksa_aug_rows(const ksa_params *p, int32_t batch, const int32_t *seqlens_host);
+
+/* Workspace bytes needed by ksa_interleave_rope / ksa_prefill_fwd for a
+ * batch of `batch` sequences (holds the per-sequence offsets and the tile
+ * list the kernels derive from cu_seqlens on the device). */
+KSA_API size_t ksa_prefill_workspace_size(const ksa_params *p, int32_t batch, int64_t total_text);
+
+/* RoPE + interleave (Eq. (1); RoPE positions of section 2.2.1).
+ *
+ * q_text [total_text, Hq, d], k_text/v_text [total_text, Hkv, d]: bf16 text
+ *   projections, packed by sequence along cu_seqlens (device int32 [batch+1],
+ *   cu_seqlens[0] = 0, non-decreasing, cu_seqlens[batch] = total_text).
+ * q_sum [total_sum, Hq, d], k_sum/v_sum [total_sum, Hkv, d]: bf16 summary
+ *   projections, total_sum = sum_b floor(n_b / k), packed the same way.
+ * q_aug [aug_rows, Hq, d], k_aug/v_aug [aug_rows, Hkv, d]: bf16 outputs in
+ *   the augmented layout; aug_rows = ksa_aug_rows(...).
+ * Q and K of text t_i are rotated at position i (local to its sequence),
+ * those of s_j at position jk+k-1 (rotate-half pairs (r, r+d/2), angle
+ * pos * theta^(-2r/d), computed in fp64); V is copied.  Padding rows are
+ * zeroed.  dev_err: device int32 error word (may be NULL: the workspace's
+ * own word is used).  An inconsistent cu_seqlens sets KSA_ERR_INVALID there
+ * and writes nothing. */
+KSA_API int ksa_interleave_rope(const ksa_params *p, int32_t batch, const int32_t *cu_seqlens,
+                        int64_t total_text, int64_t total_sum, int64_t aug_rows,
+                        const void *q_text, const void *k_text, const void *v_text,
+                        const void *q_sum, const void *k_sum, const void *v_sum,
+                        void *q_aug, void *k_aug, void *v_aug,
+                        void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                        void *stream);
+
+/* KSA prefill forward (Eqs. (2), (3), (10); block-sparse kernel of
+ * section 2.3).  q_aug/k_aug/v_aug: the augmented layout (bf16, rotated).
+ * o_aug [aug_rows, Hq, d] bf16: attention output of every real row (text
+ * and summary); lse [aug_rows, Hq] fp32 natural-log sum of exp of the
+ * scaled scores, or NULL to skip it.  Padding rows of o_aug/lse are not
+ * written.  Text rows run on the tcgen05 tensor cores, skipping every key
+ * tile the rule masks out entirely; summary rows (k+1 keys each) run on
+ * CUDA cores. */
+KSA_API int ksa_prefill_fwd(const ksa_params *p, int32_t batch, const int32_t *cu_seqlens,
+                    int64_t total_text, int64_t aug_rows,
+                    const void *q_aug, const void *k_aug, const void *v_aug,
+                    void *o_aug, float *lse,
+                    void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                    void *stream);
+
+/* ------------------------------------------------------------------------
+ * Decode cache (section 2.3.1, Figure 4).
+ *
+ * k, v: [batch, Hkv, slots, d] bf16, slots = ksa_cache_slots(p, cap).
+ * Slot map of one (sequence, kv head):
+ *   0                          scratch: the newest summary's own K/V (4c)
+ *   1 .. k                     current chunk, token r at slot k - r (4b)
+ *   k+1+b*k .. k+(b+1)*k       ring block b = chunk index mod w (4d)
+ *   1 + k + w*k + j            summary s_j, append-only (4e)
+ * state: device int32 [batch, 4] = {n_text, m, 0, err}: text tokens and
+ * summaries appended so far, and the sequence's last device error.  A
+ * fresh cache is all-zero state.  f = n_text - m*k tokens sit in the open
+ * chunk; f == k means it waits for its summary.
+ * ------------------------------------------------------------------------ */
+typedef struct ksa_cache {
+    void *k;
+    void *v;
+    int32_t *state;
+    int32_t batch;
+    int64_t cap_summaries;
+} ksa_cache;
+
+/* 1 + k + w*k + cap_summaries, or -1 on invalid input. */
+KSA_API int64_t ksa_cache_slots(const ksa_params *p, int64_t cap_summaries);
+
+/* Append one token per sequence.  kind: device int8 [batch] of KSA_TEXT,
+ * KSA_SUMMARY or KSA_SKIP.  k_new, v_new: [batch, Hkv, d] bf16, NOT
+ * rotated: K is rotated here at the token's position (text: n_text;
+ * summary: n_text - 1, its chunk's last text token) unless RoPE is off.
+ *   TEXT    (needs f < k): K/V into slot k - f; n_text += 1.       (4b)
+ *   SUMMARY (needs f == k): K/V into slot 0 (4c); slots 1..k copied over
+ *           ring block m mod w (4d); K/V into slot 1+k+w*k+m (4e); m += 1.
+ * A violated precondition sets state[b].err = KSA_ERR_STATE, a full
+ * summary buffer KSA_ERR_CAPACITY; that sequence is left unchanged. */
+KSA_API int ksa_cache_append(const ksa_params *p, const ksa_cache *cache, const int8_t *kind,
+                     const void *k_new, const void *v_new, void *stream);
+
+/* Workspace bytes for ksa_decode when no sequence has more than max_text
+ * text tokens. */
+KSA_API size_t ksa_decode_workspace_size(const ksa_params *p, int32_t batch, int64_t max_text);
+
+/* One decode step per sequence, after that step's ksa_cache_append.
+ * q: [batch, Hq, d] bf16, NOT rotated (rotated here at position n_text-1).
+ * TEXT reads slots [k-f+1, 1+k+min(m,w)*k+max(0,m-w)) with f = n_text-m*k;
+ * SUMMARY reads slots [0, k+1); SKIP writes nothing.  Each is one
+ * contiguous slice.  o: [batch, Hq, d] bf16; lse: [batch, Hq] fp32 or NULL.
+ * max_text bounds n_text over the batch (it sizes the split-K grid and
+ * must match the workspace query). */
+KSA_API int ksa_decode(const ksa_params *p, const ksa_cache *cache, const int8_t *kind, const void *q,
+               void *o, float *lse, int64_t max_text,
+               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronise `stream`, return the device error word (KSA_OK if clear) and
+ * reset it to KSA_OK.  dev_err: device int32. */
+KSA_API int ksa_get_device_error(int32_t *dev_err, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+KSA_API const char *ksa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KSA_H */

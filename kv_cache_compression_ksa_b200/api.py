@@ -1,0 +1,82 @@
+"""Tensor-level convenience calls over the C ABI (allocation of outputs and
+workspaces with torch; every computation runs in libksa.so).
+
+prefill(...)      RoPE + interleave + KSA prefill attention for a packed batch
+DecodeCache       the contiguous decode cache plus append / decode steps
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib as L
+
+
+@dataclass
+class PrefillOut:
+    o_aug: torch.Tensor        # [aug_rows, Hq, d] bf16
+    lse: torch.Tensor | None   # [aug_rows, Hq] fp32
+    q_aug: torch.Tensor
+    k_aug: torch.Tensor
+    v_aug: torch.Tensor
+
+
+def aug_rows(p: L.ksa_params, seqlens) -> int:
+    return L.ksa_aug_rows(p, seqlens)
+
+
+def prefill(p: L.ksa_params, seqlens, cu_seqlens, q_text, k_text, v_text, q_sum, k_sum, v_sum,
+            want_lse: bool = True, stream=None) -> PrefillOut:
+    """Run ksa_interleave_rope then ksa_prefill_fwd on device tensors.
+
+    seqlens: host list of text lengths (sizes the outputs); cu_seqlens: the
+    same as a device int32 prefix array [B+1]."""
+    dev = q_text.device
+    B = len(seqlens)
+    total_text = int(sum(seqlens))
+    total_sum = int(sum(n // p.k for n in seqlens))
+    rows = aug_rows(p, seqlens)
+    Hq, Hkv, d = p.num_q_heads, p.num_kv_heads, p.head_dim
+    q_aug = torch.empty(rows, Hq, d, dtype=torch.bfloat16, device=dev)
+    k_aug = torch.empty(rows, Hkv, d, dtype=torch.bfloat16, device=dev)
+    v_aug = torch.empty(rows, Hkv, d, dtype=torch.bfloat16, device=dev)
+    o_aug = torch.empty(rows, Hq, d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(rows, Hq, dtype=torch.float32, device=dev) if want_lse else None
+    ws = torch.empty(L.ksa_prefill_workspace_size(p, B, total_text), dtype=torch.uint8, device=dev)
+    L.ksa_interleave_rope(p, cu_seqlens, total_text, total_sum, rows, q_text, k_text, v_text,
+                          q_sum, k_sum, v_sum, q_aug, k_aug, v_aug, ws, stream=stream)
+    L.ksa_prefill_fwd(p, cu_seqlens, total_text, rows, q_aug, k_aug, v_aug, o_aug, lse, ws, stream=stream)
+    return PrefillOut(o_aug, lse, q_aug, k_aug, v_aug)
+
+
+class DecodeCache:
+    """K/V cache [B, Hkv, slots, d] bf16 + state [B, 4] int32 (slot map of
+    the report's Figure 4; see include/ksa.h)."""
+
+    def __init__(self, p: L.ksa_params, batch: int, cap_summaries: int, device="cuda"):
+        self.p = p
+        self.batch = batch
+        self.cap = cap_summaries
+        self.slots = L.ksa_cache_slots(p, cap_summaries)
+        shape = (batch, p.num_kv_heads, self.slots, p.head_dim)
+        self.k = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        self.v = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        self.state = torch.zeros(batch, 4, dtype=torch.int32, device=device)
+        self.desc = L.make_cache(self.k, self.v, self.state, cap_summaries)
+
+    def append(self, kind, k_new, v_new, stream=None):
+        L.ksa_cache_append(self.p, self.desc, kind, k_new, v_new, stream=stream)
+
+    def workspace(self, max_text: int):
+        n = L.ksa_decode_workspace_size(self.p, self.batch, max_text)
+        return torch.empty(max(n, 16), dtype=torch.uint8, device=self.k.device)
+
+    def decode(self, kind, q, max_text, ws=None, want_lse=True, stream=None):
+        p = self.p
+        o = torch.empty(self.batch, p.num_q_heads, p.head_dim, dtype=torch.bfloat16, device=q.device)
+        lse = torch.empty(self.batch, p.num_q_heads, dtype=torch.float32, device=q.device) if want_lse else None
+        if ws is None:
+            ws = self.workspace(max_text)
+        L.ksa_decode(p, self.desc, kind, q, o, lse, max_text, ws, stream=stream)
+        return o, lse

@@ -1,0 +1,210 @@
+// ksa_api.cu -- the extern "C" entry points of libksa.so: argument checks on
+// the host, then the kernels of rope_interleave.cu, prefill_sm100.cu and
+// cache_decode.cu.  Nothing here allocates device or host memory.
+#include <math.h>
+#include <string.h>
+
+#include "ksa_internal.cuh"
+
+namespace ksa {
+
+int sm_count()
+{
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by every call.
+static int check_params(const ksa_params *p)
+{
+    if (!p) return KSA_ERR_INVALID;
+    if (p->k < 1 || p->w < 0 || p->num_q_heads < 1 || p->num_kv_heads < 1) return KSA_ERR_INVALID;
+    if (p->num_q_heads % p->num_kv_heads != 0) return KSA_ERR_INVALID;
+    if (!(p->scale >= 0.f) || isinf(p->scale)) return KSA_ERR_INVALID;
+    if (isnan(p->rope_theta)) return KSA_ERR_INVALID;
+    if (p->head_dim != 64 && p->head_dim != 128) return KSA_ERR_UNSUPPORTED;
+    if (p->num_q_heads / p->num_kv_heads > 8) return KSA_ERR_UNSUPPORTED;
+    return KSA_OK;
+}
+
+static int check_prefill_shape(const ksa_params *p)
+{
+    int G = p->num_q_heads / p->num_kv_heads;
+    if (G * p->k > 128 || p->k > 64) return KSA_ERR_UNSUPPORTED;
+    return KSA_OK;
+}
+
+}  // namespace ksa
+
+using namespace ksa;
+
+extern "C" {
+
+const char *ksa_status_string(int s)
+{
+    switch (s) {
+    case KSA_OK: return "ok";
+    case KSA_ERR_INVALID: return "invalid argument";
+    case KSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case KSA_ERR_CAPACITY: return "capacity exceeded";
+    case KSA_ERR_CUDA: return "CUDA error";
+    case KSA_ERR_TIMEOUT: return "device wait timed out";
+    case KSA_ERR_WORKSPACE: return "workspace too small";
+    case KSA_ERR_STATE: return "decode cache order violated";
+    default: return "unknown status";
+    }
+}
+
+int64_t ksa_aug_rows(const ksa_params *p, int32_t batch, const int32_t *seqlens_host)
+{
+    if (check_params(p) != KSA_OK || batch < 0 || (batch > 0 && !seqlens_host)) return -1;
+    int64_t chunks = 0;
+    for (int b = 0; b < batch; ++b) {
+        if (seqlens_host[b] < 0) return -1;
+        chunks += (seqlens_host[b] + p->k - 1) / p->k;
+    }
+    return chunks * (p->k + 1);
+}
+
+size_t ksa_prefill_workspace_size(const ksa_params *p, int32_t batch, int64_t total_text)
+{
+    (void)p; (void)total_text;
+    if (batch < 0) return 0;
+    return plan_bytes(batch);
+}
+
+static int check_prefill_common(const ksa_params *p, int32_t batch, const int32_t *cu, int64_t total_text,
+                                int64_t aug_rows, void *ws, size_t ws_bytes)
+{
+    int rc = check_params(p);
+    if (rc != KSA_OK) return rc;
+    if (batch < 1 || !cu || total_text < 0 || aug_rows < 0 || aug_rows % (p->k + 1) != 0) return KSA_ERR_INVALID;
+    if (total_text > INT32_MAX || aug_rows / (p->k + 1) > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+    if (aug_rows < total_text) return KSA_ERR_INVALID;
+    if (!ws) return KSA_ERR_INVALID;
+    if (ws_bytes < plan_bytes(batch)) return KSA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return KSA_ERR_INVALID;
+    return KSA_OK;
+}
+
+int ksa_interleave_rope(const ksa_params *p, int32_t batch, const int32_t *cu_seqlens, int64_t total_text,
+                        int64_t total_sum, int64_t aug_rows, const void *q_text, const void *k_text,
+                        const void *v_text, const void *q_sum, const void *k_sum, const void *v_sum, void *q_aug,
+                        void *k_aug, void *v_aug, void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                        void *stream)
+{
+    int rc = check_prefill_common(p, batch, cu_seqlens, total_text, aug_rows, workspace, workspace_bytes);
+    if (rc != KSA_OK) return rc;
+    if (total_sum < 0 || total_sum > total_text / p->k) return KSA_ERR_INVALID;
+    if (total_text > 0 && (!q_text || !k_text || !v_text)) return KSA_ERR_INVALID;
+    if (total_sum > 0 && (!q_sum || !k_sum || !v_sum)) return KSA_ERR_INVALID;
+    if (aug_rows > 0 && (!q_aug || !k_aug || !v_aug)) return KSA_ERR_INVALID;
+    const void *ptrs[] = {q_text, k_text, v_text, q_sum, k_sum, v_sum, q_aug, k_aug, v_aug};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return KSA_ERR_INVALID;
+    if (reinterpret_cast<uintptr_t>(dev_err) & 3u) return KSA_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    Plan pl = plan_view(workspace, batch);
+    int32_t *err = dev_err ? dev_err : pl.err;
+    rc = launch_plan(p, batch, cu_seqlens, total_text, total_sum, aug_rows, pl, err, 0, st);
+    if (rc != KSA_OK) return rc;
+    return launch_interleave_rope(p, batch, cu_seqlens, aug_rows, q_text, k_text, v_text, q_sum, k_sum, v_sum,
+                                  q_aug, k_aug, v_aug, pl, err, st);
+}
+
+int ksa_prefill_fwd(const ksa_params *p, int32_t batch, const int32_t *cu_seqlens, int64_t total_text,
+                    int64_t aug_rows, const void *q_aug, const void *k_aug, const void *v_aug, void *o_aug,
+                    float *lse, void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream)
+{
+    int rc = check_prefill_common(p, batch, cu_seqlens, total_text, aug_rows, workspace, workspace_bytes);
+    if (rc != KSA_OK) return rc;
+    rc = check_prefill_shape(p);
+    if (rc != KSA_OK) return rc;
+    if (aug_rows > 0 && (!q_aug || !k_aug || !v_aug || !o_aug)) return KSA_ERR_INVALID;
+    const void *ptrs[] = {q_aug, k_aug, v_aug, o_aug};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return KSA_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(dev_err) & 3u))
+        return KSA_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    Plan pl = plan_view(workspace, batch);
+    int32_t *err = dev_err ? dev_err : pl.err;
+    // the summary count is implied by cu_seqlens here: -1 skips that check
+    rc = launch_plan(p, batch, cu_seqlens, total_text, -1, aug_rows, pl, err, prefill_unit_chunks(p), st);
+    if (rc != KSA_OK) return rc;
+    return launch_prefill(p, batch, cu_seqlens, total_text, aug_rows, q_aug, k_aug, v_aug, o_aug, lse, pl, err, st);
+}
+
+int64_t ksa_cache_slots(const ksa_params *p, int64_t cap_summaries)
+{
+    if (!p || p->k < 1 || p->w < 0 || cap_summaries < 0) return -1;
+    return 1 + (int64_t)p->k + (int64_t)p->w * p->k + cap_summaries;
+}
+
+static int check_cache(const ksa_params *p, const ksa_cache *c, const int8_t *kind)
+{
+    int rc = check_params(p);
+    if (rc != KSA_OK) return rc;
+    if (!c || c->batch < 0 || c->cap_summaries < 0) return KSA_ERR_INVALID;
+    if (c->batch > 0 && (!c->k || !c->v || !c->state || !kind)) return KSA_ERR_INVALID;
+    if (c->batch > 0 && (!aligned16(c->k) || !aligned16(c->v))) return KSA_ERR_INVALID;
+    if (c->batch > 65535) return KSA_ERR_UNSUPPORTED;
+    // int32 state: text positions must stay representable
+    if ((c->cap_summaries + 1) * (int64_t)p->k > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+    return KSA_OK;
+}
+
+int ksa_cache_append(const ksa_params *p, const ksa_cache *cache, const int8_t *kind, const void *k_new,
+                     const void *v_new, void *stream)
+{
+    int rc = check_cache(p, cache, kind);
+    if (rc != KSA_OK) return rc;
+    if (cache->batch > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))) return KSA_ERR_INVALID;
+    return launch_cache_append(p, cache, kind, k_new, v_new, (cudaStream_t)stream);
+}
+
+size_t ksa_decode_workspace_size(const ksa_params *p, int32_t batch, int64_t max_text)
+{
+    if (check_params(p) != KSA_OK || batch < 0 || max_text < 0) return 0;
+    return decode_workspace_bytes(p, batch, max_text);
+}
+
+int ksa_decode(const ksa_params *p, const ksa_cache *cache, const int8_t *kind, const void *q, void *o, float *lse,
+               int64_t max_text, void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_cache(p, cache, kind);
+    if (rc != KSA_OK) return rc;
+    if (max_text < 0) return KSA_ERR_INVALID;
+    if (cache->batch > 0) {
+        if (!q || !o || !workspace || !aligned16(q) || !aligned16(o) || !aligned16(workspace))
+            return KSA_ERR_INVALID;
+        if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return KSA_ERR_INVALID;
+    }
+    return launch_decode(p, cache, kind, q, o, lse, max_text, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+int ksa_get_device_error(int32_t *dev_err, void *stream)
+{
+    if (!dev_err) return KSA_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, dev_err, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return KSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KSA_ERR_CUDA;
+    if (v != KSA_OK) {
+        if (cudaMemsetAsync(dev_err, 0, sizeof(int32_t), st) != cudaSuccess) return KSA_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return KSA_ERR_CUDA;
+    }
+    return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,97 @@
+// ksa_internal.cuh -- declarations shared by the .cu files of libksa.so.
+//
+// Kwai Summary Attention Technical Report: section 2.2 (the rule), section
+// 2.3 (the block-sparse prefill kernel and the contiguous decode cache).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/ksa.h"
+
+namespace ksa {
+
+// Per-batch offsets derived on the device from cu_seqlens by plan_kernel and
+// kept at the head of the prefill workspace.
+struct Plan {
+    int32_t *err;        // error word used when the caller passes none
+    int32_t *chunk_off;  // [B+1] first chunk of each sequence (ceil(n/k) each)
+    int32_t *sum_off;    // [B+1] first summary input row (floor(n/k) each)
+    int32_t *tile_off;   // [B+1] first prefill work unit of each sequence
+};
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+// Workspace layout of the prefill calls.
+inline size_t plan_bytes(int batch)
+{
+    return align_up(16) + 3 * align_up(sizeof(int32_t) * (size_t)(batch + 1));
+}
+inline Plan plan_view(void *ws, int batch)
+{
+    char *p = static_cast<char *>(ws);
+    Plan pl;
+    pl.err = reinterpret_cast<int32_t *>(p);
+    p += align_up(16);
+    size_t a = align_up(sizeof(int32_t) * (size_t)(batch + 1));
+    pl.chunk_off = reinterpret_cast<int32_t *>(p); p += a;
+    pl.sum_off = reinterpret_cast<int32_t *>(p); p += a;
+    pl.tile_off = reinterpret_cast<int32_t *>(p);
+    return pl;
+}
+
+// Chunks covered by one prefill work unit (all rows of a unit share one kv
+// head); set by the prefill launcher, 0 for calls that need no tile list.
+int prefill_unit_chunks(const ksa_params *p);
+
+// Enqueue the plan kernel: validates cu_seqlens against the host totals and
+// fills the offsets.  unit_chunks > 0 also fills tile_off.
+int launch_plan(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text,
+                int64_t total_sum, int64_t aug_rows, const Plan &pl, int32_t *err,
+                int unit_chunks, cudaStream_t st);
+
+int launch_interleave_rope(const ksa_params *p, int batch, const int32_t *cu, int64_t aug_rows,
+                           const void *qt, const void *kt, const void *vt, const void *qs,
+                           const void *ks, const void *vs, void *qa, void *ka, void *va,
+                           const Plan &pl, int32_t *err, cudaStream_t st);
+
+int launch_prefill(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text,
+                   int64_t aug_rows, const void *qa, const void *ka, const void *va, void *oa,
+                   float *lse, const Plan &pl, int32_t *err, cudaStream_t st);
+
+int launch_cache_append(const ksa_params *p, const ksa_cache *c, const int8_t *kind,
+                        const void *k_new, const void *v_new, cudaStream_t st);
+
+size_t decode_workspace_bytes(const ksa_params *p, int batch, int64_t max_text);
+int launch_decode(const ksa_params *p, const ksa_cache *c, const int8_t *kind, const void *q,
+                  void *o, float *lse, int64_t max_text, void *ws, size_t ws_bytes,
+                  cudaStream_t st);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Record the first error only.
+__device__ __forceinline__ void set_error(int32_t *err, int code)
+{
+    if (err) atomicCAS(err, 0, code);
+}
+
+// RoPE angle of pair r (of d/2) at position pos, reduced to [-pi, pi] in
+// fp64 so that positions up to millions keep full fp32 accuracy in sincos.
+__device__ __forceinline__ void rope_cos_sin(double pos, int r, int d, double log2_theta,
+                                             float *c, float *s)
+{
+    // inv_freq = theta^(-2r/d)
+    double inv_freq = exp2(-2.0 * (double)r / (double)d * log2_theta);
+    double ang = pos * inv_freq;
+    const double two_pi = 6.283185307179586476925286766559;
+    ang = ang - two_pi * rint(ang / two_pi);
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    *c = (float)cd;
+    *s = (float)sd;
+}
+
+}  // namespace ksa

@@ -1,0 +1,88 @@
+"""The C-ABI library loads, exports every symbol include/ksa.h declares, and
+rejects bad arguments on the host before launching anything (no GPU needed:
+these calls return before their first CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ksa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from kv_cache_compression_ksa_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*KSA_API\s+(?:const\s+)?[a-z_0-9]+\s*\*?\s*(ksa_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("ksa_interleave_rope", "ksa_prefill_fwd", "ksa_cache_append", "ksa_decode"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), f"libksa.so does not export {n}"
+
+
+def test_host_side_validation(lib):
+    from kv_cache_compression_ksa_b200 import _lib as L
+    p = L.make_params(8, 8, 32, 8, 128)
+    # sizes
+    assert L.ksa_cache_slots(p, 16384) == 1 + 8 + 64 + 16384
+    assert L.ksa_aug_rows(p, [32768]) == 36864
+    assert L.ksa_aug_rows(p, [131072, 65536, 16384, 4000]) == 244116
+    assert L.ksa_aug_rows(p, [4003]) == 501 * 9
+    assert L.ksa_prefill_workspace_size(p, 4, 1000) >= 16
+    # bad parameters: returned before any launch
+    nul = ctypes.c_void_p(0)
+    bad = L.make_params(0, 8, 32, 8, 128)
+    rc = lib.ksa_prefill_fwd(ctypes.byref(bad), 1, 8, 8, 9, nul, nul, nul, nul, nul, 8, 64, nul, nul)
+    assert rc == L.KSA_ERR_INVALID
+    odd = L.make_params(8, 8, 32, 8, 96)
+    rc = lib.ksa_prefill_fwd(ctypes.byref(odd), 1, 8, 8, 9, nul, nul, nul, nul, nul, 8, 64, nul, nul)
+    assert rc == L.KSA_ERR_UNSUPPORTED
+    gqa = L.make_params(8, 8, 30, 8, 128)  # 30 % 8 != 0
+    rc = lib.ksa_prefill_fwd(ctypes.byref(gqa), 1, 8, 8, 9, nul, nul, nul, nul, nul, 8, 64, nul, nul)
+    assert rc == L.KSA_ERR_INVALID
+    # null cu_seqlens
+    rc = lib.ksa_prefill_fwd(ctypes.byref(p), 1, nul, 8, 9, nul, nul, nul, nul, nul, 16, 4096, nul, nul)
+    assert rc == L.KSA_ERR_INVALID
+    # aug_rows not a multiple of k+1
+    rc = lib.ksa_prefill_fwd(ctypes.byref(p), 1, 16, 8, 10, 16, 16, 16, 16, nul, 16, 4096, nul, nul)
+    assert rc == L.KSA_ERR_INVALID
+    # workspace too small
+    rc = lib.ksa_prefill_fwd(ctypes.byref(p), 1, 16, 8, 9, 16, 16, 16, 16, nul, 16, 8, nul, nul)
+    assert rc == L.KSA_ERR_WORKSPACE
+    # G * k > 128 is unsupported for prefill
+    big = L.make_params(64, 1, 8, 2, 128)
+    rc = lib.ksa_prefill_fwd(ctypes.byref(big), 1, 16, 64, 65, 16, 16, 16, 16, nul, 16, 4096, nul, nul)
+    assert rc == L.KSA_ERR_UNSUPPORTED
+    # decode: null cache pointers
+    cache = L.ksa_cache(None, None, None, 4, 10)
+    rc = lib.ksa_decode(ctypes.byref(p), ctypes.byref(cache), 16, 16, 16, nul, 100, 16, 1 << 20, nul)
+    assert rc == L.KSA_ERR_INVALID
+    rc = lib.ksa_cache_append(ctypes.byref(p), ctypes.byref(cache), 16, 16, 16, nul)
+    assert rc == L.KSA_ERR_INVALID
+    assert lib.ksa_get_device_error(nul, nul) == L.KSA_ERR_INVALID
+    assert L.status_string(L.KSA_ERR_STATE) == "decode cache order violated"
+
+
+def test_binding_refuses_host_tensors(lib):
+    import torch
+    from kv_cache_compression_ksa_b200 import _lib as L
+    with pytest.raises(ValueError):
+        L._ptr(torch.zeros(4))

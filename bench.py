@@ -211,6 +211,8 @@ def run_ksa(args, rank, world, local):
 
     # ---- prefill inputs (HBM resident) ----
     sl, k, w, Hq, Hkv, d = PF["seqlens"], PF["k"], PF["w"], PF["Hq"], PF["Hkv"], PF["d"]
+    if args.only == "decode":
+        sl = [256]
     x = prefill_inputs(sl, k, Hq, Hkv, d, seed=PF["seed"] + 100 * rank, scale=PF["scale"], device=dev)
     p = L.make_params(k, w, Hq, Hkv, d, 0.0, PF["theta"])
     nt, ns = sum(sl), sum(n // k for n in sl)
@@ -224,8 +226,10 @@ def run_ksa(args, rank, world, local):
     pf_flops = useful_pairs(sl, k, w) * Hq * 4 * d
     pf_text_flops = text_pairs(sl, k, w) * Hq * 4 * d
 
+    do_pf = args.only in (None, "prefill")
+    do_dc = args.only in (None, "decode")
     # ---- decode cache (HBM resident) ----
-    B, m = DC["B"], DC["m"]
+    B, m = (args.decode_batch if do_dc else 1), (DC["m"] if do_dc else 16)
     pd = L.make_params(DC["k"], DC["w"], DC["Hq"], DC["Hkv"], DC["d"], 0.0, DC["theta"])
     cache = api.DecodeCache(pd, B, cap=m + 64, device=dev)
     fill_normal_(cache.k, 1000 + rank)
@@ -253,14 +257,18 @@ def run_ksa(args, rank, world, local):
     def step(times):
         cache.state.copy_(state0)  # same step every iteration (one TEXT append + decode)
         ev[0].record(st)
-        L.ksa_interleave_rope(p, x.cu_seqlens, nt, ns, rows, x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum,
-                              x.v_sum, qa, ka, va, ws)
+        if do_pf:
+            L.ksa_interleave_rope(p, x.cu_seqlens, nt, ns, rows, x.q_text, x.k_text, x.v_text, x.q_sum,
+                                  x.k_sum, x.v_sum, qa, ka, va, ws)
         ev[1].record(st)
-        L.ksa_prefill_fwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, ws)
+        if do_pf:
+            L.ksa_prefill_fwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, ws)
         ev[2].record(st)
-        L.ksa_cache_append(pd, cache.desc, kind, kn, vn)
+        if do_dc:
+            L.ksa_cache_append(pd, cache.desc, kind, kn, vn)
         ev[3].record(st)
-        L.ksa_decode(pd, cache.desc, kind, qd, od, lsed, max_text, dws)
+        if do_dc:
+            L.ksa_decode(pd, cache.desc, kind, qd, od, lsed, max_text, dws)
         ev[4].record(st)
         if times is not None:
             torch.cuda.synchronize()
@@ -288,9 +296,11 @@ def run_ksa(args, rank, world, local):
     dec_ms_max = max_over_ranks(dec_ms, world)
     step_ms = max_over_ranks(float(np.sum(tarr, axis=1).mean()), world)
 
-    value = world * pf_flops / (pf_ms_max * 1e-3) / 1e12
-    dec_gbs = world * dec_bytes / (dec_ms_max * 1e-3) / 1e9
-    kern_tflops = pf_text_flops / (pf_ms * 1e-3) / 1e12
+    value = world * pf_flops / (pf_ms_max * 1e-3) / 1e12 if do_pf else 0.0
+    dec_gbs = world * dec_bytes / (dec_ms_max * 1e-3) / 1e9 if do_dc else 0.0
+    kern_tflops = pf_text_flops / (pf_ms * 1e-3) / 1e12 if do_pf else 0.0
+    if args.only == "decode":
+        value = dec_gbs
 
     # ---- e2e through the public API: pinned host inputs -> device -> result ----
     host = [t.cpu().pin_memory() for t in (x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum, x.v_sum)]
@@ -305,18 +315,20 @@ def run_ksa(args, rank, world, local):
         out = api.prefill(p, sl, cu_d, *dv, want_lse=False)
         out_h.copy_(out.o_aug, non_blocking=True)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(st)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
-    e2e_val = world * pf_flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms, e2e_val = None, None
+    if not args.profile and do_pf:
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(st)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+        e2e_val = world * pf_flops / (e2e_ms * 1e-3) / 1e12
 
     clocks = clk.summary()
     if rank == 0:
@@ -345,11 +357,13 @@ def run_ksa(args, rank, world, local):
                                 "kernel": "decode_split_kernel<128,4> + combine (time of ksa_decode)"},
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h), "ms": e2e_ms},
-            "gpu_launches": args.steps * 8,
+            "gpu_launches": args.steps * ((5 if do_pf else 0) + (3 if do_dc else 0)),
             "clocks": clocks,
             "timed_region_ms": total_ms,
         }
-        if world == 1:
+        if args.only == "decode":
+            line["unit"] = "GB/s"
+        if world == 1 and not args.profile and args.cpu_rows > 0:
             v, cores, nrows, dt = oracle_sample(args.cpu_rows)
             line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                     "sample": f"{nrows} evenly spaced text rows x 32 heads of the "
@@ -364,6 +378,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ksa", choices=["ksa", "reference"])
     ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="time one leg only (profiling); the JSON line then covers that leg")
+    ap.add_argument("--profile", action="store_true", help="skip the e2e and CPU legs (for ncu runs)")
+    ap.add_argument("--decode-batch", type=int, default=DC["B"])
     args = ap.parse_args()
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", 0))

@@ -54,16 +54,17 @@ class DecodeCache:
     """K/V cache [B, Hkv, slots, d] bf16 + state [B, 4] int32 (slot map of
     the report's Figure 4; see include/ksa.h)."""
 
-    def __init__(self, p: L.ksa_params, batch: int, cap_summaries: int, device="cuda"):
+    def __init__(self, p: L.ksa_params, batch: int, cap: int, device="cuda"):
+        """cap: summary-buffer capacity (chunks) of every sequence."""
         self.p = p
         self.batch = batch
-        self.cap = cap_summaries
-        self.slots = L.ksa_cache_slots(p, cap_summaries)
+        self.cap = cap
+        self.slots = L.ksa_cache_slots(p, cap)
         shape = (batch, p.num_kv_heads, self.slots, p.head_dim)
         self.k = torch.zeros(shape, dtype=torch.bfloat16, device=device)
         self.v = torch.zeros(shape, dtype=torch.bfloat16, device=device)
         self.state = torch.zeros(batch, 4, dtype=torch.int32, device=device)
-        self.desc = L.make_cache(self.k, self.v, self.state, cap_summaries)
+        self.desc = L.make_cache(self.k, self.v, self.state, cap)
 
     def append(self, kind, k_new, v_new, stream=None):
         L.ksa_cache_append(self.p, self.desc, kind, k_new, v_new, stream=stream)

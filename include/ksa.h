@@ -188,6 +188,27 @@ KSA_API int ksa_decode(const ksa_params *p, const ksa_cache *cache, const int8_t
                void *o, float *lse, int64_t max_text,
                void *workspace, size_t workspace_bytes, void *stream);
 
+/* ksa_decode without a workspace, for callers that cannot allocate device
+ * memory: a host program that owns all of the GPU's memory (for example a
+ * serving engine that reserves HBM for its own KV pools up front) or a
+ * custom op that is handed only its inputs and outputs has no allocator to
+ * take a workspace from, and a cudaMalloc of its own would break that
+ * ownership and stall the device in the middle of its decode loop.
+ * Arguments and results are those of ksa_decode minus the workspace; the
+ * split-K partials go to a 4 MiB device array that the library keeps on
+ * every GPU that loads it, until the process exits.  The first call made
+ * on a device looks up that array's device address, with that device
+ * current; make this first call before any stream capture.  A problem whose
+ * partials (ksa_decode_workspace_size) exceed 4 MiB returns
+ * KSA_ERR_CAPACITY and launches nothing.  Every call shares the one array
+ * and it keeps the last call's contents (nothing in it needs to start at
+ * zero); calls whose kernels can overlap on the GPU (other streams, other
+ * host threads) race on it, so the caller must order them.  The report has
+ * no counterpart to this call: it serves the library's callers, not the
+ * method. */
+KSA_API int ksa_decode_noalloc(const ksa_params *p, const ksa_cache *cache, const int8_t *kind,
+                               const void *q, void *o, float *lse, int64_t max_text, void *stream);
+
 /* Synchronise `stream`, return the device error word (KSA_OK if clear) and
  * reset it to KSA_OK.  dev_err: device int32. */
 KSA_API int ksa_get_device_error(int32_t *dev_err, void *stream);

@@ -74,6 +74,8 @@ SYMBOLS = {
     "ksa_decode_workspace_size": (_SZ, [ctypes.POINTER(ksa_params), _I32, _I64]),
     "ksa_decode": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _P, _P, _P,
                                   _I64, _P, _SZ, _P]),
+    "ksa_decode_noalloc": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _P, _P, _P,
+                                          _I64, _P]),
     "ksa_get_device_error": (ctypes.c_int, [_P, _P]),
     "ksa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -182,6 +184,13 @@ def ksa_decode(p, cache: ksa_cache, kind, q, o, lse, max_text, workspace, stream
                            max_text, _ptr(workspace), workspace.numel() * workspace.element_size(),
                            _stream(stream))
     _check("ksa_decode", rc)
+
+
+def ksa_decode_noalloc(p, cache: ksa_cache, kind, q, o, lse, max_text, stream=None):
+    """ksa_decode with the library's own fixed scratch instead of a workspace."""
+    rc = load().ksa_decode_noalloc(ctypes.byref(p), ctypes.byref(cache), _ptr(kind), _ptr(q), _ptr(o), _ptr(lse),
+                                   max_text, _stream(stream))
+    _check("ksa_decode_noalloc", rc)
 
 
 def ksa_get_device_error(dev_err, stream=None) -> int:

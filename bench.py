@@ -80,7 +80,7 @@ class ClockSampler:
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -127,14 +127,26 @@ def dist_setup(n_gpus):
     return 0, 1, 0
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """Slowest rank's value (timings are reported as the max over ranks)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(base, rank):
+    """Each rank runs an independent replica of the workload (weak scaling):
+    same shapes, its own inputs."""
+    return base + 100 * rank
+
+
+def whole_job_rate(work_per_rank, world, max_ms):
+    """Aggregate throughput: the work all ranks did over the slowest rank's time."""
+    return world * work_per_rank / (max_ms * 1e-3)
 
 
 def barrier(world):
@@ -213,7 +225,7 @@ def run_ksa(args, rank, world, local):
     sl, k, w, Hq, Hkv, d = PF["seqlens"], PF["k"], PF["w"], PF["Hq"], PF["Hkv"], PF["d"]
     if args.only == "decode":
         sl = [256]
-    x = prefill_inputs(sl, k, Hq, Hkv, d, seed=PF["seed"] + 100 * rank, scale=PF["scale"], device=dev)
+    x = prefill_inputs(sl, k, Hq, Hkv, d, seed=replica_seed(PF["seed"], rank), scale=PF["scale"], device=dev)
     p = L.make_params(k, w, Hq, Hkv, d, 0.0, PF["theta"])
     nt, ns = sum(sl), sum(n // k for n in sl)
     rows = L.ksa_aug_rows(p, sl)
@@ -232,8 +244,8 @@ def run_ksa(args, rank, world, local):
     B, m = (args.decode_batch if do_dc else 1), (DC["m"] if do_dc else 16)
     pd = L.make_params(DC["k"], DC["w"], DC["Hq"], DC["Hkv"], DC["d"], 0.0, DC["theta"])
     cache = api.DecodeCache(pd, B, cap=m + 64, device=dev)
-    fill_normal_(cache.k, 1000 + rank)
-    fill_normal_(cache.v, 2000 + rank)
+    fill_normal_(cache.k, replica_seed(1000, rank))
+    fill_normal_(cache.v, replica_seed(2000, rank))
     fills = uniform_ints(B, 0, DC["k"] - 1, seed=DC["seed"]).numpy()
     state0 = torch.zeros(B, 4, dtype=torch.int32)
     state0[:, 0] = torch.as_tensor(m * DC["k"] + fills, dtype=torch.int32)
@@ -296,8 +308,8 @@ def run_ksa(args, rank, world, local):
     dec_ms_max = max_over_ranks(dec_ms, world)
     step_ms = max_over_ranks(float(np.sum(tarr, axis=1).mean()), world)
 
-    value = world * pf_flops / (pf_ms_max * 1e-3) / 1e12 if do_pf else 0.0
-    dec_gbs = world * dec_bytes / (dec_ms_max * 1e-3) / 1e9 if do_dc else 0.0
+    value = whole_job_rate(pf_flops, world, pf_ms_max) / 1e12 if do_pf else 0.0
+    dec_gbs = whole_job_rate(dec_bytes, world, dec_ms_max) / 1e9 if do_dc else 0.0
     kern_tflops = pf_text_flops / (pf_ms * 1e-3) / 1e12 if do_pf else 0.0
     if args.only == "decode":
         value = dec_gbs
@@ -328,7 +340,7 @@ def run_ksa(args, rank, world, local):
         e1.record(st)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
-        e2e_val = world * pf_flops / (e2e_ms * 1e-3) / 1e12
+        e2e_val = whole_job_rate(pf_flops, world, e2e_ms) / 1e12
 
     clocks = clk.summary()
     if rank == 0:
@@ -374,7 +386,7 @@ def run_ksa(args, rank, world, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ksa", choices=["ksa", "reference"])
     ap.add_argument("--cpu-rows", type=int, default=2048)

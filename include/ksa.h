@@ -31,7 +31,8 @@
  *     kernel records a KSA_ERR_* code in a device error word and skips the
  *     affected work.  ksa_get_device_error() reads and clears such a word.
  *   - Supported: head_dim 64 or 128; num_q_heads % num_kv_heads == 0;
- *     k >= 1; w >= 0; (num_q_heads/num_kv_heads) * k <= 128 for prefill.
+ *     k >= 1; w >= 0; for prefill k <= 64 and (num_q_heads/num_kv_heads) * k
+ *     <= 128.
  */
 #ifndef KSA_H
 #define KSA_H

@@ -184,7 +184,7 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float *f)
     }
 }
 
-__device__ __forceinline__ float fast_exp2(float x)
+__device__ __forceinline__ float ex2f_approx(float x)
 {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -211,11 +211,17 @@ __device__ __forceinline__ bool decode_slice(int kind, int64_t n, int64_t m, int
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeArgs a)
+__global__ void __launch_bounds__(kDecThreads, 3) decode_split_kernel(DecodeArgs a)
 {
-    constexpr int LPK = D / 8;     // lanes per key row
-    constexpr int KPW = 32 / LPK;  // key rows per warp load
+    constexpr int LPK = D / 8;     // lanes per key row (8 dims = 16 bytes each)
+    constexpr int KPW = 32 / LPK;  // key rows per warp load instruction
+    constexpr int U = (LPK / G) < 4 ? (LPK / G) : 4;  // key rows per lane group per step
+    constexpr int NV = U * G;      // scores per lane group per step (<= LPK)
+    // after the reduce-scatter each score is complete on LPK/NV lanes: lane
+    // c8 holds score number c8 >> SH
+    constexpr int SH = (LPK / NV) == 1 ? 0 : (LPK / NV) == 2 ? 1 : (LPK / NV) == 4 ? 2 : 3;
     constexpr int HALF = D / 2;
+    static_assert(NV <= LPK && (LPK >> SH) == NV, "score layout");
     __shared__ float s_q[G][D];
     __shared__ float s_cos[HALF], s_sin[HALF];
     __shared__ float s_m[kDecWarps][G], s_l[kDecWarps][G];
@@ -258,41 +264,45 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeArgs a)
     __syncthreads();
 
     const int sub = lane / LPK;   // which key row of the warp load
-    const int c8 = lane % LPK;    // which 8 dims
+    const int c8 = lane % LPK;    // which 8 dims; after the reduce-scatter: score (u*G+g) << SH
     float qf[G][8];
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
         for (int e = 0; e < 8; ++e) qf[g][e] = s_q[g][c8 * 8 + e];
 
-    float mrun[G], lrun[G], acc[G][8];
+    // running state: max and sum of this lane's score slot (head my_g), and
+    // the accumulators of every head for this lane's 8 dims
+    float m_run = -INFINITY, l_run = 0.f, acc[G][8];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        mrun[g] = -INFINITY; lrun[g] = 0.f;
+    for (int g = 0; g < G; ++g)
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-    }
 
     const uint4 *Kb = a.K + (((int64_t)b * a.Hkv + h) * a.S) * (D / 8) + c8;
     const uint4 *Vb = a.V + (((int64_t)b * a.Hkv + h) * a.S) * (D / 8) + c8;
-    constexpr int STEP = kDecWarps * KPW * kDecU;  // rows per CTA step
-    for (int64_t base = r0; base < r1; base += STEP) {
-        uint4 kr[kDecU], vr[kDecU];
-        int64_t row[kDecU];
+    constexpr int STEP = kDecWarps * KPW * U;  // rows per CTA step
+    auto load = [&](int64_t base, uint4 *kr, uint4 *vr) {
 #pragma unroll
-        for (int u = 0; u < kDecU; ++u) {
-            row[u] = base + ((int64_t)u * kDecWarps + warp) * KPW + sub;
-            if (row[u] < r1) {
-                kr[u] = __ldcs(Kb + row[u] * (D / 8));
-                vr[u] = __ldcs(Vb + row[u] * (D / 8));
+        for (int u = 0; u < U; ++u) {
+            const int64_t row = base + ((int64_t)u * kDecWarps + warp) * KPW + sub;
+            if (row < r1) {
+                kr[u] = __ldcs(Kb + row * (D / 8));
+                vr[u] = __ldcs(Vb + row * (D / 8));
             } else {
                 kr[u] = make_uint4(0, 0, 0, 0);
                 vr[u] = kr[u];
             }
         }
-        float sc[kDecU][G];
+    };
+    uint4 kr[U], vr[U], kn[U], vn[U];
+    load(r0, kr, vr);
+    for (int64_t base = r0; base < r1; base += STEP) {
+        if (base + STEP < r1) load(base + STEP, kn, vn);   // next step's rows in flight
+        // partial scores of this lane's 8 dims: v[u*G + g]
+        float v[NV];
 #pragma unroll
-        for (int u = 0; u < kDecU; ++u) {
+        for (int u = 0; u < U; ++u) {
             float kf[8];
             bf16x8_to_f32(kr[u], kf);
 #pragma unroll
@@ -300,68 +310,105 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeArgs a)
                 float s = 0.f;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) s = fmaf(qf[g][e], kf[e], s);
-                sc[u][g] = s;
+                v[u * G + g] = s;
             }
         }
+        // reduce-scatter over the LPK lanes of a row group (top log2(NV)
+        // lane bits), then all-reduce over the remaining SH bits
 #pragma unroll
-        for (int off = LPK / 2; off >= 1; off >>= 1)
+        for (int off = LPK / 2, half = NV / 2; off >= 1; off >>= 1, half = half > 1 ? half / 2 : 0) {
+            if (half >= 1) {
+                const bool upper = (c8 & off) != 0;
 #pragma unroll
-            for (int u = 0; u < kDecU; ++u)
+                for (int i = 0; i < half; ++i) {
+                    const float send = upper ? v[i] : v[i + half];
+                    const float keep = upper ? v[i + half] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                }
+            } else {
+                v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+            }
+        }
+        const int my_u = (c8 >> SH) / G;
+        const int64_t my_row = base + ((int64_t)my_u * kDecWarps + warp) * KPW + sub;
+        float sc = my_row < r1 ? v[0] : -INFINITY;
+        // max over the U scores of this lane's head (score bits above log2 G)
+        float mx = sc;
 #pragma unroll
-                for (int g = 0; g < G; ++g) sc[u][g] += __shfl_xor_sync(0xffffffffu, sc[u][g], off);
+        for (int off = G << SH; off < LPK; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float m_new = fmaxf(m_run, mx);
+        const float corr = (m_new == -INFINITY) ? 1.f : ex2f_approx(m_run - m_new);
+        const float p = (m_new == -INFINITY) ? 0.f : ex2f_approx(sc - m_new);
+        m_run = m_new;
+        l_run = l_run * corr + p;
+        // every lane needs each head's correction and every (u, g) weight
+        const int gbase = lane & ~(LPK - 1);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            float mx = mrun[g];
+            const float cg = __shfl_sync(0xffffffffu, corr, gbase + (g << SH));
 #pragma unroll
-            for (int u = 0; u < kDecU; ++u) {
-                if (row[u] >= r1) sc[u][g] = -INFINITY;
-                mx = fmaxf(mx, sc[u][g]);
-            }
-            float corr = (mx == -INFINITY) ? 1.f : fast_exp2(mrun[g] - mx);
-            mrun[g] = mx;
-            lrun[g] *= corr;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[g][e] *= corr;
-#pragma unroll
-            for (int u = 0; u < kDecU; ++u) {
-                float pr = (mx == -INFINITY) ? 0.f : fast_exp2(sc[u][g] - mx);
-                sc[u][g] = pr;
-                lrun[g] += pr;
-            }
+            for (int e = 0; e < 8; ++e) acc[g][e] *= cg;
         }
 #pragma unroll
-        for (int u = 0; u < kDecU; ++u) {
+        for (int u = 0; u < U; ++u) {
             float vf[8];
             bf16x8_to_f32(vr[u], vf);
 #pragma unroll
-            for (int g = 0; g < G; ++g)
+            for (int g = 0; g < G; ++g) {
+                const float pg = __shfl_sync(0xffffffffu, p, gbase + ((u * G + g) << SH));
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(sc[u][g], vf[e], acc[g][e]);
+                for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pg, vf[e], acc[g][e]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) { kr[u] = kn[u]; vr[u] = vn[u]; }
+    }
+    // per head: combine the U score slots of the row group (the copies on
+    // the low SH lane bits are identical and are not summed)
+    {
+        float mx = m_run;
+#pragma unroll
+        for (int off = G << SH; off < LPK; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        float l = (mx == -INFINITY) ? 0.f : l_run * ex2f_approx(m_run - mx);
+#pragma unroll
+        for (int off = G << SH; off < LPK; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+        m_run = mx;
+        l_run = l;
+    }
+    // lanes whose score number has head g now hold (m, l) of head g; the
+    // accumulators are already relative to each head's m_run
+    float mh[G], lh[G];
+    {
+        const int gbase = lane & ~(LPK - 1);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            mh[g] = __shfl_sync(0xffffffffu, m_run, gbase + (g << SH));
+            lh[g] = __shfl_sync(0xffffffffu, l_run, gbase + (g << SH));
         }
     }
-    // merge the KPW key-row groups of the warp (lanes c8 + j*LPK)
+    // merge the KPW row groups of the warp (lanes c8 + j*LPK)
 #pragma unroll
     for (int off = LPK; off < 32; off <<= 1) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            float mo = __shfl_xor_sync(0xffffffffu, mrun[g], off);
-            float lo_ = __shfl_xor_sync(0xffffffffu, lrun[g], off);
-            float mn = fmaxf(mrun[g], mo);
-            float ca = (mn == -INFINITY) ? 0.f : fast_exp2(mrun[g] - mn);
-            float cb = (mn == -INFINITY) ? 0.f : fast_exp2(mo - mn);
-            lrun[g] = lrun[g] * ca + lo_ * cb;
+            float mo = __shfl_xor_sync(0xffffffffu, mh[g], off);
+            float lo_ = __shfl_xor_sync(0xffffffffu, lh[g], off);
+            float mn = fmaxf(mh[g], mo);
+            float ca = (mn == -INFINITY) ? 0.f : ex2f_approx(mh[g] - mn);
+            float cb = (mn == -INFINITY) ? 0.f : ex2f_approx(mo - mn);
+            lh[g] = lh[g] * ca + lo_ * cb;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 float ao = __shfl_xor_sync(0xffffffffu, acc[g][e], off);
                 acc[g][e] = acc[g][e] * ca + ao * cb;
             }
-            mrun[g] = mn;
+            mh[g] = mn;
         }
     }
     if (sub == 0) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            if (c8 == 0) { s_m[warp][g] = mrun[g]; s_l[warp][g] = lrun[g]; }
+            if (c8 == 0) { s_m[warp][g] = mh[g]; s_l[warp][g] = lh[g]; }
 #pragma unroll
             for (int e = 0; e < 8; ++e) s_acc[warp][g][c8 * 8 + e] = acc[g][e];
         }
@@ -376,7 +423,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeArgs a)
         float ll = 0.f, aa = 0.f;
 #pragma unroll
         for (int w2 = 0; w2 < kDecWarps; ++w2) {
-            float cf = (mm == -INFINITY) ? 0.f : fast_exp2(s_m[w2][g] - mm);
+            float cf = (mm == -INFINITY) ? 0.f : ex2f_approx(s_m[w2][g] - mm);
             ll += s_l[w2][g] * cf;
             aa += s_acc[w2][g][dd] * cf;
         }
@@ -404,7 +451,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeArgs a, __nv_
         float ll = 0.f, aa = 0.f;
         for (int s = 0; s < a.nsplit; ++s) {
             float ms = part[s * stride + g];
-            float cf = (ms == -INFINITY) ? 0.f : fast_exp2(ms - mm);
+            float cf = (ms == -INFINITY) ? 0.f : ex2f_approx(ms - mm);
             ll += part[s * stride + G + g] * cf;
             aa += part[s * stride + 2 * G + g * D + dd] * cf;
         }
@@ -418,8 +465,8 @@ static int decode_splits(const ksa_params *p, int batch, int64_t max_text)
 {
     int64_t max_slice = 1 + p->k + (int64_t)p->w * p->k + max_text / p->k;
     int64_t units = (int64_t)batch * p->num_kv_heads;
-    int64_t want = (4LL * sm_count() + units - 1) / units;  // ~4 CTAs per SM
-    int64_t cap = (max_slice + 255) / 256;                     // >= 256 rows per split
+    int64_t want = (32LL * sm_count() + units - 1) / units;  // ~8 waves of 4 CTAs per SM
+    int64_t cap = (max_slice + 511) / 512;                      // >= 512 rows per split
     int64_t s = want < cap ? want : cap;
     if (s < 1) s = 1;
     if (s > 1024) s = 1024;

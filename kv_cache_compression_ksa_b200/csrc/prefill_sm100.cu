@@ -37,6 +37,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "ksa_internal.cuh"
 
 namespace ksa {
@@ -44,30 +46,37 @@ namespace ksa {
 namespace pf {
 
 constexpr int BM = 128;        // rows per query tile (= TMEM lanes)
-constexpr int BN = 128;        // keys per K/V tile
-constexpr int NQ = 2;          // query tiles per CTA
-constexpr int STAGES = 2;      // K/V pipeline depth
-constexpr int kWarpTMA = 8;
-constexpr int kWarpMMA = 9;
-constexpr int kThreads = 320;
+constexpr int BN = 128;        // keys per K/V tile (N = 128 runs the MMA at full rate)
+constexpr int HC = BN / 2;     // keys per softmax half
+constexpr int NSBUF = 2;       // S buffers: QK(j+1) overlaps the softmax of tile j
+constexpr int QSTAGES = 2;     // query tiles: the next item's Q loads while this one runs
+constexpr int KSTAGES = 2;     // K pipeline depth
+constexpr int VSTAGES = 2;     // V pipeline depth
+constexpr int kWarpTMA = 8;    // loads Q and the K tiles
+constexpr int kWarpQK = 9;     // issues S = Q K^T, owns TMEM
+constexpr int kWarpPV = 10;    // issues O_h += P_h V_h
+constexpr int kWarpTMAV = 11;  // loads the V tiles (K loads never wait behind V)
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSpinLimit = 1u << 22;  // bounded waits (~0.5-4 s)
 
 template <int D>
 struct SmemLayout {
-    static constexpr int kTile = BM * D * 2;  // bytes of one 128 x D bf16 tile
+    static constexpr int kQTile = BM * D * 2;   // one 128 x D bf16 query tile
+    static constexpr int kKVTile = BN * D * 2;  // one 128 x D bf16 key or value tile
     static constexpr int kQ = 0;
-    static constexpr int kK = kQ + NQ * kTile;
-    static constexpr int kV = kK + STAGES * kTile;
-    static constexpr int kBar = kV + STAGES * kTile;
-    // barriers: q, kfull[S], kempty[S], vfull[S], vempty[S], s[NQ], p[NQ], o[NQ], drain
-    static constexpr int kNumBars = 1 + 4 * STAGES + 3 * NQ + 1;
-    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kK = kQ + QSTAGES * kQTile;
+    static constexpr int kV = kK + KSTAGES * kKVTile;
+    static constexpr int kBar = kV + VSTAGES * kKVTile;
+    // barriers: kfull[KS], kempty[KS], vfull[VS], vempty[VS], s[NSBUF], p[2 halves][NSBUF],
+    // o[NSBUF], drain x2, o free, q full[QS], q free[QS]
+    static constexpr int kNumBars = 2 * KSTAGES + 2 * VSTAGES + NSBUF + 2 * NSBUF + NSBUF + 2 + 1 + 2 * QSTAGES;
+    static constexpr int kXchg = kBar + kNumBars * 8;  // [unit parity][2 halves][2 values][128 rows] floats
+    static constexpr int kMisc = kXchg + 2 * 2 * 2 * BM * 4;
     static constexpr int kBytes = kMisc + 16;
-    // room to align the base to 1024; the rest of the SM's 227 KB is kept as
-    // slack (one CTA per SM either way: TMEM holds 512 columns)
-    static constexpr int kAlloc = 227 * 1024;
-    static_assert(kBytes + 1024 <= kAlloc, "shared memory budget");
+    static constexpr int kAlloc = kBytes + 1024;               // + alignment of the base to 1024
+    static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+    static_assert(NSBUF * BN + 2 * D <= (int)kTmemCols, "TMEM budget");  // S buffers, O_0, O_1
 };
 
 struct Params {
@@ -80,6 +89,7 @@ struct Params {
     const int32_t *cu;
     Plan pl;
     int32_t *err;
+    const __nv_bfloat16 *q;   // augmented query tensor (read row by row into TMEM)
     __nv_bfloat16 *o;
     float *lse;
 };
@@ -123,9 +133,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 
 // Bounded wait: false (after flagging the CTA and the error word) if the
 // phase did not complete within kSpinLimit polls or another role aborted.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                           int32_t *err)
 {
+    if (mbar_test(bar, parity)) return true;  // non-blocking fast path
     for (uint32_t it = 0; it < kSpinLimit; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
@@ -205,6 +229,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r)
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -245,6 +279,57 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major)
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
+
+// Named barrier shared by the two softmax warps that cover the same 32 rows
+// (warp w and w + 4): ids 1..4, 64 threads.
+__device__ __forceinline__ void pair_sync(int quarter)
+{
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+}
+
+// A work item: one query tile of 128 TMEM lanes (GQA-packed rows of one kv
+// head, unit_chunks chunks) and its list of 128-key K/V tiles: the window
+// tiles covering chunks c0-w .. cend-1, then the summary tiles.
+struct Unit {
+    int hkv, nb, mb, ncb, goff, c0, cend, cw_lo, n_win, T;
+};
+
+__device__ __forceinline__ Unit unit_of(const Params &P, int item, int n_units)
+{
+    Unit U;
+    const int rank = item / P.Hkv;
+    U.hkv = item % P.Hkv;
+    const int u = n_units - 1 - rank;  // heaviest (latest) units first
+    int lo = 0, hi = P.batch - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (P.pl.tile_off[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    U.nb = P.cu[b + 1] - P.cu[b];
+    U.mb = U.nb / P.k;
+    U.ncb = (U.nb + P.k - 1) / P.k;
+    U.goff = P.pl.chunk_off[b];
+    U.c0 = (u - P.pl.tile_off[b]) * P.unit_chunks;
+    U.cend = min(U.ncb, U.c0 + P.unit_chunks);
+    const int ns = max(min(U.mb, U.cend - 1 - P.w), 0);   // summaries any row may see
+    U.cw_lo = max(0, U.c0 - P.w);
+    U.n_win = (U.cend - U.cw_lo + P.Tk - 1) / P.Tk;
+    U.T = U.n_win + (ns + BN - 1) / BN;
+    return U;
+}
+
+// Persistent kernel: one CTA per SM walks work items blockIdx.x,
+// blockIdx.x + gridDim.x, ... (heavy first, round robin), so the loads and
+// first MMAs of the next item overlap the last tiles and the epilogue of
+// the current one.  Every role walks the same item list; barrier phases
+// follow a tile counter that runs on across items.
+//
+// The eight softmax warps split every key tile into two halves of 64 keys;
+// each half keeps its own running max, row sum and O accumulator in TMEM and
+// writes its P into its own half of the S buffer, so the two warps sharing an
+// SM sub-partition never wait for each other.  The halves merge in the
+// epilogue.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Params P)
 {
@@ -252,67 +337,54 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+    float *xchg = reinterpret_cast<float *>(smem + L::kXchg);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    // ---- work unit -------------------------------------------------------
     if (*P.err != 0) return;
     const int n_units = P.pl.tile_off[P.batch];
-    const int rank = blockIdx.x / P.Hkv;
-    const int hkv = blockIdx.x % P.Hkv;
-    if (rank >= n_units) return;
-    const int u = n_units - 1 - rank;  // longest (latest) units first
-    int b;
-    {
-        int lo = 0, hi = P.batch - 1;
-        while (lo < hi) {
-            int mid = (lo + hi + 1) >> 1;
-            if (P.pl.tile_off[mid] <= u) lo = mid; else hi = mid - 1;
-        }
-        b = lo;
-    }
-    const int nb = P.cu[b + 1] - P.cu[b];
-    const int mb = nb / P.k;                       // complete chunks = summaries
-    const int ncb = (nb + P.k - 1) / P.k;          // chunks incl. a partial one
-    const int goff = P.pl.chunk_off[b];            // first chunk in the layout
-    const int c0 = (u - P.pl.tile_off[b]) * P.unit_chunks;
-    const int cend = min(ncb, c0 + P.unit_chunks);
-    int ns = min(mb, cend - 1 - P.w);              // summaries any row may see
-    ns = max(ns, 0);
-    const int n_sum_tiles = (ns + BN - 1) / BN;
-    const int cw_lo = max(0, c0 - P.w);
-    const int n_win_tiles = (cend - cw_lo + P.Tk - 1) / P.Tk;
-    const int T = n_win_tiles + n_sum_tiles;
+    const int W = n_units * P.Hkv;   // work items
+    if ((int)blockIdx.x >= W) return;
 
     auto bar = [&](int i) { return sbase + L::kBar + 8u * (uint32_t)i; };
-    const int B_Q = 0;
-    auto B_KF = [&](int s) { return 1 + s; };
-    auto B_KE = [&](int s) { return 1 + STAGES + s; };
-    auto B_VF = [&](int s) { return 1 + 2 * STAGES + s; };
-    auto B_VE = [&](int s) { return 1 + 3 * STAGES + s; };
-    auto B_S = [&](int q) { return 1 + 4 * STAGES + q; };
-    auto B_P = [&](int q) { return 1 + 4 * STAGES + NQ + q; };
-    auto B_O = [&](int q) { return 1 + 4 * STAGES + 2 * NQ + q; };
-    const int B_DRAIN = 1 + 4 * STAGES + 3 * NQ;
+    auto B_KF = [&](int s) { return s; };
+    auto B_KE = [&](int s) { return KSTAGES + s; };
+    auto B_VF = [&](int s) { return 2 * KSTAGES + s; };
+    auto B_VE = [&](int s) { return 2 * KSTAGES + VSTAGES + s; };
+    constexpr int kB0 = 2 * KSTAGES + 2 * VSTAGES;
+    auto B_S = [&](int bf) { return kB0 + bf; };
+    auto B_P = [&](int h, int bf) { return kB0 + NSBUF + h * NSBUF + bf; };
+    auto B_O = [&](int bf) { return kB0 + 3 * NSBUF + bf; };
+    const int B_DRAIN_QK = kB0 + 4 * NSBUF;
+    const int B_DRAIN_PV = B_DRAIN_QK + 1;
+    const int B_OFREE = B_DRAIN_QK + 2;   // epilogue read O: the next item's PV may overwrite it
+    auto B_QF = [&](int q) { return B_DRAIN_QK + 3 + q; };            // query tile landed
+    auto B_QE = [&](int q) { return B_DRAIN_QK + 3 + QSTAGES + q; };  // its QKs are done
 
     // ---- setup -----------------------------------------------------------
     if (threadIdx.x == 0) {
-        mbar_init(bar(B_Q), 1);
-        for (int s = 0; s < STAGES; ++s) {
+        for (int q = 0; q < QSTAGES; ++q) {
+            mbar_init(bar(B_QF(q)), 1);
+            mbar_init(bar(B_QE(q)), 1);
+        }
+        for (int s = 0; s < KSTAGES; ++s) {
             mbar_init(bar(B_KF(s)), 1);
             mbar_init(bar(B_KE(s)), 1);
+        }
+        for (int s = 0; s < VSTAGES; ++s) {
             mbar_init(bar(B_VF(s)), 1);
             mbar_init(bar(B_VE(s)), 1);
         }
-        for (int q = 0; q < NQ; ++q) {
-            mbar_init(bar(B_S(q)), 1);
-            mbar_init(bar(B_P(q)), 128);
-            mbar_init(bar(B_O(q)), 1);
+        for (int bf = 0; bf < NSBUF; ++bf) {
+            mbar_init(bar(B_S(bf)), 1);
+            mbar_init(bar(B_P(0, bf)), 128);
+            mbar_init(bar(B_P(1, bf)), 128);
+            mbar_init(bar(B_O(bf)), 1);
         }
-        mbar_init(bar(B_DRAIN), 1);
+        mbar_init(bar(B_DRAIN_QK), 1);
+        mbar_init(bar(B_DRAIN_PV), 1);
+        mbar_init(bar(B_OFREE), 256);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -320,10 +392,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // (P is 0 there, and 0 * NaN would poison O).
     if (P.Tk * P.k < BN) {
         uint4 *vz = reinterpret_cast<uint4 *>(smem + L::kV);
-        for (int i = threadIdx.x; i < STAGES * L::kTile / 16; i += kThreads) vz[i] = make_uint4(0, 0, 0, 0);
+        for (int i = threadIdx.x; i < VSTAGES * L::kKVTile / 16; i += kThreads) vz[i] = make_uint4(0, 0, 0, 0);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == kWarpMMA) {
+    if (warp == kWarpQK) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(kTmemCols)
                      : "memory");
@@ -333,227 +405,314 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    auto S_COL = [&](int q) { return tmem + (uint32_t)(q * BN); };
-    auto O_COL = [&](int q) { return tmem + (uint32_t)(NQ * BN + q * D); };
+    auto S_COL = [&](int bf) { return tmem + (uint32_t)(bf * BN); };
+    auto O_COL = [&](int h) { return tmem + (uint32_t)(NSBUF * BN + h * D); };
 
     const uint32_t q_bytes = (uint32_t)(P.G * P.k * P.Tc) * 128u * (D / 64);
     const uint32_t win_bytes = (uint32_t)(P.k * P.Tk) * 128u * (D / 64);
     const uint32_t sum_bytes = (uint32_t)BN * 128u * (D / 64);
-    constexpr uint32_t kHalf = BM * 128;  // bytes of one 64-column half tile
+    constexpr uint32_t kQHalf = BM * 128;   // bytes of one 64-column half of the query tile
+    constexpr uint32_t kKVHalf = BN * 128;  // bytes of one 64-column half of a K/V tile
 
-    if (warp == kWarpTMA) {
-        // ================= TMA producer =================
+    if (warp == kWarpTMA || warp == kWarpTMAV) {
+        // ================= TMA producers: Q and K (warp 8), V (warp 11) =================
         if (lane == 0) {
-            int issued_k[STAGES] = {0}, issued_v[STAGES] = {0};
+            const bool isk = warp == kWarpTMA;
+            const int nst = isk ? KSTAGES : VSTAGES;
+            int issued[KSTAGES > VSTAGES ? KSTAGES : VSTAGES] = {0};
+            int q_issued[QSTAGES] = {0};
             bool ok = true;
-            mbar_expect_tx(bar(B_Q), q_bytes * NQ);
-            for (int q = 0; q < NQ; ++q)
-                for (int hf = 0; hf < D / 64; ++hf)
-                    tma_load_4d(sbase + L::kQ + q * L::kTile + hf * kHalf, &P.tm_q, bar(B_Q), hf * 64,
-                                hkv * P.G, 0, goff + c0 + q * P.Tc);
-            for (int j = 0; j < T && ok; ++j) {
-                const int s = j % STAGES;
-                const uint32_t ph = (uint32_t)((j / STAGES) - 1) & 1u;
-                const bool win = j < n_win_tiles;
-                const uint32_t bytes = win ? win_bytes : sum_bytes;
-                const CUtensorMap *mk = win ? &P.tm_kwin : &P.tm_ksum;
-                const CUtensorMap *mv = win ? &P.tm_vwin : &P.tm_vsum;
-                const int slot = win ? 0 : P.k;
-                const int chunk = goff + (win ? cw_lo + j * P.Tk : (j - n_win_tiles) * BN);
-                if (j >= STAGES && !(ok = mbar_wait(bar(B_KE(s)), ph, abort, P.err))) break;
-                mbar_expect_tx(bar(B_KF(s)), bytes);
-                for (int hf = 0; hf < D / 64; ++hf)
-                    tma_load_4d(sbase + L::kK + s * L::kTile + hf * kHalf, mk, bar(B_KF(s)), hf * 64, hkv,
-                                slot, chunk);
-                issued_k[s]++;
-                if (j >= STAGES && !(ok = mbar_wait(bar(B_VE(s)), ph, abort, P.err))) break;
-                mbar_expect_tx(bar(B_VF(s)), bytes);
-                for (int hf = 0; hf < D / 64; ++hf)
-                    tma_load_4d(sbase + L::kV + s * L::kTile + hf * kHalf, mv, bar(B_VF(s)), hf * 64, hkv,
-                                slot, chunk);
-                issued_v[s]++;
+            int gt = 0;
+            for (int item = blockIdx.x, n = 0; item < W && ok; item += gridDim.x, ++n) {
+                const Unit U = unit_of(P, item, n_units);
+                if (isk) {
+                    // query buffer n % 2 is free once the QKs of item n - 2 are done
+                    const int qb = n % QSTAGES;
+                    if (n >= QSTAGES &&
+                        !(ok = mbar_wait(bar(B_QE(qb)), (uint32_t)((n / QSTAGES) - 1) & 1u, abort, P.err)))
+                        break;
+                    mbar_expect_tx(bar(B_QF(qb)), q_bytes);
+                    for (int hf = 0; hf < D / 64; ++hf)
+                        tma_load_4d(sbase + L::kQ + qb * L::kQTile + hf * kQHalf, &P.tm_q, bar(B_QF(qb)), hf * 64,
+                                    U.hkv * P.G, 0, U.goff + U.c0);
+                    q_issued[qb]++;
+                }
+                for (int j = 0; j < U.T && ok; ++j, ++gt) {
+                    const int st = gt % nst;
+                    const bool win = j < U.n_win;
+                    const uint32_t bytes = win ? win_bytes : sum_bytes;
+                    const CUtensorMap *mp = isk ? (win ? &P.tm_kwin : &P.tm_ksum) : (win ? &P.tm_vwin : &P.tm_vsum);
+                    const int slot = win ? 0 : P.k;
+                    const int chunk = U.goff + (win ? U.cw_lo + j * P.Tk : (j - U.n_win) * BN);
+                    const int bempty = isk ? B_KE(st) : B_VE(st), bfull = isk ? B_KF(st) : B_VF(st);
+                    const uint32_t dst = sbase + (isk ? L::kK : L::kV) + st * L::kKVTile;
+                    if (gt >= nst &&
+                        !(ok = mbar_wait(bar(bempty), (uint32_t)((gt / nst) - 1) & 1u, abort, P.err)))
+                        break;
+                    mbar_expect_tx(bar(bfull), bytes);
+                    for (int hf = 0; hf < D / 64; ++hf)
+                        tma_load_4d(dst + hf * kKVHalf, mp, bar(bfull), hf * 64, U.hkv, slot, chunk);
+                    issued[st]++;
+                }
             }
             if (!ok) {
                 // drain: every load issued must land before the CTA exits
-                for (int s = 0; s < STAGES; ++s) {
-                    if (issued_k[s]) {
-                        uint32_t ph = (uint32_t)(issued_k[s] - 1) & 1u;
-                        for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_KF(s)), ph); ++it) {}
+                for (int st = 0; st < nst; ++st)
+                    if (issued[st]) {
+                        const uint32_t ph = (uint32_t)(issued[st] - 1) & 1u;
+                        const int bfull = isk ? B_KF(st) : B_VF(st);
+                        for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(bfull), ph); ++it) {}
                     }
-                    if (issued_v[s]) {
-                        uint32_t ph = (uint32_t)(issued_v[s] - 1) & 1u;
-                        for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_VF(s)), ph); ++it) {}
-                    }
-                }
-                for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_Q), 0); ++it) {}
+                if (isk)
+                    for (int qb = 0; qb < QSTAGES; ++qb)
+                        if (q_issued[qb]) {
+                            const uint32_t ph = (uint32_t)(q_issued[qb] - 1) & 1u;
+                            for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_QF(qb)), ph); ++it) {}
+                        }
             }
         }
-    } else if (warp == kWarpMMA) {
-        // ================= MMA issuer =================
+    } else if (warp == kWarpQK) {
+        // ================= S = Q K^T issuer =================
+        // S of tile gt goes to buffer gt % 2, free once both halves' PV of
+        // tile gt - 2 (which read P from it) has completed.
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16(BN, false);
-            const uint32_t id_pv = idesc_bf16(D, true);
-            bool ok = mbar_wait(bar(B_Q), 0, abort, P.err);
-            tc_fence_after();
-            for (int j = 0; j < T && ok; ++j) {
-                const int s = j % STAGES;
-                const uint32_t ph = (uint32_t)(j / STAGES) & 1u;
-                if (!(ok = mbar_wait(bar(B_KF(s)), ph, abort, P.err))) break;
-                tc_fence_after();
-                for (int q = 0; q < NQ && ok; ++q) {
-                    // S_q still holds P_q(j-1) until PV_q(j-1) has consumed it
-                    if (j > 0 && !(ok = mbar_wait(bar(B_O(q)), (uint32_t)(j - 1) & 1u, abort, P.err))) break;
+            bool ok = true;
+            int gt = 0;
+            for (int item = blockIdx.x, n = 0; item < W && ok; item += gridDim.x, ++n) {
+                const Unit U = unit_of(P, item, n_units);
+                const int qb = n % QSTAGES;
+                const uint32_t qa = sbase + L::kQ + qb * L::kQTile;
+                if (!(ok = mbar_wait(bar(B_QF(qb)), (uint32_t)(n / QSTAGES) & 1u, abort, P.err))) break;
+                for (int j = 0; j < U.T && ok; ++j, ++gt) {
+                    const int s = gt % KSTAGES, bf = gt % NSBUF;
+                    if (!(ok = mbar_wait(bar(B_KF(s)), (uint32_t)(gt / KSTAGES) & 1u, abort, P.err))) break;
+                    if (gt >= NSBUF &&
+                        !(ok = mbar_wait(bar(B_O(bf)), (uint32_t)((gt - NSBUF) / NSBUF) & 1u, abort, P.err)))
+                        break;
                     tc_fence_after();
-                    const uint32_t qa = sbase + L::kQ + q * L::kTile;
-                    const uint32_t ka = sbase + L::kK + s * L::kTile;
+                    const uint32_t ka = sbase + L::kK + s * L::kKVTile;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk / 4) * kHalf + (kk % 4) * 32;
-                        mma_ss(S_COL(q), sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), id_qk, kk > 0);
-                    }
-                    tc_commit(bar(B_S(q)));
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(S_COL(bf), sdesc(qa + (kk / 4) * kQHalf + (kk % 4) * 32, 16, 1024),
+                               sdesc(ka + (kk / 4) * kKVHalf + (kk % 4) * 32, 16, 1024), id_qk, kk > 0);
+                    tc_commit(bar(B_S(bf)));
+                    tc_commit(bar(B_KE(s)));
                 }
-                if (!ok) break;
-                tc_commit(bar(B_KE(s)));
-                if (!(ok = mbar_wait(bar(B_VF(s)), ph, abort, P.err))) break;
-                tc_fence_after();
-                for (int q = 0; q < NQ && ok; ++q) {
-                    if (!(ok = mbar_wait(bar(B_P(q)), (uint32_t)j & 1u, abort, P.err))) break;
-                    tc_fence_after();
-                    const uint32_t va = sbase + L::kV + s * L::kTile;
-#pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(O_COL(q), S_COL(q) + kk * 8, sdesc(va + kk * 2048, kHalf, 1024), id_pv,
-                               (j > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(bar(B_O(q)));
-                }
-                if (!ok) break;
-                tc_commit(bar(B_VE(s)));
+                if (ok) tc_commit(bar(B_QE(qb)));
             }
-            // all MMAs issued by this thread complete before TMEM is freed
-            tc_commit(bar(B_DRAIN));
-            for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_DRAIN), 0); ++it) {}
+            tc_commit(bar(B_DRAIN_QK));
+            for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_DRAIN_QK), 0); ++it) {}
+        }
+    } else if (warp == kWarpPV) {
+        // ================= O_h += P_h V_h issuer =================
+        // Half h's P (its 64 keys as bf16 pairs) sits in S columns
+        // [64h, 64h + 32); it multiplies V rows [64h, 64h + 64).
+        if (lane == 0) {
+            const uint32_t id_pv = idesc_bf16(D, true);
+            bool ok = true;
+            int gt = 0;
+            for (int item = blockIdx.x, n = 0; item < W && ok; item += gridDim.x, ++n) {
+                const Unit U = unit_of(P, item, n_units);
+                for (int j = 0; j < U.T && ok; ++j, ++gt) {
+                    const int s = gt % VSTAGES, bf = gt % NSBUF;
+                    if (!(ok = mbar_wait(bar(B_VF(s)), (uint32_t)(gt / VSTAGES) & 1u, abort, P.err))) break;
+                    // the previous item's epilogue must have read O before it restarts
+                    if (j == 0 && n > 0 &&
+                        !(ok = mbar_wait(bar(B_OFREE), (uint32_t)(n - 1) & 1u, abort, P.err)))
+                        break;
+                    const uint32_t va = sbase + L::kV + s * L::kKVTile;
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        if (!(ok = mbar_wait(bar(B_P(h, bf)), (uint32_t)(gt / NSBUF) & 1u, abort, P.err))) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < HC / 16; ++kk)
+                            mma_ts(O_COL(h), S_COL(bf) + h * HC + kk * 8,
+                                   sdesc(va + (h * (HC / 16) + kk) * 2048, kKVHalf, 1024), id_pv,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    if (!ok) break;
+                    tc_commit(bar(B_O(bf)));
+                    tc_commit(bar(B_VE(s)));
+                }
+            }
+            tc_commit(bar(B_DRAIN_PV));
+            for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_DRAIN_PV), 0); ++it) {}
         }
     } else {
-        // ================= softmax warpgroups =================
-        const int q = warp >> 2;                       // query tile of this warpgroup
-        const int R = (warp & 3) * 32 + lane;          // row = TMEM lane
-        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        // row -> (chunk, slot, head)
+        // ================= softmax: 8 warps, two independent key halves =================
+        const int half = warp >> 2;                    // keys [64 half, 64 half + 64) of each tile
+        const int quarter = warp & 3;
+        const int R = quarter * 32 + lane;             // row = TMEM lane
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int rows_per_chunk = P.k * P.G;
-        const int cl = R / rows_per_chunk;
+        const int cl = R / rows_per_chunk;             // row -> (chunk, slot, head)
         const int r_slot = (R / P.G) % P.k;
         const int g = R % P.G;
-        const int c = c0 + q * P.Tc + cl;
-        const int i = c * P.k + r_slot;                // local text index
-        const bool valid = cl < P.Tc && c < ncb && i < nb;
-        const int sum_lim = valid ? min(c - P.w, mb) : 0;   // sees s_j for j < sum_lim
-        const int win_lo = valid ? max(0, c - P.w) * P.k : 0;
         const float sl2 = P.scale_log2;
-
-        float m_run = -INFINITY;   // running max of raw scores used for P
-        float l_run = 0.f;
+        // An expired wait clears ok; every warp still walks all items and
+        // runs one pair barrier per item, so no barrier is left unmatched.
         bool ok = true;
-        for (int j = 0; j < T && ok; ++j) {
-            // mask interval [clo, chi) of this row in tile j
-            int clo, chi;
-            if (j < n_win_tiles) {
-                const int base = (cw_lo + j * P.Tk) * P.k;
-                clo = win_lo - base;
-                chi = valid ? i - base + 1 : 0;
-                chi = min(chi, P.Tk * P.k);
-            } else {
-                const int js = (j - n_win_tiles) * BN;
-                clo = 0;
-                chi = sum_lim - js;
-            }
-            clo = max(clo, 0);
-            chi = min(chi, BN);
-            if (chi < clo) chi = clo;
-            if (!(ok = mbar_wait(bar(B_S(q)), (uint32_t)j & 1u, abort, P.err))) break;
-            tc_fence_after();
-            uint32_t sr[BN];
-#pragma unroll
-            for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(S_COL(q) + lane_off + cc * 32, sr + cc * 32);
-            tmem_wait_ld();
-            float *s = reinterpret_cast<float *>(sr);
-            const bool full = __all_sync(0xffffffffu, clo == 0 && chi == BN);
-            float mx = -INFINITY;
-            if (full) {
-#pragma unroll
-                for (int e = 0; e < BN; ++e) mx = fmaxf(mx, s[e]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < BN; ++e) {
-                    s[e] = (e >= clo && e < chi) ? s[e] : -INFINITY;
-                    mx = fmaxf(mx, s[e]);
+        int gt = 0;
+        for (int item = blockIdx.x, n = 0; item < W; item += gridDim.x, ++n) {
+            const Unit U = unit_of(P, item, n_units);
+            const int c = U.c0 + cl;
+            const int i = c * P.k + r_slot;            // local text index
+            const bool valid = cl < P.Tc && c < U.ncb && i < U.nb;
+            const int sum_lim = valid ? min(c - P.w, U.mb) : 0;   // sees s_j for j < sum_lim
+            const int win_lo = valid ? max(0, c - P.w) * P.k : 0;
+            float m_run = -INFINITY;   // this half's running max of raw scores (the P reference)
+            float l_run = 0.f;         // this half's row sum
+            for (int j = 0; j < U.T; ++j, ++gt) {
+                if (!ok) continue;
+                const int bf = gt % NSBUF;
+                // mask interval [clo, chi) of this row in tile j, relative to this half
+                int clo, chi;
+                if (j < U.n_win) {
+                    const int base = (U.cw_lo + j * P.Tk) * P.k;
+                    clo = win_lo - base;
+                    chi = valid ? i - base + 1 : 0;
+                    chi = min(chi, P.Tk * P.k);
+                } else {
+                    const int js = (j - U.n_win) * BN;
+                    clo = 0;
+                    chi = sum_lim - js;
                 }
-            }
-            // lazy rescale: keep the old max unless the new one exceeds it by
-            // more than 8 in log2 units (P stays <= 256, exact either way)
-            const float m_new = fmaxf(m_run, mx);
-            const bool need = (m_new - m_run) * sl2 > 8.f || m_run == -INFINITY;
-            if (__any_sync(0xffffffffu, need && m_new != -INFINITY)) {
-                const float corr = (m_run == -INFINITY) ? 0.f : ex2((m_run - m_new) * sl2);
-                if (j > 0) {
-                    if (!(ok = mbar_wait(bar(B_O(q)), (uint32_t)(j - 1) & 1u, abort, P.err))) break;
+                clo = max(clo - half * HC, 0);
+                chi = min(chi - half * HC, HC);
+                if (chi < clo) chi = clo;
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S(bf)), (uint32_t)(gt / NSBUF) & 1u, abort, P.err));
+                if (!ok) continue;
+                uint32_t sr[HC];
+                float *s = reinterpret_cast<float *>(sr);
+                const bool full = __all_sync(0xffffffffu, clo == 0 && chi == HC);
+                auto load_s = [&]() {
                     tc_fence_after();
-#pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t orr[32];
-                        tmem_ld32(O_COL(q) + lane_off + cc * 32, orr);
-                        tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * corr);
-                        tmem_st32(O_COL(q) + lane_off + cc * 32, orr);
+                    for (int cc = 0; cc < HC / 32; ++cc)
+                        tmem_ld32(S_COL(bf) + lane_off + half * HC + cc * 32, sr + cc * 32);
+                    tmem_wait_ld();
+                    if (!full) {
+#pragma unroll
+                        for (int e = 0; e < HC; ++e) s[e] = (e >= clo && e < chi) ? s[e] : -INFINITY;
+                    }
+                };
+                // Pass 1: the row max and, speculatively, P against the current
+                // reference (independent, so ALU and MUFU work interleave).
+                load_s();
+                const float mb_old = (m_run == -INFINITY) ? 0.f : m_run * sl2;
+                float pm[8], ps[8];
+#pragma unroll
+                for (int a = 0; a < 8; ++a) { pm[a] = -INFINITY; ps[a] = 0.f; }
+#pragma unroll
+                for (int e = 0; e < HC; ++e) {
+                    pm[e & 7] = fmaxf(pm[e & 7], s[e]);
+                    const float pe = ex2(fmaf(s[e], sl2, -mb_old));
+                    ps[e & 7] += pe;
+                    s[e] = pe;
+                }
+                const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                       fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+                float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                // lazy rescale: keep the reference unless the max exceeds it by
+                // more than 8 in log2 units (P stays <= 256; exact either way)
+                const float m_new = fmaxf(m_run, mx);
+                const bool need = (m_new - m_run) * sl2 > 8.f || m_run == -INFINITY;
+                if (__any_sync(0xffffffffu, need && m_new != -INFINITY)) {
+                    const float corr = (m_run == -INFINITY) ? 0.f : ex2((m_run - m_new) * sl2);
+                    if (j > 0) {
+                        const int pb = (gt - 1) % NSBUF;
+                        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O(pb)), (uint32_t)((gt - 1) / NSBUF) & 1u,
+                                                               abort, P.err));
+                        if (!ok) continue;
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int cc = 0; cc < D / 32; ++cc) {
+                            uint32_t orr[32];
+                            const uint32_t oa = O_COL(half) + lane_off + cc * 32;
+                            tmem_ld32(oa, orr);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * corr);
+                            tmem_st32(oa, orr);
+                        }
+                    }
+                    l_run *= corr;
+                    m_run = m_new;
+                    // recompute P against the new reference (S is still intact)
+                    load_s();
+                    const float mb2 = (m_run == -INFINITY) ? 0.f : m_run * sl2;
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) ps[a] = 0.f;
+#pragma unroll
+                    for (int e = 0; e < HC; ++e) {
+                        const float pe = ex2(fmaf(s[e], sl2, -mb2));
+                        ps[e & 7] += pe;
+                        s[e] = pe;
+                    }
+                    sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                }
+                l_run += sum;
+                uint32_t pk[HC / 2];
+#pragma unroll
+                for (int e = 0; e < HC / 2; ++e) pk[e] = pack_bf16(s[2 * e], s[2 * e + 1]);
+                // P of this half -> S columns [64 half, 64 half + 32) (its own S region)
+                tmem_st32(S_COL(bf) + lane_off + half * HC, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(B_P(half, bf)));
+            }
+            // ---- epilogue of the item: merge the halves, O / l -> bf16 rows ----
+            if (ok)
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O((gt - 1) % NSBUF)), (uint32_t)((gt - 1) / NSBUF) & 1u,
+                                                       abort, P.err));
+            tc_fence_after();
+            float *xc = xchg + (n & 1) * 4 * BM;   // [half][m, l][row]
+            xc[(half * 2 + 0) * BM + R] = m_run;
+            xc[(half * 2 + 1) * BM + R] = l_run;
+            pair_sync(quarter);   // exactly once per item per softmax warp, on every path
+            const float m_o = xc[((1 - half) * 2 + 0) * BM + R];
+            const float l_o = xc[((1 - half) * 2 + 1) * BM + R];
+            const float m0 = half == 0 ? m_run : m_o, m1 = half == 0 ? m_o : m_run;
+            const float l0 = half == 0 ? l_run : l_o, l1 = half == 0 ? l_o : l_run;
+            const float M = fmaxf(m0, m1);
+            const float f0 = (M == -INFINITY) ? 0.f : ex2((m0 - M) * sl2);
+            const float f1 = (M == -INFINITY) ? 0.f : ex2((m1 - M) * sl2);
+            const float Lr = l0 * f0 + l1 * f1;
+            if (ok) {
+                const float inv = Lr > 0.f ? 1.f / Lr : 0.f;
+                const float g0 = f0 * inv, g1 = f1 * inv;
+                const int64_t row = (int64_t)(U.goff + c) * (P.k + 1) + r_slot;
+                const int head = U.hkv * P.G + g;
+                // this thread writes output columns [D/2 half, D/2 half + D/2)
+                uint4 *dst = reinterpret_cast<uint4 *>(P.o + (row * P.Hq + head) * D + half * (D / 2));
+#pragma unroll 1
+                for (int cc = 0; cc < D / 64; ++cc) {
+                    uint32_t a0[32], a1[32];
+                    tmem_ld32(O_COL(0) + lane_off + half * (D / 2) + cc * 32, a0);
+                    tmem_ld32(O_COL(1) + lane_off + half * (D / 2) + cc * 32, a1);
+                    tmem_wait_ld();
+                    if (valid) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float v[8];
+#pragma unroll
+                            for (int z = 0; z < 8; ++z)
+                                v[z] = __uint_as_float(a0[8 * e + z]) * g0 + __uint_as_float(a1[8 * e + z]) * g1;
+                            uint4 wv;
+                            wv.x = pack_bf16(v[0], v[1]);
+                            wv.y = pack_bf16(v[2], v[3]);
+                            wv.z = pack_bf16(v[4], v[5]);
+                            wv.w = pack_bf16(v[6], v[7]);
+                            dst[cc * 4 + e] = wv;
+                        }
                     }
                 }
-                l_run *= corr;
-                m_run = m_new;
+                if (valid && half == 0 && P.lse) P.lse[row * P.Hq + head] = M * P.scale + logf(Lr);
             }
-            const float mb2 = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-            float sum = 0.f;
-            uint32_t pk[BN / 2];
-#pragma unroll
-            for (int e = 0; e < BN / 2; ++e) {
-                float p0 = ex2(fmaf(s[2 * e], sl2, -mb2));
-                float p1 = ex2(fmaf(s[2 * e + 1], sl2, -mb2));
-                sum += p0 + p1;
-                pk[e] = pack_bf16(p0, p1);
-            }
-            l_run += sum;
-#pragma unroll
-            for (int cc = 0; cc < BN / 64; ++cc) tmem_st32(S_COL(q) + lane_off + cc * 32, pk + cc * 32);
-            tmem_wait_st();
+            // O has been read: the PV issuer may start the next item
             tc_fence_before();
-            mbar_arrive(bar(B_P(q)));
-        }
-        // ---- epilogue: O / l -> bf16 rows of the augmented layout ----
-        if (ok && T > 0) ok = mbar_wait(bar(B_O(q)), (uint32_t)(T - 1) & 1u, abort, P.err);
-        tc_fence_after();
-        if (ok) {
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            const int64_t row = (int64_t)(goff + c) * (P.k + 1) + r_slot;
-            const int head = hkv * P.G + g;
-            uint4 *dst = reinterpret_cast<uint4 *>(P.o + (row * P.Hq + head) * D);
-#pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t orr[32];
-                tmem_ld32(O_COL(q) + lane_off + cc * 32, orr);
-                tmem_wait_ld();
-                if (valid) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        uint4 v;
-                        v.x = pack_bf16(__uint_as_float(orr[8 * e + 0]) * inv, __uint_as_float(orr[8 * e + 1]) * inv);
-                        v.y = pack_bf16(__uint_as_float(orr[8 * e + 2]) * inv, __uint_as_float(orr[8 * e + 3]) * inv);
-                        v.z = pack_bf16(__uint_as_float(orr[8 * e + 4]) * inv, __uint_as_float(orr[8 * e + 5]) * inv);
-                        v.w = pack_bf16(__uint_as_float(orr[8 * e + 6]) * inv, __uint_as_float(orr[8 * e + 7]) * inv);
-                        dst[cc * 4 + e] = v;
-                    }
-                }
-            }
-            if (valid && P.lse) P.lse[row * P.Hq + head] = m_run * P.scale + logf(l_run);
+            mbar_arrive(bar(B_OFREE));
         }
     }
 
@@ -561,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kWarpMMA) {
+    if (warp == kWarpQK) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                      : "memory");
     }
@@ -584,10 +743,12 @@ struct SumArgs {
     float *lse;
 };
 
-template <int D>
+template <int D, int G>
 __global__ void __launch_bounds__(256) summary_rows_kernel(SumArgs a)
 {
-    constexpr int EPL = D / 32;  // elements per lane
+    constexpr int EPL = D / 32;  // contiguous elements per lane (8 or 4 bytes)
+    constexpr int RG = 8;        // key rows loaded together
+    using Vec = typename std::conditional<EPL == 4, uint2, uint32_t>::type;
     if (*a.err != 0) return;
     const int64_t task = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -604,38 +765,100 @@ __global__ void __launch_bounds__(256) summary_rows_kernel(SumArgs a)
     if (gc - a.pl.chunk_off[b] >= n / a.k) return;  // trailing partial chunk: no summary
     const int64_t row0 = gc * (a.k + 1);
     const int64_t srow = row0 + a.k;
-    for (int g = 0; g < a.G; ++g) {
-        const int head = h * a.G + g;
-        float qv[EPL];
-        const __nv_bfloat16 *qp = a.q + (srow * a.Hq + head) * D + lane * EPL;
+    auto unpack = [](Vec v, float *f) {
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(&v);
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) qv[e] = __bfloat162float(qp[e]);
-        float mx = -INFINITY;
-        float sc[65];
-        for (int t = 0; t <= a.k && t < 65; ++t) {
-            const __nv_bfloat16 *kp = a.kk + ((row0 + t) * a.Hkv + h) * D + lane * EPL;
-            float s = 0.f;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) s = fmaf(qv[e], __bfloat162float(kp[e]), s);
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-            sc[t] = s;
-            mx = fmaxf(mx, s);
+        for (int i = 0; i < EPL / 2; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
         }
-        float l = 0.f, acc[EPL];
+    };
+    float qv[G][EPL];
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
-        for (int t = 0; t <= a.k && t < 65; ++t) {
-            float p = ex2((sc[t] - mx) * a.scale_log2);
-            l += p;
-            const __nv_bfloat16 *vp = a.v + ((row0 + t) * a.Hkv + h) * D + lane * EPL;
+    for (int g = 0; g < G; ++g) {
+        const Vec *qp = reinterpret_cast<const Vec *>(a.q + (srow * a.Hq + h * G + g) * D) + lane;
+        unpack(*qp, qv[g]);
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[e] = fmaf(p, __bfloat162float(vp[e]), acc[e]);
+        for (int e = 0; e < EPL; ++e) qv[g][e] *= a.scale_log2;
+    }
+    float m[G], l[G], acc[G][EPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        m[g] = -INFINITY; l[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[g][e] = 0.f;
+    }
+    // the k+1 keys of s_j: rows 0..k of its chunk (k text rows, then itself)
+    for (int t0 = 0; t0 <= a.k; t0 += RG) {
+        Vec kr[RG], vr[RG];
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            const int t = t0 + r;
+            if (t <= a.k) {
+                kr[r] = reinterpret_cast<const Vec *>(a.kk + ((row0 + t) * a.Hkv + h) * D)[lane];
+                vr[r] = reinterpret_cast<const Vec *>(a.v + ((row0 + t) * a.Hkv + h) * D)[lane];
+            } else {
+                kr[r] = Vec{}; vr[r] = Vec{};
+            }
         }
-        __nv_bfloat16 *op = a.o + (srow * a.Hq + head) * D + lane * EPL;
+        float sc[G][RG];
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) op[e] = __float2bfloat16_rn(acc[e] / l);
-        if (a.lse && lane == 0) a.lse[srow * a.Hq + head] = mx * a.scale + logf(l);
+        for (int r = 0; r < RG; ++r) {
+            float kf[EPL];
+            unpack(kr[r], kf);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float s = 0.f;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) s = fmaf(qv[g][e], kf[e], s);
+                sc[g][r] = s;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int r = 0; r < RG; ++r) sc[g][r] += __shfl_xor_sync(0xffffffffu, sc[g][r], off);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float mx = m[g];
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                if (t0 + r > a.k) sc[g][r] = -INFINITY;
+                mx = fmaxf(mx, sc[g][r]);
+            }
+            const float corr = ex2(m[g] - mx);  // m = -inf on the first group: 0
+            l[g] *= corr;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[g][e] *= corr;
+            m[g] = mx;
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                sc[g][r] = ex2(sc[g][r] - mx);
+                l[g] += sc[g][r];
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            float vf[EPL];
+            unpack(vr[r], vf);
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) acc[g][e] = fmaf(sc[g][r], vf[e], acc[g][e]);
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const int head = h * G + g;
+        const float inv = 1.f / l[g];
+        Vec out;
+        uint32_t *w = reinterpret_cast<uint32_t *>(&out);
+#pragma unroll
+        for (int i = 0; i < EPL / 2; ++i) w[i] = pack_bf16(acc[g][2 * i] * inv, acc[g][2 * i + 1] * inv);
+        reinterpret_cast<Vec *>(a.o + (srow * a.Hq + head) * D)[lane] = out;
+        if (a.lse && lane == 0) a.lse[srow * a.Hq + head] = m[g] * 0.69314718055994530942f + logf(l[g]);
     }
 }
 
@@ -679,8 +902,7 @@ static bool make_map(CUtensorMap *m, const void *base, int d, int H, int k, int6
 int prefill_unit_chunks(const ksa_params *p)
 {
     int G = p->num_q_heads / p->num_kv_heads;
-    int Tc = pf::BM / (G * p->k);
-    return Tc * pf::NQ;
+    return pf::BM / (G * p->k);
 }
 
 template <int D>
@@ -697,12 +919,13 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
     P.Tk = pf::BN / k;
     if (P.Tc < 1 || P.Tk < 1) return KSA_ERR_UNSUPPORTED;
     P.batch = batch;
-    P.unit_chunks = P.Tc * pf::NQ;
+    P.unit_chunks = P.Tc;
     P.aug_rows = aug_rows;
     float scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)D);
     P.scale = scale;
     P.scale_log2 = scale * 1.4426950408889634f;
     P.cu = cu; P.pl = pl; P.err = err;
+    P.q = (const __nv_bfloat16 *)qa;
     P.o = (__nv_bfloat16 *)oa;
     P.lse = lse;
     bool ok = make_map(&P.tm_q, qa, D, Hq, k, chunks, G, k, P.Tc) &&
@@ -711,10 +934,11 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
               make_map(&P.tm_vsum, va, D, Hkv, k, chunks, 1, 1, pf::BN) &&
               make_map(&P.tm_vwin, va, D, Hkv, k, chunks, 1, k, P.Tk);
     if (!ok) return KSA_ERR_CUDA;
-    // units: an upper bound from host totals; surplus CTAs exit at once
+    // persistent: one CTA per SM (shared memory and TMEM admit one); each
+    // walks the work items round robin.  CTAs beyond the item count exit.
     int64_t units = total_text / ((int64_t)k * P.unit_chunks) + 2LL * batch + 1;
     int64_t grid = units * Hkv;
-    if (grid > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+    if (grid > sm_count()) grid = sm_count();
     static bool attr_set[2] = {false, false};
     if (!attr_set[D == 128]) {
         if (cudaFuncSetAttribute(pf::prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
@@ -733,7 +957,14 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
     s.o = (__nv_bfloat16 *)oa; s.lse = lse;
     int64_t tasks = chunks * Hkv;
     if (tasks > 0) {
-        pf::summary_rows_kernel<D><<<(unsigned)((tasks + 7) / 8), 256, 0, st>>>(s);
+        const unsigned blocks = (unsigned)((tasks + 7) / 8);
+        switch (G) {
+        case 1: pf::summary_rows_kernel<D, 1><<<blocks, 256, 0, st>>>(s); break;
+        case 2: pf::summary_rows_kernel<D, 2><<<blocks, 256, 0, st>>>(s); break;
+        case 4: pf::summary_rows_kernel<D, 4><<<blocks, 256, 0, st>>>(s); break;
+        case 8: pf::summary_rows_kernel<D, 8><<<blocks, 256, 0, st>>>(s); break;
+        default: return KSA_ERR_UNSUPPORTED;
+        }
         if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
     }
     return KSA_OK;
@@ -744,7 +975,6 @@ int launch_prefill(const ksa_params *p, int batch, const int32_t *cu, int64_t to
                    int32_t *err, cudaStream_t st)
 {
     if (aug_rows == 0) return KSA_OK;
-    if (p->k > 64) return KSA_ERR_UNSUPPORTED;  // summary-row kernel keeps <= 65 scores
     if (p->head_dim == 128)
         return launch_prefill_t<128>(p, batch, cu, total_text, aug_rows, qa, ka, va, oa, lse, pl, err, st);
     if (p->head_dim == 64)

@@ -149,17 +149,13 @@ int launch_cache_append(const ksa_params *p, const ksa_cache *c, const int8_t *k
 // ---------------------------------------------------------------------------
 // Decode: split-K over the contiguous slice.
 //
-// Grid (nsplit, Hkv, B); 4 warps per CTA.  A warp reads KPW = 32/LPK key
-// rows per 16-byte load instruction (LPK = d/8 lanes per row), U rows per
-// lane group per step, so every load instruction covers KPW*d*2 contiguous
-// bytes.  Each lane keeps the G query heads' slice of 8 dims and its own
-// running (max, sum, acc) per head; scores are completed with an xor
-// butterfly over the LPK lanes of a row.  Softmax runs in the log2 domain
-// with the scale folded into q.
+// Grid (nsplit, Hkv, B); 4 warps per CTA, each taking 16 key rows per step.
+// The per-key dot products and the P V product run on the warp-level tensor
+// core instruction (decode_split_kernel below); softmax runs in the log2
+// domain with the scale applied to the fp32 scores.
 // ---------------------------------------------------------------------------
 constexpr int kDecWarps = 4;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecU = 4;
 
 struct DecodeArgs {
     int k, w, Hkv, Hq, nsplit;
@@ -182,6 +178,12 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float *f)
         f[2 * i] = __uint_as_float(w[i] << 16);
         f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
     }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
 }
 
 __device__ __forceinline__ float ex2f_approx(float x)
@@ -210,18 +212,47 @@ __device__ __forceinline__ bool decode_slice(int kind, int64_t n, int64_t m, int
     return true;
 }
 
+// mma.sync m16n8k16, bf16 inputs, fp32 accumulate (D += A B)
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 8x8 b16 transpose across the warp, in registers
+__device__ __forceinline__ uint32_t movtrans(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t word(const uint4 &u, int i)
+{
+    return i == 0 ? u.x : i == 1 ? u.y : i == 2 ? u.z : u.w;
+}
+
+// Split-K decode on the warp-level tensor-core MMA.  The slice is read with
+// 16-byte loads: lane (g, t) = (lane / 4, lane % 4) loads dims
+// [32v + 8t, 32v + 8t + 8) of key rows g and g + 8 of each 16-row group.
+// Keys are the MMA rows: S^T = K Q^T (A = K, B = Q^T with the G query heads
+// as the 8 MMA columns) and O^T = V^T P^T.  The dot product is invariant
+// under any permutation of d applied to both q and k, so the fragment a lane
+// feeds to the MMA is exactly what it loaded; V and P fragments are turned
+// around with movmatrix.  Softmax statistics per head are merged with warp
+// shuffles.
 template <int D, int G>
 __global__ void __launch_bounds__(kDecThreads, 3) decode_split_kernel(DecodeArgs a)
 {
-    constexpr int LPK = D / 8;     // lanes per key row (8 dims = 16 bytes each)
-    constexpr int KPW = 32 / LPK;  // key rows per warp load instruction
-    constexpr int U = (LPK / G) < 4 ? (LPK / G) : 4;  // key rows per lane group per step
-    constexpr int NV = U * G;      // scores per lane group per step (<= LPK)
-    // after the reduce-scatter each score is complete on LPK/NV lanes: lane
-    // c8 holds score number c8 >> SH
-    constexpr int SH = (LPK / NV) == 1 ? 0 : (LPK / NV) == 2 ? 1 : (LPK / NV) == 4 ? 2 : 3;
+    static_assert(G <= 8, "query heads per kv head must fit the 8 MMA columns");
+    constexpr int NV = D / 32;     // 16-byte loads per key row and lane
+    constexpr int NC = D / 16;     // MMA k-chunks of the QK product
+    constexpr int NM = D / 16;     // MMA m-tiles of the PV product
     constexpr int HALF = D / 2;
-    static_assert(NV <= LPK && (LPK >> SH) == NV, "score layout");
     __shared__ float s_q[G][D];
     __shared__ float s_cos[HALF], s_sin[HALF];
     __shared__ float s_m[kDecWarps][G], s_l[kDecWarps][G];
@@ -243,7 +274,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_split_kernel(DecodeArgs
     const int64_t r0 = lo + (int64_t)split * per;
     const int64_t r1 = min(hi, r0 + per);
 
-    // rotated, pre-scaled q of the G heads of this kv head, position n - 1
+    // rotated q of the G heads of this kv head, position n - 1
     for (int r = t; r < HALF; r += kDecThreads) {
         float c = 1.f, s = 0.f;
         if (a.rotate) rope_cos_sin((double)(n - 1), r, D, a.log2_theta, &c, &s);
@@ -256,179 +287,136 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_split_kernel(DecodeArgs
         float x = __bfloat162float(qh[r]), y = __bfloat162float(qh[r + HALF]);
         float c = s_cos[r], s = s_sin[r];
         // the prefill path stores rotated q as bf16; round the same way
-        float xr = __bfloat162float(__float2bfloat16_rn(x * c - y * s));
-        float yr = __bfloat162float(__float2bfloat16_rn(y * c + x * s));
-        s_q[g][r] = xr * a.scale_log2;
-        s_q[g][r + HALF] = yr * a.scale_log2;
+        s_q[g][r] = __bfloat162float(__float2bfloat16_rn(x * c - y * s));
+        s_q[g][r + HALF] = __bfloat162float(__float2bfloat16_rn(y * c + x * s));
     }
     __syncthreads();
 
-    const int sub = lane / LPK;   // which key row of the warp load
-    const int c8 = lane % LPK;    // which 8 dims; after the reduce-scatter: score (u*G+g) << SH
-    float qf[G][8];
+    const int g = lane >> 2, tt = lane & 3;
+    // B fragments of Q^T: column (head) g, k-chunk c = 2v + hh covers dims
+    // 32v + 8tt + 4hh + {0,1} (b0) and {2,3} (b1)
+    uint32_t qb[NC][2];
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+    for (int c = 0; c < NC; ++c) {
+        const int v = c / 2, hh = c % 2;
+        const int d0 = 32 * v + 8 * tt + 4 * hh;
+        if (g < G) {
+            qb[c][0] = pack_bf16(s_q[g][d0], s_q[g][d0 + 1]);
+            qb[c][1] = pack_bf16(s_q[g][d0 + 2], s_q[g][d0 + 3]);
+        } else {
+            qb[c][0] = qb[c][1] = 0u;
+        }
+    }
+    // O^T accumulators: m-tile i = (v, pp): rows 0-7 are dims
+    // 32v + 8(row/2) + 2(2pp) + row%2, rows 8-15 the same with 2pp + 1
+    float o[NM][4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) qf[g][e] = s_q[g][c8 * 8 + e];
+    for (int i = 0; i < NM; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    // running max / sum of heads 2tt and 2tt + 1 (log2 domain)
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
-    // running state: max and sum of this lane's score slot (head my_g), and
-    // the accumulators of every head for this lane's 8 dims
-    float m_run = -INFINITY, l_run = 0.f, acc[G][8];
+    const uint4 *Kb = a.K + (((int64_t)b * a.Hkv + h) * a.S) * (D / 8);
+    const uint4 *Vb = a.V + (((int64_t)b * a.Hkv + h) * a.S) * (D / 8);
+    for (int64_t kb = r0 + 16 * warp; kb < r1; kb += 16 * kDecWarps) {
+        const int64_t key0 = kb + g, key1 = kb + g + 8;
+        const bool in0 = key0 < r1, in1 = key1 < r1;
+        uint4 kA[NV], kB[NV], vA[NV], vB[NV];
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+        for (int v = 0; v < NV; ++v) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            kA[v] = in0 ? __ldcs(Kb + key0 * (D / 8) + 4 * v + tt) : z;
+            kB[v] = in1 ? __ldcs(Kb + key1 * (D / 8) + 4 * v + tt) : z;
+            vA[v] = in0 ? __ldcs(Vb + key0 * (D / 8) + 4 * v + tt) : z;
+            vB[v] = in1 ? __ldcs(Vb + key1 * (D / 8) + 4 * v + tt) : z;
+        }
+        // S^T = K Q^T for the 16 keys
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-
-    const uint4 *Kb = a.K + (((int64_t)b * a.Hkv + h) * a.S) * (D / 8) + c8;
-    const uint4 *Vb = a.V + (((int64_t)b * a.Hkv + h) * a.S) * (D / 8) + c8;
-    constexpr int STEP = kDecWarps * KPW * U;  // rows per CTA step
-    auto load = [&](int64_t base, uint4 *kr, uint4 *vr) {
+        for (int c = 0; c < NC; ++c) {
+            const int v = c / 2, hh = c % 2;
+            mma16816(sc, word(kA[v], 2 * hh), word(kB[v], 2 * hh), word(kA[v], 2 * hh + 1),
+                     word(kB[v], 2 * hh + 1), qb[c][0], qb[c][1]);
+        }
+        // sc[0..1]: key g, heads 2tt, 2tt+1; sc[2..3]: key g + 8
+        float x[4];
+        x[0] = in0 ? sc[0] * a.scale_log2 : -INFINITY;
+        x[1] = in0 ? sc[1] * a.scale_log2 : -INFINITY;
+        x[2] = in1 ? sc[2] * a.scale_log2 : -INFINITY;
+        x[3] = in1 ? sc[3] * a.scale_log2 : -INFINITY;
+        float corr[2], pv[4];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t row = base + ((int64_t)u * kDecWarps + warp) * KPW + sub;
-            if (row < r1) {
-                kr[u] = __ldcs(Kb + row * (D / 8));
-                vr[u] = __ldcs(Vb + row * (D / 8));
-            } else {
-                kr[u] = make_uint4(0, 0, 0, 0);
-                vr[u] = kr[u];
+        for (int e = 0; e < 2; ++e) {
+            float mx = fmaxf(x[e], x[e + 2]);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float m_new = fmaxf(m_run[e], mx);
+            corr[e] = (m_new == -INFINITY) ? 1.f : ex2f_approx(m_run[e] - m_new);
+            pv[e] = (m_new == -INFINITY) ? 0.f : ex2f_approx(x[e] - m_new);
+            pv[e + 2] = (m_new == -INFINITY) ? 0.f : ex2f_approx(x[e + 2] - m_new);
+            l_run[e] = l_run[e] * corr[e] + pv[e] + pv[e + 2];
+            m_run[e] = m_new;
+        }
+        if (__any_sync(0xffffffffu, corr[0] != 1.f || corr[1] != 1.f)) {
+#pragma unroll
+            for (int i = 0; i < NM; ++i) {
+                o[i][0] *= corr[0]; o[i][1] *= corr[1];
+                o[i][2] *= corr[0]; o[i][3] *= corr[1];
             }
         }
-    };
-    uint4 kr[U], vr[U], kn[U], vn[U];
-    load(r0, kr, vr);
-    for (int64_t base = r0; base < r1; base += STEP) {
-        if (base + STEP < r1) load(base + STEP, kn, vn);   // next step's rows in flight
-        // partial scores of this lane's 8 dims: v[u*G + g]
-        float v[NV];
+        // P^T fragments (k = keys, n = heads) by transposing the S^T layout
+        const uint32_t pb0 = movtrans(pack_bf16(pv[0], pv[1]));
+        const uint32_t pb1 = movtrans(pack_bf16(pv[2], pv[3]));
+        // O^T += V^T P^T
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            float kf[8];
-            bf16x8_to_f32(kr[u], kf);
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                float s = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) s = fmaf(qf[g][e], kf[e], s);
-                v[u * G + g] = s;
-            }
-        }
-        // reduce-scatter over the LPK lanes of a row group (top log2(NV)
-        // lane bits), then all-reduce over the remaining SH bits
-#pragma unroll
-        for (int off = LPK / 2, half = NV / 2; off >= 1; off >>= 1, half = half > 1 ? half / 2 : 0) {
-            if (half >= 1) {
-                const bool upper = (c8 & off) != 0;
-#pragma unroll
-                for (int i = 0; i < half; ++i) {
-                    const float send = upper ? v[i] : v[i + half];
-                    const float keep = upper ? v[i + half] : v[i];
-                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-                }
-            } else {
-                v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
-            }
-        }
-        const int my_u = (c8 >> SH) / G;
-        const int64_t my_row = base + ((int64_t)my_u * kDecWarps + warp) * KPW + sub;
-        float sc = my_row < r1 ? v[0] : -INFINITY;
-        // max over the U scores of this lane's head (score bits above log2 G)
-        float mx = sc;
-#pragma unroll
-        for (int off = G << SH; off < LPK; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float m_new = fmaxf(m_run, mx);
-        const float corr = (m_new == -INFINITY) ? 1.f : ex2f_approx(m_run - m_new);
-        const float p = (m_new == -INFINITY) ? 0.f : ex2f_approx(sc - m_new);
-        m_run = m_new;
-        l_run = l_run * corr + p;
-        // every lane needs each head's correction and every (u, g) weight
-        const int gbase = lane & ~(LPK - 1);
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float cg = __shfl_sync(0xffffffffu, corr, gbase + (g << SH));
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[g][e] *= cg;
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            float vf[8];
-            bf16x8_to_f32(vr[u], vf);
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float pg = __shfl_sync(0xffffffffu, p, gbase + ((u * G + g) << SH));
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pg, vf[e], acc[g][e]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) { kr[u] = kn[u]; vr[u] = vn[u]; }
-    }
-    // per head: combine the U score slots of the row group (the copies on
-    // the low SH lane bits are identical and are not summed)
-    {
-        float mx = m_run;
-#pragma unroll
-        for (int off = G << SH; off < LPK; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        float l = (mx == -INFINITY) ? 0.f : l_run * ex2f_approx(m_run - mx);
-#pragma unroll
-        for (int off = G << SH; off < LPK; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-        m_run = mx;
-        l_run = l;
-    }
-    // lanes whose score number has head g now hold (m, l) of head g; the
-    // accumulators are already relative to each head's m_run
-    float mh[G], lh[G];
-    {
-        const int gbase = lane & ~(LPK - 1);
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            mh[g] = __shfl_sync(0xffffffffu, m_run, gbase + (g << SH));
-            lh[g] = __shfl_sync(0xffffffffu, l_run, gbase + (g << SH));
+        for (int i = 0; i < NM; ++i) {
+            const int v = i / 2, pp = i % 2;
+            mma16816(o[i], movtrans(word(vA[v], 2 * pp)), movtrans(word(vA[v], 2 * pp + 1)),
+                     movtrans(word(vB[v], 2 * pp)), movtrans(word(vB[v], 2 * pp + 1)), pb0, pb1);
         }
     }
-    // merge the KPW row groups of the warp (lanes c8 + j*LPK)
+    // row sums: the lanes of a head share its max, so partial sums add up
 #pragma unroll
-    for (int off = LPK; off < 32; off <<= 1) {
+    for (int e = 0; e < 2; ++e)
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float mo = __shfl_xor_sync(0xffffffffu, mh[g], off);
-            float lo_ = __shfl_xor_sync(0xffffffffu, lh[g], off);
-            float mn = fmaxf(mh[g], mo);
-            float ca = (mn == -INFINITY) ? 0.f : ex2f_approx(mh[g] - mn);
-            float cb = (mn == -INFINITY) ? 0.f : ex2f_approx(mo - mn);
-            lh[g] = lh[g] * ca + lo_ * cb;
+        for (int off = 4; off < 32; off <<= 1) l_run[e] += __shfl_xor_sync(0xffffffffu, l_run[e], off);
+    // scatter this warp's O^T into s_acc[warp][head][dim]
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                float ao = __shfl_xor_sync(0xffffffffu, acc[g][e], off);
-                acc[g][e] = acc[g][e] * ca + ao * cb;
+    for (int i = 0; i < NM; ++i) {
+        const int v = i / 2, pp = i % 2;
+        const int dA = 32 * v + 8 * (g / 2) + 2 * (2 * pp) + (g % 2);
+        const int dB = dA + 2;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int head = 2 * tt + e;
+            if (head < G) {
+                s_acc[warp][head][dA] = o[i][e];
+                s_acc[warp][head][dB] = o[i][2 + e];
             }
-            mh[g] = mn;
         }
     }
-    if (sub == 0) {
+    if (g == 0) {
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            if (c8 == 0) { s_m[warp][g] = mh[g]; s_l[warp][g] = lh[g]; }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) s_acc[warp][g][c8 * 8 + e] = acc[g][e];
+        for (int e = 0; e < 2; ++e) {
+            const int head = 2 * tt + e;
+            if (head < G) { s_m[warp][head] = m_run[e]; s_l[warp][head] = l_run[e]; }
         }
     }
     __syncthreads();
     float *out = a.part + ((((int64_t)b * a.Hkv + h) * a.nsplit) + split) * (G * (2 + D));
     for (int e = t; e < G * D; e += kDecThreads) {
-        int g = e / D, dd = e % D;
+        int gg = e / D, dd = e % D;
         float mm = -INFINITY;
 #pragma unroll
-        for (int w2 = 0; w2 < kDecWarps; ++w2) mm = fmaxf(mm, s_m[w2][g]);
+        for (int w2 = 0; w2 < kDecWarps; ++w2) mm = fmaxf(mm, s_m[w2][gg]);
         float ll = 0.f, aa = 0.f;
 #pragma unroll
         for (int w2 = 0; w2 < kDecWarps; ++w2) {
-            float cf = (mm == -INFINITY) ? 0.f : ex2f_approx(s_m[w2][g] - mm);
-            ll += s_l[w2][g] * cf;
-            aa += s_acc[w2][g][dd] * cf;
+            float cf = (mm == -INFINITY) ? 0.f : ex2f_approx(s_m[w2][gg] - mm);
+            ll += s_l[w2][gg] * cf;
+            aa += s_acc[w2][gg][dd] * cf;
         }
-        out[2 * G + g * D + dd] = aa;
-        if (dd == 0) { out[g] = mm; out[G + g] = ll; }
+        out[2 * G + gg * D + dd] = aa;
+        if (dd == 0) { out[gg] = mm; out[G + gg] = ll; }
     }
 }
 

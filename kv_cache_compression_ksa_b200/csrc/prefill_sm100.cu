@@ -67,20 +67,22 @@ struct SmemLayout {
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + QSTAGES * kQTile;
     static constexpr int kV = kK + KSTAGES * kKVTile;
-    static constexpr int kBar = kV + VSTAGES * kKVTile;
+    static constexpr int kO = kV + VSTAGES * kKVTile;           // output tile staging for the TMA store
+    static constexpr int kBar = kO + kQTile;
     // barriers: kfull[KS], kempty[KS], vfull[VS], vempty[VS], s[NSBUF], p[2 halves][NSBUF],
     // o[NSBUF], drain x2, o free, q full[QS], q free[QS]
     static constexpr int kNumBars = 2 * KSTAGES + 2 * VSTAGES + NSBUF + 2 * NSBUF + NSBUF + 2 + 1 + 2 * QSTAGES;
-    static constexpr int kXchg = kBar + kNumBars * 8;  // [unit parity][2 halves][2 values][128 rows] floats
-    static constexpr int kMisc = kXchg + 2 * 2 * 2 * BM * 4;
+    static constexpr int kXchg = kBar + kNumBars * 8;  // [2 halves][2 values][128 rows] floats
+    static constexpr int kMisc = kXchg + 2 * 2 * BM * 4;
     static constexpr int kBytes = kMisc + 16;
-    static constexpr int kAlloc = kBytes + 1024;               // + alignment of the base to 1024
+    // the dynamic shared memory base is 1024-byte aligned (checked at run time)
+    static constexpr int kAlloc = kBytes;
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
     static_assert(NSBUF * BN + 2 * D <= (int)kTmemCols, "TMEM budget");  // S buffers, O_0, O_1
 };
 
 struct Params {
-    CUtensorMap tm_q, tm_ksum, tm_kwin, tm_vsum, tm_vwin;
+    CUtensorMap tm_q, tm_ksum, tm_kwin, tm_vsum, tm_vwin, tm_o;
     int k, w, G, Hq, Hkv, Tc, Tk, batch;
     int unit_chunks;
     int64_t aug_rows;
@@ -167,6 +169,15 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
         " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
+}
+
+// shared -> global tiled store (bulk group; completion via wait_group)
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2, int c3)
+{
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -334,8 +345,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Params P)
 {
     using L = SmemLayout<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw;
     const uint32_t sbase = smem_u32(smem);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
@@ -343,6 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (*P.err != 0) return;
+    if (sbase & 1023u) {   // the 128-byte swizzled tiles need a 1024-byte aligned base
+        if (threadIdx.x == 0) set_error(P.err, KSA_ERR_UNSUPPORTED);
+        return;
+    }
     const int n_units = P.pl.tile_off[P.batch];
     const int W = n_units * P.Hkv;   // work items
     if ((int)blockIdx.x >= W) return;
@@ -551,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const int g = R % P.G;
         const float sl2 = P.scale_log2;
         // An expired wait clears ok; every warp still walks all items and
-        // runs one pair barrier per item, so no barrier is left unmatched.
+        // runs two pair barriers per item, so no barrier is left unmatched.
         bool ok = true;
         int gt = 0;
         for (int item = blockIdx.x, n = 0; item < W; item += gridDim.x, ++n) {
@@ -667,53 +682,80 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O((gt - 1) % NSBUF)), (uint32_t)((gt - 1) / NSBUF) & 1u,
                                                        abort, P.err));
             tc_fence_after();
-            float *xc = xchg + (n & 1) * 4 * BM;   // [half][m, l][row]
+            float *xc = xchg;   // [half][m, l][row]
             xc[(half * 2 + 0) * BM + R] = m_run;
             xc[(half * 2 + 1) * BM + R] = l_run;
-            pair_sync(quarter);   // exactly once per item per softmax warp, on every path
+            pair_sync(quarter);   // twice per item per softmax warp, on every path
             const float m_o = xc[((1 - half) * 2 + 0) * BM + R];
             const float l_o = xc[((1 - half) * 2 + 1) * BM + R];
+            pair_sync(quarter);   // both read: the next item may overwrite the exchange
             const float m0 = half == 0 ? m_run : m_o, m1 = half == 0 ? m_o : m_run;
             const float l0 = half == 0 ? l_run : l_o, l1 = half == 0 ? l_o : l_run;
             const float M = fmaxf(m0, m1);
             const float f0 = (M == -INFINITY) ? 0.f : ex2((m0 - M) * sl2);
             const float f1 = (M == -INFINITY) ? 0.f : ex2((m1 - M) * sl2);
             const float Lr = l0 * f0 + l1 * f1;
-            if (ok) {
-                const float inv = Lr > 0.f ? 1.f / Lr : 0.f;
-                const float g0 = f0 * inv, g1 = f1 * inv;
-                const int64_t row = (int64_t)(U.goff + c) * (P.k + 1) + r_slot;
-                const int head = U.hkv * P.G + g;
-                // this thread writes output columns [D/2 half, D/2 half + D/2)
-                uint4 *dst = reinterpret_cast<uint4 *>(P.o + (row * P.Hq + head) * D + half * (D / 2));
+            // Units whose chunks are all whole leave through a TMA store of the
+            // staged tile (the query tile's box over o); the last unit of a
+            // sequence stores its real rows one by one, so no padding row is written.
+            const bool tma_out = U.c0 + P.Tc <= U.mb;
+            if (tma_out) {
+                // the staging buffer is free once the previous store has read it
+                if (warp == 0 && lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                asm volatile("bar.sync 13, 256;" ::: "memory");
+            }
+            const float inv = Lr > 0.f ? 1.f / Lr : 0.f;
+            const float g0 = f0 * inv, g1 = f1 * inv;
+            const int64_t row = (int64_t)(U.goff + c) * (P.k + 1) + r_slot;
+            const int head = U.hkv * P.G + g;
+            // this thread holds output columns [D/2 half, D/2 half + D/2) of its row
+            uint4 *dst = reinterpret_cast<uint4 *>(P.o + (row * P.Hq + head) * D + half * (D / 2));
+            const uint32_t stage_row = sbase + L::kO + (uint32_t)R * 128u;
 #pragma unroll 1
-                for (int cc = 0; cc < D / 64; ++cc) {
-                    uint32_t a0[32], a1[32];
-                    tmem_ld32(O_COL(0) + lane_off + half * (D / 2) + cc * 32, a0);
-                    tmem_ld32(O_COL(1) + lane_off + half * (D / 2) + cc * 32, a1);
-                    tmem_wait_ld();
-                    if (valid) {
+            for (int cc = 0; cc < D / 64 && ok; ++cc) {
+                uint32_t a0[32], a1[32];
+                tmem_ld32(O_COL(0) + lane_off + half * (D / 2) + cc * 32, a0);
+                tmem_ld32(O_COL(1) + lane_off + half * (D / 2) + cc * 32, a1);
+                tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float v[8];
+                for (int e = 0; e < 4; ++e) {
+                    float v[8];
 #pragma unroll
-                            for (int z = 0; z < 8; ++z)
-                                v[z] = __uint_as_float(a0[8 * e + z]) * g0 + __uint_as_float(a1[8 * e + z]) * g1;
-                            uint4 wv;
-                            wv.x = pack_bf16(v[0], v[1]);
-                            wv.y = pack_bf16(v[2], v[3]);
-                            wv.z = pack_bf16(v[4], v[5]);
-                            wv.w = pack_bf16(v[6], v[7]);
-                            dst[cc * 4 + e] = wv;
-                        }
+                    for (int z = 0; z < 8; ++z)
+                        v[z] = __uint_as_float(a0[8 * e + z]) * g0 + __uint_as_float(a1[8 * e + z]) * g1;
+                    const uint4 wv = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                                                pack_bf16(v[6], v[7]));
+                    if (tma_out) {
+                        // column col of row R: 64-column half col / 64, 16-byte chunk
+                        // j = (col % 64) / 8, stored at chunk j ^ (R % 8) (128-byte swizzle)
+                        const int col = half * (D / 2) + cc * 32 + 8 * e;
+                        const uint32_t hoff = (uint32_t)(col / 64) * kQHalf;
+                        const uint32_t j = (uint32_t)((col % 64) / 8);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stage_row + hoff + ((j ^ (uint32_t)(R & 7)) << 4)),
+                                     "r"(wv.x), "r"(wv.y), "r"(wv.z), "r"(wv.w)
+                                     : "memory");
+                    } else if (valid) {
+                        dst[cc * 4 + e] = wv;
                     }
                 }
-                if (valid && half == 0 && P.lse) P.lse[row * P.Hq + head] = M * P.scale + logf(Lr);
             }
+            if (ok && valid && half == 0 && P.lse) P.lse[row * P.Hq + head] = M * P.scale + logf(Lr);
             // O has been read: the PV issuer may start the next item
             tc_fence_before();
             mbar_arrive(bar(B_OFREE));
+            if (tma_out) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                asm volatile("bar.sync 13, 256;" ::: "memory");
+                if (warp == 0 && lane == 0 && ok) {
+#pragma unroll
+                    for (int hf = 0; hf < D / 64; ++hf)
+                        tma_store_4d(&P.tm_o, sbase + L::kO + hf * kQHalf, hf * 64, U.hkv * P.G, 0, U.goff + U.c0);
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                }
+            }
         }
+        // every store has finished reading shared memory before the CTA exits
+        if (warp == 0 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
 
     // ---- teardown --------------------------------------------------------
@@ -932,7 +974,8 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
               make_map(&P.tm_ksum, ka, D, Hkv, k, chunks, 1, 1, pf::BN) &&
               make_map(&P.tm_kwin, ka, D, Hkv, k, chunks, 1, k, P.Tk) &&
               make_map(&P.tm_vsum, va, D, Hkv, k, chunks, 1, 1, pf::BN) &&
-              make_map(&P.tm_vwin, va, D, Hkv, k, chunks, 1, k, P.Tk);
+              make_map(&P.tm_vwin, va, D, Hkv, k, chunks, 1, k, P.Tk) &&
+              make_map(&P.tm_o, oa, D, Hq, k, chunks, G, k, P.Tc);
     if (!ok) return KSA_ERR_CUDA;
     // persistent: one CTA per SM (shared memory and TMEM admit one); each
     // walks the work items round robin.  CTAs beyond the item count exit.

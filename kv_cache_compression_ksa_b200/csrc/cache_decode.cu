@@ -19,6 +19,7 @@
 #include <math.h>
 
 #include "ksa_internal.cuh"
+#include "warp_mma.cuh"
 
 namespace ksa {
 
@@ -212,29 +213,9 @@ __device__ __forceinline__ bool decode_slice(int kind, int64_t n, int64_t m, int
     return true;
 }
 
-// mma.sync m16n8k16, bf16 inputs, fp32 accumulate (D += A B)
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// 8x8 b16 transpose across the warp, in registers
-__device__ __forceinline__ uint32_t movtrans(uint32_t x)
-{
-    uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-    return y;
-}
-
-__device__ __forceinline__ uint32_t word(const uint4 &u, int i)
-{
-    return i == 0 ? u.x : i == 1 ? u.y : i == 2 ? u.z : u.w;
-}
+using wm::mma16816;
+using wm::movtrans;
+using wm::word;
 
 // Split-K decode on the warp-level tensor-core MMA.  The slice is read with
 // 16-byte loads: lane (g, t) = (lane / 4, lane % 4) loads dims

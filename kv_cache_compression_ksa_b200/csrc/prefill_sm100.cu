@@ -40,6 +40,7 @@
 #include <type_traits>
 
 #include "ksa_internal.cuh"
+#include "warp_mma.cuh"
 
 namespace ksa {
 
@@ -770,8 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
 // ---------------------------------------------------------------------------
 // Summary rows: s_j over the k text rows of its chunk and itself, which are
-// exactly the k+1 contiguous rows of chunk j in the augmented layout.  One
-// warp per (chunk, kv head); CUDA cores (k+1 keys per row).
+// exactly the k+1 contiguous rows of chunk j in the augmented layout.
 // ---------------------------------------------------------------------------
 struct SumArgs {
     int k, G, Hq, Hkv, batch;
@@ -785,16 +785,25 @@ struct SumArgs {
     float *lse;
 };
 
+// One warp per (chunk, kv head) on the warp-level tensor-core MMA: the keys
+// are the MMA rows (S^T = K Q^T, O^T = V^T P^T, G query heads as the 8 MMA
+// columns), 16 keys per step with an online softmax across steps.  Lane
+// (g, t) = (lane / 4, lane % 4) loads dims [32v + 8t, 32v + 8t + 8) of key
+// rows g and g + 8 with 16-byte loads and feeds them to the MMA as they are
+// (the dot product is invariant under a common permutation of d).
+constexpr int kSumWarps = 4;
+
 template <int D, int G>
-__global__ void __launch_bounds__(256) summary_rows_kernel(SumArgs a)
+__global__ void __launch_bounds__(kSumWarps * 32) summary_rows_kernel(SumArgs a)
 {
-    constexpr int EPL = D / 32;  // contiguous elements per lane (8 or 4 bytes)
-    constexpr int RG = 8;        // key rows loaded together
-    using Vec = typename std::conditional<EPL == 4, uint2, uint32_t>::type;
+    static_assert(G <= 8, "query heads per kv head must fit the 8 MMA columns");
+    constexpr int NV = D / 32, NC = D / 16, NM = D / 16;
+    __shared__ float s_o[kSumWarps][G][D];
+    __shared__ float s_ml[kSumWarps][2][G];
     if (*a.err != 0) return;
-    const int64_t task = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (task >= a.chunks * a.Hkv) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t task = (int64_t)blockIdx.x * kSumWarps + warp;
+    if (task >= a.chunks * a.Hkv) return;   // warp-uniform; only warp-level syncs below
     const int64_t gc = task / a.Hkv;
     const int h = (int)(task % a.Hkv);
     int lo = 0, hi = a.batch - 1;
@@ -807,101 +816,118 @@ __global__ void __launch_bounds__(256) summary_rows_kernel(SumArgs a)
     if (gc - a.pl.chunk_off[b] >= n / a.k) return;  // trailing partial chunk: no summary
     const int64_t row0 = gc * (a.k + 1);
     const int64_t srow = row0 + a.k;
-    auto unpack = [](Vec v, float *f) {
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(&v);
+    const int g = lane >> 2, tt = lane & 3;
+    // B fragments of Q^T: column (head) g, k-chunk c = 2v + hh covers dims
+    // 32v + 8tt + 4hh + {0,1} (b0) and {2,3} (b1): two bf16 words of q
+    uint32_t qb[NC][2];
 #pragma unroll
-        for (int i = 0; i < EPL / 2; ++i) {
-            f[2 * i] = __uint_as_float(w[i] << 16);
-            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    for (int c = 0; c < NC; ++c) {
+        const int d0 = 32 * (c / 2) + 8 * tt + 4 * (c % 2);
+        if (g < G) {
+            const uint32_t *qp = reinterpret_cast<const uint32_t *>(a.q + (srow * a.Hq + (int64_t)h * G + g) * D + d0);
+            qb[c][0] = qp[0];
+            qb[c][1] = qp[1];
+        } else {
+            qb[c][0] = qb[c][1] = 0u;
         }
-    };
-    float qv[G][EPL];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const Vec *qp = reinterpret_cast<const Vec *>(a.q + (srow * a.Hq + h * G + g) * D) + lane;
-        unpack(*qp, qv[g]);
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) qv[g][e] *= a.scale_log2;
     }
-    float m[G], l[G], acc[G][EPL];
+    float o[NM][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        m[g] = -INFINITY; l[g] = 0.f;
+    for (int i = 0; i < NM; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};   // heads 2tt, 2tt + 1 (log2 units)
+    const int64_t rstride = (int64_t)a.Hkv * (D / 8);   // uint4 per augmented row
+    const uint4 *Kb = reinterpret_cast<const uint4 *>(a.kk) + row0 * rstride + (int64_t)h * (D / 8);
+    const uint4 *Vb = reinterpret_cast<const uint4 *>(a.v) + row0 * rstride + (int64_t)h * (D / 8);
+    // keys: rows 0 .. k of the chunk (its k text rows, then the summary itself)
+    for (int kb = 0; kb <= a.k; kb += 16) {
+        const int r0 = kb + g, r1 = kb + g + 8;
+        const bool in0 = r0 <= a.k, in1 = r1 <= a.k;
+        uint4 kA[NV], kB[NV], vA[NV], vB[NV];
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[g][e] = 0.f;
-    }
-    // the k+1 keys of s_j: rows 0..k of its chunk (k text rows, then itself)
-    for (int t0 = 0; t0 <= a.k; t0 += RG) {
-        Vec kr[RG], vr[RG];
-#pragma unroll
-        for (int r = 0; r < RG; ++r) {
-            const int t = t0 + r;
-            if (t <= a.k) {
-                kr[r] = reinterpret_cast<const Vec *>(a.kk + ((row0 + t) * a.Hkv + h) * D)[lane];
-                vr[r] = reinterpret_cast<const Vec *>(a.v + ((row0 + t) * a.Hkv + h) * D)[lane];
-            } else {
-                kr[r] = Vec{}; vr[r] = Vec{};
-            }
+        for (int v = 0; v < NV; ++v) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            kA[v] = in0 ? Kb[r0 * rstride + 4 * v + tt] : z;
+            kB[v] = in1 ? Kb[r1 * rstride + 4 * v + tt] : z;
+            vA[v] = in0 ? Vb[r0 * rstride + 4 * v + tt] : z;
+            vB[v] = in1 ? Vb[r1 * rstride + 4 * v + tt] : z;
         }
-        float sc[G][RG];
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int r = 0; r < RG; ++r) {
-            float kf[EPL];
-            unpack(kr[r], kf);
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                float s = 0.f;
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) s = fmaf(qv[g][e], kf[e], s);
-                sc[g][r] = s;
-            }
+        for (int c = 0; c < NC; ++c) {
+            const int v = c / 2, hh = c % 2;
+            wm::mma16816(sc, wm::word(kA[v], 2 * hh), wm::word(kB[v], 2 * hh), wm::word(kA[v], 2 * hh + 1),
+                         wm::word(kB[v], 2 * hh + 1), qb[c][0], qb[c][1]);
         }
+        // sc[0..1]: key r0, heads 2tt, 2tt+1; sc[2..3]: key r1
+        float x[4];
+        x[0] = in0 ? sc[0] * a.scale_log2 : -INFINITY;
+        x[1] = in0 ? sc[1] * a.scale_log2 : -INFINITY;
+        x[2] = in1 ? sc[2] * a.scale_log2 : -INFINITY;
+        x[3] = in1 ? sc[3] * a.scale_log2 : -INFINITY;
+        float corr[2], pv[4];
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1)
+        for (int e = 0; e < 2; ++e) {
+            float mx = fmaxf(x[e], x[e + 2]);
 #pragma unroll
-            for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int r = 0; r < RG; ++r) sc[g][r] += __shfl_xor_sync(0xffffffffu, sc[g][r], off);
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float mx = m[g];
-#pragma unroll
-            for (int r = 0; r < RG; ++r) {
-                if (t0 + r > a.k) sc[g][r] = -INFINITY;
-                mx = fmaxf(mx, sc[g][r]);
-            }
-            const float corr = ex2(m[g] - mx);  // m = -inf on the first group: 0
-            l[g] *= corr;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[g][e] *= corr;
-            m[g] = mx;
-#pragma unroll
-            for (int r = 0; r < RG; ++r) {
-                sc[g][r] = ex2(sc[g][r] - mx);
-                l[g] += sc[g][r];
-            }
+            for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float m_new = fmaxf(m_run[e], mx);   // finite: key 0 is always present
+            corr[e] = wm::ex2(m_run[e] - m_new);       // 0 on the first step
+            pv[e] = wm::ex2(x[e] - m_new);
+            pv[e + 2] = wm::ex2(x[e + 2] - m_new);
+            l_run[e] = l_run[e] * corr[e] + pv[e] + pv[e + 2];
+            m_run[e] = m_new;
         }
 #pragma unroll
-        for (int r = 0; r < RG; ++r) {
-            float vf[EPL];
-            unpack(vr[r], vf);
+        for (int i = 0; i < NM; ++i) {
+            o[i][0] *= corr[0]; o[i][1] *= corr[1];
+            o[i][2] *= corr[0]; o[i][3] *= corr[1];
+        }
+        const uint32_t pb0 = wm::movtrans(wm::pack2(pv[0], pv[1]));
+        const uint32_t pb1 = wm::movtrans(wm::pack2(pv[2], pv[3]));
 #pragma unroll
-            for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) acc[g][e] = fmaf(sc[g][r], vf[e], acc[g][e]);
+        for (int i = 0; i < NM; ++i) {
+            const int v = i / 2, pp = i % 2;
+            wm::mma16816(o[i], wm::movtrans(wm::word(vA[v], 2 * pp)), wm::movtrans(wm::word(vA[v], 2 * pp + 1)),
+                         wm::movtrans(wm::word(vB[v], 2 * pp)), wm::movtrans(wm::word(vB[v], 2 * pp + 1)), pb0, pb1);
         }
     }
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const int head = h * G + g;
-        const float inv = 1.f / l[g];
-        Vec out;
-        uint32_t *w = reinterpret_cast<uint32_t *>(&out);
+    for (int e = 0; e < 2; ++e)
 #pragma unroll
-        for (int i = 0; i < EPL / 2; ++i) w[i] = pack_bf16(acc[g][2 * i] * inv, acc[g][2 * i + 1] * inv);
-        reinterpret_cast<Vec *>(a.o + (srow * a.Hq + head) * D)[lane] = out;
-        if (a.lse && lane == 0) a.lse[srow * a.Hq + head] = m[g] * 0.69314718055994530942f + logf(l[g]);
+        for (int off = 4; off < 32; off <<= 1) l_run[e] += __shfl_xor_sync(0xffffffffu, l_run[e], off);
+    // O^T rows: m-tile i = (v, pp), row g -> dim 32v + 8(g/2) + 4pp + (g%2), row g+8 -> that + 2
+#pragma unroll
+    for (int i = 0; i < NM; ++i) {
+        const int v = i / 2, pp = i % 2;
+        const int dA = 32 * v + 8 * (g / 2) + 4 * pp + (g % 2);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int head = 2 * tt + e;
+            if (head < G) {
+                s_o[warp][head][dA] = o[i][e];
+                s_o[warp][head][dA + 2] = o[i][2 + e];
+            }
+        }
     }
+    if (g == 0) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+            if (2 * tt + e < G) {
+                s_ml[warp][0][2 * tt + e] = m_run[e];
+                s_ml[warp][1][2 * tt + e] = l_run[e];
+            }
+    }
+    __syncwarp();
+    // the G output rows of s_j: bf16 pairs, 128 contiguous bytes per instruction
+    for (int idx = lane; idx < G * (D / 2); idx += 32) {
+        const int gg = idx / (D / 2), w2 = idx % (D / 2);
+        const float inv = 1.f / s_ml[warp][1][gg];
+        const uint32_t pr = wm::pack2(s_o[warp][gg][2 * w2] * inv, s_o[warp][gg][2 * w2 + 1] * inv);
+        reinterpret_cast<uint32_t *>(a.o + (srow * a.Hq + (int64_t)h * G + gg) * D)[w2] = pr;
+    }
+    if (a.lse && lane < G)
+        a.lse[srow * a.Hq + (int64_t)h * G + lane] =
+            (s_ml[warp][0][lane] + log2f(s_ml[warp][1][lane])) * 0.69314718055994530942f;
 }
 
 }  // namespace pf
@@ -1000,12 +1026,13 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
     s.o = (__nv_bfloat16 *)oa; s.lse = lse;
     int64_t tasks = chunks * Hkv;
     if (tasks > 0) {
-        const unsigned blocks = (unsigned)((tasks + 7) / 8);
+        const unsigned blocks = (unsigned)((tasks + pf::kSumWarps - 1) / pf::kSumWarps);
+        const unsigned thr = pf::kSumWarps * 32;
         switch (G) {
-        case 1: pf::summary_rows_kernel<D, 1><<<blocks, 256, 0, st>>>(s); break;
-        case 2: pf::summary_rows_kernel<D, 2><<<blocks, 256, 0, st>>>(s); break;
-        case 4: pf::summary_rows_kernel<D, 4><<<blocks, 256, 0, st>>>(s); break;
-        case 8: pf::summary_rows_kernel<D, 8><<<blocks, 256, 0, st>>>(s); break;
+        case 1: pf::summary_rows_kernel<D, 1><<<blocks, thr, 0, st>>>(s); break;
+        case 2: pf::summary_rows_kernel<D, 2><<<blocks, thr, 0, st>>>(s); break;
+        case 4: pf::summary_rows_kernel<D, 4><<<blocks, thr, 0, st>>>(s); break;
+        case 8: pf::summary_rows_kernel<D, 8><<<blocks, thr, 0, st>>>(s); break;
         default: return KSA_ERR_UNSUPPORTED;
         }
         if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;

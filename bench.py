@@ -31,6 +31,14 @@ sys.path.insert(0, ROOT)
 
 # workloads
 PF = dict(seqlens=[32768], k=8, w=8, Hq=32, Hkv=8, d=128, scale=0.5, seed=1, theta=1e6)
+# DRAM bytes (read + write) per launch of the dominant kernels, from the ncu
+# captures summarised under profiles/ for the kernels as they now stand (to be
+# set to None whenever one of those kernels changes, until it is captured again).
+# The decode capture ran at batch 16; its traffic grows in proportion to the batch.
+TRAFFIC = {
+    "prefill": (660.3e6, "profiles/prefill_kernel_qwen3_4b_32k.md (prefill_kernel<128>)"),
+    "decode_per_seq": (1.0851e9 / 16, "profiles/decode_split_kernel_b16_m16384.md (batch 16 capture, per sequence)"),
+}
 DC = dict(B=64, m=16384, k=8, w=8, Hq=32, Hkv=8, d=128, seed=3, theta=1e6)
 
 
@@ -361,11 +369,14 @@ def run_ksa(args, rank, world, local):
             "decode": {"ms": dec_ms, "append_ms": app_ms, "gbs": dec_gbs / world,
                        "frac_of_hbm_peak": (dec_gbs / world) / hbm_peak, "batch": B, "summaries": m},
             "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": tc_peak, "unit": "TFLOP/s",
-                         "frac": kern_tflops / tc_peak, "traffic": None,
+                         "frac": kern_tflops / tc_peak,
+                         "traffic": TRAFFIC["prefill"][0], "traffic_source": TRAFFIC["prefill"][1],
                          "kernel": "prefill_kernel<128> (text rows; time of the ksa_prefill_fwd call)",
                          "peak_source": f"{peak_src} burst bf16", "peak_sustained": tc_sus},
             "roofline_decode": {"bound": "hbm", "achieved": dec_gbs / world, "peak": hbm_peak, "unit": "GB/s",
-                                "frac": (dec_gbs / world) / hbm_peak, "traffic": None,
+                                "frac": (dec_gbs / world) / hbm_peak,
+                                "traffic": (TRAFFIC["decode_per_seq"][0] * B if m == DC["m"] else None),
+                                "traffic_source": TRAFFIC["decode_per_seq"][1],
                                 "kernel": "decode_split_kernel<128,4> + combine (time of ksa_decode)"},
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h), "ms": e2e_ms},
@@ -383,6 +394,131 @@ def run_ksa(args, rank, world, local):
         print(json.dumps(line))
 
 
+# ---------------------------------------------------------------------------
+# sweep (not the bench line): the long varlen prefill batch and the decode
+# grid of batch x context, one JSON line per point
+# ---------------------------------------------------------------------------
+SWEEP_PREFILL = [
+    dict(name="varlen 131072+65536+16384+4000", seqlens=[131072, 65536, 16384, 4000], k=8, w=16, seed=2),
+    dict(name="varlen 131072+65536+16384+4003", seqlens=[131072, 65536, 16384, 4003], k=8, w=16, seed=2),
+]
+SWEEP_DECODE = dict(batches=[1, 16, 128], contexts=[4096, 32768, 131072, 1048576], k=8, w=8, Hq=32, Hkv=8,
+                    d=128, seed=7, text_steps=64)
+
+
+def run_sweep(args):
+    import torch
+    from kv_cache_compression_ksa_b200 import _lib as L
+    from kv_cache_compression_ksa_b200 import api, build
+    from kv_cache_compression_ksa_b200.inputs import fill_normal_, prefill_inputs, uniform_ints
+
+    build.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    hbm_peak, tc_peak, tc_sus, peak_src = load_peaks()
+    Hq, Hkv, d = 32, 8, 128
+
+    def ev_time(fn, warm=3, reps=10):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return float(np.median(ts))
+
+    for cfg in SWEEP_PREFILL:
+        sl, k, w = cfg["seqlens"], cfg["k"], cfg["w"]
+        x = prefill_inputs(sl, k, Hq, Hkv, d, seed=cfg["seed"], scale=1.0, device=dev)
+        p = L.make_params(k, w, Hq, Hkv, d, 0.0, 1e6)
+        nt, ns = sum(sl), sum(n // k for n in sl)
+        rows = L.ksa_aug_rows(p, sl)
+        qa = torch.empty(rows, Hq, d, dtype=torch.bfloat16, device=dev)
+        ka = torch.empty(rows, Hkv, d, dtype=torch.bfloat16, device=dev)
+        va = torch.empty_like(ka)
+        oa = torch.empty_like(qa)
+        lse = torch.empty(rows, Hq, dtype=torch.float32, device=dev)
+        ws = torch.empty(L.ksa_prefill_workspace_size(p, len(sl), nt), dtype=torch.uint8, device=dev)
+        rope_ms = ev_time(lambda: L.ksa_interleave_rope(p, x.cu_seqlens, nt, ns, rows, x.q_text, x.k_text, x.v_text,
+                                                        x.q_sum, x.k_sum, x.v_sum, qa, ka, va, ws))
+        ms = ev_time(lambda: L.ksa_prefill_fwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, ws))
+        flops = useful_pairs(sl, k, w) * Hq * 4 * d
+        tf = flops / (ms * 1e-3) / 1e12
+        print(json.dumps({"sweep": "prefill", "workload": cfg["name"] + f", 32q/8kv, d128, k{k}, w{w}, N(0,1) bf16",
+                          "useful_tflop": flops / 1e12, "ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / tc_peak,
+                          "rope_interleave_ms": rope_ms}), flush=True)
+        del x, qa, ka, va, oa, lse, ws
+        torch.cuda.empty_cache()
+
+    S = SWEEP_DECODE
+    k, w = S["k"], S["w"]
+    pd = L.make_params(k, w, S["Hq"], S["Hkv"], S["d"], 0.0, 1e6)
+    cycle = k + 1                       # k TEXT steps and one SUMMARY step per chunk
+    nsteps = S["text_steps"] // k * cycle
+    replays = 4
+    for B in S["batches"]:
+        for n in S["contexts"]:
+            m = n // k
+            extra = (replays + 2) * (S["text_steps"] // k)
+            cache = api.DecodeCache(pd, B, cap=m + extra, device=dev)
+            fill_normal_(cache.k, 1000 + B)
+            fill_normal_(cache.v, 2000 + B)
+            fills = uniform_ints(B, 0, k - 1, seed=S["seed"]).numpy()
+            state0 = torch.zeros(B, 4, dtype=torch.int32)
+            state0[:, 0] = torch.as_tensor(m * k + fills, dtype=torch.int32)
+            state0[:, 1] = m
+            cache.state.copy_(state0.to(dev))
+            # per step and sequence: SUMMARY when its open chunk is full, else TEXT;
+            # nsteps is a whole number of cycles, so every replay starts from the same fills
+            kinds = np.zeros((nsteps, B), np.int8)
+            nbytes = 0.0
+            f = fills.copy()
+            mm = np.full(B, m, np.int64)
+            for j in range(nsteps):
+                full = f == k
+                kinds[j] = np.where(full, 1, 0)
+                rows_j = np.where(full, k + 1, f + 1 + np.minimum(mm, w) * k + np.maximum(0, mm - w))
+                nbytes += float(rows_j.sum()) * S["Hkv"] * S["d"] * 2 * 2
+                mm = np.where(full, mm + 1, mm)
+                f = np.where(full, 0, f + 1)
+            kinds_d = torch.as_tensor(kinds, device=dev)
+            gen = torch.Generator(device=dev).manual_seed(S["seed"])
+            kn = torch.randn(B, S["Hkv"], S["d"], generator=gen, device=dev).to(torch.bfloat16)
+            vn = torch.randn(B, S["Hkv"], S["d"], generator=gen, device=dev).to(torch.bfloat16)
+            qd = torch.randn(B, S["Hq"], S["d"], generator=gen, device=dev).to(torch.bfloat16)
+            max_text = (m + extra + 1) * k
+            dws = cache.workspace(max_text)
+            od = torch.empty(B, S["Hq"], S["d"], dtype=torch.bfloat16, device=dev)
+            lsed = torch.empty(B, S["Hq"], dtype=torch.float32, device=dev)
+
+            def steps():
+                for j in range(nsteps):
+                    L.ksa_cache_append(pd, cache.desc, kinds_d[j], kn, vn)
+                    L.ksa_decode(pd, cache.desc, kinds_d[j], qd, od, lsed, max_text, dws)
+
+            steps()   # eager pass: loads the kernels, advances one whole number of cycles
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                steps()
+            ms = ev_time(g.replay, warm=1, reps=replays - 1)
+            st = cache.state.cpu().numpy()
+            assert (st[:, 3] == 0).all(), f"cache state error {st[:, 3]}"
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            print(json.dumps({"sweep": "decode", "batch": B, "context": n, "summaries": m,
+                              "text_steps": S["text_steps"], "summary_steps": nsteps - S["text_steps"],
+                              "ms_per_text_step": ms / S["text_steps"], "graph_ms": ms,
+                              "gb_per_graph": nbytes / 1e9, "gbs": gbs, "frac_of_hbm_peak": gbs / hbm_peak}),
+                  flush=True)
+            del g, cache, dws, kinds_d, kn, vn, qd, od, lsed
+            torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -394,7 +530,12 @@ def main():
                     help="time one leg only (profiling); the JSON line then covers that leg")
     ap.add_argument("--profile", action="store_true", help="skip the e2e and CPU legs (for ncu runs)")
     ap.add_argument("--decode-batch", type=int, default=DC["B"])
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the long varlen prefill batch and the decode batch x context grid (one JSON line per point)")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", 0))
         world = int(os.environ.get("WORLD_SIZE", 1))

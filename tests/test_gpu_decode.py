@@ -151,12 +151,13 @@ def _prefilled_cache(B, k, w, Hq, Hkv, d, m_chunks, fills, seed):
     return p, cache
 
 
-@pytest.mark.parametrize("B,m_chunks,nsample", [(64, 16384, 6), (3, 40, 3)])
+@pytest.mark.parametrize("B,m_chunks,nsample", [(64, 16384, 6), (2, 131072, 2), (3, 40, 3)])
 def test_decode_full_size_against_cache_model(B, m_chunks, nsample):
     """The long-context decode step (64 sequences, 16384 summaries each, full
-    64-token ring, fill 0..7): one TEXT append + decode in the launch
-    configuration the benchmark times, checked on sampled sequences against
-    the oracle's cache-model decode of the same cache image."""
+    64-token ring, fill 0..7; and the 1M-token context, 131072 summaries, of
+    the decode sweep): one TEXT append + decode in the launch configuration
+    the benchmark times, checked on sampled sequences against the oracle's
+    cache-model decode of the same cache image."""
     k, w, Hq, Hkv, d = 8, 8, 32, 8, 128
     fills = uniform_ints(B, 0, k - 1, seed=3).numpy()
     p, cache = _prefilled_cache(B, k, w, Hq, Hkv, d, m_chunks, fills, seed=9)

@@ -452,7 +452,15 @@ def run_sweep(args):
         print(json.dumps({"sweep": "prefill", "workload": cfg["name"] + f", 32q/8kv, d128, k{k}, w{w}, N(0,1) bf16",
                           "useful_tflop": flops / 1e12, "ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / tc_peak,
                           "rope_interleave_ms": rope_ms}), flush=True)
-        del x, qa, ka, va, oa, lse, ws
+        # prefill -> decode hand-off of the same batch: bytes read and written
+        cache = api.DecodeCache(p, len(sl), cap=max(n // k for n in sl) + 8, device=dev)
+        hms = ev_time(lambda: cache.from_prefill(x.cu_seqlens, nt, ka, va, ws))
+        hrows = sum(n // k + min(n // k, w) * k + (n - (n // k) * k) for n in sl)
+        hbytes = hrows * Hkv * d * 2 * 2 * 2
+        print(json.dumps({"sweep": "handoff", "workload": cfg["name"] + f", Hkv 8, d128, k{k}, w{w}",
+                          "rows": hrows, "ms": hms, "gbs": hbytes / (hms * 1e-3) / 1e9,
+                          "frac_of_hbm_peak": hbytes / (hms * 1e-3) / 1e9 / hbm_peak}), flush=True)
+        del x, qa, ka, va, oa, lse, ws, cache
         torch.cuda.empty_cache()
 
     S = SWEEP_DECODE

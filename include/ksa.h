@@ -174,6 +174,25 @@ KSA_API int64_t ksa_cache_slots(const ksa_params *p, int64_t cap_summaries);
 KSA_API int ksa_cache_append(const ksa_params *p, const ksa_cache *cache, const int8_t *kind,
                      const void *k_new, const void *v_new, void *stream);
 
+/* Build the decode cache of a prefilled batch in one pass: the hand-off from
+ * prefill to decode (the report fills the cache token by token, Figure 4;
+ * this writes the state that sequence of appends reaches, section 2.3.1).
+ * k_aug, v_aug: the augmented K/V that ksa_interleave_rope wrote for the same
+ * cu_seqlens (device int32 [cache->batch + 1]), i.e. already rotated.  For
+ * sequence b with n_b text tokens, m_b = floor(n_b / k) summaries and
+ * f_b = n_b - m_b k open tokens it writes: summary s_j at slot 1+k+w*k+j;
+ * chunk c of its last min(m_b, w) complete chunks at ring block c mod w,
+ * token r at slot k+1+(c mod w)*k+(k-1-r); open token r at slot k - r; and
+ * state[b] = {n_b, m_b, 0, 0}.  Other slots are left as they are (they hold
+ * nothing a later decode reads).  A sequence with m_b > cap_summaries is
+ * not written and gets state[b].err = KSA_ERR_CAPACITY.  workspace:
+ * ksa_prefill_workspace_size(p, batch, total_text) bytes; dev_err as for
+ * ksa_interleave_rope (an inconsistent cu_seqlens sets KSA_ERR_INVALID
+ * there and nothing is written). */
+KSA_API int ksa_cache_from_prefill(const ksa_params *p, const ksa_cache *cache, const int32_t *cu_seqlens,
+                           int64_t total_text, int64_t aug_rows, const void *k_aug, const void *v_aug,
+                           void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream);
+
 /* Workspace bytes for ksa_decode when no sequence has more than max_text
  * text tokens. */
 KSA_API size_t ksa_decode_workspace_size(const ksa_params *p, int32_t batch, int64_t max_text);

@@ -71,6 +71,8 @@ SYMBOLS = {
                                        _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "ksa_cache_slots": (_I64, [ctypes.POINTER(ksa_params), _I64]),
     "ksa_cache_append": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _P, _P, _P]),
+    "ksa_cache_from_prefill": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _I64, _I64,
+                                              _P, _P, _P, _SZ, _P, _P]),
     "ksa_decode_workspace_size": (_SZ, [ctypes.POINTER(ksa_params), _I32, _I64]),
     "ksa_decode": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _P, _P, _P,
                                   _I64, _P, _SZ, _P]),
@@ -173,6 +175,14 @@ def ksa_cache_append(p, cache: ksa_cache, kind, k_new, v_new, stream=None):
     rc = load().ksa_cache_append(ctypes.byref(p), ctypes.byref(cache), _ptr(kind), _ptr(k_new), _ptr(v_new),
                                  _stream(stream))
     _check("ksa_cache_append", rc)
+
+
+def ksa_cache_from_prefill(p, cache: ksa_cache, cu_seqlens, total_text, aug_rows, k_aug, v_aug, workspace,
+                           dev_err=None, stream=None):
+    rc = load().ksa_cache_from_prefill(ctypes.byref(p), ctypes.byref(cache), _ptr(cu_seqlens), total_text, aug_rows,
+                                       _ptr(k_aug), _ptr(v_aug), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _ptr(dev_err), _stream(stream))
+    _check("ksa_cache_from_prefill", rc)
 
 
 def ksa_decode_workspace_size(p: ksa_params, batch: int, max_text: int) -> int:

@@ -69,6 +69,12 @@ class DecodeCache:
     def append(self, kind, k_new, v_new, stream=None):
         L.ksa_cache_append(self.p, self.desc, kind, k_new, v_new, stream=stream)
 
+    def from_prefill(self, cu_seqlens, total_text: int, k_aug, v_aug, workspace, stream=None):
+        """Fill the cache with the state a prefill of these sequences leaves
+        (k_aug / v_aug: the rotated augmented K/V of ksa_interleave_rope)."""
+        L.ksa_cache_from_prefill(self.p, self.desc, cu_seqlens, total_text, k_aug.shape[0], k_aug, v_aug, workspace,
+                                 stream=stream)
+
     def workspace(self, max_text: int):
         n = L.ksa_decode_workspace_size(self.p, self.batch, max_text)
         return torch.empty(max(n, 16), dtype=torch.uint8, device=self.k.device)

@@ -148,6 +148,98 @@ int launch_cache_append(const ksa_params *p, const ksa_cache *c, const int8_t *k
 }
 
 // ---------------------------------------------------------------------------
+// Hand-off: the decode cache of a prefilled batch in one pass.  Sequence b
+// (blockIdx.y) lists its rows as: m summaries, then the k tokens of each of
+// its last R = min(m, w) complete chunks, then its f open tokens; every
+// (row, kv head, 16-byte piece) is one item of a grid-stride loop, so one
+// warp copies 512 contiguous bytes of a source row (two heads) and writes
+// each head's 256 bytes to its own slot.  HBM-bound copy.
+// ---------------------------------------------------------------------------
+struct BuildArgs {
+    int k, w, Hkv, D8;        // D8: 16-byte pieces per head row
+    int64_t S, cap;
+    const int32_t *cu;
+    Plan pl;
+    const int32_t *err;
+    const uint4 *ka, *va;     // [aug_rows, Hkv, d]
+    uint4 *K, *V;             // [B, Hkv, S, d]
+    int32_t *state;
+};
+
+constexpr int kBuildThreads = 256;
+
+__global__ void __launch_bounds__(kBuildThreads) cache_build_kernel(BuildArgs a)
+{
+    const int b = blockIdx.y;
+    if (*a.err != 0) return;   // the plan found cu_seqlens inconsistent
+    const int n = a.cu[b + 1] - a.cu[b];
+    const int k = a.k, m = n / k, f = n - m * k;
+    const int64_t cs = a.pl.chunk_off[b];
+    const bool lead = blockIdx.x == 0 && threadIdx.x == 0;
+    if ((int64_t)m > a.cap) {
+        if (lead) a.state[4 * (int64_t)b + 3] = KSA_ERR_CAPACITY;
+        return;
+    }
+    if (lead) {
+        a.state[4 * (int64_t)b + 0] = n;
+        a.state[4 * (int64_t)b + 1] = m;
+        a.state[4 * (int64_t)b + 2] = 0;
+        a.state[4 * (int64_t)b + 3] = 0;
+    }
+    const int R = min(m, a.w);
+    const int64_t rows = (int64_t)m + (int64_t)R * k + f;
+    const int64_t total = rows * a.Hkv * a.D8;
+    for (int64_t it = (int64_t)blockIdx.x * kBuildThreads + threadIdx.x; it < total;
+         it += (int64_t)gridDim.x * kBuildThreads) {
+        const int j = (int)(it % a.D8);
+        const int64_t t = it / a.D8;
+        const int h = (int)(t % a.Hkv);
+        const int64_t idx = t / a.Hkv;
+        int64_t src_row, slot;
+        if (idx < m) {                       // summary s_idx
+            src_row = (cs + idx) * (k + 1) + k;
+            slot = 1 + k + (int64_t)a.w * k + idx;
+        } else if (idx < m + (int64_t)R * k) {   // ring: chunk c, token r
+            const int64_t q = idx - m;
+            const int64_t c = m - R + q / k;
+            const int r = (int)(q % k);
+            src_row = (cs + c) * (k + 1) + r;
+            slot = k + 1 + (c % a.w) * k + (k - 1 - r);
+        } else {                             // open chunk m, token r
+            const int r = (int)(idx - m - (int64_t)R * k);
+            src_row = (cs + m) * (k + 1) + r;
+            slot = k - r;
+        }
+        const int64_t src = (src_row * a.Hkv + h) * a.D8 + j;
+        const int64_t dst = (((int64_t)b * a.Hkv + h) * a.S + slot) * a.D8 + j;
+        a.K[dst] = a.ka[src];
+        a.V[dst] = a.va[src];
+    }
+}
+
+int launch_cache_build(const ksa_params *p, const ksa_cache *c, const int32_t *cu, const void *k_aug,
+                       const void *v_aug, const Plan &pl, int32_t *err, cudaStream_t st)
+{
+    if (c->batch == 0) return KSA_OK;
+    BuildArgs a;
+    a.k = p->k; a.w = p->w; a.Hkv = p->num_kv_heads; a.D8 = p->head_dim / 8;
+    a.S = ksa_cache_slots(p, c->cap_summaries);
+    a.cap = c->cap_summaries;
+    a.cu = cu; a.pl = pl; a.err = err;
+    a.ka = (const uint4 *)k_aug; a.va = (const uint4 *)v_aug;
+    a.K = (uint4 *)c->k; a.V = (uint4 *)c->v;
+    a.state = c->state;
+    // rows per sequence are at most cap + w k + k; the grid-stride loop covers the rest
+    const int64_t max_items = (c->cap_summaries + (int64_t)p->w * p->k + p->k) * a.Hkv * a.D8;
+    int64_t gx = (max_items + kBuildThreads - 1) / kBuildThreads;
+    const int64_t gmax = 4LL * sm_count();
+    if (gx > gmax) gx = gmax;
+    if (gx < 1) gx = 1;
+    cache_build_kernel<<<dim3((unsigned)gx, (unsigned)c->batch), kBuildThreads, 0, st>>>(a);
+    return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 // Decode: split-K over the contiguous slice.
 //
 // Grid (nsplit, Hkv, B); 4 warps per CTA, each taking 16 key rows per step.

@@ -173,6 +173,29 @@ int ksa_cache_append(const ksa_params *p, const ksa_cache *cache, const int8_t *
     return launch_cache_append(p, cache, kind, k_new, v_new, (cudaStream_t)stream);
 }
 
+int ksa_cache_from_prefill(const ksa_params *p, const ksa_cache *cache, const int32_t *cu_seqlens,
+                           int64_t total_text, int64_t aug_rows, const void *k_aug, const void *v_aug,
+                           void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream)
+{
+    int rc = check_params(p);
+    if (rc != KSA_OK) return rc;
+    if (!cache || cache->batch < 0 || cache->cap_summaries < 0) return KSA_ERR_INVALID;
+    if (cache->batch == 0) return KSA_OK;
+    if (!cache->k || !cache->v || !cache->state || !aligned16(cache->k) || !aligned16(cache->v)) return KSA_ERR_INVALID;
+    if (cache->batch > 65535) return KSA_ERR_UNSUPPORTED;
+    if ((cache->cap_summaries + 1) * (int64_t)p->k > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+    rc = check_prefill_common(p, cache->batch, cu_seqlens, total_text, aug_rows, workspace, workspace_bytes);
+    if (rc != KSA_OK) return rc;
+    if (aug_rows > 0 && (!k_aug || !v_aug || !aligned16(k_aug) || !aligned16(v_aug))) return KSA_ERR_INVALID;
+    if (reinterpret_cast<uintptr_t>(dev_err) & 3u) return KSA_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    Plan pl = plan_view(workspace, cache->batch);
+    int32_t *err = dev_err ? dev_err : pl.err;
+    rc = launch_plan(p, cache->batch, cu_seqlens, total_text, -1, aug_rows, pl, err, 0, st);
+    if (rc != KSA_OK) return rc;
+    return launch_cache_build(p, cache, cu_seqlens, k_aug, v_aug, pl, err, st);
+}
+
 size_t ksa_decode_workspace_size(const ksa_params *p, int32_t batch, int64_t max_text)
 {
     if (check_params(p) != KSA_OK || batch < 0 || max_text < 0) return 0;

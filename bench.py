@@ -401,6 +401,10 @@ def run_ksa(args, rank, world, local):
 SWEEP_PREFILL = [
     dict(name="varlen 131072+65536+16384+4000", seqlens=[131072, 65536, 16384, 4000], k=8, w=16, seed=2),
     dict(name="varlen 131072+65536+16384+4003", seqlens=[131072, 65536, 16384, 4003], k=8, w=16, seed=2),
+    dict(name="1x32768, sliding chunk number 128", seqlens=[32768], k=8, w=128, seed=1),
+    dict(name="1x32768, chunk 16", seqlens=[32768], k=16, w=8, seed=1),
+    dict(name="1x32768, chunk 32", seqlens=[32768], k=32, w=8, seed=1),
+    dict(name="1x32768, chunk 64 (q heads split over 2 tiles)", seqlens=[32768], k=64, w=8, seed=1),
 ]
 SWEEP_DECODE = dict(batches=[1, 16, 128], contexts=[4096, 32768, 131072, 1048576], k=8, w=8, Hq=32, Hkv=8,
                     d=128, seed=7, text_steps=64)

@@ -30,9 +30,11 @@
  *     a full summary buffer, a pipeline wait that ran out) never trap: the
  *     kernel records a KSA_ERR_* code in a device error word and skips the
  *     affected work.  ksa_get_device_error() reads and clears such a word.
- *   - Supported: head_dim 64 or 128; num_q_heads % num_kv_heads == 0;
- *     k >= 1; w >= 0; for prefill k <= 64 and (num_q_heads/num_kv_heads) * k
- *     <= 128.
+ *   - Supported: head_dim 64 or 128; num_q_heads % num_kv_heads == 0 with
+ *     at most 8 q heads per kv head; k >= 1; w >= 0; for prefill k <= 128
+ *     and 1, 2, 4 or 8 q heads per kv head (when (q heads per kv head) * k
+ *     exceeds 128 rows, a kv head's q heads are split over several query
+ *     tiles, each reading the same key/value tiles).
  */
 #ifndef KSA_H
 #define KSA_H

@@ -39,8 +39,10 @@ static int check_params(const ksa_params *p)
 
 static int check_prefill_shape(const ksa_params *p)
 {
-    int G = p->num_q_heads / p->num_kv_heads;
-    if (G * p->k > 128 || p->k > 64) return KSA_ERR_UNSUPPORTED;
+    // query tiles hold min(G, 128/k) heads of k slots; G must split evenly
+    if (prefill_heads_per_tile(p) < 1) return KSA_ERR_UNSUPPORTED;
+    const int G = p->num_q_heads / p->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return KSA_ERR_UNSUPPORTED;   // summary-row kernel
     return KSA_OK;
 }
 

@@ -45,6 +45,7 @@ inline Plan plan_view(void *ws, int batch)
 // Chunks covered by one prefill work unit (all rows of a unit share one kv
 // head); set by the prefill launcher, 0 for calls that need no tile list.
 int prefill_unit_chunks(const ksa_params *p);
+int prefill_heads_per_tile(const ksa_params *p);
 
 // Enqueue the plan kernel: validates cu_seqlens against the host totals and
 // fills the offsets.  unit_chunks > 0 also fills tile_off.

@@ -85,6 +85,7 @@ struct SmemLayout {
 struct Params {
     CUtensorMap tm_q, tm_ksum, tm_kwin, tm_vsum, tm_vwin, tm_o;
     int k, w, G, Hq, Hkv, Tc, Tk, batch;
+    int Gp, HP;          // q heads per query tile (min(G, 128/k)) and head parts per kv head (G / Gp)
     int unit_chunks;
     int64_t aug_rows;
     float scale_log2;   // scale * log2(e)
@@ -299,18 +300,22 @@ __device__ __forceinline__ void pair_sync(int quarter)
     asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
 }
 
-// A work item: one query tile of 128 TMEM lanes (GQA-packed rows of one kv
-// head, unit_chunks chunks) and its list of 128-key K/V tiles: the window
-// tiles covering chunks c0-w .. cend-1, then the summary tiles.
+// A work item: one query tile of 128 TMEM lanes (GQA-packed rows: Gp of the
+// G q heads of one kv head, starting at q head h0, for unit_chunks chunks)
+// and its list of 128-key K/V tiles: the window tiles covering chunks
+// c0-w .. cend-1, then the summary tiles.  When G k > 128 the G heads are
+// split over G / Gp items, each loading the same K/V tiles.
 struct Unit {
-    int hkv, nb, mb, ncb, goff, c0, cend, cw_lo, n_win, T;
+    int hkv, h0, nb, mb, ncb, goff, c0, cend, cw_lo, n_win, T;
 };
 
 __device__ __forceinline__ Unit unit_of(const Params &P, int item, int n_units)
 {
     Unit U;
-    const int rank = item / P.Hkv;
-    U.hkv = item % P.Hkv;
+    const int per = P.Hkv * P.HP;
+    const int rank = item / per;
+    U.hkv = (item % per) / P.HP;
+    U.h0 = U.hkv * P.G + ((item % per) % P.HP) * P.Gp;
     const int u = n_units - 1 - rank;  // heaviest (latest) units first
     int lo = 0, hi = P.batch - 1;
     while (lo < hi) {
@@ -360,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         return;
     }
     const int n_units = P.pl.tile_off[P.batch];
-    const int W = n_units * P.Hkv;   // work items
+    const int W = n_units * P.Hkv * P.HP;   // work items
     if ((int)blockIdx.x >= W) return;
 
     auto bar = [&](int i) { return sbase + L::kBar + 8u * (uint32_t)i; };
@@ -424,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     auto S_COL = [&](int bf) { return tmem + (uint32_t)(bf * BN); };
     auto O_COL = [&](int h) { return tmem + (uint32_t)(NSBUF * BN + h * D); };
 
-    const uint32_t q_bytes = (uint32_t)(P.G * P.k * P.Tc) * 128u * (D / 64);
+    const uint32_t q_bytes = (uint32_t)(P.Gp * P.k * P.Tc) * 128u * (D / 64);
     const uint32_t win_bytes = (uint32_t)(P.k * P.Tk) * 128u * (D / 64);
     const uint32_t sum_bytes = (uint32_t)BN * 128u * (D / 64);
     constexpr uint32_t kQHalf = BM * 128;   // bytes of one 64-column half of the query tile
@@ -450,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     mbar_expect_tx(bar(B_QF(qb)), q_bytes);
                     for (int hf = 0; hf < D / 64; ++hf)
                         tma_load_4d(sbase + L::kQ + qb * L::kQTile + hf * kQHalf, &P.tm_q, bar(B_QF(qb)), hf * 64,
-                                    U.hkv * P.G, 0, U.goff + U.c0);
+                                    U.h0, 0, U.goff + U.c0);
                     q_issued[qb]++;
                 }
                 for (int j = 0; j < U.T && ok; ++j, ++gt) {
@@ -561,10 +566,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const int quarter = warp & 3;
         const int R = quarter * 32 + lane;             // row = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const int rows_per_chunk = P.k * P.G;
+        const int rows_per_chunk = P.k * P.Gp;
         const int cl = R / rows_per_chunk;             // row -> (chunk, slot, head)
-        const int r_slot = (R / P.G) % P.k;
-        const int g = R % P.G;
+        const int r_slot = (R / P.Gp) % P.k;
+        const int g = R % P.Gp;
         const float sl2 = P.scale_log2;
         // An expired wait clears ok; every warp still walks all items and
         // runs two pair barriers per item, so no barrier is left unmatched.
@@ -708,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             const float inv = Lr > 0.f ? 1.f / Lr : 0.f;
             const float g0 = f0 * inv, g1 = f1 * inv;
             const int64_t row = (int64_t)(U.goff + c) * (P.k + 1) + r_slot;
-            const int head = U.hkv * P.G + g;
+            const int head = U.h0 + g;
             // this thread holds output columns [D/2 half, D/2 half + D/2) of its row
             uint4 *dst = reinterpret_cast<uint4 *>(P.o + (row * P.Hq + head) * D + half * (D / 2));
             const uint32_t stage_row = sbase + L::kO + (uint32_t)R * 128u;
@@ -750,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 if (warp == 0 && lane == 0 && ok) {
 #pragma unroll
                     for (int hf = 0; hf < D / 64; ++hf)
-                        tma_store_4d(&P.tm_o, sbase + L::kO + hf * kQHalf, hf * 64, U.hkv * P.G, 0, U.goff + U.c0);
+                        tma_store_4d(&P.tm_o, sbase + L::kO + hf * kQHalf, hf * 64, U.h0, 0, U.goff + U.c0);
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 }
             }
@@ -967,10 +972,20 @@ static bool make_map(CUtensorMap *m, const void *base, int d, int H, int k, int6
     return r == CUDA_SUCCESS;
 }
 
+// q heads per query tile: all G of a kv head when G k <= 128 rows, else as
+// many as fit (128 / k); 0 when the shape is not supported.
+int prefill_heads_per_tile(const ksa_params *p)
+{
+    const int G = p->num_q_heads / p->num_kv_heads;
+    if (p->k < 1 || p->k > pf::BM) return 0;
+    const int Gp = G < pf::BM / p->k ? G : pf::BM / p->k;
+    return (Gp >= 1 && G % Gp == 0) ? Gp : 0;
+}
+
 int prefill_unit_chunks(const ksa_params *p)
 {
-    int G = p->num_q_heads / p->num_kv_heads;
-    return pf::BM / (G * p->k);
+    const int Gp = prefill_heads_per_tile(p);
+    return Gp ? pf::BM / (Gp * p->k) : 0;
 }
 
 template <int D>
@@ -983,7 +998,10 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
     const int k = p->k, Hq = p->num_q_heads, Hkv = p->num_kv_heads, G = Hq / Hkv;
     const int64_t chunks = aug_rows / (k + 1);
     P.k = k; P.w = p->w; P.G = G; P.Hq = Hq; P.Hkv = Hkv;
-    P.Tc = pf::BM / (G * k);
+    P.Gp = prefill_heads_per_tile(p);
+    if (P.Gp < 1) return KSA_ERR_UNSUPPORTED;
+    P.HP = G / P.Gp;
+    P.Tc = pf::BM / (P.Gp * k);
     P.Tk = pf::BN / k;
     if (P.Tc < 1 || P.Tk < 1) return KSA_ERR_UNSUPPORTED;
     P.batch = batch;
@@ -996,17 +1014,17 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
     P.q = (const __nv_bfloat16 *)qa;
     P.o = (__nv_bfloat16 *)oa;
     P.lse = lse;
-    bool ok = make_map(&P.tm_q, qa, D, Hq, k, chunks, G, k, P.Tc) &&
+    bool ok = make_map(&P.tm_q, qa, D, Hq, k, chunks, P.Gp, k, P.Tc) &&
               make_map(&P.tm_ksum, ka, D, Hkv, k, chunks, 1, 1, pf::BN) &&
               make_map(&P.tm_kwin, ka, D, Hkv, k, chunks, 1, k, P.Tk) &&
               make_map(&P.tm_vsum, va, D, Hkv, k, chunks, 1, 1, pf::BN) &&
               make_map(&P.tm_vwin, va, D, Hkv, k, chunks, 1, k, P.Tk) &&
-              make_map(&P.tm_o, oa, D, Hq, k, chunks, G, k, P.Tc);
+              make_map(&P.tm_o, oa, D, Hq, k, chunks, P.Gp, k, P.Tc);
     if (!ok) return KSA_ERR_CUDA;
     // persistent: one CTA per SM (shared memory and TMEM admit one); each
     // walks the work items round robin.  CTAs beyond the item count exit.
     int64_t units = total_text / ((int64_t)k * P.unit_chunks) + 2LL * batch + 1;
-    int64_t grid = units * Hkv;
+    int64_t grid = units * Hkv * P.HP;
     if (grid > sm_count()) grid = sm_count();
     static bool attr_set[2] = {false, false};
     if (!attr_set[D == 128]) {

@@ -67,9 +67,13 @@ def test_host_side_validation(lib):
     # workspace too small
     rc = lib.ksa_prefill_fwd(ctypes.byref(p), 1, 16, 8, 9, 16, 16, 16, 16, nul, 16, 8, nul, nul)
     assert rc == L.KSA_ERR_WORKSPACE
-    # G * k > 128 is unsupported for prefill
-    big = L.make_params(64, 1, 8, 2, 128)
-    rc = lib.ksa_prefill_fwd(ctypes.byref(big), 1, 16, 64, 65, 16, 16, 16, 16, nul, 16, 4096, nul, nul)
+    # prefill: k > 128 (a chunk's slots exceed a query tile) and 3 q heads per
+    # kv head (no summary-row kernel) are unsupported
+    big = L.make_params(129, 1, 8, 2, 128)
+    rc = lib.ksa_prefill_fwd(ctypes.byref(big), 1, 16, 129, 130, 16, 16, 16, 16, nul, 16, 4096, nul, nul)
+    assert rc == L.KSA_ERR_UNSUPPORTED
+    g3 = L.make_params(8, 1, 6, 2, 128)
+    rc = lib.ksa_prefill_fwd(ctypes.byref(g3), 1, 16, 8, 9, 16, 16, 16, 16, nul, 16, 4096, nul, nul)
     assert rc == L.KSA_ERR_UNSUPPORTED
     # decode: null cache pointers
     cache = L.ksa_cache(None, None, None, 4, 10)

@@ -27,6 +27,11 @@ CASES = [
     ("two_summary_tiles", [2000], 8, 8, 32, 8, 128, 0.5, 15),
     ("window_covers_all", [200], 8, 100, 4, 1, 128, 1.0, 16),
     ("gqa8_k16", [700], 16, 2, 16, 2, 64, 1.0, 17),
+    ("k16_gqa4_w8", [4096], 16, 8, 32, 8, 128, 1.0, 22),       # k ablation shapes of the report's Table 7
+    ("k32_gqa4_w4", [1500, 333], 32, 4, 32, 8, 128, 1.0, 18),
+    ("k64_gqa4_head_split", [2000, 130], 64, 2, 32, 8, 128, 1.0, 19),   # 4 heads x 64 slots > 128 rows
+    ("k128_gqa8_head_split", [1300], 128, 1, 16, 2, 64, 1.0, 20),
+    ("w128_k8", [3000], 8, 128, 8, 2, 128, 0.5, 21),           # the report's sliding chunk number
 ]
 
 
@@ -103,7 +108,7 @@ def test_interleave_rope_matches_oracle(name, seqlens, k, w, Hq, Hkv, d, scale, 
 
 
 @pytest.mark.parametrize("seqlens,k,w,Hq,Hkv", [([100], 8, 2, 4, 1), ([37, 5, 50], 4, 1, 2, 2),
-                                                ([40, 50], 3, 0, 8, 1)])
+                                                ([40, 50], 3, 0, 8, 1), ([64], 64, 0, 8, 2)])
 def test_visible_set_bit_exact_one_hot(seqlens, k, w, Hq, Hkv):
     """Q = K = 0 makes the softmax uniform over the visible keys; V of the key
     at augmented row a is e_a.  The output row is then nonzero exactly on the

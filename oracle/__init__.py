@@ -9,7 +9,8 @@ together the per-sequence calls of a packed (varlen) batch.
 Citations are to "Kwai Summary Attention Technical Report": the augmented
 sequence is section 2.2.1 Eq. (1); visibility is section 2.2.1 (summary rule)
 and section 2.2.2 Eqs. (2)-(3); the attention is Eq. (10); the decode cache is
-section 2.3.1 with Figure 4.
+section 2.3.1 with Figure 4.  The prefill backward (ksa_attention_bwd) is the
+textbook gradient of Eq. (10) under the same mask, written in numpy.
 """
 from __future__ import annotations
 
@@ -294,3 +295,74 @@ def decode_image(k, C, cap, n_text, m, kind, K, V, q, scale=None):
     lib().oracle_decode_image(k, C, Hkv, d, cap, n_text, m, kind, _p(K), _p(V),
                               Hq, float(scale), _p(q), _p(o), _p(lse))
     return o, lse
+
+
+# --------------------------------------------------------------------------
+# Prefill backward (gradients of Eq. (10) under the KSA mask)
+# --------------------------------------------------------------------------
+def aug_index(n: int, k: int) -> np.ndarray:
+    """Rows of the padded augmented layout (chunk * (k+1) + slot, the layout
+    of the CUDA library) that hold the n + floor(n/k) rows of Eq. (1), in
+    Eq. (1) order (dense_mask's order)."""
+    m = n // k
+    idx = [c * (k + 1) + s for c in range(m) for s in range(k + 1)]
+    idx += [m * (k + 1) + r for r in range(n - m * k)]
+    return np.asarray(idx, dtype=np.int64)
+
+
+def ksa_attention_bwd(n, k, C, q, kk, v, do, scale=None):
+    """Gradients of the loss sum(do * o), o = softmax(scale q k^T + M_KSA) v
+    (Eq. (10)), for one sequence.
+
+    q, do [L, Hq, d] and kk, v [L, Hkv, d]: the L = n + floor(n/k) augmented
+    rows of Eq. (1), already rotated (the tensors attention sees).  Query
+    head h uses kv head h // (Hq / Hkv).  Returns (dq, dk, dv, o, lse) in
+    fp64, written out from the definition: with P the masked softmax,
+    dP = do v^T, D = rowsum(do * o), dS = P * (dP - D), dq = scale dS k,
+    dk = scale dS^T q and dv = P^T do, the last two summed over the q heads
+    that share a kv head.
+    """
+    q, kk, v, do = (_f64(a) for a in (q, kk, v, do))
+    L, Hq, d = q.shape
+    Hkv = kk.shape[1]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    M = dense_mask(n, k, C).astype(bool)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(kk)
+    dv = np.zeros_like(v)
+    o = np.zeros_like(q)
+    lse = np.zeros((L, Hq))
+    for h in range(Hq):
+        g = h // G
+        S = scale * (q[:, h] @ kk[:, g].T)
+        S = np.where(M, S, -np.inf)
+        mx = S.max(axis=1, keepdims=True)
+        E = np.exp(S - mx)
+        den = E.sum(axis=1, keepdims=True)
+        P = E / den
+        o[:, h] = P @ v[:, g]
+        lse[:, h] = (mx + np.log(den))[:, 0]
+        dP = do[:, h] @ v[:, g].T
+        D = (do[:, h] * o[:, h]).sum(axis=1)
+        dS = P * (dP - D[:, None])
+        dq[:, h] = scale * (dS @ kk[:, g])
+        dk[:, g] += scale * (dS.T @ q[:, h])
+        dv[:, g] += P.T @ do[:, h]
+    return dq, dk, dv, o, lse
+
+
+def ksa_prefill_bwd_aug(seqlens, k, C, q_aug, k_aug, v_aug, do_aug, scale=None):
+    """ksa_attention_bwd over a packed batch in the padded augmented layout
+    ([rows, H, d] with chunk * (k+1) + slot rows per sequence).  Returns
+    (dq, dk, dv) in that layout; padding rows are zero."""
+    q_aug, k_aug, v_aug, do_aug = (_f64(a) for a in (q_aug, k_aug, v_aug, do_aug))
+    dq, dk, dv = np.zeros_like(q_aug), np.zeros_like(k_aug), np.zeros_like(v_aug)
+    base = 0
+    for n in seqlens:
+        rows = base + aug_index(n, k)
+        g = ksa_attention_bwd(n, k, C, q_aug[rows], k_aug[rows], v_aug[rows], do_aug[rows], scale)
+        dq[rows], dk[rows], dv[rows] = g[0], g[1], g[2]
+        base += ((n + k - 1) // k) * (k + 1)
+    return dq, dk, dv

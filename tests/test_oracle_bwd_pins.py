@@ -1,0 +1,103 @@
+"""Pins of the oracle's prefill backward (gradients of Eq. (10) of the Kwai
+Summary Attention Technical Report under the KSA mask of section 2.2):
+central finite differences of the loss sum(do * o), the causal-attention
+special case (window covering the whole sequence) against autograd of
+PyTorch's fp64 scaled_dot_product_attention, and two exact identities of
+softmax attention (the key gradients of a kv head sum to zero; the value
+gradients sum to the output gradients of its q heads)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+
+def _inputs(n, k, Hq, Hkv, d, seed):
+    L = n + n // k
+    rng = np.random.default_rng(seed)
+    f = lambda H: rng.standard_normal((L, H, d))
+    return f(Hq), f(Hkv), f(Hkv), f(Hq)
+
+
+@pytest.mark.parametrize("n,k,C,Hq,Hkv,d", [(11, 3, 1, 4, 2, 8), (9, 4, 0, 2, 1, 8), (7, 1, 2, 2, 2, 4),
+                                            (17, 4, 1, 2, 1, 6)])
+def test_bwd_matches_finite_differences(n, k, C, Hq, Hkv, d):
+    q, kk, v, do = _inputs(n, k, Hq, Hkv, d, seed=n + 10 * k + C)
+    dq, dk, dv, o, _ = oracle.ksa_attention_bwd(n, k, C, q, kk, v, do)
+
+    def loss(q_, k_, v_):
+        return float((oracle.ksa_attention_bwd(n, k, C, q_, k_, v_, do)[3] * do).sum())
+
+    eps = 1e-6
+    rng = np.random.default_rng(1)
+    for which, arr, grad in (("q", q, dq), ("k", kk, dk), ("v", v, dv)):
+        for _ in range(12):
+            idx = tuple(int(rng.integers(0, s)) for s in arr.shape)
+            args = {"q": q, "k": kk, "v": v}
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += eps
+            minus[idx] -= eps
+            lp = loss(*(plus if nm == which else args[nm] for nm in ("q", "k", "v")))
+            lm = loss(*(minus if nm == which else args[nm] for nm in ("q", "k", "v")))
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (which, idx, fd, grad[idx])
+
+
+@pytest.mark.parametrize("n,k,Hq,Hkv,d", [(24, 4, 4, 2, 16), (13, 3, 2, 1, 8)])
+def test_bwd_full_window_equals_causal_sdpa_autograd(n, k, Hq, Hkv, d):
+    """With the window covering the whole sequence (C >= n/k) text rows attend
+    causally to all text and see no summary; with zero output gradient on the
+    summary rows the text gradients are those of causal attention."""
+    C = n // k + 1
+    q, kk, v, do = _inputs(n, k, Hq, Hkv, d, seed=3)
+    idx = oracle.aug_index(n, k)
+    L = len(idx)
+    text = np.array([a for a in range(L) if not (a < (n // k) * (k + 1) and a % (k + 1) == k)])
+    summ = np.setdiff1d(np.arange(L), text)
+    do[summ] = 0
+    dq, dk, dv, _, _ = oracle.ksa_attention_bwd(n, k, C, q, kk, v, do)
+    G = Hq // Hkv
+    tq = torch.tensor(q[text], dtype=torch.float64).transpose(0, 1).requires_grad_(True)   # [Hq, n, d]
+    tk = torch.tensor(kk[text], dtype=torch.float64).transpose(0, 1).requires_grad_(True)
+    tv = torch.tensor(v[text], dtype=torch.float64).transpose(0, 1).requires_grad_(True)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk.repeat_interleave(G, dim=0), tv.repeat_interleave(G, dim=0), is_causal=True)
+    (out * torch.tensor(do[text], dtype=torch.float64).transpose(0, 1)).sum().backward()
+    np.testing.assert_allclose(dq[text], tq.grad.transpose(0, 1).numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk[text], tk.grad.transpose(0, 1).numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv[text], tv.grad.transpose(0, 1).numpy(), rtol=1e-10, atol=1e-12)
+    # summaries are invisible to text queries, and the summary rows' own
+    # output gradient is zero: nothing flows into them
+    assert np.abs(dk[summ]).max() == 0 and np.abs(dv[summ]).max() == 0 and np.abs(dq[summ]).max() == 0
+
+
+@pytest.mark.parametrize("n,k,C", [(40, 4, 2), (33, 8, 1), (64, 8, 0)])
+def test_bwd_identities(n, k, C):
+    Hq, Hkv, d = 4, 2, 16
+    q, kk, v, do = _inputs(n, k, Hq, Hkv, d, seed=7)
+    dq, dk, dv, _, _ = oracle.ksa_attention_bwd(n, k, C, q, kk, v, do)
+    L = q.shape[0]
+    G = Hq // Hkv
+    assert np.abs(dk.sum(axis=0)).max() < 1e-11
+    want = do.reshape(L, Hkv, G, d).sum(axis=(0, 2))
+    np.testing.assert_allclose(dv.sum(axis=0), want, rtol=1e-12, atol=1e-11)
+
+
+def test_bwd_padded_layout():
+    """The packed, padded augmented layout of the library: each sequence's
+    rows map to its own gradients; padding rows stay zero."""
+    seqlens, k, C, Hq, Hkv, d = [10, 8, 3], 4, 1, 2, 1, 8
+    rows = sum(((n + k - 1) // k) * (k + 1) for n in seqlens)
+    rng = np.random.default_rng(5)
+    qa, ka, va, doa = (rng.standard_normal((rows, H, d)) for H in (Hq, Hkv, Hkv, Hq))
+    dq, dk, dv = oracle.ksa_prefill_bwd_aug(seqlens, k, C, qa, ka, va, doa)
+    base = 0
+    live = np.zeros(rows, bool)
+    for n in seqlens:
+        r = base + oracle.aug_index(n, k)
+        live[r] = True
+        g = oracle.ksa_attention_bwd(n, k, C, qa[r], ka[r], va[r], doa[r])
+        np.testing.assert_array_equal(dq[r], g[0])
+        np.testing.assert_array_equal(dk[r], g[1])
+        base += ((n + k - 1) // k) * (k + 1)
+    assert np.abs(dq[~live]).max() == 0 and np.abs(dk[~live]).max() == 0 and np.abs(dv[~live]).max() == 0

@@ -139,6 +139,27 @@ KSA_API int ksa_prefill_fwd(const ksa_params *p, int32_t batch, const int32_t *c
                     void *workspace, size_t workspace_bytes, int32_t *dev_err,
                     void *stream);
 
+/* Workspace bytes for ksa_prefill_bwd (the batch plan, block offsets and an
+ * fp32 [aug_rows, Hq] buffer for rowsum(dO * O)). */
+KSA_API size_t ksa_prefill_bwd_workspace_size(const ksa_params *p, int32_t batch, int64_t aug_rows);
+
+/* KSA prefill backward: gradients of Eq. (10) under the KSA mask (sections
+ * 2.2.1-2.2.2, Eqs. (2)-(3)) with respect to the augmented, rotated inputs
+ * of ksa_prefill_fwd.  q_aug, k_aug, v_aug, o_aug, lse: as given to and
+ * returned by ksa_prefill_fwd (lse is required); do_aug [aug_rows, Hq, d]
+ * bf16: the gradient of the loss with respect to o_aug.  Writes
+ * dq_aug [aug_rows, Hq, d], dk_aug / dv_aug [aug_rows, Hkv, d] (bf16) for
+ * every real row (text and summary); padding rows are not written.  dk and
+ * dv sum over the q heads that share a kv head.  Runs on the warp-level
+ * tensor-core MMA, skipping the key/query block pairs the rule masks out
+ * entirely.  dev_err and cu_seqlens as for ksa_prefill_fwd. */
+KSA_API int ksa_prefill_bwd(const ksa_params *p, int32_t batch, const int32_t *cu_seqlens,
+                    int64_t total_text, int64_t aug_rows,
+                    const void *q_aug, const void *k_aug, const void *v_aug,
+                    const void *o_aug, const float *lse, const void *do_aug,
+                    void *dq_aug, void *dk_aug, void *dv_aug,
+                    void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream);
+
 /* ------------------------------------------------------------------------
  * Decode cache (section 2.3.1, Figure 4).
  *

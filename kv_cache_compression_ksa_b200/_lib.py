@@ -69,6 +69,9 @@ SYMBOLS = {
                                            _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "ksa_prefill_fwd": (ctypes.c_int, [ctypes.POINTER(ksa_params), _I32, _P, _I64, _I64,
                                        _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "ksa_prefill_bwd_workspace_size": (_SZ, [ctypes.POINTER(ksa_params), _I32, _I64]),
+    "ksa_prefill_bwd": (ctypes.c_int, [ctypes.POINTER(ksa_params), _I32, _P, _I64, _I64, _P, _P, _P, _P, _P, _P,
+                                       _P, _P, _P, _P, _SZ, _P, _P]),
     "ksa_cache_slots": (_I64, [ctypes.POINTER(ksa_params), _I64]),
     "ksa_cache_append": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _P, _P, _P]),
     "ksa_cache_from_prefill": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _I64, _I64,
@@ -161,6 +164,19 @@ def ksa_prefill_fwd(p, cu_seqlens, total_text, aug_rows, q_aug, k_aug, v_aug, o_
         _ptr(q_aug), _ptr(k_aug), _ptr(v_aug), _ptr(o_aug), _ptr(lse),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_err), _stream(stream))
     _check("ksa_prefill_fwd", rc)
+
+
+def ksa_prefill_bwd_workspace_size(p: ksa_params, batch: int, aug_rows: int) -> int:
+    return int(load().ksa_prefill_bwd_workspace_size(ctypes.byref(p), batch, aug_rows))
+
+
+def ksa_prefill_bwd(p, cu_seqlens, total_text, aug_rows, q_aug, k_aug, v_aug, o_aug, lse, do_aug, dq_aug, dk_aug,
+                    dv_aug, workspace, dev_err=None, stream=None):
+    rc = load().ksa_prefill_bwd(
+        ctypes.byref(p), cu_seqlens.numel() - 1, _ptr(cu_seqlens), total_text, aug_rows, _ptr(q_aug), _ptr(k_aug),
+        _ptr(v_aug), _ptr(o_aug), _ptr(lse), _ptr(do_aug), _ptr(dq_aug), _ptr(dk_aug), _ptr(dv_aug),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_err), _stream(stream))
+    _check("ksa_prefill_bwd", rc)
 
 
 def ksa_cache_slots(p: ksa_params, cap_summaries: int) -> int:

@@ -147,6 +147,36 @@ int ksa_prefill_fwd(const ksa_params *p, int32_t batch, const int32_t *cu_seqlen
     return launch_prefill(p, batch, cu_seqlens, total_text, aug_rows, q_aug, k_aug, v_aug, o_aug, lse, pl, err, st);
 }
 
+size_t ksa_prefill_bwd_workspace_size(const ksa_params *p, int32_t batch, int64_t aug_rows)
+{
+    if (check_params(p) != KSA_OK || batch < 0 || aug_rows < 0) return 0;
+    return prefill_bwd_workspace_bytes(p, batch, aug_rows);
+}
+
+int ksa_prefill_bwd(const ksa_params *p, int32_t batch, const int32_t *cu_seqlens, int64_t total_text,
+                    int64_t aug_rows, const void *q_aug, const void *k_aug, const void *v_aug, const void *o_aug,
+                    const float *lse, const void *do_aug, void *dq_aug, void *dk_aug, void *dv_aug, void *workspace,
+                    size_t workspace_bytes, int32_t *dev_err, void *stream)
+{
+    int rc = check_prefill_common(p, batch, cu_seqlens, total_text, aug_rows, workspace, workspace_bytes);
+    if (rc != KSA_OK) return rc;
+    if (workspace_bytes < prefill_bwd_workspace_bytes(p, batch, aug_rows)) return KSA_ERR_WORKSPACE;
+    if (aug_rows > 0) {
+        const void *ptrs[] = {q_aug, k_aug, v_aug, o_aug, do_aug, dq_aug, dk_aug, dv_aug};
+        for (const void *x : ptrs)
+            if (!x || !aligned16(x)) return KSA_ERR_INVALID;
+        if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u)) return KSA_ERR_INVALID;
+    }
+    if (reinterpret_cast<uintptr_t>(dev_err) & 3u) return KSA_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    Plan pl = plan_view(workspace, batch);
+    int32_t *err = dev_err ? dev_err : pl.err;
+    rc = launch_plan(p, batch, cu_seqlens, total_text, -1, aug_rows, pl, err, 0, st);
+    if (rc != KSA_OK) return rc;
+    return launch_prefill_bwd(p, batch, cu_seqlens, total_text, aug_rows, q_aug, k_aug, v_aug, o_aug, lse, do_aug,
+                              dq_aug, dk_aug, dv_aug, workspace, pl, err, st);
+}
+
 int64_t ksa_cache_slots(const ksa_params *p, int64_t cap_summaries)
 {
     if (!p || p->k < 1 || p->w < 0 || cap_summaries < 0) return -1;

@@ -58,6 +58,12 @@ int launch_interleave_rope(const ksa_params *p, int batch, const int32_t *cu, in
                            const void *ks, const void *vs, void *qa, void *ka, void *va,
                            const Plan &pl, int32_t *err, cudaStream_t st);
 
+// Prefill backward (prefill_bwd.cu).
+size_t prefill_bwd_workspace_bytes(const ksa_params *p, int batch, int64_t aug_rows);
+int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,
+                       const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
+                       void *dq, void *dk, void *dv, void *ws, const Plan &pl, int32_t *err, cudaStream_t st);
+
 // Decode cache from the augmented K/V of a prefilled batch (cache_decode.cu).
 int launch_cache_build(const ksa_params *p, const ksa_cache *c, const int32_t *cu, const void *k_aug,
                        const void *v_aug, const Plan &pl, int32_t *err, cudaStream_t st);

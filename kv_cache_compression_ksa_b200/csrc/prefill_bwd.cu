@@ -1,0 +1,525 @@
+// prefill_bwd.cu -- backward of the KSA prefill attention: dq, dk, dv of the
+// augmented (rotated) Q, K, V given dO, O and the forward's LSE.
+//
+// Kwai Summary Attention Technical Report: the forward is Eq. (10),
+// softmax(Q K^T / sqrt(d) + M_KSA) V, with the mask of section 2.2.1 (a
+// summary sees its chunk's k text tokens and itself) and section 2.2.2,
+// Eqs. (2)-(3) (text t_i sees text chunks c-w .. c causally and the
+// summaries s_0 .. s_{c-w-1}).  The gradients are the textbook ones under the
+// same mask: P = exp(S - lse), dP = dO V^T, D = rowsum(dO * O),
+// dS = P * (dP - D), dq = scale dS K, dk = scale dS^T Q, dv = P^T dO.
+//
+// Work is cut the way the forward skips tiles: a block holds 64 rows of one
+// kind (64 consecutive text tokens or 64 consecutive summaries of one
+// sequence), and a query block only meets the key blocks its rows can see
+// (summaries 0 .. c_last-w-1 and the text of chunks c_first-w .. c_last), and
+// a key block only the query blocks that can see it.  Inside a pair of blocks
+// the mask is evaluated per element from the rows' coordinates.
+//
+//   bwd_dot_kernel   D = rowsum(dO * O)                          (HBM)
+//   bwd_dq_kernel    query-stationary: dq of 64 rows of one q head
+//   bwd_dkv_kernel   key-stationary: dk, dv of 64 rows of one kv head,
+//                    over all q heads of its group
+// Both attention kernels use the warp-level tensor-core MMA (m16n8k16, bf16
+// in, fp32 accumulate) with operands staged in shared memory and read with
+// ldmatrix; each warp owns 16 rows of its block.  No atomics: every output
+// row belongs to exactly one block.
+#include <math.h>
+
+#include "ksa_internal.cuh"
+#include "warp_mma.cuh"
+
+namespace ksa {
+namespace bw {
+
+constexpr int RB = 64;          // rows per block
+constexpr int kThreads = 128;   // 4 warps x 16 rows
+constexpr int TEXT_ROWS = 0, SUM_ROWS = 1;
+
+struct Args {
+    int k, w, Hq, Hkv, G, batch;
+    float scale, scale_log2;
+    const int32_t *cu;
+    Plan pl;
+    const int32_t *tb_off, *sb_off;   // [B+1] first text / summary block of each sequence
+    int32_t *err;
+    const __nv_bfloat16 *q, *kk, *v, *o, *dout;
+    const float *lse;                 // [rows, Hq] natural log
+    float *dsum;                      // [rows, Hq] D = rowsum(dO * O)
+    __nv_bfloat16 *dq, *dk, *dv;
+};
+
+// A block: rows of one kind of sequence b.
+struct Blk {
+    int b, kind, idx0, cnt, n, m;
+    int64_t c0;    // first chunk of the sequence in the augmented layout
+};
+
+__device__ __forceinline__ int64_t aug_row(const Args &a, const Blk &B, int idx)
+{
+    return B.kind == TEXT_ROWS ? (B.c0 + idx / a.k) * (a.k + 1) + idx % a.k : (B.c0 + idx) * (a.k + 1) + a.k;
+}
+
+__device__ __forceinline__ int find_seq(const int32_t *off, int batch, int id)
+{
+    int lo = 0, hi = batch - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= id) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// block id -> (sequence, kind, rows): text blocks of all sequences first
+__device__ __forceinline__ bool block_of(const Args &a, int id, Blk &B)
+{
+    const int nt = a.tb_off[a.batch];
+    int b, kind, j;
+    if (id < nt) {
+        b = find_seq(a.tb_off, a.batch, id); kind = TEXT_ROWS; j = id - a.tb_off[b];
+    } else {
+        id -= nt;
+        if (id >= a.sb_off[a.batch]) return false;
+        b = find_seq(a.sb_off, a.batch, id); kind = SUM_ROWS; j = id - a.sb_off[b];
+    }
+    B.b = b; B.kind = kind;
+    B.n = a.cu[b + 1] - a.cu[b];
+    B.m = B.n / a.k;
+    B.c0 = a.pl.chunk_off[b];
+    B.idx0 = j * RB;
+    B.cnt = min(RB, (kind == TEXT_ROWS ? B.n : B.m) - B.idx0);
+    return B.cnt > 0;
+}
+
+// KSA visibility of key (kk_kind, ki) to query (qk, qi) of one sequence
+__device__ __forceinline__ bool visible(const Args &a, int m, int qk, int qi, int kk_kind, int ki)
+{
+    if (qk == TEXT_ROWS) {
+        const int c = qi / a.k;
+        if (kk_kind == TEXT_ROWS) return ki <= qi && ki >= max(0, c - a.w) * a.k;
+        return ki < min(c - a.w, m);
+    }
+    if (kk_kind == TEXT_ROWS) return ki / a.k == qi;
+    return ki == qi;
+}
+
+// 64 rows x D bf16 of one head into shared memory, rows padded by 16 bytes
+// (row pitch D + 8 elements keeps ldmatrix's 8-row reads conflict-free);
+// rows at or beyond cnt are zero.
+template <int D>
+__device__ __forceinline__ void load_rows(__nv_bfloat16 (*dst)[D + 8], const __nv_bfloat16 *src, int H, int head,
+                                          const Args &a, const Blk &B, int first, int cnt)
+{
+    constexpr int V8 = D / 8;
+    for (int e = threadIdx.x; e < RB * V8; e += kThreads) {
+        const int r = e / V8, c8 = e % V8;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (r < cnt) val = reinterpret_cast<const uint4 *>(src + (aug_row(a, B, first + r) * H + head) * D)[c8];
+        *reinterpret_cast<uint4 *>(&dst[r][c8 * 8]) = val;
+    }
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p)
+{
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void *p)
+{
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
+}
+
+// A fragment (16 rows x 16 cols) at (row0, col0) of a row-major tile
+template <int D>
+__device__ __forceinline__ void frag_a(uint32_t (&r)[4], const __nv_bfloat16 (*t)[D + 8], int row0, int col0)
+{
+    const int l = threadIdx.x & 31;
+    ldsm_x4(r, &t[row0 + (l & 7) + 8 * ((l >> 3) & 1)][col0 + 8 * (l >> 4)]);
+}
+
+// B fragments of two n-tiles from a tile stored [n][k] (rows = n): n-tiles
+// n0 .. n0+7 and n0+8 .. n0+15, k-chunk k0 .. k0+15.  r = {b0, b1 of the
+// first n-tile, b0, b1 of the second}.
+template <int D>
+__device__ __forceinline__ void frag_b_nk(uint32_t (&r)[4], const __nv_bfloat16 (*t)[D + 8], int n0, int k0)
+{
+    const int l = threadIdx.x & 31;
+    ldsm_x4(r, &t[n0 + (l & 7) + 8 * (l >> 4)][k0 + 8 * ((l >> 3) & 1)]);
+}
+
+// B fragments of two n-tiles from a tile stored [k][n] (rows = k): k-chunk
+// k0 .. k0+15, n-tiles n0 .. n0+7 and n0+8 .. n0+15 (transposing load).
+template <int D>
+__device__ __forceinline__ void frag_b_kn(uint32_t (&r)[4], const __nv_bfloat16 (*t)[D + 8], int k0, int n0)
+{
+    const int l = threadIdx.x & 31;
+    ldsm_x4_t(r, &t[k0 + (l & 7) + 8 * ((l >> 3) & 1)][n0 + 8 * (l >> 4)]);
+}
+
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) bwd_dot_kernel(Args a, int64_t rows, int D)
+{
+    // one thread per (row, head): D = dO . O over d
+    const int64_t t = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    if (t >= rows * a.Hq) return;
+    const uint4 *x = reinterpret_cast<const uint4 *>(a.dout + t * D);
+    const uint4 *y = reinterpret_cast<const uint4 *>(a.o + t * D);
+    float s = 0.f;
+    for (int c = 0; c < D / 8; ++c) {
+        const uint4 u = x[c], w = y[c];
+        const uint32_t uu[4] = {u.x, u.y, u.z, u.w}, ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            s = fmaf(__uint_as_float(uu[i] << 16), __uint_as_float(ww[i] << 16), s);
+            s = fmaf(__uint_as_float(uu[i] & 0xffff0000u), __uint_as_float(ww[i] & 0xffff0000u), s);
+        }
+    }
+    a.dsum[t] = s;
+}
+
+// ---------------------------------------------------------------------------
+// dq: one CTA = one query block x one q head.
+template <int D>
+__global__ void __launch_bounds__(kThreads) bwd_dq_kernel(Args a)
+{
+    constexpr int KC = D / 16, NT = D / 8;
+    using Row = __nv_bfloat16[D + 8];
+    extern __shared__ __align__(16) uint8_t bw_smem[];
+    Row *sQ = reinterpret_cast<Row *>(bw_smem), *sO = sQ + RB, *sK = sO + RB, *sV = sK + RB;
+    if (*a.err != 0) return;
+    Blk Q;
+    if (!block_of(a, blockIdx.x, Q)) return;
+    const int h = blockIdx.y, g = h / a.G;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tt = lane & 3;
+    load_rows<D>(sQ, a.q, a.Hq, h, a, Q, Q.idx0, Q.cnt);
+    load_rows<D>(sO, a.dout, a.Hq, h, a, Q, Q.idx0, Q.cnt);
+    // this warp's two rows per lane: 16 warp + gr and + 8
+    float lse2[2], dd[2];
+    int qi[2];
+    bool live[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        const int r = 16 * warp + gr + 8 * x;
+        live[x] = r < Q.cnt;
+        qi[x] = Q.idx0 + r;
+        const int64_t row = live[x] ? aug_row(a, Q, qi[x]) : 0;
+        lse2[x] = live[x] ? a.lse[row * a.Hq + h] * 1.4426950408889634f : 0.f;
+        dd[x] = live[x] ? a.dsum[row * a.Hq + h] : 0.f;
+    }
+    __syncthreads();
+    uint32_t qf[KC][4], of[KC][4];
+#pragma unroll
+    for (int c = 0; c < KC; ++c) {
+        frag_a<D>(qf[c], sQ, 16 * warp, 16 * c);
+        frag_a<D>(of[c], sO, 16 * warp, 16 * c);
+    }
+    float acc[NT][4];
+#pragma unroll
+    for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+    // the key blocks these rows can see
+    int nsb = 0, t_lo = 0, t_hi = 0, s_lo = 0;
+    if (Q.kind == TEXT_ROWS) {
+        const int ca = Q.idx0 / a.k, cb = (Q.idx0 + Q.cnt - 1) / a.k;
+        const int ns = max(0, min(cb - a.w, Q.m));
+        nsb = (ns + RB - 1) / RB;            // summary key blocks [0, ns)
+        t_lo = max(0, ca - a.w) * a.k;       // text keys [t_lo, t_hi)
+        t_hi = Q.idx0 + Q.cnt;
+    } else {
+        t_lo = Q.idx0 * a.k;
+        t_hi = (Q.idx0 + Q.cnt) * a.k;
+        nsb = 1;                             // the block's own summaries (each sees itself)
+        s_lo = Q.idx0;
+    }
+    const int ntb = (t_hi - t_lo + RB - 1) / RB;
+    for (int kb = 0; kb < nsb + ntb; ++kb) {
+        Blk K = Q;
+        if (kb < nsb) {
+            K.kind = SUM_ROWS; K.idx0 = s_lo + kb * RB;
+            K.cnt = min(RB, (Q.kind == TEXT_ROWS ? max(0, min((Q.idx0 + Q.cnt - 1) / a.k - a.w, Q.m)) : Q.idx0 + Q.cnt) - K.idx0);
+        } else {
+            K.kind = TEXT_ROWS; K.idx0 = t_lo + (kb - nsb) * RB;
+            K.cnt = min(RB, t_hi - K.idx0);
+        }
+        __syncthreads();   // the previous key block has been read
+        load_rows<D>(sK, a.kk, a.Hkv, g, a, K, K.idx0, K.cnt);
+        load_rows<D>(sV, a.v, a.Hkv, g, a, K, K.idx0, K.cnt);
+        __syncthreads();
+        // S = Q K^T and dP = dO V^T: 16 rows x 64 keys
+        float s[8][4], dp[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
+#pragma unroll
+        for (int c = 0; c < KC; ++c)
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bk[4], bv[4];
+                frag_b_nk<D>(bk, sK, 16 * np, 16 * c);
+                frag_b_nk<D>(bv, sV, 16 * np, 16 * c);
+                wm::mma16816(s[2 * np], qf[c][0], qf[c][1], qf[c][2], qf[c][3], bk[0], bk[1]);
+                wm::mma16816(s[2 * np + 1], qf[c][0], qf[c][1], qf[c][2], qf[c][3], bk[2], bk[3]);
+                wm::mma16816(dp[2 * np], of[c][0], of[c][1], of[c][2], of[c][3], bv[0], bv[1]);
+                wm::mma16816(dp[2 * np + 1], of[c][0], of[c][1], of[c][2], of[c][3], bv[2], bv[3]);
+            }
+        // dS = P * (dP - D), P = exp(S - lse) on visible pairs, as bf16 A fragments
+        uint32_t dsf[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            float e[4];
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+                const int x = z >> 1, col = 8 * nt + 2 * tt + (z & 1);
+                const bool vis = live[x] && col < K.cnt && visible(a, Q.m, Q.kind, qi[x], K.kind, K.idx0 + col);
+                const float p = vis ? wm::ex2(s[nt][z] * a.scale_log2 - lse2[x]) : 0.f;
+                e[z] = p * (dp[nt][z] - dd[x]);
+            }
+            const int j = nt >> 1;
+            if ((nt & 1) == 0) { dsf[j][0] = wm::pack2(e[0], e[1]); dsf[j][1] = wm::pack2(e[2], e[3]); }
+            else { dsf[j][2] = wm::pack2(e[0], e[1]); dsf[j][3] = wm::pack2(e[2], e[3]); }
+        }
+        // dq += dS K (k = keys, n = dims)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int np = 0; np < NT / 2; ++np) {
+                uint32_t bk[4];
+                frag_b_kn<D>(bk, sK, 16 * j, 16 * np);
+                wm::mma16816(acc[2 * np], dsf[j][0], dsf[j][1], dsf[j][2], dsf[j][3], bk[0], bk[1]);
+                wm::mma16816(acc[2 * np + 1], dsf[j][0], dsf[j][1], dsf[j][2], dsf[j][3], bk[2], bk[3]);
+            }
+    }
+    // dq rows: acc[nt] holds (row gr, dims 8nt + 2tt, +1) and (row gr + 8, same dims)
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        if (!live[x]) continue;
+        __nv_bfloat16 *dst = a.dq + (aug_row(a, Q, qi[x]) * a.Hq + h) * D;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            *reinterpret_cast<uint32_t *>(dst + 8 * nt + 2 * tt) =
+                wm::pack2(acc[nt][2 * x] * a.scale, acc[nt][2 * x + 1] * a.scale);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// dk, dv: one CTA = one key block x one kv head, over the q heads of its group.
+template <int D>
+__global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
+{
+    constexpr int KC = D / 16, NT = D / 8;
+    using Row = __nv_bfloat16[D + 8];
+    extern __shared__ __align__(16) uint8_t bw_smem[];
+    Row *sK = reinterpret_cast<Row *>(bw_smem), *sV = sK + RB, *sQ = sV + RB, *sO = sQ + RB;
+    float *sL = reinterpret_cast<float *>(sO + RB), *sD = sL + RB;
+    if (*a.err != 0) return;
+    Blk K;
+    if (!block_of(a, blockIdx.x, K)) return;
+    const int g = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tt = lane & 3;
+    load_rows<D>(sK, a.kk, a.Hkv, g, a, K, K.idx0, K.cnt);
+    load_rows<D>(sV, a.v, a.Hkv, g, a, K, K.idx0, K.cnt);
+    int ki[2];
+    bool live[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        const int r = 16 * warp + gr + 8 * x;
+        live[x] = r < K.cnt;
+        ki[x] = K.idx0 + r;
+    }
+    float dk[NT][4], dv[NT][4];
+#pragma unroll
+    for (int i = 0; i < NT; ++i) dk[i][0] = dk[i][1] = dk[i][2] = dk[i][3] = dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
+
+    // the query blocks that can see these keys
+    int t_lo, t_hi, s_lo, s_hi;
+    if (K.kind == TEXT_ROWS) {
+        const int ca = K.idx0 / a.k, cb = (K.idx0 + K.cnt - 1) / a.k;
+        t_lo = K.idx0;
+        t_hi = min(K.n, (cb + a.w + 1) * a.k);
+        s_lo = ca;
+        s_hi = min(cb + 1, K.m);
+    } else {
+        t_lo = min(K.n, (K.idx0 + a.w + 1) * a.k);
+        t_hi = K.n;
+        s_lo = K.idx0;
+        s_hi = K.idx0 + K.cnt;
+    }
+    const int ntb = (t_hi - t_lo + RB - 1) / RB;
+    const int nsb = s_hi > s_lo ? 1 : 0;   // at most 64 summaries see this block's keys
+    for (int hh = 0; hh < a.G; ++hh) {
+        const int h = g * a.G + hh;
+        for (int qb = 0; qb < ntb + nsb; ++qb) {
+            Blk Q = K;
+            if (qb < ntb) {
+                Q.kind = TEXT_ROWS; Q.idx0 = t_lo + qb * RB; Q.cnt = min(RB, t_hi - Q.idx0);
+            } else {
+                Q.kind = SUM_ROWS; Q.idx0 = s_lo; Q.cnt = s_hi - s_lo;
+            }
+            __syncthreads();   // the previous query block has been read
+            load_rows<D>(sQ, a.q, a.Hq, h, a, Q, Q.idx0, Q.cnt);
+            load_rows<D>(sO, a.dout, a.Hq, h, a, Q, Q.idx0, Q.cnt);
+            for (int r = threadIdx.x; r < RB; r += kThreads) {
+                const bool ok = r < Q.cnt;
+                const int64_t row = ok ? aug_row(a, Q, Q.idx0 + r) : 0;
+                sL[r] = ok ? a.lse[row * a.Hq + h] * 1.4426950408889634f : 0.f;
+                sD[r] = ok ? a.dsum[row * a.Hq + h] : 0.f;
+            }
+            __syncthreads();
+            // two halves of 32 queries: S^T = K Q^T, dP^T = V dO^T (16 keys x 32 queries)
+#pragma unroll 1
+            for (int hq = 0; hq < 2; ++hq) {
+                const int q0 = 32 * hq;
+                if (q0 >= Q.cnt) break;
+                float s[4][4], dp[4][4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
+#pragma unroll
+                for (int c = 0; c < KC; ++c) {
+                    uint32_t ak[4], av[4];
+                    frag_a<D>(ak, sK, 16 * warp, 16 * c);
+                    frag_a<D>(av, sV, 16 * warp, 16 * c);
+#pragma unroll
+                    for (int np = 0; np < 2; ++np) {
+                        uint32_t bq[4], bo[4];
+                        frag_b_nk<D>(bq, sQ, q0 + 16 * np, 16 * c);
+                        frag_b_nk<D>(bo, sO, q0 + 16 * np, 16 * c);
+                        wm::mma16816(s[2 * np], ak[0], ak[1], ak[2], ak[3], bq[0], bq[1]);
+                        wm::mma16816(s[2 * np + 1], ak[0], ak[1], ak[2], ak[3], bq[2], bq[3]);
+                        wm::mma16816(dp[2 * np], av[0], av[1], av[2], av[3], bo[0], bo[1]);
+                        wm::mma16816(dp[2 * np + 1], av[0], av[1], av[2], av[3], bo[2], bo[3]);
+                    }
+                }
+                // P^T and dS^T as bf16 A fragments (16 keys x 32 queries = 2 k-chunks)
+                uint32_t pf[2][4], dsf[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    float pe[4], de[4];
+#pragma unroll
+                    for (int z = 0; z < 4; ++z) {
+                        const int x = z >> 1, col = q0 + 8 * nt + 2 * tt + (z & 1);
+                        const bool vis = live[x] && col < Q.cnt && visible(a, K.m, Q.kind, Q.idx0 + col, K.kind, ki[x]);
+                        const float p = vis ? wm::ex2(s[nt][z] * a.scale_log2 - sL[col]) : 0.f;
+                        pe[z] = p;
+                        de[z] = p * (dp[nt][z] - sD[col]);
+                    }
+                    const int j = nt >> 1;
+                    if ((nt & 1) == 0) {
+                        pf[j][0] = wm::pack2(pe[0], pe[1]); pf[j][1] = wm::pack2(pe[2], pe[3]);
+                        dsf[j][0] = wm::pack2(de[0], de[1]); dsf[j][1] = wm::pack2(de[2], de[3]);
+                    } else {
+                        pf[j][2] = wm::pack2(pe[0], pe[1]); pf[j][3] = wm::pack2(pe[2], pe[3]);
+                        dsf[j][2] = wm::pack2(de[0], de[1]); dsf[j][3] = wm::pack2(de[2], de[3]);
+                    }
+                }
+                // dv += P^T dO, dk += dS^T Q (k = queries, n = dims)
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        uint32_t bo[4], bq[4];
+                        frag_b_kn<D>(bo, sO, q0 + 16 * j, 16 * np);
+                        frag_b_kn<D>(bq, sQ, q0 + 16 * j, 16 * np);
+                        wm::mma16816(dv[2 * np], pf[j][0], pf[j][1], pf[j][2], pf[j][3], bo[0], bo[1]);
+                        wm::mma16816(dv[2 * np + 1], pf[j][0], pf[j][1], pf[j][2], pf[j][3], bo[2], bo[3]);
+                        wm::mma16816(dk[2 * np], dsf[j][0], dsf[j][1], dsf[j][2], dsf[j][3], bq[0], bq[1]);
+                        wm::mma16816(dk[2 * np + 1], dsf[j][0], dsf[j][1], dsf[j][2], dsf[j][3], bq[2], bq[3]);
+                    }
+            }
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        if (!live[x]) continue;
+        const int64_t row = aug_row(a, K, ki[x]);
+        __nv_bfloat16 *pk = a.dk + (row * a.Hkv + g) * D;
+        __nv_bfloat16 *pv = a.dv + (row * a.Hkv + g) * D;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            *reinterpret_cast<uint32_t *>(pk + 8 * nt + 2 * tt) = wm::pack2(dk[nt][2 * x] * a.scale, dk[nt][2 * x + 1] * a.scale);
+            *reinterpret_cast<uint32_t *>(pv + 8 * nt + 2 * tt) = wm::pack2(dv[nt][2 * x], dv[nt][2 * x + 1]);
+        }
+    }
+}
+
+// per-sequence block counts: text blocks ceil(n/64), summary blocks ceil(m/64)
+__global__ void bwd_blocks_kernel(int batch, const int32_t *cu, int k, int32_t *tb_off, int32_t *sb_off)
+{
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    int t = 0, s = 0;
+    for (int b = 0; b < batch; ++b) {
+        tb_off[b] = t;
+        sb_off[b] = s;
+        const int n = max(cu[b + 1] - cu[b], 0);
+        t += (n + RB - 1) / RB;
+        s += (n / k + RB - 1) / RB;
+    }
+    tb_off[batch] = t;
+    sb_off[batch] = s;
+}
+
+}  // namespace bw
+
+// four 64-row tiles of D + 8 bf16 per row (+ per-query LSE and D for dk, dv)
+template <int D>
+static int bw_launch(const bw::Args &a, int64_t nblk, cudaStream_t st)
+{
+    const int tiles = 4 * bw::RB * (D + 8) * 2;
+    const int dkv = tiles + 2 * bw::RB * 4;
+    static bool attr[2] = {false, false};
+    if (!attr[D == 128]) {
+        if (cudaFuncSetAttribute(bw::bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, tiles) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(bw::bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv) != cudaSuccess)
+            return KSA_ERR_CUDA;
+        attr[D == 128] = true;
+    }
+    bw::bwd_dq_kernel<D><<<dim3((unsigned)nblk, a.Hq), bw::kThreads, tiles, st>>>(a);
+    bw::bwd_dkv_kernel<D><<<dim3((unsigned)nblk, a.Hkv), bw::kThreads, dkv, st>>>(a);
+    return KSA_OK;
+}
+
+size_t prefill_bwd_workspace_bytes(const ksa_params *p, int batch, int64_t aug_rows)
+{
+    return plan_bytes(batch) + 2 * align_up(sizeof(int32_t) * (size_t)(batch + 1)) +
+           align_up(sizeof(float) * (size_t)aug_rows * p->num_q_heads);
+}
+
+int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,
+                       const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
+                       void *dq, void *dk, void *dv, void *ws, const Plan &pl, int32_t *err, cudaStream_t st)
+{
+    if (aug_rows == 0) return KSA_OK;
+    char *w = static_cast<char *>(ws) + plan_bytes(batch);
+    const size_t ab = align_up(sizeof(int32_t) * (size_t)(batch + 1));
+    bw::Args a;
+    a.tb_off = reinterpret_cast<int32_t *>(w);
+    a.sb_off = reinterpret_cast<int32_t *>(w + ab);
+    a.dsum = reinterpret_cast<float *>(w + 2 * ab);
+    a.k = p->k; a.w = p->w; a.Hq = p->num_q_heads; a.Hkv = p->num_kv_heads; a.G = a.Hq / a.Hkv; a.batch = batch;
+    a.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->head_dim);
+    a.scale_log2 = a.scale * 1.4426950408889634f;
+    a.cu = cu; a.pl = pl; a.err = err;
+    a.q = (const __nv_bfloat16 *)q; a.kk = (const __nv_bfloat16 *)k; a.v = (const __nv_bfloat16 *)v;
+    a.o = (const __nv_bfloat16 *)o; a.dout = (const __nv_bfloat16 *)dout; a.lse = lse;
+    a.dq = (__nv_bfloat16 *)dq; a.dk = (__nv_bfloat16 *)dk; a.dv = (__nv_bfloat16 *)dv;
+    bw::bwd_blocks_kernel<<<1, 32, 0, st>>>(batch, cu, p->k, const_cast<int32_t *>(a.tb_off),
+                                            const_cast<int32_t *>(a.sb_off));
+    const int64_t cells = aug_rows * a.Hq;
+    bw::bwd_dot_kernel<<<(unsigned)((cells + 255) / 256), 256, 0, st>>>(a, aug_rows, p->head_dim);
+    // upper bound of the block count; CTAs past the real count exit
+    const int64_t nblk = total_text / bw::RB + (total_text / p->k) / bw::RB + 2LL * batch;
+    if (nblk > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
+    if (p->head_dim == 128) {
+        if (bw_launch<128>(a, nblk, st) != KSA_OK) return KSA_ERR_CUDA;
+    } else if (p->head_dim == 64) {
+        if (bw_launch<64>(a, nblk, st) != KSA_OK) return KSA_ERR_CUDA;
+    } else {
+        return KSA_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
+}
+
+}  // namespace ksa

@@ -1,0 +1,73 @@
+"""GPU parity of ksa_prefill_bwd (gradients of Eq. (10) of the Kwai Summary
+Attention Technical Report under the KSA mask, sections 2.2.1-2.2.2) against
+the oracle's fp64 backward, over varlen batches with partial chunks, GQA,
+w = 0 and k = 1.
+
+Tolerance: the kernels feed P and dS to the tensor cores in bf16 (relative
+rounding 2^-9 each) and write bf16 gradients, accumulating in fp32, so the
+gradients carry a few bf16 ulps of relative error: relative Frobenius error
+<= 1e-2 per tensor and max-abs error <= 3e-2 of the tensor's largest entry."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_compression_ksa_b200 import _lib as L
+from kv_cache_compression_ksa_b200.inputs import prefill_inputs
+from ksa_testutil import to_f64
+
+pytestmark = pytest.mark.gpu
+THETA = 1e6
+REL_FROB = 1e-2
+MAX_REL = 3e-2
+
+CASES = [
+    ("varlen_partial_chunks", [100, 37, 8, 3], 8, 2, 8, 2, 128, 11),
+    ("k1_w0", [150, 41], 1, 0, 4, 4, 64, 13),
+    ("k4_gqa4_w3", [300], 4, 3, 16, 4, 128, 12),
+    ("long_summaries", [1500], 8, 4, 8, 2, 128, 15),
+    ("k16_d64", [700, 333], 16, 2, 8, 4, 64, 17),
+]
+
+
+def _check(name, got, want, live):
+    g, w = got[live], want[live]
+    err = np.linalg.norm(g - w) / max(np.linalg.norm(w), 1e-30)
+    mx = np.abs(g - w).max() / max(np.abs(w).max(), 1e-30)
+    assert err <= REL_FROB and mx <= MAX_REL, f"{name}: rel-Frob {err:.3e}, max-abs/max {mx:.3e}"
+
+
+@pytest.mark.parametrize("name,seqlens,k,w,Hq,Hkv,d,seed", CASES, ids=[c[0] for c in CASES])
+def test_prefill_bwd_matches_oracle(name, seqlens, k, w, Hq, Hkv, d, seed):
+    dev = torch.device("cuda")
+    x = prefill_inputs(seqlens, k, Hq, Hkv, d, seed=seed, device=dev)
+    p = L.make_params(k, w, Hq, Hkv, d, 0.0, THETA)
+    nt, ns = sum(seqlens), sum(n // k for n in seqlens)
+    rows = L.ksa_aug_rows(p, seqlens)
+    qa = torch.empty(rows, Hq, d, dtype=torch.bfloat16, device=dev)
+    ka = torch.empty(rows, Hkv, d, dtype=torch.bfloat16, device=dev)
+    va = torch.empty_like(ka)
+    oa = torch.empty_like(qa)
+    lse = torch.empty(rows, Hq, dtype=torch.float32, device=dev)
+    ws = torch.empty(L.ksa_prefill_workspace_size(p, len(seqlens), nt), dtype=torch.uint8, device=dev)
+    L.ksa_interleave_rope(p, x.cu_seqlens, nt, ns, rows, x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum, x.v_sum,
+                          qa, ka, va, ws)
+    L.ksa_prefill_fwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, ws)
+    gen = torch.Generator(device=dev).manual_seed(seed + 100)
+    do = torch.randn(rows, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+    dq = torch.zeros_like(qa)
+    dk = torch.zeros_like(ka)
+    dv = torch.zeros_like(va)
+    wsb = torch.empty(L.ksa_prefill_bwd_workspace_size(p, len(seqlens), rows), dtype=torch.uint8, device=dev)
+    L.ksa_prefill_bwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, do, dq, dk, dv, wsb)
+    torch.cuda.synchronize()
+    assert L.ksa_get_device_error(wsb) == 0
+    want = oracle.ksa_prefill_bwd_aug(seqlens, k, w, to_f64(qa), to_f64(ka), to_f64(va), to_f64(do))
+    live = np.zeros(rows, bool)
+    base = 0
+    for n in seqlens:
+        live[base + oracle.aug_index(n, k)] = True
+        base += ((n + k - 1) // k) * (k + 1)
+    _check(name + " dq", to_f64(dq), want[0], live)
+    _check(name + " dk", to_f64(dk), want[1], live)
+    _check(name + " dv", to_f64(dv), want[2], live)

@@ -467,6 +467,35 @@ def run_sweep(args):
         del x, qa, ka, va, oa, lse, ws, cache
         torch.cuda.empty_cache()
 
+    # backward of the 32768-token prefill (bench shape): useful FLOPs 2.5x the
+    # forward's (five products per visible pair: S, dP, dV, dQ, dK)
+    sl, k, w = PF["seqlens"], PF["k"], PF["w"]
+    x = prefill_inputs(sl, k, Hq, Hkv, d, seed=PF["seed"], scale=PF["scale"], device=dev)
+    p = L.make_params(k, w, Hq, Hkv, d, 0.0, PF["theta"])
+    nt, ns = sum(sl), sum(n // k for n in sl)
+    rows = L.ksa_aug_rows(p, sl)
+    qa = torch.empty(rows, Hq, d, dtype=torch.bfloat16, device=dev)
+    ka = torch.empty(rows, Hkv, d, dtype=torch.bfloat16, device=dev)
+    va = torch.empty_like(ka)
+    oa = torch.empty_like(qa)
+    lse = torch.empty(rows, Hq, dtype=torch.float32, device=dev)
+    ws = torch.empty(L.ksa_prefill_workspace_size(p, len(sl), nt), dtype=torch.uint8, device=dev)
+    L.ksa_interleave_rope(p, x.cu_seqlens, nt, ns, rows, x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum, x.v_sum,
+                          qa, ka, va, ws)
+    L.ksa_prefill_fwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, ws)
+    do = torch.randn(rows, Hq, d, device=dev).to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(qa), torch.empty_like(ka), torch.empty_like(va)
+    wsb = torch.empty(L.ksa_prefill_bwd_workspace_size(p, len(sl), rows), dtype=torch.uint8, device=dev)
+    ms = ev_time(lambda: L.ksa_prefill_bwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, do, dq, dk, dv, wsb))
+    flops = 2.5 * useful_pairs(sl, k, w) * Hq * 4 * d
+    tf = flops / (ms * 1e-3) / 1e12
+    print(json.dumps({"sweep": "prefill_bwd", "workload": "1x32768, 32q/8kv, d128, k8, w8, N(0,1)*0.5 bf16",
+                      "useful_tflop": flops / 1e12, "ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / tc_peak,
+                      "note": "warp-level mma.sync kernels; S and dP are computed in both the dq and the dk/dv pass"}),
+          flush=True)
+    del x, qa, ka, va, oa, lse, ws, do, dq, dk, dv, wsb
+    torch.cuda.empty_cache()
+
     S = SWEEP_DECODE
     k, w = S["k"], S["w"]
     pd = L.make_params(k, w, S["Hq"], S["Hkv"], S["d"], 0.0, 1e6)

@@ -139,8 +139,10 @@ KSA_API int ksa_prefill_fwd(const ksa_params *p, int32_t batch, const int32_t *c
                     void *workspace, size_t workspace_bytes, int32_t *dev_err,
                     void *stream);
 
-/* Workspace bytes for ksa_prefill_bwd (the batch plan, block offsets and an
- * fp32 [aug_rows, Hq] buffer for rowsum(dO * O)). */
+/* Workspace bytes for ksa_prefill_bwd: the batch plan, block offsets, an
+ * fp32 [aug_rows, Hq] buffer for rowsum(dO * O) and fp32 [aug_rows, Hkv, d]
+ * accumulators for dk and dv (a key block's query range is split over
+ * several CTAs that add their shares). */
 KSA_API size_t ksa_prefill_bwd_workspace_size(const ksa_params *p, int32_t batch, int64_t aug_rows);
 
 /* KSA prefill backward: gradients of Eq. (10) under the KSA mask (sections

@@ -18,12 +18,16 @@
 //
 //   bwd_dot_kernel   D = rowsum(dO * O)                          (HBM)
 //   bwd_dq_kernel    query-stationary: dq of 64 rows of one q head
-//   bwd_dkv_kernel   key-stationary: dk, dv of 64 rows of one kv head,
-//                    over all q heads of its group
+//   bwd_dkv_kernel   key-stationary: dk, dv of 64 rows of one kv head, over
+//                    all q heads of its group and (grid z) a share of at
+//                    most 16 of the query blocks that see them, added into
+//                    fp32 accumulators (the first summaries are seen by every
+//                    later text row, so their query ranges are split)
+//   bwd_dkv_out_kernel  accumulators -> bf16
 // Both attention kernels use the warp-level tensor-core MMA (m16n8k16, bf16
 // in, fp32 accumulate) with operands staged in shared memory and read with
-// ldmatrix; each warp owns 16 rows of its block.  No atomics: every output
-// row belongs to exactly one block.
+// ldmatrix; each warp owns 16 rows of its block.  dq rows belong to exactly
+// one block and are written once.
 #include <math.h>
 
 #include "ksa_internal.cuh"
@@ -35,6 +39,7 @@ namespace bw {
 constexpr int RB = 64;          // rows per block
 constexpr int kThreads = 128;   // 4 warps x 16 rows
 constexpr int TEXT_ROWS = 0, SUM_ROWS = 1;
+constexpr int QB_SPLIT = 16;    // query blocks per dk/dv CTA: long query ranges are split
 
 struct Args {
     int k, w, Hq, Hkv, G, batch;
@@ -46,6 +51,8 @@ struct Args {
     const __nv_bfloat16 *q, *kk, *v, *o, *dout;
     const float *lse;                 // [rows, Hq] natural log
     float *dsum;                      // [rows, Hq] D = rowsum(dO * O)
+    float *dk32, *dv32;               // [rows, Hkv, d] fp32 accumulators of the split dk/dv pass
+    int nblk;                         // upper bound of the block count (grid x)
     __nv_bfloat16 *dq, *dk, *dv;
 };
 
@@ -192,7 +199,11 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(Args a)
     Row *sQ = reinterpret_cast<Row *>(bw_smem), *sO = sQ + RB, *sK = sO + RB, *sV = sK + RB;
     if (*a.err != 0) return;
     Blk Q;
-    if (!block_of(a, blockIdx.x, Q)) return;
+    // text blocks late in a sequence see the most summaries: reverse order
+    // puts them first
+    const int nreal = a.tb_off[a.batch] + a.sb_off[a.batch];
+    const int id = (int)blockIdx.x < nreal ? nreal - 1 - (int)blockIdx.x : (int)blockIdx.x;
+    if (!block_of(a, id, Q)) return;
     const int h = blockIdx.y, g = h / a.G;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tt = lane & 3;
     load_rows<D>(sQ, a.q, a.Hq, h, a, Q, Q.idx0, Q.cnt);
@@ -349,9 +360,12 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
     }
     const int ntb = (t_hi - t_lo + RB - 1) / RB;
     const int nsb = s_hi > s_lo ? 1 : 0;   // at most 64 summaries see this block's keys
+    // this CTA's share of the query blocks (split z of ceil((ntb + nsb) / QB_SPLIT))
+    const int qb_lo = (int)blockIdx.z * QB_SPLIT, qb_hi = min(ntb + nsb, qb_lo + QB_SPLIT);
+    if (qb_lo >= ntb + nsb) return;
     for (int hh = 0; hh < a.G; ++hh) {
         const int h = g * a.G + hh;
-        for (int qb = 0; qb < ntb + nsb; ++qb) {
+        for (int qb = qb_lo; qb < qb_hi; ++qb) {
             Blk Q = K;
             if (qb < ntb) {
                 Q.kind = TEXT_ROWS; Q.idx0 = t_lo + qb * RB; Q.cnt = min(RB, t_hi - Q.idx0);
@@ -430,17 +444,34 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
             }
         }
     }
+    // partial sums of this split into the fp32 accumulators
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
         if (!live[x]) continue;
         const int64_t row = aug_row(a, K, ki[x]);
-        __nv_bfloat16 *pk = a.dk + (row * a.Hkv + g) * D;
-        __nv_bfloat16 *pv = a.dv + (row * a.Hkv + g) * D;
+        float *pk = a.dk32 + (row * a.Hkv + g) * D;
+        float *pv = a.dv32 + (row * a.Hkv + g) * D;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            *reinterpret_cast<uint32_t *>(pk + 8 * nt + 2 * tt) = wm::pack2(dk[nt][2 * x] * a.scale, dk[nt][2 * x + 1] * a.scale);
-            *reinterpret_cast<uint32_t *>(pv + 8 * nt + 2 * tt) = wm::pack2(dv[nt][2 * x], dv[nt][2 * x + 1]);
+            atomicAdd(pk + 8 * nt + 2 * tt, dk[nt][2 * x] * a.scale);
+            atomicAdd(pk + 8 * nt + 2 * tt + 1, dk[nt][2 * x + 1] * a.scale);
+            atomicAdd(pv + 8 * nt + 2 * tt, dv[nt][2 * x]);
+            atomicAdd(pv + 8 * nt + 2 * tt + 1, dv[nt][2 * x + 1]);
         }
+    }
+}
+
+// fp32 accumulators -> bf16 dk, dv of the real rows (padding rows untouched)
+__global__ void __launch_bounds__(256) bwd_dkv_out_kernel(Args a, int D)
+{
+    Blk K;
+    if (!block_of(a, blockIdx.x, K)) return;
+    const int g = blockIdx.y;
+    for (int e = threadIdx.x; e < K.cnt * (D / 2); e += 256) {
+        const int r = e / (D / 2), c2 = e % (D / 2);
+        const int64_t off = (aug_row(a, K, K.idx0 + r) * a.Hkv + g) * D + 2 * c2;
+        *reinterpret_cast<uint32_t *>(a.dk + off) = wm::pack2(a.dk32[off], a.dk32[off + 1]);
+        *reinterpret_cast<uint32_t *>(a.dv + off) = wm::pack2(a.dv32[off], a.dv32[off + 1]);
     }
 }
 
@@ -464,7 +495,7 @@ __global__ void bwd_blocks_kernel(int batch, const int32_t *cu, int k, int32_t *
 
 // four 64-row tiles of D + 8 bf16 per row (+ per-query LSE and D for dk, dv)
 template <int D>
-static int bw_launch(const bw::Args &a, int64_t nblk, cudaStream_t st)
+static int bw_launch(const bw::Args &a, int64_t nblk, int64_t zsplits, cudaStream_t st)
 {
     const int tiles = 4 * bw::RB * (D + 8) * 2;
     const int dkv = tiles + 2 * bw::RB * 4;
@@ -477,14 +508,16 @@ static int bw_launch(const bw::Args &a, int64_t nblk, cudaStream_t st)
         attr[D == 128] = true;
     }
     bw::bwd_dq_kernel<D><<<dim3((unsigned)nblk, a.Hq), bw::kThreads, tiles, st>>>(a);
-    bw::bwd_dkv_kernel<D><<<dim3((unsigned)nblk, a.Hkv), bw::kThreads, dkv, st>>>(a);
+    bw::bwd_dkv_kernel<D><<<dim3((unsigned)nblk, a.Hkv, (unsigned)zsplits), bw::kThreads, dkv, st>>>(a);
+    bw::bwd_dkv_out_kernel<<<dim3((unsigned)nblk, a.Hkv), 256, 0, st>>>(a, D);
     return KSA_OK;
 }
 
 size_t prefill_bwd_workspace_bytes(const ksa_params *p, int batch, int64_t aug_rows)
 {
     return plan_bytes(batch) + 2 * align_up(sizeof(int32_t) * (size_t)(batch + 1)) +
-           align_up(sizeof(float) * (size_t)aug_rows * p->num_q_heads);
+           align_up(sizeof(float) * (size_t)aug_rows * p->num_q_heads) +
+           2 * align_up(sizeof(float) * (size_t)aug_rows * p->num_kv_heads * p->head_dim);
 }
 
 int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,
@@ -498,6 +531,11 @@ int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_
     a.tb_off = reinterpret_cast<int32_t *>(w);
     a.sb_off = reinterpret_cast<int32_t *>(w + ab);
     a.dsum = reinterpret_cast<float *>(w + 2 * ab);
+    const size_t dsb = align_up(sizeof(float) * (size_t)aug_rows * p->num_q_heads);
+    const size_t accb = align_up(sizeof(float) * (size_t)aug_rows * p->num_kv_heads * p->head_dim);
+    a.dk32 = reinterpret_cast<float *>(w + 2 * ab + dsb);
+    a.dv32 = reinterpret_cast<float *>(w + 2 * ab + dsb + accb);
+    if (cudaMemsetAsync(a.dk32, 0, 2 * accb, st) != cudaSuccess) return KSA_ERR_CUDA;
     a.k = p->k; a.w = p->w; a.Hq = p->num_q_heads; a.Hkv = p->num_kv_heads; a.G = a.Hq / a.Hkv; a.batch = batch;
     a.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->head_dim);
     a.scale_log2 = a.scale * 1.4426950408889634f;
@@ -512,10 +550,14 @@ int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_
     // upper bound of the block count; CTAs past the real count exit
     const int64_t nblk = total_text / bw::RB + (total_text / p->k) / bw::RB + 2LL * batch;
     if (nblk > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
+    a.nblk = (int)nblk;
+    // query blocks any key block can meet: at most total_text/64 + 2 (text + one summary block)
+    const int64_t zsplits = (total_text / bw::RB + 2 + bw::QB_SPLIT - 1) / bw::QB_SPLIT;
+    if (zsplits > 65535) return KSA_ERR_UNSUPPORTED;
     if (p->head_dim == 128) {
-        if (bw_launch<128>(a, nblk, st) != KSA_OK) return KSA_ERR_CUDA;
+        if (bw_launch<128>(a, nblk, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
     } else if (p->head_dim == 64) {
-        if (bw_launch<64>(a, nblk, st) != KSA_OK) return KSA_ERR_CUDA;
+        if (bw_launch<64>(a, nblk, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
     } else {
         return KSA_ERR_UNSUPPORTED;
     }

@@ -366,3 +366,42 @@ def ksa_prefill_bwd_aug(seqlens, k, C, q_aug, k_aug, v_aug, do_aug, scale=None):
         dq[rows], dk[rows], dv[rows] = g[0], g[1], g[2]
         base += ((n + k - 1) // k) * (k + 1)
     return dq, dk, dv
+
+
+def visible_keys(n: int, k: int, C: int, a: int) -> np.ndarray:
+    """Eq. (1) indices of the keys the query at Eq. (1) index a sees
+    (section 2.2.1: a summary sees its chunk's text and itself; Eqs. (2)-(3):
+    text t_i sees text t_{max(0, c-C)k} .. t_i and summaries s_j, j < c - C)."""
+    m = n // k
+    txt = lambda i: i + i // k                       # Eq. (1) index of text i
+    if a < m * (k + 1) and a % (k + 1) == k:         # summary j
+        j = a // (k + 1)
+        return np.concatenate([txt(np.arange(j * k, j * k + k)), [a]]).astype(np.int64)
+    i = a - min(a // (k + 1), m)                      # text token index
+    c = i // k
+    lo = max(0, c - C) * k
+    summ = np.arange(0, max(0, min(c - C, m))) * (k + 1) + k
+    return np.concatenate([summ, txt(np.arange(lo, i + 1))]).astype(np.int64)
+
+
+def ksa_attention_bwd_dq_rows(n, k, C, q, kk, v, do, rows, scale=None):
+    """dq of the given Eq. (1) query rows only (each row's gradient needs just
+    its own visible keys): the same formulas as ksa_attention_bwd."""
+    q, kk, v, do = (_f64(a) for a in (q, kk, v, do))
+    Hq, d = q.shape[1], q.shape[2]
+    G = Hq // kk.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.zeros((len(rows), Hq, d))
+    for r, a in enumerate(rows):
+        keys = visible_keys(n, k, C, int(a))
+        for h in range(Hq):
+            g = h // G
+            s = scale * (kk[keys, g] @ q[a, h])
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            o = p @ v[keys, g]
+            dp = v[keys, g] @ do[a, h]
+            ds = p * (dp - float(do[a, h] @ o))
+            out[r, h] = scale * (ds @ kk[keys, g])
+    return out

@@ -71,3 +71,47 @@ def test_prefill_bwd_matches_oracle(name, seqlens, k, w, Hq, Hkv, d, seed):
     _check(name + " dq", to_f64(dq), want[0], live)
     _check(name + " dk", to_f64(dk), want[1], live)
     _check(name + " dv", to_f64(dv), want[2], live)
+
+
+def test_prefill_bwd_full_size_identities_and_sampled_rows():
+    """The 32768-token Qwen3-4B-layer prefill (32 q / 8 kv heads, d 128, k 8,
+    w 8): per kv head the key gradients sum to zero and the value gradients
+    sum to the output gradients of its q heads (exact for softmax attention;
+    checked to 1e-2 of the summed magnitudes); sampled dq rows against the
+    oracle's per-row backward."""
+    dev = torch.device("cuda")
+    seqlens, k, w, Hq, Hkv, d = [32768], 8, 8, 32, 8, 128
+    x = prefill_inputs(seqlens, k, Hq, Hkv, d, seed=1, scale=0.5, device=dev)
+    p = L.make_params(k, w, Hq, Hkv, d, 0.0, THETA)
+    nt, ns = sum(seqlens), sum(n // k for n in seqlens)
+    rows = L.ksa_aug_rows(p, seqlens)
+    qa = torch.empty(rows, Hq, d, dtype=torch.bfloat16, device=dev)
+    ka = torch.empty(rows, Hkv, d, dtype=torch.bfloat16, device=dev)
+    va = torch.empty_like(ka)
+    oa = torch.empty_like(qa)
+    lse = torch.empty(rows, Hq, dtype=torch.float32, device=dev)
+    ws = torch.empty(L.ksa_prefill_workspace_size(p, 1, nt), dtype=torch.uint8, device=dev)
+    L.ksa_interleave_rope(p, x.cu_seqlens, nt, ns, rows, x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum, x.v_sum,
+                          qa, ka, va, ws)
+    L.ksa_prefill_fwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, ws)
+    gen = torch.Generator(device=dev).manual_seed(7)
+    do = torch.randn(rows, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(qa), torch.empty_like(ka), torch.empty_like(va)
+    wsb = torch.empty(L.ksa_prefill_bwd_workspace_size(p, 1, rows), dtype=torch.uint8, device=dev)
+    L.ksa_prefill_bwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, do, dq, dk, dv, wsb)
+    torch.cuda.synchronize()
+    assert L.ksa_get_device_error(wsb) == 0
+    # n % k == 0: no padding rows
+    dkf, dvf, dof = dk.double(), dv.double(), do.double()
+    sk = dkf.sum(0)
+    assert (sk.abs().sum(-1) <= 1e-2 * dkf.abs().sum(0).sum(-1)).all()
+    want_v = dof.view(rows, Hkv, Hq // Hkv, d).sum((0, 2))
+    assert ((dvf.sum(0) - want_v).abs().sum(-1) <= 1e-2 * dvf.abs().sum(0).sum(-1)).all()
+    # sampled dq rows (Eq. (1) order = the layout here): text rows early, mid
+    # and late, and summary rows
+    sample = np.array([0, 5, 80, 9 * 1000 + 3, 9 * 2047 + 8, 9 * 3000 + 4, rows - 2, rows - 1])
+    n = seqlens[0]
+    want = oracle.ksa_attention_bwd_dq_rows(n, k, w, to_f64(qa), to_f64(ka), to_f64(va), to_f64(do), sample)
+    got = to_f64(dq)[sample]
+    err = np.linalg.norm(got - want) / np.linalg.norm(want)
+    assert err <= REL_FROB, f"sampled dq rel-Frob {err:.3e}"

@@ -101,3 +101,18 @@ def test_bwd_padded_layout():
         np.testing.assert_array_equal(dk[r], g[1])
         base += ((n + k - 1) // k) * (k + 1)
     assert np.abs(dq[~live]).max() == 0 and np.abs(dk[~live]).max() == 0 and np.abs(dv[~live]).max() == 0
+
+
+@pytest.mark.parametrize("n,k,C", [(40, 4, 2), (35, 8, 1), (13, 1, 0)])
+def test_bwd_dq_rows_match_dense(n, k, C):
+    """The per-row form (closed-form visible set) equals the dense backward,
+    and the visible sets equal the rows of the dense mask."""
+    Hq, Hkv, d = 4, 2, 8
+    q, kk, v, do = _inputs(n, k, Hq, Hkv, d, seed=9)
+    dq = oracle.ksa_attention_bwd(n, k, C, q, kk, v, do)[0]
+    M = oracle.dense_mask(n, k, C)
+    rows = np.arange(q.shape[0])
+    for a in rows:
+        np.testing.assert_array_equal(np.sort(oracle.visible_keys(n, k, C, int(a))), np.nonzero(M[a])[0])
+    np.testing.assert_allclose(oracle.ksa_attention_bwd_dq_rows(n, k, C, q, kk, v, do, rows), dq, rtol=1e-12,
+                               atol=1e-12)

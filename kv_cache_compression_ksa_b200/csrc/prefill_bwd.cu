@@ -126,6 +126,29 @@ __device__ __forceinline__ void load_rows(__nv_bfloat16 (*dst)[D + 8], const __n
     }
 }
 
+// the same, issued as 16-byte cp.async copies (one commit group per call);
+// zero rows are written directly
+template <int D>
+__device__ __forceinline__ void load_rows_async(__nv_bfloat16 (*dst)[D + 8], const __nv_bfloat16 *src, int H, int head,
+                                                const Args &a, const Blk &B, int first, int cnt)
+{
+    constexpr int V8 = D / 8;
+    for (int e = threadIdx.x; e < RB * V8; e += kThreads) {
+        const int r = e / V8, c8 = e % V8;
+        if (r < cnt) {
+            const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(&dst[r][c8 * 8]));
+            const void *g = reinterpret_cast<const uint4 *>(src + (aug_row(a, B, first + r) * H + head) * D) + c8;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(g) : "memory");
+        } else {
+            *reinterpret_cast<uint4 *>(&dst[r][c8 * 8]) = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p)
 {
     const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -196,7 +219,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(Args a)
     constexpr int KC = D / 16, NT = D / 8;
     using Row = __nv_bfloat16[D + 8];
     extern __shared__ __align__(16) uint8_t bw_smem[];
-    Row *sQ = reinterpret_cast<Row *>(bw_smem), *sO = sQ + RB, *sK = sO + RB, *sV = sK + RB;
+    // Q, dO, then two buffers of (K, V)
+    Row *sQ = reinterpret_cast<Row *>(bw_smem), *sO = sQ + RB, *sKV = sO + RB;
     if (*a.err != 0) return;
     Blk Q;
     // text blocks late in a sequence see the most summaries: reverse order
@@ -247,19 +271,35 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(Args a)
         s_lo = Q.idx0;
     }
     const int ntb = (t_hi - t_lo + RB - 1) / RB;
-    for (int kb = 0; kb < nsb + ntb; ++kb) {
+    const int s_end = Q.kind == TEXT_ROWS ? max(0, min((Q.idx0 + Q.cnt - 1) / a.k - a.w, Q.m)) : Q.idx0 + Q.cnt;
+    auto key_block = [&](int kb) {
         Blk K = Q;
         if (kb < nsb) {
-            K.kind = SUM_ROWS; K.idx0 = s_lo + kb * RB;
-            K.cnt = min(RB, (Q.kind == TEXT_ROWS ? max(0, min((Q.idx0 + Q.cnt - 1) / a.k - a.w, Q.m)) : Q.idx0 + Q.cnt) - K.idx0);
+            K.kind = SUM_ROWS; K.idx0 = s_lo + kb * RB; K.cnt = min(RB, s_end - K.idx0);
         } else {
-            K.kind = TEXT_ROWS; K.idx0 = t_lo + (kb - nsb) * RB;
-            K.cnt = min(RB, t_hi - K.idx0);
+            K.kind = TEXT_ROWS; K.idx0 = t_lo + (kb - nsb) * RB; K.cnt = min(RB, t_hi - K.idx0);
         }
-        __syncthreads();   // the previous key block has been read
-        load_rows<D>(sK, a.kk, a.Hkv, g, a, K, K.idx0, K.cnt);
-        load_rows<D>(sV, a.v, a.Hkv, g, a, K, K.idx0, K.cnt);
-        __syncthreads();
+        return K;
+    };
+    auto prefetch = [&](int kb) {   // key block kb -> buffer kb % 2 (one commit group)
+        const Blk K = key_block(kb);
+        Row *b = sKV + (kb & 1) * 2 * RB;
+        load_rows_async<D>(b, a.kk, a.Hkv, g, a, K, K.idx0, K.cnt);
+        load_rows_async<D>(b + RB, a.v, a.Hkv, g, a, K, K.idx0, K.cnt);
+        cp_commit();
+    };
+    const int nkb = nsb + ntb;
+    if (nkb > 0) prefetch(0);
+    for (int kb = 0; kb < nkb; ++kb) {
+        const Blk K = key_block(kb);
+        if (kb + 1 < nkb) {
+            prefetch(kb + 1);
+            cp_wait<1>();
+        } else {
+            cp_wait<0>();
+        }
+        __syncthreads();   // key block kb has landed for every thread
+        Row *sK = sKV + (kb & 1) * 2 * RB, *sV = sK + RB;
         // S = Q K^T and dP = dO V^T: 16 rows x 64 keys
         float s[8][4], dp[8][4];
 #pragma unroll
@@ -302,6 +342,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(Args a)
                 wm::mma16816(acc[2 * np], dsf[j][0], dsf[j][1], dsf[j][2], dsf[j][3], bk[0], bk[1]);
                 wm::mma16816(acc[2 * np + 1], dsf[j][0], dsf[j][1], dsf[j][2], dsf[j][3], bk[2], bk[3]);
             }
+        __syncthreads();   // buffer kb % 2 is read: the next prefetch may overwrite it
     }
     // dq rows: acc[nt] holds (row gr, dims 8nt + 2tt, +1) and (row gr + 8, same dims)
 #pragma unroll
@@ -323,15 +364,14 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
     constexpr int KC = D / 16, NT = D / 8;
     using Row = __nv_bfloat16[D + 8];
     extern __shared__ __align__(16) uint8_t bw_smem[];
-    Row *sK = reinterpret_cast<Row *>(bw_smem), *sV = sK + RB, *sQ = sV + RB, *sO = sQ + RB;
-    float *sL = reinterpret_cast<float *>(sO + RB), *sD = sL + RB;
+    // K, V, then two buffers of (Q, dO), then two buffers of (LSE, D)
+    Row *sK = reinterpret_cast<Row *>(bw_smem), *sV = sK + RB, *sQO = sV + RB;
+    float *sLD = reinterpret_cast<float *>(sQO + 4 * RB);
     if (*a.err != 0) return;
     Blk K;
     if (!block_of(a, blockIdx.x, K)) return;
     const int g = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tt = lane & 3;
-    load_rows<D>(sK, a.kk, a.Hkv, g, a, K, K.idx0, K.cnt);
-    load_rows<D>(sV, a.v, a.Hkv, g, a, K, K.idx0, K.cnt);
     int ki[2];
     bool live[2];
 #pragma unroll
@@ -362,26 +402,48 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
     const int nsb = s_hi > s_lo ? 1 : 0;   // at most 64 summaries see this block's keys
     // this CTA's share of the query blocks (split z of ceil((ntb + nsb) / QB_SPLIT))
     const int qb_lo = (int)blockIdx.z * QB_SPLIT, qb_hi = min(ntb + nsb, qb_lo + QB_SPLIT);
-    if (qb_lo >= ntb + nsb) return;
-    for (int hh = 0; hh < a.G; ++hh) {
-        const int h = g * a.G + hh;
-        for (int qb = qb_lo; qb < qb_hi; ++qb) {
-            Blk Q = K;
-            if (qb < ntb) {
-                Q.kind = TEXT_ROWS; Q.idx0 = t_lo + qb * RB; Q.cnt = min(RB, t_hi - Q.idx0);
+    if (qb_lo >= ntb + nsb) return;   // an empty share (block-uniform), before any load
+    load_rows<D>(sK, a.kk, a.Hkv, g, a, K, K.idx0, K.cnt);
+    load_rows<D>(sV, a.v, a.Hkv, g, a, K, K.idx0, K.cnt);
+    const int nq = qb_hi - qb_lo;   // query blocks per head in this share
+    auto query_block = [&](int qb) {
+        Blk Q = K;
+        if (qb < ntb) {
+            Q.kind = TEXT_ROWS; Q.idx0 = t_lo + qb * RB; Q.cnt = min(RB, t_hi - Q.idx0);
+        } else {
+            Q.kind = SUM_ROWS; Q.idx0 = s_lo; Q.cnt = s_hi - s_lo;
+        }
+        return Q;
+    };
+    auto prefetch = [&](int it) {   // step it = (head, query block) -> buffer it % 2
+        const int h = g * a.G + it / nq;
+        const Blk Q = query_block(qb_lo + it % nq);
+        Row *b = sQO + (it & 1) * 2 * RB;
+        load_rows_async<D>(b, a.q, a.Hq, h, a, Q, Q.idx0, Q.cnt);
+        load_rows_async<D>(b + RB, a.dout, a.Hq, h, a, Q, Q.idx0, Q.cnt);
+        float *ld = sLD + (it & 1) * 2 * RB;
+        for (int r = threadIdx.x; r < RB; r += kThreads) {
+            const bool ok = r < Q.cnt;
+            const int64_t row = ok ? aug_row(a, Q, Q.idx0 + r) : 0;
+            ld[r] = ok ? a.lse[row * a.Hq + h] * 1.4426950408889634f : 0.f;
+            ld[RB + r] = ok ? a.dsum[row * a.Hq + h] : 0.f;
+        }
+        cp_commit();
+    };
+    const int nsteps = a.G * nq;
+    prefetch(0);
+    for (int it = 0; it < nsteps; ++it) {
+        {
+            const Blk Q = query_block(qb_lo + it % nq);
+            if (it + 1 < nsteps) {
+                prefetch(it + 1);
+                cp_wait<1>();
             } else {
-                Q.kind = SUM_ROWS; Q.idx0 = s_lo; Q.cnt = s_hi - s_lo;
+                cp_wait<0>();
             }
-            __syncthreads();   // the previous query block has been read
-            load_rows<D>(sQ, a.q, a.Hq, h, a, Q, Q.idx0, Q.cnt);
-            load_rows<D>(sO, a.dout, a.Hq, h, a, Q, Q.idx0, Q.cnt);
-            for (int r = threadIdx.x; r < RB; r += kThreads) {
-                const bool ok = r < Q.cnt;
-                const int64_t row = ok ? aug_row(a, Q, Q.idx0 + r) : 0;
-                sL[r] = ok ? a.lse[row * a.Hq + h] * 1.4426950408889634f : 0.f;
-                sD[r] = ok ? a.dsum[row * a.Hq + h] : 0.f;
-            }
-            __syncthreads();
+            __syncthreads();   // step it has landed for every thread
+            Row *sQ = sQO + (it & 1) * 2 * RB, *sO = sQ + RB;
+            const float *sL = sLD + (it & 1) * 2 * RB, *sD = sL + RB;
             // two halves of 32 queries: S^T = K Q^T, dP^T = V dO^T (16 keys x 32 queries)
 #pragma unroll 1
             for (int hq = 0; hq < 2; ++hq) {
@@ -442,6 +504,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
                         wm::mma16816(dk[2 * np + 1], dsf[j][0], dsf[j][1], dsf[j][2], dsf[j][3], bq[2], bq[3]);
                     }
             }
+            __syncthreads();   // buffer it % 2 is read: the next prefetch may overwrite it
         }
     }
     // partial sums of this split into the fp32 accumulators
@@ -497,8 +560,8 @@ __global__ void bwd_blocks_kernel(int batch, const int32_t *cu, int k, int32_t *
 template <int D>
 static int bw_launch(const bw::Args &a, int64_t nblk, int64_t zsplits, cudaStream_t st)
 {
-    const int tiles = 4 * bw::RB * (D + 8) * 2;
-    const int dkv = tiles + 2 * bw::RB * 4;
+    const int tiles = 6 * bw::RB * (D + 8) * 2;              // Q, dO + two (K, V) / K, V + two (Q, dO)
+    const int dkv = tiles + 2 * 2 * bw::RB * 4;               // + two (LSE, D)
     static bool attr[2] = {false, false};
     if (!attr[D == 128]) {
         if (cudaFuncSetAttribute(bw::bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, tiles) !=

@@ -124,6 +124,21 @@ KSA_API int ksa_interleave_rope(const ksa_params *p, int32_t batch, const int32_
                         void *workspace, size_t workspace_bytes, int32_t *dev_err,
                         void *stream);
 
+/* Backward of ksa_interleave_rope: from the gradients of the augmented rows
+ * (dq_aug [aug_rows, Hq, d], dk_aug / dv_aug [aug_rows, Hkv, d], e.g. from
+ * ksa_prefill_bwd) to the gradients of the text and summary projections,
+ * laid out as the forward's inputs (dq_text [total_text, Hq, d] ...,
+ * dq_sum [total_sum, Hq, d] ...).  The rotation is orthogonal: q and k
+ * gradients are rotated by the opposite angle at the same positions; v
+ * gradients are copied.  Padding rows are ignored.  Arguments otherwise as
+ * for ksa_interleave_rope. */
+KSA_API int ksa_interleave_rope_bwd(const ksa_params *p, int32_t batch, const int32_t *cu_seqlens,
+                            int64_t total_text, int64_t total_sum, int64_t aug_rows,
+                            const void *dq_aug, const void *dk_aug, const void *dv_aug,
+                            void *dq_text, void *dk_text, void *dv_text,
+                            void *dq_sum, void *dk_sum, void *dv_sum,
+                            void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream);
+
 /* KSA prefill forward (Eqs. (2), (3), (10); block-sparse kernel of
  * section 2.3).  q_aug/k_aug/v_aug: the augmented layout (bf16, rotated).
  * o_aug [aug_rows, Hq, d] bf16: attention output of every real row (text

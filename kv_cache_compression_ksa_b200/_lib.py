@@ -67,6 +67,8 @@ SYMBOLS = {
     "ksa_prefill_workspace_size": (_SZ, [ctypes.POINTER(ksa_params), _I32, _I64]),
     "ksa_interleave_rope": (ctypes.c_int, [ctypes.POINTER(ksa_params), _I32, _P, _I64, _I64, _I64,
                                            _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "ksa_interleave_rope_bwd": (ctypes.c_int, [ctypes.POINTER(ksa_params), _I32, _P, _I64, _I64, _I64,
+                                               _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "ksa_prefill_fwd": (ctypes.c_int, [ctypes.POINTER(ksa_params), _I32, _P, _I64, _I64,
                                        _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "ksa_prefill_bwd_workspace_size": (_SZ, [ctypes.POINTER(ksa_params), _I32, _I64]),
@@ -155,6 +157,16 @@ def ksa_interleave_rope(p, cu_seqlens, total_text, total_sum, aug_rows, q_text, 
         _ptr(q_aug), _ptr(k_aug), _ptr(v_aug), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(dev_err), _stream(stream))
     _check("ksa_interleave_rope", rc)
+
+
+def ksa_interleave_rope_bwd(p, cu_seqlens, total_text, total_sum, aug_rows, dq_aug, dk_aug, dv_aug,
+                            dq_text, dk_text, dv_text, dq_sum, dk_sum, dv_sum, workspace, dev_err=None, stream=None):
+    rc = load().ksa_interleave_rope_bwd(
+        ctypes.byref(p), cu_seqlens.numel() - 1, _ptr(cu_seqlens), total_text, total_sum, aug_rows,
+        _ptr(dq_aug), _ptr(dk_aug), _ptr(dv_aug), _ptr(dq_text), _ptr(dk_text), _ptr(dv_text), _ptr(dq_sum),
+        _ptr(dk_sum), _ptr(dv_sum), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_err),
+        _stream(stream))
+    _check("ksa_interleave_rope_bwd", rc)
 
 
 def ksa_prefill_fwd(p, cu_seqlens, total_text, aug_rows, q_aug, k_aug, v_aug, o_aug, lse, workspace,

@@ -124,6 +124,31 @@ int ksa_interleave_rope(const ksa_params *p, int32_t batch, const int32_t *cu_se
                                   q_aug, k_aug, v_aug, pl, err, st);
 }
 
+int ksa_interleave_rope_bwd(const ksa_params *p, int32_t batch, const int32_t *cu_seqlens, int64_t total_text,
+                            int64_t total_sum, int64_t aug_rows, const void *dq_aug, const void *dk_aug,
+                            const void *dv_aug, void *dq_text, void *dk_text, void *dv_text, void *dq_sum,
+                            void *dk_sum, void *dv_sum, void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                            void *stream)
+{
+    int rc = check_prefill_common(p, batch, cu_seqlens, total_text, aug_rows, workspace, workspace_bytes);
+    if (rc != KSA_OK) return rc;
+    if (total_sum < 0 || total_sum > total_text / p->k) return KSA_ERR_INVALID;
+    if (total_text > 0 && (!dq_text || !dk_text || !dv_text)) return KSA_ERR_INVALID;
+    if (total_sum > 0 && (!dq_sum || !dk_sum || !dv_sum)) return KSA_ERR_INVALID;
+    if (aug_rows > 0 && (!dq_aug || !dk_aug || !dv_aug)) return KSA_ERR_INVALID;
+    const void *ptrs[] = {dq_text, dk_text, dv_text, dq_sum, dk_sum, dv_sum, dq_aug, dk_aug, dv_aug};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return KSA_ERR_INVALID;
+    if (reinterpret_cast<uintptr_t>(dev_err) & 3u) return KSA_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    Plan pl = plan_view(workspace, batch);
+    int32_t *err = dev_err ? dev_err : pl.err;
+    rc = launch_plan(p, batch, cu_seqlens, total_text, total_sum, aug_rows, pl, err, 0, st);
+    if (rc != KSA_OK) return rc;
+    return launch_interleave_rope_bwd(p, batch, cu_seqlens, aug_rows, dq_aug, dk_aug, dv_aug, dq_text, dk_text,
+                                      dv_text, dq_sum, dk_sum, dv_sum, pl, err, st);
+}
+
 int ksa_prefill_fwd(const ksa_params *p, int32_t batch, const int32_t *cu_seqlens, int64_t total_text,
                     int64_t aug_rows, const void *q_aug, const void *k_aug, const void *v_aug, void *o_aug,
                     float *lse, void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream)

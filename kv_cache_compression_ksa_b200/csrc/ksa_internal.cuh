@@ -58,6 +58,10 @@ int launch_interleave_rope(const ksa_params *p, int batch, const int32_t *cu, in
                            const void *ks, const void *vs, void *qa, void *ka, void *va,
                            const Plan &pl, int32_t *err, cudaStream_t st);
 
+int launch_interleave_rope_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_t aug_rows,
+                               const void *dqa, const void *dka, const void *dva, void *dqt, void *dkt, void *dvt,
+                               void *dqs, void *dks, void *dvs, const Plan &pl, int32_t *err, cudaStream_t st);
+
 // Prefill backward (prefill_bwd.cu).
 size_t prefill_bwd_workspace_bytes(const ksa_params *p, int batch, int64_t aug_rows);
 int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,

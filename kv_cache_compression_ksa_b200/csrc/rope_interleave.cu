@@ -124,6 +124,12 @@ __device__ __forceinline__ void rot8(uint4 &lo, uint4 &hi, const float *cs, cons
     }
 }
 
+// BWD: the backward (gradients of the augmented rows -> gradients of the
+// text and summary projections).  The rotation is orthogonal, so its
+// transpose is the rotation by the opposite angle; V is copied back; padding
+// rows have no source and are skipped.  In that mode qa/ka/va are read and
+// qt/kt/vt/qs/ks/vs written.
+template <bool BWD>
 __global__ void __launch_bounds__(kRopeThreads)
 interleave_rope_kernel(RopeArgs a)
 {
@@ -170,7 +176,7 @@ interleave_rope_kernel(RopeArgs a)
         float c = 1.f, s = 0.f;
         if (a.rotate) rope_cos_sin((double)s_pos[r], pr, a.d, a.log2_theta, &c, &s);
         s_cos[r][pr] = c;
-        s_sin[r][pr] = s;
+        s_sin[r][pr] = BWD ? -s : s;
     }
     __syncthreads();
     const int qv = a.Hq * a.d / 16;   // rotate items per Q row (8 pairs each)
@@ -191,6 +197,17 @@ interleave_rope_kernel(RopeArgs a)
             int h = j / chunks_half, c = j % chunks_half;
             // uint4 index of element (row, h, 8c) with d/8 uint4 per head row
             int64_t base_out = (R * H + h) * (a.d / 8);
+            if (BWD) {
+                if (src < 0) continue;
+                const uint4 *in = isq ? a.qa : a.ka;
+                uint4 lo = in[base_out + c], hi = in[base_out + c + chunks_half];
+                rot8(lo, hi, cs + 8 * c, sn + 8 * c);
+                uint4 *out = const_cast<uint4 *>(isq ? (s_is_sum[r] ? a.qs : a.qt) : (s_is_sum[r] ? a.ks : a.kt));
+                int64_t base_in = (src * H + h) * (a.d / 8);
+                out[base_in + c] = lo;
+                out[base_in + c + chunks_half] = hi;
+                continue;
+            }
             uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
             if (src >= 0) {
                 const uint4 *in = isq ? (s_is_sum[r] ? a.qs : a.qt) : (s_is_sum[r] ? a.ks : a.kt);
@@ -205,6 +222,12 @@ interleave_rope_kernel(RopeArgs a)
         } else {
             int j = it - qv - kv;
             int64_t o = R * (int64_t)a.Hkv * (a.d / 8) + j;
+            if (BWD) {
+                if (src < 0) continue;
+                uint4 *out = const_cast<uint4 *>(s_is_sum[r] ? a.vs : a.vt);
+                out[src * (int64_t)a.Hkv * (a.d / 8) + j] = a.va[o];
+                continue;
+            }
             uint4 val = make_uint4(0, 0, 0, 0);
             if (src >= 0) {
                 const uint4 *in = s_is_sum[r] ? a.vs : a.vt;
@@ -232,7 +255,27 @@ int launch_interleave_rope(const ksa_params *p, int batch, const int32_t *cu, in
     a.qa = (uint4 *)qa; a.ka = (uint4 *)ka; a.va = (uint4 *)va;
     int64_t blocks = (aug_rows + kRows - 1) / kRows;
     if (blocks > INT32_MAX) return KSA_ERR_UNSUPPORTED;
-    interleave_rope_kernel<<<(unsigned)blocks, kRopeThreads, 0, st>>>(a);
+    interleave_rope_kernel<false><<<(unsigned)blocks, kRopeThreads, 0, st>>>(a);
+    return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
+}
+
+int launch_interleave_rope_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_t aug_rows,
+                               const void *dqa, const void *dka, const void *dva, void *dqt, void *dkt, void *dvt,
+                               void *dqs, void *dks, void *dvs, const Plan &pl, int32_t *err, cudaStream_t st)
+{
+    if (aug_rows == 0) return KSA_OK;
+    RopeArgs a;
+    a.batch = batch; a.k = p->k; a.Hq = p->num_q_heads; a.Hkv = p->num_kv_heads; a.d = p->head_dim;
+    a.aug_rows = aug_rows;
+    a.rotate = p->rope_theta > 0.0;
+    a.log2_theta = a.rotate ? log2(p->rope_theta) : 0.0;
+    a.cu = cu; a.pl = pl; a.err = err;
+    a.qt = (const uint4 *)dqt; a.kt = (const uint4 *)dkt; a.vt = (const uint4 *)dvt;
+    a.qs = (const uint4 *)dqs; a.ks = (const uint4 *)dks; a.vs = (const uint4 *)dvs;
+    a.qa = (uint4 *)dqa; a.ka = (uint4 *)dka; a.va = (uint4 *)dva;
+    int64_t blocks = (aug_rows + kRows - 1) / kRows;
+    if (blocks > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+    interleave_rope_kernel<true><<<(unsigned)blocks, kRopeThreads, 0, st>>>(a);
     return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
 }
 

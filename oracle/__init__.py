@@ -405,3 +405,29 @@ def ksa_attention_bwd_dq_rows(n, k, C, q, kk, v, do, rows, scale=None):
             ds = p * (dp - float(do[a, h] @ o))
             out[r, h] = scale * (ds @ kk[keys, g])
     return out
+
+
+def interleave_rope_bwd(seqlens, k, theta, dq_aug, dk_aug, dv_aug):
+    """Gradients of the text and summary projections from those of the
+    augmented rows: the transpose of Eq. (1)'s interleave and of RoPE (an
+    orthogonal rotation, so its transpose rotates by the opposite angle).
+    Returns (dq_text, dk_text, dv_text, dq_sum, dk_sum, dv_sum), packed by
+    sequence like the forward's inputs."""
+    dq_aug, dk_aug, dv_aug = (_f64(a) for a in (dq_aug, dk_aug, dv_aug))
+    out = [[], [], [], [], [], []]
+    base = 0
+    for n in seqlens:
+        m = n // k
+        i = np.arange(n)
+        tr = base + (i // k) * (k + 1) + i % k
+        sr = base + np.arange(m) * (k + 1) + k
+        pt, ps = text_positions(n), summary_positions(n, k)
+        neg = lambda x, pos: rope(x, -pos, theta) if theta and theta > 0 else x
+        out[0].append(neg(dq_aug[tr], pt))
+        out[1].append(neg(dk_aug[tr], pt))
+        out[2].append(dv_aug[tr])
+        out[3].append(neg(dq_aug[sr], ps) if m else dq_aug[sr])
+        out[4].append(neg(dk_aug[sr], ps) if m else dk_aug[sr])
+        out[5].append(dv_aug[sr])
+        base += ((n + k - 1) // k) * (k + 1)
+    return tuple(np.concatenate(x) for x in out)

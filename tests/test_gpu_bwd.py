@@ -115,3 +115,62 @@ def test_prefill_bwd_full_size_identities_and_sampled_rows():
     got = to_f64(dq)[sample]
     err = np.linalg.norm(got - want) / np.linalg.norm(want)
     assert err <= REL_FROB, f"sampled dq rel-Frob {err:.3e}"
+
+
+@pytest.mark.parametrize("seqlens,k,w,Hq,Hkv,d", [([100, 37, 8, 3], 8, 2, 8, 2, 128), ([150, 41], 4, 1, 4, 4, 64)])
+def test_training_chain_gradients_of_the_projections(seqlens, k, w, Hq, Hkv, d):
+    """The whole prefill training step: text/summary projections -> RoPE +
+    interleave -> attention -> loss sum(dO * O) and back through
+    ksa_prefill_bwd and ksa_interleave_rope_bwd, against the oracle's chain
+    (its own fp64 rotation of the same inputs, its backward, the transpose of
+    the rotation)."""
+    dev = torch.device("cuda")
+    x = prefill_inputs(seqlens, k, Hq, Hkv, d, seed=21, device=dev)
+    p = L.make_params(k, w, Hq, Hkv, d, 0.0, THETA)
+    nt, ns = sum(seqlens), sum(n // k for n in seqlens)
+    rows = L.ksa_aug_rows(p, seqlens)
+    qa = torch.empty(rows, Hq, d, dtype=torch.bfloat16, device=dev)
+    ka = torch.empty(rows, Hkv, d, dtype=torch.bfloat16, device=dev)
+    va = torch.empty_like(ka)
+    oa = torch.empty_like(qa)
+    lse = torch.empty(rows, Hq, dtype=torch.float32, device=dev)
+    ws = torch.empty(L.ksa_prefill_workspace_size(p, len(seqlens), nt), dtype=torch.uint8, device=dev)
+    L.ksa_interleave_rope(p, x.cu_seqlens, nt, ns, rows, x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum, x.v_sum,
+                          qa, ka, va, ws)
+    L.ksa_prefill_fwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, ws)
+    gen = torch.Generator(device=dev).manual_seed(22)
+    do = torch.randn(rows, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+    dqa, dka, dva = torch.zeros_like(qa), torch.zeros_like(ka), torch.zeros_like(va)
+    wsb = torch.empty(L.ksa_prefill_bwd_workspace_size(p, len(seqlens), rows), dtype=torch.uint8, device=dev)
+    L.ksa_prefill_bwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, do, dqa, dka, dva, wsb)
+    outs = [torch.empty_like(t) for t in (x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum, x.v_sum)]
+    L.ksa_interleave_rope_bwd(p, x.cu_seqlens, nt, ns, rows, dqa, dka, dva, *outs, ws)
+    torch.cuda.synchronize()
+    # the oracle's chain from the same bf16 inputs
+    f64 = lambda t: to_f64(t)
+    base = 0
+    qa64, ka64, va64 = (np.zeros((rows, H, d)) for H in (Hq, Hkv, Hkv))
+    t0 = s0 = 0
+    for n in seqlens:
+        m = n // k
+        i = np.arange(n)
+        tr = base + (i // k) * (k + 1) + i % k
+        sr = base + np.arange(m) * (k + 1) + k
+        pt, ps = oracle.text_positions(n), oracle.summary_positions(n, k)
+        qa64[tr] = oracle.rope(f64(x.q_text[t0:t0 + n]), pt, THETA)
+        ka64[tr] = oracle.rope(f64(x.k_text[t0:t0 + n]), pt, THETA)
+        va64[tr] = f64(x.v_text[t0:t0 + n])
+        if m:
+            qa64[sr] = oracle.rope(f64(x.q_sum[s0:s0 + m]), ps, THETA)
+            ka64[sr] = oracle.rope(f64(x.k_sum[s0:s0 + m]), ps, THETA)
+            va64[sr] = f64(x.v_sum[s0:s0 + m])
+        base += ((n + k - 1) // k) * (k + 1)
+        t0 += n
+        s0 += m
+    g = oracle.ksa_prefill_bwd_aug(seqlens, k, w, qa64, ka64, va64, f64(do))
+    want = oracle.interleave_rope_bwd(seqlens, k, THETA, *g)
+    names = ["dq_text", "dk_text", "dv_text", "dq_sum", "dk_sum", "dv_sum"]
+    for nm, got, wt in zip(names, outs, want):
+        allrows = np.ones(wt.shape[0], bool)
+        if wt.shape[0]:
+            _check(nm, f64(got), wt, allrows)

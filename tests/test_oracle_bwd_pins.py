@@ -116,3 +116,45 @@ def test_bwd_dq_rows_match_dense(n, k, C):
         np.testing.assert_array_equal(np.sort(oracle.visible_keys(n, k, C, int(a))), np.nonzero(M[a])[0])
     np.testing.assert_allclose(oracle.ksa_attention_bwd_dq_rows(n, k, C, q, kk, v, do, rows), dq, rtol=1e-12,
                                atol=1e-12)
+
+
+def test_rope_transpose_and_inverse():
+    """RoPE is a rotation: rotating by -pos undoes it, and it is its own
+    transpose's inverse (<R x, g> = <x, R^T g>)."""
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((50, 3, 16))
+    g = rng.standard_normal((50, 3, 16))
+    pos = rng.integers(0, 100000, 50)
+    rx = oracle.rope(x, pos, 1e6)
+    np.testing.assert_allclose(oracle.rope(rx, -pos, 1e6), x, rtol=1e-12, atol=1e-12)
+    assert abs((rx * g).sum() - (x * oracle.rope(g, -pos, 1e6)).sum()) < 1e-9
+
+
+def test_interleave_rope_bwd_is_the_transpose():
+    """<interleave_rope(inputs), G> = <inputs, interleave_rope_bwd(G)> for the
+    augmented gradients G (the definition of the backward of a linear map)."""
+    seqlens, k, Hq, Hkv, d, theta = [11, 8, 5], 4, 2, 1, 8, 1e6
+    rng = np.random.default_rng(12)
+    nt, ns = sum(seqlens), sum(n // k for n in seqlens)
+    qt, kt, vt = (rng.standard_normal((nt, H, d)) for H in (Hq, Hkv, Hkv))
+    qs, ks, vs = (rng.standard_normal((ns, H, d)) for H in (Hq, Hkv, Hkv))
+    rows = sum(((n + k - 1) // k) * (k + 1) for n in seqlens)
+    qa, ka, va = np.zeros((rows, Hq, d)), np.zeros((rows, Hkv, d)), np.zeros((rows, Hkv, d))
+    base = t0 = s0 = 0
+    for n in seqlens:
+        m = n // k
+        i = np.arange(n)
+        tr = base + (i // k) * (k + 1) + i % k
+        sr = base + np.arange(m) * (k + 1) + k
+        pt, ps = oracle.text_positions(n), oracle.summary_positions(n, k)
+        qa[tr], ka[tr], va[tr] = oracle.rope(qt[t0:t0 + n], pt, theta), oracle.rope(kt[t0:t0 + n], pt, theta), vt[t0:t0 + n]
+        if m:
+            qa[sr], ka[sr], va[sr] = oracle.rope(qs[s0:s0 + m], ps, theta), oracle.rope(ks[s0:s0 + m], ps, theta), vs[s0:s0 + m]
+        base += ((n + k - 1) // k) * (k + 1)
+        t0 += n
+        s0 += m
+    G = [rng.standard_normal(a.shape) for a in (qa, ka, va)]
+    back = oracle.interleave_rope_bwd(seqlens, k, theta, *G)
+    lhs = sum((a * g).sum() for a, g in zip((qa, ka, va), G))
+    rhs = sum((a * b).sum() for a, b in zip((qt, kt, vt, qs, ks, vs), back))
+    assert abs(lhs - rhs) < 1e-8 * max(1.0, abs(lhs))

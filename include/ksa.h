@@ -233,6 +233,42 @@ KSA_API int ksa_cache_from_prefill(const ksa_params *p, const ksa_cache *cache, 
                            int64_t total_text, int64_t aug_rows, const void *k_aug, const void *v_aug,
                            void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream);
 
+/* Workspace bytes for ksa_prefill_chunk: per-sequence snapshots and block
+ * offsets, and the rotated q and k of the block (total_text + total_sum
+ * rows of Hq + Hkv heads, bf16). */
+KSA_API size_t ksa_prefill_chunk_workspace_size(const ksa_params *p, int32_t batch, int64_t total_text,
+                                                int64_t total_sum);
+
+/* Chunked prefill: a block of new text tokens per sequence, attended against
+ * the sequence's decode cache, then appended to it.  The rows are the
+ * prefill's (Eq. (10) under the rule of sections 2.2.1-2.2.2) for text
+ * positions n0 .. n0+T_b-1 and summaries m0 .. m0+S_b-1 of sequence b, whose
+ * first n0 tokens and m0 summaries are in the cache (state {n0, m0}); the
+ * older keys are read from the slots of section 2.3.1 (Figure 4).
+ * cu_text / cu_sum: device int32 [cache->batch + 1], the new text tokens and
+ * new summaries per sequence (prefix sums; the totals are total_text and
+ * total_sum).  S_b must be floor((f0 + T_b) / k), f0 = n0 - m0 k: each chunk
+ * the block completes brings its summary.  Inputs (bf16, NOT rotated; rotated
+ * here at those positions, a summary at its chunk's last text position):
+ * q_text [total_text, Hq, d], k_text / v_text [total_text, Hkv, d], and the
+ * summary tensors likewise with total_sum rows.  Outputs: o_text
+ * [total_text, Hq, d], o_sum [total_sum, Hq, d] (bf16); lse_text
+ * [total_text, Hq], lse_sum [total_sum, Hq] (fp32, natural log) or NULL.
+ * Afterwards the cache holds what the token-by-token appends (ksa_cache_append)
+ * of the same tokens would leave in every slot a later decode reads, and
+ * state[b] = {n0 + T_b, m0 + S_b}.  A sequence whose state has an error, an
+ * f0 outside [0, k] or the wrong S_b gets state[b].err = KSA_ERR_STATE (too
+ * many summaries for cap_summaries: KSA_ERR_CAPACITY) and neither its rows
+ * nor its cache are written.  Inconsistent cu arrays set *dev_err (or the
+ * workspace's own word when dev_err is NULL) to KSA_ERR_INVALID and nothing
+ * is written.  Supported: d in {64, 128}, any G <= 8, k >= 1, w >= 0.
+ * Runs on the warp-level tensor-core MMA. */
+KSA_API int ksa_prefill_chunk(const ksa_params *p, const ksa_cache *cache, const int32_t *cu_text,
+                              int64_t total_text, const int32_t *cu_sum, int64_t total_sum, const void *q_text,
+                              const void *k_text, const void *v_text, const void *q_sum, const void *k_sum,
+                              const void *v_sum, void *o_text, void *o_sum, float *lse_text, float *lse_sum,
+                              void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream);
+
 /* Workspace bytes for ksa_decode when no sequence has more than max_text
  * text tokens. */
 KSA_API size_t ksa_decode_workspace_size(const ksa_params *p, int32_t batch, int64_t max_text);

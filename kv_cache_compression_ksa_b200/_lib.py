@@ -78,6 +78,9 @@ SYMBOLS = {
     "ksa_cache_append": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _P, _P, _P]),
     "ksa_cache_from_prefill": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _I64, _I64,
                                               _P, _P, _P, _SZ, _P, _P]),
+    "ksa_prefill_chunk_workspace_size": (_SZ, [ctypes.POINTER(ksa_params), _I32, _I64, _I64]),
+    "ksa_prefill_chunk": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _I64, _P, _I64,
+                                         _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "ksa_decode_workspace_size": (_SZ, [ctypes.POINTER(ksa_params), _I32, _I64]),
     "ksa_decode": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _P, _P, _P,
                                   _I64, _P, _SZ, _P]),
@@ -211,6 +214,20 @@ def ksa_cache_from_prefill(p, cache: ksa_cache, cu_seqlens, total_text, aug_rows
                                        _ptr(k_aug), _ptr(v_aug), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _ptr(dev_err), _stream(stream))
     _check("ksa_cache_from_prefill", rc)
+
+
+def ksa_prefill_chunk_workspace_size(p: ksa_params, batch: int, total_text: int, total_sum: int) -> int:
+    return int(load().ksa_prefill_chunk_workspace_size(ctypes.byref(p), batch, total_text, total_sum))
+
+
+def ksa_prefill_chunk(p, cache: ksa_cache, cu_text, total_text, cu_sum, total_sum, q_text, k_text, v_text, q_sum,
+                      k_sum, v_sum, o_text, o_sum, lse_text, lse_sum, workspace, dev_err=None, stream=None):
+    rc = load().ksa_prefill_chunk(
+        ctypes.byref(p), ctypes.byref(cache), _ptr(cu_text), total_text, _ptr(cu_sum), total_sum, _ptr(q_text),
+        _ptr(k_text), _ptr(v_text), _ptr(q_sum), _ptr(k_sum), _ptr(v_sum), _ptr(o_text), _ptr(o_sum),
+        _ptr(lse_text), _ptr(lse_sum), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(dev_err), _stream(stream))
+    _check("ksa_prefill_chunk", rc)
 
 
 def ksa_decode_workspace_size(p: ksa_params, batch: int, max_text: int) -> int:

@@ -75,6 +75,27 @@ class DecodeCache:
         L.ksa_cache_from_prefill(self.p, self.desc, cu_seqlens, total_text, k_aug.shape[0], k_aug, v_aug, workspace,
                                  stream=stream)
 
+    def chunk_workspace(self, total_text: int, total_sum: int):
+        n = L.ksa_prefill_chunk_workspace_size(self.p, self.batch, total_text, total_sum)
+        return torch.empty(max(n, 16), dtype=torch.uint8, device=self.k.device)
+
+    def prefill_chunk(self, cu_text, total_text: int, cu_sum, total_sum: int, q_text, k_text, v_text,
+                      q_sum, k_sum, v_sum, ws=None, want_lse=True, stream=None):
+        """Chunked prefill: attend a block of new tokens per sequence against
+        the cache, then append them (ksa_prefill_chunk).  Returns
+        (o_text, o_sum, lse_text, lse_sum)."""
+        p = self.p
+        dev = self.k.device
+        o_t = torch.empty(total_text, p.num_q_heads, p.head_dim, dtype=torch.bfloat16, device=dev)
+        o_s = torch.empty(total_sum, p.num_q_heads, p.head_dim, dtype=torch.bfloat16, device=dev)
+        l_t = torch.empty(total_text, p.num_q_heads, dtype=torch.float32, device=dev) if want_lse else None
+        l_s = torch.empty(total_sum, p.num_q_heads, dtype=torch.float32, device=dev) if want_lse else None
+        if ws is None:
+            ws = self.chunk_workspace(total_text, total_sum)
+        L.ksa_prefill_chunk(p, self.desc, cu_text, total_text, cu_sum, total_sum, q_text, k_text, v_text, q_sum,
+                            k_sum, v_sum, o_t, o_s, l_t, l_s, ws, stream=stream)
+        return o_t, o_s, l_t, l_s
+
     def workspace(self, max_text: int):
         n = L.ksa_decode_workspace_size(self.p, self.batch, max_text)
         return torch.empty(max(n, 16), dtype=torch.uint8, device=self.k.device)

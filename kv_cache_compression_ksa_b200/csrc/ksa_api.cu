@@ -253,6 +253,44 @@ int ksa_cache_from_prefill(const ksa_params *p, const ksa_cache *cache, const in
     return launch_cache_build(p, cache, cu_seqlens, k_aug, v_aug, pl, err, st);
 }
 
+size_t ksa_prefill_chunk_workspace_size(const ksa_params *p, int32_t batch, int64_t total_text, int64_t total_sum)
+{
+    if (check_params(p) != KSA_OK || batch < 0 || total_text < 0 || total_sum < 0) return 0;
+    return prefill_chunk_workspace_bytes(p, batch, total_text, total_sum);
+}
+
+int ksa_prefill_chunk(const ksa_params *p, const ksa_cache *cache, const int32_t *cu_text, int64_t total_text,
+                      const int32_t *cu_sum, int64_t total_sum, const void *q_text, const void *k_text,
+                      const void *v_text, const void *q_sum, const void *k_sum, const void *v_sum, void *o_text,
+                      void *o_sum, float *lse_text, float *lse_sum, void *workspace, size_t workspace_bytes,
+                      int32_t *dev_err, void *stream)
+{
+    int rc = check_params(p);
+    if (rc != KSA_OK) return rc;
+    if (!cache || cache->batch < 0 || cache->cap_summaries < 0) return KSA_ERR_INVALID;
+    if (total_text < 0 || total_sum < 0) return KSA_ERR_INVALID;
+    if (total_text > INT32_MAX || total_sum > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+    if (cache->batch == 0) return KSA_OK;
+    if (!cache->k || !cache->v || !cache->state || !aligned16(cache->k) || !aligned16(cache->v)) return KSA_ERR_INVALID;
+    if (cache->batch > 65535) return KSA_ERR_UNSUPPORTED;
+    if ((cache->cap_summaries + 1) * (int64_t)p->k > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+    if (!cu_text || !cu_sum || !workspace || !aligned16(workspace)) return KSA_ERR_INVALID;
+    const void *need_t[] = {q_text, k_text, v_text, o_text};
+    const void *need_s[] = {q_sum, k_sum, v_sum, o_sum};
+    for (const void *x : need_t)
+        if (total_text > 0 && (!x || !aligned16(x))) return KSA_ERR_INVALID;
+    for (const void *x : need_s)
+        if (total_sum > 0 && (!x || !aligned16(x))) return KSA_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(lse_text) & 3u) || (reinterpret_cast<uintptr_t>(lse_sum) & 3u) ||
+        (reinterpret_cast<uintptr_t>(dev_err) & 3u))
+        return KSA_ERR_INVALID;
+    if (workspace_bytes < prefill_chunk_workspace_bytes(p, cache->batch, total_text, total_sum))
+        return KSA_ERR_WORKSPACE;
+    return launch_prefill_chunk(p, cache, cu_text, total_text, cu_sum, total_sum, q_text, k_text, v_text, q_sum,
+                                k_sum, v_sum, o_text, o_sum, lse_text, lse_sum, workspace, dev_err,
+                                (cudaStream_t)stream);
+}
+
 size_t ksa_decode_workspace_size(const ksa_params *p, int32_t batch, int64_t max_text)
 {
     if (check_params(p) != KSA_OK || batch < 0 || max_text < 0) return 0;

@@ -72,6 +72,13 @@ int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_
 int launch_cache_build(const ksa_params *p, const ksa_cache *c, const int32_t *cu, const void *k_aug,
                        const void *v_aug, const Plan &pl, int32_t *err, cudaStream_t st);
 
+// Chunked prefill against a decode cache (prefill_chunk.cu).
+size_t prefill_chunk_workspace_bytes(const ksa_params *p, int batch, int64_t total_text, int64_t total_sum);
+int launch_prefill_chunk(const ksa_params *p, const ksa_cache *c, const int32_t *cu_t, int64_t total_t,
+                         const int32_t *cu_s, int64_t total_s, const void *qt, const void *kt, const void *vt,
+                         const void *qs, const void *ks, const void *vs, void *ot, void *os, float *lt, float *ls,
+                         void *ws, int32_t *dev_err, cudaStream_t st);
+
 int launch_prefill(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text,
                    int64_t aug_rows, const void *qa, const void *ka, const void *va, void *oa,
                    float *lse, const Plan &pl, int32_t *err, cudaStream_t st);
@@ -107,6 +114,26 @@ __device__ __forceinline__ void rope_cos_sin(double pos, int r, int d, double lo
     sincos(ang, &sd, &cd);
     *c = (float)cd;
     *s = (float)sd;
+}
+
+// Rotate-half RoPE of 8 pairs: lo holds x_r .. x_{r+7}, hi holds
+// x_{r+d/2} .. x_{r+d/2+7} (bf16); cs / sn the pairs' cos / sin.  fp32
+// arithmetic, bf16 round-to-nearest-even.  Every kernel that rotates keys
+// uses this one routine, so keys rotated by different calls are identical.
+__device__ __forceinline__ void rope_rot8(uint4 &lo, uint4 &hi, const float *cs, const float *sn)
+{
+    __nv_bfloat162 *a = reinterpret_cast<__nv_bfloat162 *>(&lo);
+    __nv_bfloat162 *b = reinterpret_cast<__nv_bfloat162 *>(&hi);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float2 x = __bfloat1622float2(a[e]);
+        float2 y = __bfloat1622float2(b[e]);
+        float c0 = cs[2 * e], c1 = cs[2 * e + 1], s0 = sn[2 * e], s1 = sn[2 * e + 1];
+        float2 xo = make_float2(x.x * c0 - y.x * s0, x.y * c1 - y.y * s1);
+        float2 yo = make_float2(y.x * c0 + x.x * s0, y.y * c1 + x.y * s1);
+        a[e] = __float22bfloat162_rn(xo);
+        b[e] = __float22bfloat162_rn(yo);
+    }
 }
 
 }  // namespace ksa

@@ -145,50 +145,11 @@ __device__ __forceinline__ void load_rows_async(__nv_bfloat16 (*dst)[D + 8], con
     }
 }
 
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p)
-{
-    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void *p)
-{
-    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
-}
-
-// A fragment (16 rows x 16 cols) at (row0, col0) of a row-major tile
-template <int D>
-__device__ __forceinline__ void frag_a(uint32_t (&r)[4], const __nv_bfloat16 (*t)[D + 8], int row0, int col0)
-{
-    const int l = threadIdx.x & 31;
-    ldsm_x4(r, &t[row0 + (l & 7) + 8 * ((l >> 3) & 1)][col0 + 8 * (l >> 4)]);
-}
-
-// B fragments of two n-tiles from a tile stored [n][k] (rows = n): n-tiles
-// n0 .. n0+7 and n0+8 .. n0+15, k-chunk k0 .. k0+15.  r = {b0, b1 of the
-// first n-tile, b0, b1 of the second}.
-template <int D>
-__device__ __forceinline__ void frag_b_nk(uint32_t (&r)[4], const __nv_bfloat16 (*t)[D + 8], int n0, int k0)
-{
-    const int l = threadIdx.x & 31;
-    ldsm_x4(r, &t[n0 + (l & 7) + 8 * (l >> 4)][k0 + 8 * ((l >> 3) & 1)]);
-}
-
-// B fragments of two n-tiles from a tile stored [k][n] (rows = k): k-chunk
-// k0 .. k0+15, n-tiles n0 .. n0+7 and n0+8 .. n0+15 (transposing load).
-template <int D>
-__device__ __forceinline__ void frag_b_kn(uint32_t (&r)[4], const __nv_bfloat16 (*t)[D + 8], int k0, int n0)
-{
-    const int l = threadIdx.x & 31;
-    ldsm_x4_t(r, &t[k0 + (l & 7) + 8 * ((l >> 3) & 1)][n0 + 8 * (l >> 4)]);
-}
+using wm::cp_commit;
+using wm::cp_wait;
+using wm::frag_a;
+using wm::frag_b_kn;
+using wm::frag_b_nk;
 
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) bwd_dot_kernel(Args a, int64_t rows, int D)

@@ -108,22 +108,6 @@ struct RopeArgs {
     uint4 *qa, *ka, *va;
 };
 
-__device__ __forceinline__ void rot8(uint4 &lo, uint4 &hi, const float *cs, const float *sn)
-{
-    __nv_bfloat162 *a = reinterpret_cast<__nv_bfloat162 *>(&lo);
-    __nv_bfloat162 *b = reinterpret_cast<__nv_bfloat162 *>(&hi);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        float2 x = __bfloat1622float2(a[e]);
-        float2 y = __bfloat1622float2(b[e]);
-        float c0 = cs[2 * e], c1 = cs[2 * e + 1], s0 = sn[2 * e], s1 = sn[2 * e + 1];
-        float2 xo = make_float2(x.x * c0 - y.x * s0, x.y * c1 - y.y * s1);
-        float2 yo = make_float2(y.x * c0 + x.x * s0, y.y * c1 + x.y * s1);
-        a[e] = __float22bfloat162_rn(xo);
-        b[e] = __float22bfloat162_rn(yo);
-    }
-}
-
 // BWD: the backward (gradients of the augmented rows -> gradients of the
 // text and summary projections).  The rotation is orthogonal, so its
 // transpose is the rotation by the opposite angle; V is copied back; padding
@@ -201,7 +185,7 @@ interleave_rope_kernel(RopeArgs a)
                 if (src < 0) continue;
                 const uint4 *in = isq ? a.qa : a.ka;
                 uint4 lo = in[base_out + c], hi = in[base_out + c + chunks_half];
-                rot8(lo, hi, cs + 8 * c, sn + 8 * c);
+                rope_rot8(lo, hi, cs + 8 * c, sn + 8 * c);
                 uint4 *out = const_cast<uint4 *>(isq ? (s_is_sum[r] ? a.qs : a.qt) : (s_is_sum[r] ? a.ks : a.kt));
                 int64_t base_in = (src * H + h) * (a.d / 8);
                 out[base_in + c] = lo;
@@ -214,7 +198,7 @@ interleave_rope_kernel(RopeArgs a)
                 int64_t base_in = (src * H + h) * (a.d / 8);
                 lo = in[base_in + c];
                 hi = in[base_in + c + chunks_half];
-                rot8(lo, hi, cs + 8 * c, sn + 8 * c);
+                rope_rot8(lo, hi, cs + 8 * c, sn + 8 * c);
             }
             uint4 *out = isq ? a.qa : a.ka;
             out[base_out + c] = lo;

@@ -9,8 +9,10 @@ together the per-sequence calls of a packed (varlen) batch.
 Citations are to "Kwai Summary Attention Technical Report": the augmented
 sequence is section 2.2.1 Eq. (1); visibility is section 2.2.1 (summary rule)
 and section 2.2.2 Eqs. (2)-(3); the attention is Eq. (10); the decode cache is
-section 2.3.1 with Figure 4.  The prefill backward (ksa_attention_bwd) is the
-textbook gradient of Eq. (10) under the same mask, written in numpy.
+section 2.3.1 with Figure 4; a chunked prefill (ksa_prefill_chunk) is, by
+definition, a range of rows of the prefill.  The prefill backward
+(ksa_attention_bwd) is the textbook gradient of Eq. (10) under the same mask,
+written in numpy.
 """
 from __future__ import annotations
 
@@ -431,3 +433,20 @@ def interleave_rope_bwd(seqlens, k, theta, dq_aug, dk_aug, dv_aug):
         out[5].append(dv_aug[sr])
         base += ((n + k - 1) // k) * (k + 1)
     return tuple(np.concatenate(x) for x in out)
+
+
+# --------------------------------------------------------------------------
+# Chunked prefill
+# --------------------------------------------------------------------------
+def ksa_prefill_chunk(n0, m0, T, k, C, qt, kt, vt, qs, ks, vs, theta, scale=None):
+    """Rows of a block of T new text tokens appended to a sequence that holds
+    n0 text tokens and m0 summaries (0 <= n0 - m0 k <= k): by definition the
+    prefill rows (Eq. (10) under the KSA mask) of text positions n0 .. n0+T-1
+    and of the summaries m0 .. m1-1, m1 = floor((n0+T)/k), of the sequence's
+    first n0 + T tokens.  qt/kt/vt hold at least n0 + T text rows and qs/ks/vs
+    at least m1 summary rows (not rotated).  Returns one SeqResult."""
+    n1 = n0 + T
+    m1 = n1 // k
+    assert 0 <= n0 - m0 * k <= k and m0 <= m1
+    return ksa_prefill([n1], k, C, qt[:n1], kt[:n1], vt[:n1], qs[:m1], ks[:m1], vs[:m1], theta, scale,
+                       text_rows=[np.arange(n0, n1)], sum_rows=[np.arange(m0, m1)])[0]

@@ -278,6 +278,59 @@ def test_cache_decode_equals_prefill_rows(k, C):
     assert cache.n_text == n and cache.m == m
 
 
+@pytest.mark.parametrize("k,C,n0,pending,T", [
+    (4, 2, 0, False, 23),    # a block from an empty cache
+    (4, 2, 10, False, 13),   # open chunk with 2 cached tokens, ring wraps inside the block
+    (4, 2, 12, True, 9),     # chunk 2 complete, its summary still to come
+    (3, 1, 7, False, 0),     # an empty block
+    (8, 0, 16, True, 0),     # only the pending summary
+    (1, 2, 5, False, 6),     # k = 1: every token completes a chunk
+    (2, 4, 9, False, 21),    # w larger than the chunks before the block
+])
+def test_chunk_rows_equal_decode_steps(k, C, n0, pending, T):
+    """A chunked prefill's rows (by definition, prefill rows n0 .. n0+T-1 and
+    the summaries of the chunks the block completes) equal the decode steps
+    of the same tokens against the cache of the first n0 -- two mechanisms
+    (Eq. (3) enumeration vs the slot map of Figure 4) that must agree."""
+    rng = np.random.default_rng(100 + 13 * k + n0 + T)
+    Hq, Hkv, d, theta = 4, 2, 8, 1e6
+    n1 = n0 + T
+    m1 = n1 // k
+    m0 = n0 // k - (1 if pending else 0)
+    qt, kt, vt = _rand(rng, n1, Hq, d), _rand(rng, n1, Hkv, d), _rand(rng, n1, Hkv, d)
+    qs, ks, vs = _rand(rng, m1, Hq, d), _rand(rng, m1, Hkv, d), _rand(rng, m1, Hkv, d)
+    ref = oracle.ksa_prefill_chunk(n0, m0, T, k, C, qt, kt, vt, qs, ks, vs, theta)
+    assert ref.text_o.shape[0] == T and ref.sum_o.shape[0] == m1 - m0
+    pt, ps = oracle.text_positions(n1), oracle.summary_positions(n1, k)
+    rq, rk = oracle.rope(qt, pt, theta), oracle.rope(kt, pt, theta)
+    sq = oracle.rope(qs, ps, theta) if m1 else qs
+    sk = oracle.rope(ks, ps, theta) if m1 else ks
+    cache = oracle.Cache(k, C, Hkv, d, cap=m1 + 1)
+    for i in range(n0):
+        assert cache.append_text(rk[i], vt[i]) == 0
+        if (i + 1) % k == 0 and (i + 1) // k - 1 < m0:
+            assert cache.append_summary(sk[(i + 1) // k - 1], vs[(i + 1) // k - 1]) == 0
+    assert cache.n_text == n0 and cache.m == m0
+    if pending:
+        assert cache.append_summary(sk[m0], vs[m0]) == 0
+        o, l = cache.decode(oracle.SUMMARY, sq[m0])
+        np.testing.assert_allclose(o, ref.sum_o[0], atol=1e-12)
+        np.testing.assert_allclose(l, ref.sum_lse[0], atol=1e-12)
+    for t in range(T):
+        i = n0 + t
+        assert cache.append_text(rk[i], vt[i]) == 0
+        o, l = cache.decode(oracle.TEXT, rq[i])
+        np.testing.assert_allclose(o, ref.text_o[t], atol=1e-12)
+        np.testing.assert_allclose(l, ref.text_lse[t], atol=1e-12)
+        if (i + 1) % k == 0:
+            j = (i + 1) // k - 1
+            assert cache.append_summary(sk[j], vs[j]) == 0
+            o, l = cache.decode(oracle.SUMMARY, sq[j])
+            np.testing.assert_allclose(o, ref.sum_o[j - m0], atol=1e-12)
+            np.testing.assert_allclose(l, ref.sum_lse[j - m0], atol=1e-12)
+    assert cache.n_text == n1 and cache.m == m1
+
+
 def test_cache_slot_map_contents():
     """The documented slot map, checked slot by slot after a run that wraps
     the ring: scratch = newest summary, summaries in order from slot

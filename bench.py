@@ -36,7 +36,7 @@ PF = dict(seqlens=[32768], k=8, w=8, Hq=32, Hkv=8, d=128, scale=0.5, seed=1, the
 # set to None whenever one of those kernels changes, until it is captured again).
 # The decode capture ran at batch 16; its traffic grows in proportion to the batch.
 TRAFFIC = {
-    "prefill": (660.3e6, "profiles/prefill_kernel_qwen3_4b_32k.md (prefill_kernel<128>)"),
+    "prefill": (661.1e6, "profiles/prefill_kernel_qwen3_4b_32k.md (prefill_kernel<128>)"),
     "decode_per_seq": (1.0851e9 / 16, "profiles/decode_split_kernel_b16_m16384.md (batch 16 capture, per sequence)"),
 }
 DC = dict(B=64, m=16384, k=8, w=8, Hq=32, Hkv=8, d=128, seed=3, theta=1e6)
@@ -55,6 +55,16 @@ def useful_pairs(seqlens, k, w):
 
 def text_pairs(seqlens, k, w):
     return useful_pairs(seqlens, k, w) - sum((n // k) * (k + 1) for n in seqlens)
+
+
+def chunk_pairs(n0, m0, T, k, w):
+    """Visible (query, key) pairs per head of a chunked-prefill block: text
+    positions n0 .. n0+T-1 (Eqs. (2)-(3)) and the summaries m0 .. m1-1 of the
+    chunks it completes (k + 1 keys each)."""
+    i = np.arange(n0, n0 + T, dtype=np.int64)
+    c = i // k
+    text = int(((i - np.maximum(c - w, 0) * k + 1) + np.maximum(c - w, 0)).sum())
+    return text + ((n0 + T) // k - m0) * (k + 1)
 
 
 def decode_slice_rows(m, k, w, fills):
@@ -406,6 +416,12 @@ SWEEP_PREFILL = [
     dict(name="1x32768, chunk 32", seqlens=[32768], k=32, w=8, seed=1),
     dict(name="1x32768, chunk 64 (q heads split over 2 tiles)", seqlens=[32768], k=64, w=8, seed=1),
 ]
+# chunked prefill: (batch, cached tokens per sequence, new tokens per sequence)
+SWEEP_CHUNK = [
+    dict(name="1 x 4096-token block onto a 126976-token cache", B=1, n0=126976, T=4096),
+    dict(name="8 x 2048-token blocks onto 30720-token caches", B=8, n0=30720, T=2048),
+    dict(name="64 x 512-token blocks onto 32765-token caches", B=64, n0=32765, T=512),
+]
 SWEEP_DECODE = dict(batches=[1, 16, 128], contexts=[4096, 32768, 131072, 1048576], k=8, w=8, Hq=32, Hkv=8,
                     d=128, seed=7, text_steps=64)
 
@@ -436,7 +452,8 @@ def run_sweep(args):
             ts.append(a.elapsed_time(b))
         return float(np.median(ts))
 
-    for cfg in SWEEP_PREFILL:
+    parts = set(args.sweep_parts.split(","))
+    for cfg in SWEEP_PREFILL if "prefill" in parts else []:
         sl, k, w = cfg["seqlens"], cfg["k"], cfg["w"]
         x = prefill_inputs(sl, k, Hq, Hkv, d, seed=cfg["seed"], scale=1.0, device=dev)
         p = L.make_params(k, w, Hq, Hkv, d, 0.0, 1e6)
@@ -467,6 +484,55 @@ def run_sweep(args):
         del x, qa, ka, va, oa, lse, ws, cache
         torch.cuda.empty_cache()
 
+    # chunked prefill against a decode cache whose slots are filled straight
+    # from N(0,1) (the cached values do not change the work); each timed call
+    # starts from the same state (n0, m0), restored before the call
+    for cfg in SWEEP_CHUNK if "chunk" in parts else []:
+        k, w, B, n0, T = 8, 8, cfg["B"], cfg["n0"], cfg["T"]
+        p = L.make_params(k, w, Hq, Hkv, d, 0.0, 1e6)
+        m0 = n0 // k
+        S = (n0 - m0 * k + T) // k
+        cache = api.DecodeCache(p, B, cap=m0 + S + 1, device=dev)
+        fill_normal_(cache.k, 31)
+        fill_normal_(cache.v, 32)
+        st0 = torch.tensor([[n0, m0, 0, 0]] * B, dtype=torch.int32, device=dev)
+        gen = torch.Generator(device=dev).manual_seed(33)
+        rnd = lambda r, h: torch.randn(r, h, d, generator=gen, device=dev).to(torch.bfloat16)
+        tx = [rnd(B * T, Hq), rnd(B * T, Hkv), rnd(B * T, Hkv)]
+        sm = [rnd(B * S, Hq), rnd(B * S, Hkv), rnd(B * S, Hkv)]
+        cu_t = torch.arange(0, B + 1, dtype=torch.int32, device=dev) * T
+        cu_s = torch.arange(0, B + 1, dtype=torch.int32, device=dev) * S
+        o_t = torch.empty(B * T, Hq, d, dtype=torch.bfloat16, device=dev)
+        o_s = torch.empty(B * S, Hq, d, dtype=torch.bfloat16, device=dev)
+        l_t = torch.empty(B * T, Hq, dtype=torch.float32, device=dev)
+        l_s = torch.empty(B * S, Hq, dtype=torch.float32, device=dev)
+        cws = cache.chunk_workspace(B * T, B * S)
+        ts = []
+        for it in range(13):
+            cache.state.copy_(st0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            L.ksa_prefill_chunk(p, cache.desc, cu_t, B * T, cu_s, B * S, *tx, *sm, o_t, o_s, l_t, l_s, cws)
+            b.record()
+            torch.cuda.synchronize()
+            if it >= 3:
+                ts.append(a.elapsed_time(b))
+        st = cache.state.cpu().numpy()
+        assert (st[:, 3] == 0).all() and (st[:, 0] == n0 + T).all(), f"chunk state {st[0]}"
+        ms = float(np.median(ts))
+        flops = B * chunk_pairs(n0, m0, T, k, w) * Hq * 4 * d
+        tf = flops / (ms * 1e-3) / 1e12
+        print(json.dumps({"sweep": "prefill_chunk", "workload": cfg["name"] + ", 32q/8kv, d128, k8, w8, N(0,1) bf16",
+                          "useful_tflop": flops / 1e12, "ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / tc_peak,
+                          "note": "whole ksa_prefill_chunk call: plan, RoPE, attention (warp-level mma.sync), "
+                                  "cache append"}), flush=True)
+        del cache, tx, sm, o_t, o_s, l_t, l_s, cws
+        torch.cuda.empty_cache()
+
+    if "bwd" not in parts and "decode" not in parts:
+        return
+    if "bwd" not in parts:
+        return run_decode_sweep(args, L, api, fill_normal_, uniform_ints, dev, hbm_peak, ev_time)
     # backward of the 32768-token prefill (bench shape): useful FLOPs 2.5x the
     # forward's (five products per visible pair: S, dP, dV, dQ, dK)
     sl, k, w = PF["seqlens"], PF["k"], PF["w"]
@@ -495,7 +561,12 @@ def run_sweep(args):
           flush=True)
     del x, qa, ka, va, oa, lse, ws, do, dq, dk, dv, wsb
     torch.cuda.empty_cache()
+    if "decode" in parts:
+        run_decode_sweep(args, L, api, fill_normal_, uniform_ints, dev, hbm_peak, ev_time)
 
+
+def run_decode_sweep(args, L, api, fill_normal_, uniform_ints, dev, hbm_peak, ev_time):
+    import torch
     S = SWEEP_DECODE
     k, w = S["k"], S["w"]
     pd = L.make_params(k, w, S["Hq"], S["Hkv"], S["d"], 0.0, 1e6)
@@ -571,6 +642,8 @@ def main():
                     help="time one leg only (profiling); the JSON line then covers that leg")
     ap.add_argument("--profile", action="store_true", help="skip the e2e and CPU legs (for ncu runs)")
     ap.add_argument("--decode-batch", type=int, default=DC["B"])
+    ap.add_argument("--sweep-parts", default="prefill,chunk,bwd,decode",
+                    help="comma list of the sweep's parts: prefill, chunk, bwd, decode")
     ap.add_argument("--sweep", action="store_true",
                     help="time the long varlen prefill batch and the decode batch x context grid (one JSON line per point)")
     args = ap.parse_args()

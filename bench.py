@@ -422,6 +422,8 @@ SWEEP_CHUNK = [
     dict(name="8 x 2048-token blocks onto 30720-token caches", B=8, n0=30720, T=2048),
     dict(name="64 x 512-token blocks onto 32765-token caches", B=64, n0=32765, T=512),
 ]
+# decode over an MLA latent cache, Table 1's MLA shape (128 heads, d_c 512, d_r 64)
+SWEEP_MLA = dict(batches=[1, 16, 64], contexts=[32768, 131072], k=8, w=8, H=128, seed=9)
 SWEEP_DECODE = dict(batches=[1, 16, 128], contexts=[4096, 32768, 131072, 1048576], k=8, w=8, Hq=32, Hkv=8,
                     d=128, seed=7, text_steps=64)
 
@@ -528,6 +530,41 @@ def run_sweep(args):
                                   "cache append"}), flush=True)
         del cache, tx, sm, o_t, o_s, l_t, l_s, cws
         torch.cuda.empty_cache()
+
+    if "mla" in parts:
+        M = SWEEP_MLA
+        k, w, H = M["k"], M["w"], M["H"]
+        pm = L.make_mla_params(k, w, H, 512, 64, 0.0, 1e6)
+        for B in M["batches"]:
+            for n in M["contexts"]:
+                m = n // k
+                cache = api.MlaCache(pm, B, cap=m + 1, device=dev)
+                fill_normal_(cache.latent, M["seed"] + B)
+                fills = uniform_ints(B, 1, k, seed=M["seed"]).numpy()
+                st = torch.zeros(B, 4, dtype=torch.int32)
+                st[:, 0] = torch.as_tensor(m * k + fills, dtype=torch.int32)
+                st[:, 1] = m
+                cache.state.copy_(st.to(dev))
+                gen = torch.Generator(device=dev).manual_seed(M["seed"])
+                q = torch.randn(B, H, 576, generator=gen, device=dev).to(torch.bfloat16)
+                kind = torch.zeros(B, dtype=torch.int8, device=dev)
+                max_text = m * k + k
+                mws = cache.workspace(max_text)
+                o = torch.empty(B, H, 512, dtype=torch.bfloat16, device=dev)
+                lse_m = torch.empty(B, H, dtype=torch.float32, device=dev)
+                ms = ev_time(lambda: L.ksa_mla_decode(pm, cache.desc, kind, q, o, lse_m, max_text, mws))
+                assert (cache.state[:, 3] == 0).all()
+                rows = float((fills + min(m, w) * k + max(0, m - w)).sum())
+                gbs = rows * 576 * 2 / (ms * 1e-3) / 1e9
+                tf = rows * H * (576 + 512) * 2 / (ms * 1e-3) / 1e12
+                print(json.dumps({"sweep": "mla_decode", "batch": B, "context": n, "summaries": m, "heads": H,
+                                  "ms": ms, "slice_gb": rows * 576 * 2 / 1e9, "gbs": gbs,
+                                  "frac_of_hbm_peak": gbs / hbm_peak, "tflops": tf,
+                                  "frac_of_bf16_peak": tf / tc_peak,
+                                  "note": "one TEXT step over latent rows of d_c 512 + d_r 64; warp-level mma.sync"}),
+                      flush=True)
+                del cache, q, o, lse_m, mws
+                torch.cuda.empty_cache()
 
     if "bwd" not in parts and "decode" not in parts:
         return
@@ -642,8 +679,8 @@ def main():
                     help="time one leg only (profiling); the JSON line then covers that leg")
     ap.add_argument("--profile", action="store_true", help="skip the e2e and CPU legs (for ncu runs)")
     ap.add_argument("--decode-batch", type=int, default=DC["B"])
-    ap.add_argument("--sweep-parts", default="prefill,chunk,bwd,decode",
-                    help="comma list of the sweep's parts: prefill, chunk, bwd, decode")
+    ap.add_argument("--sweep-parts", default="prefill,chunk,mla,bwd,decode",
+                    help="comma list of the sweep's parts: prefill, chunk, mla, bwd, decode")
     ap.add_argument("--sweep", action="store_true",
                     help="time the long varlen prefill batch and the decode batch x context grid (one JSON line per point)")
     args = ap.parse_args()

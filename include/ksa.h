@@ -305,6 +305,62 @@ KSA_API int ksa_decode(const ksa_params *p, const ksa_cache *cache, const int8_t
 KSA_API int ksa_decode_noalloc(const ksa_params *p, const ksa_cache *cache, const int8_t *kind,
                                const void *q, void *o, float *lse, int64_t max_text, void *stream);
 
+/* ------------------------------------------------------------------------
+ * KSA over an MLA latent cache (section 3.2, Eq. (6); MLA as described in
+ * section 3.1: a d_c latent block holding the non-RoPE keys and values and a
+ * decoupled d_r RoPE key block per cached token).
+ *
+ * The cache keeps the slot map of section 2.3.1 above, one latent row of
+ * d_c + d_r bf16 values per slot: latent [batch, slots, d_c + d_r], state as
+ * for ksa_cache.  Decoding uses the absorbed form of MLA: the caller folds
+ * the key up-projection into the query (q_c, d_c values per head) and maps
+ * the d_c-dim output through the value up-projection afterwards.  A head's
+ * score against slot j is scale * (q_c . c_j + q_r . r_j), its output
+ * sum_j softmax_j c_j: multi-query attention over the latent rows.
+ * Supported: d_c = 512, d_r = 64, any num_heads.
+ * ------------------------------------------------------------------------ */
+typedef struct ksa_mla_params {
+    int32_t k;            /* chunk size (>= 1)                                   */
+    int32_t w;            /* sliding chunk number (>= 0)                         */
+    int32_t num_heads;    /* query heads (all read the same latent rows)         */
+    int32_t kv_lora_rank; /* d_c: 512                                            */
+    int32_t rope_dim;     /* d_r: 64                                             */
+    float scale;          /* softmax scale; 0 selects 1/sqrt(d_c + d_r)          */
+    double rope_theta;    /* RoPE base of the d_r part; <= 0 disables RoPE       */
+} ksa_mla_params;
+
+typedef struct ksa_mla_cache {
+    void *latent;          /* [batch, slots, d_c + d_r] bf16                     */
+    int32_t *state;        /* [batch, 4] {n_text, m, 0, err} as for ksa_cache    */
+    int32_t batch;
+    int64_t cap_summaries;
+} ksa_mla_cache;
+
+/* 1 + k + w*k + cap_summaries, or -1 on invalid input. */
+KSA_API int64_t ksa_mla_cache_slots(const ksa_mla_params *p, int64_t cap_summaries);
+
+/* Append one token per sequence to a latent cache: as ksa_cache_append,
+ * with x [batch, d_c + d_r] bf16 the new latent rows (c, then r NOT
+ * rotated; r is rotated here, rotate-half over its d_r dims, at the token's
+ * position: text n_text, summary n_text - 1). */
+KSA_API int ksa_mla_cache_append(const ksa_mla_params *p, const ksa_mla_cache *cache, const int8_t *kind,
+                                 const void *x, void *stream);
+
+/* Workspace bytes for ksa_mla_decode (split shares of each slice: fp32
+ * partial outputs and softmax statistics). */
+KSA_API size_t ksa_mla_decode_workspace_size(const ksa_mla_params *p, int32_t batch, int64_t max_text);
+
+/* One decode step per sequence over its latent slice, after that step's
+ * ksa_mla_cache_append.  q: [batch, num_heads, d_c + d_r] bf16 (q_c, then
+ * q_r NOT rotated; rotated here at position n_text - 1).  Slices and kinds
+ * as for ksa_decode.  o: [batch, num_heads, d_c] bf16, the latent output;
+ * lse: [batch, num_heads] fp32 (natural log) or NULL.  max_text bounds
+ * n_text over the batch and must match the workspace query.  Runs on the
+ * warp-level tensor-core MMA. */
+KSA_API int ksa_mla_decode(const ksa_mla_params *p, const ksa_mla_cache *cache, const int8_t *kind, const void *q,
+                           void *o, float *lse, int64_t max_text, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
 /* Synchronise `stream`, return the device error word (KSA_OK if clear) and
  * reset it to KSA_OK.  dev_err: device int32. */
 KSA_API int ksa_get_device_error(int32_t *dev_err, void *stream);

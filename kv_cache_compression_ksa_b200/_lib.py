@@ -55,6 +55,27 @@ class KsaError(RuntimeError):
         self.status = status
 
 
+class ksa_mla_params(ctypes.Structure):
+    _fields_ = [
+        ("k", ctypes.c_int32),
+        ("w", ctypes.c_int32),
+        ("num_heads", ctypes.c_int32),
+        ("kv_lora_rank", ctypes.c_int32),
+        ("rope_dim", ctypes.c_int32),
+        ("scale", ctypes.c_float),
+        ("rope_theta", ctypes.c_double),
+    ]
+
+
+class ksa_mla_cache(ctypes.Structure):
+    _fields_ = [
+        ("latent", ctypes.c_void_p),
+        ("state", ctypes.c_void_p),
+        ("batch", ctypes.c_int32),
+        ("cap_summaries", ctypes.c_int64),
+    ]
+
+
 _lib = None
 _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
@@ -86,6 +107,12 @@ SYMBOLS = {
                                   _I64, _P, _SZ, _P]),
     "ksa_decode_noalloc": (ctypes.c_int, [ctypes.POINTER(ksa_params), ctypes.POINTER(ksa_cache), _P, _P, _P, _P,
                                           _I64, _P]),
+    "ksa_mla_cache_slots": (_I64, [ctypes.POINTER(ksa_mla_params), _I64]),
+    "ksa_mla_cache_append": (ctypes.c_int, [ctypes.POINTER(ksa_mla_params), ctypes.POINTER(ksa_mla_cache), _P, _P,
+                                            _P]),
+    "ksa_mla_decode_workspace_size": (_SZ, [ctypes.POINTER(ksa_mla_params), _I32, _I64]),
+    "ksa_mla_decode": (ctypes.c_int, [ctypes.POINTER(ksa_mla_params), ctypes.POINTER(ksa_mla_cache), _P, _P, _P, _P,
+                                      _I64, _P, _SZ, _P]),
     "ksa_get_device_error": (ctypes.c_int, [_P, _P]),
     "ksa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -246,6 +273,35 @@ def ksa_decode_noalloc(p, cache: ksa_cache, kind, q, o, lse, max_text, stream=No
     rc = load().ksa_decode_noalloc(ctypes.byref(p), ctypes.byref(cache), _ptr(kind), _ptr(q), _ptr(o), _ptr(lse),
                                    max_text, _stream(stream))
     _check("ksa_decode_noalloc", rc)
+
+
+def make_mla_params(k: int, w: int, num_heads: int, kv_lora_rank: int = 512, rope_dim: int = 64,
+                    scale: float = 0.0, rope_theta: float = 1e6) -> ksa_mla_params:
+    return ksa_mla_params(k, w, num_heads, kv_lora_rank, rope_dim, scale, rope_theta)
+
+
+def make_mla_cache(latent, state, cap_summaries) -> ksa_mla_cache:
+    return ksa_mla_cache(_ptr(latent), _ptr(state), state.shape[0], cap_summaries)
+
+
+def ksa_mla_cache_slots(p: ksa_mla_params, cap_summaries: int) -> int:
+    return int(load().ksa_mla_cache_slots(ctypes.byref(p), cap_summaries))
+
+
+def ksa_mla_cache_append(p, cache: ksa_mla_cache, kind, x, stream=None):
+    rc = load().ksa_mla_cache_append(ctypes.byref(p), ctypes.byref(cache), _ptr(kind), _ptr(x), _stream(stream))
+    _check("ksa_mla_cache_append", rc)
+
+
+def ksa_mla_decode_workspace_size(p: ksa_mla_params, batch: int, max_text: int) -> int:
+    return int(load().ksa_mla_decode_workspace_size(ctypes.byref(p), batch, max_text))
+
+
+def ksa_mla_decode(p, cache: ksa_mla_cache, kind, q, o, lse, max_text, workspace, stream=None):
+    rc = load().ksa_mla_decode(ctypes.byref(p), ctypes.byref(cache), _ptr(kind), _ptr(q), _ptr(o), _ptr(lse),
+                               max_text, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream))
+    _check("ksa_mla_decode", rc)
 
 
 def ksa_get_device_error(dev_err, stream=None) -> int:

@@ -108,3 +108,34 @@ class DecodeCache:
             ws = self.workspace(max_text)
         L.ksa_decode(p, self.desc, kind, q, o, lse, max_text, ws, stream=stream)
         return o, lse
+
+
+class MlaCache:
+    """Latent (MLA) cache [B, slots, d_c + d_r] bf16 + state [B, 4] int32 under
+    the same slot map (include/ksa.h, ksa_mla_*)."""
+
+    def __init__(self, p: L.ksa_mla_params, batch: int, cap: int, device="cuda"):
+        self.p = p
+        self.batch = batch
+        self.cap = cap
+        self.slots = L.ksa_mla_cache_slots(p, cap)
+        self.latent = torch.zeros(batch, self.slots, p.kv_lora_rank + p.rope_dim, dtype=torch.bfloat16,
+                                  device=device)
+        self.state = torch.zeros(batch, 4, dtype=torch.int32, device=device)
+        self.desc = L.make_mla_cache(self.latent, self.state, cap)
+
+    def append(self, kind, x, stream=None):
+        L.ksa_mla_cache_append(self.p, self.desc, kind, x, stream=stream)
+
+    def workspace(self, max_text: int):
+        n = L.ksa_mla_decode_workspace_size(self.p, self.batch, max_text)
+        return torch.empty(max(n, 16), dtype=torch.uint8, device=self.latent.device)
+
+    def decode(self, kind, q, max_text, ws=None, want_lse=True, stream=None):
+        p = self.p
+        o = torch.empty(self.batch, p.num_heads, p.kv_lora_rank, dtype=torch.bfloat16, device=q.device)
+        lse = torch.empty(self.batch, p.num_heads, dtype=torch.float32, device=q.device) if want_lse else None
+        if ws is None:
+            ws = self.workspace(max_text)
+        L.ksa_mla_decode(p, self.desc, kind, q, o, lse, max_text, ws, stream=stream)
+        return o, lse

@@ -286,25 +286,6 @@ __device__ __forceinline__ float ex2f_approx(float x)
     return y;
 }
 
-// Slice of one sequence after its append: [lo, hi) in slots.  Returns false
-// (and records the error) if the state cannot hold a query of this kind.
-__device__ __forceinline__ bool decode_slice(int kind, int64_t n, int64_t m, int k, int w,
-                                             int64_t *lo, int64_t *hi)
-{
-    int64_t f = n - m * k;
-    if (kind == KSA_SUMMARY) {
-        if (m < 1 || f != 0) return false;
-        *lo = 0; *hi = k + 1;
-        return true;
-    }
-    if (f < 1 || f > k) return false;
-    int64_t ring = m < w ? m : w;
-    int64_t far = m > w ? m - w : 0;
-    *lo = k - f + 1;
-    *hi = 1 + k + ring * k + far;
-    return true;
-}
-
 using wm::mma16816;
 using wm::movtrans;
 using wm::word;

@@ -46,6 +46,19 @@ static int check_prefill_shape(const ksa_params *p)
     return KSA_OK;
 }
 
+static int check_mla(const ksa_mla_params *p, const ksa_mla_cache *c, const int8_t *kind)
+{
+    if (!p || !c) return KSA_ERR_INVALID;
+    if (p->k < 1 || p->w < 0 || p->num_heads < 1 || p->kv_lora_rank < 1 || p->rope_dim < 0) return KSA_ERR_INVALID;
+    if (!(p->scale >= 0.f) || isinf(p->scale) || isnan(p->rope_theta)) return KSA_ERR_INVALID;
+    if (p->kv_lora_rank != 512 || p->rope_dim != 64) return KSA_ERR_UNSUPPORTED;
+    if (c->batch < 0 || c->cap_summaries < 0) return KSA_ERR_INVALID;
+    if (c->batch > 0 && (!c->latent || !c->state || !kind || !aligned16(c->latent))) return KSA_ERR_INVALID;
+    if (c->batch > 65535) return KSA_ERR_UNSUPPORTED;
+    if ((c->cap_summaries + 1) * (int64_t)p->k > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+    return KSA_OK;
+}
+
 }  // namespace ksa
 
 using namespace ksa;
@@ -309,6 +322,41 @@ int ksa_decode(const ksa_params *p, const ksa_cache *cache, const int8_t *kind, 
         if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return KSA_ERR_INVALID;
     }
     return launch_decode(p, cache, kind, q, o, lse, max_text, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+int64_t ksa_mla_cache_slots(const ksa_mla_params *p, int64_t cap_summaries)
+{
+    if (!p || p->k < 1 || p->w < 0 || cap_summaries < 0) return -1;
+    return 1 + (int64_t)p->k + (int64_t)p->w * p->k + cap_summaries;
+}
+
+int ksa_mla_cache_append(const ksa_mla_params *p, const ksa_mla_cache *cache, const int8_t *kind, const void *x,
+                         void *stream)
+{
+    int rc = check_mla(p, cache, kind);
+    if (rc != KSA_OK) return rc;
+    if (cache->batch > 0 && (!x || !aligned16(x))) return KSA_ERR_INVALID;
+    return launch_mla_append(p, cache, kind, x, (cudaStream_t)stream);
+}
+
+size_t ksa_mla_decode_workspace_size(const ksa_mla_params *p, int32_t batch, int64_t max_text)
+{
+    if (!p || p->k < 1 || p->w < 0 || p->num_heads < 1 || batch < 0 || max_text < 0) return 0;
+    if (p->kv_lora_rank != 512 || p->rope_dim != 64) return 0;
+    return mla_decode_workspace_bytes(p, batch, max_text);
+}
+
+int ksa_mla_decode(const ksa_mla_params *p, const ksa_mla_cache *cache, const int8_t *kind, const void *q, void *o,
+                   float *lse, int64_t max_text, void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_mla(p, cache, kind);
+    if (rc != KSA_OK) return rc;
+    if (max_text < 0) return KSA_ERR_INVALID;
+    if (cache->batch > 0) {
+        if (!q || !o || !workspace || !aligned16(q) || !aligned16(o) || !aligned16(workspace)) return KSA_ERR_INVALID;
+        if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return KSA_ERR_INVALID;
+    }
+    return launch_mla_decode(p, cache, kind, q, o, lse, max_text, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 int ksa_get_device_error(int32_t *dev_err, void *stream)

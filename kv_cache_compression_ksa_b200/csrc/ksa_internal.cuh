@@ -79,6 +79,13 @@ int launch_prefill_chunk(const ksa_params *p, const ksa_cache *c, const int32_t 
                          const void *qs, const void *ks, const void *vs, void *ot, void *os, float *lt, float *ls,
                          void *ws, int32_t *dev_err, cudaStream_t st);
 
+// Decode over an MLA latent cache (mla_decode.cu).
+size_t mla_decode_workspace_bytes(const ksa_mla_params *p, int batch, int64_t max_text);
+int launch_mla_append(const ksa_mla_params *p, const ksa_mla_cache *c, const int8_t *kind, const void *x,
+                      cudaStream_t st);
+int launch_mla_decode(const ksa_mla_params *p, const ksa_mla_cache *c, const int8_t *kind, const void *q, void *o,
+                      float *lse, int64_t max_text, void *ws, size_t ws_bytes, cudaStream_t st);
+
 int launch_prefill(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text,
                    int64_t aug_rows, const void *qa, const void *ka, const void *va, void *oa,
                    float *lse, const Plan &pl, int32_t *err, cudaStream_t st);
@@ -134,6 +141,25 @@ __device__ __forceinline__ void rope_rot8(uint4 &lo, uint4 &hi, const float *cs,
         a[e] = __float22bfloat162_rn(xo);
         b[e] = __float22bfloat162_rn(yo);
     }
+}
+
+// Slice of one sequence after its append: [lo, hi) in slots.  Returns false
+// (and records the error) if the state cannot hold a query of this kind.
+__device__ __forceinline__ bool decode_slice(int kind, int64_t n, int64_t m, int k, int w,
+                                             int64_t *lo, int64_t *hi)
+{
+    int64_t f = n - m * k;
+    if (kind == KSA_SUMMARY) {
+        if (m < 1 || f != 0) return false;
+        *lo = 0; *hi = k + 1;
+        return true;
+    }
+    if (f < 1 || f > k) return false;
+    int64_t ring = m < w ? m : w;
+    int64_t far = m > w ? m - w : 0;
+    *lo = k - f + 1;
+    *hi = 1 + k + ring * k + far;
+    return true;
 }
 
 }  // namespace ksa

@@ -10,7 +10,9 @@ Citations are to "Kwai Summary Attention Technical Report": the augmented
 sequence is section 2.2.1 Eq. (1); visibility is section 2.2.1 (summary rule)
 and section 2.2.2 Eqs. (2)-(3); the attention is Eq. (10); the decode cache is
 section 2.3.1 with Figure 4; a chunked prefill (ksa_prefill_chunk) is, by
-definition, a range of rows of the prefill.  The prefill backward
+definition, a range of rows of the prefill; KSA over an MLA latent cache
+(section 3.2, Eq. (6)) is absorbed MLA written as multi-query attention over
+the same slot map (mla_decode_image).  The prefill backward
 (ksa_attention_bwd) is the textbook gradient of Eq. (10) under the same mask,
 written in numpy.
 """
@@ -450,3 +452,43 @@ def ksa_prefill_chunk(n0, m0, T, k, C, qt, kt, vt, qs, ks, vs, theta, scale=None
     assert 0 <= n0 - m0 * k <= k and m0 <= m1
     return ksa_prefill([n1], k, C, qt[:n1], kt[:n1], vt[:n1], qs[:m1], ks[:m1], vs[:m1], theta, scale,
                        text_rows=[np.arange(n0, n1)], sum_rows=[np.arange(m0, m1)])[0]
+
+
+# --------------------------------------------------------------------------
+# KSA over an MLA latent cache (section 3.2, Eq. (6); MLA per section 3.1)
+# --------------------------------------------------------------------------
+def mla_kv_rows(lat, pos, theta, d_c):
+    """K and V rows of absorbed MLA written as multi-query attention: a
+    latent row [c (d_c), r (d_r)] gives K = [c, RoPE(r, pos)] and
+    V = [c, 0] (the value is the latent; the zero tail keeps one row width).
+    lat: [n, d_c + d_r] not rotated; pos: [n]."""
+    lat = _f64(lat)
+    K = lat.copy()
+    if theta and theta > 0:
+        K[:, d_c:] = rope(lat[:, None, d_c:], np.asarray(pos), theta)[:, 0]
+    V = lat.copy()
+    V[:, d_c:] = 0.0
+    return K, V
+
+
+def mla_query(q, pos, theta, d_c):
+    """[q_c, RoPE(q_r, pos)] for q [H, d_c + d_r] of one query."""
+    q = _f64(q).copy()
+    if theta and theta > 0:
+        q[:, d_c:] = rope(q[None, :, d_c:], np.asarray([pos]), theta)[0]
+    return q
+
+
+def mla_decode_image(k, C, cap, n_text, m, kind, lat_img, q, scale, theta, d_c=512):
+    """Absorbed-MLA decode of one sequence against a latent cache image
+    lat_img [S, d_c + d_r] (rope part already rotated) in the slot map:
+    scores scale (q_c . c_j + RoPE(q_r) . r_j) over the slice the map makes
+    visible, output sum_j p_j c_j.  q: [H, d_c + d_r], q_r not rotated
+    (rotated at position n_text - 1).  Returns (o [H, d_c], lse [H])."""
+    lat_img = _f64(lat_img)
+    K = lat_img[:, None, :]
+    V = lat_img.copy()
+    V[:, d_c:] = 0.0
+    qq = mla_query(q, n_text - 1, theta, d_c)
+    o, lse = decode_image(k, C, cap, n_text, m, kind, K, V[:, None, :], qq, scale)
+    return o[:, :d_c], lse

@@ -382,3 +382,61 @@ def test_table1_cache_ratios():
     assert abs(slots / n - 1 / k) < 1e-4
     h, g = 128, 8
     assert abs(slots * g / (n * h) - 0.0078125) < 1e-6
+
+
+# ---------------------------------------------------------------------------
+# KSA over an MLA latent cache (section 3.2, Eq. (6); MLA of section 3.1)
+# ---------------------------------------------------------------------------
+def test_mla_absorbed_equals_explicit_per_head_attention():
+    """The oracle's latent decode (absorbed MLA as multi-query attention over
+    [c, r] rows) equals MLA computed the explicit way: per-head keys
+    [W_UK c, r] and values W_UV c rebuilt from random up-projections, softmax
+    over the visible slots, then compared after mapping the latent output
+    through W_UV."""
+    rng = np.random.default_rng(77)
+    k, C, H, d_c, d_r, d_nope, d_v, theta = 4, 2, 3, 16, 8, 6, 5, 1e6
+    n = 6 * k + 3
+    m = n // k
+    cap = m + 1
+    lat_t = rng.standard_normal((n, d_c + d_r))
+    lat_s = rng.standard_normal((m, d_c + d_r))
+    W_uk = rng.standard_normal((H, d_nope, d_c))
+    W_uv = rng.standard_normal((H, d_v, d_c))
+    q_nope = rng.standard_normal((H, d_nope))
+    q_rope = rng.standard_normal((H, d_r))
+    scale = 1.0 / math.sqrt(d_nope + d_r)
+    cache = oracle.Cache(k, C, 1, d_c + d_r, cap)
+    Kt, Vt = oracle.mla_kv_rows(lat_t, np.arange(n), theta, d_c)
+    Ks, Vs = oracle.mla_kv_rows(lat_s, oracle.summary_positions(n, k), theta, d_c)
+    for i in range(n):
+        cache.append_text(Kt[i:i + 1], Vt[i:i + 1])
+        if (i + 1) % k == 0:
+            cache.append_summary(Ks[(i + 1) // k - 1:(i + 1) // k], Vs[(i + 1) // k - 1:(i + 1) // k])
+    # absorbed: q_c = W_UK^T q_nope
+    q_abs = np.concatenate([np.einsum("hnc,hn->hc", W_uk, q_nope), q_rope], axis=1)
+    o_lat, lse = oracle.mla_decode_image(k, C, cap, n, m, oracle.TEXT, cache.K()[:, 0], q_abs, scale, theta, d_c)
+    # explicit: visible keys of text token n-1 by the rule (Eqs. (2)-(3))
+    i = n - 1
+    c = i // k
+    txt = [j for j in range(max(0, c - C) * k, i + 1)]
+    sm = [j for j in range(max(0, c - C))]
+    rows = [Kt[j] for j in txt] + [Ks[j] for j in sm]
+    qr = oracle.rope(q_rope[None], np.array([i]), theta)[0]
+    for h in range(H):
+        keys = np.stack([np.concatenate([W_uk[h] @ r[:d_c], r[d_c:]]) for r in rows])
+        vals = np.stack([W_uv[h] @ r[:d_c] for r in rows])
+        s = scale * keys @ np.concatenate([q_nope[h], qr[h]])
+        p = np.exp(s - s.max())
+        want = (p / p.sum()) @ vals
+        np.testing.assert_allclose(W_uv[h] @ o_lat[h], want, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(lse[h], s.max() + np.log(np.exp(s - s.max()).sum()), atol=1e-12)
+
+
+def test_mla_table1_cache_ratio():
+    """Eq. (6) against Table 1's setting (h = 128, d = 128, d_c = 512,
+    d_r = 64, k = 8): KSA + MLA keeps (d_c + d_r) / k values per token, 576/8
+    = 72, i.e. 72 / (2 h d) = 0.22 % of MHA's 2 h d per token."""
+    h, d, d_c, d_r, k = 128, 128, 512, 64, 8
+    per_token = (d_c + d_r) / k
+    assert per_token == 72
+    assert round(100 * per_token / (2 * h * d), 2) == 0.22

@@ -262,7 +262,12 @@ KSA_API size_t ksa_prefill_chunk_workspace_size(const ksa_params *p, int32_t bat
  * nor its cache are written.  Inconsistent cu arrays set *dev_err (or the
  * workspace's own word when dev_err is NULL) to KSA_ERR_INVALID and nothing
  * is written.  Supported: d in {64, 128}, any G <= 8, k >= 1, w >= 0.
- * Runs on the warp-level tensor-core MMA. */
+ * The text rows run on the tcgen05 prefill kernel when its shape rules hold
+ * (1, 2, 4 or 8 q heads per kv head), reading summary keys straight from
+ * the cache in tiles of 128 slots, so every slot of cache->k / cache->v must
+ * hold finite values (zero the cache once when allocating it); the block's
+ * summaries are written to the cache before its text rows are attended.
+ * Other shapes and the summary rows use the warp-level tensor-core MMA. */
 KSA_API int ksa_prefill_chunk(const ksa_params *p, const ksa_cache *cache, const int32_t *cu_text,
                               int64_t total_text, const int32_t *cu_sum, int64_t total_sum, const void *q_text,
                               const void *k_text, const void *v_text, const void *q_sum, const void *k_sum,

@@ -72,6 +72,25 @@ int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_
 int launch_cache_build(const ksa_params *p, const ksa_cache *c, const int32_t *cu, const void *k_aug,
                        const void *v_aug, const Plan &pl, int32_t *err, cudaStream_t st);
 
+// The tensor-core prefill kernel in chunk mode: the text rows of a block of
+// new tokens against a decode cache.  The caller (prefill_chunk.cu) gathers
+// the block's rotated query rows and its window of text keys into augmented
+// buffers ([chunks, k+1, H, d]) and fills the per-sequence arrays; summary
+// key tiles are read from the cache's summary slots.
+struct ChunkTiles {
+    const int32_t *tile_off;   // [B+1] first work unit of each sequence
+    const int32_t *cbeg;       // [B] first query chunk (absolute)
+    const int32_t *ntot;       // [B] text tokens after the block
+    const int32_t *qbase;      // [B] q/o buffer chunk of absolute chunk 0
+    const int32_t *kvbase;     // [B] window buffer chunk of absolute chunk 0
+    int64_t q_chunks, kv_chunks, max_units;
+    const void *qa, *ka, *va;
+    void *oa;
+    float *lse;
+};
+int launch_prefill_cache(const ksa_params *p, const ksa_cache *c, const ChunkTiles &t, int32_t *err,
+                         cudaStream_t st);
+
 // Chunked prefill against a decode cache (prefill_chunk.cu).
 size_t prefill_chunk_workspace_bytes(const ksa_params *p, int batch, int64_t total_text, int64_t total_sum);
 int launch_prefill_chunk(const ksa_params *p, const ksa_cache *c, const int32_t *cu_t, int64_t total_t,

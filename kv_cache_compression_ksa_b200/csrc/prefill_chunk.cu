@@ -15,8 +15,19 @@
 // rotated once into the workspace).  Then the block is written into the
 // cache in the state that the token-by-token appends of Figure 4 reach.
 //
-//   chunk_plan_kernel    validate each sequence, snapshot (n0, m0), block offsets
+//   chunk_plan_kernel    validate each sequence, snapshot (n0, m0), offsets
 //   chunk_rope_kernel    rotate the block's q and k at their positions
+// text rows, tensor-core path (shapes the prefill kernel takes):
+//   chunk_sumwrite_kernel  the block's summaries into the cache's summary
+//                        slots first (append-only slots no query reads yet),
+//                        so all summary keys sit in one contiguous run
+//   chunk_gather_kernel  the block's query rows and its window of text keys
+//                        (cached ring / open-chunk tokens and new tokens)
+//                        into small augmented buffers
+//   prefill_kernel       (prefill_sm100.cu, chunk mode) summary tiles by TMA
+//                        from the cache, window tiles from the gathered rows
+//   chunk_scatter_kernel outputs of the new rows back to [T, Hq, d]
+// text rows otherwise, and the summary rows always:
 //   chunk_attn_kernel    64 query rows of one q head against their visible keys
 //                        (warp-level tensor-core MMA, online softmax)
 //   chunk_append_kernel  write the block into the cache, advance the state
@@ -47,6 +58,14 @@ struct Args {
     int64_t total_t, total_s;
     Snap *snap;                         // [B]
     int32_t *tb_off, *sb_off;           // [B+1] first text / summary query block
+    // tensor-core path (uc > 0: query chunks per prefill work unit)
+    int uc;
+    int32_t *cbeg, *kvbeg, *ntot, *qbase, *kvbase;   // [B]
+    int32_t *qoff, *kvoff, *uoff;                    // [B+1] gathered q chunks, window chunks, work units
+    int64_t q_chunks, kv_chunks;                     // buffer extents (chunks of k + 1 rows)
+    __nv_bfloat16 *qa, *ka, *va, *oa;                // gathered buffers
+    float *la;
+    int sum_only;                                    // attention kernel: summary blocks only
     int32_t *state;                     // cache state [B, 4]
     int32_t *err;
     __nv_bfloat16 *ck, *cv;             // cache [B, Hkv, S, d]
@@ -74,9 +93,35 @@ __device__ __forceinline__ int find_seq(const int32_t *off, int batch, int id)
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
 
+// State checks of sequence b for a block of T tokens and S summaries.
+__device__ __forceinline__ int chunk_state_code(const Args &a, int b, int T, int S, int32_t *n0p, int32_t *m0p)
+{
+    const int32_t *st = a.state + 4 * (int64_t)b;
+    const int32_t n0 = st[0], m0 = st[1];
+    *n0p = n0; *m0p = m0;
+    if (st[3] != 0) return st[3];
+    const int64_t f0 = (int64_t)n0 - (int64_t)m0 * a.k;
+    if (n0 < 0 || m0 < 0 || f0 < 0 || f0 > a.k || (int64_t)S != (f0 + T) / a.k) return KSA_ERR_STATE;
+    if ((int64_t)m0 + S > a.cap || (int64_t)n0 + T > (int64_t)INT32_MAX) return KSA_ERR_CAPACITY;
+    return KSA_OK;
+}
+
+// Chunks of the tensor-core path for a valid sequence: query chunks
+// [cbeg, ncb) and window chunks [kvb, ncb), kvb covering both the first
+// query chunk's window and the chunk of the first new summary.
+__device__ __forceinline__ void chunk_ranges(const Args &a, int32_t n0, int32_t m0, int T, int *cbeg, int *kvb,
+                                             int *ncb)
+{
+    const int64_t n1 = (int64_t)n0 + T;
+    *cbeg = n0 / a.k;
+    *ncb = (int)((n1 + a.k - 1) / a.k);
+    *kvb = max(0, min(*cbeg - a.w, m0));
+}
+
 __global__ void __launch_bounds__(kPlanThreads) chunk_plan_kernel(Args a, int reset_err)
 {
-    __shared__ int32_t s_tb[kPlanThreads], s_sb[kPlanThreads];
+    constexpr int NA = 5;   // text blocks, summary blocks, work units, query chunks, window chunks
+    __shared__ int32_t s_sc[NA][kPlanThreads];
     __shared__ int s_bad;
     const int t = threadIdx.x;
     if (t == 0) {
@@ -86,21 +131,30 @@ __global__ void __launch_bounds__(kPlanThreads) chunk_plan_kernel(Args a, int re
     __syncthreads();
     const int per = (a.batch + kPlanThreads - 1) / kPlanThreads;
     const int b0 = min(a.batch, t * per), b1 = min(a.batch, b0 + per);
-    int tb = 0, sb = 0, bad = 0;
+    int32_t acc[NA] = {0, 0, 0, 0, 0};
+    int bad = 0;
     for (int b = b0; b < b1; ++b) {
         const int T = a.cu_t[b + 1] - a.cu_t[b], S = a.cu_s[b + 1] - a.cu_s[b];
         if (T < 0 || S < 0) { bad = 1; continue; }
-        tb += (T + RB - 1) / RB;
-        sb += (S + RB - 1) / RB;
+        acc[0] += (T + RB - 1) / RB;
+        acc[1] += (S + RB - 1) / RB;
+        int32_t n0, m0;
+        if (a.uc > 0 && T > 0 && chunk_state_code(a, b, T, S, &n0, &m0) == KSA_OK) {
+            int cb, kb, nc;
+            chunk_ranges(a, n0, m0, T, &cb, &kb, &nc);
+            acc[2] += (nc - cb + a.uc - 1) / a.uc;
+            acc[3] += nc - cb;
+            acc[4] += nc - kb;
+        }
     }
-    s_tb[t] = tb; s_sb[t] = sb;
+    for (int i = 0; i < NA; ++i) s_sc[i][t] = acc[i];
     if (bad) s_bad = 1;
     __syncthreads();
     for (int off = 1; off < kPlanThreads; off <<= 1) {
-        int32_t x = 0, y = 0;
-        if (t >= off) { x = s_tb[t - off]; y = s_sb[t - off]; }
+        int32_t x[NA];
+        for (int i = 0; i < NA; ++i) x[i] = t >= off ? s_sc[i][t - off] : 0;
         __syncthreads();
-        s_tb[t] += x; s_sb[t] += y;
+        for (int i = 0; i < NA; ++i) s_sc[i][t] += x[i];
         __syncthreads();
     }
     const bool cu_ok = !s_bad && a.cu_t[0] == 0 && a.cu_s[0] == 0 && (int64_t)a.cu_t[a.batch] == a.total_t &&
@@ -109,28 +163,40 @@ __global__ void __launch_bounds__(kPlanThreads) chunk_plan_kernel(Args a, int re
         if (t == 0) set_error(a.err, KSA_ERR_INVALID);
         return;
     }
-    int32_t tb0 = t ? s_tb[t - 1] : 0, sb0 = t ? s_sb[t - 1] : 0;
+    int32_t o[NA];
+    for (int i = 0; i < NA; ++i) o[i] = t ? s_sc[i][t - 1] : 0;
     for (int b = b0; b < b1; ++b) {
         const int T = a.cu_t[b + 1] - a.cu_t[b], S = a.cu_s[b + 1] - a.cu_s[b];
-        int32_t *st = a.state + 4 * (int64_t)b;
-        const int32_t n0 = st[0], m0 = st[1];
-        int ok = 0;
-        if (st[3] == 0) {
-            const int64_t f0 = (int64_t)n0 - (int64_t)m0 * a.k;
-            int code = KSA_OK;
-            if (n0 < 0 || m0 < 0 || f0 < 0 || f0 > a.k || (int64_t)S != (f0 + T) / a.k) code = KSA_ERR_STATE;
-            else if ((int64_t)m0 + S > a.cap || (int64_t)n0 + T > (int64_t)INT32_MAX) code = KSA_ERR_CAPACITY;
-            if (code != KSA_OK) st[3] = code; else ok = 1;
-        }
+        int32_t n0, m0;
+        const int code = chunk_state_code(a, b, T, S, &n0, &m0);
+        if (code != KSA_OK && a.state[4 * (int64_t)b + 3] == 0) a.state[4 * (int64_t)b + 3] = code;
+        const int ok = code == KSA_OK;
         a.snap[b] = Snap{n0, m0, ok, 0};
-        a.tb_off[b] = tb0;
-        a.sb_off[b] = sb0;
-        tb0 += (T + RB - 1) / RB;
-        sb0 += (S + RB - 1) / RB;
+        a.tb_off[b] = o[0];
+        a.sb_off[b] = o[1];
+        o[0] += (T + RB - 1) / RB;
+        o[1] += (S + RB - 1) / RB;
+        if (a.uc > 0) {
+            int cb = 0, kb = 0, nc = 0;
+            if (ok && T > 0) chunk_ranges(a, n0, m0, T, &cb, &kb, &nc);
+            a.uoff[b] = o[2]; a.qoff[b] = o[3]; a.kvoff[b] = o[4];
+            a.cbeg[b] = cb; a.kvbeg[b] = kb; a.ntot[b] = n0 + T;
+            a.qbase[b] = o[3] - cb; a.kvbase[b] = o[4] - kb;
+            if (ok && T > 0) {
+                o[2] += (nc - cb + a.uc - 1) / a.uc;
+                o[3] += nc - cb;
+                o[4] += nc - kb;
+            }
+        }
     }
     if (t == kPlanThreads - 1) {
-        a.tb_off[a.batch] = s_tb[t];
-        a.sb_off[a.batch] = s_sb[t];
+        a.tb_off[a.batch] = s_sc[0][t];
+        a.sb_off[a.batch] = s_sc[1][t];
+        if (a.uc > 0) {
+            a.uoff[a.batch] = s_sc[2][t];
+            a.qoff[a.batch] = s_sc[3][t];
+            a.kvoff[a.batch] = s_sc[4][t];
+        }
     }
 }
 
@@ -242,7 +308,7 @@ __global__ void __launch_bounds__(kThreads) chunk_attn_kernel(Args a)
     extern __shared__ __align__(16) uint8_t ck_smem[];
     Row *sKV = reinterpret_cast<Row *>(ck_smem);   // two buffers of (K, V), RB rows each
     if (*a.err != 0) return;
-    const int nt = a.tb_off[a.batch], ns = a.sb_off[a.batch];
+    const int nt = a.sum_only ? 0 : a.tb_off[a.batch], ns = a.sb_off[a.batch];
     const int x = blockIdx.x;
     int kind, id;
     if (x < nt) { kind = TEXT_ROWS; id = nt - 1 - x; }   // late text blocks first
@@ -442,6 +508,127 @@ __global__ void __launch_bounds__(kThreads) chunk_attn_kernel(Args a)
 }
 
 // ---------------------------------------------------------------------------
+// Tensor-core path helpers.
+// ---------------------------------------------------------------------------
+constexpr int kCopyThreads = 256;
+
+// The block's summaries (rotated K, V) into slots 1 + k + w k + m0 + s.  No
+// query of this call reads those slots through the warp-level kernel (it
+// takes new summaries from the workspace), and no earlier state reads them.
+__global__ void __launch_bounds__(kCopyThreads) chunk_sumwrite_kernel(Args a)
+{
+    if (*a.err != 0) return;
+    const int b = blockIdx.x, g = blockIdx.y;
+    const Snap sn = a.snap[b];
+    if (!sn.ok) return;
+    const int V8 = a.d / 8;
+    const int S = a.cu_s[b + 1] - a.cu_s[b];
+    uint4 *K = reinterpret_cast<uint4 *>(a.ck) + ((int64_t)b * a.Hkv + g) * a.S * V8;
+    uint4 *V = reinterpret_cast<uint4 *>(a.cv) + ((int64_t)b * a.Hkv + g) * a.S * V8;
+    const uint4 *ks = reinterpret_cast<const uint4 *>(a.ksr), *vs = reinterpret_cast<const uint4 *>(a.vs);
+    for (int64_t e = threadIdx.x; e < (int64_t)S * V8; e += kCopyThreads) {
+        const int64_t s = e / V8, c = e % V8;
+        const int64_t slot = 1 + a.k + (int64_t)a.w * a.k + sn.m0 + s;
+        const int64_t src = ((int64_t)a.cu_s[b] + s) * a.Hkv + g;
+        K[slot * V8 + c] = ks[src * V8 + c];
+        V[slot * V8 + c] = vs[src * V8 + c];
+    }
+}
+
+// One CTA per chunk of the gathered buffers (grid = the window buffer's
+// extent, which is at least the query buffer's).  Window chunk x of sequence
+// b is absolute chunk kvbeg + (x - kvoff): text slot r holds position
+// c k + r from the cache (older than the block), the block, or zero past
+// the block; the summary slot is zero (summary keys come from the cache).
+// Query chunk x likewise: the rotated q of new positions, zero elsewhere.
+// Chunks past the last sequence are zero, so no tile ever loads stale bytes.
+__global__ void __launch_bounds__(kCopyThreads) chunk_gather_kernel(Args a)
+{
+    if (*a.err != 0) return;
+    const int x = blockIdx.x, V8 = a.d / 8;
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    // window rows (K and V)
+    {
+        const int nkv = a.kvoff[a.batch];
+        int b = -1;
+        int64_t c = 0;
+        if (x < nkv) {
+            b = find_seq(a.kvoff, a.batch, x);
+            c = (int64_t)a.kvbeg[b] + (x - a.kvoff[b]);
+        }
+        uint4 *dk = reinterpret_cast<uint4 *>(a.ka) + (int64_t)x * (a.k + 1) * a.Hkv * V8;
+        uint4 *dv = reinterpret_cast<uint4 *>(a.va) + (int64_t)x * (a.k + 1) * a.Hkv * V8;
+        const int items = (a.k + 1) * a.Hkv * V8;
+        for (int e = threadIdx.x; e < items; e += kCopyThreads) {
+            const int r = e / (a.Hkv * V8), rem = e % (a.Hkv * V8), g = rem / V8, cc = rem % V8;
+            uint4 kv = zero, vv = zero;
+            if (b >= 0 && r < a.k) {
+                const Snap sn = a.snap[b];
+                const int64_t p = c * a.k + r;
+                if (p < sn.n0) {
+                    const int64_t cp = p / a.k, rr = p - cp * a.k;
+                    int64_t slot;
+                    if (cp >= sn.m0) slot = a.k - rr;
+                    else slot = a.w > 0 ? a.k + 1 + (cp % a.w) * a.k + (a.k - 1 - rr) : 0;
+                    const int64_t row = ((int64_t)b * a.Hkv + g) * a.S + slot;
+                    kv = reinterpret_cast<const uint4 *>(a.ck)[row * V8 + cc];
+                    vv = reinterpret_cast<const uint4 *>(a.cv)[row * V8 + cc];
+                } else if (p < a.ntot[b]) {
+                    const int64_t row = ((int64_t)a.cu_t[b] + p - sn.n0) * a.Hkv + g;
+                    kv = reinterpret_cast<const uint4 *>(a.ktr)[row * V8 + cc];
+                    vv = reinterpret_cast<const uint4 *>(a.vt)[row * V8 + cc];
+                }
+            }
+            dk[e] = kv;
+            dv[e] = vv;
+        }
+    }
+    // query rows
+    if (x < a.q_chunks) {
+        const int nq = a.qoff[a.batch];
+        int b = -1;
+        int64_t c = 0;
+        if (x < nq) {
+            b = find_seq(a.qoff, a.batch, x);
+            c = (int64_t)a.cbeg[b] + (x - a.qoff[b]);
+        }
+        uint4 *dq = reinterpret_cast<uint4 *>(a.qa) + (int64_t)x * (a.k + 1) * a.Hq * V8;
+        const int items = (a.k + 1) * a.Hq * V8;
+        for (int e = threadIdx.x; e < items; e += kCopyThreads) {
+            const int r = e / (a.Hq * V8), rem = e % (a.Hq * V8), h = rem / V8, cc = rem % V8;
+            uint4 qv = zero;
+            if (b >= 0 && r < a.k) {
+                const int64_t p = c * a.k + r, n0 = a.snap[b].n0;
+                if (p >= n0 && p < a.ntot[b]) {
+                    const int64_t row = ((int64_t)a.cu_t[b] + p - n0) * a.Hq + h;
+                    qv = reinterpret_cast<const uint4 *>(a.qtr)[row * V8 + cc];
+                }
+            }
+            dq[e] = qv;
+        }
+    }
+}
+
+// The new text rows' outputs (and LSE) from the gathered layout to
+// [total_text, Hq, d]: one CTA per row.
+__global__ void __launch_bounds__(kCopyThreads) chunk_scatter_kernel(Args a)
+{
+    if (*a.err != 0) return;
+    const int64_t i = blockIdx.x;
+    const int b = find_seq(a.cu_t, a.batch, (int)i);
+    const Snap sn = a.snap[b];
+    if (!sn.ok) return;
+    const int64_t p = sn.n0 + (i - a.cu_t[b]);
+    const int64_t row = ((int64_t)a.qbase[b] + p / a.k) * (a.k + 1) + p % a.k;
+    const int V8 = a.d / 8;
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.oa) + row * a.Hq * V8;
+    uint4 *dst = reinterpret_cast<uint4 *>(a.ot) + i * a.Hq * V8;
+    for (int e = threadIdx.x; e < a.Hq * V8; e += kCopyThreads) dst[e] = src[e];
+    if (a.lt)
+        for (int h = threadIdx.x; h < a.Hq; h += kCopyThreads) a.lt[i * a.Hq + h] = a.la[row * a.Hq + h];
+}
+
+// ---------------------------------------------------------------------------
 // Extend the cache of (sequence, kv head) by the block (Figure 4):
 //  (4d) when the block completes the open chunk m0, that chunk's f0 cached
 //       tokens move from slots k - r to its ring block (if it is among the
@@ -504,8 +691,20 @@ __global__ void __launch_bounds__(kAppendThreads) chunk_append_kernel(Args a)
 }
 
 // ---------------------------------------------------------------------------
+// Query chunks of the tensor-core path (0 when the shape is not one the
+// prefill kernel takes).
+static int tc_unit_chunks(const ksa_params *p)
+{
+    const int G = p->num_q_heads / p->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
+    if (p->head_dim != 64 && p->head_dim != 128) return 0;
+    return prefill_unit_chunks(p);
+}
+
 struct Layout {
-    size_t err, snap, tb, sb, qtr, ktr, qsr, ksr, total;
+    size_t err, snap, tb, sb, qtr, ktr, qsr, ksr;
+    size_t arr[8], qa, ka, va, oa, la, total;
+    int64_t q_chunks, kv_chunks, max_units;
 };
 
 static Layout layout(const ksa_params *p, int batch, int64_t total_t, int64_t total_s)
@@ -521,6 +720,22 @@ static Layout layout(const ksa_params *p, int batch, int64_t total_t, int64_t to
     L.ktr = o; o += align_up((size_t)total_t * Hkv * d * 2);
     L.qsr = o; o += align_up((size_t)total_s * Hq * d * 2);
     L.ksr = o; o += align_up((size_t)total_s * Hkv * d * 2);
+    const int uc = tc_unit_chunks(p);
+    L.q_chunks = L.kv_chunks = L.max_units = 0;
+    if (uc > 0 && total_t > 0) {
+        // a sequence's query chunks number at most T/k + 2 and its window
+        // chunks at most w + 1 more
+        L.q_chunks = total_t / p->k + 2LL * batch;
+        L.kv_chunks = L.q_chunks + (int64_t)batch * (p->w + 1);
+        L.max_units = L.q_chunks / uc + batch;
+        for (int i = 0; i < 8; ++i) { L.arr[i] = o; o += align_up(sizeof(int32_t) * (size_t)(batch + 1)); }
+        const size_t rows_q = (size_t)L.q_chunks * (p->k + 1), rows_kv = (size_t)L.kv_chunks * (p->k + 1);
+        L.qa = o; o += align_up(rows_q * Hq * d * 2);
+        L.oa = o; o += align_up(rows_q * Hq * d * 2);
+        L.la = o; o += align_up(rows_q * Hq * 4);
+        L.ka = o; o += align_up(rows_kv * Hkv * d * 2);
+        L.va = o; o += align_up(rows_kv * Hkv * d * 2);
+    }
     L.total = o;
     return L;
 }
@@ -574,6 +789,25 @@ int launch_prefill_chunk(const ksa_params *p, const ksa_cache *c, const int32_t 
     a.qtr = reinterpret_cast<__nv_bfloat16 *>(w + L.qtr); a.ktr = reinterpret_cast<__nv_bfloat16 *>(w + L.ktr);
     a.qsr = reinterpret_cast<__nv_bfloat16 *>(w + L.qsr); a.ksr = reinterpret_cast<__nv_bfloat16 *>(w + L.ksr);
     a.ot = (__nv_bfloat16 *)ot; a.os = (__nv_bfloat16 *)os; a.lt = lt; a.ls = ls;
+    // tensor-core path for the text rows when the shape allows and the cache
+    // coordinates fit the tensor maps
+    const bool tc = L.q_chunks > 0 && a.S <= INT32_MAX && L.kv_chunks * (p->k + 1) <= INT32_MAX;
+    a.uc = tc ? tc_unit_chunks(p) : 0;
+    a.sum_only = 0;
+    a.q_chunks = L.q_chunks; a.kv_chunks = L.kv_chunks;
+    if (tc) {
+        int32_t *arr[8];
+        for (int i = 0; i < 8; ++i) arr[i] = reinterpret_cast<int32_t *>(w + L.arr[i]);
+        a.cbeg = arr[0]; a.kvbeg = arr[1]; a.ntot = arr[2]; a.qbase = arr[3]; a.kvbase = arr[4];
+        a.qoff = arr[5]; a.kvoff = arr[6]; a.uoff = arr[7];
+        a.qa = reinterpret_cast<__nv_bfloat16 *>(w + L.qa); a.oa = reinterpret_cast<__nv_bfloat16 *>(w + L.oa);
+        a.ka = reinterpret_cast<__nv_bfloat16 *>(w + L.ka); a.va = reinterpret_cast<__nv_bfloat16 *>(w + L.va);
+        a.la = reinterpret_cast<float *>(w + L.la);
+    } else {
+        a.cbeg = a.kvbeg = a.ntot = a.qbase = a.kvbase = a.qoff = a.kvoff = a.uoff = nullptr;
+        a.qa = a.oa = a.ka = a.va = nullptr;
+        a.la = nullptr;
+    }
 
     chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(a, a.err == own_err);
     if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
@@ -583,7 +817,24 @@ int launch_prefill_chunk(const ksa_params *p, const ksa_cache *c, const int32_t 
         if (rb > INT32_MAX) return KSA_ERR_UNSUPPORTED;
         chunk_rope_kernel<<<(unsigned)rb, kRopeThreads, 0, st>>>(a);
         if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
-        const int64_t blocks = (total_t / RB + B) + (total_s / RB + B);
+        if (tc) {
+            dim3 sg((unsigned)B, (unsigned)a.Hkv);
+            chunk_sumwrite_kernel<<<sg, kCopyThreads, 0, st>>>(a);
+            if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
+            if (L.kv_chunks > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+            chunk_gather_kernel<<<(unsigned)L.kv_chunks, kCopyThreads, 0, st>>>(a);
+            if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
+            ChunkTiles t;
+            t.tile_off = a.uoff; t.cbeg = a.cbeg; t.ntot = a.ntot; t.qbase = a.qbase; t.kvbase = a.kvbase;
+            t.q_chunks = L.q_chunks; t.kv_chunks = L.kv_chunks; t.max_units = L.max_units;
+            t.qa = a.qa; t.ka = a.ka; t.va = a.va; t.oa = a.oa; t.lse = a.la;
+            int rc = launch_prefill_cache(p, c, t, a.err, st);
+            if (rc != KSA_OK) return rc;
+            chunk_scatter_kernel<<<(unsigned)total_t, kCopyThreads, 0, st>>>(a);
+            if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
+            a.sum_only = 1;
+        }
+        const int64_t blocks = (a.sum_only ? 0 : total_t / RB + B) + (total_s / RB + B);
         if (blocks > INT32_MAX) return KSA_ERR_UNSUPPORTED;
         const int rc = p->head_dim == 128 ? launch_attn<128>(a, blocks, st) : launch_attn<64>(a, blocks, st);
         if (rc != KSA_OK) return rc;

@@ -96,6 +96,19 @@ struct Params {
     const __nv_bfloat16 *q;   // augmented query tensor (read row by row into TMEM)
     __nv_bfloat16 *o;
     float *lse;
+    // Chunk mode (a block of new tokens against a decode cache): per-sequence
+    // arrays of the chunk plan, all null in the plain prefill.  Chunks and
+    // summaries are then numbered from the sequence's start (absolute), and
+    // each map has its own origin: q/o map chunk = qbase + c, window map
+    // chunk = kvbase + c.  The summary maps then cover the cache itself,
+    // dims (d, slot, kv head, sequence), summary j at slot sum_slot0 + j
+    // (the plain prefill: all origins are the sequence's first chunk and
+    // summary j is slot k of chunk j).
+    const int32_t *ck_tile_off;   // [B+1] first work unit of each sequence
+    const int32_t *ck_cbeg;       // [B] first query chunk
+    const int32_t *ck_ntot;       // [B] text tokens after the block
+    const int32_t *ck_qbase, *ck_kvbase;
+    int sum_slot0;
 };
 
 // ---------------------------------------------------------------------------
@@ -306,7 +319,7 @@ __device__ __forceinline__ void pair_sync(int quarter)
 // c0-w .. cend-1, then the summary tiles.  When G k > 128 the G heads are
 // split over G / Gp items, each loading the same K/V tiles.
 struct Unit {
-    int hkv, h0, nb, mb, ncb, goff, c0, cend, cw_lo, n_win, T;
+    int hkv, h0, b, nb, mb, ncb, qbase, kvbase, sbase, c0, cend, cw_lo, n_win, T;
 };
 
 __device__ __forceinline__ Unit unit_of(const Params &P, int item, int n_units)
@@ -317,17 +330,27 @@ __device__ __forceinline__ Unit unit_of(const Params &P, int item, int n_units)
     U.hkv = (item % per) / P.HP;
     U.h0 = U.hkv * P.G + ((item % per) % P.HP) * P.Gp;
     const int u = n_units - 1 - rank;  // heaviest (latest) units first
+    const int32_t *toff = P.ck_tile_off ? P.ck_tile_off : P.pl.tile_off;
     int lo = 0, hi = P.batch - 1;
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
-        if (P.pl.tile_off[mid] <= u) lo = mid; else hi = mid - 1;
+        if (toff[mid] <= u) lo = mid; else hi = mid - 1;
     }
     const int b = lo;
-    U.nb = P.cu[b + 1] - P.cu[b];
+    U.b = b;
+    if (P.ck_tile_off) {
+        U.nb = P.ck_ntot[b];
+        U.qbase = P.ck_qbase[b];
+        U.kvbase = P.ck_kvbase[b];
+        U.sbase = P.sum_slot0;
+        U.c0 = P.ck_cbeg[b] + (u - toff[b]) * P.unit_chunks;
+    } else {
+        U.nb = P.cu[b + 1] - P.cu[b];
+        U.qbase = U.kvbase = U.sbase = P.pl.chunk_off[b];
+        U.c0 = (u - toff[b]) * P.unit_chunks;
+    }
     U.mb = U.nb / P.k;
     U.ncb = (U.nb + P.k - 1) / P.k;
-    U.goff = P.pl.chunk_off[b];
-    U.c0 = (u - P.pl.tile_off[b]) * P.unit_chunks;
     U.cend = min(U.ncb, U.c0 + P.unit_chunks);
     const int ns = max(min(U.mb, U.cend - 1 - P.w), 0);   // summaries any row may see
     U.cw_lo = max(0, U.c0 - P.w);
@@ -364,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         if (threadIdx.x == 0) set_error(P.err, KSA_ERR_UNSUPPORTED);
         return;
     }
-    const int n_units = P.pl.tile_off[P.batch];
+    const int n_units = P.ck_tile_off ? P.ck_tile_off[P.batch] : P.pl.tile_off[P.batch];
     const int W = n_units * P.Hkv * P.HP;   // work items
     if ((int)blockIdx.x >= W) return;
 
@@ -455,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     mbar_expect_tx(bar(B_QF(qb)), q_bytes);
                     for (int hf = 0; hf < D / 64; ++hf)
                         tma_load_4d(sbase + L::kQ + qb * L::kQTile + hf * kQHalf, &P.tm_q, bar(B_QF(qb)), hf * 64,
-                                    U.h0, 0, U.goff + U.c0);
+                                    U.h0, 0, U.qbase + U.c0);
                     q_issued[qb]++;
                 }
                 for (int j = 0; j < U.T && ok; ++j, ++gt) {
@@ -463,8 +486,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     const bool win = j < U.n_win;
                     const uint32_t bytes = win ? win_bytes : sum_bytes;
                     const CUtensorMap *mp = isk ? (win ? &P.tm_kwin : &P.tm_ksum) : (win ? &P.tm_vwin : &P.tm_vsum);
-                    const int slot = win ? 0 : P.k;
-                    const int chunk = U.goff + (win ? U.cw_lo + j * P.Tk : (j - U.n_win) * BN);
+                    // window: (d, head, slot 0, chunk); summaries: (d, head, slot k,
+                    // chunk) over the augmented rows, or (d, slot, head, sequence)
+                    // over the cache in chunk mode
+                    int c1 = U.hkv, c2 = win ? 0 : P.k;
+                    int c3 = win ? U.kvbase + U.cw_lo + j * P.Tk : U.sbase + (j - U.n_win) * BN;
+                    if (!win && P.ck_tile_off) { c1 = c3; c2 = U.hkv; c3 = U.b; }
                     const int bempty = isk ? B_KE(st) : B_VE(st), bfull = isk ? B_KF(st) : B_VF(st);
                     const uint32_t dst = sbase + (isk ? L::kK : L::kV) + st * L::kKVTile;
                     if (gt >= nst &&
@@ -472,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                         break;
                     mbar_expect_tx(bar(bfull), bytes);
                     for (int hf = 0; hf < D / 64; ++hf)
-                        tma_load_4d(dst + hf * kKVHalf, mp, bar(bfull), hf * 64, U.hkv, slot, chunk);
+                        tma_load_4d(dst + hf * kKVHalf, mp, bar(bfull), hf * 64, c1, c2, c3);
                     issued[st]++;
                 }
             }
@@ -712,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             }
             const float inv = Lr > 0.f ? 1.f / Lr : 0.f;
             const float g0 = f0 * inv, g1 = f1 * inv;
-            const int64_t row = (int64_t)(U.goff + c) * (P.k + 1) + r_slot;
+            const int64_t row = (int64_t)(U.qbase + c) * (P.k + 1) + r_slot;
             const int head = U.h0 + g;
             // this thread holds output columns [D/2 half, D/2 half + D/2) of its row
             uint4 *dst = reinterpret_cast<uint4 *>(P.o + (row * P.Hq + head) * D + half * (D / 2));
@@ -755,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 if (warp == 0 && lane == 0 && ok) {
 #pragma unroll
                     for (int hf = 0; hf < D / 64; ++hf)
-                        tma_store_4d(&P.tm_o, sbase + L::kO + hf * kQHalf, hf * 64, U.h0, 0, U.goff + U.c0);
+                        tma_store_4d(&P.tm_o, sbase + L::kO + hf * kQHalf, hf * 64, U.h0, 0, U.qbase + U.c0);
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 }
             }
@@ -1014,6 +1041,8 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
     P.q = (const __nv_bfloat16 *)qa;
     P.o = (__nv_bfloat16 *)oa;
     P.lse = lse;
+    P.ck_tile_off = P.ck_cbeg = P.ck_ntot = P.ck_qbase = P.ck_kvbase = nullptr;
+    P.sum_slot0 = 0;
     bool ok = make_map(&P.tm_q, qa, D, Hq, k, chunks, P.Gp, k, P.Tc) &&
               make_map(&P.tm_ksum, ka, D, Hkv, k, chunks, 1, 1, pf::BN) &&
               make_map(&P.tm_kwin, ka, D, Hkv, k, chunks, 1, k, P.Tk) &&
@@ -1056,6 +1085,81 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
         if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
     }
     return KSA_OK;
+}
+
+// Summary tiles straight from a decode cache [B, Hkv, S, d]: dims (d, slot,
+// kv head, sequence), boxes of 128 slots of one (sequence, kv head).  Slots
+// past S are outside the map and load as zeros.
+static bool make_cache_map(CUtensorMap *m, const void *base, int d, int Hkv, int64_t S, int B)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)S, (cuuint64_t)Hkv, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)S * d * 2, (cuuint64_t)Hkv * S * d * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)pf::BN, 1, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D>
+static int launch_prefill_cache_t(const ksa_params *p, const ksa_cache *c, const ChunkTiles &t, int32_t *err,
+                                  cudaStream_t st)
+{
+    using L = pf::SmemLayout<D>;
+    pf::Params P;
+    const int k = p->k, Hq = p->num_q_heads, Hkv = p->num_kv_heads, G = Hq / Hkv;
+    P.k = k; P.w = p->w; P.G = G; P.Hq = Hq; P.Hkv = Hkv;
+    P.Gp = prefill_heads_per_tile(p);
+    if (P.Gp < 1) return KSA_ERR_UNSUPPORTED;
+    P.HP = G / P.Gp;
+    P.Tc = pf::BM / (P.Gp * k);
+    P.Tk = pf::BN / k;
+    if (P.Tc < 1 || P.Tk < 1) return KSA_ERR_UNSUPPORTED;
+    P.batch = c->batch;
+    P.unit_chunks = P.Tc;
+    P.aug_rows = t.q_chunks * (k + 1);
+    const float scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)D);
+    P.scale = scale;
+    P.scale_log2 = scale * 1.4426950408889634f;
+    P.cu = nullptr;
+    P.pl = Plan{nullptr, nullptr, nullptr, nullptr};
+    P.err = err;
+    P.q = (const __nv_bfloat16 *)t.qa;
+    P.o = (__nv_bfloat16 *)t.oa;
+    P.lse = t.lse;
+    P.ck_tile_off = t.tile_off; P.ck_cbeg = t.cbeg; P.ck_ntot = t.ntot;
+    P.ck_qbase = t.qbase; P.ck_kvbase = t.kvbase;
+    P.sum_slot0 = 1 + k + p->w * k;
+    const int64_t S = 1 + (int64_t)k + (int64_t)p->w * k + c->cap_summaries;
+    bool ok = make_map(&P.tm_q, t.qa, D, Hq, k, t.q_chunks, P.Gp, k, P.Tc) &&
+              make_map(&P.tm_o, t.oa, D, Hq, k, t.q_chunks, P.Gp, k, P.Tc) &&
+              make_map(&P.tm_kwin, t.ka, D, Hkv, k, t.kv_chunks, 1, k, P.Tk) &&
+              make_map(&P.tm_vwin, t.va, D, Hkv, k, t.kv_chunks, 1, k, P.Tk) &&
+              make_cache_map(&P.tm_ksum, c->k, D, Hkv, S, c->batch) &&
+              make_cache_map(&P.tm_vsum, c->v, D, Hkv, S, c->batch);
+    if (!ok) return KSA_ERR_CUDA;
+    int64_t grid = t.max_units * Hkv * P.HP;
+    if (grid > sm_count()) grid = sm_count();
+    if (grid < 1) return KSA_OK;
+    static bool attr_set[2] = {false, false};
+    if (!attr_set[D == 128]) {
+        if (cudaFuncSetAttribute(pf::prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
+            cudaSuccess)
+            return KSA_ERR_CUDA;
+        attr_set[D == 128] = true;
+    }
+    pf::prefill_kernel<D><<<(unsigned)grid, pf::kThreads, L::kAlloc, st>>>(P);
+    return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
+}
+
+int launch_prefill_cache(const ksa_params *p, const ksa_cache *c, const ChunkTiles &t, int32_t *err, cudaStream_t st)
+{
+    if (p->head_dim == 128) return launch_prefill_cache_t<128>(p, c, t, err, st);
+    if (p->head_dim == 64) return launch_prefill_cache_t<64>(p, c, t, err, st);
+    return KSA_ERR_UNSUPPORTED;
 }
 
 int launch_prefill(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,

@@ -5,7 +5,10 @@ A block of new tokens per sequence is attended against a cache that holds
 the sequence's first n0 tokens; its rows must equal the oracle's prefill
 rows n0 .. n0+T-1 (and the summaries of the chunks the block completes),
 and afterwards the cache must hold, in every slot a decode reads, what the
-oracle's cache model holds after appending the same tokens one by one."""
+oracle's cache model holds after appending the same tokens one by one.
+Shapes the tensor-core prefill kernel takes run its text rows there (summary
+tiles straight from the cache); the 3-heads-per-kv-head case runs them on
+the warp-level kernel."""
 import numpy as np
 import pytest
 import torch
@@ -83,6 +86,11 @@ CASES = {
     "k16_w3_gqa4": (16, 3, 8, 2, 128, [(130, False, 200), (45, False, 3), (160, True, 40)]),
     "k1_gqa4": (1, 2, 4, 1, 64, [(10, False, 10), (0, False, 7)]),
     "gqa8": (8, 4, 16, 2, 128, [(300, False, 257), (64, True, 64)]),
+    # 3 q heads per kv head: not a tensor-core prefill shape, the text rows
+    # take the warp-level kernel
+    "gqa3_warp_path": (4, 2, 6, 2, 64, [(37, False, 50), (16, True, 5), (0, False, 9)]),
+    # k 32 with 8 q heads per kv head: each kv head's heads split over 2 tiles
+    "k32_gqa8_head_split": (32, 2, 16, 2, 128, [(100, False, 300), (64, True, 70)]),
 }
 
 

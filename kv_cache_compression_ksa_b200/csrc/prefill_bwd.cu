@@ -98,18 +98,6 @@ __device__ __forceinline__ bool block_of(const Args &a, int id, Blk &B)
     return B.cnt > 0;
 }
 
-// KSA visibility of key (kk_kind, ki) to query (qk, qi) of one sequence
-__device__ __forceinline__ bool visible(const Args &a, int m, int qk, int qi, int kk_kind, int ki)
-{
-    if (qk == TEXT_ROWS) {
-        const int c = qi / a.k;
-        if (kk_kind == TEXT_ROWS) return ki <= qi && ki >= max(0, c - a.w) * a.k;
-        return ki < min(c - a.w, m);
-    }
-    if (kk_kind == TEXT_ROWS) return ki / a.k == qi;
-    return ki == qi;
-}
-
 // 64 rows x D bf16 of one head into shared memory, rows padded by 16 bytes
 // (row pitch D + 8 elements keeps ldmatrix's 8-row reads conflict-free);
 // rows at or beyond cnt are zero.
@@ -216,6 +204,21 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(Args a)
     float acc[NT][4];
 #pragma unroll
     for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    // per row, the keys it sees: text [lt_lo, lt_hi], summaries [ls_lo, ls_hi)
+    int lt_lo[2], lt_hi[2], ls_lo[2], ls_hi[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        if (!live[x]) {
+            lt_lo[x] = 1; lt_hi[x] = 0; ls_lo[x] = ls_hi[x] = 0;
+        } else if (Q.kind == TEXT_ROWS) {
+            const int c = qi[x] / a.k;
+            lt_lo[x] = max(0, c - a.w) * a.k; lt_hi[x] = qi[x];
+            ls_lo[x] = 0; ls_hi[x] = max(0, min(c - a.w, Q.m));
+        } else {
+            lt_lo[x] = qi[x] * a.k; lt_hi[x] = qi[x] * a.k + a.k - 1;
+            ls_lo[x] = qi[x]; ls_hi[x] = qi[x] + 1;
+        }
+    }
 
     // the key blocks these rows can see
     int nsb = 0, t_lo = 0, t_hi = 0, s_lo = 0;
@@ -261,6 +264,13 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(Args a)
         }
         __syncthreads();   // key block kb has landed for every thread
         Row *sK = sKV + (kb & 1) * 2 * RB, *sV = sK + RB;
+        // a whole key block inside every text row's range needs no mask
+        bool full = K.cnt == RB && Q.kind == TEXT_ROWS;
+        if (full) {
+            const int ia = Q.idx0, ib = Q.idx0 + Q.cnt - 1, ca = ia / a.k, cb = ib / a.k;
+            full = K.kind == SUM_ROWS ? K.idx0 + K.cnt - 1 < min(ca - a.w, Q.m)
+                                      : (K.idx0 + K.cnt - 1 <= ia && K.idx0 >= max(0, cb - a.w) * a.k);
+        }
         // S = Q K^T and dP = dO V^T: 16 rows x 64 keys
         float s[8][4], dp[8][4];
 #pragma unroll
@@ -284,8 +294,9 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(Args a)
             float e[4];
 #pragma unroll
             for (int z = 0; z < 4; ++z) {
-                const int x = z >> 1, col = 8 * nt + 2 * tt + (z & 1);
-                const bool vis = live[x] && col < K.cnt && visible(a, Q.m, Q.kind, qi[x], K.kind, K.idx0 + col);
+                const int x = z >> 1, col = 8 * nt + 2 * tt + (z & 1), key = K.idx0 + col;
+                const bool vis = full || (col < K.cnt && (K.kind == TEXT_ROWS ? key >= lt_lo[x] && key <= lt_hi[x]
+                                                                                : key >= ls_lo[x] && key < ls_hi[x]));
                 const float p = vis ? wm::ex2(s[nt][z] * a.scale_log2 - lse2[x]) : 0.f;
                 e[z] = p * (dp[nt][z] - dd[x]);
             }
@@ -335,11 +346,27 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tt = lane & 3;
     int ki[2];
     bool live[2];
+    // per key row, the queries that see it (the rule inverted): text
+    // queries [qt_lo, qt_hi], summary queries [qs_lo, qs_hi).  Text key p of
+    // chunk c_p: text queries p .. (c_p + w + 1) k - 1 and summary c_p (if
+    // that chunk is complete); summary key j: text queries from
+    // (j + w + 1) k on and summary j.
+    int qt_lo[2], qt_hi[2], qs_lo[2], qs_hi[2];
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
         const int r = 16 * warp + gr + 8 * x;
         live[x] = r < K.cnt;
         ki[x] = K.idx0 + r;
+        if (!live[x]) {
+            qt_lo[x] = 1; qt_hi[x] = 0; qs_lo[x] = qs_hi[x] = 0;
+        } else if (K.kind == TEXT_ROWS) {
+            const int cp = ki[x] / a.k;
+            qt_lo[x] = ki[x]; qt_hi[x] = (cp + a.w + 1) * a.k - 1;
+            qs_lo[x] = cp; qs_hi[x] = cp < K.m ? cp + 1 : cp;
+        } else {
+            qt_lo[x] = (ki[x] + a.w + 1) * a.k; qt_hi[x] = INT32_MAX;
+            qs_lo[x] = ki[x]; qs_hi[x] = ki[x] + 1;
+        }
     }
     float dk[NT][4], dv[NT][4];
 #pragma unroll
@@ -405,6 +432,13 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
             __syncthreads();   // step it has landed for every thread
             Row *sQ = sQO + (it & 1) * 2 * RB, *sO = sQ + RB;
             const float *sL = sLD + (it & 1) * 2 * RB, *sD = sL + RB;
+            // a whole text query block that sees every live key of the block
+            bool full = Q.cnt == RB && Q.kind == TEXT_ROWS;
+            if (full) {
+                const int k_last = K.idx0 + K.cnt - 1;
+                full = K.kind == SUM_ROWS ? Q.idx0 >= (k_last + a.w + 1) * a.k
+                                          : (Q.idx0 >= k_last && Q.idx0 + RB - 1 <= (K.idx0 / a.k + a.w + 1) * a.k - 1);
+            }
             // two halves of 32 queries: S^T = K Q^T, dP^T = V dO^T (16 keys x 32 queries)
 #pragma unroll 1
             for (int hq = 0; hq < 2; ++hq) {
@@ -436,8 +470,9 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
                     float pe[4], de[4];
 #pragma unroll
                     for (int z = 0; z < 4; ++z) {
-                        const int x = z >> 1, col = q0 + 8 * nt + 2 * tt + (z & 1);
-                        const bool vis = live[x] && col < Q.cnt && visible(a, K.m, Q.kind, Q.idx0 + col, K.kind, ki[x]);
+                        const int x = z >> 1, col = q0 + 8 * nt + 2 * tt + (z & 1), qi = Q.idx0 + col;
+                        const bool vis = full || (col < Q.cnt && (Q.kind == TEXT_ROWS ? qi >= qt_lo[x] && qi <= qt_hi[x]
+                                                                                      : qi >= qs_lo[x] && qi < qs_hi[x]));
                         const float p = vis ? wm::ex2(s[nt][z] * a.scale_log2 - sL[col]) : 0.f;
                         pe[z] = p;
                         de[z] = p * (dp[nt][z] - sD[col]);

@@ -27,7 +27,9 @@
 //   prefill_kernel       (prefill_sm100.cu, chunk mode) summary tiles by TMA
 //                        from the cache, window tiles from the gathered rows
 //   chunk_scatter_kernel outputs of the new rows back to [T, Hq, d]
-// text rows otherwise, and the summary rows always:
+//   chunk_sum_kernel     the block's summary rows: k + 1 keys each, one warp
+//                        per (summary, kv head)
+// text and summary rows otherwise (q heads per kv head not 1, 2, 4 or 8):
 //   chunk_attn_kernel    64 query rows of one q head against their visible keys
 //                        (warp-level tensor-core MMA, online softmax)
 //   chunk_append_kernel  write the block into the cache, advance the state
@@ -65,7 +67,6 @@ struct Args {
     int64_t q_chunks, kv_chunks;                     // buffer extents (chunks of k + 1 rows)
     __nv_bfloat16 *qa, *ka, *va, *oa;                // gathered buffers
     float *la;
-    int sum_only;                                    // attention kernel: summary blocks only
     int32_t *state;                     // cache state [B, 4]
     int32_t *err;
     __nv_bfloat16 *ck, *cv;             // cache [B, Hkv, S, d]
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(kThreads) chunk_attn_kernel(Args a)
     extern __shared__ __align__(16) uint8_t ck_smem[];
     Row *sKV = reinterpret_cast<Row *>(ck_smem);   // two buffers of (K, V), RB rows each
     if (*a.err != 0) return;
-    const int nt = a.sum_only ? 0 : a.tb_off[a.batch], ns = a.sb_off[a.batch];
+    const int nt = a.tb_off[a.batch], ns = a.sb_off[a.batch];
     const int x = blockIdx.x;
     int kind, id;
     if (x < nt) { kind = TEXT_ROWS; id = nt - 1 - x; }   // late text blocks first
@@ -508,6 +509,166 @@ __global__ void __launch_bounds__(kThreads) chunk_attn_kernel(Args a)
 }
 
 // ---------------------------------------------------------------------------
+// Summary rows of the block: summary s_j sees the k text tokens of chunk j
+// and itself (section 2.2.1), k + 1 keys.  One warp per (new summary, kv
+// head): the keys are the rows of a 16-row MMA tile (S^T = K Q^T with the G
+// query heads of the kv head as MMA columns, O^T = V^T P^T), 16 keys per
+// step with an online softmax across steps.  Lane (g, t) loads dims
+// [32v + 8t, +8) of key rows g and g + 8 with 16-byte loads and hands the
+// words to the MMA unchanged; q is loaded in the same permuted order, so the
+// dot products are unchanged.  A key row is read where it lives: a token of
+// the open chunk from its cache slot, a new token from the block, the
+// summary from the block.
+// ---------------------------------------------------------------------------
+constexpr int kSumWarps = 4;
+
+template <int D, int G>
+__global__ void __launch_bounds__(kSumWarps * 32) chunk_sum_kernel(Args a)
+{
+    static_assert(G <= 8, "query heads per kv head must fit the 8 MMA columns");
+    constexpr int NV = D / 32, NC = D / 16, NM = D / 16;
+    __shared__ float s_o[kSumWarps][G][D];
+    __shared__ float s_ml[kSumWarps][2][G];
+    if (*a.err != 0) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t task = (int64_t)blockIdx.x * kSumWarps + warp;
+    if (task >= a.total_s * a.Hkv) return;   // warp-uniform; only warp-level syncs below
+    const int64_t row = task / a.Hkv;         // the summary's input row
+    const int h = (int)(task % a.Hkv);
+    const int b = find_seq(a.cu_s, a.batch, (int)row);
+    const Snap sn = a.snap[b];
+    if (!sn.ok) return;
+    const int64_t j = sn.m0 + (row - a.cu_s[b]);   // its chunk
+    const int g = lane >> 2, tt = lane & 3;
+    uint32_t qb[NC][2];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const int d0 = 32 * (c / 2) + 8 * tt + 4 * (c % 2);
+        if (g < G) {
+            const uint32_t *qp = reinterpret_cast<const uint32_t *>(a.qsr + (row * a.Hq + (int64_t)h * G + g) * D + d0);
+            qb[c][0] = qp[0];
+            qb[c][1] = qp[1];
+        } else {
+            qb[c][0] = qb[c][1] = 0u;
+        }
+    }
+    // uint4 base of key row r (r < k: text position j k + r; r = k: the summary)
+    auto key_row = [&](int r, const uint4 *&kp, const uint4 *&vp) {
+        int64_t off;
+        if (r == a.k) {
+            off = (row * a.Hkv + h) * (D / 8);
+            kp = reinterpret_cast<const uint4 *>(a.ksr) + off;
+            vp = reinterpret_cast<const uint4 *>(a.vs) + off;
+            return;
+        }
+        const int64_t p = j * a.k + r;
+        if (p < sn.n0) {   // a token of the open chunk m0, cached at slot k - r
+            off = (((int64_t)b * a.Hkv + h) * a.S + (a.k - (p - (int64_t)sn.m0 * a.k))) * (D / 8);
+            kp = reinterpret_cast<const uint4 *>(a.ck) + off;
+            vp = reinterpret_cast<const uint4 *>(a.cv) + off;
+        } else {
+            off = (((int64_t)a.cu_t[b] + p - sn.n0) * a.Hkv + h) * (D / 8);
+            kp = reinterpret_cast<const uint4 *>(a.ktr) + off;
+            vp = reinterpret_cast<const uint4 *>(a.vt) + off;
+        }
+    };
+    float o[NM][4];
+#pragma unroll
+    for (int i = 0; i < NM; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};   // heads 2tt, 2tt + 1 (log2 units)
+    for (int kb = 0; kb <= a.k; kb += 16) {
+        const int r0 = kb + g, r1 = kb + g + 8;
+        const bool in0 = r0 <= a.k, in1 = r1 <= a.k;
+        const uint4 *k0p = nullptr, *v0p = nullptr, *k1p = nullptr, *v1p = nullptr;
+        if (in0) key_row(r0, k0p, v0p);
+        if (in1) key_row(r1, k1p, v1p);
+        uint4 kA[NV], kB[NV], vA[NV], vB[NV];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            kA[v] = in0 ? k0p[4 * v + tt] : z;
+            kB[v] = in1 ? k1p[4 * v + tt] : z;
+            vA[v] = in0 ? v0p[4 * v + tt] : z;
+            vB[v] = in1 ? v1p[4 * v + tt] : z;
+        }
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const int v = c / 2, hh = c % 2;
+            wm::mma16816(sc, wm::word(kA[v], 2 * hh), wm::word(kB[v], 2 * hh), wm::word(kA[v], 2 * hh + 1),
+                         wm::word(kB[v], 2 * hh + 1), qb[c][0], qb[c][1]);
+        }
+        float x[4];
+        x[0] = in0 ? sc[0] * a.scale_log2 : -INFINITY;
+        x[1] = in0 ? sc[1] * a.scale_log2 : -INFINITY;
+        x[2] = in1 ? sc[2] * a.scale_log2 : -INFINITY;
+        x[3] = in1 ? sc[3] * a.scale_log2 : -INFINITY;
+        float corr[2], pv[4];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float mx = fmaxf(x[e], x[e + 2]);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float m_new = fmaxf(m_run[e], mx);   // finite: key 0 is always present
+            corr[e] = wm::ex2(m_run[e] - m_new);
+            pv[e] = wm::ex2(x[e] - m_new);
+            pv[e + 2] = wm::ex2(x[e + 2] - m_new);
+            l_run[e] = l_run[e] * corr[e] + pv[e] + pv[e + 2];
+            m_run[e] = m_new;
+        }
+#pragma unroll
+        for (int i = 0; i < NM; ++i) {
+            o[i][0] *= corr[0]; o[i][1] *= corr[1];
+            o[i][2] *= corr[0]; o[i][3] *= corr[1];
+        }
+        const uint32_t pb0 = wm::movtrans(wm::pack2(pv[0], pv[1]));
+        const uint32_t pb1 = wm::movtrans(wm::pack2(pv[2], pv[3]));
+#pragma unroll
+        for (int i = 0; i < NM; ++i) {
+            const int v = i / 2, pp = i % 2;
+            wm::mma16816(o[i], wm::movtrans(wm::word(vA[v], 2 * pp)), wm::movtrans(wm::word(vA[v], 2 * pp + 1)),
+                         wm::movtrans(wm::word(vB[v], 2 * pp)), wm::movtrans(wm::word(vB[v], 2 * pp + 1)), pb0, pb1);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) l_run[e] += __shfl_xor_sync(0xffffffffu, l_run[e], off);
+    // O^T rows: m-tile i = (v, pp), row g -> dim 32v + 8(g/2) + 4pp + (g%2), row g+8 -> that + 2
+#pragma unroll
+    for (int i = 0; i < NM; ++i) {
+        const int v = i / 2, pp = i % 2;
+        const int dA = 32 * v + 8 * (g / 2) + 4 * pp + (g % 2);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int head = 2 * tt + e;
+            if (head < G) {
+                s_o[warp][head][dA] = o[i][e];
+                s_o[warp][head][dA + 2] = o[i][2 + e];
+            }
+        }
+    }
+    if (g == 0) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+            if (2 * tt + e < G) {
+                s_ml[warp][0][2 * tt + e] = m_run[e];
+                s_ml[warp][1][2 * tt + e] = l_run[e];
+            }
+    }
+    __syncwarp();
+    for (int idx = lane; idx < G * (D / 2); idx += 32) {
+        const int gg = idx / (D / 2), w2 = idx % (D / 2);
+        const float inv = 1.f / s_ml[warp][1][gg];
+        const uint32_t pr = wm::pack2(s_o[warp][gg][2 * w2] * inv, s_o[warp][gg][2 * w2 + 1] * inv);
+        reinterpret_cast<uint32_t *>(a.os + (row * a.Hq + (int64_t)h * G + gg) * D)[w2] = pr;
+    }
+    if (a.ls && lane < G)
+        a.ls[row * a.Hq + (int64_t)h * G + lane] =
+            (s_ml[warp][0][lane] + log2f(s_ml[warp][1][lane])) * 0.69314718055994530942f;
+}
+
+// ---------------------------------------------------------------------------
 // Tensor-core path helpers.
 // ---------------------------------------------------------------------------
 constexpr int kCopyThreads = 256;
@@ -518,20 +679,20 @@ constexpr int kCopyThreads = 256;
 __global__ void __launch_bounds__(kCopyThreads) chunk_sumwrite_kernel(Args a)
 {
     if (*a.err != 0) return;
-    const int b = blockIdx.x, g = blockIdx.y;
-    const Snap sn = a.snap[b];
-    if (!sn.ok) return;
     const int V8 = a.d / 8;
-    const int S = a.cu_s[b + 1] - a.cu_s[b];
-    uint4 *K = reinterpret_cast<uint4 *>(a.ck) + ((int64_t)b * a.Hkv + g) * a.S * V8;
-    uint4 *V = reinterpret_cast<uint4 *>(a.cv) + ((int64_t)b * a.Hkv + g) * a.S * V8;
+    const int64_t items = a.total_s * a.Hkv * V8;
     const uint4 *ks = reinterpret_cast<const uint4 *>(a.ksr), *vs = reinterpret_cast<const uint4 *>(a.vs);
-    for (int64_t e = threadIdx.x; e < (int64_t)S * V8; e += kCopyThreads) {
-        const int64_t s = e / V8, c = e % V8;
-        const int64_t slot = 1 + a.k + (int64_t)a.w * a.k + sn.m0 + s;
-        const int64_t src = ((int64_t)a.cu_s[b] + s) * a.Hkv + g;
-        K[slot * V8 + c] = ks[src * V8 + c];
-        V[slot * V8 + c] = vs[src * V8 + c];
+    for (int64_t e = (int64_t)blockIdx.x * kCopyThreads + threadIdx.x; e < items;
+         e += (int64_t)gridDim.x * kCopyThreads) {
+        const int64_t row = e / ((int64_t)a.Hkv * V8), rem = e % ((int64_t)a.Hkv * V8);
+        const int g = (int)(rem / V8), c = (int)(rem % V8);
+        const int b = find_seq(a.cu_s, a.batch, (int)row);
+        const Snap sn = a.snap[b];
+        if (!sn.ok) continue;
+        const int64_t slot = 1 + a.k + (int64_t)a.w * a.k + sn.m0 + (row - a.cu_s[b]);
+        const int64_t dst = (((int64_t)b * a.Hkv + g) * a.S + slot) * V8 + c;
+        reinterpret_cast<uint4 *>(a.ck)[dst] = ks[e];
+        reinterpret_cast<uint4 *>(a.cv)[dst] = vs[e];
     }
 }
 
@@ -664,7 +825,10 @@ __global__ void __launch_bounds__(kAppendThreads) chunk_append_kernel(Args a)
     }
     __syncthreads();   // the open chunk's slots are read before new tokens overwrite them
     const uint4 *kt = reinterpret_cast<const uint4 *>(a.ktr), *vt = reinterpret_cast<const uint4 *>(a.vt);
-    for (int64_t e = t; e < (int64_t)T * V8; e += kAppendThreads) {
+    // only the open chunk and the last w complete chunks are kept: start at
+    // the first kept position
+    const int64_t keep = max(n0, (w > 0 ? max((int64_t)0, m1 - w) : m1) * k);
+    for (int64_t e = (keep - n0) * V8 + t; e < (int64_t)T * V8; e += kAppendThreads) {
         const int64_t tq = e / V8, c = e % V8;
         const int64_t p = n0 + tq, cp = p / k, r = p - cp * k;
         int64_t slot;
@@ -676,7 +840,8 @@ __global__ void __launch_bounds__(kAppendThreads) chunk_append_kernel(Args a)
         V[slot * V8 + c] = vt[src * V8 + c];
     }
     const uint4 *ks = reinterpret_cast<const uint4 *>(a.ksr), *vs = reinterpret_cast<const uint4 *>(a.vs);
-    for (int64_t e = t; e < (int64_t)S * V8; e += kAppendThreads) {
+    // (the tensor-core path wrote the summaries before its attention)
+    for (int64_t e = t; e < (a.uc > 0 ? 0 : (int64_t)S * V8); e += kAppendThreads) {
         const int64_t s = e / V8, c = e % V8;
         const int64_t slot = 1 + k + (int64_t)w * k + m0 + s;
         const int64_t src = ((int64_t)a.cu_s[b] + s) * a.Hkv + g;
@@ -751,6 +916,24 @@ static int launch_attn(const Args &a, int64_t blocks, cudaStream_t st)
     return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
 }
 
+template <int D>
+static int launch_sum_d(int G, const Args &a, unsigned blocks, cudaStream_t st)
+{
+    switch (G) {
+    case 1: chunk_sum_kernel<D, 1><<<blocks, kSumWarps * 32, 0, st>>>(a); break;
+    case 2: chunk_sum_kernel<D, 2><<<blocks, kSumWarps * 32, 0, st>>>(a); break;
+    case 4: chunk_sum_kernel<D, 4><<<blocks, kSumWarps * 32, 0, st>>>(a); break;
+    case 8: chunk_sum_kernel<D, 8><<<blocks, kSumWarps * 32, 0, st>>>(a); break;
+    default: return KSA_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
+}
+
+static int launch_sum(int d, int G, const Args &a, unsigned blocks, cudaStream_t st)
+{
+    return d == 128 ? launch_sum_d<128>(G, a, blocks, st) : launch_sum_d<64>(G, a, blocks, st);
+}
+
 }  // namespace ck
 
 size_t prefill_chunk_workspace_bytes(const ksa_params *p, int batch, int64_t total_text, int64_t total_sum)
@@ -793,7 +976,6 @@ int launch_prefill_chunk(const ksa_params *p, const ksa_cache *c, const int32_t 
     // coordinates fit the tensor maps
     const bool tc = L.q_chunks > 0 && a.S <= INT32_MAX && L.kv_chunks * (p->k + 1) <= INT32_MAX;
     a.uc = tc ? tc_unit_chunks(p) : 0;
-    a.sum_only = 0;
     a.q_chunks = L.q_chunks; a.kv_chunks = L.kv_chunks;
     if (tc) {
         int32_t *arr[8];
@@ -818,8 +1000,9 @@ int launch_prefill_chunk(const ksa_params *p, const ksa_cache *c, const int32_t 
         chunk_rope_kernel<<<(unsigned)rb, kRopeThreads, 0, st>>>(a);
         if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
         if (tc) {
-            dim3 sg((unsigned)B, (unsigned)a.Hkv);
-            chunk_sumwrite_kernel<<<sg, kCopyThreads, 0, st>>>(a);
+            const int64_t sitems = total_s * a.Hkv * (p->head_dim / 8);
+            const int64_t sblocks = sitems > 0 ? min((int64_t)4 * sm_count(), (sitems + kCopyThreads - 1) / kCopyThreads) : 0;
+            if (sblocks > 0) chunk_sumwrite_kernel<<<(unsigned)sblocks, kCopyThreads, 0, st>>>(a);
             if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
             if (L.kv_chunks > INT32_MAX) return KSA_ERR_UNSUPPORTED;
             chunk_gather_kernel<<<(unsigned)L.kv_chunks, kCopyThreads, 0, st>>>(a);
@@ -832,12 +1015,22 @@ int launch_prefill_chunk(const ksa_params *p, const ksa_cache *c, const int32_t 
             if (rc != KSA_OK) return rc;
             chunk_scatter_kernel<<<(unsigned)total_t, kCopyThreads, 0, st>>>(a);
             if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
-            a.sum_only = 1;
         }
-        const int64_t blocks = (a.sum_only ? 0 : total_t / RB + B) + (total_s / RB + B);
-        if (blocks > INT32_MAX) return KSA_ERR_UNSUPPORTED;
-        const int rc = p->head_dim == 128 ? launch_attn<128>(a, blocks, st) : launch_attn<64>(a, blocks, st);
-        if (rc != KSA_OK) return rc;
+        if (tc) {
+            // summary rows: one warp per (summary, kv head)
+            const int64_t tasks = total_s * a.Hkv;
+            if (tasks > 0) {
+                const int64_t sb = (tasks + kSumWarps - 1) / kSumWarps;
+                if (sb > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+                const int rc = launch_sum(p->head_dim, a.G, a, (unsigned)sb, st);
+                if (rc != KSA_OK) return rc;
+            }
+        } else {
+            const int64_t blocks = (total_t / RB + B) + (total_s / RB + B);
+            if (blocks > INT32_MAX) return KSA_ERR_UNSUPPORTED;
+            const int rc = p->head_dim == 128 ? launch_attn<128>(a, blocks, st) : launch_attn<64>(a, blocks, st);
+            if (rc != KSA_OK) return rc;
+        }
     }
     dim3 grid((unsigned)B, (unsigned)a.Hkv);
     chunk_append_kernel<<<grid, kAppendThreads, 0, st>>>(a);

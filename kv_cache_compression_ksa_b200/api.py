@@ -2,7 +2,11 @@
 workspaces with torch; every computation runs in libksa.so).
 
 prefill(...)      RoPE + interleave + KSA prefill attention for a packed batch
-DecodeCache       the contiguous decode cache plus append / decode steps
+KSAAttention      the same as a torch.autograd.Function (backward through
+                  ksa_prefill_bwd and ksa_interleave_rope_bwd)
+DecodeCache       the contiguous decode cache plus append / decode / chunked
+                  prefill steps
+MlaCache          the latent (MLA) cache plus append / decode steps
 """
 from __future__ import annotations
 
@@ -48,6 +52,46 @@ def prefill(p: L.ksa_params, seqlens, cu_seqlens, q_text, k_text, v_text, q_sum,
                           q_sum, k_sum, v_sum, q_aug, k_aug, v_aug, ws, stream=stream)
     L.ksa_prefill_fwd(p, cu_seqlens, total_text, rows, q_aug, k_aug, v_aug, o_aug, lse, ws, stream=stream)
     return PrefillOut(o_aug, lse, q_aug, k_aug, v_aug)
+
+
+class KSAAttention(torch.autograd.Function):
+    """KSA prefill attention with autograd, for training.
+
+    forward(p, seqlens, cu_seqlens, q_text, k_text, v_text, q_sum, k_sum,
+    v_sum) -> o_aug [aug_rows, Hq, d] bf16 in the augmented layout
+    (include/ksa.h): ksa_interleave_rope + ksa_prefill_fwd, keeping the
+    rotated q/k/v, O and LSE for the backward.  backward: ksa_prefill_bwd
+    then ksa_interleave_rope_bwd give the gradients of the six projections.
+    Padding rows of o_aug are unspecified and their incoming gradient is
+    ignored.  Use: o = KSAAttention.apply(p, seqlens, cu, qt, kt, vt, qs, ks, vs).
+    """
+
+    @staticmethod
+    def forward(ctx, p, seqlens, cu_seqlens, q_text, k_text, v_text, q_sum, k_sum, v_sum):
+        out = prefill(p, seqlens, cu_seqlens, q_text, k_text, v_text, q_sum, k_sum, v_sum, want_lse=True)
+        ctx.p = p
+        ctx.seqlens = [int(n) for n in seqlens]
+        ctx.save_for_backward(cu_seqlens, out.q_aug, out.k_aug, out.v_aug, out.o_aug, out.lse)
+        ctx.in_shapes = [tuple(t.shape) for t in (q_text, k_text, v_text, q_sum, k_sum, v_sum)]
+        return out.o_aug
+
+    @staticmethod
+    def backward(ctx, do_aug):
+        cu, qa, ka, va, oa, lse = ctx.saved_tensors
+        p, seqlens = ctx.p, ctx.seqlens
+        dev = qa.device
+        B = len(seqlens)
+        total_text = sum(seqlens)
+        total_sum = sum(n // p.k for n in seqlens)
+        rows = qa.shape[0]
+        do = do_aug.to(torch.bfloat16).contiguous()
+        dqa, dka, dva = torch.empty_like(qa), torch.empty_like(ka), torch.empty_like(va)
+        wsb = torch.empty(L.ksa_prefill_bwd_workspace_size(p, B, rows), dtype=torch.uint8, device=dev)
+        L.ksa_prefill_bwd(p, cu, total_text, rows, qa, ka, va, oa, lse, do, dqa, dka, dva, wsb)
+        grads = [torch.empty(sh, dtype=torch.bfloat16, device=dev) for sh in ctx.in_shapes]
+        ws = torch.empty(L.ksa_prefill_workspace_size(p, B, total_text), dtype=torch.uint8, device=dev)
+        L.ksa_interleave_rope_bwd(p, cu, total_text, total_sum, rows, dqa, dka, dva, *grads, ws)
+        return (None, None, None, *grads)
 
 
 class DecodeCache:

@@ -174,3 +174,40 @@ def test_training_chain_gradients_of_the_projections(seqlens, k, w, Hq, Hkv, d):
         allrows = np.ones(wt.shape[0], bool)
         if wt.shape[0]:
             _check(nm, f64(got), wt, allrows)
+
+
+def test_autograd_function_matches_the_library_chain():
+    """KSAAttention (torch.autograd over the library) gives, bit for bit, the
+    gradients of the explicit chain interleave -> prefill -> prefill_bwd ->
+    interleave_bwd that test_training_chain_gradients_of_the_projections
+    checks against the oracle; padding rows' incoming gradient is ignored."""
+    from kv_cache_compression_ksa_b200.api import KSAAttention
+    seqlens, k, w, Hq, Hkv, d = [37, 64, 5], 4, 2, 4, 2, 64
+    dev = torch.device("cuda")
+    x = prefill_inputs(seqlens, k, Hq, Hkv, d, seed=31, device=dev)
+    p = L.make_params(k, w, Hq, Hkv, d, 0.0, THETA)
+    ins = [t.clone().requires_grad_(True) for t in (x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum, x.v_sum)]
+    o = KSAAttention.apply(p, seqlens, x.cu_seqlens, *ins)
+    gen = torch.Generator(device=dev).manual_seed(32)
+    G = torch.randn(o.shape, generator=gen, device=dev).to(torch.bfloat16)
+    grads = torch.autograd.grad((o.float() * G.float()).sum(), ins)
+    # the same chain through the C ABI
+    nt, ns = sum(seqlens), sum(n // k for n in seqlens)
+    rows = L.ksa_aug_rows(p, seqlens)
+    qa = torch.empty(rows, Hq, d, dtype=torch.bfloat16, device=dev)
+    ka = torch.empty(rows, Hkv, d, dtype=torch.bfloat16, device=dev)
+    va, oa = torch.empty_like(ka), torch.empty_like(qa)
+    lse = torch.empty(rows, Hq, dtype=torch.float32, device=dev)
+    ws = torch.empty(L.ksa_prefill_workspace_size(p, len(seqlens), nt), dtype=torch.uint8, device=dev)
+    L.ksa_interleave_rope(p, x.cu_seqlens, nt, ns, rows, x.q_text, x.k_text, x.v_text, x.q_sum, x.k_sum, x.v_sum,
+                          qa, ka, va, ws)
+    L.ksa_prefill_fwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, ws)
+    dqa, dka, dva = torch.empty_like(qa), torch.empty_like(ka), torch.empty_like(va)
+    wsb = torch.empty(L.ksa_prefill_bwd_workspace_size(p, len(seqlens), rows), dtype=torch.uint8, device=dev)
+    L.ksa_prefill_bwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, G, dqa, dka, dva, wsb)
+    want = [torch.empty_like(t) for t in ins]
+    L.ksa_interleave_rope_bwd(p, x.cu_seqlens, nt, ns, rows, dqa, dka, dva, *want, ws)
+    torch.cuda.synchronize()
+    for g_, w_ in zip(grads, want):
+        assert g_.dtype == torch.bfloat16 and g_.shape == w_.shape
+        assert torch.equal(g_, w_)

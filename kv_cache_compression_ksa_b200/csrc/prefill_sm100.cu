@@ -645,23 +645,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                         for (int e = 0; e < HC; ++e) s[e] = (e >= clo && e < chi) ? s[e] : -INFINITY;
                     }
                 };
-                // Pass 1: the row max and, speculatively, P against the current
-                // reference (independent, so ALU and MUFU work interleave).
                 load_s();
-                const float mb_old = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-                float pm[8], ps[8];
+                // the row max of this half's 64 keys
+                float pm[8];
 #pragma unroll
-                for (int a = 0; a < 8; ++a) { pm[a] = -INFINITY; ps[a] = 0.f; }
+                for (int a = 0; a < 8; ++a) pm[a] = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < HC; ++e) {
-                    pm[e & 7] = fmaxf(pm[e & 7], s[e]);
-                    const float pe = ex2(fmaf(s[e], sl2, -mb_old));
-                    ps[e & 7] += pe;
-                    s[e] = pe;
-                }
+                for (int e = 0; e < HC; ++e) pm[e & 7] = fmaxf(pm[e & 7], s[e]);
                 const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                                        fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-                float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 // lazy rescale: keep the reference unless the max exceeds it by
                 // more than 8 in log2 units (P stays <= 256; exact either way)
                 const float m_new = fmaxf(m_run, mx);
@@ -687,25 +679,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     }
                     l_run *= corr;
                     m_run = m_new;
-                    // recompute P against the new reference (S is still intact)
-                    load_s();
-                    const float mb2 = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-#pragma unroll
-                    for (int a = 0; a < 8; ++a) ps[a] = 0.f;
-#pragma unroll
-                    for (int e = 0; e < HC; ++e) {
-                        const float pe = ex2(fmaf(s[e], sl2, -mb2));
-                        ps[e & 7] += pe;
-                        s[e] = pe;
-                    }
-                    sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 }
-                l_run += sum;
-                uint32_t pk[HC / 2];
+                // P in two groups of 32 keys; each group's bf16 pairs go to TMEM
+                // as soon as they are packed, so the first store overlaps the
+                // second group's exponentials
+                const float mb = (m_run == -INFINITY) ? 0.f : m_run * sl2;
+                float ps[8];
 #pragma unroll
-                for (int e = 0; e < HC / 2; ++e) pk[e] = pack_bf16(s[2 * e], s[2 * e + 1]);
-                // P of this half -> S columns [64 half, 64 half + 32) (its own S region)
-                tmem_st32(S_COL(bf) + lane_off + half * HC, pk);
+                for (int a = 0; a < 8; ++a) ps[a] = 0.f;
+#pragma unroll
+                for (int grp = 0; grp < 2; ++grp) {
+                    uint32_t pk[HC / 4];
+#pragma unroll
+                    for (int e2 = 0; e2 < HC / 4; ++e2) {
+                        const int e = grp * (HC / 2) + 2 * e2;
+                        const float p0 = ex2(fmaf(s[e], sl2, -mb)), p1 = ex2(fmaf(s[e + 1], sl2, -mb));
+                        ps[e & 7] += p0;
+                        ps[(e + 1) & 7] += p1;
+                        pk[e2] = pack_bf16(p0, p1);
+                    }
+                    // P of this half -> S columns [64 half + 16 grp, +16) (its own S region)
+                    tmem_st16(S_COL(bf) + lane_off + half * HC + grp * (HC / 4), pk);
+                }
+                l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(B_P(half, bf)));

@@ -83,34 +83,49 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """nvidia-smi clock / throttle sampling during the timed region.
+
+    The sampler starts before the warm-up (so the process is running when
+    the timed region begins) and the summary keeps only the samples whose
+    timestamps fall inside the window given to mark()."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
+        import tempfile
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.window = None
+        self.path = os.path.join(tempfile.gettempdir(), f"ksa_bench_clocks_{os.getpid()}_{index}.csv")
 
-    def __enter__(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    def start(self):
         try:
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return self
+        for _ in range(150):   # up to ~3 s for the first line
+            if os.path.getsize(self.path) > 0 or self.proc.poll() is not None:
+                break
+            time.sleep(0.02)
         return self
 
-    def __exit__(self, *a):
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
+
+    def stop(self):
         if self.proc:
             self.proc.terminate()
             self.proc.wait()
             self.f.close()
 
     def summary(self):
+        from datetime import datetime
         if not self.proc:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         sm, mx, reasons = [], None, set()
@@ -118,16 +133,24 @@ class ClockSampler:
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    mx = float(parts[2])
+                    ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    clk, cmax = float(parts[2]), float(parts[3])
                 except ValueError:
                     continue
-                for nm, v in zip(names, parts[5:9]):
+                if self.window and not (self.window[0] - 0.03 <= ts <= self.window[1] + 0.03):
+                    continue
+                sm.append(clk)
+                mx = cmax
+                for nm, v in zip(names, parts[6:10]):
                     if v.lower() == "active":
                         reasons.add(nm)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
 
@@ -304,20 +327,23 @@ def run_ksa(args, rank, world, local):
             torch.cuda.synchronize()
             times.append([ev[i].elapsed_time(ev[i + 1]) for i in range(4)])
 
+    clk = ClockSampler(local).start()
     for _ in range(args.warmup):
         step(None)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     times = []
-    with ClockSampler(local) as clk:
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(st)
-        for _ in range(args.steps):
-            step(times)
-        t_end.record(st)
-        torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    t_start.record(st)
+    for _ in range(args.steps):
+        step(times)
+    t_end.record(st)
+    torch.cuda.synchronize()
+    clk.mark(w0, time.time())
+    clk.stop()
     barrier(world)
     total_ms = t_start.elapsed_time(t_end)
     tarr = np.asarray(times)  # [steps, 4] ms: rope, prefill, append, decode

@@ -350,6 +350,255 @@ __global__ void __launch_bounds__(64 * MT) mla_decode_kernel(Args a)
         }
 }
 
+// ---------------------------------------------------------------------------
+// Warp-specialised form for 64-head CTAs.  Warps 0-3 (one warpgroup) each
+// take 16 heads: they keep those heads' q fragments in registers for the
+// whole slice, compute S = Q K^T of a 32-slot block and its softmax (a row
+// never leaves its warp), and publish P and the rescale factors.  Warps 4-11
+// each own 64 latent dims of O for all 64 heads and load the latent blocks.
+// Blocks and P are double-buffered; named barriers hand them over:
+//   1 + b  block in buffer b landed        (PV warps arrive, QK warps sync)
+//   3 + b  P and factors of buffer b ready (QK warps arrive, PV warps sync)
+//   5 + b  P buffer b read                 (PV warps arrive, QK warps sync)
+// Each barrier alternates strictly between the two groups, and both groups
+// walk the same blocks, so every phase gets its 384 threads.  Registers move
+// from the PV warps (168 -> 160) to the QK warps (168 -> 184, room for their
+// 144 q-fragment registers): 4 x 32 x 184 + 8 x 32 x 160 = 384 x 168, exactly
+// the launch allocation, so the increase always finds its registers.
+// ---------------------------------------------------------------------------
+constexpr int WS_THREADS = 384;
+
+struct WsSmem {
+    static constexpr int HEADS = 64;
+    static constexpr size_t q = 0;
+    static constexpr size_t kv = q + (size_t)HEADS * PITCH * 2;
+    static constexpr size_t p = kv + 2ull * KB * PITCH * 2;            // two P buffers
+    static constexpr size_t alpha = p + 2ull * HEADS * PPITCH * 2;     // two factor buffers
+    static constexpr size_t bytes = alpha + 2ull * HEADS * 4;
+};
+
+__device__ __forceinline__ void nb_sync(int id) { asm volatile("bar.sync %0, 384;" ::"r"(id) : "memory"); }
+__device__ __forceinline__ void nb_arrive(int id) { asm volatile("bar.arrive %0, 384;" ::"r"(id) : "memory"); }
+
+__global__ void __launch_bounds__(WS_THREADS, 1) mla_decode_ws_kernel(Args a)
+{
+    constexpr int HEADS = 64, NC = DL / 16;
+    using L = WsSmem;
+    using Row = __nv_bfloat16[PITCH];
+    using PRow = __nv_bfloat16[PPITCH];
+    extern __shared__ __align__(16) uint8_t mla_smem[];
+    Row *sQ = reinterpret_cast<Row *>(mla_smem + L::q);
+    Row *sK = reinterpret_cast<Row *>(mla_smem + L::kv);
+    PRow *sP = reinterpret_cast<PRow *>(mla_smem + L::p);
+    float *sA = reinterpret_cast<float *>(mla_smem + L::alpha);
+    __shared__ float s_cos[DR / 2], s_sin[DR / 2];
+
+    const int split = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tt = lane & 3;
+    const int h0 = hg * HEADS;
+    const int64_t pidx = ((int64_t)split * a.batch + b) * a.H + h0;
+    const int kind = a.kind[b];
+    const int64_t n = a.state[4 * (int64_t)b], m = a.state[4 * (int64_t)b + 1];
+    int64_t lo = 0, hi = 0;
+    if (kind == KSA_SKIP || a.state[4 * (int64_t)b + 3] != 0) return;
+    if (!decode_slice(kind, n, m, a.k, a.w, &lo, &hi) || hi > a.S) {
+        if (split == 0 && hg == 0 && threadIdx.x == 0) a.state[4 * (int64_t)b + 3] = KSA_ERR_STATE;
+        return;
+    }
+    const int64_t s0 = lo + (int64_t)split * a.per, s1 = min(hi, s0 + a.per);
+    const int nblk = s1 > s0 ? (int)((s1 - s0 + KB - 1) / KB) : 0;
+
+    // q of this CTA's heads in shared memory, the d_r part rotated at n - 1
+    const int64_t pos = n - 1;
+    for (int r = threadIdx.x; r < DR / 2; r += WS_THREADS) {
+        float c = 1.f, s = 0.f;
+        if (a.rotate) rope_cos_sin((double)pos, r, DR, a.log2_theta, &c, &s);
+        s_cos[r] = c; s_sin[r] = s;
+    }
+    __syncthreads();
+    {
+        constexpr int V8 = DL / 8;
+        const uint4 *qg = reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * a.H + h0) * DL);
+        for (int e = threadIdx.x; e < HEADS * (DC / 8); e += WS_THREADS) {
+            const int h = e / (DC / 8), c = e % (DC / 8);
+            *reinterpret_cast<uint4 *>(&sQ[h][8 * c]) = h0 + h < a.H ? qg[(int64_t)h * V8 + c] : make_uint4(0, 0, 0, 0);
+        }
+        for (int e = threadIdx.x; e < HEADS * (DR / 16); e += WS_THREADS) {
+            const int h = e / (DR / 16), c = e % (DR / 16);
+            uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = lo4;
+            if (h0 + h < a.H) {
+                lo4 = qg[(int64_t)h * V8 + DC / 8 + c];
+                hi4 = qg[(int64_t)h * V8 + DC / 8 + c + DR / 16];
+                rope_rot8(lo4, hi4, s_cos + 8 * c, s_sin + 8 * c);
+            }
+            *reinterpret_cast<uint4 *>(&sQ[h][DC + 8 * c]) = lo4;
+            *reinterpret_cast<uint4 *>(&sQ[h][DC + DR / 2 + 8 * c]) = hi4;
+        }
+    }
+    __syncthreads();
+
+    if (warp < 4) {
+        // ================= QK and softmax: heads 16 warp .. 16 warp + 15 =================
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 184;" ::: "memory");
+        uint32_t qf[NC][4];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) wm::frag_a<PITCH - 8>(qf[c], sQ, 16 * warp, 16 * c);
+        const int rA = 16 * warp + gr, rB = rA + 8;
+        float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+        for (int kb = 0; kb < nblk; ++kb) {
+            const int bb = kb & 1;
+            const int cnt = (int)min((int64_t)KB, s1 - (s0 + (int64_t)kb * KB));
+            nb_sync(1 + bb);   // block kb landed
+            const Row *K = sK + bb * KB;
+            float sc[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                uint32_t k0[4], k1[4];
+                wm::frag_b_nk<PITCH - 8>(k0, K, 0, 16 * c);
+                wm::frag_b_nk<PITCH - 8>(k1, K, 16, 16 * c);
+                wm::mma16816(sc[0], qf[c][0], qf[c][1], qf[c][2], qf[c][3], k0[0], k0[1]);
+                wm::mma16816(sc[1], qf[c][0], qf[c][1], qf[c][2], qf[c][3], k0[2], k0[3]);
+                wm::mma16816(sc[2], qf[c][0], qf[c][1], qf[c][2], qf[c][3], k1[0], k1[1]);
+                wm::mma16816(sc[3], qf[c][0], qf[c][1], qf[c][2], qf[c][3], k1[2], k1[3]);
+            }
+            // scale, mask the tail, softmax over the block's 32 slots
+            float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int z = 0; z < 4; ++z) {
+                    const int col = 8 * nt + 2 * tt + (z & 1);
+                    const float v = col < cnt ? sc[nt][z] * a.scale_log2 : -INFINITY;
+                    sc[nt][z] = v;
+                    mx[z >> 1] = fmaxf(mx[z >> 1], v);
+                }
+            float base[2], alpha[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                mx[x] = fmaxf(mx[x], __shfl_xor_sync(0xffffffffu, mx[x], 1));
+                mx[x] = fmaxf(mx[x], __shfl_xor_sync(0xffffffffu, mx[x], 2));
+                const float mn = fmaxf(mrow[x], mx[x]);
+                base[x] = mn == -INFINITY ? 0.f : mn;
+                alpha[x] = wm::ex2(mrow[x] - base[x]);
+                mrow[x] = mn;
+                lrow[x] *= alpha[x];
+            }
+            uint32_t pw[4][2];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                float e[4];
+#pragma unroll
+                for (int z = 0; z < 4; ++z) {
+                    e[z] = wm::ex2(sc[nt][z] - base[z >> 1]);
+                    lrow[z >> 1] += e[z];
+                }
+                pw[nt][0] = wm::pack2(e[0], e[1]);
+                pw[nt][1] = wm::pack2(e[2], e[3]);
+            }
+            if (kb >= 2) nb_sync(5 + bb);   // the PV warps have read P buffer bb (block kb - 2)
+            PRow *Pb = sP + bb * HEADS;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                *reinterpret_cast<uint32_t *>(&Pb[rA][8 * nt + 2 * tt]) = pw[nt][0];
+                *reinterpret_cast<uint32_t *>(&Pb[rB][8 * nt + 2 * tt]) = pw[nt][1];
+            }
+            if (tt == 0) { sA[bb * HEADS + rA] = alpha[0]; sA[bb * HEADS + rB] = alpha[1]; }
+            nb_arrive(3 + bb);   // P and factors of block kb ready
+        }
+        // share statistics: max (log2 units) and sum of this share
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            float l = lrow[x];
+            l += __shfl_xor_sync(0xffffffffu, l, 1);
+            l += __shfl_xor_sync(0xffffffffu, l, 2);
+            const int h = x ? rB : rA;
+            if (tt == 0 && h0 + h < a.H) {
+                a.part_ml[(pidx + h) * 2] = mrow[x];
+                a.part_ml[(pidx + h) * 2 + 1] = l;
+            }
+        }
+    } else {
+        // ================= PV: latent dims 64 pw .. 64 pw + 63 of all 64 heads =================
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 160;" ::: "memory");
+        constexpr int NTW = 8, NPT = 256;   // n-tiles of this warp's dims; threads of the group
+        const int pw = warp - 4, tid = threadIdx.x - 128;
+        const __nv_bfloat16 *rows = a.lat + (int64_t)b * a.S * DL;
+        auto issue = [&](int kb) {   // block kb -> buffer kb % 2 (one commit group)
+            Row *dst = sK + (kb & 1) * KB;
+            const int64_t r0 = s0 + (int64_t)kb * KB;
+            const int cnt = (int)min((int64_t)KB, s1 - r0);
+            for (int e = tid; e < KB * (DL / 8); e += NPT) {
+                const int r = e / (DL / 8), c = e % (DL / 8);
+                if (r < cnt) wm::cp_async16(&dst[r][8 * c], rows + (r0 + r) * DL + 8 * c);
+                else *reinterpret_cast<uint4 *>(&dst[r][8 * c]) = make_uint4(0, 0, 0, 0);
+            }
+            wm::cp_commit();
+        };
+        float acc[4][NTW][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < NTW; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+        if (nblk > 0) {
+            issue(0);
+            if (nblk > 1) { issue(1); wm::cp_wait<1>(); } else { wm::cp_wait<0>(); }
+            nb_arrive(1 + 0);   // block 0 landed
+        }
+        for (int kb = 0; kb < nblk; ++kb) {
+            const int bb = kb & 1;
+            if (kb + 1 < nblk) {   // block kb + 1 (issued one block ago) landed
+                wm::cp_wait<0>();
+                nb_arrive(1 + (bb ^ 1));
+            }
+            nb_sync(3 + bb);   // P of block kb ready
+            const Row *V = sK + bb * KB;
+            const PRow *Pb = sP + bb * HEADS;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float a0 = sA[bb * HEADS + 16 * i + gr], a1 = sA[bb * HEADS + 16 * i + gr + 8];
+#pragma unroll
+                for (int j = 0; j < NTW; ++j) {
+                    acc[i][j][0] *= a0; acc[i][j][1] *= a0;
+                    acc[i][j][2] *= a1; acc[i][j][3] *= a1;
+                }
+            }
+#pragma unroll
+            for (int kc = 0; kc < KB / 16; ++kc) {
+                uint32_t pa[4][4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) wm::frag_a<PPITCH - 8>(pa[i], Pb, 16 * i, 16 * kc);
+#pragma unroll
+                for (int np = 0; np < NTW / 2; ++np) {
+                    uint32_t vb[4];
+                    wm::frag_b_kn<PITCH - 8>(vb, V, 16 * kc, 64 * pw + 16 * np);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        wm::mma16816(acc[i][2 * np], pa[i][0], pa[i][1], pa[i][2], pa[i][3], vb[0], vb[1]);
+                        wm::mma16816(acc[i][2 * np + 1], pa[i][0], pa[i][1], pa[i][2], pa[i][3], vb[2], vb[3]);
+                    }
+                }
+            }
+            if (kb + 2 < nblk) {
+                nb_arrive(5 + bb);   // P buffer bb read; block kb's buffer is free
+                issue(kb + 2);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int h = 16 * i + gr + 8 * x;
+                if (h0 + h >= a.H) continue;
+                float *dst = a.part_o + (pidx + h) * DC + 64 * pw;
+#pragma unroll
+                for (int j = 0; j < NTW; ++j)
+                    *reinterpret_cast<float2 *>(dst + 8 * j + 2 * tt) = make_float2(acc[i][j][2 * x], acc[i][j][2 * x + 1]);
+            }
+    }
+}
+
 // One CTA per (head, sequence): merge the shares.
 constexpr int kCombineThreads = 128;
 
@@ -447,6 +696,17 @@ static int launch_mla_t(const mla::Args &a, int groups, cudaStream_t st)
     return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
 }
 
+static int launch_mla_ws(const mla::Args &a, int groups, cudaStream_t st)
+{
+    const size_t smem = mla::WsSmem::bytes;
+    if (cudaFuncSetAttribute(mla::mla_decode_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return KSA_ERR_CUDA;
+    dim3 grid((unsigned)a.splits, (unsigned)groups, (unsigned)a.batch);
+    mla::mla_decode_ws_kernel<<<grid, mla::WS_THREADS, smem, st>>>(a);
+    return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
+}
+
 int launch_mla_decode(const ksa_mla_params *p, const ksa_mla_cache *c, const int8_t *kind, const void *q, void *o,
                       float *lse, int64_t max_text, void *ws, size_t ws_bytes, cudaStream_t st)
 {
@@ -470,8 +730,8 @@ int launch_mla_decode(const ksa_mla_params *p, const ksa_mla_cache *c, const int
     a.part_ml = reinterpret_cast<float *>(static_cast<char *>(ws) + align_up(rows * mla::DC * 4));
     a.o = (__nv_bfloat16 *)o;
     a.lse = lse;
-    int rc = P.mt == 4 ? launch_mla_t<4>(a, P.groups, st) : P.mt == 2 ? launch_mla_t<2>(a, P.groups, st)
-                                                                       : launch_mla_t<1>(a, P.groups, st);
+    int rc = P.mt == 4 ? launch_mla_ws(a, P.groups, st) : P.mt == 2 ? launch_mla_t<2>(a, P.groups, st)
+                                                                     : launch_mla_t<1>(a, P.groups, st);
     if (rc != KSA_OK) return rc;
     dim3 grid((unsigned)p->num_heads, (unsigned)c->batch);
     mla::mla_combine_kernel<<<grid, mla::kCombineThreads, 0, st>>>(a);

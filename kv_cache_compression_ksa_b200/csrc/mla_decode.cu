@@ -645,12 +645,24 @@ static Plan plan(const ksa_mla_params *p, int batch, int64_t max_text)
     P.groups = (p->num_heads + 16 * P.mt - 1) / (16 * P.mt);
     const int64_t mmax = max_text / p->k;
     const int64_t lmax = (int64_t)p->k + 1 + (int64_t)p->w * p->k + (mmax > p->w ? mmax - p->w : 0);
-    // enough CTAs for two per SM, each share at least 4 blocks
-    const int64_t ctas = (int64_t)batch * P.groups;
-    const int64_t want = ctas > 0 ? (2LL * sm_count() + ctas - 1) / ctas : 1;
+    // Enough shares for two CTAs per SM, each at least 4 blocks.  Then, while
+    // a share keeps at least 1024 slots (so the partial outputs stay small
+    // against the slice), a larger count up to twice the four-wave count may
+    // be taken if its last wave is fuller (one CTA per SM fits).
+    const int64_t ctas = (int64_t)batch * P.groups, sms = sm_count();
+    const int64_t want = ctas > 0 ? (2 * sms + ctas - 1) / ctas : 1;
     const int64_t most = (lmax + 4 * KB - 1) / (4 * KB);
     int64_t sp = want < most ? want : most;
     if (sp < 1) sp = 1;
+    const int64_t four = ctas > 0 ? (4 * sms + ctas - 1) / ctas : 1;
+    int64_t top = (four > sp ? four : sp) * 2;
+    if (top > lmax / 1024) top = lmax / 1024;
+    double best = -1.0;
+    for (int64_t c = sp, c0 = sp; c <= (top > c0 ? top : c0) && ctas > 0; ++c) {
+        const double waves = (double)(ctas * c) / (double)sms;
+        const double eff = waves / (double)((ctas * c + sms - 1) / sms);
+        if (eff > best + 1e-9) { best = eff; sp = c; }
+    }
     if (sp > 1024) sp = 1024;
     int64_t per = (lmax + sp - 1) / sp;
     per = (per + KB - 1) / KB * KB;

@@ -53,6 +53,7 @@ struct Args {
     float *dsum;                      // [rows, Hq] D = rowsum(dO * O)
     float *dk32, *dv32;               // [rows, Hkv, d] fp32 accumulators of the split dk/dv pass
     int nblk;                         // upper bound of the block count (grid x)
+    int sumq_only;                    // dk/dv pass: only the summary query rows (the text rows run on tcgen05)
     __nv_bfloat16 *dq, *dk, *dv;
 };
 
@@ -386,7 +387,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
         s_lo = K.idx0;
         s_hi = K.idx0 + K.cnt;
     }
-    const int ntb = (t_hi - t_lo + RB - 1) / RB;
+    const int ntb = a.sumq_only ? 0 : (t_hi - t_lo + RB - 1) / RB;
     const int nsb = s_hi > s_lo ? 1 : 0;   // at most 64 summaries see this block's keys
     // this CTA's share of the query blocks (split z of ceil((ntb + nsb) / QB_SPLIT))
     const int qb_lo = (int)blockIdx.z * QB_SPLIT, qb_hi = min(ntb + nsb, qb_lo + QB_SPLIT);
@@ -576,7 +577,8 @@ size_t prefill_bwd_workspace_bytes(const ksa_params *p, int batch, int64_t aug_r
 {
     return plan_bytes(batch) + 2 * align_up(sizeof(int32_t) * (size_t)(batch + 1)) +
            align_up(sizeof(float) * (size_t)aug_rows * p->num_q_heads) +
-           2 * align_up(sizeof(float) * (size_t)aug_rows * p->num_kv_heads * p->head_dim);
+           2 * align_up(sizeof(float) * (size_t)aug_rows * p->num_kv_heads * p->head_dim) +
+           prefill_bwd_tc_workspace_bytes(batch, aug_rows);
 }
 
 int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,
@@ -611,8 +613,18 @@ int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_
     if (nblk > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
     a.nblk = (int)nblk;
     // query blocks any key block can meet: at most total_text/64 + 2 (text + one summary block)
-    const int64_t zsplits = (total_text / bw::RB + 2 + bw::QB_SPLIT - 1) / bw::QB_SPLIT;
+    int64_t zsplits = (total_text / bw::RB + 2 + bw::QB_SPLIT - 1) / bw::QB_SPLIT;
     if (zsplits > 65535) return KSA_ERR_UNSUPPORTED;
+    // dk, dv from the text query rows on the tensor-core kernel where the
+    // shape allows; the warp-level dk/dv pass then only adds the summary rows'
+    a.sumq_only = 0;
+    if (prefill_bwd_tc_supported(p)) {
+        const int r = launch_prefill_bwd_dkv_tc(p, batch, cu, total_text, aug_rows, q, k, v, dout, lse, a.dsum, a.dk32,
+                                                a.dv32, w + 2 * ab + dsb + 2 * accb, pl, err, st);
+        if (r != KSA_OK) return r;
+        a.sumq_only = 1;
+        zsplits = 1;
+    }
     if (p->head_dim == 128) {
         if (bw_launch<128>(a, nblk, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
     } else if (p->head_dim == 64) {

@@ -1,0 +1,564 @@
+// prefill_bwd_sm100.cu -- dk, dv of the KSA prefill from the text query rows
+// on tcgen05 (TMA -> SMEM -> tcgen05.mma -> TMEM).
+//
+// Kwai Summary Attention Technical Report: the forward is Eq. (10),
+// softmax(Q K^T / sqrt(d) + M_KSA) V, under the mask of section 2.2.2,
+// Eqs. (2)-(3): text t_i (chunk c = floor(i/k)) sees the text of chunks
+// c-w .. c causally and the summaries s_0 .. s_{c-w-1}.  Read from the key
+// side, text key p (chunk c_p) is seen by the text queries p ..
+// (c_p + w + 1) k - 1 and summary key j by the text queries from
+// (j + w + 1) k on.  The gradients are the textbook ones: P = exp(S - lse),
+// dP = dO V^T, dS = P (dP - D) with D = rowsum(dO * O), dv = P^T dO,
+// dk = scale dS^T Q.
+//
+// Design.  A CTA owns one tile of 128 keys of one kind (128 consecutive text
+// tokens or 128 consecutive summaries of one sequence) of one kv head: its K
+// and V sit in shared memory for the whole CTA and its rows are the 128
+// TMEM lanes.  It walks a share of at most kSplit steps; a step is one q head
+// of the kv head's group x 128 consecutive text query positions (TMA boxes
+// over the augmented layout's text slots), and takes four MMAs:
+//     S^T  = K Q^T      (SS, M 128 keys, N 128 queries, K d)
+//     dP^T = V dO^T     (SS)
+//     dV  += P^T dO     (TS: P^T written as bf16 over S^T, B = dO MN-major)
+//     dK  += dS^T Q     (TS: dS^T written as bf16 over dP^T)
+// TMEM holds S^T, dP^T, dV and dK (128 + 128 + 2 d columns).  Eight
+// elementwise warps (two per TMEM lane quarter, 64 query columns each) turn
+// S^T into P^T and dP^T into dS^T; the mask of a key row inside a step is
+// one interval of columns, from coordinates.  The summary query rows (a
+// summary sees its own chunk and itself) are left to the warp-level kernel of
+// prefill_bwd.cu.  Shares of the same key tile (long summary ranges) add
+// their dK, dV into fp32 accumulators.  All mbarrier waits are bounded.
+#include <cuda.h>
+#include <math.h>
+
+#include "ksa_internal.cuh"
+#include "tc_sm100.cuh"
+
+namespace ksa {
+namespace bt {
+
+using namespace tc;
+
+constexpr int BK = 128;       // keys per tile (TMEM lanes)
+constexpr int BQ = 128;       // query positions per step (MMA N)
+constexpr int HQ = BQ / 2;    // query columns per elementwise warp
+constexpr int QST = 2;        // Q / dO stages
+constexpr int kSplit = 32;    // steps per CTA
+constexpr int kWarpTMA = 8;   // K, V once, then Q and dO per step
+constexpr int kWarpMMA = 9;   // MMA issuer, TMEM owner
+constexpr int kWarpLD = 10;   // per-step LSE and D, zero rows past the sequence
+constexpr int kThreads = 352;
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Smem {
+    static constexpr int kTile = BK * D * 2;   // one 128 x D bf16 tile
+    static constexpr int kK = 0;
+    static constexpr int kV = kK + kTile;
+    static constexpr int kQ = kV + kTile;            // [QST] query tiles
+    static constexpr int kDO = kQ + QST * kTile;     // [QST] dO tiles
+    static constexpr int kLD = kDO + QST * kTile;    // [QST][lse2, D][BQ] floats
+    static constexpr int kBar = kLD + QST * 2 * BQ * 4;
+    // kv, qt[QST], qf[QST], qe[QST], s, dp, p, ds, dv, dk, drain
+    static constexpr int kNumBars = 1 + 3 * QST + 7;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16;
+    static_assert(kBytes <= 227 * 1024, "shared memory budget");
+    static_assert(2 * BQ + 2 * D <= (int)kTmemCols, "TMEM budget");
+};
+
+struct TArgs {
+    CUtensorMap tm_kt, tm_ks, tm_vt, tm_vs, tm_q, tm_do;
+    int k, w, G, Hq, Hkv, batch;
+    float scale, scale_log2;
+    const int32_t *cu;
+    Plan pl;
+    const int32_t *ks_off, *kt_off;   // [B+1] first summary / text key tile of each sequence
+    const int32_t *item_off;          // [tiles+1] first CTA of each key tile (summary tiles first)
+    int max_tiles;
+    int32_t *err;
+    const float *lse, *dsum;
+    float *dk32, *dv32;
+};
+
+// A key tile and the text query range that sees it.
+struct KTile {
+    int b, sum, j0, kcnt, n, m, c0, qlo, qhi, nq;   // nq: query tiles of 128 positions
+};
+
+__device__ __forceinline__ int find_off(const int32_t *off, int batch, int id)
+{
+    int lo = 0, hi = batch - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= id) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ void key_tile(const TArgs &a, int tile, KTile &T)
+{
+    const int ns = a.ks_off[a.batch];
+    T.sum = tile < ns;
+    const int32_t *off = T.sum ? a.ks_off : a.kt_off;
+    const int id = T.sum ? tile : tile - ns;
+    T.b = find_off(off, a.batch, id);
+    T.j0 = (id - off[T.b]) * BK;
+    T.n = a.cu[T.b + 1] - a.cu[T.b];
+    T.m = T.n / a.k;
+    T.c0 = a.pl.chunk_off[T.b];
+    if (T.sum) {
+        T.kcnt = min(BK, T.m - T.j0);
+        T.qlo = min(T.n, (T.j0 + a.w + 1) * a.k);   // first text query of summary j0
+        T.qhi = T.n;
+    } else {
+        T.kcnt = min(BK, T.n - T.j0);
+        const int cb = (T.j0 + T.kcnt - 1) / a.k;
+        T.qlo = T.j0;
+        T.qhi = min(T.n, (cb + a.w + 1) * a.k);     // past the last text query of chunk cb's keys
+    }
+    T.nq = T.qhi > T.qlo ? (T.qhi - T.qlo + BQ - 1) / BQ : 0;
+}
+
+// Key tiles (summary tiles of all sequences, then text tiles) and the CTA
+// offsets of their shares of ceil(G nq / kSplit) CTAs each.
+__global__ void __launch_bounds__(1024) bt_plan_kernel(TArgs a, int32_t *ks_off, int32_t *kt_off, int32_t *item_off)
+{
+    __shared__ int part[1024];
+    __shared__ int s_nt;
+    if (threadIdx.x == 0) {
+        int s = 0, t = 0;
+        for (int b = 0; b < a.batch; ++b) {
+            ks_off[b] = s;
+            kt_off[b] = t;
+            const int n = max(a.cu[b + 1] - a.cu[b], 0);
+            s += (n / a.k + BK - 1) / BK;
+            t += (n + BK - 1) / BK;
+        }
+        ks_off[a.batch] = s;
+        kt_off[a.batch] = t;
+        s_nt = s + t;
+        if (s + t > a.max_tiles) {
+            set_error(a.err, KSA_ERR_UNSUPPORTED);
+            s_nt = 0;
+        }
+    }
+    __syncthreads();
+    const int NT = s_nt;
+    const int per = (NT + 1023) / 1024;
+    const int lo = min(NT, (int)threadIdx.x * per), hi = min(NT, lo + per);
+    int sum = 0;
+    for (int t = lo; t < hi; ++t) {
+        KTile T;
+        key_tile(a, t, T);
+        sum += (a.G * T.nq + kSplit - 1) / kSplit;
+    }
+    part[threadIdx.x] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {   // exclusive scan of the 1024 partial counts
+        int run = 0;
+        for (int i = 0; i < 1024; ++i) {
+            const int v = part[i];
+            part[i] = run;
+            run += v;
+        }
+        item_off[NT] = run;
+    }
+    __syncthreads();
+    int run = part[threadIdx.x];
+    for (int t = lo; t < hi; ++t) {
+        item_off[t] = run;
+        KTile T;
+        key_tile(a, t, T);
+        run += (a.G * T.nq + kSplit - 1) / kSplit;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_constant__ TArgs a)
+{
+    using L = Smem<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw;
+    const uint32_t sbase = smem_u32(smem);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (*a.err != 0) return;
+    if (sbase & 1023u) {
+        if (threadIdx.x == 0) set_error(a.err, KSA_ERR_UNSUPPORTED);
+        return;
+    }
+    // this CTA's key tile and share (uniform over the CTA; empty CTAs leave
+    // before any barrier or TMEM is touched)
+    const int NT = a.ks_off[a.batch] + a.kt_off[a.batch];
+    if (NT > a.max_tiles) return;
+    const int item = blockIdx.x;
+    if (item >= a.item_off[NT]) return;
+    const int tile = find_off(a.item_off, NT, item);
+    KTile T;
+    key_tile(a, tile, T);
+    const int g = blockIdx.y;
+    const int s_lo = (item - a.item_off[tile]) * kSplit;
+    const int n_steps = min(a.G * T.nq, s_lo + kSplit) - s_lo;
+    if (n_steps <= 0) return;
+
+    auto bar = [&](int i) { return sbase + L::kBar + 8u * (uint32_t)i; };
+    constexpr int B_KV = 0;
+    auto B_QT = [](int s) { return 1 + s; };              // Q, dO landed
+    auto B_QF = [](int s) { return 1 + QST + s; };        // + LSE, D, zero rows: ready
+    auto B_QE = [](int s) { return 1 + 2 * QST + s; };    // stage free
+    constexpr int B_S = 1 + 3 * QST, B_DP = B_S + 1, B_P = B_S + 2, B_DS = B_S + 3, B_DV = B_S + 4,
+                  B_DK = B_S + 5, B_DRAIN = B_S + 6;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_KV), 1);
+        for (int s = 0; s < QST; ++s) {
+            mbar_init(bar(B_QT(s)), 1);
+            mbar_init(bar(B_QF(s)), 32);
+            mbar_init(bar(B_QE(s)), 1);
+        }
+        mbar_init(bar(B_S), 1);
+        mbar_init(bar(B_DP), 1);
+        mbar_init(bar(B_P), 256);
+        mbar_init(bar(B_DS), 256);
+        mbar_init(bar(B_DV), 1);
+        mbar_init(bar(B_DK), 1);
+        mbar_init(bar(B_DRAIN), 1);
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == kWarpMMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t T_S = tmem, T_DP = tmem + BQ, T_DV = tmem + 2 * BQ, T_DK = tmem + 2 * BQ + D;
+    constexpr uint32_t kHalf = BK * 128;   // bytes of one 64-column half of a tile
+    constexpr uint32_t kTileBytes = (uint32_t)L::kTile;
+
+    // step s of the share -> (query tile, q head)
+    auto step_q0 = [&](int s) { return T.qlo + ((s_lo + s) / a.G) * BQ; };
+    auto step_h = [&](int s) { return g * a.G + (s_lo + s) % a.G; };
+
+    if (warp == kWarpTMA) {
+        if (lane == 0) {
+            bool ok = true;
+            int q_issued[QST] = {0};
+            mbar_expect_tx(bar(B_KV), 2 * kTileBytes);
+            for (int hf = 0; hf < D / 64; ++hf) {
+                if (T.sum) {
+                    tma_load_4d(sbase + L::kK + hf * kHalf, &a.tm_ks, bar(B_KV), hf * 64, g, a.k, T.c0 + T.j0);
+                    tma_load_4d(sbase + L::kV + hf * kHalf, &a.tm_vs, bar(B_KV), hf * 64, g, a.k, T.c0 + T.j0);
+                } else {
+                    tma_load_4d(sbase + L::kK + hf * kHalf, &a.tm_kt, bar(B_KV), hf * 64, g, 0, T.c0 + T.j0 / a.k);
+                    tma_load_4d(sbase + L::kV + hf * kHalf, &a.tm_vt, bar(B_KV), hf * 64, g, 0, T.c0 + T.j0 / a.k);
+                }
+            }
+            for (int s = 0; s < n_steps; ++s) {
+                const int st = s % QST;
+                if (s >= QST && !(ok = mbar_wait(bar(B_QE(st)), (uint32_t)((s / QST) - 1) & 1u, abort, a.err)))
+                    break;
+                const int chunk = T.c0 + step_q0(s) / a.k, h = step_h(s);
+                mbar_expect_tx(bar(B_QT(st)), 2 * kTileBytes);
+                for (int hf = 0; hf < D / 64; ++hf) {
+                    tma_load_4d(sbase + L::kQ + st * kTileBytes + hf * kHalf, &a.tm_q, bar(B_QT(st)), hf * 64, h, 0,
+                                chunk);
+                    tma_load_4d(sbase + L::kDO + st * kTileBytes + hf * kHalf, &a.tm_do, bar(B_QT(st)), hf * 64, h,
+                                0, chunk);
+                }
+                q_issued[st]++;
+            }
+            // every load issued lands before the CTA exits
+            for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_KV), 0); ++it) {}
+            if (!ok)
+                for (int st = 0; st < QST; ++st)
+                    if (q_issued[st]) {
+                        const uint32_t ph = (uint32_t)(q_issued[st] - 1) & 1u;
+                        for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_QT(st)), ph); ++it) {}
+                    }
+        }
+    } else if (warp == kWarpLD) {
+        // per step: wait for the tiles, zero the query rows past the sequence
+        // (they meet P = 0 and dS = 0 in the MMAs, which need them finite),
+        // then the step's LSE (log2 units) and D into shared memory
+        bool ok = true;
+        for (int s = 0; s < n_steps && ok; ++s) {
+            const int st = s % QST;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QT(st)), (uint32_t)(s / QST) & 1u, abort, a.err));
+            if (!ok) break;
+            const int q0 = step_q0(s), h = step_h(s);
+            const int qn = min(BQ, T.n - q0);
+            if (qn < BQ) {
+                const int per_row = 8 * (D / 64);   // 16-byte words of a row over both halves
+                for (int e = lane; e < (BQ - qn) * per_row; e += 32) {
+                    const int r = qn + e / per_row, hf = (e % per_row) / 8, c = e % 8;
+                    const uint32_t off = (uint32_t)(hf * kHalf + r * 128 + c * 16);
+                    *reinterpret_cast<uint4 *>(smem + L::kQ + st * kTileBytes + off) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(smem + L::kDO + st * kTileBytes + off) = make_uint4(0, 0, 0, 0);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            }
+            float *ld = reinterpret_cast<float *>(smem + L::kLD) + st * 2 * BQ;
+            for (int r = lane; r < BQ; r += 32) {
+                float l2 = 0.f, dd = 0.f;
+                if (r < qn) {
+                    const int pos = q0 + r;
+                    const int64_t row = (int64_t)(T.c0 + pos / a.k) * (a.k + 1) + pos % a.k;
+                    l2 = a.lse[row * a.Hq + h] * 1.4426950408889634f;
+                    dd = a.dsum[row * a.Hq + h];
+                }
+                ld[r] = l2;
+                ld[BQ + r] = dd;
+            }
+            mbar_arrive(bar(B_QF(st)));
+        }
+    } else if (warp == kWarpMMA) {
+        if (lane == 0) {
+            const uint32_t id_ss = idesc_f16(BK, BQ, false);
+            const uint32_t id_ts = idesc_f16(BK, D, true);
+            bool ok = mbar_wait(bar(B_KV), 0, abort, a.err);
+            for (int s = 0; s < n_steps && ok; ++s) {
+                const int st = s % QST;
+                const uint32_t ph = (uint32_t)s & 1u, php = (uint32_t)(s - 1) & 1u;
+                if (!(ok = mbar_wait(bar(B_QF(st)), (uint32_t)(s / QST) & 1u, abort, a.err))) break;
+                const uint32_t qa = sbase + L::kQ + st * kTileBytes, da = sbase + L::kDO + st * kTileBytes;
+                // S^T = K Q^T into the S columns, free once the previous dV has read P^T
+                if (s > 0 && !(ok = mbar_wait(bar(B_DV), php, abort, a.err))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(T_S, sdesc(sbase + L::kK + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024),
+                           sdesc(qa + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024), id_ss, kk > 0);
+                tc_commit(bar(B_S));
+                // dP^T = V dO^T, once the previous dK has read dS^T
+                if (s > 0 && !(ok = mbar_wait(bar(B_DK), php, abort, a.err))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(T_DP, sdesc(sbase + L::kV + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024),
+                           sdesc(da + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024), id_ss, kk > 0);
+                tc_commit(bar(B_DP));
+                // dV += P^T dO: half h's P^T (64 queries as bf16 pairs) sits in
+                // S columns [64h, 64h + 32) and meets dO rows [64h, 64h + 64)
+                if (!(ok = mbar_wait(bar(B_P), ph, abort, a.err))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int kk = 0; kk < HQ / 16; ++kk)
+                        mma_ts(T_DV, T_S + h * HQ + kk * 8, sdesc(da + (h * (HQ / 16) + kk) * 2048, kHalf, 1024), id_ts,
+                               (s > 0 || h > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(bar(B_DV));
+                // dK += dS^T Q
+                if (!(ok = mbar_wait(bar(B_DS), ph, abort, a.err))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int kk = 0; kk < HQ / 16; ++kk)
+                        mma_ts(T_DK, T_DP + h * HQ + kk * 8, sdesc(qa + (h * (HQ / 16) + kk) * 2048, kHalf, 1024),
+                               id_ts, (s > 0 || h > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(bar(B_DK));
+                tc_commit(bar(B_QE(st)));
+            }
+            tc_commit(bar(B_DRAIN));
+            for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_DRAIN), 0); ++it) {}
+        }
+    } else if (warp < 8) {
+        // ================= elementwise: 8 warps, 64 query columns each =================
+        const int half = warp >> 2, quarter = warp & 3;
+        const int r = quarter * 32 + lane;   // key row = TMEM lane
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const bool live = r < T.kcnt;
+        const int key = T.j0 + r;            // text position or summary index
+        const float sl2 = a.scale_log2;
+        bool ok = true;
+        for (int s = 0; s < n_steps; ++s) {
+            const int st = s % QST;
+            const uint32_t ph = (uint32_t)s & 1u;
+            const int q0 = step_q0(s);
+            const int qn = min(BQ, T.n - q0);
+            // this row's visible columns [lo, hi) of the step, inside this half
+            int lo, hi;
+            if (T.sum) {
+                lo = (key + a.w + 1) * a.k - q0;
+                hi = qn;
+            } else {
+                lo = key - q0;
+                hi = min(qn, (key / a.k + a.w + 1) * a.k - q0);
+            }
+            if (!live) lo = hi = 0;
+            lo = max(lo - half * HQ, 0);
+            hi = min(hi - half * HQ, HQ);
+            if (hi < lo) hi = lo;
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(B_QF(st)), (uint32_t)(s / QST) & 1u, abort, a.err));
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(B_S), ph, abort, a.err));
+            if (!ok) break;
+            const float *l2 = reinterpret_cast<const float *>(smem + L::kLD) + st * 2 * BQ + half * HQ;
+            const float *dd = l2 + BQ;
+            float p[HQ];
+            {
+                uint32_t sr[HQ];
+                tc_fence_after();
+                tmem_ld32(T_S + lane_off + half * HQ, sr);
+                tmem_ld32(T_S + lane_off + half * HQ + 32, sr + 32);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < HQ; ++e) {
+                    const float x = fmaf(__uint_as_float(sr[e]), sl2, -l2[e]);
+                    p[e] = (e >= lo && e < hi) ? ex2(x) : 0.f;
+                }
+#pragma unroll
+                for (int grp = 0; grp < 2; ++grp) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e2 = 0; e2 < 16; ++e2) pk[e2] = pack_bf16(p[grp * 32 + 2 * e2], p[grp * 32 + 2 * e2 + 1]);
+                    tmem_st16(T_S + lane_off + half * HQ + grp * 16, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(B_P));
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DP), ph, abort, a.err));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int grp = 0; grp < 2; ++grp) {
+                uint32_t dr[32], pk[16];
+                tmem_ld32(T_DP + lane_off + half * HQ + grp * 32, dr);
+                tmem_wait_ld();
+                float ds[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int c = grp * 32 + e;
+                    ds[e] = (c >= lo && c < hi) ? p[c] * (__uint_as_float(dr[e]) - dd[c]) : 0.f;
+                }
+#pragma unroll
+                for (int e2 = 0; e2 < 16; ++e2) pk[e2] = pack_bf16(ds[2 * e2], ds[2 * e2 + 1]);
+                // dS^T of this half -> dP^T columns [64 half + 16 grp, +16); the
+                // second group's load above read columns at or past 64 half + 32
+                tmem_st16(T_DP + lane_off + half * HQ + grp * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(B_DS));
+        }
+        // ---- epilogue: dK (scaled) and dV rows into the fp32 accumulators ----
+        if (ok)
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DK), (uint32_t)(n_steps - 1) & 1u, abort, a.err));
+        if (ok) {
+            tc_fence_after();
+            const int64_t row = T.sum ? (int64_t)(T.c0 + key) * (a.k + 1) + a.k
+                                      : (int64_t)(T.c0 + key / a.k) * (a.k + 1) + key % a.k;
+            float4 *pk = reinterpret_cast<float4 *>(a.dk32 + (row * a.Hkv + g) * D + half * (D / 2));
+            float4 *pv = reinterpret_cast<float4 *>(a.dv32 + (row * a.Hkv + g) * D + half * (D / 2));
+#pragma unroll 1
+            for (int cc = 0; cc < D / 64; ++cc) {
+                uint32_t vk[32], vv[32];
+                tmem_ld32(T_DK + lane_off + half * (D / 2) + cc * 32, vk);
+                tmem_ld32(T_DV + lane_off + half * (D / 2) + cc * 32, vv);
+                tmem_wait_ld();
+                if (live) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        atomicAdd(pk + cc * 8 + e,
+                                  make_float4(__uint_as_float(vk[4 * e]) * a.scale, __uint_as_float(vk[4 * e + 1]) * a.scale,
+                                              __uint_as_float(vk[4 * e + 2]) * a.scale,
+                                              __uint_as_float(vk[4 * e + 3]) * a.scale));
+                        atomicAdd(pv + cc * 8 + e, make_float4(__uint_as_float(vv[4 * e]), __uint_as_float(vv[4 * e + 1]),
+                                                               __uint_as_float(vv[4 * e + 2]),
+                                                               __uint_as_float(vv[4 * e + 3])));
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- teardown --------------------------------------------------------
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpMMA) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace bt
+
+bool prefill_bwd_tc_supported(const ksa_params *p)
+{
+    return (p->head_dim == 128 || p->head_dim == 64) && p->k >= 1 && p->k <= bt::BQ && bt::BQ % p->k == 0 &&
+           p->num_kv_heads > 0 && p->num_q_heads % p->num_kv_heads == 0;
+}
+
+size_t prefill_bwd_tc_workspace_bytes(int batch, int64_t aug_rows)
+{
+    const int64_t tiles = aug_rows / bt::BK + 2LL * batch + 2;
+    return 2 * align_up(sizeof(int32_t) * (size_t)(batch + 1)) + align_up(sizeof(int32_t) * (size_t)(tiles + 1));
+}
+
+template <int D>
+static int bt_launch(const bt::TArgs &a, int64_t grid, cudaStream_t st)
+{
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(bt::bt_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 bt::Smem<D>::kBytes) != cudaSuccess)
+            return KSA_ERR_CUDA;
+        attr = true;
+    }
+    bt::bt_dkv_kernel<D><<<dim3((unsigned)grid, a.Hkv), bt::kThreads, bt::Smem<D>::kBytes, st>>>(a);
+    return KSA_OK;
+}
+
+int launch_prefill_bwd_dkv_tc(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,
+                              const void *q, const void *k, const void *v, const void *dout, const float *lse,
+                              const float *dsum, float *dk32, float *dv32, void *ws, const Plan &pl, int32_t *err,
+                              cudaStream_t st)
+{
+    bt::TArgs a;
+    const int d = p->head_dim, kk = p->k;
+    const int64_t chunks = aug_rows / (kk + 1);
+    const int qrows = bt::BQ / kk;   // chunks per query / text key box
+    bool ok = make_map(&a.tm_kt, k, d, p->num_kv_heads, kk, chunks, 1, kk, qrows) &&
+              make_map(&a.tm_vt, v, d, p->num_kv_heads, kk, chunks, 1, kk, qrows) &&
+              make_map(&a.tm_ks, k, d, p->num_kv_heads, kk, chunks, 1, 1, bt::BK) &&
+              make_map(&a.tm_vs, v, d, p->num_kv_heads, kk, chunks, 1, 1, bt::BK) &&
+              make_map(&a.tm_q, q, d, p->num_q_heads, kk, chunks, 1, kk, qrows) &&
+              make_map(&a.tm_do, dout, d, p->num_q_heads, kk, chunks, 1, kk, qrows);
+    if (!ok) return KSA_ERR_CUDA;
+    a.k = kk; a.w = p->w; a.Hq = p->num_q_heads; a.Hkv = p->num_kv_heads; a.G = a.Hq / a.Hkv; a.batch = batch;
+    a.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)d);
+    a.scale_log2 = a.scale * 1.4426950408889634f;
+    a.cu = cu; a.pl = pl; a.err = err;
+    a.lse = lse; a.dsum = dsum; a.dk32 = dk32; a.dv32 = dv32;
+    char *w = static_cast<char *>(ws);
+    const size_t ab = align_up(sizeof(int32_t) * (size_t)(batch + 1));
+    int32_t *ks_off = reinterpret_cast<int32_t *>(w), *kt_off = reinterpret_cast<int32_t *>(w + ab);
+    int32_t *item_off = reinterpret_cast<int32_t *>(w + 2 * ab);
+    const int64_t max_tiles = aug_rows / bt::BK + 2LL * batch + 2;
+    if (max_tiles > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
+    a.ks_off = ks_off; a.kt_off = kt_off; a.item_off = item_off; a.max_tiles = (int)max_tiles;
+    bt::bt_plan_kernel<<<1, 1024, 0, st>>>(a, ks_off, kt_off, item_off);
+    // CTAs: at most one per key tile plus G nq / kSplit per tile; a summary
+    // tile's queries number at most total_text, a text tile's 128 + (w+1) k
+    const int64_t ns_tiles = (total_text / kk) / bt::BK + batch, nt_tiles = total_text / bt::BK + batch;
+    const int64_t G = a.G;
+    const int64_t q_sum = (total_text + bt::BQ - 1) / bt::BQ + 1;
+    const int64_t q_txt = (bt::BK + (int64_t)(p->w + 1) * kk + bt::BQ - 1) / bt::BQ + 1;
+    const int64_t grid = ns_tiles * (1 + (G * q_sum) / bt::kSplit) + nt_tiles * (1 + (G * q_txt) / bt::kSplit);
+    if (grid > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
+    if (grid == 0) return KSA_OK;
+    const int r = d == 128 ? bt_launch<128>(a, grid, st) : bt_launch<64>(a, grid, st);
+    if (r != KSA_OK) return r;
+    return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
+}
+
+}  // namespace ksa

@@ -68,15 +68,16 @@ int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_
                        const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
                        void *dq, void *dk, void *dv, void *ws, const Plan &pl, int32_t *err, cudaStream_t st);
 
-// Tensor-core dk, dv of the text query rows (prefill_bwd_sm100.cu): adds into
-// the fp32 accumulators dk32, dv32 ([aug_rows, Hkv, d], zeroed by the caller);
-// ws holds prefill_bwd_tc_workspace_bytes.
+// Tensor-core backward of the text query rows (prefill_bwd_sm100.cu): dk, dv
+// added into the fp32 accumulators dk32, dv32 ([aug_rows, Hkv, d], zeroed by
+// the caller), dq of the text rows written as bf16; ws holds
+// prefill_bwd_tc_workspace_bytes.
 bool prefill_bwd_tc_supported(const ksa_params *p);
 size_t prefill_bwd_tc_workspace_bytes(int batch, int64_t aug_rows);
-int launch_prefill_bwd_dkv_tc(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,
-                              const void *q, const void *k, const void *v, const void *dout, const float *lse,
-                              const float *dsum, float *dk32, float *dv32, void *ws, const Plan &pl, int32_t *err,
-                              cudaStream_t st);
+int launch_prefill_bwd_tc(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,
+                          const void *q, const void *k, const void *v, const void *dout, const float *lse,
+                          const float *dsum, float *dk32, float *dv32, void *dq, void *ws, const Plan &pl,
+                          int32_t *err, cudaStream_t st);
 
 // Decode cache from the augmented K/V of a prefilled batch (cache_decode.cu).
 int launch_cache_build(const ksa_params *p, const ksa_cache *c, const int32_t *cu, const void *k_aug,

@@ -53,7 +53,8 @@ struct Args {
     float *dsum;                      // [rows, Hq] D = rowsum(dO * O)
     float *dk32, *dv32;               // [rows, Hkv, d] fp32 accumulators of the split dk/dv pass
     int nblk;                         // upper bound of the block count (grid x)
-    int sumq_only;                    // dk/dv pass: only the summary query rows (the text rows run on tcgen05)
+    int sumq_only;                    // only the summary query rows (the text rows run on tcgen05):
+                                      // dk/dv from them, and dq of them
     __nv_bfloat16 *dq, *dk, *dv;
 };
 
@@ -176,7 +177,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(Args a)
     // text blocks late in a sequence see the most summaries: reverse order
     // puts them first
     const int nreal = a.tb_off[a.batch] + a.sb_off[a.batch];
-    const int id = (int)blockIdx.x < nreal ? nreal - 1 - (int)blockIdx.x : (int)blockIdx.x;
+    const int id = a.sumq_only ? a.tb_off[a.batch] + (int)blockIdx.x
+                               : ((int)blockIdx.x < nreal ? nreal - 1 - (int)blockIdx.x : (int)blockIdx.x);
     if (!block_of(a, id, Q)) return;
     const int h = blockIdx.y, g = h / a.G;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tt = lane & 3;
@@ -555,7 +557,7 @@ __global__ void bwd_blocks_kernel(int batch, const int32_t *cu, int k, int32_t *
 
 // four 64-row tiles of D + 8 bf16 per row (+ per-query LSE and D for dk, dv)
 template <int D>
-static int bw_launch(const bw::Args &a, int64_t nblk, int64_t zsplits, cudaStream_t st)
+static int bw_launch(const bw::Args &a, int64_t nblk, int64_t nblk_dq, int64_t zsplits, cudaStream_t st)
 {
     const int tiles = 6 * bw::RB * (D + 8) * 2;              // Q, dO + two (K, V) / K, V + two (Q, dO)
     const int dkv = tiles + 2 * 2 * bw::RB * 4;               // + two (LSE, D)
@@ -567,7 +569,7 @@ static int bw_launch(const bw::Args &a, int64_t nblk, int64_t zsplits, cudaStrea
             return KSA_ERR_CUDA;
         attr[D == 128] = true;
     }
-    bw::bwd_dq_kernel<D><<<dim3((unsigned)nblk, a.Hq), bw::kThreads, tiles, st>>>(a);
+    if (nblk_dq > 0) bw::bwd_dq_kernel<D><<<dim3((unsigned)nblk_dq, a.Hq), bw::kThreads, tiles, st>>>(a);
     bw::bwd_dkv_kernel<D><<<dim3((unsigned)nblk, a.Hkv, (unsigned)zsplits), bw::kThreads, dkv, st>>>(a);
     bw::bwd_dkv_out_kernel<<<dim3((unsigned)nblk, a.Hkv), 256, 0, st>>>(a, D);
     return KSA_OK;
@@ -615,20 +617,22 @@ int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_
     // query blocks any key block can meet: at most total_text/64 + 2 (text + one summary block)
     int64_t zsplits = (total_text / bw::RB + 2 + bw::QB_SPLIT - 1) / bw::QB_SPLIT;
     if (zsplits > 65535) return KSA_ERR_UNSUPPORTED;
-    // dk, dv from the text query rows on the tensor-core kernel where the
-    // shape allows; the warp-level dk/dv pass then only adds the summary rows'
+    // dq, dk, dv of the text query rows on the tensor-core kernels where the
+    // shape allows; the warp-level passes then only take the summary rows
     a.sumq_only = 0;
+    int64_t nblk_dq = nblk;
     if (prefill_bwd_tc_supported(p)) {
-        const int r = launch_prefill_bwd_dkv_tc(p, batch, cu, total_text, aug_rows, q, k, v, dout, lse, a.dsum, a.dk32,
-                                                a.dv32, w + 2 * ab + dsb + 2 * accb, pl, err, st);
+        const int r = launch_prefill_bwd_tc(p, batch, cu, total_text, aug_rows, q, k, v, dout, lse, a.dsum, a.dk32,
+                                            a.dv32, dq, w + 2 * ab + dsb + 2 * accb, pl, err, st);
         if (r != KSA_OK) return r;
         a.sumq_only = 1;
         zsplits = 1;
+        nblk_dq = (total_text / p->k) / bw::RB + batch;   // summary query blocks only
     }
     if (p->head_dim == 128) {
-        if (bw_launch<128>(a, nblk, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
+        if (bw_launch<128>(a, nblk, nblk_dq, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
     } else if (p->head_dim == 64) {
-        if (bw_launch<64>(a, nblk, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
+        if (bw_launch<64>(a, nblk, nblk_dq, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
     } else {
         return KSA_ERR_UNSUPPORTED;
     }

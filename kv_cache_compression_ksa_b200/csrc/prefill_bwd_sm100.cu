@@ -490,6 +490,312 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
     }
 }
 
+// ---------------------------------------------------------------------------
+// dq of the text query rows.  A CTA owns 128 consecutive text query
+// positions of one q head (rows = TMEM lanes; Q and dO stay in shared
+// memory) and walks the key tiles those rows can see: the summary tiles
+// s_0 .. s_{c_last-w-1}, then the text tiles from chunk c_first - w on.  A
+// step is three MMAs:
+//     S   = Q K^T      (SS, M 128 queries, N 128 keys)
+//     dP  = dO V^T     (SS, into one of two dP buffers)
+//     dQ += dS K       (TS: dS written as bf16 over its dP buffer, B = K
+//                       MN-major)
+// S is released as soon as the elementwise warps have loaded it, so the
+// next step's S runs while they form dS; the two dP buffers let dP(j+1)
+// run before dQ(j) has read dS(j).  TMEM: S, dP x 2, dQ.
+constexpr int KST = 3;   // K stages (a K tile is read by S(j) and by dQ(j) one step later)
+constexpr int VST = 2;   // V stages
+
+template <int D>
+struct SmemQ {
+    static constexpr int kTile = BK * D * 2;
+    static constexpr int kQ = 0;
+    static constexpr int kDO = kQ + kTile;
+    static constexpr int kK = kDO + kTile;            // [KST]
+    static constexpr int kV = kK + KST * kTile;       // [VST]
+    static constexpr int kBar = kV + VST * kTile;
+    // q, kf[KST], ke[KST], vf[VST], ve[VST], s, sc, dp, ds, dq, drain
+    static constexpr int kNumBars = 1 + 2 * KST + 2 * VST + 6;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16;
+    static_assert(kBytes <= 227 * 1024, "shared memory budget");
+    static_assert(3 * BK + D <= (int)kTmemCols, "TMEM budget");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constant__ TArgs a, __nv_bfloat16 *dq)
+{
+    using L = SmemQ<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw;
+    const uint32_t sbase = smem_u32(smem);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (*a.err != 0) return;
+    if (sbase & 1023u) {
+        if (threadIdx.x == 0) set_error(a.err, KSA_ERR_UNSUPPORTED);
+        return;
+    }
+    // query tile: text tiles in reverse (late tiles see the most summaries)
+    const int ntt = a.kt_off[a.batch];
+    if ((int)blockIdx.x >= ntt) return;
+    const int qt = ntt - 1 - (int)blockIdx.x;
+    const int b = find_off(a.kt_off, a.batch, qt);
+    const int n = a.cu[b + 1] - a.cu[b], m = n / a.k, c0 = a.pl.chunk_off[b];
+    const int q0 = (qt - a.kt_off[b]) * BQ;
+    const int qn = min(BQ, n - q0);
+    const int h = blockIdx.y, g = h / a.G;
+    const int c_first = q0 / a.k, c_last = (q0 + qn - 1) / a.k;
+    const int ns = max(0, min(m, c_last - a.w));          // summaries any row may see
+    const int n_sum = (ns + BK - 1) / BK;
+    const int t_lo = max(0, c_first - a.w) * a.k;         // text keys [t_lo, q0 + qn)
+    const int n_win = (q0 + qn - t_lo + BK - 1) / BK;
+    const int n_steps = n_sum + n_win;                    // >= 1: every row sees itself
+
+    auto bar = [&](int i) { return sbase + L::kBar + 8u * (uint32_t)i; };
+    constexpr int B_Q = 0;
+    auto B_KF = [](int s) { return 1 + s; };
+    auto B_KE = [](int s) { return 1 + KST + s; };
+    auto B_VF = [](int s) { return 1 + 2 * KST + s; };
+    auto B_VE = [](int s) { return 1 + 2 * KST + VST + s; };
+    constexpr int B_S = 1 + 2 * KST + 2 * VST, B_SC = B_S + 1, B_DP = B_S + 2, B_DS = B_S + 3, B_DQ = B_S + 4,
+                  B_DRAIN = B_S + 5;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_Q), 1);
+        for (int s = 0; s < KST; ++s) {
+            mbar_init(bar(B_KF(s)), 1);
+            mbar_init(bar(B_KE(s)), 1);
+        }
+        for (int s = 0; s < VST; ++s) {
+            mbar_init(bar(B_VF(s)), 1);
+            mbar_init(bar(B_VE(s)), 1);
+        }
+        mbar_init(bar(B_S), 1);
+        mbar_init(bar(B_SC), 256);
+        mbar_init(bar(B_DP), 1);
+        mbar_init(bar(B_DS), 256);
+        mbar_init(bar(B_DQ), 1);
+        mbar_init(bar(B_DRAIN), 1);
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == kWarpMMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t T_S = tmem, T_DQ = tmem + 3 * BK;
+    auto T_DP = [&](int j) { return tmem + (uint32_t)(BK + (j & 1) * BK); };
+    constexpr uint32_t kHalf = BK * 128;
+    constexpr uint32_t kTileBytes = (uint32_t)L::kTile;
+
+    if (warp == kWarpTMA) {
+        if (lane == 0) {
+            bool ok = true;
+            int k_issued[KST] = {0}, v_issued[VST] = {0};
+            mbar_expect_tx(bar(B_Q), 2 * kTileBytes);
+            for (int hf = 0; hf < D / 64; ++hf) {
+                tma_load_4d(sbase + L::kQ + hf * kHalf, &a.tm_q, bar(B_Q), hf * 64, h, 0, c0 + c_first);
+                tma_load_4d(sbase + L::kDO + hf * kHalf, &a.tm_do, bar(B_Q), hf * 64, h, 0, c0 + c_first);
+            }
+            // K of step j, then V of step j: K runs a stage further ahead
+            for (int j = 0; j < n_steps && ok; ++j) {
+                const bool sum = j < n_sum;
+                const int c1 = g, c2 = sum ? a.k : 0;
+                const int c3 = sum ? c0 + j * BK : c0 + (t_lo + (j - n_sum) * BK) / a.k;
+                const CUtensorMap *mk = sum ? &a.tm_ks : &a.tm_kt, *mv = sum ? &a.tm_vs : &a.tm_vt;
+                const int sk = j % KST, sv = j % VST;
+                if (j >= KST && !(ok = mbar_wait(bar(B_KE(sk)), (uint32_t)((j / KST) - 1) & 1u, abort, a.err)))
+                    break;
+                mbar_expect_tx(bar(B_KF(sk)), kTileBytes);
+                for (int hf = 0; hf < D / 64; ++hf)
+                    tma_load_4d(sbase + L::kK + sk * kTileBytes + hf * kHalf, mk, bar(B_KF(sk)), hf * 64, c1, c2, c3);
+                k_issued[sk]++;
+                if (j >= VST && !(ok = mbar_wait(bar(B_VE(sv)), (uint32_t)((j / VST) - 1) & 1u, abort, a.err)))
+                    break;
+                mbar_expect_tx(bar(B_VF(sv)), kTileBytes);
+                for (int hf = 0; hf < D / 64; ++hf)
+                    tma_load_4d(sbase + L::kV + sv * kTileBytes + hf * kHalf, mv, bar(B_VF(sv)), hf * 64, c1, c2, c3);
+                v_issued[sv]++;
+            }
+            for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_Q), 0); ++it) {}
+            if (!ok) {
+                for (int s = 0; s < KST; ++s)
+                    if (k_issued[s]) {
+                        const uint32_t ph = (uint32_t)(k_issued[s] - 1) & 1u;
+                        for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_KF(s)), ph); ++it) {}
+                    }
+                for (int s = 0; s < VST; ++s)
+                    if (v_issued[s]) {
+                        const uint32_t ph = (uint32_t)(v_issued[s] - 1) & 1u;
+                        for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_VF(s)), ph); ++it) {}
+                    }
+            }
+        }
+    } else if (warp == kWarpMMA) {
+        if (lane == 0) {
+            const uint32_t id_ss = idesc_f16(BK, BK, false);
+            const uint32_t id_ts = idesc_f16(BK, D, true);
+            // dQ(j) = dS(j) K(j): dS(j) (128 keys as bf16 pairs) sits in
+            // dP buffer j % 2, columns [64h, 64h + 32) for key half h
+            auto issue_dq = [&](int j) -> bool {
+                if (!mbar_wait(bar(B_DS), (uint32_t)j & 1u, abort, a.err)) return false;
+                tc_fence_after();
+                const uint32_t ka = sbase + L::kK + (j % KST) * kTileBytes;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                    for (int kk = 0; kk < HQ / 16; ++kk)
+                        mma_ts(T_DQ, T_DP(j) + hh * HQ + kk * 8, sdesc(ka + (hh * (HQ / 16) + kk) * 2048, kHalf, 1024),
+                               id_ts, (j > 0 || hh > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(bar(B_DQ));
+                tc_commit(bar(B_KE(j % KST)));
+                return true;
+            };
+            bool ok = mbar_wait(bar(B_Q), 0, abort, a.err);
+            for (int j = 0; j < n_steps && ok; ++j) {
+                const int sk = j % KST, sv = j % VST;
+                // S(j) once K(j) landed and the elementwise warps loaded S(j-1)
+                if (!(ok = mbar_wait(bar(B_KF(sk)), (uint32_t)(j / KST) & 1u, abort, a.err))) break;
+                if (j > 0 && !(ok = mbar_wait(bar(B_SC), (uint32_t)(j - 1) & 1u, abort, a.err))) break;
+                tc_fence_after();
+                const uint32_t ka = sbase + L::kK + sk * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(T_S, sdesc(sbase + L::kQ + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024),
+                           sdesc(ka + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024), id_ss, kk > 0);
+                tc_commit(bar(B_S));
+                // dP(j) into buffer j % 2, free once dQ(j-2) has read dS(j-2);
+                // it also waits for dS(j-1), so B_DP never completes a phase
+                // the elementwise warps have not waited for yet (a parity wait
+                // only tells the current phase from the one before it)
+                if (!(ok = mbar_wait(bar(B_VF(sv)), (uint32_t)(j / VST) & 1u, abort, a.err))) break;
+                if (j > 0 && !(ok = mbar_wait(bar(B_DS), (uint32_t)(j - 1) & 1u, abort, a.err))) break;
+                if (j > 1 && !(ok = mbar_wait(bar(B_DQ), (uint32_t)(j - 2) & 1u, abort, a.err))) break;
+                tc_fence_after();
+                const uint32_t va = sbase + L::kV + sv * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(T_DP(j), sdesc(sbase + L::kDO + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024),
+                           sdesc(va + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024), id_ss, kk > 0);
+                tc_commit(bar(B_DP));
+                tc_commit(bar(B_VE(sv)));
+                if (j > 0 && !(ok = issue_dq(j - 1))) break;
+            }
+            if (ok) ok = issue_dq(n_steps - 1);
+            tc_commit(bar(B_DRAIN));
+            for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_DRAIN), 0); ++it) {}
+        }
+    } else if (warp < 8) {
+        // ================= elementwise: 8 warps, 64 key columns each =================
+        const int half = warp >> 2, quarter = warp & 3;
+        const int r = quarter * 32 + lane;   // query row = TMEM lane
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const bool live = r < qn;
+        const int qp = q0 + r, c = qp / a.k;
+        const int64_t row = (int64_t)(c0 + c) * (a.k + 1) + qp % a.k;
+        const float lse2 = live ? a.lse[row * a.Hq + h] * 1.4426950408889634f : 0.f;
+        const float dd = live ? a.dsum[row * a.Hq + h] : 0.f;
+        const int sum_lim = live ? min(c - a.w, m) : 0;   // sees s_j for j < sum_lim
+        const int win_lo = max(0, c - a.w) * a.k;
+        const float sl2 = a.scale_log2;
+        bool ok = true;
+        for (int j = 0; j < n_steps; ++j) {
+            int lo, hi;
+            if (j < n_sum) {
+                lo = 0;
+                hi = sum_lim - j * BK;
+            } else {
+                const int kb = t_lo + (j - n_sum) * BK;
+                lo = win_lo - kb;
+                hi = live ? qp - kb + 1 : 0;
+            }
+            lo = max(lo - half * HQ, 0);
+            hi = min(hi - half * HQ, HQ);
+            if (hi < lo) hi = lo;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S), (uint32_t)j & 1u, abort, a.err));
+            if (!ok) break;
+            float p[HQ];
+            {
+                uint32_t sr[HQ];
+                tc_fence_after();
+                tmem_ld32(T_S + lane_off + half * HQ, sr);
+                tmem_ld32(T_S + lane_off + half * HQ + 32, sr + 32);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar(B_SC));   // S may be overwritten by the next step's QK
+#pragma unroll
+                for (int e = 0; e < HQ; ++e) {
+                    const float x = fmaf(__uint_as_float(sr[e]), sl2, -lse2);
+                    p[e] = (e >= lo && e < hi) ? ex2(x) : 0.f;
+                }
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DP), (uint32_t)j & 1u, abort, a.err));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t dpb = T_DP(j) + lane_off + half * HQ;
+#pragma unroll
+            for (int grp = 0; grp < 2; ++grp) {
+                uint32_t dr[32], pk[16];
+                tmem_ld32(dpb + grp * 32, dr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e2 = 0; e2 < 16; ++e2) {
+                    const int e = grp * 32 + 2 * e2;
+                    const float d0 = (e >= lo && e < hi) ? p[e] * (__uint_as_float(dr[2 * e2]) - dd) : 0.f;
+                    const float d1 = (e + 1 >= lo && e + 1 < hi) ? p[e + 1] * (__uint_as_float(dr[2 * e2 + 1]) - dd) : 0.f;
+                    pk[e2] = pack_bf16(d0, d1);
+                }
+                // dS of this half -> columns [64 half + 16 grp, +16) of its dP
+                // buffer, which this thread has already loaded
+                tmem_st16(dpb + grp * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(B_DS));
+        }
+        // ---- epilogue: dq = scale dQ -> bf16, this thread's 64 (or 32) columns ----
+        // (the drain barrier completes once, after every MMA of the CTA)
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DRAIN), 0, abort, a.err));
+        if (ok) {
+            tc_fence_after();
+            uint4 *dst = reinterpret_cast<uint4 *>(dq + (row * a.Hq + h) * D + half * (D / 2));
+#pragma unroll 1
+            for (int cc = 0; cc < D / 64; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(T_DQ + lane_off + half * (D / 2) + cc * 32, v);
+                tmem_wait_ld();
+                if (live) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int z = 0; z < 4; ++z)
+                            w4[z] = pack_bf16(__uint_as_float(v[8 * e + 2 * z]) * a.scale,
+                                              __uint_as_float(v[8 * e + 2 * z + 1]) * a.scale);
+                        dst[cc * 4 + e] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpMMA) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
 }  // namespace bt
 
 bool prefill_bwd_tc_supported(const ksa_params *p)
@@ -505,23 +811,26 @@ size_t prefill_bwd_tc_workspace_bytes(int batch, int64_t aug_rows)
 }
 
 template <int D>
-static int bt_launch(const bt::TArgs &a, int64_t grid, cudaStream_t st)
+static int bt_launch(const bt::TArgs &a, int64_t grid, int64_t grid_q, __nv_bfloat16 *dq, cudaStream_t st)
 {
     static bool attr = false;
     if (!attr) {
         if (cudaFuncSetAttribute(bt::bt_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 bt::Smem<D>::kBytes) != cudaSuccess)
+                                 bt::Smem<D>::kBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(bt::bq_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 bt::SmemQ<D>::kBytes) != cudaSuccess)
             return KSA_ERR_CUDA;
         attr = true;
     }
     bt::bt_dkv_kernel<D><<<dim3((unsigned)grid, a.Hkv), bt::kThreads, bt::Smem<D>::kBytes, st>>>(a);
+    bt::bq_dq_kernel<D><<<dim3((unsigned)grid_q, a.Hq), bt::kThreads, bt::SmemQ<D>::kBytes, st>>>(a, dq);
     return KSA_OK;
 }
 
-int launch_prefill_bwd_dkv_tc(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,
-                              const void *q, const void *k, const void *v, const void *dout, const float *lse,
-                              const float *dsum, float *dk32, float *dv32, void *ws, const Plan &pl, int32_t *err,
-                              cudaStream_t st)
+int launch_prefill_bwd_tc(const ksa_params *p, int batch, const int32_t *cu, int64_t total_text, int64_t aug_rows,
+                          const void *q, const void *k, const void *v, const void *dout, const float *lse,
+                          const float *dsum, float *dk32, float *dv32, void *dq, void *ws, const Plan &pl,
+                          int32_t *err, cudaStream_t st)
 {
     bt::TArgs a;
     const int d = p->head_dim, kk = p->k;
@@ -556,7 +865,9 @@ int launch_prefill_bwd_dkv_tc(const ksa_params *p, int batch, const int32_t *cu,
     const int64_t grid = ns_tiles * (1 + (G * q_sum) / bt::kSplit) + nt_tiles * (1 + (G * q_txt) / bt::kSplit);
     if (grid > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
     if (grid == 0) return KSA_OK;
-    const int r = d == 128 ? bt_launch<128>(a, grid, st) : bt_launch<64>(a, grid, st);
+    const int64_t grid_q = nt_tiles;   // query tiles of 128 text positions (CTAs past the real count exit)
+    __nv_bfloat16 *dqb = static_cast<__nv_bfloat16 *>(dq);
+    const int r = d == 128 ? bt_launch<128>(a, grid, grid_q, dqb, st) : bt_launch<64>(a, grid, grid_q, dqb, st);
     if (r != KSA_OK) return r;
     return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
 }

@@ -47,7 +47,8 @@ constexpr int kSplit = 32;    // steps per CTA
 constexpr int kWarpTMA = 8;   // K, V once, then Q and dO per step
 constexpr int kWarpMMA = 9;   // MMA issuer, TMEM owner
 constexpr int kWarpLD = 10;   // per-step LSE and D, zero rows past the sequence
-constexpr int kThreads = 352;
+constexpr int kWarpMMA2 = 11; // second MMA issuer (an issuing thread sustains ~70 cycles per MMA)
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
         for (int s = 0; s < QST; ++s) {
             mbar_init(bar(B_QT(s)), 1);
             mbar_init(bar(B_QF(s)), 32);
-            mbar_init(bar(B_QE(s)), 1);
+            mbar_init(bar(B_QE(s)), 2);   // one commit per issuer
         }
         mbar_init(bar(B_S), 1);
         mbar_init(bar(B_DP), 1);
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
         mbar_init(bar(B_DS), 256);
         mbar_init(bar(B_DV), 1);
         mbar_init(bar(B_DK), 1);
-        mbar_init(bar(B_DRAIN), 1);
+        mbar_init(bar(B_DRAIN), 2);   // one commit per issuer, after its last MMA
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -284,16 +285,30 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
                     }
         }
     } else if (warp == kWarpLD) {
-        // per step: wait for the tiles, zero the query rows past the sequence
-        // (they meet P = 0 and dS = 0 in the MMAs, which need them finite),
-        // then the step's LSE (log2 units) and D into shared memory
+        // per step: the step's LSE (log2 units) and D, fetched one step ahead
+        // into registers (the loads of step s + 1 are in flight while step s
+        // waits for its tiles); once the tiles have landed, zero the query
+        // rows past the sequence (they meet P = 0 and dS = 0 in the MMAs,
+        // which need them finite) and publish LSE and D in shared memory
+        constexpr int PER = BQ / 32;
+        float l2v[PER], ddv[PER];
+        auto fetch = [&](int s) {
+            const int q0 = step_q0(s), h = step_h(s), qn = min(BQ, T.n - q0);
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int r = lane + 32 * u, pos = q0 + r;
+                const int64_t row = (int64_t)(T.c0 + pos / a.k) * (a.k + 1) + pos % a.k;
+                l2v[u] = r < qn ? a.lse[row * a.Hq + h] : 0.f;
+                ddv[u] = r < qn ? a.dsum[row * a.Hq + h] : 0.f;
+            }
+        };
         bool ok = true;
+        fetch(0);
         for (int s = 0; s < n_steps && ok; ++s) {
             const int st = s % QST;
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QT(st)), (uint32_t)(s / QST) & 1u, abort, a.err));
             if (!ok) break;
-            const int q0 = step_q0(s), h = step_h(s);
-            const int qn = min(BQ, T.n - q0);
+            const int qn = min(BQ, T.n - step_q0(s));
             if (qn < BQ) {
                 const int per_row = 8 * (D / 64);   // 16-byte words of a row over both halves
                 for (int e = lane; e < (BQ - qn) * per_row; e += 32) {
@@ -305,66 +320,53 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
             float *ld = reinterpret_cast<float *>(smem + L::kLD) + st * 2 * BQ;
-            for (int r = lane; r < BQ; r += 32) {
-                float l2 = 0.f, dd = 0.f;
-                if (r < qn) {
-                    const int pos = q0 + r;
-                    const int64_t row = (int64_t)(T.c0 + pos / a.k) * (a.k + 1) + pos % a.k;
-                    l2 = a.lse[row * a.Hq + h] * 1.4426950408889634f;
-                    dd = a.dsum[row * a.Hq + h];
-                }
-                ld[r] = l2;
-                ld[BQ + r] = dd;
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                ld[lane + 32 * u] = l2v[u] * 1.4426950408889634f;
+                ld[BQ + lane + 32 * u] = ddv[u];
             }
             mbar_arrive(bar(B_QF(st)));
+            if (s + 1 < n_steps) fetch(s + 1);
         }
-    } else if (warp == kWarpMMA) {
+    } else if (warp == kWarpMMA || warp == kWarpMMA2) {
+        // Two issuers, one per chain: kWarpMMA the P side (S^T = K Q^T, then
+        // dV += P^T dO), kWarpMMA2 the dS side (dP^T = V dO^T, then
+        // dK += dS^T Q).  Each side's product columns are free again once
+        // its own accumulation of the step before has read them.
         if (lane == 0) {
+            const bool pside = warp == kWarpMMA;
             const uint32_t id_ss = idesc_f16(BK, BQ, false);
             const uint32_t id_ts = idesc_f16(BK, D, true);
+            const uint32_t T_X = pside ? T_S : T_DP, T_ACC = pside ? T_DV : T_DK;
+            const int b_x = pside ? B_S : B_DP, b_in = pside ? B_P : B_DS, b_acc = pside ? B_DV : B_DK;
+            const uint64_t dA = sdesc(sbase + (pside ? L::kK : L::kV), 16, 1024);   // SS A: K or V
             bool ok = mbar_wait(bar(B_KV), 0, abort, a.err);
             for (int s = 0; s < n_steps && ok; ++s) {
                 const int st = s % QST;
                 const uint32_t ph = (uint32_t)s & 1u, php = (uint32_t)(s - 1) & 1u;
                 if (!(ok = mbar_wait(bar(B_QF(st)), (uint32_t)(s / QST) & 1u, abort, a.err))) break;
                 const uint32_t qa = sbase + L::kQ + st * kTileBytes, da = sbase + L::kDO + st * kTileBytes;
-                // S^T = K Q^T into the S columns, free once the previous dV has read P^T
-                if (s > 0 && !(ok = mbar_wait(bar(B_DV), php, abort, a.err))) break;
+                const uint64_t dB = sdesc(pside ? qa : da, 16, 1024);      // SS B: Q or dO (K-major)
+                const uint64_t dC = sdesc(pside ? da : qa, kHalf, 1024);   // TS B: dO or Q (MN-major)
+                if (s > 0 && !(ok = mbar_wait(bar(b_acc), php, abort, a.err))) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(T_S, sdesc(sbase + L::kK + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024),
-                           sdesc(qa + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024), id_ss, kk > 0);
-                tc_commit(bar(B_S));
-                // dP^T = V dO^T, once the previous dK has read dS^T
-                if (s > 0 && !(ok = mbar_wait(bar(B_DK), php, abort, a.err))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(T_DP, sdesc(sbase + L::kV + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024),
-                           sdesc(da + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024), id_ss, kk > 0);
-                tc_commit(bar(B_DP));
-                // dV += P^T dO: half h's P^T (64 queries as bf16 pairs) sits in
-                // S columns [64h, 64h + 32) and meets dO rows [64h, 64h + 64)
-                if (!(ok = mbar_wait(bar(B_P), ph, abort, a.err))) break;
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (uint32_t)((kk / 4) * kHalf + (kk % 4) * 32) >> 4;
+                    mma_ss(T_X, dA + off, dB + off, id_ss, kk > 0);
+                }
+                tc_commit(bar(b_x));
+                // half h's bf16 pairs sit in columns [64h, 64h + 32) of S^T / dP^T
+                // and meet rows [64h, 64h + 64) of dO / Q
+                if (!(ok = mbar_wait(bar(b_in), ph, abort, a.err))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int kk = 0; kk < HQ / 16; ++kk)
-                        mma_ts(T_DV, T_S + h * HQ + kk * 8, sdesc(da + (h * (HQ / 16) + kk) * 2048, kHalf, 1024), id_ts,
+                        mma_ts(T_ACC, T_X + h * HQ + kk * 8, dC + (uint32_t)(((h * (HQ / 16) + kk) * 2048) >> 4), id_ts,
                                (s > 0 || h > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(bar(B_DV));
-                // dK += dS^T Q
-                if (!(ok = mbar_wait(bar(B_DS), ph, abort, a.err))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int kk = 0; kk < HQ / 16; ++kk)
-                        mma_ts(T_DK, T_DP + h * HQ + kk * 8, sdesc(qa + (h * (HQ / 16) + kk) * 2048, kHalf, 1024),
-                               id_ts, (s > 0 || h > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(bar(B_DK));
+                tc_commit(bar(b_acc));
                 tc_commit(bar(B_QE(st)));
             }
             tc_commit(bar(B_DRAIN));
@@ -397,6 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
             lo = max(lo - half * HQ, 0);
             hi = min(hi - half * HQ, HQ);
             if (hi < lo) hi = lo;
+            // every column of this half visible to every row of the warp: no mask
+            const bool full = __all_sync(0xffffffffu, lo == 0 && hi == HQ);
             ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(B_QF(st)), (uint32_t)(s / QST) & 1u, abort, a.err));
             ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(B_S), ph, abort, a.err));
             if (!ok) break;
@@ -409,10 +413,15 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
                 tmem_ld32(T_S + lane_off + half * HQ, sr);
                 tmem_ld32(T_S + lane_off + half * HQ + 32, sr + 32);
                 tmem_wait_ld();
+                if (full) {
 #pragma unroll
-                for (int e = 0; e < HQ; ++e) {
-                    const float x = fmaf(__uint_as_float(sr[e]), sl2, -l2[e]);
-                    p[e] = (e >= lo && e < hi) ? ex2(x) : 0.f;
+                    for (int e = 0; e < HQ; ++e) p[e] = ex2(fmaf(__uint_as_float(sr[e]), sl2, -l2[e]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < HQ; ++e) {
+                        const float x = fmaf(__uint_as_float(sr[e]), sl2, -l2[e]);
+                        p[e] = (e >= lo && e < hi) ? ex2(x) : 0.f;
+                    }
                 }
 #pragma unroll
                 for (int grp = 0; grp < 2; ++grp) {
@@ -434,10 +443,15 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
                 tmem_ld32(T_DP + lane_off + half * HQ + grp * 32, dr);
                 tmem_wait_ld();
                 float ds[32];
+                if (full) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = grp * 32 + e;
-                    ds[e] = (c >= lo && c < hi) ? p[c] * (__uint_as_float(dr[e]) - dd[c]) : 0.f;
+                    for (int e = 0; e < 32; ++e) ds[e] = p[grp * 32 + e] * (__uint_as_float(dr[e]) - dd[grp * 32 + e]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int c = grp * 32 + e;
+                        ds[e] = (c >= lo && c < hi) ? p[c] * (__uint_as_float(dr[e]) - dd[c]) : 0.f;
+                    }
                 }
 #pragma unroll
                 for (int e2 = 0; e2 < 16; ++e2) pk[e2] = pack_bf16(ds[2 * e2], ds[2 * e2 + 1]);
@@ -450,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
             mbar_arrive(bar(B_DS));
         }
         // ---- epilogue: dK (scaled) and dV rows into the fp32 accumulators ----
-        if (ok)
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DK), (uint32_t)(n_steps - 1) & 1u, abort, a.err));
+        // (the drain barrier completes once, after every MMA of both issuers)
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DRAIN), 0, abort, a.err));
         if (ok) {
             tc_fence_after();
             const int64_t row = T.sum ? (int64_t)(T.c0 + key) * (a.k + 1) + a.k
@@ -577,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constan
         mbar_init(bar(B_DP), 1);
         mbar_init(bar(B_DS), 256);
         mbar_init(bar(B_DQ), 1);
-        mbar_init(bar(B_DRAIN), 1);
+        mbar_init(bar(B_DRAIN), 2);   // one commit per issuer, after its last MMA
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -639,57 +653,73 @@ __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constan
                     }
             }
         }
-    } else if (warp == kWarpMMA) {
+    } else if (warp == kWarpMMA || warp == kWarpMMA2) {
+        // Two issuers: kWarpMMA issues S(j) = Q K(j)^T as soon as K(j) has
+        // landed and the elementwise warps have loaded S(j-1); kWarpMMA2
+        // issues dP(j) = dO V(j)^T and dQ += dS(j-1) K(j-1).
         if (lane == 0) {
             const uint32_t id_ss = idesc_f16(BK, BK, false);
             const uint32_t id_ts = idesc_f16(BK, D, true);
-            // dQ(j) = dS(j) K(j): dS(j) (128 keys as bf16 pairs) sits in
-            // dP buffer j % 2, columns [64h, 64h + 32) for key half h
-            auto issue_dq = [&](int j) -> bool {
-                if (!mbar_wait(bar(B_DS), (uint32_t)j & 1u, abort, a.err)) return false;
-                tc_fence_after();
-                const uint32_t ka = sbase + L::kK + (j % KST) * kTileBytes;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                    for (int kk = 0; kk < HQ / 16; ++kk)
-                        mma_ts(T_DQ, T_DP(j) + hh * HQ + kk * 8, sdesc(ka + (hh * (HQ / 16) + kk) * 2048, kHalf, 1024),
-                               id_ts, (j > 0 || hh > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(bar(B_DQ));
-                tc_commit(bar(B_KE(j % KST)));
-                return true;
-            };
             bool ok = mbar_wait(bar(B_Q), 0, abort, a.err);
-            for (int j = 0; j < n_steps && ok; ++j) {
-                const int sk = j % KST, sv = j % VST;
-                // S(j) once K(j) landed and the elementwise warps loaded S(j-1)
-                if (!(ok = mbar_wait(bar(B_KF(sk)), (uint32_t)(j / KST) & 1u, abort, a.err))) break;
-                if (j > 0 && !(ok = mbar_wait(bar(B_SC), (uint32_t)(j - 1) & 1u, abort, a.err))) break;
-                tc_fence_after();
-                const uint32_t ka = sbase + L::kK + sk * kTileBytes;
+            if (warp == kWarpMMA) {
+                const uint64_t dQd = sdesc(sbase + L::kQ, 16, 1024);
+                for (int j = 0; j < n_steps && ok; ++j) {
+                    const int sk = j % KST;
+                    if (!(ok = mbar_wait(bar(B_KF(sk)), (uint32_t)(j / KST) & 1u, abort, a.err))) break;
+                    if (j > 0 && !(ok = mbar_wait(bar(B_SC), (uint32_t)(j - 1) & 1u, abort, a.err))) break;
+                    tc_fence_after();
+                    const uint64_t dKd = sdesc(sbase + L::kK + sk * kTileBytes, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(T_S, sdesc(sbase + L::kQ + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024),
-                           sdesc(ka + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024), id_ss, kk > 0);
-                tc_commit(bar(B_S));
-                // dP(j) into buffer j % 2, free once dQ(j-2) has read dS(j-2);
-                // it also waits for dS(j-1), so B_DP never completes a phase
-                // the elementwise warps have not waited for yet (a parity wait
-                // only tells the current phase from the one before it)
-                if (!(ok = mbar_wait(bar(B_VF(sv)), (uint32_t)(j / VST) & 1u, abort, a.err))) break;
-                if (j > 0 && !(ok = mbar_wait(bar(B_DS), (uint32_t)(j - 1) & 1u, abort, a.err))) break;
-                if (j > 1 && !(ok = mbar_wait(bar(B_DQ), (uint32_t)(j - 2) & 1u, abort, a.err))) break;
-                tc_fence_after();
-                const uint32_t va = sbase + L::kV + sv * kTileBytes;
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (uint32_t)((kk / 4) * kHalf + (kk % 4) * 32) >> 4;
+                        mma_ss(T_S, dQd + off, dKd + off, id_ss, kk > 0);
+                    }
+                    tc_commit(bar(B_S));
+                }
+            } else {
+                const uint64_t dOd = sdesc(sbase + L::kDO, 16, 1024);
+                // dQ(j) = dS(j) K(j): dS(j) (128 keys as bf16 pairs) sits in
+                // dP buffer j % 2, columns [64h, 64h + 32) for key half h.  K(j)'s
+                // stage is released here; S(j) read it before dS(j) existed.
+                // Inside the loop dS(j) was waited for just before dP(j+1); a
+                // second parity wait there could miss the phase if dS(j+1)
+                // completed in between, so only the last step waits here.
+                auto issue_dq = [&](int j, bool wait_ds) -> bool {
+                    if (wait_ds && !mbar_wait(bar(B_DS), (uint32_t)j & 1u, abort, a.err)) return false;
+                    tc_fence_after();
+                    const uint64_t dKm = sdesc(sbase + L::kK + (j % KST) * kTileBytes, kHalf, 1024);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(T_DP(j), sdesc(sbase + L::kDO + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024),
-                           sdesc(va + (kk / 4) * kHalf + (kk % 4) * 32, 16, 1024), id_ss, kk > 0);
-                tc_commit(bar(B_DP));
-                tc_commit(bar(B_VE(sv)));
-                if (j > 0 && !(ok = issue_dq(j - 1))) break;
+                    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                        for (int kk = 0; kk < HQ / 16; ++kk)
+                            mma_ts(T_DQ, T_DP(j) + hh * HQ + kk * 8, dKm + (uint32_t)(((hh * (HQ / 16) + kk) * 2048) >> 4),
+                                   id_ts, (j > 0 || hh > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(bar(B_DQ));
+                    tc_commit(bar(B_KE(j % KST)));
+                    return true;
+                };
+                for (int j = 0; j < n_steps && ok; ++j) {
+                    const int sv = j % VST;
+                    // dP(j) into buffer j % 2, free once dQ(j-2) has read dS(j-2);
+                    // it also waits for dS(j-1), so B_DP never completes a phase
+                    // the elementwise warps have not waited for yet (a parity wait
+                    // only tells the current phase from the one before it)
+                    if (!(ok = mbar_wait(bar(B_VF(sv)), (uint32_t)(j / VST) & 1u, abort, a.err))) break;
+                    if (j > 0 && !(ok = mbar_wait(bar(B_DS), (uint32_t)(j - 1) & 1u, abort, a.err))) break;
+                    if (j > 1 && !(ok = mbar_wait(bar(B_DQ), (uint32_t)(j - 2) & 1u, abort, a.err))) break;
+                    tc_fence_after();
+                    const uint64_t dVd = sdesc(sbase + L::kV + sv * kTileBytes, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (uint32_t)((kk / 4) * kHalf + (kk % 4) * 32) >> 4;
+                        mma_ss(T_DP(j), dOd + off, dVd + off, id_ss, kk > 0);
+                    }
+                    tc_commit(bar(B_DP));
+                    tc_commit(bar(B_VE(sv)));
+                    if (j > 0 && !(ok = issue_dq(j - 1, false))) break;
+                }
+                if (ok) ok = issue_dq(n_steps - 1, true);
             }
-            if (ok) ok = issue_dq(n_steps - 1);
             tc_commit(bar(B_DRAIN));
             for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_DRAIN), 0); ++it) {}
         }
@@ -720,6 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constan
             lo = max(lo - half * HQ, 0);
             hi = min(hi - half * HQ, HQ);
             if (hi < lo) hi = lo;
+            const bool full = __all_sync(0xffffffffu, lo == 0 && hi == HQ);
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S), (uint32_t)j & 1u, abort, a.err));
             if (!ok) break;
             float p[HQ];
@@ -731,10 +762,15 @@ __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constan
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(bar(B_SC));   // S may be overwritten by the next step's QK
+                if (full) {
 #pragma unroll
-                for (int e = 0; e < HQ; ++e) {
-                    const float x = fmaf(__uint_as_float(sr[e]), sl2, -lse2);
-                    p[e] = (e >= lo && e < hi) ? ex2(x) : 0.f;
+                    for (int e = 0; e < HQ; ++e) p[e] = ex2(fmaf(__uint_as_float(sr[e]), sl2, -lse2));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < HQ; ++e) {
+                        const float x = fmaf(__uint_as_float(sr[e]), sl2, -lse2);
+                        p[e] = (e >= lo && e < hi) ? ex2(x) : 0.f;
+                    }
                 }
             }
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DP), (uint32_t)j & 1u, abort, a.err));
@@ -746,12 +782,22 @@ __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constan
                 uint32_t dr[32], pk[16];
                 tmem_ld32(dpb + grp * 32, dr);
                 tmem_wait_ld();
+                if (full) {
 #pragma unroll
-                for (int e2 = 0; e2 < 16; ++e2) {
-                    const int e = grp * 32 + 2 * e2;
-                    const float d0 = (e >= lo && e < hi) ? p[e] * (__uint_as_float(dr[2 * e2]) - dd) : 0.f;
-                    const float d1 = (e + 1 >= lo && e + 1 < hi) ? p[e + 1] * (__uint_as_float(dr[2 * e2 + 1]) - dd) : 0.f;
-                    pk[e2] = pack_bf16(d0, d1);
+                    for (int e2 = 0; e2 < 16; ++e2) {
+                        const int e = grp * 32 + 2 * e2;
+                        pk[e2] = pack_bf16(p[e] * (__uint_as_float(dr[2 * e2]) - dd),
+                                           p[e + 1] * (__uint_as_float(dr[2 * e2 + 1]) - dd));
+                    }
+                } else {
+#pragma unroll
+                    for (int e2 = 0; e2 < 16; ++e2) {
+                        const int e = grp * 32 + 2 * e2;
+                        const float d0 = (e >= lo && e < hi) ? p[e] * (__uint_as_float(dr[2 * e2]) - dd) : 0.f;
+                        const float d1 =
+                            (e + 1 >= lo && e + 1 < hi) ? p[e + 1] * (__uint_as_float(dr[2 * e2 + 1]) - dd) : 0.f;
+                        pk[e2] = pack_bf16(d0, d1);
+                    }
                 }
                 // dS of this half -> columns [64 half + 16 grp, +16) of its dP
                 // buffer, which this thread has already loaded

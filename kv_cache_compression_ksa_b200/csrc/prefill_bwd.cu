@@ -53,8 +53,6 @@ struct Args {
     float *dsum;                      // [rows, Hq] D = rowsum(dO * O)
     float *dk32, *dv32;               // [rows, Hkv, d] fp32 accumulators of the split dk/dv pass
     int nblk;                         // upper bound of the block count (grid x)
-    int sumq_only;                    // only the summary query rows (the text rows run on tcgen05):
-                                      // dk/dv from them, and dq of them
     __nv_bfloat16 *dq, *dk, *dv;
 };
 
@@ -177,8 +175,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(Args a)
     // text blocks late in a sequence see the most summaries: reverse order
     // puts them first
     const int nreal = a.tb_off[a.batch] + a.sb_off[a.batch];
-    const int id = a.sumq_only ? a.tb_off[a.batch] + (int)blockIdx.x
-                               : ((int)blockIdx.x < nreal ? nreal - 1 - (int)blockIdx.x : (int)blockIdx.x);
+    const int id = (int)blockIdx.x < nreal ? nreal - 1 - (int)blockIdx.x : (int)blockIdx.x;
     if (!block_of(a, id, Q)) return;
     const int h = blockIdx.y, g = h / a.G;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, tt = lane & 3;
@@ -389,7 +386,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
         s_lo = K.idx0;
         s_hi = K.idx0 + K.cnt;
     }
-    const int ntb = a.sumq_only ? 0 : (t_hi - t_lo + RB - 1) / RB;
+    const int ntb = (t_hi - t_lo + RB - 1) / RB;
     const int nsb = s_hi > s_lo ? 1 : 0;   // at most 64 summaries see this block's keys
     // this CTA's share of the query blocks (split z of ceil((ntb + nsb) / QB_SPLIT))
     const int qb_lo = (int)blockIdx.z * QB_SPLIT, qb_hi = min(ntb + nsb, qb_lo + QB_SPLIT);
@@ -537,6 +534,121 @@ __global__ void __launch_bounds__(256) bwd_dkv_out_kernel(Args a, int D)
     }
 }
 
+// The summary query rows of the tensor-core path and the output conversion,
+// fused: one warp per (chunk, kv head).  Summary s_j (section 2.2.1, Figure
+// 4c) attends to the k text rows of chunk j and to itself, i.e. exactly the
+// k + 1 rows of the chunk; its G q heads give P and dS over those rows
+// (CUDA cores, warp-wide dot products), dq of s_j = scale dS K, and the rows'
+// dk += scale dS^T q_sj, dv += P^T dO_sj are added to the fp32 accumulators
+// of the text query rows as they are converted to bf16.  Lane l holds
+// columns [D/32 l, D/32 (l + 1)).  sm: [4 warps][P, dS][G][k + 1] floats.
+template <int D>
+__global__ void __launch_bounds__(128) bwd_sum_rows_kernel(Args a, int64_t chunks)
+{
+    constexpr int CPL = D / 32;
+    extern __shared__ float bw_sum_sm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t gc = (int64_t)blockIdx.x * 4 + warp;
+    if (*a.err != 0 || gc >= chunks) return;   // warp-uniform; only warp-level syncs below
+    const int g = blockIdx.y, K1 = a.k + 1, G = a.G;
+    float *sP = bw_sum_sm + (size_t)warp * 2 * G * K1, *sS = sP + G * K1;
+    const int b = find_seq(a.pl.chunk_off, a.batch, (int)gc);
+    const int j = (int)(gc - a.pl.chunk_off[b]);
+    const int n = a.cu[b + 1] - a.cu[b], m = n / a.k;
+    if (j * a.k >= n) return;                  // past the sequence (a padding chunk cannot occur)
+    const bool has_sum = j < m;
+    const int64_t row0 = gc * K1, srow = row0 + a.k;
+    const int col0 = lane * CPL;
+    auto ld = [&](const __nv_bfloat16 *p, float *f) {
+        if constexpr (CPL == 4) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(p);
+            f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
+            f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
+        } else {
+            const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
+            f[0] = __uint_as_float(u << 16); f[1] = __uint_as_float(u & 0xffff0000u);
+        }
+    };
+    auto st = [&](__nv_bfloat16 *p, const float *f) {
+        if constexpr (CPL == 4)
+            *reinterpret_cast<uint2 *>(p) = make_uint2(wm::pack2(f[0], f[1]), wm::pack2(f[2], f[3]));
+        else
+            *reinterpret_cast<uint32_t *>(p) = wm::pack2(f[0], f[1]);
+    };
+    if (has_sum) {
+        for (int r = 0; r < K1; ++r) {
+            float kr[CPL], vr[CPL];
+            ld(a.kk + ((row0 + r) * a.Hkv + g) * D + col0, kr);
+            ld(a.v + ((row0 + r) * a.Hkv + g) * D + col0, vr);
+            for (int hh = 0; hh < G; ++hh) {
+                const int h = g * G + hh;
+                float qv[CPL], ov[CPL];
+                ld(a.q + (srow * a.Hq + h) * D + col0, qv);
+                ld(a.dout + (srow * a.Hq + h) * D + col0, ov);
+                float sc = 0.f, dp = 0.f;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    sc = fmaf(qv[c], kr[c], sc);
+                    dp = fmaf(ov[c], vr[c], dp);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    sc += __shfl_xor_sync(0xffffffffu, sc, off);
+                    dp += __shfl_xor_sync(0xffffffffu, dp, off);
+                }
+                const float pr = wm::ex2(sc * a.scale_log2 - a.lse[srow * a.Hq + h] * 1.4426950408889634f);
+                if (lane == 0) {
+                    sP[hh * K1 + r] = pr;
+                    sS[hh * K1 + r] = pr * (dp - a.dsum[srow * a.Hq + h]);
+                }
+            }
+        }
+        __syncwarp();
+        // dq of s_j, head by head
+        for (int hh = 0; hh < G; ++hh) {
+            float acc[CPL] = {};
+            for (int r = 0; r < K1; ++r) {
+                float kr[CPL];
+                ld(a.kk + ((row0 + r) * a.Hkv + g) * D + col0, kr);
+                const float w = sS[hh * K1 + r];
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) acc[c] = fmaf(w, kr[c], acc[c]);
+            }
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) acc[c] *= a.scale;
+            st(a.dq + (srow * a.Hq + g * G + hh) * D + col0, acc);
+        }
+    }
+    // dk, dv of the chunk's real rows: its text rows, then s_j
+    const int ntext = min(a.k, n - j * a.k);
+    for (int r = 0; r < K1; ++r) {
+        if (r < a.k ? r >= ntext : !has_sum) continue;
+        const int64_t off = ((row0 + r) * a.Hkv + g) * D + col0;
+        float dk[CPL], dv[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            dk[c] = a.dk32[off + c];
+            dv[c] = a.dv32[off + c];
+        }
+        if (has_sum) {
+            for (int hh = 0; hh < G; ++hh) {
+                const int h = g * G + hh;
+                float qv[CPL], ov[CPL];
+                ld(a.q + (srow * a.Hq + h) * D + col0, qv);
+                ld(a.dout + (srow * a.Hq + h) * D + col0, ov);
+                const float ws = sS[hh * K1 + r] * a.scale, wp = sP[hh * K1 + r];
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    dk[c] = fmaf(ws, qv[c], dk[c]);
+                    dv[c] = fmaf(wp, ov[c], dv[c]);
+                }
+            }
+        }
+        st(a.dk + off, dk);
+        st(a.dv + off, dv);
+    }
+}
+
 // per-sequence block counts: text blocks ceil(n/64), summary blocks ceil(m/64)
 __global__ void bwd_blocks_kernel(int batch, const int32_t *cu, int k, int32_t *tb_off, int32_t *sb_off)
 {
@@ -556,8 +668,26 @@ __global__ void bwd_blocks_kernel(int batch, const int32_t *cu, int k, int32_t *
 }  // namespace bw
 
 // four 64-row tiles of D + 8 bf16 per row (+ per-query LSE and D for dk, dv)
+// Summary query rows and the output conversion after the tensor-core kernels.
 template <int D>
-static int bw_launch(const bw::Args &a, int64_t nblk, int64_t nblk_dq, int64_t zsplits, cudaStream_t st)
+static int bw_sum_launch(const bw::Args &a, int64_t chunks, cudaStream_t st)
+{
+    const size_t smem = (size_t)4 * 2 * a.G * (a.k + 1) * sizeof(float);
+    if (smem > 48 * 1024) {
+        static size_t attr = 0;
+        if (smem > attr) {
+            if (cudaFuncSetAttribute(bw::bwd_sum_rows_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem) != cudaSuccess)
+                return KSA_ERR_UNSUPPORTED;
+            attr = smem;
+        }
+    }
+    bw::bwd_sum_rows_kernel<D><<<dim3((unsigned)((chunks + 3) / 4), a.Hkv), 128, smem, st>>>(a, chunks);
+    return KSA_OK;
+}
+
+template <int D>
+static int bw_launch(const bw::Args &a, int64_t nblk, int64_t zsplits, cudaStream_t st)
 {
     const int tiles = 6 * bw::RB * (D + 8) * 2;              // Q, dO + two (K, V) / K, V + two (Q, dO)
     const int dkv = tiles + 2 * 2 * bw::RB * 4;               // + two (LSE, D)
@@ -569,7 +699,7 @@ static int bw_launch(const bw::Args &a, int64_t nblk, int64_t nblk_dq, int64_t z
             return KSA_ERR_CUDA;
         attr[D == 128] = true;
     }
-    if (nblk_dq > 0) bw::bwd_dq_kernel<D><<<dim3((unsigned)nblk_dq, a.Hq), bw::kThreads, tiles, st>>>(a);
+    bw::bwd_dq_kernel<D><<<dim3((unsigned)nblk, a.Hq), bw::kThreads, tiles, st>>>(a);
     bw::bwd_dkv_kernel<D><<<dim3((unsigned)nblk, a.Hkv, (unsigned)zsplits), bw::kThreads, dkv, st>>>(a);
     bw::bwd_dkv_out_kernel<<<dim3((unsigned)nblk, a.Hkv), 256, 0, st>>>(a, D);
     return KSA_OK;
@@ -615,24 +745,24 @@ int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_
     if (nblk > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
     a.nblk = (int)nblk;
     // query blocks any key block can meet: at most total_text/64 + 2 (text + one summary block)
-    int64_t zsplits = (total_text / bw::RB + 2 + bw::QB_SPLIT - 1) / bw::QB_SPLIT;
+    const int64_t zsplits = (total_text / bw::RB + 2 + bw::QB_SPLIT - 1) / bw::QB_SPLIT;
     if (zsplits > 65535) return KSA_ERR_UNSUPPORTED;
     // dq, dk, dv of the text query rows on the tensor-core kernels where the
-    // shape allows; the warp-level passes then only take the summary rows
-    a.sumq_only = 0;
-    int64_t nblk_dq = nblk;
+    // shape allows, then the summary query rows fused with the conversion;
+    // otherwise the warp-level passes take every row
     if (prefill_bwd_tc_supported(p)) {
         const int r = launch_prefill_bwd_tc(p, batch, cu, total_text, aug_rows, q, k, v, dout, lse, a.dsum, a.dk32,
                                             a.dv32, dq, w + 2 * ab + dsb + 2 * accb, pl, err, st);
         if (r != KSA_OK) return r;
-        a.sumq_only = 1;
-        zsplits = 1;
-        nblk_dq = (total_text / p->k) / bw::RB + batch;   // summary query blocks only
+        const int64_t chunks = aug_rows / (p->k + 1);
+        const int rs = p->head_dim == 128 ? bw_sum_launch<128>(a, chunks, st) : bw_sum_launch<64>(a, chunks, st);
+        if (rs != KSA_OK) return rs;
+        return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
     }
     if (p->head_dim == 128) {
-        if (bw_launch<128>(a, nblk, nblk_dq, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
+        if (bw_launch<128>(a, nblk, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
     } else if (p->head_dim == 64) {
-        if (bw_launch<64>(a, nblk, nblk_dq, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
+        if (bw_launch<64>(a, nblk, zsplits, st) != KSA_OK) return KSA_ERR_CUDA;
     } else {
         return KSA_ERR_UNSUPPORTED;
     }

@@ -650,7 +650,8 @@ def run_sweep(args):
     tf = flops / (ms * 1e-3) / 1e12
     print(json.dumps({"sweep": "prefill_bwd", "workload": "1x32768, 32q/8kv, d128, k8, w8, N(0,1)*0.5 bf16",
                       "useful_tflop": flops / 1e12, "ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / tc_peak,
-                      "note": "warp-level mma.sync kernels; S and dP are computed in both the dq and the dk/dv pass"}),
+                      "note": "tcgen05 kernels for the text query rows (dk/dv key-stationary, dq query-stationary: "
+                              "S and dP are computed in both), summary query rows on CUDA cores"}),
           flush=True)
     del x, qa, ka, va, oa, lse, ws, do, dq, dk, dv, wsb
     torch.cuda.empty_cache()

@@ -155,9 +155,10 @@ KSA_API int ksa_prefill_fwd(const ksa_params *p, int32_t batch, const int32_t *c
                     void *stream);
 
 /* Workspace bytes for ksa_prefill_bwd: the batch plan, block offsets, an
- * fp32 [aug_rows, Hq] buffer for rowsum(dO * O) and fp32 [aug_rows, Hkv, d]
- * accumulators for dk and dv (a key block's query range is split over
- * several CTAs that add their shares). */
+ * fp32 [aug_rows, Hq] buffer for rowsum(dO * O), fp32 [aug_rows, Hkv, d]
+ * accumulators for dk and dv (a key tile's query range is split over
+ * several CTAs that add their shares) and the key-tile work list of the
+ * tensor-core kernels. */
 KSA_API size_t ksa_prefill_bwd_workspace_size(const ksa_params *p, int32_t batch, int64_t aug_rows);
 
 /* KSA prefill backward: gradients of Eq. (10) under the KSA mask (sections
@@ -167,9 +168,16 @@ KSA_API size_t ksa_prefill_bwd_workspace_size(const ksa_params *p, int32_t batch
  * bf16: the gradient of the loss with respect to o_aug.  Writes
  * dq_aug [aug_rows, Hq, d], dk_aug / dv_aug [aug_rows, Hkv, d] (bf16) for
  * every real row (text and summary); padding rows are not written.  dk and
- * dv sum over the q heads that share a kv head.  Runs on the warp-level
- * tensor-core MMA, skipping the key/query block pairs the rule masks out
- * entirely.  dev_err and cu_seqlens as for ksa_prefill_fwd. */
+ * dv sum over the q heads that share a kv head.  The text query rows run on
+ * the tcgen05 tensor cores (dk, dv key-stationary over 128-key tiles; dq
+ * query-stationary over 128-query tiles), skipping every tile pair the rule
+ * masks out entirely; the summary query rows (k+1 keys each) run on CUDA
+ * cores, fused with the conversion of the fp32 accumulators.  Shapes with
+ * 128 % k != 0 or d not in {64, 128} run every row on the warp-level MMA.
+ * The padding rows of k_aug and v_aug must hold finite values (as
+ * ksa_interleave_rope leaves them: zeros); those of q_aug and do_aug are
+ * never read into a result.  dev_err and cu_seqlens as for
+ * ksa_prefill_fwd. */
 KSA_API int ksa_prefill_bwd(const ksa_params *p, int32_t batch, const int32_t *cu_seqlens,
                     int64_t total_text, int64_t aug_rows,
                     const void *q_aug, const void *k_aug, const void *v_aug,

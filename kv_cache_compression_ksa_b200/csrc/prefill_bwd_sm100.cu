@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
             }
             for (int s = 0; s < n_steps; ++s) {
                 const int st = s % QST;
-                if (s >= QST && !(ok = mbar_wait(bar(B_QE(st)), (uint32_t)((s / QST) - 1) & 1u, abort, a.err)))
+                if (s >= QST && !(ok = mbar_wait_sleep(bar(B_QE(st)), (uint32_t)((s / QST) - 1) & 1u, abort, a.err)))
                     break;
                 const int chunk = T.c0 + step_q0(s) / a.k, h = step_h(s);
                 mbar_expect_tx(bar(B_QT(st)), 2 * kTileBytes);
@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
         fetch(0);
         for (int s = 0; s < n_steps && ok; ++s) {
             const int st = s % QST;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QT(st)), (uint32_t)(s / QST) & 1u, abort, a.err));
+            ok = __all_sync(0xffffffffu, mbar_wait_sleep(bar(B_QT(st)), (uint32_t)(s / QST) & 1u, abort, a.err));
             if (!ok) break;
             const int qn = min(BQ, T.n - step_q0(s));
             if (qn < BQ) {
@@ -340,15 +340,15 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
             const uint32_t T_X = pside ? T_S : T_DP, T_ACC = pside ? T_DV : T_DK;
             const int b_x = pside ? B_S : B_DP, b_in = pside ? B_P : B_DS, b_acc = pside ? B_DV : B_DK;
             const uint64_t dA = sdesc(sbase + (pside ? L::kK : L::kV), 16, 1024);   // SS A: K or V
-            bool ok = mbar_wait(bar(B_KV), 0, abort, a.err);
+            bool ok = mbar_wait_sleep(bar(B_KV), 0, abort, a.err);
             for (int s = 0; s < n_steps && ok; ++s) {
                 const int st = s % QST;
                 const uint32_t ph = (uint32_t)s & 1u, php = (uint32_t)(s - 1) & 1u;
-                if (!(ok = mbar_wait(bar(B_QF(st)), (uint32_t)(s / QST) & 1u, abort, a.err))) break;
+                if (!(ok = mbar_wait_sleep(bar(B_QF(st)), (uint32_t)(s / QST) & 1u, abort, a.err))) break;
                 const uint32_t qa = sbase + L::kQ + st * kTileBytes, da = sbase + L::kDO + st * kTileBytes;
                 const uint64_t dB = sdesc(pside ? qa : da, 16, 1024);      // SS B: Q or dO (K-major)
                 const uint64_t dC = sdesc(pside ? da : qa, kHalf, 1024);   // TS B: dO or Q (MN-major)
-                if (s > 0 && !(ok = mbar_wait(bar(b_acc), php, abort, a.err))) break;
+                if (s > 0 && !(ok = mbar_wait_sleep(bar(b_acc), php, abort, a.err))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
                 tc_commit(bar(b_x));
                 // half h's bf16 pairs sit in columns [64h, 64h + 32) of S^T / dP^T
                 // and meet rows [64h, 64h + 64) of dO / Q
-                if (!(ok = mbar_wait(bar(b_in), ph, abort, a.err))) break;
+                if (!(ok = mbar_wait_sleep(bar(b_in), ph, abort, a.err))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
@@ -626,13 +626,13 @@ __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constan
                 const int c3 = sum ? c0 + j * BK : c0 + (t_lo + (j - n_sum) * BK) / a.k;
                 const CUtensorMap *mk = sum ? &a.tm_ks : &a.tm_kt, *mv = sum ? &a.tm_vs : &a.tm_vt;
                 const int sk = j % KST, sv = j % VST;
-                if (j >= KST && !(ok = mbar_wait(bar(B_KE(sk)), (uint32_t)((j / KST) - 1) & 1u, abort, a.err)))
+                if (j >= KST && !(ok = mbar_wait_sleep(bar(B_KE(sk)), (uint32_t)((j / KST) - 1) & 1u, abort, a.err)))
                     break;
                 mbar_expect_tx(bar(B_KF(sk)), kTileBytes);
                 for (int hf = 0; hf < D / 64; ++hf)
                     tma_load_4d(sbase + L::kK + sk * kTileBytes + hf * kHalf, mk, bar(B_KF(sk)), hf * 64, c1, c2, c3);
                 k_issued[sk]++;
-                if (j >= VST && !(ok = mbar_wait(bar(B_VE(sv)), (uint32_t)((j / VST) - 1) & 1u, abort, a.err)))
+                if (j >= VST && !(ok = mbar_wait_sleep(bar(B_VE(sv)), (uint32_t)((j / VST) - 1) & 1u, abort, a.err)))
                     break;
                 mbar_expect_tx(bar(B_VF(sv)), kTileBytes);
                 for (int hf = 0; hf < D / 64; ++hf)
@@ -660,13 +660,13 @@ __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constan
         if (lane == 0) {
             const uint32_t id_ss = idesc_f16(BK, BK, false);
             const uint32_t id_ts = idesc_f16(BK, D, true);
-            bool ok = mbar_wait(bar(B_Q), 0, abort, a.err);
+            bool ok = mbar_wait_sleep(bar(B_Q), 0, abort, a.err);
             if (warp == kWarpMMA) {
                 const uint64_t dQd = sdesc(sbase + L::kQ, 16, 1024);
                 for (int j = 0; j < n_steps && ok; ++j) {
                     const int sk = j % KST;
-                    if (!(ok = mbar_wait(bar(B_KF(sk)), (uint32_t)(j / KST) & 1u, abort, a.err))) break;
-                    if (j > 0 && !(ok = mbar_wait(bar(B_SC), (uint32_t)(j - 1) & 1u, abort, a.err))) break;
+                    if (!(ok = mbar_wait_sleep(bar(B_KF(sk)), (uint32_t)(j / KST) & 1u, abort, a.err))) break;
+                    if (j > 0 && !(ok = mbar_wait_sleep(bar(B_SC), (uint32_t)(j - 1) & 1u, abort, a.err))) break;
                     tc_fence_after();
                     const uint64_t dKd = sdesc(sbase + L::kK + sk * kTileBytes, 16, 1024);
 #pragma unroll
@@ -685,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constan
                 // second parity wait there could miss the phase if dS(j+1)
                 // completed in between, so only the last step waits here.
                 auto issue_dq = [&](int j, bool wait_ds) -> bool {
-                    if (wait_ds && !mbar_wait(bar(B_DS), (uint32_t)j & 1u, abort, a.err)) return false;
+                    if (wait_ds && !mbar_wait_sleep(bar(B_DS), (uint32_t)j & 1u, abort, a.err)) return false;
                     tc_fence_after();
                     const uint64_t dKm = sdesc(sbase + L::kK + (j % KST) * kTileBytes, kHalf, 1024);
 #pragma unroll
@@ -704,9 +704,9 @@ __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constan
                     // it also waits for dS(j-1), so B_DP never completes a phase
                     // the elementwise warps have not waited for yet (a parity wait
                     // only tells the current phase from the one before it)
-                    if (!(ok = mbar_wait(bar(B_VF(sv)), (uint32_t)(j / VST) & 1u, abort, a.err))) break;
-                    if (j > 0 && !(ok = mbar_wait(bar(B_DS), (uint32_t)(j - 1) & 1u, abort, a.err))) break;
-                    if (j > 1 && !(ok = mbar_wait(bar(B_DQ), (uint32_t)(j - 2) & 1u, abort, a.err))) break;
+                    if (!(ok = mbar_wait_sleep(bar(B_VF(sv)), (uint32_t)(j / VST) & 1u, abort, a.err))) break;
+                    if (j > 0 && !(ok = mbar_wait_sleep(bar(B_DS), (uint32_t)(j - 1) & 1u, abort, a.err))) break;
+                    if (j > 1 && !(ok = mbar_wait_sleep(bar(B_DQ), (uint32_t)(j - 2) & 1u, abort, a.err))) break;
                     tc_fence_after();
                     const uint64_t dVd = sdesc(sbase + L::kV + sv * kTileBytes, 16, 1024);
 #pragma unroll

@@ -13,7 +13,13 @@
 namespace ksa {
 namespace tc {
 
-constexpr uint32_t kSpinLimit = 1u << 22;  // bounded waits (~0.5-4 s)
+constexpr uint32_t kSpinLimit = 1u << 22;  // bounded polls of the drain loops (~0.5-4 s)
+// mbar_wait sleeps in mbarrier.try_wait until the phase completes, at most
+// kSuspendNs per call, and gives up after kWaitLimit calls (~2.6 s).  A
+// waiting warp that instead polls takes issue slots from the compute warps
+// of its SM sub-partition.
+constexpr uint32_t kSuspendNs = 20000;
+constexpr uint32_t kWaitLimit = 1u << 17;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -49,8 +55,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait: false (after flagging the CTA and the error word) if the
-// phase did not complete within kSpinLimit polls or another role aborted.
+// try_wait that suspends the thread until the phase completes or kSuspendNs
+// have passed
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
@@ -64,12 +83,30 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Bounded waits: false (after flagging the CTA and the error word) if the
+// phase did not complete in time or another role aborted.  mbar_wait polls
+// (for the warps on the critical path, which must resume at once);
+// mbar_wait_sleep suspends between checks (for producer and issuer warps,
+// which would otherwise take issue slots from the compute warps).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                           int32_t *err)
 {
     if (mbar_test(bar, parity)) return true;  // non-blocking fast path
     for (uint32_t it = 0; it < kSpinLimit; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+    }
+    *abort = 1;
+    set_error(err, KSA_ERR_TIMEOUT);
+    return false;
+}
+
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, volatile int *abort,
+                                                int32_t *err)
+{
+    if (mbar_test(bar, parity)) return true;
+    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*abort) return false;
     }
     *abort = 1;

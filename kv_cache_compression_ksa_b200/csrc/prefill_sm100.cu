@@ -30,9 +30,12 @@
 //     tiles covering chunks c_first-w .. c_last.  Every other tile of the
 //     L x L plane is skipped without being looked at.  Inside a tile the
 //     mask of a row is one interval of columns, computed from coordinates.
-//   * Warp roles: warps 0-7 softmax (two warpgroups), warp 8 TMA producer,
-//     warp 9 MMA issuer and TMEM owner.  All mbarrier waits are bounded; on
-//     expiry the CTA records KSA_ERR_TIMEOUT, drains, frees TMEM and exits.
+//   * Warp roles: warps 0-7 softmax (two key halves), warp 8 TMA for Q and
+//     K, warp 9 the QK issuer and TMEM owner, warp 10 the PV issuer, warp 11
+//     TMA for V, warps 12-15 the epilogue (merge the halves, O / l -> bf16,
+//     LSE), which runs while the softmax warps start the next work item.
+//     All mbarrier waits are bounded; on expiry the CTA records
+//     KSA_ERR_TIMEOUT, drains, frees TMEM and exits.
 //   * Summary query rows (k+1 keys each) run in a separate CUDA-core kernel.
 #include <cuda.h>
 #include <math.h>
@@ -58,7 +61,10 @@ constexpr int kWarpTMA = 8;    // loads Q and the K tiles
 constexpr int kWarpQK = 9;     // issues S = Q K^T, owns TMEM
 constexpr int kWarpPV = 10;    // issues O_h += P_h V_h
 constexpr int kWarpTMAV = 11;  // loads the V tiles (K loads never wait behind V)
-constexpr int kThreads = 384;
+constexpr int kWarpEpi = 12;   // warps 12-15: the epilogue of each work item (one row per thread)
+constexpr int kThreads = 512;
+// 512 threads at 128 registers each fill the register file; every role fits
+// (the softmax no longer holds the epilogue's O rows).
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -71,9 +77,9 @@ struct SmemLayout {
     static constexpr int kO = kV + VSTAGES * kKVTile;           // output tile staging for the TMA store
     static constexpr int kBar = kO + kQTile;
     // barriers: kfull[KS], kempty[KS], vfull[VS], vempty[VS], s[NSBUF], p[2 halves][NSBUF],
-    // o[NSBUF], drain x2, o free, q full[QS], q free[QS]
-    static constexpr int kNumBars = 2 * KSTAGES + 2 * VSTAGES + NSBUF + 2 * NSBUF + NSBUF + 2 + 1 + 2 * QSTAGES;
-    static constexpr int kXchg = kBar + kNumBars * 8;  // [2 halves][2 values][128 rows] floats
+    // o[NSBUF], drain x2, o free, q full[QS], q free[QS], item done
+    static constexpr int kNumBars = 2 * KSTAGES + 2 * VSTAGES + NSBUF + 2 * NSBUF + NSBUF + 2 + 1 + 2 * QSTAGES + 1;
+    static constexpr int kXchg = kBar + kNumBars * 8;  // [2 halves][m, l][128 rows] floats
     static constexpr int kMisc = kXchg + 2 * 2 * BM * 4;
     static constexpr int kBytes = kMisc + 16;
     // the dynamic shared memory base is 1024-byte aligned (checked at run time)
@@ -122,13 +128,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) { retu
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-
-// Named barrier shared by the two softmax warps that cover the same 32 rows
-// (warp w and w + 4): ids 1..4, 64 threads.
-__device__ __forceinline__ void pair_sync(int quarter)
-{
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
-}
 
 // A work item: one query tile of 128 TMEM lanes (GQA-packed rows: Gp of the
 // G q heads of one kv head, starting at q head h0, for unit_chunks chunks)
@@ -222,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const int B_OFREE = B_DRAIN_QK + 2;   // epilogue read O: the next item's PV may overwrite it
     auto B_QF = [&](int q) { return B_DRAIN_QK + 3 + q; };            // query tile landed
     auto B_QE = [&](int q) { return B_DRAIN_QK + 3 + QSTAGES + q; };  // its QKs are done
+    const int B_UDONE = B_DRAIN_QK + 3 + 2 * QSTAGES;                  // softmax finished the item
 
     // ---- setup -----------------------------------------------------------
     if (threadIdx.x == 0) {
@@ -245,7 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         }
         mbar_init(bar(B_DRAIN_QK), 1);
         mbar_init(bar(B_DRAIN_PV), 1);
-        mbar_init(bar(B_OFREE), 256);
+        mbar_init(bar(B_OFREE), 128);   // the epilogue warps
+        mbar_init(bar(B_UDONE), 256);   // the softmax warps
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -404,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             tc_commit(bar(B_DRAIN_PV));
             for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_DRAIN_PV), 0); ++it) {}
         }
-    } else {
+    } else if (warp < 8) {
         // ================= softmax: 8 warps, two independent key halves =================
         const int half = warp >> 2;                    // keys [64 half, 64 half + 64) of each tile
         const int quarter = warp & 3;
@@ -413,10 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const int rows_per_chunk = P.k * P.Gp;
         const int cl = R / rows_per_chunk;             // row -> (chunk, slot, head)
         const int r_slot = (R / P.Gp) % P.k;
-        const int g = R % P.Gp;
         const float sl2 = P.scale_log2;
-        // An expired wait clears ok; every warp still walks all items and
-        // runs two pair barriers per item, so no barrier is left unmatched.
+        // An expired wait clears ok; every warp still walks all items.
         bool ok = true;
         int gt = 0;
         for (int item = blockIdx.x, n = 0; item < W; item += gridDim.x, ++n) {
@@ -523,20 +522,47 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 tc_fence_before();
                 mbar_arrive(bar(B_P(half, bf)));
             }
-            // ---- epilogue of the item: merge the halves, O / l -> bf16 rows ----
-            if (ok)
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O((gt - 1) % NSBUF)), (uint32_t)((gt - 1) / NSBUF) & 1u,
-                                                       abort, P.err));
-            tc_fence_after();
+            // ---- end of the item: this half's (m, l) to the epilogue warps,
+            // which merge the halves once the item's last PV has completed.
+            // The exchange buffer is free once the previous item's epilogue
+            // has read it (it reads before releasing O). ----
+            if (n > 0)
+                ok = ok && __all_sync(0xffffffffu,
+                                      mbar_wait(bar(B_OFREE), (uint32_t)(n - 1) & 1u, abort, P.err));
             float *xc = xchg;   // [half][m, l][row]
             xc[(half * 2 + 0) * BM + R] = m_run;
             xc[(half * 2 + 1) * BM + R] = l_run;
-            pair_sync(quarter);   // twice per item per softmax warp, on every path
-            const float m_o = xc[((1 - half) * 2 + 0) * BM + R];
-            const float l_o = xc[((1 - half) * 2 + 1) * BM + R];
-            pair_sync(quarter);   // both read: the next item may overwrite the exchange
-            const float m0 = half == 0 ? m_run : m_o, m1 = half == 0 ? m_o : m_run;
-            const float l0 = half == 0 ? l_run : l_o, l1 = half == 0 ? l_o : l_run;
+            mbar_arrive(bar(B_UDONE));
+        }
+    } else if (warp >= kWarpEpi) {
+        // ================= epilogue: 4 warps, one row per thread =================
+        // Merges the two halves' (m, l, O) of each item and stores O / l as
+        // bf16 (and the LSE) while the softmax warps run the next item.  O is
+        // free for the next item's first PV once it has been read (B_OFREE);
+        // that PV waits for it, which bounds how far the softmax runs ahead.
+        const int quarter = warp & 3;
+        const int R = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int rows_per_chunk = P.k * P.Gp;
+        const int cl = R / rows_per_chunk;
+        const int r_slot = (R / P.Gp) % P.k;
+        const int g = R % P.Gp;
+        const float sl2 = P.scale_log2;
+        const bool leader = warp == kWarpEpi && lane == 0;
+        bool ok = true;
+        int gt = 0;   // tiles up to and including this item
+        for (int item = blockIdx.x, n = 0; item < W; item += gridDim.x, ++n) {
+            const Unit U = unit_of(P, item, n_units);
+            gt += U.T;
+            const int c = U.c0 + cl;
+            const int i = c * P.k + r_slot;
+            const bool valid = cl < P.Tc && c < U.ncb && i < U.nb;
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(B_UDONE), (uint32_t)n & 1u, abort, P.err));
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(B_O((gt - 1) % NSBUF)), (uint32_t)((gt - 1) / NSBUF) & 1u,
+                                                         abort, P.err));
+            tc_fence_after();
+            const float *xc = xchg;
+            const float m0 = xc[0 * BM + R], l0 = xc[1 * BM + R], m1 = xc[2 * BM + R], l1 = xc[3 * BM + R];
             const float M = fmaxf(m0, m1);
             const float f0 = (M == -INFINITY) ? 0.f : ex2((m0 - M) * sl2);
             const float f1 = (M == -INFINITY) ? 0.f : ex2((m1 - M) * sl2);
@@ -547,21 +573,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             const bool tma_out = U.c0 + P.Tc <= U.mb;
             if (tma_out) {
                 // the staging buffer is free once the previous store has read it
-                if (warp == 0 && lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-                asm volatile("bar.sync 13, 256;" ::: "memory");
+                if (leader) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                asm volatile("bar.sync 13, 128;" ::: "memory");
             }
             const float inv = Lr > 0.f ? 1.f / Lr : 0.f;
             const float g0 = f0 * inv, g1 = f1 * inv;
             const int64_t row = (int64_t)(U.qbase + c) * (P.k + 1) + r_slot;
             const int head = U.h0 + g;
-            // this thread holds output columns [D/2 half, D/2 half + D/2) of its row
-            uint4 *dst = reinterpret_cast<uint4 *>(P.o + (row * P.Hq + head) * D + half * (D / 2));
+            uint4 *dst = reinterpret_cast<uint4 *>(P.o + (row * P.Hq + head) * D);
             const uint32_t stage_row = sbase + L::kO + (uint32_t)R * 128u;
 #pragma unroll 1
-            for (int cc = 0; cc < D / 64 && ok; ++cc) {
+            for (int cc = 0; cc < D / 32 && ok; ++cc) {
                 uint32_t a0[32], a1[32];
-                tmem_ld32(O_COL(0) + lane_off + half * (D / 2) + cc * 32, a0);
-                tmem_ld32(O_COL(1) + lane_off + half * (D / 2) + cc * 32, a1);
+                tmem_ld32(O_COL(0) + lane_off + cc * 32, a0);
+                tmem_ld32(O_COL(1) + lane_off + cc * 32, a1);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -574,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     if (tma_out) {
                         // column col of row R: 64-column half col / 64, 16-byte chunk
                         // j = (col % 64) / 8, stored at chunk j ^ (R % 8) (128-byte swizzle)
-                        const int col = half * (D / 2) + cc * 32 + 8 * e;
+                        const int col = cc * 32 + 8 * e;
                         const uint32_t hoff = (uint32_t)(col / 64) * kQHalf;
                         const uint32_t j = (uint32_t)((col % 64) / 8);
                         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stage_row + hoff + ((j ^ (uint32_t)(R & 7)) << 4)),
@@ -585,14 +610,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     }
                 }
             }
-            if (ok && valid && half == 0 && P.lse) P.lse[row * P.Hq + head] = M * P.scale + logf(Lr);
+            if (ok && valid && P.lse) P.lse[row * P.Hq + head] = M * P.scale + logf(Lr);
             // O has been read: the PV issuer may start the next item
             tc_fence_before();
             mbar_arrive(bar(B_OFREE));
             if (tma_out) {
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                asm volatile("bar.sync 13, 256;" ::: "memory");
-                if (warp == 0 && lane == 0 && ok) {
+                asm volatile("bar.sync 13, 128;" ::: "memory");
+                if (leader && ok) {
 #pragma unroll
                     for (int hf = 0; hf < D / 64; ++hf)
                         tma_store_4d(&P.tm_o, sbase + L::kO + hf * kQHalf, hf * 64, U.h0, 0, U.qbase + U.c0);
@@ -601,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             }
         }
         // every store has finished reading shared memory before the CTA exits
-        if (warp == 0 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
 
     // ---- teardown --------------------------------------------------------

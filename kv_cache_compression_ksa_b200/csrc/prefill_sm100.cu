@@ -463,13 +463,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 };
                 load_s();
                 // the row max of this half's 64 keys
-                float pm[8];
+                static_assert(HC == 64, "the max tree below covers 64 scores");
+                float pm[8];   // three-input max: columns a, a+8, ..., a+56 into pm[a]
 #pragma unroll
-                for (int a = 0; a < 8; ++a) pm[a] = -INFINITY;
-#pragma unroll
-                for (int e = 0; e < HC; ++e) pm[e & 7] = fmaxf(pm[e & 7], s[e]);
-                const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                       fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+                for (int a = 0; a < 8; ++a) {
+                    pm[a] = max3(s[a], s[a + 8], s[a + 16]);
+                    pm[a] = max3(pm[a], s[a + 24], s[a + 32]);
+                    pm[a] = max3(pm[a], s[a + 40], s[a + 48]);
+                    pm[a] = fmaxf(pm[a], s[a + 56]);
+                }
+                const float mx = max3(max3(pm[0], pm[1], pm[2]), max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
                 // lazy rescale: keep the reference unless the max exceeds it by
                 // more than 8 in log2 units (P stays <= 256; exact either way)
                 const float m_new = fmaxf(m_run, mx);
@@ -500,23 +503,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 // as soon as they are packed, so the first store overlaps the
                 // second group's exponentials
                 const float mb = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-                float ps[8];
+                // x = s sl2 - mb and the row sums on packed fp32 pairs; the
+                // sums keep eight partials (element e in partial e % 8)
+                const uint64_t sl2x2 = f2_pack(sl2, sl2), nmbx2 = f2_pack(-mb, -mb);
+                uint64_t ps2[4];
 #pragma unroll
-                for (int a = 0; a < 8; ++a) ps[a] = 0.f;
+                for (int a = 0; a < 4; ++a) ps2[a] = 0ull;
 #pragma unroll
                 for (int grp = 0; grp < 2; ++grp) {
                     uint32_t pk[HC / 4];
 #pragma unroll
                     for (int e2 = 0; e2 < HC / 4; ++e2) {
                         const int e = grp * (HC / 2) + 2 * e2;
-                        const float p0 = ex2(fmaf(s[e], sl2, -mb)), p1 = ex2(fmaf(s[e + 1], sl2, -mb));
-                        ps[e & 7] += p0;
-                        ps[(e + 1) & 7] += p1;
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sl2x2, nmbx2), x0, x1);
+                        const float p0 = ex2(x0), p1 = ex2(x1);
+                        ps2[(e & 7) >> 1] = f2_add(ps2[(e & 7) >> 1], f2_pack(p0, p1));
                         pk[e2] = pack_bf16(p0, p1);
                     }
                     // P of this half -> S columns [64 half + 16 grp, +16) (its own S region)
                     tmem_st16(S_COL(bf) + lane_off + half * HC + grp * (HC / 4), pk);
                 }
+                float ps[8];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) f2_unpack(ps2[a], ps[2 * a], ps[2 * a + 1]);
                 l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 tmem_wait_st();
                 tc_fence_before();

@@ -43,7 +43,7 @@ constexpr int BK = 128;       // keys per tile (TMEM lanes)
 constexpr int BQ = 128;       // query positions per step (MMA N)
 constexpr int HQ = BQ / 2;    // query columns per elementwise warp
 constexpr int QST = 2;        // Q / dO stages
-constexpr int kSplit = 32;    // steps per CTA
+constexpr int kSplit = 128;   // steps per CTA
 constexpr int kWarpTMA = 8;   // K, V once, then Q and dO per step
 constexpr int kWarpMMA = 9;   // MMA issuer, TMEM owner
 constexpr int kWarpLD = 10;   // per-step LSE and D, zero rows past the sequence

@@ -14,20 +14,23 @@
 // Design.  A CTA owns one tile of 128 keys of one kind (128 consecutive text
 // tokens or 128 consecutive summaries of one sequence) of one kv head: its K
 // and V sit in shared memory for the whole CTA and its rows are the 128
-// TMEM lanes.  It walks a share of at most kSplit steps; a step is one q head
-// of the kv head's group x 128 consecutive text query positions (TMA boxes
-// over the augmented layout's text slots), and takes four MMAs:
-//     S^T  = K Q^T      (SS, M 128 keys, N 128 queries, K d)
+// TMEM lanes.  It walks a share of its steps; a step is one q head of the kv
+// head's group x NQ consecutive text query positions (TMA boxes over the
+// augmented layout's text slots; NQ = 64 when k divides 64, else 128), and
+// takes four MMAs:
+//     S^T  = K Q^T      (SS, M 128 keys, N NQ queries, K d)
 //     dP^T = V dO^T     (SS)
 //     dV  += P^T dO     (TS: P^T written as bf16 over S^T, B = dO MN-major)
 //     dK  += dS^T Q     (TS: dS^T written as bf16 over dP^T)
-// TMEM holds S^T, dP^T, dV and dK (128 + 128 + 2 d columns).  Eight
-// elementwise warps (two per TMEM lane quarter, 64 query columns each) turn
-// S^T into P^T and dP^T into dS^T; the mask of a key row inside a step is
-// one interval of columns, from coordinates.  The summary query rows (a
-// summary sees its own chunk and itself) are left to the warp-level kernel of
-// prefill_bwd.cu.  Shares of the same key tile (long summary ranges) add
-// their dK, dV into fp32 accumulators.  All mbarrier waits are bounded.
+// TMEM holds S^T and dP^T (two buffers each at NQ = 64, so the next step's
+// products run while this step's accumulations read P^T and dS^T), dV and
+// dK.  Eight elementwise warps (two per TMEM lane quarter, NQ / 2 query
+// columns each) turn S^T into P^T and dP^T into dS^T; the mask of a key row
+// inside a step is one interval of columns, from coordinates.  The summary
+// query rows (a summary sees its own chunk and itself) are left to a
+// CUDA-core kernel of prefill_bwd.cu.  Shares of the same key tile (long
+// summary ranges) add their dK, dV into fp32 accumulators.  All mbarrier
+// waits are bounded.
 #include <cuda.h>
 #include <math.h>
 
@@ -40,10 +43,8 @@ namespace bt {
 using namespace tc;
 
 constexpr int BK = 128;       // keys per tile (TMEM lanes)
-constexpr int BQ = 128;       // query positions per step (MMA N)
-constexpr int HQ = BQ / 2;    // query columns per elementwise warp
-constexpr int QST = 2;        // Q / dO stages
-constexpr int kSplit = 128;   // steps per CTA
+constexpr int BQ = 128;       // query positions per dq tile (MMA M) and per key tile's query tiles of dq
+constexpr int HQ = BQ / 2;    // key columns per elementwise warp of dq
 constexpr int kWarpTMA = 8;   // K, V once, then Q and dO per step
 constexpr int kWarpMMA = 9;   // MMA issuer, TMEM owner
 constexpr int kWarpLD = 10;   // per-step LSE and D, zero rows past the sequence
@@ -51,25 +52,36 @@ constexpr int kWarpMMA2 = 11; // second MMA issuer (an issuing thread sustains ~
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 
-template <int D>
-struct Smem {
-    static constexpr int kTile = BK * D * 2;   // one 128 x D bf16 tile
+// dk/dv geometry: NQ query positions per step (64 when k divides 64, else
+// 128) and NBUF S^T / dP^T buffers (two at NQ = 64: the next step's products
+// go to the other buffer while dV and dK read this one's P^T and dS^T).
+template <int D, int NQ>
+struct DkvCfg {
+    static constexpr int HQ2 = NQ / 2;              // query columns per elementwise warp
+    static constexpr int NBUF = NQ == 64 ? 2 : 1;
+    static constexpr int QS = NQ == 64 ? 4 : 2;     // Q / dO stages
+    static constexpr int kSplit = NQ == 64 ? 256 : 128;   // steps per CTA (16384 query positions)
+    static constexpr int kTile = BK * D * 2;        // a 128 x D bf16 K or V tile
+    static constexpr int kQTile = NQ * D * 2;       // an NQ x D bf16 Q or dO tile
+    static constexpr int kQHalf = NQ * 128;         // one 64-column half of it
     static constexpr int kK = 0;
     static constexpr int kV = kK + kTile;
-    static constexpr int kQ = kV + kTile;            // [QST] query tiles
-    static constexpr int kDO = kQ + QST * kTile;     // [QST] dO tiles
-    static constexpr int kLD = kDO + QST * kTile;    // [QST][lse2, D][BQ] floats
-    static constexpr int kBar = kLD + QST * 2 * BQ * 4;
-    // kv, qt[QST], qf[QST], qe[QST], s, dp, p, ds, dv, dk, drain
-    static constexpr int kNumBars = 1 + 3 * QST + 7;
+    static constexpr int kQ = kV + kTile;           // [QS] query tiles
+    static constexpr int kDO = kQ + QS * kQTile;    // [QS] dO tiles
+    static constexpr int kLD = kDO + QS * kQTile;   // [QS][lse2, D][NQ] floats
+    static constexpr int kBar = kLD + QS * 2 * NQ * 4;
+    // kv, qt[QS], qf[QS], qe[QS], s[NBUF], dp[NBUF], p[NBUF], ds[NBUF], dv, dk, drain
+    static constexpr int kNumBars = 1 + 3 * QS + 4 * NBUF + 3;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static_assert(kBytes <= 227 * 1024, "shared memory budget");
-    static_assert(2 * BQ + 2 * D <= (int)kTmemCols, "TMEM budget");
+    static_assert(2 * NBUF * NQ + 2 * D <= (int)kTmemCols, "TMEM budget");
+    static_assert(HQ2 % 32 == 0, "elementwise column groups");
 };
 
 struct TArgs {
-    CUtensorMap tm_kt, tm_ks, tm_vt, tm_vs, tm_q, tm_do;
+    CUtensorMap tm_kt, tm_ks, tm_vt, tm_vs, tm_q, tm_do;   // 128-row boxes (dq: query tiles; K/V tiles)
+    CUtensorMap tm_qs, tm_dos;                             // nqs-row boxes: the dk/dv steps' Q and dO
     int k, w, G, Hq, Hkv, batch;
     float scale, scale_log2;
     const int32_t *cu;
@@ -77,6 +89,7 @@ struct TArgs {
     const int32_t *ks_off, *kt_off;   // [B+1] first summary / text key tile of each sequence
     const int32_t *item_off;          // [tiles+1] first CTA of each key tile (summary tiles first)
     int max_tiles;
+    int nqs, split;                   // dk/dv: query positions per step, steps per CTA
     int32_t *err;
     const float *lse, *dsum;
     float *dk32, *dv32;
@@ -118,11 +131,11 @@ __device__ __forceinline__ void key_tile(const TArgs &a, int tile, KTile &T)
         T.qlo = T.j0;
         T.qhi = min(T.n, (cb + a.w + 1) * a.k);     // past the last text query of chunk cb's keys
     }
-    T.nq = T.qhi > T.qlo ? (T.qhi - T.qlo + BQ - 1) / BQ : 0;
+    T.nq = T.qhi > T.qlo ? (T.qhi - T.qlo + a.nqs - 1) / a.nqs : 0;   // dk/dv steps per q head
 }
 
 // Key tiles (summary tiles of all sequences, then text tiles) and the CTA
-// offsets of their shares of ceil(G nq / kSplit) CTAs each.
+// offsets of their shares of ceil(G nq / split) CTAs each.
 __global__ void __launch_bounds__(1024) bt_plan_kernel(TArgs a, int32_t *ks_off, int32_t *kt_off, int32_t *item_off)
 {
     __shared__ int part[1024];
@@ -152,7 +165,7 @@ __global__ void __launch_bounds__(1024) bt_plan_kernel(TArgs a, int32_t *ks_off,
     for (int t = lo; t < hi; ++t) {
         KTile T;
         key_tile(a, t, T);
-        sum += (a.G * T.nq + kSplit - 1) / kSplit;
+        sum += (a.G * T.nq + a.split - 1) / a.split;
     }
     part[threadIdx.x] = sum;
     __syncthreads();
@@ -171,14 +184,15 @@ __global__ void __launch_bounds__(1024) bt_plan_kernel(TArgs a, int32_t *ks_off,
         item_off[t] = run;
         KTile T;
         key_tile(a, t, T);
-        run += (a.G * T.nq + kSplit - 1) / kSplit;
+        run += (a.G * T.nq + a.split - 1) / a.split;
     }
 }
 
-template <int D>
+template <int D, int NQ>
 __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_constant__ TArgs a)
 {
-    using L = Smem<D>;
+    using L = DkvCfg<D, NQ>;
+    constexpr int QS = L::QS, NBUF = L::NBUF, HQ2 = L::HQ2;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw;
     const uint32_t sbase = smem_u32(smem);
@@ -200,29 +214,34 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
     KTile T;
     key_tile(a, tile, T);
     const int g = blockIdx.y;
-    const int s_lo = (item - a.item_off[tile]) * kSplit;
-    const int n_steps = min(a.G * T.nq, s_lo + kSplit) - s_lo;
+    const int s_lo = (item - a.item_off[tile]) * L::kSplit;
+    const int n_steps = min(a.G * T.nq, s_lo + L::kSplit) - s_lo;
     if (n_steps <= 0) return;
 
     auto bar = [&](int i) { return sbase + L::kBar + 8u * (uint32_t)i; };
     constexpr int B_KV = 0;
     auto B_QT = [](int s) { return 1 + s; };              // Q, dO landed
-    auto B_QF = [](int s) { return 1 + QST + s; };        // + LSE, D, zero rows: ready
-    auto B_QE = [](int s) { return 1 + 2 * QST + s; };    // stage free
-    constexpr int B_S = 1 + 3 * QST, B_DP = B_S + 1, B_P = B_S + 2, B_DS = B_S + 3, B_DV = B_S + 4,
-                  B_DK = B_S + 5, B_DRAIN = B_S + 6;
+    auto B_QF = [](int s) { return 1 + QS + s; };         // + LSE, D, zero rows: ready
+    auto B_QE = [](int s) { return 1 + 2 * QS + s; };     // stage free
+    auto B_S = [](int b) { return 1 + 3 * QS + b; };      // S^T of buffer b computed
+    auto B_DP = [](int b) { return 1 + 3 * QS + NBUF + b; };
+    auto B_P = [](int b) { return 1 + 3 * QS + 2 * NBUF + b; };    // P^T written
+    auto B_DS = [](int b) { return 1 + 3 * QS + 3 * NBUF + b; };   // dS^T written
+    constexpr int B_DV = 1 + 3 * QS + 4 * NBUF, B_DK = B_DV + 1, B_DRAIN = B_DV + 2;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_KV), 1);
-        for (int s = 0; s < QST; ++s) {
+        for (int s = 0; s < QS; ++s) {
             mbar_init(bar(B_QT(s)), 1);
             mbar_init(bar(B_QF(s)), 32);
             mbar_init(bar(B_QE(s)), 2);   // one commit per issuer
         }
-        mbar_init(bar(B_S), 1);
-        mbar_init(bar(B_DP), 1);
-        mbar_init(bar(B_P), 256);
-        mbar_init(bar(B_DS), 256);
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(bar(B_S(b)), 1);
+            mbar_init(bar(B_DP(b)), 1);
+            mbar_init(bar(B_P(b)), 256);
+            mbar_init(bar(B_DS(b)), 256);
+        }
         mbar_init(bar(B_DV), 1);
         mbar_init(bar(B_DK), 1);
         mbar_init(bar(B_DRAIN), 2);   // one commit per issuer, after its last MMA
@@ -239,18 +258,22 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t T_S = tmem, T_DP = tmem + BQ, T_DV = tmem + 2 * BQ, T_DK = tmem + 2 * BQ + D;
-    constexpr uint32_t kHalf = BK * 128;   // bytes of one 64-column half of a tile
-    constexpr uint32_t kTileBytes = (uint32_t)L::kTile;
+    // TMEM: S^T[NBUF], dP^T[NBUF] (NQ columns each), dV, dK (D columns each)
+    auto T_S = [&](int b) { return tmem + (uint32_t)(b * NQ); };
+    auto T_DP = [&](int b) { return tmem + (uint32_t)((NBUF + b) * NQ); };
+    const uint32_t T_DV = tmem + 2 * NBUF * NQ, T_DK = T_DV + D;
+    constexpr uint32_t kHalf = BK * 128;   // one 64-column half of a K or V tile
+    constexpr uint32_t kTileBytes = (uint32_t)L::kTile, kQBytes = (uint32_t)L::kQTile;
+    constexpr uint32_t kQHalf = (uint32_t)L::kQHalf;
 
     // step s of the share -> (query tile, q head)
-    auto step_q0 = [&](int s) { return T.qlo + ((s_lo + s) / a.G) * BQ; };
+    auto step_q0 = [&](int s) { return T.qlo + ((s_lo + s) / a.G) * NQ; };
     auto step_h = [&](int s) { return g * a.G + (s_lo + s) % a.G; };
 
     if (warp == kWarpTMA) {
         if (lane == 0) {
             bool ok = true;
-            int q_issued[QST] = {0};
+            int q_issued[QS] = {0};
             mbar_expect_tx(bar(B_KV), 2 * kTileBytes);
             for (int hf = 0; hf < D / 64; ++hf) {
                 if (T.sum) {
@@ -262,15 +285,15 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
                 }
             }
             for (int s = 0; s < n_steps; ++s) {
-                const int st = s % QST;
-                if (s >= QST && !(ok = mbar_wait_sleep(bar(B_QE(st)), (uint32_t)((s / QST) - 1) & 1u, abort, a.err)))
+                const int st = s % QS;
+                if (s >= QS && !(ok = mbar_wait_sleep(bar(B_QE(st)), (uint32_t)((s / QS) - 1) & 1u, abort, a.err)))
                     break;
                 const int chunk = T.c0 + step_q0(s) / a.k, h = step_h(s);
-                mbar_expect_tx(bar(B_QT(st)), 2 * kTileBytes);
+                mbar_expect_tx(bar(B_QT(st)), 2 * kQBytes);
                 for (int hf = 0; hf < D / 64; ++hf) {
-                    tma_load_4d(sbase + L::kQ + st * kTileBytes + hf * kHalf, &a.tm_q, bar(B_QT(st)), hf * 64, h, 0,
+                    tma_load_4d(sbase + L::kQ + st * kQBytes + hf * kQHalf, &a.tm_qs, bar(B_QT(st)), hf * 64, h, 0,
                                 chunk);
-                    tma_load_4d(sbase + L::kDO + st * kTileBytes + hf * kHalf, &a.tm_do, bar(B_QT(st)), hf * 64, h,
+                    tma_load_4d(sbase + L::kDO + st * kQBytes + hf * kQHalf, &a.tm_dos, bar(B_QT(st)), hf * 64, h,
                                 0, chunk);
                 }
                 q_issued[st]++;
@@ -278,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
             // every load issued lands before the CTA exits
             for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_KV), 0); ++it) {}
             if (!ok)
-                for (int st = 0; st < QST; ++st)
+                for (int st = 0; st < QS; ++st)
                     if (q_issued[st]) {
                         const uint32_t ph = (uint32_t)(q_issued[st] - 1) & 1u;
                         for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_QT(st)), ph); ++it) {}
@@ -290,10 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
         // waits for its tiles); once the tiles have landed, zero the query
         // rows past the sequence (they meet P = 0 and dS = 0 in the MMAs,
         // which need them finite) and publish LSE and D in shared memory
-        constexpr int PER = BQ / 32;
+        constexpr int PER = NQ / 32;
         float l2v[PER], ddv[PER];
         auto fetch = [&](int s) {
-            const int q0 = step_q0(s), h = step_h(s), qn = min(BQ, T.n - q0);
+            const int q0 = step_q0(s), h = step_h(s), qn = min(NQ, T.n - q0);
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
                 const int r = lane + 32 * u, pos = q0 + r;
@@ -305,25 +328,25 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
         bool ok = true;
         fetch(0);
         for (int s = 0; s < n_steps && ok; ++s) {
-            const int st = s % QST;
-            ok = __all_sync(0xffffffffu, mbar_wait_sleep(bar(B_QT(st)), (uint32_t)(s / QST) & 1u, abort, a.err));
+            const int st = s % QS;
+            ok = __all_sync(0xffffffffu, mbar_wait_sleep(bar(B_QT(st)), (uint32_t)(s / QS) & 1u, abort, a.err));
             if (!ok) break;
-            const int qn = min(BQ, T.n - step_q0(s));
-            if (qn < BQ) {
+            const int qn = min(NQ, T.n - step_q0(s));
+            if (qn < NQ) {
                 const int per_row = 8 * (D / 64);   // 16-byte words of a row over both halves
-                for (int e = lane; e < (BQ - qn) * per_row; e += 32) {
+                for (int e = lane; e < (NQ - qn) * per_row; e += 32) {
                     const int r = qn + e / per_row, hf = (e % per_row) / 8, c = e % 8;
-                    const uint32_t off = (uint32_t)(hf * kHalf + r * 128 + c * 16);
-                    *reinterpret_cast<uint4 *>(smem + L::kQ + st * kTileBytes + off) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(smem + L::kDO + st * kTileBytes + off) = make_uint4(0, 0, 0, 0);
+                    const uint32_t off = (uint32_t)(hf * kQHalf + r * 128 + c * 16);
+                    *reinterpret_cast<uint4 *>(smem + L::kQ + st * kQBytes + off) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(smem + L::kDO + st * kQBytes + off) = make_uint4(0, 0, 0, 0);
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
-            float *ld = reinterpret_cast<float *>(smem + L::kLD) + st * 2 * BQ;
+            float *ld = reinterpret_cast<float *>(smem + L::kLD) + st * 2 * NQ;
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
                 ld[lane + 32 * u] = l2v[u] * 1.4426950408889634f;
-                ld[BQ + lane + 32 * u] = ddv[u];
+                ld[NQ + lane + 32 * u] = ddv[u];
             }
             mbar_arrive(bar(B_QF(st)));
             if (s + 1 < n_steps) fetch(s + 1);
@@ -331,49 +354,59 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
     } else if (warp == kWarpMMA || warp == kWarpMMA2) {
         // Two issuers, one per chain: kWarpMMA the P side (S^T = K Q^T, then
         // dV += P^T dO), kWarpMMA2 the dS side (dP^T = V dO^T, then
-        // dK += dS^T Q).  Each side's product columns are free again once
-        // its own accumulation of the step before has read them.
+        // dK += dS^T Q).  With two buffers a side issues step t's product
+        // before the accumulation of step t - 1, which reads the other
+        // buffer; a buffer is reused once this side's accumulation of the
+        // step two back has read it.
         if (lane == 0) {
             const bool pside = warp == kWarpMMA;
-            const uint32_t id_ss = idesc_f16(BK, BQ, false);
+            const uint32_t id_ss = idesc_f16(BK, NQ, false);
             const uint32_t id_ts = idesc_f16(BK, D, true);
-            const uint32_t T_X = pside ? T_S : T_DP, T_ACC = pside ? T_DV : T_DK;
-            const int b_x = pside ? B_S : B_DP, b_in = pside ? B_P : B_DS, b_acc = pside ? B_DV : B_DK;
+            const int b_in0 = pside ? B_P(0) : B_DS(0), b_x0 = pside ? B_S(0) : B_DP(0);
+            const int b_acc = pside ? B_DV : B_DK;
+            const uint32_t T_ACC = pside ? T_DV : T_DK;
             const uint64_t dA = sdesc(sbase + (pside ? L::kK : L::kV), 16, 1024);   // SS A: K or V
             bool ok = mbar_wait_sleep(bar(B_KV), 0, abort, a.err);
-            for (int s = 0; s < n_steps && ok; ++s) {
-                const int st = s % QST;
-                const uint32_t ph = (uint32_t)s & 1u, php = (uint32_t)(s - 1) & 1u;
-                if (!(ok = mbar_wait_sleep(bar(B_QF(st)), (uint32_t)(s / QST) & 1u, abort, a.err))) break;
-                const uint32_t qa = sbase + L::kQ + st * kTileBytes, da = sbase + L::kDO + st * kTileBytes;
-                const uint64_t dB = sdesc(pside ? qa : da, 16, 1024);      // SS B: Q or dO (K-major)
-                const uint64_t dC = sdesc(pside ? da : qa, kHalf, 1024);   // TS B: dO or Q (MN-major)
-                if (s > 0 && !(ok = mbar_wait_sleep(bar(b_acc), php, abort, a.err))) break;
-                tc_fence_after();
+            for (int t = 0; t < n_steps + NBUF - 1 && ok; ++t) {
+                if (t < n_steps) {
+                    const int st = t % QS, b = t % NBUF;
+                    if (!(ok = mbar_wait_sleep(bar(B_QF(st)), (uint32_t)(t / QS) & 1u, abort, a.err))) break;
+                    if (t >= NBUF && !(ok = mbar_wait_sleep(bar(b_acc), (uint32_t)(t - NBUF) & 1u, abort, a.err)))
+                        break;
+                    tc_fence_after();
+                    const uint64_t dB =
+                        sdesc(sbase + (pside ? L::kQ : L::kDO) + st * kQBytes, 16, 1024);   // SS B: Q or dO
+                    const uint32_t T_X = pside ? T_S(b) : T_DP(b);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk / 4) * kHalf + (kk % 4) * 32) >> 4;
-                    mma_ss(T_X, dA + off, dB + off, id_ss, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(T_X, dA + ((uint32_t)((kk / 4) * kHalf + (kk % 4) * 32) >> 4),
+                               dB + ((uint32_t)((kk / 4) * kQHalf + (kk % 4) * 32) >> 4), id_ss, kk > 0);
+                    tc_commit(bar(b_x0 + b));
                 }
-                tc_commit(bar(b_x));
-                // half h's bf16 pairs sit in columns [64h, 64h + 32) of S^T / dP^T
-                // and meet rows [64h, 64h + 64) of dO / Q
-                if (!(ok = mbar_wait_sleep(bar(b_in), ph, abort, a.err))) break;
-                tc_fence_after();
+                const int s = t - (NBUF - 1);
+                if (s >= 0) {
+                    const int st = s % QS, b = s % NBUF;
+                    if (!(ok = mbar_wait_sleep(bar(b_in0 + b), (uint32_t)(s / NBUF) & 1u, abort, a.err))) break;
+                    tc_fence_after();
+                    // half h's bf16 pairs sit in columns [HQ2 h, HQ2 h + HQ2/2) of
+                    // S^T / dP^T and meet rows [HQ2 h, HQ2 h + HQ2) of dO / Q
+                    const uint64_t dC = sdesc(sbase + (pside ? L::kDO : L::kQ) + st * kQBytes, kQHalf, 1024);
+                    const uint32_t T_X = pside ? T_S(b) : T_DP(b);
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+                    for (int h = 0; h < 2; ++h)
 #pragma unroll
-                    for (int kk = 0; kk < HQ / 16; ++kk)
-                        mma_ts(T_ACC, T_X + h * HQ + kk * 8, dC + (uint32_t)(((h * (HQ / 16) + kk) * 2048) >> 4), id_ts,
-                               (s > 0 || h > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(bar(b_acc));
-                tc_commit(bar(B_QE(st)));
+                        for (int kk = 0; kk < HQ2 / 16; ++kk)
+                            mma_ts(T_ACC, T_X + h * HQ2 + kk * 8, dC + (uint32_t)(((h * (HQ2 / 16) + kk) * 2048) >> 4),
+                                   id_ts, (s > 0 || h > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(bar(b_acc));
+                    tc_commit(bar(B_QE(st)));
+                }
             }
             tc_commit(bar(B_DRAIN));
             for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(bar(B_DRAIN), 0); ++it) {}
         }
     } else if (warp < 8) {
-        // ================= elementwise: 8 warps, 64 query columns each =================
+        // ================= elementwise: 8 warps, HQ2 query columns each =================
         const int half = warp >> 2, quarter = warp & 3;
         const int r = quarter * 32 + lane;   // key row = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -382,10 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
         const float sl2 = a.scale_log2;
         bool ok = true;
         for (int s = 0; s < n_steps; ++s) {
-            const int st = s % QST;
-            const uint32_t ph = (uint32_t)s & 1u;
+            const int st = s % QS, b = s % NBUF;
+            const uint32_t ph = (uint32_t)(s / NBUF) & 1u;
             const int q0 = step_q0(s);
-            const int qn = min(BQ, T.n - q0);
+            const int qn = min(NQ, T.n - q0);
             // this row's visible columns [lo, hi) of the step, inside this half
             int lo, hi;
             if (T.sum) {
@@ -396,51 +429,51 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
                 hi = min(qn, (key / a.k + a.w + 1) * a.k - q0);
             }
             if (!live) lo = hi = 0;
-            lo = max(lo - half * HQ, 0);
-            hi = min(hi - half * HQ, HQ);
+            lo = max(lo - half * HQ2, 0);
+            hi = min(hi - half * HQ2, HQ2);
             if (hi < lo) hi = lo;
             // every column of this half visible to every row of the warp: no mask
-            const bool full = __all_sync(0xffffffffu, lo == 0 && hi == HQ);
-            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(B_QF(st)), (uint32_t)(s / QST) & 1u, abort, a.err));
-            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(B_S), ph, abort, a.err));
+            const bool full = __all_sync(0xffffffffu, lo == 0 && hi == HQ2);
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(B_QF(st)), (uint32_t)(s / QS) & 1u, abort, a.err));
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(B_S(b)), ph, abort, a.err));
             if (!ok) break;
-            const float *l2 = reinterpret_cast<const float *>(smem + L::kLD) + st * 2 * BQ + half * HQ;
-            const float *dd = l2 + BQ;
-            float p[HQ];
+            const float *l2 = reinterpret_cast<const float *>(smem + L::kLD) + st * 2 * NQ + half * HQ2;
+            const float *dd = l2 + NQ;
+            float p[HQ2];
             {
-                uint32_t sr[HQ];
+                uint32_t sr[HQ2];
                 tc_fence_after();
-                tmem_ld32(T_S + lane_off + half * HQ, sr);
-                tmem_ld32(T_S + lane_off + half * HQ + 32, sr + 32);
+#pragma unroll
+                for (int cc = 0; cc < HQ2 / 32; ++cc) tmem_ld32(T_S(b) + lane_off + half * HQ2 + cc * 32, sr + cc * 32);
                 tmem_wait_ld();
                 if (full) {
 #pragma unroll
-                    for (int e = 0; e < HQ; ++e) p[e] = ex2(fmaf(__uint_as_float(sr[e]), sl2, -l2[e]));
+                    for (int e = 0; e < HQ2; ++e) p[e] = ex2(fmaf(__uint_as_float(sr[e]), sl2, -l2[e]));
                 } else {
 #pragma unroll
-                    for (int e = 0; e < HQ; ++e) {
+                    for (int e = 0; e < HQ2; ++e) {
                         const float x = fmaf(__uint_as_float(sr[e]), sl2, -l2[e]);
                         p[e] = (e >= lo && e < hi) ? ex2(x) : 0.f;
                     }
                 }
 #pragma unroll
-                for (int grp = 0; grp < 2; ++grp) {
+                for (int grp = 0; grp < HQ2 / 32; ++grp) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e2 = 0; e2 < 16; ++e2) pk[e2] = pack_bf16(p[grp * 32 + 2 * e2], p[grp * 32 + 2 * e2 + 1]);
-                    tmem_st16(T_S + lane_off + half * HQ + grp * 16, pk);
+                    tmem_st16(T_S(b) + lane_off + half * HQ2 + grp * 16, pk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(bar(B_P));
+                mbar_arrive(bar(B_P(b)));
             }
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DP), ph, abort, a.err));
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DP(b)), ph, abort, a.err));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int grp = 0; grp < 2; ++grp) {
+            for (int grp = 0; grp < HQ2 / 32; ++grp) {
                 uint32_t dr[32], pk[16];
-                tmem_ld32(T_DP + lane_off + half * HQ + grp * 32, dr);
+                tmem_ld32(T_DP(b) + lane_off + half * HQ2 + grp * 32, dr);
                 tmem_wait_ld();
                 float ds[32];
                 if (full) {
@@ -455,13 +488,13 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
                 }
 #pragma unroll
                 for (int e2 = 0; e2 < 16; ++e2) pk[e2] = pack_bf16(ds[2 * e2], ds[2 * e2 + 1]);
-                // dS^T of this half -> dP^T columns [64 half + 16 grp, +16); the
-                // second group's load above read columns at or past 64 half + 32
-                tmem_st16(T_DP + lane_off + half * HQ + grp * 16, pk);
+                // dS^T of this half -> dP^T columns [HQ2 half + 16 grp, +16), which
+                // this thread has already loaded
+                tmem_st16(T_DP(b) + lane_off + half * HQ2 + grp * 16, pk);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(B_DS));
+            mbar_arrive(bar(B_DS(b)));
         }
         // ---- epilogue: dK (scaled) and dV rows into the fp32 accumulators ----
         // (the drain barrier completes once, after every MMA of both issuers)
@@ -856,19 +889,20 @@ size_t prefill_bwd_tc_workspace_bytes(int batch, int64_t aug_rows)
     return 2 * align_up(sizeof(int32_t) * (size_t)(batch + 1)) + align_up(sizeof(int32_t) * (size_t)(tiles + 1));
 }
 
-template <int D>
+template <int D, int NQ>
 static int bt_launch(const bt::TArgs &a, int64_t grid, int64_t grid_q, __nv_bfloat16 *dq, cudaStream_t st)
 {
+    using C = bt::DkvCfg<D, NQ>;
     static bool attr = false;
     if (!attr) {
-        if (cudaFuncSetAttribute(bt::bt_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 bt::Smem<D>::kBytes) != cudaSuccess ||
+        if (cudaFuncSetAttribute(bt::bt_dkv_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kBytes) !=
+                cudaSuccess ||
             cudaFuncSetAttribute(bt::bq_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  bt::SmemQ<D>::kBytes) != cudaSuccess)
             return KSA_ERR_CUDA;
         attr = true;
     }
-    bt::bt_dkv_kernel<D><<<dim3((unsigned)grid, a.Hkv), bt::kThreads, bt::Smem<D>::kBytes, st>>>(a);
+    bt::bt_dkv_kernel<D, NQ><<<dim3((unsigned)grid, a.Hkv), bt::kThreads, C::kBytes, st>>>(a);
     bt::bq_dq_kernel<D><<<dim3((unsigned)grid_q, a.Hq), bt::kThreads, bt::SmemQ<D>::kBytes, st>>>(a, dq);
     return KSA_OK;
 }
@@ -882,7 +916,13 @@ int launch_prefill_bwd_tc(const ksa_params *p, int batch, const int32_t *cu, int
     const int d = p->head_dim, kk = p->k;
     const int64_t chunks = aug_rows / (kk + 1);
     const int qrows = bt::BQ / kk;   // chunks per query / text key box
-    bool ok = make_map(&a.tm_kt, k, d, p->num_kv_heads, kk, chunks, 1, kk, qrows) &&
+    // dk/dv steps of 64 query positions (two S^T / dP^T buffers) when k
+    // divides 64, else of 128
+    const int nqs = 64 % kk == 0 ? 64 : bt::BQ;
+    const int split = nqs == 64 ? bt::DkvCfg<128, 64>::kSplit : bt::DkvCfg<128, 128>::kSplit;
+    bool ok = make_map(&a.tm_qs, q, d, p->num_q_heads, kk, chunks, 1, kk, nqs / kk) &&
+              make_map(&a.tm_dos, dout, d, p->num_q_heads, kk, chunks, 1, kk, nqs / kk) &&
+              make_map(&a.tm_kt, k, d, p->num_kv_heads, kk, chunks, 1, kk, qrows) &&
               make_map(&a.tm_vt, v, d, p->num_kv_heads, kk, chunks, 1, kk, qrows) &&
               make_map(&a.tm_ks, k, d, p->num_kv_heads, kk, chunks, 1, 1, bt::BK) &&
               make_map(&a.tm_vs, v, d, p->num_kv_heads, kk, chunks, 1, 1, bt::BK) &&
@@ -894,6 +934,7 @@ int launch_prefill_bwd_tc(const ksa_params *p, int batch, const int32_t *cu, int
     a.scale_log2 = a.scale * 1.4426950408889634f;
     a.cu = cu; a.pl = pl; a.err = err;
     a.lse = lse; a.dsum = dsum; a.dk32 = dk32; a.dv32 = dv32;
+    a.nqs = nqs; a.split = split;
     char *w = static_cast<char *>(ws);
     const size_t ab = align_up(sizeof(int32_t) * (size_t)(batch + 1));
     int32_t *ks_off = reinterpret_cast<int32_t *>(w), *kt_off = reinterpret_cast<int32_t *>(w + ab);
@@ -902,18 +943,22 @@ int launch_prefill_bwd_tc(const ksa_params *p, int batch, const int32_t *cu, int
     if (max_tiles > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
     a.ks_off = ks_off; a.kt_off = kt_off; a.item_off = item_off; a.max_tiles = (int)max_tiles;
     bt::bt_plan_kernel<<<1, 1024, 0, st>>>(a, ks_off, kt_off, item_off);
-    // CTAs: at most one per key tile plus G nq / kSplit per tile; a summary
+    // CTAs: at most one per key tile plus G nq / split per tile; a summary
     // tile's queries number at most total_text, a text tile's 128 + (w+1) k
     const int64_t ns_tiles = (total_text / kk) / bt::BK + batch, nt_tiles = total_text / bt::BK + batch;
     const int64_t G = a.G;
-    const int64_t q_sum = (total_text + bt::BQ - 1) / bt::BQ + 1;
-    const int64_t q_txt = (bt::BK + (int64_t)(p->w + 1) * kk + bt::BQ - 1) / bt::BQ + 1;
-    const int64_t grid = ns_tiles * (1 + (G * q_sum) / bt::kSplit) + nt_tiles * (1 + (G * q_txt) / bt::kSplit);
+    const int64_t q_sum = (total_text + nqs - 1) / nqs + 1;
+    const int64_t q_txt = (bt::BK + (int64_t)(p->w + 1) * kk + nqs - 1) / nqs + 1;
+    const int64_t grid = ns_tiles * (1 + (G * q_sum) / split) + nt_tiles * (1 + (G * q_txt) / split);
     if (grid > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
     if (grid == 0) return KSA_OK;
     const int64_t grid_q = nt_tiles;   // query tiles of 128 text positions (CTAs past the real count exit)
     __nv_bfloat16 *dqb = static_cast<__nv_bfloat16 *>(dq);
-    const int r = d == 128 ? bt_launch<128>(a, grid, grid_q, dqb, st) : bt_launch<64>(a, grid, grid_q, dqb, st);
+    int r;
+    if (nqs == 64)
+        r = d == 128 ? bt_launch<128, 64>(a, grid, grid_q, dqb, st) : bt_launch<64, 64>(a, grid, grid_q, dqb, st);
+    else
+        r = d == 128 ? bt_launch<128, 128>(a, grid, grid_q, dqb, st) : bt_launch<64, 128>(a, grid, grid_q, dqb, st);
     if (r != KSA_OK) return r;
     return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
 }

@@ -1,0 +1,368 @@
+"""Discrete-event models of the mbarrier protocols of the tensor-core kernels
+(csrc/prefill_sm100.cu prefill_kernel, csrc/prefill_bwd_sm100.cu
+bt_dkv_kernel and bq_dq_kernel), checked for deadlock and for parity aliasing
+under many random interleavings.
+
+Each role of a kernel (TMA producers, MMA issuers, elementwise and epilogue
+warps) is restated as the sequence of its waits, arrivals and MMA commits, in
+the kernel's order.  The engine follows PTX semantics:
+  * an mbarrier completes a phase when its expected arrival count is reached;
+  * mbarrier.try_wait.parity(P) succeeds iff the number of completed phases
+    has the other parity than P, so a waiter for phase p that is two phases
+    behind the barrier succeeds wrongly (flagged as aliasing) and one that is
+    two phases ahead hangs (a deadlock);
+  * a TMA load arrives on its barrier some time after it is issued;
+  * tcgen05.commit arrives once every MMA its thread issued before it has
+    completed; each issuing thread's MMAs complete in issue order.
+A mutation test checks that the engine catches a protocol bug of this kind.
+"""
+import random
+
+import pytest
+
+
+class _Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.done = count, 0, 0
+
+    def arrive(self):
+        self.pending += 1
+        if self.pending == self.count:
+            self.pending, self.done = 0, self.done + 1
+
+
+def _simulate(bars, roles, seed, max_rounds=400000):
+    """roles: name -> generator yielding ("wait", bar, phase), ("arrive", bar),
+    ("load", bar) (a TMA load completing later on bar) or ("mma", issuer) /
+    ("commit", issuer, bar).  Returns (status, stuck waits, aliasing events)."""
+    rng = random.Random(seed)
+    B = {name: _Bar(count) for name, count in bars.items()}
+    aliasing, loads, mma = [], [], {}
+    cur = {k: None for k in roles}
+    done = set()
+
+    def wait_ok(name, p):
+        d = B[name].done
+        ok = (d & 1) != (p & 1)
+        if ok and d < p + 1:
+            aliasing.append((name, p, d))
+        return ok
+
+    for _ in range(max_rounds):
+        if len(done) == len(roles):
+            return "ok", None, aliasing
+        progressed = False
+        order = list(roles) + ["loads"] + ["mma:" + k for k in mma]
+        rng.shuffle(order)
+        for c in order:
+            if c == "loads":
+                if loads and rng.random() < 0.5:
+                    B[loads.pop(0)].arrive()
+                    progressed = True
+            elif c.startswith("mma:"):
+                q = mma[c[4:]]
+                if q and rng.random() < 0.5:
+                    e = q.pop(0)
+                    if e is not None:
+                        B[e].arrive()
+                    progressed = True
+            elif c not in done:
+                while True:
+                    if cur[c] is None:
+                        try:
+                            cur[c] = next(roles[c])
+                        except StopIteration:
+                            done.add(c)
+                            break
+                    a = cur[c]
+                    if a[0] == "wait":
+                        if not wait_ok(a[1], a[2]):
+                            break
+                    elif a[0] == "arrive":
+                        B[a[1]].arrive()
+                    elif a[0] == "load":
+                        loads.append(a[1])
+                    elif a[0] == "mma":
+                        mma.setdefault(a[1], []).append(None)
+                    elif a[0] == "commit":
+                        mma.setdefault(a[1], []).append(a[2])
+                    cur[c] = None
+                    progressed = True
+        if not progressed and not loads and not any(mma.values()):
+            return "deadlock", {k: cur[k] for k in roles if k not in done}, aliasing
+    return "timeout", None, aliasing
+
+
+# ---------------------------------------------------------------- prefill_kernel
+def _prefill_roles(tiles, rescale_rng):
+    """tiles[n]: K/V tiles of work item n.  Two S buffers, two Q, K, V stages;
+    softmax halves h = 0, 1; the epilogue warpgroup releases O (B_OFREE)."""
+    NS = QS = KS = VS = 2
+    bars = {"OFREE": 1, "UDONE": 2}
+    for i in range(2):
+        bars.update({f"QF{i}": 1, f"QE{i}": 1, f"KF{i}": 1, f"KE{i}": 1, f"VF{i}": 1, f"VE{i}": 1,
+                     f"S{i}": 1, f"P0_{i}": 1, f"P1_{i}": 1, f"O{i}": 1})
+
+    def tma_qk():
+        gt = 0
+        for n, T in enumerate(tiles):
+            if n >= QS:
+                yield ("wait", f"QE{n % QS}", n // QS - 1)
+            yield ("load", f"QF{n % QS}")
+            for _ in range(T):
+                if gt >= KS:
+                    yield ("wait", f"KE{gt % KS}", gt // KS - 1)
+                yield ("load", f"KF{gt % KS}")
+                gt += 1
+
+    def tma_v():
+        gt = 0
+        for T in tiles:
+            for _ in range(T):
+                if gt >= VS:
+                    yield ("wait", f"VE{gt % VS}", gt // VS - 1)
+                yield ("load", f"VF{gt % VS}")
+                gt += 1
+
+    def qk():
+        gt = 0
+        for n, T in enumerate(tiles):
+            yield ("wait", f"QF{n % QS}", n // QS)
+            for _ in range(T):
+                bf = gt % NS
+                yield ("wait", f"KF{gt % KS}", gt // KS)
+                if gt >= NS:
+                    yield ("wait", f"O{bf}", (gt - NS) // NS)   # S buffer free: PV two tiles back done
+                yield ("mma", "qk")
+                yield ("commit", "qk", f"S{bf}")
+                yield ("commit", "qk", f"KE{gt % KS}")
+                gt += 1
+            yield ("commit", "qk", f"QE{n % QS}")
+
+    def pv():
+        gt = 0
+        for n, T in enumerate(tiles):
+            for j in range(T):
+                bf = gt % NS
+                yield ("wait", f"VF{gt % VS}", gt // VS)
+                if j == 0 and n > 0:
+                    yield ("wait", "OFREE", n - 1)
+                for h in range(2):
+                    yield ("wait", f"P{h}_{bf}", gt // NS)
+                    yield ("mma", "pv")
+                yield ("commit", "pv", f"O{bf}")
+                yield ("commit", "pv", f"VE{gt % VS}")
+                gt += 1
+
+    def softmax(h):
+        gt = 0
+        for n, T in enumerate(tiles):
+            for j in range(T):
+                yield ("wait", f"S{gt % NS}", gt // NS)
+                if j > 0 and rescale_rng.random() < 0.3:   # the lazy rescale reads O after the last PV
+                    yield ("wait", f"O{(gt - 1) % NS}", (gt - 1) // NS)
+                yield ("arrive", f"P{h}_{gt % NS}")
+                gt += 1
+            if n > 0:
+                yield ("wait", "OFREE", n - 1)   # exchange buffer read by the last epilogue
+            yield ("arrive", "UDONE")
+
+    def epilogue():
+        gt = 0
+        for n, T in enumerate(tiles):
+            gt += T
+            yield ("wait", "UDONE", n)
+            yield ("wait", f"O{(gt - 1) % NS}", (gt - 1) // NS)
+            yield ("arrive", "OFREE")
+
+    roles = {"tma_qk": tma_qk(), "tma_v": tma_v(), "qk": qk(), "pv": pv(), "s0": softmax(0), "s1": softmax(1),
+             "epi": epilogue()}
+    return bars, roles
+
+
+def _cases(seed, n_cases, max_items, max_len):
+    rng = random.Random(seed)
+    return [[1], [2], [1, 1], [3, 1, 2]] + [[rng.randint(1, max_len) for _ in range(rng.randint(1, max_items))]
+                                            for _ in range(n_cases)]
+
+
+def test_prefill_kernel_protocol():
+    for items in _cases(3, 30, 6, 6):
+        for seed in range(25):
+            bars, roles = _prefill_roles(items, random.Random(seed + 1000))
+            status, stuck, aliasing = _simulate(bars, roles, seed)
+            assert status == "ok" and not aliasing, (items, seed, status, stuck, aliasing)
+
+
+# ---------------------------------------------------------------- bt_dkv_kernel
+def _dkv_roles(n, nbuf, qs):
+    bars = {"KV": 1, "DV": 1, "DK": 1, "DRAIN": 2}
+    for s in range(qs):
+        bars.update({f"QT{s}": 1, f"QF{s}": 1, f"QE{s}": 2})
+    for b in range(nbuf):
+        bars.update({f"S{b}": 1, f"DP{b}": 1, f"P{b}": 1, f"DS{b}": 1})
+
+    def tma():
+        yield ("load", "KV")
+        for s in range(n):
+            if s >= qs:
+                yield ("wait", f"QE{s % qs}", s // qs - 1)
+            yield ("load", f"QT{s % qs}")
+
+    def loader():
+        for s in range(n):
+            yield ("wait", f"QT{s % qs}", s // qs)
+            yield ("arrive", f"QF{s % qs}")
+
+    def issuer(side):
+        prod, inp, acc = ("S", "P", "DV") if side == "p" else ("DP", "DS", "DK")
+        yield ("wait", "KV", 0)
+        for t in range(n + nbuf - 1):
+            if t < n:
+                yield ("wait", f"QF{t % qs}", t // qs)
+                if t >= nbuf:
+                    yield ("wait", acc, t - nbuf)   # buffer free: this side's accumulation nbuf steps back
+                yield ("mma", side)
+                yield ("commit", side, f"{prod}{t % nbuf}")
+            s = t - (nbuf - 1)
+            if s >= 0:
+                yield ("wait", f"{inp}{s % nbuf}", s // nbuf)
+                yield ("mma", side)
+                yield ("commit", side, acc)
+                yield ("commit", side, f"QE{s % qs}")
+        yield ("commit", side, "DRAIN")
+
+    def elementwise():
+        for s in range(n):
+            b = s % nbuf
+            yield ("wait", f"QF{s % qs}", s // qs)
+            yield ("wait", f"S{b}", s // nbuf)
+            yield ("arrive", f"P{b}")
+            yield ("wait", f"DP{b}", s // nbuf)
+            yield ("arrive", f"DS{b}")
+        yield ("wait", "DRAIN", 0)
+
+    return bars, {"tma": tma(), "ld": loader(), "p": issuer("p"), "d": issuer("d"), "ew": elementwise()}
+
+
+@pytest.mark.parametrize("nbuf,qs", [(2, 4), (1, 2)], ids=["64-query steps, two buffers", "128-query steps"])
+def test_dkv_kernel_protocol(nbuf, qs):
+    for n in range(1, 13):
+        for seed in range(40):
+            bars, roles = _dkv_roles(n, nbuf, qs)
+            status, stuck, aliasing = _simulate(bars, roles, seed)
+            assert status == "ok" and not aliasing, (n, seed, status, stuck, aliasing)
+
+
+# ---------------------------------------------------------------- bq_dq_kernel
+def _dq_roles(items, boundary_bug=False):
+    """items[n]: key-tile steps of the n-th query tile a CTA walks (the kernel
+    takes one; the persistent form, several, with Q/dO and dQ handed over
+    between tiles)."""
+    KST, VST = 3, 2
+    bars = {"Q": 1, "QFREE": 2, "S": 1, "SC": 1, "DP": 1, "DS": 1, "DQ": 1, "DQDONE": 1, "DQFREE": 1, "DRAIN": 2}
+    for s in range(KST):
+        bars.update({f"KF{s}": 1, f"KE{s}": 1})
+    for s in range(VST):
+        bars.update({f"VF{s}": 1, f"VE{s}": 1})
+    state = {"gj": 0}
+
+    def tma():
+        gj = 0
+
+        def load_kv():
+            nonlocal gj
+            if gj >= KST:
+                yield ("wait", f"KE{gj % KST}", gj // KST - 1)
+            yield ("load", f"KF{gj % KST}")
+            if gj >= VST:
+                yield ("wait", f"VE{gj % VST}", gj // VST - 1)
+            yield ("load", f"VF{gj % VST}")
+            gj += 1
+        for n, ns in enumerate(items):
+            yield from load_kv()
+            if n > 0:
+                yield ("wait", "QFREE", n - 1)
+            yield ("load", "Q")
+            for _ in range(1, ns):
+                yield from load_kv()
+
+    def issuer_s():
+        gj = 0
+        for n, ns in enumerate(items):
+            yield ("wait", "Q", n)
+            for _ in range(ns):
+                yield ("wait", f"KF{gj % KST}", gj // KST)
+                if gj > 0:
+                    yield ("wait", "SC", gj - 1)
+                yield ("mma", "a")
+                yield ("commit", "a", "S")
+                gj += 1
+            yield ("commit", "a", "QFREE")
+        yield ("commit", "a", "DRAIN")
+
+    def issuer_dp_dq():
+        gj = 0
+
+        def dq(x, first, n):
+            if first and n > 0:
+                yield ("wait", "DQFREE", n - 1)
+            yield ("mma", "b")
+            yield ("commit", "b", "DQ")
+            yield ("commit", "b", f"KE{x % KST}")
+        for n, ns in enumerate(items):
+            yield ("wait", "Q", n)
+            for j in range(ns):
+                yield ("wait", f"VF{gj % VST}", gj // VST)
+                if gj > 0:
+                    yield ("wait", "DS", gj - 1)
+                if j == 0 and gj > 0 and not boundary_bug:
+                    yield ("wait", "DQ", gj - 1)
+                elif gj > 1:
+                    yield ("wait", "DQ", gj - 2)
+                yield ("mma", "b")
+                yield ("commit", "b", "DP")
+                yield ("commit", "b", f"VE{gj % VST}")
+                if j > 0:
+                    yield from dq(gj - 1, j == 1, n)
+                gj += 1
+            yield ("commit", "b", "QFREE")
+            yield ("wait", "DS", gj - 1)
+            yield from dq(gj - 1, ns == 1, n)
+            yield ("commit", "b", "DQDONE")
+        yield ("commit", "b", "DRAIN")
+
+    def elementwise():
+        gj = 0
+        for n, ns in enumerate(items):
+            for _ in range(ns):
+                yield ("wait", "S", gj)
+                yield ("arrive", "SC")
+                yield ("wait", "DP", gj)
+                yield ("arrive", "DS")
+                gj += 1
+            yield ("wait", "DQDONE", n)
+            yield ("arrive", "DQFREE")
+
+    return bars, {"tma": tma(), "a": issuer_s(), "b": issuer_dp_dq(), "ew": elementwise()}
+
+
+def test_dq_kernel_protocol():
+    for items in [[n] for n in range(1, 12)] + _cases(7, 25, 5, 6):
+        for seed in range(30):
+            bars, roles = _dq_roles(items)
+            status, stuck, aliasing = _simulate(bars, roles, seed)
+            assert status == "ok" and not aliasing, (items, seed, status, stuck, aliasing)
+
+
+def test_engine_catches_a_parity_aliasing_bug():
+    """The dq protocol with several query tiles per CTA and the wait for
+    dQ(gj-2) kept at a tile's first step (where the previous tile's last dQ,
+    dQ(gj-1), may already have completed) deadlocks under some interleaving."""
+    failures = 0
+    for items in ([3, 3], [2, 1], [5, 4]):
+        for seed in range(30):
+            bars, roles = _dq_roles(items, boundary_bug=True)
+            status, _, aliasing = _simulate(bars, roles, seed)
+            failures += status != "ok" or bool(aliasing)
+    assert failures > 0

@@ -73,6 +73,25 @@ def decode_slice_rows(m, k, w, fills):
     return np.asarray(fills) + 1 + min(m, w) * k + max(0, m - w)
 
 
+METRIC = "KSA prefill TFLOP/s (useful pairs) & decode KV GB/s"
+
+
+def workload_config(world):
+    """The config of the default bench line, shared by both arms."""
+    from kv_cache_compression_ksa_b200.inputs import uniform_ints
+    sl = PF["seqlens"]
+    fills = uniform_ints(DC["B"], 0, DC["k"] - 1, seed=DC["seed"]).numpy()
+    rows = decode_slice_rows(DC["m"], DC["k"], DC["w"], fills)
+    return {
+        "workload": "prefill 1x32768 text tokens (Qwen3-4B layer: 32q/8kv heads, d128), k8, w8, "
+                    "N(0,1)*0.5 bf16, RoPE 1e6, fp32 LSE; + decode 64 seqs x 131072 prior tokens",
+        "global_batch": world, "seq_len": sl[0], "parallelism": f"replicas x{world}",
+        "l2": "inputs larger than L2 (prefill q_aug 302 MB; decode slice 4.3 GB)",
+        "useful_prefill_tflop": useful_pairs(sl, PF["k"], PF["w"]) * PF["Hq"] * 4 * PF["d"] / 1e12,
+        "decode_slice_gb": float(rows.sum()) * DC["Hkv"] * DC["d"] * 2 * 2 / 1e9,
+    }
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -235,13 +254,14 @@ def run_reference(args, rank, world):
             t_total += dt
     v = float(np.mean(vals))
     line = {
-        "impl": "reference", "metric": "KSA prefill TFLOP/s (useful pairs)", "value": v, "unit": "TFLOP/s",
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_total / max(args.steps, 1) * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "prefill 1x32768 text tokens, 32q/8kv heads, d128, k8, w8 (sampled rows)"},
+        "config": workload_config(world),
         "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{nrows} evenly spaced text rows x 32 heads of the 32768-token prefill"},
+                         "sample": f"{nrows} evenly spaced text rows x 32 heads of the 32768-token prefill "
+                                   "(the prefill leg: the oracle's TFLOP/s on those rows)"},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -415,17 +435,12 @@ def run_ksa(args, rank, world, local):
     clocks = clk.summary()
     if rank == 0:
         line = {
-            "metric": "KSA prefill TFLOP/s (useful pairs) & decode KV GB/s",
+            "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {
-                "workload": "prefill 1x32768 text tokens (Qwen3-4B layer: 32q/8kv heads, d128), k8, w8, "
-                            "N(0,1)*0.5 bf16, RoPE 1e6, fp32 LSE; + decode 64 seqs x 131072 prior tokens",
-                "global_batch": world, "seq_len": sl[0], "parallelism": f"replicas x{world}",
-                "l2": "inputs larger than L2 (prefill q_aug 302 MB; decode slice 4.3 GB)",
-                "useful_prefill_tflop": pf_flops / 1e12, "decode_slice_gb": dec_bytes / 1e9,
-            },
+            "config": dict(workload_config(world), useful_prefill_tflop=pf_flops / 1e12,
+                           decode_slice_gb=dec_bytes / 1e9),
             "prefill": {"ms": pf_ms, "rope_interleave_ms": rope_ms, "tflops": value / world,
                         "frac_of_bf16_peak": (value / world) / tc_peak},
             "decode": {"ms": dec_ms, "append_ms": app_ms, "gbs": dec_gbs / world,

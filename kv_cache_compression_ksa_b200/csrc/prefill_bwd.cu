@@ -9,14 +9,23 @@
 // same mask: P = exp(S - lse), dP = dO V^T, D = rowsum(dO * O),
 // dS = P * (dP - D), dq = scale dS K, dk = scale dS^T Q, dv = P^T dO.
 //
-// Work is cut the way the forward skips tiles: a block holds 64 rows of one
-// kind (64 consecutive text tokens or 64 consecutive summaries of one
-// sequence), and a query block only meets the key blocks its rows can see
-// (summaries 0 .. c_last-w-1 and the text of chunks c_first-w .. c_last), and
-// a key block only the query blocks that can see it.  Inside a pair of blocks
-// the mask is evaluated per element from the rows' coordinates.
+// launch_prefill_bwd runs D = rowsum(dO * O), then, where the shape allows
+// (k divides 128, d of 64 or 128), the tensor-core kernels of
+// prefill_bwd_sm100.cu for the text query rows and bwd_sum_rows_kernel for
+// the summary query rows fused with the fp32 -> bf16 conversion; every other
+// shape runs on the warp-level kernels below.
+//
+// Warp-level path.  Work is cut the way the forward skips tiles: a block
+// holds 64 rows of one kind (64 consecutive text tokens or 64 consecutive
+// summaries of one sequence), and a query block only meets the key blocks its
+// rows can see (summaries 0 .. c_last-w-1 and the text of chunks c_first-w ..
+// c_last), and a key block only the query blocks that can see it.  Inside a
+// pair of blocks the mask is evaluated per element from the rows' coordinates.
 //
 //   bwd_dot_kernel   D = rowsum(dO * O)                          (HBM)
+//   bwd_sum_rows_kernel  tensor-core path: the summary query rows (k+1 keys
+//                    each) on CUDA cores, added into the accumulators as they
+//                    are converted to bf16
 //   bwd_dq_kernel    query-stationary: dq of 64 rows of one q head
 //   bwd_dkv_kernel   key-stationary: dk, dv of 64 rows of one kv head, over
 //                    all q heads of its group and (grid z) a share of at

@@ -3,8 +3,8 @@ Attention Technical Report under the KSA mask, sections 2.2.1-2.2.2) against
 the oracle's fp64 backward, over varlen batches with partial chunks, GQA,
 w = 0, k = 1, a k that does not divide the 128-row tiles of the tensor-core
 kernels (warp-level path), k = 128 (dk/dv steps of 128 queries instead of
-64) and a sequence long enough that the summary key tiles' text queries are
-split over several CTAs.
+64), k = 64 (a dk/dv step is one chunk) and a sequence long enough that the
+summary key tiles' text queries are split over several CTAs.
 
 Tolerance: the kernels feed P and dS to the tensor cores in bf16 (relative
 rounding 2^-9 each) and write bf16 gradients, accumulating in fp32, so the
@@ -33,6 +33,7 @@ CASES = [
     ("k6_warp_path", [200, 50], 6, 2, 8, 2, 128, 19),          # k does not divide 128: warp-level dk/dv
     ("summary_shares", [2600, 300], 8, 1, 8, 2, 128, 23),      # summary key tiles split over several CTAs
     ("k128_steps_of_128", [700, 300], 128, 1, 4, 2, 128, 29),  # k does not divide 64: 128-query dk/dv steps
+    ("k64_one_chunk_steps", [1300, 260], 64, 2, 8, 2, 128, 31),  # a dk/dv step is one chunk of 64 slots
 ]
 
 

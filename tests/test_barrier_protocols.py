@@ -1,7 +1,8 @@
-"""Discrete-event models of the mbarrier protocols of the tensor-core kernels
-(csrc/prefill_sm100.cu prefill_kernel, csrc/prefill_bwd_sm100.cu
-bt_dkv_kernel and bq_dq_kernel), checked for deadlock and for parity aliasing
-under many random interleavings.
+"""Discrete-event models of the barrier protocols of the warp-specialised
+kernels (csrc/prefill_sm100.cu prefill_kernel, csrc/prefill_bwd_sm100.cu
+bt_dkv_kernel and bq_dq_kernel on mbarriers; csrc/mla_decode.cu
+mla_decode_ws_kernel on named barriers), checked for deadlock, parity
+aliasing and mismatched named-barrier use under many random interleavings.
 
 Each role of a kernel (TMA producers, MMA issuers, elementwise and epilogue
 warps) is restated as the sequence of its waits, arrivals and MMA commits, in
@@ -366,3 +367,93 @@ def test_engine_catches_a_parity_aliasing_bug():
             status, _, aliasing = _simulate(bars, roles, seed)
             failures += status != "ok" or bool(aliasing)
     assert failures > 0
+
+
+# ---------------------------------------------------------------- mla_decode_ws_kernel
+def _simulate_named(nblk, seed, skip_p_read_sync=False):
+    """Named barriers (bar.sync / bar.arrive with 384 threads: the QK
+    warpgroup, 128, and the eight PV warps, 256).  A barrier completes a
+    generation when both groups have arrived; bar.sync also waits for that
+    generation.  A group arriving twice in one generation (its next use
+    counted toward the current one) is flagged."""
+    rng = random.Random(seed)
+    gen = {i: 0 for i in range(1, 7)}
+    arrived = {i: set() for i in range(1, 7)}
+    misuse = []
+
+    def arrive(i, who):
+        if who in arrived[i]:
+            misuse.append((i, who, gen[i]))
+        arrived[i].add(who)
+        if arrived[i] == {"qk", "pv"}:
+            arrived[i] = set()
+            gen[i] += 1
+            return gen[i] - 1
+        return gen[i]
+
+    def qk():
+        for kb in range(nblk):
+            bb = kb & 1
+            yield ("sync", 1 + bb)          # block kb landed
+            if kb >= 2 and not skip_p_read_sync:
+                yield ("sync", 5 + bb)      # P buffer bb read by the PV warps (block kb - 2)
+            yield ("arrive", 3 + bb)        # P of block kb ready
+
+    def pv():
+        if nblk > 0:
+            yield ("arrive", 1)             # block 0 landed
+        for kb in range(nblk):
+            bb = kb & 1
+            if kb + 1 < nblk:
+                yield ("arrive", 1 + (bb ^ 1))   # block kb + 1 landed
+            yield ("sync", 3 + bb)          # P of block kb ready
+            if kb + 2 < nblk:
+                yield ("arrive", 5 + bb)    # P buffer bb read
+
+    roles = {"qk": qk(), "pv": pv()}
+    cur = {"qk": None, "pv": None}
+    waiting = {}   # role -> (barrier, generation it waits to complete)
+    done = set()
+    for _ in range(100000):
+        if len(done) == 2:
+            return "ok", misuse
+        progressed = False
+        for who in rng.sample(list(roles), 2):
+            if who in done:
+                continue
+            if who in waiting:
+                i, g = waiting[who]
+                if gen[i] > g:
+                    del waiting[who]
+                    progressed = True
+                continue
+            try:
+                a = next(roles[who])
+            except StopIteration:
+                done.add(who)
+                progressed = True
+                continue
+            g = arrive(a[1], who)
+            if a[0] == "sync" and gen[a[1]] <= g:
+                waiting[who] = (a[1], g)
+            progressed = True
+        if not progressed:
+            return "deadlock", misuse
+    return "timeout", misuse
+
+
+def test_mla_ws_kernel_named_barrier_protocol():
+    for nblk in range(0, 12):
+        for seed in range(40):
+            status, misuse = _simulate_named(nblk, seed)
+            assert status == "ok" and not misuse, (nblk, seed, status, misuse)
+
+
+def test_named_barrier_engine_catches_a_missing_sync():
+    """Without the QK warps' wait for "P buffer read", the PV warps' arrivals
+    pile up on that barrier (two arrivals of one group in a generation)."""
+    flagged = 0
+    for seed in range(20):
+        status, misuse = _simulate_named(6, seed, skip_p_read_sync=True)
+        flagged += status != "ok" or bool(misuse)
+    assert flagged > 0

@@ -36,7 +36,10 @@ PF = dict(seqlens=[32768], k=8, w=8, Hq=32, Hkv=8, d=128, scale=0.5, seed=1, the
 # set to None whenever one of those kernels changes, until it is captured again).
 # The decode capture ran at batch 16; its traffic grows in proportion to the batch.
 TRAFFIC = {
-    "prefill": (661.2e6, "profiles/prefill_kernel_qwen3_4b_32k.md (prefill_kernel<128>)"),
+    # the softmax changed (three-input max, packed fp32 pairs) after the last
+    # capture (661.2 MB of the previous build, profiles/prefill_kernel_qwen3_4b_32k.md)
+    "prefill": (None, "not captured for this build; 661.2 MB for the previous one in "
+                      "profiles/prefill_kernel_qwen3_4b_32k.md (prefill_kernel<128>)"),
     "decode_per_seq": (1.0851e9 / 16, "profiles/decode_split_kernel_b16_m16384.md (batch 16 capture, per sequence)"),
 }
 DC = dict(B=64, m=16384, k=8, w=8, Hq=32, Hkv=8, d=128, seed=3, theta=1e6)

@@ -174,8 +174,9 @@ __device__ __forceinline__ void rope_rot8(uint4 &lo, uint4 &hi, const float *cs,
 }
 
 // Slice of one sequence after its append: [lo, hi) in slots.  Returns false
-// (and records the error) if the state cannot hold a query of this kind.
-__device__ __forceinline__ bool decode_slice(int kind, int64_t n, int64_t m, int k, int w,
+// if the state cannot hold a query of this kind (the caller records the error).
+// Host-callable too, for CPU tests against a reference cache.
+__host__ __device__ __forceinline__ bool decode_slice(int kind, int64_t n, int64_t m, int k, int w,
                                              int64_t *lo, int64_t *hi)
 {
     int64_t f = n - m * k;

@@ -95,12 +95,13 @@ struct TArgs {
     float *dk32, *dv32;
 };
 
-// A key tile and the text query range that sees it.
+// A key tile and the text query range that sees it.  key_tile is
+// host-callable too, for CPU tests of the ranges against the dense mask.
 struct KTile {
     int b, sum, j0, kcnt, n, m, c0, qlo, qhi, nq;   // nq: query tiles of 128 positions
 };
 
-__device__ __forceinline__ int find_off(const int32_t *off, int batch, int id)
+__host__ __device__ __forceinline__ int find_off(const int32_t *off, int batch, int id)
 {
     int lo = 0, hi = batch - 1;
     while (lo < hi) {
@@ -110,7 +111,7 @@ __device__ __forceinline__ int find_off(const int32_t *off, int batch, int id)
     return lo;
 }
 
-__device__ __forceinline__ void key_tile(const TArgs &a, int tile, KTile &T)
+__host__ __device__ __forceinline__ void key_tile(const TArgs &a, int tile, KTile &T)
 {
     const int ns = a.ks_off[a.batch];
     T.sum = tile < ns;

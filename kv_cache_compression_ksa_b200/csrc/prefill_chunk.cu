@@ -95,7 +95,7 @@ __device__ __forceinline__ int find_seq(const int32_t *off, int batch, int id)
 constexpr int kPlanThreads = 1024;
 
 // State checks of sequence b for a block of T tokens and S summaries.
-__device__ __forceinline__ int chunk_state_code(const Args &a, int b, int T, int S, int32_t *n0p, int32_t *m0p)
+__host__ __device__ __forceinline__ int chunk_state_code(const Args &a, int b, int T, int S, int32_t *n0p, int32_t *m0p)
 {
     const int32_t *st = a.state + 4 * (int64_t)b;
     const int32_t n0 = st[0], m0 = st[1];
@@ -107,10 +107,11 @@ __device__ __forceinline__ int chunk_state_code(const Args &a, int b, int T, int
     return KSA_OK;
 }
 
+// (chunk_state_code and chunk_ranges are host-callable too, for CPU tests.)
 // Chunks of the tensor-core path for a valid sequence: query chunks
 // [cbeg, ncb) and window chunks [kvb, ncb), kvb covering both the first
 // query chunk's window and the chunk of the first new summary.
-__device__ __forceinline__ void chunk_ranges(const Args &a, int32_t n0, int32_t m0, int T, int *cbeg, int *kvb,
+__host__ __device__ __forceinline__ void chunk_ranges(const Args &a, int32_t n0, int32_t m0, int T, int *cbeg, int *kvb,
                                              int *ncb)
 {
     const int64_t n1 = (int64_t)n0 + T;

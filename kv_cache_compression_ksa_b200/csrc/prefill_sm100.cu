@@ -133,12 +133,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) { retu
 // G q heads of one kv head, starting at q head h0, for unit_chunks chunks)
 // and its list of 128-key K/V tiles: the window tiles covering chunks
 // c0-w .. cend-1, then the summary tiles.  When G k > 128 the G heads are
-// split over G / Gp items, each loading the same K/V tiles.
+// split over G / Gp items, each loading the same K/V tiles.  unit_of is
+// host-callable too, so that CPU tests can check the tile lists it yields
+// against the dense mask.
 struct Unit {
     int hkv, h0, b, nb, mb, ncb, qbase, kvbase, sbase, c0, cend, cw_lo, n_win, T;
 };
 
-__device__ __forceinline__ Unit unit_of(const Params &P, int item, int n_units)
+__host__ __device__ __forceinline__ Unit unit_of(const Params &P, int item, int n_units)
 {
     Unit U;
     const int per = P.Hkv * P.HP;

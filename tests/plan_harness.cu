@@ -1,0 +1,213 @@
+// plan_harness.cu -- a host build of the CUDA library's work decomposition,
+// for CPU tests of its tile lists against the KSA mask.
+//
+// The library's sources are compiled into this program whole, so the
+// functions under test are the kernels' own, marked __host__ __device__:
+//   pf::unit_of           the forward's work items and their K/V tiles
+//                         (plain prefill and chunk mode),
+//   bt::key_tile          the backward's key tiles and the text query range
+//                         that sees each,
+//   ck::chunk_state_code, ck::chunk_ranges, ck::layout
+//                         the chunked prefill's state checks, gathered
+//                         chunk ranges and buffer sizes,
+//   decode_slice          the live cache slots of a decode query.
+// Only the prefix sums that the plan kernels compute on the device (one
+// scan per array) are written out here, as plain loops, together with the
+// per-call constants the launch functions set (Gp, Tc, Tk).
+//
+// Input: one query per line on stdin.  Output: integer lines, each query's
+// block closed by a line "end".
+//   fwd   k w Hq Hkv B n_0 .. n_{B-1}
+//         "W Gp HP Tc Tk", then per work item
+//         "hkv h0 b nb mb ncb qbase kvbase sbase c0 cend cw_lo n_win T"
+//   chunk k w Hq Hkv B (n0 m0 T)_0 .. (n0 m0 T)_{B-1}
+//         per sequence "code cbeg kvb ncb qoff kvoff"; then
+//         "sum_q sum_kv units L.q_chunks L.kv_chunks L.max_units sum_slot0";
+//         then the work items as for fwd
+//   bwd   k w Hq Hkv nqs B n_0 .. n_{B-1}
+//         "ns nt", then per key tile "b sum j0 kcnt n m c0 qlo qhi nq"
+//   slice k w kind n m
+//         "ok lo hi"
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../kv_cache_compression_ksa_b200/csrc/prefill_sm100.cu"
+#include "../kv_cache_compression_ksa_b200/csrc/prefill_bwd_sm100.cu"
+#include "../kv_cache_compression_ksa_b200/csrc/prefill_chunk.cu"
+
+namespace ksa {
+int sm_count() { return 148; }   // the launch functions are not called here
+}
+
+using namespace ksa;
+
+static ksa_params params(int k, int w, int Hq, int Hkv)
+{
+    ksa_params p;
+    std::memset(&p, 0, sizeof(p));
+    p.k = k; p.w = w; p.num_q_heads = Hq; p.num_kv_heads = Hkv; p.head_dim = 128;
+    return p;
+}
+
+// Per-call constants of the forward, as the launch functions set them.
+static bool fwd_consts(const ksa_params &p, pf::Params &P)
+{
+    std::memset(&P, 0, sizeof(P));
+    const int G = p.num_q_heads / p.num_kv_heads;
+    P.k = p.k; P.w = p.w; P.G = G; P.Hq = p.num_q_heads; P.Hkv = p.num_kv_heads;
+    P.Gp = prefill_heads_per_tile(&p);
+    if (P.Gp < 1) return false;
+    P.HP = G / P.Gp;
+    P.Tc = pf::BM / (P.Gp * p.k);
+    P.Tk = pf::BN / p.k;
+    if (P.Tc < 1 || P.Tk < 1) return false;
+    P.unit_chunks = P.Tc;
+    return true;
+}
+
+static void print_items(const pf::Params &P, int n_units)
+{
+    const int W = n_units * P.Hkv * P.HP;
+    std::printf("%d %d %d %d %d\n", W, P.Gp, P.HP, P.Tc, P.Tk);
+    for (int item = 0; item < W; ++item) {
+        const pf::Unit U = pf::unit_of(P, item, n_units);
+        std::printf("%d %d %d %d %d %d %d %d %d %d %d %d %d %d\n", U.hkv, U.h0, U.b, U.nb, U.mb, U.ncb, U.qbase,
+                    U.kvbase, U.sbase, U.c0, U.cend, U.cw_lo, U.n_win, U.T);
+    }
+}
+
+static void run_fwd(int k, int w, int Hq, int Hkv, const std::vector<int> &n)
+{
+    const ksa_params p = params(k, w, Hq, Hkv);
+    pf::Params P;
+    if (!fwd_consts(p, P)) { std::printf("unsupported\n"); return; }
+    const int B = (int)n.size();
+    std::vector<int32_t> cu(B + 1, 0), chunk_off(B + 1, 0), tile_off(B + 1, 0);
+    for (int b = 0; b < B; ++b) {
+        const int c = (n[b] + k - 1) / k;
+        cu[b + 1] = cu[b] + n[b];
+        chunk_off[b + 1] = chunk_off[b] + c;
+        tile_off[b + 1] = tile_off[b] + (c + P.unit_chunks - 1) / P.unit_chunks;
+    }
+    P.batch = B;
+    P.cu = cu.data();
+    P.pl.chunk_off = chunk_off.data();
+    P.pl.tile_off = tile_off.data();
+    print_items(P, tile_off[B]);
+}
+
+static void run_chunk(int k, int w, int Hq, int Hkv, const std::vector<int> &trip)
+{
+    const ksa_params p = params(k, w, Hq, Hkv);
+    const int B = (int)trip.size() / 3;
+    const int64_t cap = 1 << 20;
+    ck::Args a;
+    std::memset(&a, 0, sizeof(a));
+    a.k = k; a.w = w; a.Hq = Hq; a.Hkv = Hkv; a.G = Hq / Hkv; a.batch = B; a.d = 128;
+    a.cap = cap;
+    a.S = 1 + (int64_t)k + (int64_t)w * k + cap;
+    a.uc = ck::tc_unit_chunks(&p);
+    std::vector<int32_t> state(4 * B, 0);
+    int64_t total_t = 0, total_s = 0;
+    std::vector<int> T(B), S(B);
+    for (int b = 0; b < B; ++b) {
+        const int n0 = trip[3 * b], m0 = trip[3 * b + 1];
+        T[b] = trip[3 * b + 2];
+        state[4 * b] = n0;
+        state[4 * b + 1] = m0;
+        const int64_t f0 = (int64_t)n0 - (int64_t)m0 * k;
+        S[b] = f0 >= 0 ? (int)((f0 + T[b]) / k) : 0;   // the summaries the block completes
+        total_t += T[b];
+        total_s += S[b];
+    }
+    a.state = state.data();
+    pf::Params P;
+    if (a.uc < 1 || !fwd_consts(p, P)) { std::printf("unsupported\n"); return; }
+    std::vector<int32_t> cbeg(B), ntot(B), qbase(B), kvbase(B), uoff(B + 1, 0);
+    int32_t oq = 0, okv = 0;
+    for (int b = 0; b < B; ++b) {
+        int32_t n0, m0;
+        const int code = ck::chunk_state_code(a, b, T[b], S[b], &n0, &m0);
+        int cb = 0, kb = 0, nc = 0;
+        if (code == KSA_OK && T[b] > 0) ck::chunk_ranges(a, n0, m0, T[b], &cb, &kb, &nc);
+        std::printf("%d %d %d %d %d %d\n", code, cb, kb, nc, oq, okv);
+        cbeg[b] = cb; ntot[b] = n0 + T[b];
+        qbase[b] = oq - cb; kvbase[b] = okv - kb;
+        uoff[b + 1] = uoff[b];
+        if (code == KSA_OK && T[b] > 0) {
+            uoff[b + 1] += (nc - cb + a.uc - 1) / a.uc;
+            oq += nc - cb;
+            okv += nc - kb;
+        }
+    }
+    const ck::Layout L = ck::layout(&p, B, total_t, total_s);
+    P.batch = B;
+    P.ck_tile_off = uoff.data(); P.ck_cbeg = cbeg.data(); P.ck_ntot = ntot.data();
+    P.ck_qbase = qbase.data(); P.ck_kvbase = kvbase.data();
+    P.sum_slot0 = 1 + k + w * k;
+    std::printf("%d %d %d %lld %lld %lld %d\n", oq, okv, uoff[B], (long long)L.q_chunks, (long long)L.kv_chunks,
+                (long long)L.max_units, P.sum_slot0);
+    print_items(P, uoff[B]);
+}
+
+static void run_bwd(int k, int w, int Hq, int Hkv, int nqs, const std::vector<int> &n)
+{
+    const int B = (int)n.size();
+    std::vector<int32_t> cu(B + 1, 0), chunk_off(B + 1, 0), ks_off(B + 1, 0), kt_off(B + 1, 0);
+    for (int b = 0; b < B; ++b) {
+        cu[b + 1] = cu[b] + n[b];
+        chunk_off[b + 1] = chunk_off[b] + (n[b] + k - 1) / k;
+        ks_off[b + 1] = ks_off[b] + (n[b] / k + bt::BK - 1) / bt::BK;
+        kt_off[b + 1] = kt_off[b] + (n[b] + bt::BK - 1) / bt::BK;
+    }
+    bt::TArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.k = k; a.w = w; a.G = Hq / Hkv; a.Hq = Hq; a.Hkv = Hkv; a.batch = B;
+    a.cu = cu.data();
+    a.pl.chunk_off = chunk_off.data();
+    a.ks_off = ks_off.data();
+    a.kt_off = kt_off.data();
+    a.nqs = nqs;
+    const int ns = ks_off[B], nt = kt_off[B];
+    std::printf("%d %d\n", ns, nt);
+    for (int t = 0; t < ns + nt; ++t) {
+        bt::KTile T;
+        bt::key_tile(a, t, T);
+        std::printf("%d %d %d %d %d %d %d %d %d %d\n", T.b, T.sum, T.j0, T.kcnt, T.n, T.m, T.c0, T.qlo, T.qhi, T.nq);
+    }
+}
+
+int main()
+{
+    char line[1 << 16];
+    while (std::fgets(line, sizeof(line), stdin)) {
+        char mode[16] = {0};
+        int off = 0;
+        if (std::sscanf(line, "%15s%n", mode, &off) != 1) continue;
+        std::vector<long long> v;
+        const char *s = line + off;
+        long long x;
+        int used;
+        while (std::sscanf(s, "%lld%n", &x, &used) == 1) { v.push_back(x); s += used; }
+        const std::string m(mode);
+        auto ints = [&](size_t from) { return std::vector<int>(v.begin() + from, v.end()); };
+        if (m == "fwd" && v.size() >= 5 && v.size() == 5 + (size_t)v[4]) {
+            run_fwd((int)v[0], (int)v[1], (int)v[2], (int)v[3], ints(5));
+        } else if (m == "chunk" && v.size() >= 5 && v.size() == 5 + 3 * (size_t)v[4]) {
+            run_chunk((int)v[0], (int)v[1], (int)v[2], (int)v[3], ints(5));
+        } else if (m == "bwd" && v.size() >= 6 && v.size() == 6 + (size_t)v[5]) {
+            run_bwd((int)v[0], (int)v[1], (int)v[2], (int)v[3], (int)v[4], ints(6));
+        } else if (m == "slice" && v.size() == 5) {
+            int64_t lo = 0, hi = 0;
+            const bool ok = decode_slice((int)v[2], v[3], v[4], (int)v[0], (int)v[1], &lo, &hi);
+            std::printf("%d %lld %lld\n", ok ? 1 : 0, (long long)lo, (long long)hi);
+        } else {
+            std::printf("bad query\n");
+        }
+        std::printf("end\n");
+        std::fflush(stdout);
+    }
+    return 0;
+}

@@ -1,0 +1,320 @@
+"""CPU checks of the CUDA library's work decomposition against the KSA mask.
+
+The block-sparse kernels never look at the L x L mask: each one derives its
+list of tiles from chunk coordinates.  The parity tests on the GPU show that
+the outputs are right; a tile list that reads a tile too many still passes
+them.  These tests run the kernels' own index functions, compiled for the
+host (tests/plan_harness.cu), over many shapes, and check each list against
+the oracle's dense mask:
+  - every row (sequence, q head, text token) belongs to exactly one work item;
+  - every key that a row of a work item sees lies in one of its tiles;
+  - every tile holds at least one key that some row of the item sees, so no
+    fully masked tile is ever loaded or multiplied ("Kwai Summary Attention
+    Technical Report", section 2.3 "Kernel Design": only block pairs the mask
+    does not zero out entirely are computed);
+  - the backward's key tiles split the keys, and the text query range of
+    each tile is exactly the span of the queries that see it;
+  - the chunked prefill's gathered buffers hold what its work items read,
+    within the sizes the workspace reserves;
+  - the decode's live slots match the oracle's cache (section 2.3.1,
+    Figure 4) in every reachable state, and unreachable states are refused.
+The visibility rule is section 2.2.1 (summaries) and section 2.2.2,
+Eqs. (2)-(3) (text).
+"""
+from __future__ import annotations
+
+import functools
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "plan_harness.cu")
+BM = BN = BK = 128   # query-tile rows, K/V-tile keys (forward), key-tile keys (backward)
+TEXT, SUMMARY = 0, 1
+
+
+@pytest.fixture(scope="module")
+def harness(tmp_path_factory):
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not found")
+    exe = str(tmp_path_factory.mktemp("plan") / "plan_harness")
+    # PTX only: the kernels are compiled along with the host code, never run
+    subprocess.check_call([nvcc, "-gencode", "arch=compute_100a,code=compute_100a", "-std=c++17", "-O1",
+                           "-o", exe, SRC])
+    proc = subprocess.Popen([exe], stdin=subprocess.PIPE, stdout=subprocess.PIPE, text=True)
+
+    def query(*words):
+        proc.stdin.write(" ".join(str(x) for x in words) + "\n")
+        proc.stdin.flush()
+        rows = []
+        while True:
+            line = proc.stdout.readline()
+            assert line, "harness exited"
+            line = line.strip()
+            if line == "end":
+                return rows
+            assert line not in ("bad query", "unsupported"), (words, line)
+            rows.append([int(x) for x in line.split()])
+
+    yield query
+    proc.stdin.close()
+    proc.wait(timeout=30)
+
+
+# ---------------------------------------------------------------------------
+# The mask, as [text query, text key] and [text query, summary] booleans
+# ---------------------------------------------------------------------------
+@functools.lru_cache(maxsize=None)
+def text_views(n: int, k: int, w: int):
+    m = n // k
+    M = oracle.dense_mask(n, k, w).astype(bool)
+    t = np.arange(n)
+    pt = (t // k) * (k + 1) + t % k          # Eq. (1) position of text token t
+    ps = np.arange(m) * (k + 1) + k          # and of summary s_j
+    return M[np.ix_(pt, pt)], M[np.ix_(pt, ps)]
+
+
+def offsets(counts):
+    return np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+
+
+# ---------------------------------------------------------------------------
+# Forward work items
+# ---------------------------------------------------------------------------
+FIELDS = ("hkv", "h0", "b", "nb", "mb", "ncb", "qbase", "kvbase", "sbase", "c0", "cend", "cw_lo", "n_win", "T")
+
+
+def check_items(rows, k, w, Hq, Hkv, seq, row_lo=None):
+    """Checks the work items printed by the harness.  seq[b] = (ntot, first
+    query chunk, first window chunk held or None, q-buffer / window-buffer
+    chunk bases or None); row_lo[b]: the first row the call must produce."""
+    W, Gp, HP, Tc, Tk = rows[0]
+    items = [dict(zip(FIELDS, r)) for r in rows[1:]]
+    G = Hq // Hkv
+    assert len(items) == W
+    assert Gp * HP == G and Gp * k * Tc <= BM and Tk == BN // k
+    assert Gp == min(G, BM // k) and Tc == BM // (Gp * k)
+    covered = {}
+    for it in items:
+        b = it["b"]
+        ntot, cbeg, kvb, bases = seq[b]
+        n, m, ncb = ntot, ntot // k, -(-ntot // k)
+        assert (it["nb"], it["mb"], it["ncb"]) == (n, m, ncb)
+        if bases is not None:
+            assert (it["qbase"], it["kvbase"]) == bases
+        assert it["hkv"] * G <= it["h0"] and it["h0"] + Gp <= (it["hkv"] + 1) * G
+        assert (it["h0"] - it["hkv"] * G) % Gp == 0
+        c0, cend = it["c0"], it["cend"]
+        assert cbeg <= c0 < cend <= ncb and cend - c0 <= Tc
+        assert (c0 - cbeg) % Tc == 0 and (cend == c0 + Tc or cend == ncb)
+        for h in range(it["h0"], it["h0"] + Gp):
+            for c in range(c0, cend):
+                key = (b, h, c)
+                assert key not in covered, ("row covered twice", key)
+                covered[key] = True
+        # keys the item's rows see, against its tiles
+        vt, vs = text_views(n, k, w)
+        r0, r1 = c0 * k, min(cend * k, n)
+        seen_t = np.flatnonzero(vt[r0:r1].any(axis=0))
+        seen_s = np.flatnonzero(vs[r0:r1].any(axis=0))
+        cw_lo, n_win, T = it["cw_lo"], it["n_win"], it["T"]
+        assert cw_lo == max(0, c0 - w)
+        if kvb is not None:
+            assert cw_lo >= kvb, "a window tile starts before the chunks the buffer holds"
+            assert seen_t.size == 0 or (seen_t[0] >= kvb * k and seen_t[-1] < ncb * k)
+        lo, hi = cw_lo * k, (cw_lo + n_win * Tk) * k
+        assert seen_t.size and seen_t[0] >= lo and seen_t[-1] < hi, "a visible text key outside the window tiles"
+        for j in range(n_win):
+            a, z = lo + j * Tk * k, lo + (j + 1) * Tk * k
+            assert np.any((seen_t >= a) & (seen_t < z)), ("fully masked window tile", it, j)
+        n_sum = T - n_win
+        assert n_sum >= 0
+        assert seen_s.size == 0 or seen_s[-1] < n_sum * BN, "a visible summary outside the summary tiles"
+        if seen_s.size:
+            assert seen_s[0] == 0 and seen_s.size == seen_s[-1] + 1   # a prefix s_0 .. s_{ns-1}
+        for j in range(n_sum):
+            assert np.any((seen_s >= j * BN) & (seen_s < (j + 1) * BN)), ("fully masked summary tile", it, j)
+    # every (sequence, q head, chunk) the call must produce
+    for b, (ntot, cbeg, _, _) in enumerate(seq):
+        ncb = -(-ntot // k)
+        first = cbeg if row_lo is None else row_lo[b] // k
+        for h in range(Hq):
+            for c in range(first, ncb):
+                assert (b, h, c) in covered, ("row not covered", b, h, c)
+    return items
+
+
+def fwd_case(harness, k, w, Hq, Hkv, seqlens):
+    rows = harness("fwd", k, w, Hq, Hkv, len(seqlens), *seqlens)
+    coff = offsets([-(-n // k) for n in seqlens])
+    seq = [(n, 0, None, (int(coff[b]), int(coff[b]))) for b, n in enumerate(seqlens)]
+    items = check_items(rows, k, w, Hq, Hkv, seq)
+    for it in items:
+        assert it["sbase"] == it["qbase"]
+    return items
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 5, 8, 12, 16, 24, 32, 64, 100, 128])
+@pytest.mark.parametrize("w", [0, 1, 2, 5, 16])
+def test_forward_items_cover_the_mask_and_skip_masked_tiles(harness, k, w):
+    rng = np.random.default_rng(1000 * k + w)
+    Hq, Hkv = [(8, 8), (16, 8), (32, 8), (64, 4)][(k + w) % 4]
+    lens = [int(x) for x in rng.integers(1, 700 if k > 2 else 300, size=3)] + [k, k + 1, max(k - 1, 1)]
+    fwd_case(harness, k, w, Hq, Hkv, lens)
+
+
+@pytest.mark.parametrize("k,Hq,Hkv", [(8, 32, 8), (16, 128, 8), (64, 16, 1), (128, 8, 4), (7, 72, 4)])
+def test_forward_items_split_heads_when_a_kv_group_exceeds_the_tile(harness, k, Hq, Hkv):
+    """G k > 128: the q heads of a kv head split over several items, each
+    with the same K/V tiles (Gp = 128 / k heads per item)."""
+    items = fwd_case(harness, k, 3, Hq, Hkv, [900, 130, 1])
+    G = Hq // Hkv
+    if G * k > BM:
+        assert max(it["h0"] - it["hkv"] * G for it in items) > 0
+
+
+def test_forward_items_empty_sequences_and_heavy_first_order(harness):
+    k, w = 8, 2
+    lens = [0, 300, 0, 5, 0, 1200]
+    items = fwd_case(harness, k, w, 32, 8, lens)
+    assert all(it["b"] not in (0, 2, 4) for it in items)
+    # round robin hands out the latest units of the last sequence first
+    assert items[0]["b"] == 5 and items[0]["cend"] == -(-1200 // k)
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill: a block of T new tokens against a cache holding n0 / m0
+# ---------------------------------------------------------------------------
+def chunk_case(harness, k, w, Hq, Hkv, states):
+    trip = [x for s in states for x in s]
+    rows = harness("chunk", k, w, Hq, Hkv, len(states), *trip)
+    B = len(states)
+    per, tail, item_rows = rows[:B], rows[B], rows[B + 1:]
+    sum_q, sum_kv, units, Lq, Lkv, Lunits, slot0 = tail
+    assert slot0 == 1 + k + w * k
+    # the gathered buffers and the unit list fit the workspace the call reserves
+    assert sum_q <= Lq and sum_kv <= Lkv and units <= Lunits
+    seq, row_lo = [], []
+    for (n0, m0, T), (code, cb, kvb, ncb, qoff, kvoff) in zip(states, per):
+        f0 = n0 - m0 * k
+        valid = 0 <= f0 <= k and n0 >= 0 and m0 >= 0
+        assert (code == 0) == valid, (n0, m0, T, code)
+        if valid and T > 0:
+            assert cb == n0 // k and ncb == -(-(n0 + T) // k)
+            assert kvb == max(0, min(cb - w, m0))
+            # the chunk of the first new summary is among the window chunks
+            assert kvb <= m0
+        seq.append((n0 + T, cb, kvb, (qoff - cb, kvoff - kvb)))
+        row_lo.append(n0)
+    active = [b for b, (s, p) in enumerate(zip(states, per)) if p[0] == 0 and s[2] > 0]
+    check_items(item_rows, k, w, Hq, Hkv, [seq[b] if b in active else (0, 0, 0, None) for b in range(B)],
+                row_lo=[row_lo[b] if b in active else 0 for b in range(B)])
+
+
+@pytest.mark.parametrize("k,w", [(1, 0), (2, 3), (4, 1), (8, 2), (8, 8), (16, 4), (32, 1), (64, 2), (128, 0), (6, 3)])
+def test_chunk_items_read_only_their_own_buffers(harness, k, w):
+    rng = np.random.default_rng(77 + k * 10 + w)
+    states = []
+    for _ in range(5):
+        n0 = int(rng.integers(0, 600))
+        T = int(rng.integers(1, 400))
+        states.append((n0, n0 // k, T))
+    # a full chunk whose summary is still pending (f0 = k), a block that
+    # starts on a chunk boundary, a one-token block, an empty block
+    states += [(3 * k, 2, 5), (4 * k, 4, 2 * k), (k + 1, 1, 1), (50, 50 // k, 0)]
+    chunk_case(harness, k, w, 32, 8, states)
+
+
+def test_chunk_invalid_states_get_no_work(harness):
+    k, w = 8, 2
+    states = [(20, 1, 10),   # f0 = 12 > k
+              (20, 3, 10),   # f0 < 0
+              (16, 2, 30),   # valid: f0 = 0
+              (-1, 0, 5)]
+    chunk_case(harness, k, w, 32, 8, states)
+
+
+# ---------------------------------------------------------------------------
+# Backward key tiles
+# ---------------------------------------------------------------------------
+KT = ("b", "sum", "j0", "kcnt", "n", "m", "c0", "qlo", "qhi", "nq")
+
+
+def bwd_case(harness, k, w, Hq, Hkv, nqs, seqlens):
+    rows = harness("bwd", k, w, Hq, Hkv, nqs, len(seqlens), *seqlens)
+    ns, nt = rows[0]
+    tiles = [dict(zip(KT, r)) for r in rows[1:]]
+    assert len(tiles) == ns + nt
+    coff = offsets([-(-n // k) for n in seqlens])
+    got_s = {b: [] for b in range(len(seqlens))}
+    got_t = {b: [] for b in range(len(seqlens))}
+    for i, T in enumerate(tiles):
+        b = T["b"]
+        n = seqlens[b]
+        m = n // k
+        assert (T["n"], T["m"], T["c0"]) == (n, m, coff[b])
+        assert bool(T["sum"]) == (i < ns), "summary tiles come first"
+        j0, kc = T["j0"], T["kcnt"]
+        assert j0 % BK == 0 and 1 <= kc <= BK
+        vt, vs = text_views(n, k, w)
+        if T["sum"]:
+            assert j0 + kc <= m and (kc == BK or j0 + kc == m)
+            got_s[b].append(j0)
+            q = np.flatnonzero(vs[:, j0:j0 + kc].any(axis=1))
+        else:
+            assert j0 + kc <= n and (kc == BK or j0 + kc == n)
+            got_t[b].append(j0)
+            q = np.flatnonzero(vt[:, j0:j0 + kc].any(axis=1))
+        qlo, qhi = T["qlo"], T["qhi"]
+        if q.size:
+            assert (qlo, qhi) == (q[0], q[-1] + 1), ("query range not the span of the queries that see it", T)
+        else:
+            assert qhi <= qlo
+        assert T["nq"] == (-(-(qhi - qlo) // nqs) if qhi > qlo else 0)
+    for b, n in enumerate(seqlens):
+        assert got_s[b] == list(range(0, n // k, BK))
+        assert got_t[b] == list(range(0, n, BK))
+
+
+@pytest.mark.parametrize("k", [1, 2, 4, 6, 8, 16, 32, 64, 100, 128])
+@pytest.mark.parametrize("w", [0, 1, 3, 8])
+def test_backward_key_tiles_and_query_ranges(harness, k, w):
+    rng = np.random.default_rng(500 + 10 * k + w)
+    lens = [int(x) for x in rng.integers(1, 900 if k > 2 else 350, size=3)] + [0, k, 2 * BK * max(1, k // 8)]
+    lens = [min(n, 1400) for n in lens]
+    nqs = 64 if 64 % k == 0 else 128
+    bwd_case(harness, k, w, 32, 8, nqs, lens)
+
+
+# ---------------------------------------------------------------------------
+# Decode slice
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("k,w", [(1, 0), (1, 3), (3, 2), (4, 0), (8, 1), (8, 8), (16, 3), (64, 2)])
+def test_decode_slice_matches_the_oracle_cache(harness, k, w):
+    n_tokens = 40 * k if k <= 8 else 6 * k
+    cache = oracle.Cache(k, w, 1, 2, n_tokens // k + 1)
+    row = np.zeros((1, 2))
+    n = m = 0
+    for _ in range(n_tokens):
+        assert cache.append_text(row, row) >= 0
+        n += 1
+        ok, lo, hi = harness("slice", k, w, TEXT, n, m)[0]
+        assert ok == 1 and (lo, hi) == cache.slice(TEXT), (n, m)
+        # a summary query is refused while the chunk is incomplete
+        assert harness("slice", k, w, SUMMARY, n, m)[0][0] == (1 if n - m * k == 0 and m >= 1 else 0)
+        if n % k == 0:
+            assert cache.append_summary(row, row) >= 0
+            m += 1
+            ok, lo, hi = harness("slice", k, w, SUMMARY, n, m)[0]
+            assert ok == 1 and (lo, hi) == cache.slice(SUMMARY), (n, m)
+            # a text query needs its token in the cache: f = n - m k >= 1
+            assert harness("slice", k, w, TEXT, n, m)[0][0] == 0
+    assert harness("slice", k, w, SUMMARY, 0, 0)[0][0] == 0
+    assert harness("slice", k, w, TEXT, k + 1, 0)[0][0] == 0   # f > k

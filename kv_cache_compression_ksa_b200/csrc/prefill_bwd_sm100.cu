@@ -570,6 +570,34 @@ struct SmemQ {
     static_assert(3 * BK + D <= (int)kTmemCols, "TMEM budget");
 };
 
+// The query tile of a dq CTA and its key tiles: text tiles in reverse order
+// (late tiles see the most summaries); ceil(ns / 128) summary tiles, then
+// the text keys [t_lo, q0 + qn) in tiles of 128.  Host-callable too, for
+// CPU tests of the tile list against the dense mask.
+struct QTile {
+    int b, n, m, c0, q0, qn, c_first, ns, n_sum, t_lo, n_win;
+};
+
+__host__ __device__ __forceinline__ bool q_tile(const TArgs &a, int cta, QTile &Q)
+{
+    const int ntt = a.kt_off[a.batch];
+    if (cta >= ntt) return false;
+    const int qt = ntt - 1 - cta;
+    Q.b = find_off(a.kt_off, a.batch, qt);
+    Q.n = a.cu[Q.b + 1] - a.cu[Q.b];
+    Q.m = Q.n / a.k;
+    Q.c0 = a.pl.chunk_off[Q.b];
+    Q.q0 = (qt - a.kt_off[Q.b]) * BQ;
+    Q.qn = min(BQ, Q.n - Q.q0);
+    Q.c_first = Q.q0 / a.k;
+    const int c_last = (Q.q0 + Q.qn - 1) / a.k;
+    Q.ns = max(0, min(Q.m, c_last - a.w));              // summaries any row may see
+    Q.n_sum = (Q.ns + BK - 1) / BK;
+    Q.t_lo = max(0, Q.c_first - a.w) * a.k;
+    Q.n_win = (Q.q0 + Q.qn - Q.t_lo + BK - 1) / BK;
+    return true;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constant__ TArgs a, __nv_bfloat16 *dq)
 {
@@ -585,21 +613,13 @@ __global__ void __launch_bounds__(kThreads, 1) bq_dq_kernel(const __grid_constan
         if (threadIdx.x == 0) set_error(a.err, KSA_ERR_UNSUPPORTED);
         return;
     }
-    // query tile: text tiles in reverse (late tiles see the most summaries)
-    const int ntt = a.kt_off[a.batch];
-    if ((int)blockIdx.x >= ntt) return;
-    const int qt = ntt - 1 - (int)blockIdx.x;
-    const int b = find_off(a.kt_off, a.batch, qt);
-    const int n = a.cu[b + 1] - a.cu[b], m = n / a.k, c0 = a.pl.chunk_off[b];
-    const int q0 = (qt - a.kt_off[b]) * BQ;
-    const int qn = min(BQ, n - q0);
+    QTile Q;
+    if (!q_tile(a, (int)blockIdx.x, Q)) return;
+    const int m = Q.m, c0 = Q.c0, q0 = Q.q0, qn = Q.qn;
     const int h = blockIdx.y, g = h / a.G;
-    const int c_first = q0 / a.k, c_last = (q0 + qn - 1) / a.k;
-    const int ns = max(0, min(m, c_last - a.w));          // summaries any row may see
-    const int n_sum = (ns + BK - 1) / BK;
-    const int t_lo = max(0, c_first - a.w) * a.k;         // text keys [t_lo, q0 + qn)
-    const int n_win = (q0 + qn - t_lo + BK - 1) / BK;
-    const int n_steps = n_sum + n_win;                    // >= 1: every row sees itself
+    const int c_first = Q.c_first;
+    const int n_sum = Q.n_sum, t_lo = Q.t_lo;
+    const int n_steps = n_sum + Q.n_win;                  // >= 1: every row sees itself
 
     auto bar = [&](int i) { return sbase + L::kBar + 8u * (uint32_t)i; };
     constexpr int B_Q = 0;
@@ -884,9 +904,40 @@ bool prefill_bwd_tc_supported(const ksa_params *p)
            p->num_kv_heads > 0 && p->num_q_heads % p->num_kv_heads == 0;
 }
 
+// Host-side sizing of the tensor-core backward, shared by the launch, the
+// workspace query and the CPU tests of the work list.
+//
+// Key tiles: at most aug_rows / 128 + 2 batch + 2 (a sequence's text and
+// summary rows each end in at most one partial tile).
+static int64_t bt_max_tiles(int batch, int64_t aug_rows) { return aug_rows / bt::BK + 2LL * batch + 2; }
+
+// dk/dv steps of 64 query positions (two S^T / dP^T buffers) when k divides
+// 64, else of 128; steps per CTA to match.
+static void bt_step_shape(int k, int *nqs, int *split)
+{
+    *nqs = 64 % k == 0 ? 64 : bt::BQ;
+    *split = *nqs == 64 ? bt::DkvCfg<128, 64>::kSplit : bt::DkvCfg<128, 128>::kSplit;
+}
+
+// CTAs of the dk/dv launch: an upper bound on the plan's share count (CTAs
+// past it exit).  At most one CTA per key tile plus G nq / split per tile; a
+// summary tile's queries number at most total_text, a text tile's
+// 128 + (w+1) k.
+static int64_t bt_dkv_grid(int64_t total_text, int batch, int k, int w, int G, int nqs, int split)
+{
+    const int64_t ns_tiles = (total_text / k) / bt::BK + batch, nt_tiles = total_text / bt::BK + batch;
+    const int64_t q_sum = (total_text + nqs - 1) / nqs + 1;
+    const int64_t q_txt = (bt::BK + (int64_t)(w + 1) * k + nqs - 1) / nqs + 1;
+    return ns_tiles * (1 + ((int64_t)G * q_sum) / split) + nt_tiles * (1 + ((int64_t)G * q_txt) / split);
+}
+
+// CTAs of the dq launch: an upper bound on the query tiles of 128 text
+// positions, which are the text key tiles (CTAs past the real count exit).
+static int64_t bt_dq_grid(int64_t total_text, int batch) { return total_text / bt::BK + batch; }
+
 size_t prefill_bwd_tc_workspace_bytes(int batch, int64_t aug_rows)
 {
-    const int64_t tiles = aug_rows / bt::BK + 2LL * batch + 2;
+    const int64_t tiles = bt_max_tiles(batch, aug_rows);
     return 2 * align_up(sizeof(int32_t) * (size_t)(batch + 1)) + align_up(sizeof(int32_t) * (size_t)(tiles + 1));
 }
 
@@ -917,10 +968,8 @@ int launch_prefill_bwd_tc(const ksa_params *p, int batch, const int32_t *cu, int
     const int d = p->head_dim, kk = p->k;
     const int64_t chunks = aug_rows / (kk + 1);
     const int qrows = bt::BQ / kk;   // chunks per query / text key box
-    // dk/dv steps of 64 query positions (two S^T / dP^T buffers) when k
-    // divides 64, else of 128
-    const int nqs = 64 % kk == 0 ? 64 : bt::BQ;
-    const int split = nqs == 64 ? bt::DkvCfg<128, 64>::kSplit : bt::DkvCfg<128, 128>::kSplit;
+    int nqs, split;
+    bt_step_shape(kk, &nqs, &split);
     bool ok = make_map(&a.tm_qs, q, d, p->num_q_heads, kk, chunks, 1, kk, nqs / kk) &&
               make_map(&a.tm_dos, dout, d, p->num_q_heads, kk, chunks, 1, kk, nqs / kk) &&
               make_map(&a.tm_kt, k, d, p->num_kv_heads, kk, chunks, 1, kk, qrows) &&
@@ -940,20 +989,14 @@ int launch_prefill_bwd_tc(const ksa_params *p, int batch, const int32_t *cu, int
     const size_t ab = align_up(sizeof(int32_t) * (size_t)(batch + 1));
     int32_t *ks_off = reinterpret_cast<int32_t *>(w), *kt_off = reinterpret_cast<int32_t *>(w + ab);
     int32_t *item_off = reinterpret_cast<int32_t *>(w + 2 * ab);
-    const int64_t max_tiles = aug_rows / bt::BK + 2LL * batch + 2;
+    const int64_t max_tiles = bt_max_tiles(batch, aug_rows);
     if (max_tiles > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
     a.ks_off = ks_off; a.kt_off = kt_off; a.item_off = item_off; a.max_tiles = (int)max_tiles;
     bt::bt_plan_kernel<<<1, 1024, 0, st>>>(a, ks_off, kt_off, item_off);
-    // CTAs: at most one per key tile plus G nq / split per tile; a summary
-    // tile's queries number at most total_text, a text tile's 128 + (w+1) k
-    const int64_t ns_tiles = (total_text / kk) / bt::BK + batch, nt_tiles = total_text / bt::BK + batch;
-    const int64_t G = a.G;
-    const int64_t q_sum = (total_text + nqs - 1) / nqs + 1;
-    const int64_t q_txt = (bt::BK + (int64_t)(p->w + 1) * kk + nqs - 1) / nqs + 1;
-    const int64_t grid = ns_tiles * (1 + (G * q_sum) / split) + nt_tiles * (1 + (G * q_txt) / split);
+    const int64_t grid = bt_dkv_grid(total_text, batch, kk, p->w, a.G, nqs, split);
     if (grid > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;
     if (grid == 0) return KSA_OK;
-    const int64_t grid_q = nt_tiles;   // query tiles of 128 text positions (CTAs past the real count exit)
+    const int64_t grid_q = bt_dq_grid(total_text, batch);
     __nv_bfloat16 *dqb = static_cast<__nv_bfloat16 *>(dq);
     int r;
     if (nqs == 64)

@@ -5,8 +5,12 @@
 // functions under test are the kernels' own, marked __host__ __device__:
 //   pf::unit_of           the forward's work items and their K/V tiles
 //                         (plain prefill and chunk mode),
-//   bt::key_tile          the backward's key tiles and the text query range
-//                         that sees each,
+//   bt::key_tile, bt::q_tile
+//                         the backward's key tiles with the text query range
+//                         that sees each (dk/dv), and its query tiles with
+//                         their key tiles (dq),
+//   bt_step_shape, bt_max_tiles, bt_dkv_grid, bt_dq_grid
+//                         the backward's step shape and launch bounds,
 //   ck::chunk_state_code, ck::chunk_ranges, ck::layout
 //                         the chunked prefill's state checks, gathered
 //                         chunk ranges and buffer sizes,
@@ -24,8 +28,10 @@
 //         per sequence "code cbeg kvb ncb qoff kvoff"; then
 //         "sum_q sum_kv units L.q_chunks L.kv_chunks L.max_units sum_slot0";
 //         then the work items as for fwd
-//   bwd   k w Hq Hkv nqs B n_0 .. n_{B-1}
-//         "ns nt", then per key tile "b sum j0 kcnt n m c0 qlo qhi nq"
+//   bwd   k w Hq Hkv B n_0 .. n_{B-1}
+//         "ns nt nqs split max_tiles dkv_grid dq_grid dkv_ctas", then per key
+//         tile "b sum j0 kcnt n m c0 qlo qhi nq", then "ntt" and per dq CTA
+//         "b n m c0 q0 qn c_first ns n_sum t_lo n_win"
 //   slice k w kind n m
 //         "ok lo hi"
 #include <cstdio>
@@ -152,9 +158,11 @@ static void run_chunk(int k, int w, int Hq, int Hkv, const std::vector<int> &tri
     print_items(P, uoff[B]);
 }
 
-static void run_bwd(int k, int w, int Hq, int Hkv, int nqs, const std::vector<int> &n)
+static void run_bwd(int k, int w, int Hq, int Hkv, const std::vector<int> &n)
 {
     const int B = (int)n.size();
+    int nqs, split;
+    bt_step_shape(k, &nqs, &split);
     std::vector<int32_t> cu(B + 1, 0), chunk_off(B + 1, 0), ks_off(B + 1, 0), kt_off(B + 1, 0);
     for (int b = 0; b < B; ++b) {
         cu[b + 1] = cu[b] + n[b];
@@ -170,12 +178,27 @@ static void run_bwd(int k, int w, int Hq, int Hkv, int nqs, const std::vector<in
     a.ks_off = ks_off.data();
     a.kt_off = kt_off.data();
     a.nqs = nqs;
+    a.split = split;
     const int ns = ks_off[B], nt = kt_off[B];
-    std::printf("%d %d\n", ns, nt);
+    const int64_t total_text = cu[B], aug_rows = (int64_t)chunk_off[B] * (k + 1);
+    // the plan's CTA shares: ceil(G nq / split) per key tile
+    int64_t ctas = 0;
+    std::vector<bt::KTile> tiles(ns + nt);
     for (int t = 0; t < ns + nt; ++t) {
-        bt::KTile T;
-        bt::key_tile(a, t, T);
+        bt::key_tile(a, t, tiles[t]);
+        ctas += (a.G * tiles[t].nq + split - 1) / split;
+    }
+    std::printf("%d %d %d %d %lld %lld %lld %lld\n", ns, nt, nqs, split, (long long)bt_max_tiles(B, aug_rows),
+                (long long)bt_dkv_grid(total_text, B, k, w, a.G, nqs, split), (long long)bt_dq_grid(total_text, B),
+                (long long)ctas);
+    for (const bt::KTile &T : tiles)
         std::printf("%d %d %d %d %d %d %d %d %d %d\n", T.b, T.sum, T.j0, T.kcnt, T.n, T.m, T.c0, T.qlo, T.qhi, T.nq);
+    std::printf("%d\n", nt);
+    for (int cta = 0;; ++cta) {
+        bt::QTile Q;
+        if (!bt::q_tile(a, cta, Q)) break;
+        std::printf("%d %d %d %d %d %d %d %d %d %d %d\n", Q.b, Q.n, Q.m, Q.c0, Q.q0, Q.qn, Q.c_first, Q.ns, Q.n_sum,
+                    Q.t_lo, Q.n_win);
     }
 }
 
@@ -197,8 +220,8 @@ int main()
             run_fwd((int)v[0], (int)v[1], (int)v[2], (int)v[3], ints(5));
         } else if (m == "chunk" && v.size() >= 5 && v.size() == 5 + 3 * (size_t)v[4]) {
             run_chunk((int)v[0], (int)v[1], (int)v[2], (int)v[3], ints(5));
-        } else if (m == "bwd" && v.size() >= 6 && v.size() == 6 + (size_t)v[5]) {
-            run_bwd((int)v[0], (int)v[1], (int)v[2], (int)v[3], (int)v[4], ints(6));
+        } else if (m == "bwd" && v.size() >= 5 && v.size() == 5 + (size_t)v[4]) {
+            run_bwd((int)v[0], (int)v[1], (int)v[2], (int)v[3], ints(5));
         } else if (m == "slice" && v.size() == 5) {
             int64_t lo = 0, hi = 0;
             const bool ok = decode_slice((int)v[2], v[3], v[4], (int)v[0], (int)v[1], &lo, &hi);

@@ -13,7 +13,9 @@ the oracle's dense mask:
     Technical Report", section 2.3 "Kernel Design": only block pairs the mask
     does not zero out entirely are computed);
   - the backward's key tiles split the keys, and the text query range of
-    each tile is exactly the span of the queries that see it;
+    each tile is exactly the span of the queries that see it; its query
+    tiles split the text rows and hold what those rows see; its grids and
+    workspace bound the work lists;
   - the chunked prefill's gathered buffers hold what its work items read,
     within the sizes the workspace reserves;
   - the decode's live slots match the oracle's cache (section 2.3.1,
@@ -245,13 +247,19 @@ def test_chunk_invalid_states_get_no_work(harness):
 # Backward key tiles
 # ---------------------------------------------------------------------------
 KT = ("b", "sum", "j0", "kcnt", "n", "m", "c0", "qlo", "qhi", "nq")
+QT = ("b", "n", "m", "c0", "q0", "qn", "c_first", "ns", "n_sum", "t_lo", "n_win")
 
 
-def bwd_case(harness, k, w, Hq, Hkv, nqs, seqlens):
-    rows = harness("bwd", k, w, Hq, Hkv, nqs, len(seqlens), *seqlens)
-    ns, nt = rows[0]
-    tiles = [dict(zip(KT, r)) for r in rows[1:]]
-    assert len(tiles) == ns + nt
+def bwd_case(harness, k, w, Hq, Hkv, seqlens):
+    rows = harness("bwd", k, w, Hq, Hkv, len(seqlens), *seqlens)
+    ns, nt, nqs, split, max_tiles, dkv_grid, dq_grid, dkv_ctas = rows[0]
+    G = Hq // Hkv
+    # steps of 64 query positions when k divides 64, else of 128
+    assert nqs == (64 if 64 % k == 0 else 128) and nqs % k == 0
+    # launch bounds: the plan never needs more tiles, or CTAs, than reserved
+    assert ns + nt <= max_tiles and dkv_ctas <= dkv_grid and nt <= dq_grid
+    tiles = [dict(zip(KT, r)) for r in rows[1:1 + ns + nt]]
+    check_dq_tiles(rows[1 + ns + nt:], k, w, seqlens, nt)
     coff = offsets([-(-n // k) for n in seqlens])
     got_s = {b: [] for b in range(len(seqlens))}
     got_t = {b: [] for b in range(len(seqlens))}
@@ -281,16 +289,54 @@ def bwd_case(harness, k, w, Hq, Hkv, nqs, seqlens):
     for b, n in enumerate(seqlens):
         assert got_s[b] == list(range(0, n // k, BK))
         assert got_t[b] == list(range(0, n, BK))
+    assert dkv_ctas == sum(-(-(G * T["nq"]) // split) for T in tiles)
 
 
-@pytest.mark.parametrize("k", [1, 2, 4, 6, 8, 16, 32, 64, 100, 128])
+def check_dq_tiles(rows, k, w, seqlens, nt):
+    """dq: one CTA per 128 text rows (latest first), each with its summary
+    tiles and text key tiles of 128 from t_lo."""
+    assert rows[0] == [nt] and len(rows) == 1 + nt
+    coff = offsets([-(-n // k) for n in seqlens])
+    covered = {b: [] for b in range(len(seqlens))}
+    for r in rows[1:]:
+        Q = dict(zip(QT, r))
+        b, n = Q["b"], seqlens[Q["b"]]
+        assert (Q["n"], Q["m"], Q["c0"]) == (n, n // k, coff[b])
+        q0, qn = Q["q0"], Q["qn"]
+        assert q0 % BK == 0 and 1 <= qn <= BK and q0 + qn <= n and (qn == BK or q0 + qn == n)
+        assert Q["c_first"] == q0 // k
+        covered[b].append(q0)
+        vt, vs = text_views(n, k, w)
+        seen_t = np.flatnonzero(vt[q0:q0 + qn].any(axis=0))
+        seen_s = np.flatnonzero(vs[q0:q0 + qn].any(axis=0))
+        t_lo, n_win, n_sum = Q["t_lo"], Q["n_win"], Q["n_sum"]
+        assert t_lo % k == 0, "a text key box starts on a chunk"
+        assert seen_t[0] >= t_lo and seen_t[-1] < t_lo + n_win * BK
+        for j in range(n_win):
+            assert np.any((seen_t >= t_lo + j * BK) & (seen_t < t_lo + (j + 1) * BK)), ("fully masked text tile", Q, j)
+        assert seen_s.size == Q["ns"] and (seen_s.size == 0 or seen_s[-1] == seen_s.size - 1)
+        assert n_sum == -(-Q["ns"] // BK)
+    for b, n in enumerate(seqlens):
+        assert sorted(covered[b]) == list(range(0, n, BK))
+
+
+@pytest.mark.parametrize("k", [1, 2, 4, 8, 16, 32, 64, 128])   # the tensor-core backward's k: divisors of 128
 @pytest.mark.parametrize("w", [0, 1, 3, 8])
 def test_backward_key_tiles_and_query_ranges(harness, k, w):
     rng = np.random.default_rng(500 + 10 * k + w)
     lens = [int(x) for x in rng.integers(1, 900 if k > 2 else 350, size=3)] + [0, k, 2 * BK * max(1, k // 8)]
     lens = [min(n, 1400) for n in lens]
-    nqs = 64 if 64 % k == 0 else 128
-    bwd_case(harness, k, w, 32, 8, nqs, lens)
+    Hq, Hkv = [(32, 8), (8, 8), (64, 4)][(k + w) % 3]
+    bwd_case(harness, k, w, Hq, Hkv, lens)
+
+
+@pytest.mark.parametrize("k,w,G", [(1, 0, 16), (8, 0, 1), (8, 64, 4), (64, 1, 8), (128, 0, 4), (2, 300, 2)])
+def test_backward_launch_bounds_at_their_edges(harness, k, w, G):
+    """Shapes that push the grid bounds: one long sequence (a summary tile's
+    query range is the whole sequence), many short ones (partial tiles per
+    sequence), a window wider than the sequence."""
+    for lens in ([4000], [1] * 40, [k] * 17 + [k + 1] * 5, [129, 257, 383]):
+        bwd_case(harness, k, w, 8 * G, 8, lens)
 
 
 # ---------------------------------------------------------------------------

@@ -40,7 +40,11 @@ TRAFFIC = {
     # capture (661.2 MB of the previous build, profiles/prefill_kernel_qwen3_4b_32k.md)
     "prefill": (None, "not captured for this build; 661.2 MB for the previous one in "
                       "profiles/prefill_kernel_qwen3_4b_32k.md (prefill_kernel<128>)"),
-    "decode_per_seq": (1.0851e9 / 16, "profiles/decode_split_kernel_b16_m16384.md (batch 16 capture, per sequence)"),
+    # the decode kernel gained a state check (slice within the cache's slots,
+    # no negative counts) after its capture; the capture read 1.0851 GB per
+    # 16 sequences, 1.007x the algorithmic bytes
+    "decode_per_seq": (None, "not captured for this build; 1.0851e9 B per 16 sequences for the previous one in "
+                             "profiles/decode_split_kernel_b16_m16384.md (batch 16 capture)"),
 }
 DC = dict(B=64, m=16384, k=8, w=8, Hq=32, Hkv=8, d=128, seed=3, theta=1e6)
 
@@ -455,7 +459,8 @@ def run_ksa(args, rank, world, local):
                          "peak_source": f"{peak_src} burst bf16", "peak_sustained": tc_sus},
             "roofline_decode": {"bound": "hbm", "achieved": dec_gbs / world, "peak": hbm_peak, "unit": "GB/s",
                                 "frac": (dec_gbs / world) / hbm_peak,
-                                "traffic": (TRAFFIC["decode_per_seq"][0] * B if m == DC["m"] else None),
+                                "traffic": (TRAFFIC["decode_per_seq"][0] * B
+                                            if m == DC["m"] and TRAFFIC["decode_per_seq"][0] is not None else None),
                                 "traffic_source": TRAFFIC["decode_per_seq"][1],
                                 "kernel": "decode_split_kernel<128,4> + combine (time of ksa_decode)"},
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),

@@ -217,8 +217,9 @@ KSA_API int64_t ksa_cache_slots(const ksa_params *p, int64_t cap_summaries);
  *   TEXT    (needs f < k): K/V into slot k - f; n_text += 1.       (4b)
  *   SUMMARY (needs f == k): K/V into slot 0 (4c); slots 1..k copied over
  *           ring block m mod w (4d); K/V into slot 1+k+w*k+m (4e); m += 1.
- * A violated precondition sets state[b].err = KSA_ERR_STATE, a full
- * summary buffer KSA_ERR_CAPACITY; that sequence is left unchanged. */
+ * A violated precondition, or a state no sequence of appends reaches
+ * (negative counts), sets state[b].err = KSA_ERR_STATE, a full summary
+ * buffer KSA_ERR_CAPACITY; that sequence is left unchanged. */
 KSA_API int ksa_cache_append(const ksa_params *p, const ksa_cache *cache, const int8_t *kind,
                      const void *k_new, const void *v_new, void *stream);
 
@@ -292,7 +293,10 @@ KSA_API size_t ksa_decode_workspace_size(const ksa_params *p, int32_t batch, int
  * SUMMARY reads slots [0, k+1); SKIP writes nothing.  Each is one
  * contiguous slice.  o: [batch, Hq, d] bf16; lse: [batch, Hq] fp32 or NULL.
  * max_text bounds n_text over the batch (it sizes the split-K grid and
- * must match the workspace query). */
+ * must match the workspace query).  A sequence whose state cannot hold a
+ * query of its kind (negative counts, f outside [1, k] for TEXT, f != 0 or
+ * m = 0 for SUMMARY, a slice past the cache's slots) gets state[b].err =
+ * KSA_ERR_STATE and no output. */
 KSA_API int ksa_decode(const ksa_params *p, const ksa_cache *cache, const int8_t *kind, const void *q,
                void *o, float *lse, int64_t max_text,
                void *workspace, size_t workspace_bytes, void *stream);

@@ -50,11 +50,12 @@ __global__ void __launch_bounds__(kAppendThreads) cache_append_kernel(AppendArgs
         int kind = a.kind[b];
         int64_t n = st[0], m = st[1];
         int64_t f = n - m * a.k;
+        const bool reachable = n >= 0 && m >= 0;   // slots below are only in range for these
         int act = 0;
         if (kind == KSA_TEXT) {
-            if (f >= 0 && f < a.k) act = 1; else st[3] = KSA_ERR_STATE;
+            if (reachable && f >= 0 && f < a.k) act = 1; else st[3] = KSA_ERR_STATE;
         } else if (kind == KSA_SUMMARY) {
-            if (f != a.k) st[3] = KSA_ERR_STATE;
+            if (!reachable || f != a.k) st[3] = KSA_ERR_STATE;
             else if (m >= a.cap) st[3] = KSA_ERR_CAPACITY;
             else act = 2;
         } else if (kind != KSA_SKIP) {
@@ -318,7 +319,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_split_kernel(DecodeArgs
     if (kind == KSA_SKIP) return;
     const int64_t n = a.state[4 * (int64_t)b], m = a.state[4 * (int64_t)b + 1];
     int64_t lo, hi;
-    if (!decode_slice(kind, n, m, a.k, a.w, &lo, &hi)) {
+    if (!decode_slice(kind, n, m, a.k, a.w, &lo, &hi) || hi > a.S) {
         if (split == 0 && h == 0 && t == 0) a.state[4 * (int64_t)b + 3] = KSA_ERR_STATE;
         return;
     }
@@ -482,7 +483,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeArgs a, __nv_
     const int kind = a.kind[b];
     if (kind == KSA_SKIP) return;
     int64_t lo, hi;
-    if (!decode_slice(kind, a.state[4 * (int64_t)b], a.state[4 * (int64_t)b + 1], a.k, a.w, &lo, &hi))
+    if (!decode_slice(kind, a.state[4 * (int64_t)b], a.state[4 * (int64_t)b + 1], a.k, a.w, &lo, &hi) ||
+        hi > a.S)
         return;
     const float *part = a.part + (((int64_t)b * a.Hkv + h) * a.nsplit) * (G * (2 + D));
     const int stride = G * (2 + D);

@@ -179,6 +179,7 @@ __device__ __forceinline__ void rope_rot8(uint4 &lo, uint4 &hi, const float *cs,
 __host__ __device__ __forceinline__ bool decode_slice(int kind, int64_t n, int64_t m, int k, int w,
                                              int64_t *lo, int64_t *hi)
 {
+    if (n < 0 || m < 0) return false;   // no sequence of appends reaches it
     int64_t f = n - m * k;
     if (kind == KSA_SUMMARY) {
         if (m < 1 || f != 0) return false;

@@ -72,11 +72,12 @@ __global__ void __launch_bounds__(kAppendThreads) mla_append_kernel(AppendArgs a
     if (t == 0) {
         const int kind = a.kind[b];
         const int64_t n = st[0], m = st[1], f = n - m * a.k;
+        const bool reachable = n >= 0 && m >= 0;   // slots below are only in range for these
         int act = 0;
         if (kind == KSA_TEXT) {
-            if (f >= 0 && f < a.k) act = 1; else st[3] = KSA_ERR_STATE;
+            if (reachable && f >= 0 && f < a.k) act = 1; else st[3] = KSA_ERR_STATE;
         } else if (kind == KSA_SUMMARY) {
-            if (f != a.k) st[3] = KSA_ERR_STATE;
+            if (!reachable || f != a.k) st[3] = KSA_ERR_STATE;
             else if (m >= a.cap) st[3] = KSA_ERR_CAPACITY;
             else act = 2;
         } else if (kind != KSA_SKIP) {

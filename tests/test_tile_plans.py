@@ -353,6 +353,7 @@ def test_decode_slice_matches_the_oracle_cache(harness, k, w):
         n += 1
         ok, lo, hi = harness("slice", k, w, TEXT, n, m)[0]
         assert ok == 1 and (lo, hi) == cache.slice(TEXT), (n, m)
+        assert 1 <= lo < hi <= 1 + k + w * k + m   # within a cache whose capacity is m
         # a summary query is refused while the chunk is incomplete
         assert harness("slice", k, w, SUMMARY, n, m)[0][0] == (1 if n - m * k == 0 and m >= 1 else 0)
         if n % k == 0:
@@ -364,3 +365,7 @@ def test_decode_slice_matches_the_oracle_cache(harness, k, w):
             assert harness("slice", k, w, TEXT, n, m)[0][0] == 0
     assert harness("slice", k, w, SUMMARY, 0, 0)[0][0] == 0
     assert harness("slice", k, w, TEXT, k + 1, 0)[0][0] == 0   # f > k
+    # counts no sequence of appends reaches, even where f would pass
+    for n_, m_ in ((-k, -2), (1 - k, -1), (-1, 0), (k, -1)):
+        assert harness("slice", k, w, TEXT, n_, m_)[0][0] == 0
+        assert harness("slice", k, w, SUMMARY, n_, m_)[0][0] == 0

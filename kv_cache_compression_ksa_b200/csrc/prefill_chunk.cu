@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kRopeThreads) chunk_rope_kernel(Args a)
 
 // K and V rows (D elements) of a key of sequence b, kv head g.
 template <int D>
-__device__ __forceinline__ void key_rows(const Args &a, const Snap &sn, int b, int g, int kind, int idx,
+__host__ __device__ __forceinline__ void key_rows(const Args &a, const Snap &sn, int b, int g, int kind, int idx,
                                          const __nv_bfloat16 *&pk, const __nv_bfloat16 *&pv)
 {
     const int64_t cache_row = ((int64_t)b * a.Hkv + g) * a.S;

@@ -11,9 +11,10 @@
 //                         their key tiles (dq),
 //   bt_step_shape, bt_max_tiles, bt_dkv_grid, bt_dq_grid
 //                         the backward's step shape and launch bounds,
-//   ck::chunk_state_code, ck::chunk_ranges, ck::layout
+//   ck::chunk_state_code, ck::chunk_ranges, ck::layout, ck::key_rows
 //                         the chunked prefill's state checks, gathered
-//                         chunk ranges and buffer sizes,
+//                         chunk ranges, buffer sizes and the cache slot or
+//                         block row each key is read from,
 //   decode_slice          the live cache slots of a decode query.
 // Only the prefix sums that the plan kernels compute on the device (one
 // scan per array) are written out here, as plain loops, together with the
@@ -34,6 +35,10 @@
 //         "b n m c0 q0 qn c_first ns n_sum t_lo n_win"
 //   slice k w kind n m
 //         "ok lo hi"
+//   keys  k w n0 m0 T
+//         per text key p < n0 + T "0 p src at", then per summary
+//         j < m0 + S "1 j src at": src 0 = cache slot at, 1 = row at of the
+//         block's input (one sequence, one kv head)
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -202,6 +207,46 @@ static void run_bwd(int k, int w, int Hq, int Hkv, const std::vector<int> &n)
     }
 }
 
+static void run_keys(int k, int w, int n0, int m0, int T)
+{
+    constexpr int D = 64;
+    const int64_t f0 = (int64_t)n0 - (int64_t)m0 * k;
+    const int S_new = f0 >= 0 ? (int)((f0 + T) / k) : 0;
+    const int64_t cap = m0 + S_new + 1;
+    ck::Args a;
+    std::memset(&a, 0, sizeof(a));
+    a.k = k; a.w = w; a.Hkv = 1; a.Hq = 1; a.G = 1; a.batch = 1; a.d = D;
+    a.cap = cap;
+    a.S = 1 + (int64_t)k + (int64_t)w * k + cap;
+    const int32_t cu_t[2] = {0, T}, cu_s[2] = {0, S_new};
+    a.cu_t = cu_t; a.cu_s = cu_s;
+    std::vector<__nv_bfloat16> ck_(a.S * D), cv_(a.S * D), kt_((size_t)T * D + D), vt_((size_t)T * D + D),
+        ks_((size_t)S_new * D + D), vs_((size_t)S_new * D + D);
+    a.ck = ck_.data(); a.cv = cv_.data();
+    a.ktr = kt_.data(); a.vt = vt_.data();
+    a.ksr = ks_.data(); a.vs = vs_.data();
+    const ck::Snap sn{n0, m0, 1, 0};
+    auto locate = [&](const __nv_bfloat16 *pk, const __nv_bfloat16 *pv, const __nv_bfloat16 *kb,
+                      const __nv_bfloat16 *vb, size_t rows, int64_t *at) {
+        if (pk < kb || pk >= kb + rows * D) return false;
+        *at = (pk - kb) / D;
+        return (pk - kb) % D == 0 && pv == vb + *at * D;   // K and V from the same row
+    };
+    for (int kind = 0; kind < 2; ++kind) {
+        const int count = kind == 0 ? n0 + T : m0 + S_new;
+        for (int idx = 0; idx < count; ++idx) {
+            const __nv_bfloat16 *pk = nullptr, *pv = nullptr;
+            ck::key_rows<D>(a, sn, 0, 0, kind == 0 ? ck::TEXT_ROWS : ck::SUM_ROWS, idx, pk, pv);
+            int64_t at = -1;
+            int src = -1;
+            if (locate(pk, pv, a.ck, a.cv, (size_t)a.S, &at)) src = 0;
+            else if (kind == 0 && locate(pk, pv, a.ktr, a.vt, (size_t)T, &at)) src = 1;
+            else if (kind == 1 && locate(pk, pv, a.ksr, a.vs, (size_t)S_new, &at)) src = 1;
+            std::printf("%d %d %d %lld\n", kind, idx, src, (long long)at);
+        }
+    }
+}
+
 int main()
 {
     char line[1 << 16];
@@ -222,6 +267,8 @@ int main()
             run_chunk((int)v[0], (int)v[1], (int)v[2], (int)v[3], ints(5));
         } else if (m == "bwd" && v.size() >= 5 && v.size() == 5 + (size_t)v[4]) {
             run_bwd((int)v[0], (int)v[1], (int)v[2], (int)v[3], ints(5));
+        } else if (m == "keys" && v.size() == 5) {
+            run_keys((int)v[0], (int)v[1], (int)v[2], (int)v[3], (int)v[4]);
         } else if (m == "slice" && v.size() == 5) {
             int64_t lo = 0, hi = 0;
             const bool ok = decode_slice((int)v[2], v[3], v[4], (int)v[0], (int)v[1], &lo, &hi);

@@ -17,7 +17,9 @@ the oracle's dense mask:
     tiles split the text rows and hold what those rows see; its grids and
     workspace bound the work lists;
   - the chunked prefill's gathered buffers hold what its work items read,
-    within the sizes the workspace reserves;
+    within the sizes the workspace reserves, and every key its rows see is
+    read from the cache slot where the oracle's cache holds that key (or
+    from the block's own input rows);
   - the decode's live slots match the oracle's cache (section 2.3.1,
     Figure 4) in every reachable state, and unreachable states are refused.
 The visibility rule is section 2.2.1 (summaries) and section 2.2.2,
@@ -369,3 +371,62 @@ def test_decode_slice_matches_the_oracle_cache(harness, k, w):
     for n_, m_ in ((-k, -2), (1 - k, -1), (-1, 0), (k, -1)):
         assert harness("slice", k, w, TEXT, n_, m_)[0][0] == 0
         assert harness("slice", k, w, SUMMARY, n_, m_)[0][0] == 0
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill: where each key is read from
+# ---------------------------------------------------------------------------
+def oracle_cache_image(k, w, n0, m0, cap):
+    """The oracle's cache after n0 text appends and m0 summaries (in the
+    order of section 2.3.1), each K row holding its key's id: text p -> p + 1,
+    summary j -> -(j + 1)."""
+    cache = oracle.Cache(k, w, 1, 1, cap)
+    m = 0
+    for p in range(n0):
+        assert cache.append_text(np.full((1, 1), p + 1.0), np.zeros((1, 1))) == 0
+        if (p + 1) % k == 0 and m < m0:
+            assert cache.append_summary(np.full((1, 1), -(m + 1.0)), np.zeros((1, 1))) == 0
+            m += 1
+    assert (cache.n_text, cache.m) == (n0, m0)
+    return cache.K()[:, 0, 0]
+
+
+@pytest.mark.parametrize("k,w", [(1, 0), (1, 2), (2, 1), (3, 2), (4, 1), (4, 4), (8, 2), (8, 8), (16, 3), (5, 0)])
+def test_chunk_keys_are_read_where_the_cache_holds_them(harness, k, w):
+    rng = np.random.default_rng(900 + 10 * k + w)
+    states = [(0, 0, 3 * k + 1), (k - 1, 0, 2), (2 * k, 2, k), (3 * k, 2, 1), (3 * k, 2, 2 * k + 3)]
+    for _ in range(4):
+        n0 = int(rng.integers(0, 12 * k + 5))
+        pending = n0 > 0 and n0 % k == 0 and rng.random() < 0.5   # a full chunk still waiting for its summary
+        states.append((n0, n0 // k - (1 if pending else 0), int(rng.integers(1, 4 * k + 3))))
+    for n0, m0, T in states:
+        f0 = n0 - m0 * k
+        S_new = (f0 + T) // k
+        n1, m1 = n0 + T, m0 + S_new
+        img = oracle_cache_image(k, w, n0, m0, m1 + 1)
+        where = {}
+        for kind, idx, src, at in harness("keys", k, w, n0, m0, T):
+            where[(kind, idx)] = (src, at)
+        M = oracle.dense_mask(n1, k, w).astype(bool)
+        # Eq. (1) positions of text p and summary j, and the rows the block computes
+        tpos = lambda p: (p // k) * (k + 1) + p % k
+        spos = lambda j: j * (k + 1) + k
+        rows = [tpos(p) for p in range(n0, n1)] + [spos(j) for j in range(m0, m1)]
+        seen = M[rows].any(axis=0)
+        for p in range(n1):
+            if not seen[tpos(p)]:
+                continue
+            src, at = where[(TEXT, p)]
+            if p < n0:
+                assert src == 0 and img[at] == p + 1, ("cached text key read from the wrong slot", n0, m0, T, p, at)
+            else:
+                assert (src, at) == (1, p - n0)
+        for j in range(m1):
+            if not seen[spos(j)]:
+                continue
+            src, at = where[(SUMMARY, j)]
+            if j < m0:
+                assert src == 0 and img[at] == -(j + 1), ("cached summary read from the wrong slot", n0, m0, T, j, at)
+            else:
+                assert (src, at) == (1, j - m0)
+

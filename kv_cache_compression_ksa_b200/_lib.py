@@ -140,11 +140,20 @@ def status_string(status: int) -> str:
         return "library not loaded"
 
 
-def _ptr(t):
+# element types the ABI documents for its tensor arguments (include/ksa.h)
+BF16, F32, I32, I8 = torch.bfloat16, torch.float32, torch.int32, torch.int8
+
+
+def _ptr(t, dtype=None):
+    """Device pointer of a contiguous CUDA tensor of the given element type
+    (None: any, e.g. a byte workspace).  An int passes through as a raw
+    device address."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"tensor must be {dtype}, got {t.dtype}")
     if not t.is_cuda:
         raise ValueError("tensor must live on a CUDA device")
     if not t.is_contiguous():
@@ -182,29 +191,29 @@ def ksa_prefill_workspace_size(p: ksa_params, batch: int, total_text: int) -> in
 def ksa_interleave_rope(p, cu_seqlens, total_text, total_sum, aug_rows, q_text, k_text, v_text,
                         q_sum, k_sum, v_sum, q_aug, k_aug, v_aug, workspace, dev_err=None, stream=None):
     rc = load().ksa_interleave_rope(
-        ctypes.byref(p), cu_seqlens.numel() - 1, _ptr(cu_seqlens), total_text, total_sum, aug_rows,
-        _ptr(q_text), _ptr(k_text), _ptr(v_text), _ptr(q_sum), _ptr(k_sum), _ptr(v_sum),
-        _ptr(q_aug), _ptr(k_aug), _ptr(v_aug), _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _ptr(dev_err), _stream(stream))
+        ctypes.byref(p), cu_seqlens.numel() - 1, _ptr(cu_seqlens, I32), total_text, total_sum, aug_rows,
+        _ptr(q_text, BF16), _ptr(k_text, BF16), _ptr(v_text, BF16), _ptr(q_sum, BF16), _ptr(k_sum, BF16),
+        _ptr(v_sum, BF16), _ptr(q_aug, BF16), _ptr(k_aug, BF16), _ptr(v_aug, BF16), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_err, I32), _stream(stream))
     _check("ksa_interleave_rope", rc)
 
 
 def ksa_interleave_rope_bwd(p, cu_seqlens, total_text, total_sum, aug_rows, dq_aug, dk_aug, dv_aug,
                             dq_text, dk_text, dv_text, dq_sum, dk_sum, dv_sum, workspace, dev_err=None, stream=None):
     rc = load().ksa_interleave_rope_bwd(
-        ctypes.byref(p), cu_seqlens.numel() - 1, _ptr(cu_seqlens), total_text, total_sum, aug_rows,
-        _ptr(dq_aug), _ptr(dk_aug), _ptr(dv_aug), _ptr(dq_text), _ptr(dk_text), _ptr(dv_text), _ptr(dq_sum),
-        _ptr(dk_sum), _ptr(dv_sum), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_err),
-        _stream(stream))
+        ctypes.byref(p), cu_seqlens.numel() - 1, _ptr(cu_seqlens, I32), total_text, total_sum, aug_rows,
+        _ptr(dq_aug, BF16), _ptr(dk_aug, BF16), _ptr(dv_aug, BF16), _ptr(dq_text, BF16), _ptr(dk_text, BF16),
+        _ptr(dv_text, BF16), _ptr(dq_sum, BF16), _ptr(dk_sum, BF16), _ptr(dv_sum, BF16), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_err, I32), _stream(stream))
     _check("ksa_interleave_rope_bwd", rc)
 
 
 def ksa_prefill_fwd(p, cu_seqlens, total_text, aug_rows, q_aug, k_aug, v_aug, o_aug, lse, workspace,
                     dev_err=None, stream=None):
     rc = load().ksa_prefill_fwd(
-        ctypes.byref(p), cu_seqlens.numel() - 1, _ptr(cu_seqlens), total_text, aug_rows,
-        _ptr(q_aug), _ptr(k_aug), _ptr(v_aug), _ptr(o_aug), _ptr(lse),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_err), _stream(stream))
+        ctypes.byref(p), cu_seqlens.numel() - 1, _ptr(cu_seqlens, I32), total_text, aug_rows,
+        _ptr(q_aug, BF16), _ptr(k_aug, BF16), _ptr(v_aug, BF16), _ptr(o_aug, BF16), _ptr(lse, F32),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_err, I32), _stream(stream))
     _check("ksa_prefill_fwd", rc)
 
 
@@ -215,9 +224,10 @@ def ksa_prefill_bwd_workspace_size(p: ksa_params, batch: int, aug_rows: int) -> 
 def ksa_prefill_bwd(p, cu_seqlens, total_text, aug_rows, q_aug, k_aug, v_aug, o_aug, lse, do_aug, dq_aug, dk_aug,
                     dv_aug, workspace, dev_err=None, stream=None):
     rc = load().ksa_prefill_bwd(
-        ctypes.byref(p), cu_seqlens.numel() - 1, _ptr(cu_seqlens), total_text, aug_rows, _ptr(q_aug), _ptr(k_aug),
-        _ptr(v_aug), _ptr(o_aug), _ptr(lse), _ptr(do_aug), _ptr(dq_aug), _ptr(dk_aug), _ptr(dv_aug),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_err), _stream(stream))
+        ctypes.byref(p), cu_seqlens.numel() - 1, _ptr(cu_seqlens, I32), total_text, aug_rows, _ptr(q_aug, BF16),
+        _ptr(k_aug, BF16), _ptr(v_aug, BF16), _ptr(o_aug, BF16), _ptr(lse, F32), _ptr(do_aug, BF16),
+        _ptr(dq_aug, BF16), _ptr(dk_aug, BF16), _ptr(dv_aug, BF16), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_err, I32), _stream(stream))
     _check("ksa_prefill_bwd", rc)
 
 
@@ -226,20 +236,21 @@ def ksa_cache_slots(p: ksa_params, cap_summaries: int) -> int:
 
 
 def make_cache(k, v, state, cap_summaries) -> ksa_cache:
-    return ksa_cache(_ptr(k), _ptr(v), _ptr(state), state.shape[0], cap_summaries)
+    return ksa_cache(_ptr(k, BF16), _ptr(v, BF16), _ptr(state, I32), state.shape[0], cap_summaries)
 
 
 def ksa_cache_append(p, cache: ksa_cache, kind, k_new, v_new, stream=None):
-    rc = load().ksa_cache_append(ctypes.byref(p), ctypes.byref(cache), _ptr(kind), _ptr(k_new), _ptr(v_new),
-                                 _stream(stream))
+    rc = load().ksa_cache_append(ctypes.byref(p), ctypes.byref(cache), _ptr(kind, I8), _ptr(k_new, BF16),
+                                 _ptr(v_new, BF16), _stream(stream))
     _check("ksa_cache_append", rc)
 
 
 def ksa_cache_from_prefill(p, cache: ksa_cache, cu_seqlens, total_text, aug_rows, k_aug, v_aug, workspace,
                            dev_err=None, stream=None):
-    rc = load().ksa_cache_from_prefill(ctypes.byref(p), ctypes.byref(cache), _ptr(cu_seqlens), total_text, aug_rows,
-                                       _ptr(k_aug), _ptr(v_aug), _ptr(workspace),
-                                       workspace.numel() * workspace.element_size(), _ptr(dev_err), _stream(stream))
+    rc = load().ksa_cache_from_prefill(ctypes.byref(p), ctypes.byref(cache), _ptr(cu_seqlens, I32), total_text,
+                                       aug_rows, _ptr(k_aug, BF16), _ptr(v_aug, BF16), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _ptr(dev_err, I32),
+                                       _stream(stream))
     _check("ksa_cache_from_prefill", rc)
 
 
@@ -250,10 +261,10 @@ def ksa_prefill_chunk_workspace_size(p: ksa_params, batch: int, total_text: int,
 def ksa_prefill_chunk(p, cache: ksa_cache, cu_text, total_text, cu_sum, total_sum, q_text, k_text, v_text, q_sum,
                       k_sum, v_sum, o_text, o_sum, lse_text, lse_sum, workspace, dev_err=None, stream=None):
     rc = load().ksa_prefill_chunk(
-        ctypes.byref(p), ctypes.byref(cache), _ptr(cu_text), total_text, _ptr(cu_sum), total_sum, _ptr(q_text),
-        _ptr(k_text), _ptr(v_text), _ptr(q_sum), _ptr(k_sum), _ptr(v_sum), _ptr(o_text), _ptr(o_sum),
-        _ptr(lse_text), _ptr(lse_sum), _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _ptr(dev_err), _stream(stream))
+        ctypes.byref(p), ctypes.byref(cache), _ptr(cu_text, I32), total_text, _ptr(cu_sum, I32), total_sum,
+        _ptr(q_text, BF16), _ptr(k_text, BF16), _ptr(v_text, BF16), _ptr(q_sum, BF16), _ptr(k_sum, BF16),
+        _ptr(v_sum, BF16), _ptr(o_text, BF16), _ptr(o_sum, BF16), _ptr(lse_text, F32), _ptr(lse_sum, F32),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_err, I32), _stream(stream))
     _check("ksa_prefill_chunk", rc)
 
 
@@ -262,16 +273,16 @@ def ksa_decode_workspace_size(p: ksa_params, batch: int, max_text: int) -> int:
 
 
 def ksa_decode(p, cache: ksa_cache, kind, q, o, lse, max_text, workspace, stream=None):
-    rc = load().ksa_decode(ctypes.byref(p), ctypes.byref(cache), _ptr(kind), _ptr(q), _ptr(o), _ptr(lse),
-                           max_text, _ptr(workspace), workspace.numel() * workspace.element_size(),
+    rc = load().ksa_decode(ctypes.byref(p), ctypes.byref(cache), _ptr(kind, I8), _ptr(q, BF16), _ptr(o, BF16),
+                           _ptr(lse, F32), max_text, _ptr(workspace), workspace.numel() * workspace.element_size(),
                            _stream(stream))
     _check("ksa_decode", rc)
 
 
 def ksa_decode_noalloc(p, cache: ksa_cache, kind, q, o, lse, max_text, stream=None):
     """ksa_decode with the library's own fixed scratch instead of a workspace."""
-    rc = load().ksa_decode_noalloc(ctypes.byref(p), ctypes.byref(cache), _ptr(kind), _ptr(q), _ptr(o), _ptr(lse),
-                                   max_text, _stream(stream))
+    rc = load().ksa_decode_noalloc(ctypes.byref(p), ctypes.byref(cache), _ptr(kind, I8), _ptr(q, BF16),
+                                   _ptr(o, BF16), _ptr(lse, F32), max_text, _stream(stream))
     _check("ksa_decode_noalloc", rc)
 
 
@@ -281,7 +292,7 @@ def make_mla_params(k: int, w: int, num_heads: int, kv_lora_rank: int = 512, rop
 
 
 def make_mla_cache(latent, state, cap_summaries) -> ksa_mla_cache:
-    return ksa_mla_cache(_ptr(latent), _ptr(state), state.shape[0], cap_summaries)
+    return ksa_mla_cache(_ptr(latent, BF16), _ptr(state, I32), state.shape[0], cap_summaries)
 
 
 def ksa_mla_cache_slots(p: ksa_mla_params, cap_summaries: int) -> int:
@@ -289,7 +300,8 @@ def ksa_mla_cache_slots(p: ksa_mla_params, cap_summaries: int) -> int:
 
 
 def ksa_mla_cache_append(p, cache: ksa_mla_cache, kind, x, stream=None):
-    rc = load().ksa_mla_cache_append(ctypes.byref(p), ctypes.byref(cache), _ptr(kind), _ptr(x), _stream(stream))
+    rc = load().ksa_mla_cache_append(ctypes.byref(p), ctypes.byref(cache), _ptr(kind, I8), _ptr(x, BF16),
+                                     _stream(stream))
     _check("ksa_mla_cache_append", rc)
 
 
@@ -298,11 +310,11 @@ def ksa_mla_decode_workspace_size(p: ksa_mla_params, batch: int, max_text: int) 
 
 
 def ksa_mla_decode(p, cache: ksa_mla_cache, kind, q, o, lse, max_text, workspace, stream=None):
-    rc = load().ksa_mla_decode(ctypes.byref(p), ctypes.byref(cache), _ptr(kind), _ptr(q), _ptr(o), _ptr(lse),
-                               max_text, _ptr(workspace), workspace.numel() * workspace.element_size(),
-                               _stream(stream))
+    rc = load().ksa_mla_decode(ctypes.byref(p), ctypes.byref(cache), _ptr(kind, I8), _ptr(q, BF16),
+                               _ptr(o, BF16), _ptr(lse, F32), max_text, _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
     _check("ksa_mla_decode", rc)
 
 
 def ksa_get_device_error(dev_err, stream=None) -> int:
-    return int(load().ksa_get_device_error(_ptr(dev_err), _stream(stream)))
+    return int(load().ksa_get_device_error(_ptr(dev_err, I32), _stream(stream)))

@@ -90,3 +90,43 @@ def test_binding_refuses_host_tensors(lib):
     from kv_cache_compression_ksa_b200 import _lib as L
     with pytest.raises(ValueError):
         L._ptr(torch.zeros(4))
+
+
+def test_binding_checks_element_types(lib):
+    """Each tensor argument must have the element type include/ksa.h
+    documents (bf16 data, fp32 LSE, int32 offsets / state / error words,
+    int8 kinds).  The check runs before the device check, so a wrong type
+    is named even on a host without a GPU; an int stands for a raw device
+    address and passes through, so the arguments before the one under test
+    are given as ints."""
+    import torch
+    from kv_cache_compression_ksa_b200 import _lib as L
+    p = L.make_params(8, 2, 8, 2, 64)
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    cu = torch.tensor([0, 16], dtype=torch.int32)
+    ws = torch.zeros(64, dtype=torch.uint8)
+    A = 256   # a stand-in device address
+    # prefill: int64 offsets are refused by the call; fp16 data and bf16 LSE
+    # by the marshalling every call uses
+    with pytest.raises(ValueError, match="int32"):
+        L.ksa_prefill_fwd(p, cu.long(), 16, 18, A, A, A, A, None, ws)
+    with pytest.raises(ValueError, match="bfloat16"):
+        L._ptr(bf(18, 8, 64).half(), L.BF16)
+    with pytest.raises(ValueError, match="float32"):
+        L._ptr(bf(18, 8), L.F32)
+    # the right type on the host gets as far as the device check
+    with pytest.raises(ValueError, match="CUDA device"):
+        L._ptr(torch.zeros(18, 8), L.F32)
+    # decode cache: int64 state; int32 / uint8 kinds
+    with pytest.raises(ValueError, match="int32"):
+        L.make_cache(A, A, torch.zeros(1, 4, dtype=torch.int64), 4)
+    cache = L.ksa_cache(0, 0, 0, 1, 4)
+    with pytest.raises(ValueError, match="int8"):
+        L.ksa_decode(p, cache, torch.zeros(1, dtype=torch.int32), A, A, None, 16, ws)
+    with pytest.raises(ValueError, match="int8"):
+        L.ksa_cache_append(p, cache, torch.zeros(1, dtype=torch.uint8), A, A)
+    # MLA: fp32 latent rows
+    pm = L.make_mla_params(8, 2, 16)
+    mc = L.ksa_mla_cache(0, 0, 1, 4)
+    with pytest.raises(ValueError, match="bfloat16"):
+        L.ksa_mla_cache_append(pm, mc, A, torch.zeros(1, 576))

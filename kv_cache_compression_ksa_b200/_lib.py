@@ -317,4 +317,7 @@ def ksa_mla_decode(p, cache: ksa_mla_cache, kind, q, o, lse, max_text, workspace
 
 
 def ksa_get_device_error(dev_err, stream=None) -> int:
-    return int(load().ksa_get_device_error(_ptr(dev_err, I32), _stream(stream)))
+    """Read and clear a device error word: an int32 word, or a byte
+    workspace whose first word the calls used because they were given none."""
+    ptr = _ptr(dev_err) if isinstance(dev_err, torch.Tensor) and dev_err.dtype == torch.uint8 else _ptr(dev_err, I32)
+    return int(load().ksa_get_device_error(ptr, _stream(stream)))

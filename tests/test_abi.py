@@ -125,6 +125,11 @@ def test_binding_checks_element_types(lib):
         L.ksa_decode(p, cache, torch.zeros(1, dtype=torch.int32), A, A, None, 16, ws)
     with pytest.raises(ValueError, match="int8"):
         L.ksa_cache_append(p, cache, torch.zeros(1, dtype=torch.uint8), A, A)
+    # an error word is int32, or the byte workspace that holds the default one
+    with pytest.raises(ValueError, match="int32"):
+        L.ksa_get_device_error(torch.zeros(1, dtype=torch.int64))
+    with pytest.raises(ValueError, match="CUDA device"):
+        L.ksa_get_device_error(torch.zeros(16, dtype=torch.uint8))
     # MLA: fp32 latent rows
     pm = L.make_mla_params(8, 2, 16)
     mc = L.ksa_mla_cache(0, 0, 1, 4)

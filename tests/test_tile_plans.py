@@ -430,3 +430,12 @@ def test_chunk_keys_are_read_where_the_cache_holds_them(harness, k, w):
             else:
                 assert (src, at) == (1, j - m0)
 
+
+
+def test_wide_window_tile_lists(harness):
+    """The sliding chunk number 128 of the benchmarked sweep (a 1024-token
+    window at k = 8): a work item's window spans many K/V tiles; forward
+    items, chunked-prefill items and backward tiles all stay exact."""
+    fwd_case(harness, 8, 128, 32, 8, [3000, 1100, 9])
+    chunk_case(harness, 8, 128, 32, 8, [(1500, 187, 700), (2048, 255, 64), (7, 0, 1200)])
+    bwd_case(harness, 8, 128, 32, 8, [3000, 1100, 9])

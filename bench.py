@@ -49,14 +49,22 @@ TRAFFIC = {
 DC = dict(B=64, m=16384, k=8, w=8, Hq=32, Hkv=8, d=128, seed=3, theta=1e6)
 
 
+def text_row_keys(i, k, w, m):
+    """Keys text rows i see (Eqs. (2)-(3)): the window text from chunk
+    max(c - w, 0) up to the row itself, and the summaries s_0 .. s_{c-w-1}
+    (of m in the sequence); c = i // k."""
+    i = np.asarray(i, dtype=np.int64)
+    c = i // k
+    return (i - np.maximum(c - w, 0) * k + 1) + np.clip(c - w, 0, m)
+
+
 def useful_pairs(seqlens, k, w):
-    """Visible (query, key) pairs per head (closed form of Eqs. (2)-(3))."""
+    """Visible (query, key) pairs per head: the text rows' keys plus k + 1
+    for each summary row."""
     tot = 0
     for n in seqlens:
-        i = np.arange(n, dtype=np.int64)
-        c = i // k
         m = n // k
-        tot += int(((i - np.maximum(c - w, 0) * k + 1) + np.clip(c - w, 0, m)).sum()) + m * (k + 1)
+        tot += int(text_row_keys(np.arange(n), k, w, m).sum()) + m * (k + 1)
     return tot
 
 
@@ -68,9 +76,7 @@ def chunk_pairs(n0, m0, T, k, w):
     """Visible (query, key) pairs per head of a chunked-prefill block: text
     positions n0 .. n0+T-1 (Eqs. (2)-(3)) and the summaries m0 .. m1-1 of the
     chunks it completes (k + 1 keys each)."""
-    i = np.arange(n0, n0 + T, dtype=np.int64)
-    c = i // k
-    text = int(((i - np.maximum(c - w, 0) * k + 1) + np.maximum(c - w, 0)).sum())
+    text = int(text_row_keys(np.arange(n0, n0 + T), k, w, (n0 + T) // k).sum())
     return text + ((n0 + T) // k - m0) * (k + 1)
 
 
@@ -242,9 +248,7 @@ def oracle_sample(sample_rows: int, seed: int = 1):
     t0 = time.perf_counter()
     oracle.ksa_attention(n, k, w, qt, kt, vt, qs, ks, vs, tq_idx=rows, sq_idx=np.zeros(0, np.int64))
     dt = time.perf_counter() - t0
-    c = rows // k
-    keys = (rows - np.maximum(c - w, 0) * k + 1) + np.clip(c - w, 0, n // k)
-    flops = float(keys.sum()) * PF["Hq"] * 4 * PF["d"]
+    flops = float(text_row_keys(rows, k, w, n // k).sum()) * PF["Hq"] * 4 * PF["d"]
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return flops / dt / 1e12, cores, len(rows), dt
 

@@ -87,3 +87,13 @@ def test_decode_slice_rows_equal_the_oracle_cache(k, w):
             n = m * k + fill + 1
             M, tpos, _ = mask_views(n, k, w)
             assert bench.decode_slice_rows(m, k, w, [fill])[0] == hi - lo == int(M[tpos(n - 1)].sum())
+
+
+@pytest.mark.parametrize("k,w", [(1, 0), (3, 2), (8, 8), (16, 1)])
+def test_text_row_keys_row_by_row(k, w):
+    """The per-row key count (shared by the pair totals and the CPU
+    baseline's FLOP count) equals each text row's mask row."""
+    for n in (1, k, 5 * k + 3, 200):
+        M, tpos, _ = mask_views(n, k, w)
+        want = [int(M[tpos(p)].sum()) for p in range(n)]
+        assert bench.text_row_keys(np.arange(n), k, w, n // k).tolist() == want

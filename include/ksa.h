@@ -55,7 +55,8 @@ extern "C" {
 /* Shape and method parameters shared by all calls. */
 typedef struct ksa_params {
     int32_t k;            /* chunk size: text tokens per chunk (>= 1)           */
-    int32_t w;            /* sliding chunk number C of Eqs. (2)-(3) (>= 0)      */
+    int32_t w;            /* sliding chunk number C of Eqs. (2)-(3) (>= 0;      *
+                           * (w+1)*k <= 2^30, else KSA_ERR_UNSUPPORTED)        */
     int32_t num_q_heads;  /* Hq                                                 */
     int32_t num_kv_heads; /* Hkv; q head h reads kv head h / (Hq/Hkv)           */
     int32_t head_dim;     /* d: 64 or 128                                       */
@@ -338,7 +339,7 @@ KSA_API int ksa_decode_noalloc(const ksa_params *p, const ksa_cache *cache, cons
  * ------------------------------------------------------------------------ */
 typedef struct ksa_mla_params {
     int32_t k;            /* chunk size (>= 1)                                   */
-    int32_t w;            /* sliding chunk number (>= 0)                         */
+    int32_t w;            /* sliding chunk number (>= 0; (w+1)*k <= 2^30)        */
     int32_t num_heads;    /* query heads (all read the same latent rows)         */
     int32_t kv_lora_rank; /* d_c: 512                                            */
     int32_t rope_dim;     /* d_r: 64                                             */

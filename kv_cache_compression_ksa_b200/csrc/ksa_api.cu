@@ -25,10 +25,18 @@ int sm_count()
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shape checks shared by every call.
+// The window the kernels index in 32-bit arithmetic: (w + 1) k text tokens.
+// A larger w (e.g. INT32_MAX for "every chunk") is refused, not wrapped;
+// w = the chunk count of the longest sequence gives full attention.
+constexpr int64_t kMaxWindowTokens = 1LL << 30;
+
+static bool window_fits(int k, int w) { return ((int64_t)w + 1) * (int64_t)k <= kMaxWindowTokens; }
+
 static int check_params(const ksa_params *p)
 {
     if (!p) return KSA_ERR_INVALID;
     if (p->k < 1 || p->w < 0 || p->num_q_heads < 1 || p->num_kv_heads < 1) return KSA_ERR_INVALID;
+    if (!window_fits(p->k, p->w)) return KSA_ERR_UNSUPPORTED;
     if (p->num_q_heads % p->num_kv_heads != 0) return KSA_ERR_INVALID;
     if (!(p->scale >= 0.f) || isinf(p->scale)) return KSA_ERR_INVALID;
     if (isnan(p->rope_theta)) return KSA_ERR_INVALID;
@@ -50,6 +58,7 @@ static int check_mla(const ksa_mla_params *p, const ksa_mla_cache *c, const int8
 {
     if (!p || !c) return KSA_ERR_INVALID;
     if (p->k < 1 || p->w < 0 || p->num_heads < 1 || p->kv_lora_rank < 1 || p->rope_dim < 0) return KSA_ERR_INVALID;
+    if (!window_fits(p->k, p->w)) return KSA_ERR_UNSUPPORTED;
     if (!(p->scale >= 0.f) || isinf(p->scale) || isnan(p->rope_theta)) return KSA_ERR_INVALID;
     if (p->kv_lora_rank != 512 || p->rope_dim != 64) return KSA_ERR_UNSUPPORTED;
     if (c->batch < 0 || c->cap_summaries < 0) return KSA_ERR_INVALID;
@@ -342,7 +351,7 @@ int ksa_mla_cache_append(const ksa_mla_params *p, const ksa_mla_cache *cache, co
 size_t ksa_mla_decode_workspace_size(const ksa_mla_params *p, int32_t batch, int64_t max_text)
 {
     if (!p || p->k < 1 || p->w < 0 || p->num_heads < 1 || batch < 0 || max_text < 0) return 0;
-    if (p->kv_lora_rank != 512 || p->rope_dim != 64) return 0;
+    if (!window_fits(p->k, p->w) || p->kv_lora_rank != 512 || p->rope_dim != 64) return 0;
     return mla_decode_workspace_bytes(p, batch, max_text);
 }
 

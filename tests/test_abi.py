@@ -135,3 +135,26 @@ def test_binding_checks_element_types(lib):
     mc = L.ksa_mla_cache(0, 0, 1, 4)
     with pytest.raises(ValueError, match="bfloat16"):
         L.ksa_mla_cache_append(pm, mc, A, torch.zeros(1, 576))
+
+
+def test_window_bound(lib):
+    """The kernels index the window ((w + 1) k text tokens) in 32-bit
+    arithmetic, so a larger window is refused before any launch instead of
+    wrapping; the largest allowed one is accepted."""
+    from kv_cache_compression_ksa_b200 import _lib as L
+    nul = ctypes.c_void_p(0)
+    edge = L.make_params(8, (1 << 27) - 1, 32, 8, 128)       # (w + 1) k = 2^30
+    over = L.make_params(8, 1 << 27, 32, 8, 128)
+    full = L.make_params(8, 2 ** 31 - 1, 32, 8, 128)        # "every chunk"
+    assert L.ksa_decode_workspace_size(edge, 4, 1000) > 0
+    assert L.ksa_decode_workspace_size(over, 4, 1000) == 0
+    assert L.ksa_prefill_bwd_workspace_size(full, 1, 9) == 0
+    for p in (over, full):
+        rc = lib.ksa_prefill_fwd(ctypes.byref(p), 1, 8, 8, 9, nul, nul, nul, nul, nul, 8, 64, nul, nul)
+        assert rc == L.KSA_ERR_UNSUPPORTED
+        cache = L.ksa_cache(16, 16, 16, 1, 4)
+        rc = lib.ksa_decode(ctypes.byref(p), ctypes.byref(cache), 16, 16, 16, nul, 100, 16, 1 << 20, nul)
+        assert rc == L.KSA_ERR_UNSUPPORTED
+    pm = L.make_mla_params(8, 1 << 27, 16)
+    assert L.ksa_mla_decode_workspace_size(pm, 4, 1000) == 0
+    assert L.ksa_mla_decode_workspace_size(L.make_mla_params(8, (1 << 27) - 1, 16), 4, 1000) > 0

@@ -439,3 +439,13 @@ def test_wide_window_tile_lists(harness):
     fwd_case(harness, 8, 128, 32, 8, [3000, 1100, 9])
     chunk_case(harness, 8, 128, 32, 8, [(1500, 187, 700), (2048, 255, 64), (7, 0, 1200)])
     bwd_case(harness, 8, 128, 32, 8, [3000, 1100, 9])
+
+
+def test_largest_accepted_window(harness):
+    """(w + 1) k = 2^30, the largest window the library accepts: the tile
+    lists' 32-bit index arithmetic does not wrap (every row sees all of its
+    sequence's earlier text and no summary)."""
+    w = (1 << 27) - 1
+    fwd_case(harness, 8, w, 32, 8, [1000, 300])
+    bwd_case(harness, 8, w, 32, 8, [1000, 300])
+    chunk_case(harness, 8, w, 32, 8, [(500, 62, 300)])

@@ -532,6 +532,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
 // fp32 accumulators -> bf16 dk, dv of the real rows (padding rows untouched)
 __global__ void __launch_bounds__(256) bwd_dkv_out_kernel(Args a, int D)
 {
+    if (*a.err != 0) return;   // the plan found cu_seqlens inconsistent: its rows may lie outside the buffers
     Blk K;
     if (!block_of(a, blockIdx.x, K)) return;
     const int g = blockIdx.y;

@@ -4,7 +4,8 @@ the oracle's fp64 backward, over varlen batches with partial chunks, GQA,
 w = 0, k = 1, a k that does not divide the 128-row tiles of the tensor-core
 kernels (warp-level path), k = 128 (dk/dv steps of 128 queries instead of
 64), k = 64 (a dk/dv step is one chunk) and a sequence long enough that the
-summary key tiles' text queries are split over several CTAs.
+summary key tiles' text queries are split over several CTAs; and
+inconsistent cu_seqlens on both paths (error recorded, nothing written).
 
 Tolerance: the kernels feed P and dS to the tensor cores in bf16 (relative
 rounding 2^-9 each) and write bf16 gradients, accumulating in fp32, so the
@@ -218,3 +219,30 @@ def test_autograd_function_matches_the_library_chain():
     for g_, w_ in zip(grads, want):
         assert g_.dtype == torch.bfloat16 and g_.shape == w_.shape
         assert torch.equal(g_, w_)
+
+
+@pytest.mark.parametrize("k", [8, 6])   # tensor-core path; warp-level path (6 does not divide 128)
+def test_prefill_bwd_inconsistent_cu_seqlens_writes_nothing(k):
+    """cu_seqlens that disagree with the host totals: the plan kernel records
+    KSA_ERR_INVALID in the caller's error word and every kernel of the call
+    returns before writing a gradient (the offsets it would use are wrong)."""
+    w, Hq, Hkv, d = 2, 4, 2, 64
+    p = L.make_params(k, w, Hq, Hkv, d, 0.0, THETA)
+    dev = torch.device("cuda")
+    n = 10 * k
+    rows = L.ksa_aug_rows(p, [n])
+    bad_cu = torch.tensor([0, n + k], dtype=torch.int32, device=dev)   # says n + k, the host says n
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(7)
+    qa = torch.randn(rows, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+    ka = torch.randn(rows, Hkv, d, generator=gen, device=dev).to(torch.bfloat16)
+    oa = torch.randn(rows, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+    lse = torch.zeros(rows, Hq, dtype=torch.float32, device=dev)
+    dq = torch.full((rows, Hq, d), 5.0, dtype=torch.bfloat16, device=dev)
+    dk = torch.full((rows, Hkv, d), 5.0, dtype=torch.bfloat16, device=dev)
+    dv = torch.full((rows, Hkv, d), 5.0, dtype=torch.bfloat16, device=dev)
+    wsb = torch.empty(L.ksa_prefill_bwd_workspace_size(p, 1, rows), dtype=torch.uint8, device=dev)
+    L.ksa_prefill_bwd(p, bad_cu, n, rows, qa, ka, ka, oa, lse, oa, dq, dk, dv, wsb, dev_err=err)
+    assert L.ksa_get_device_error(err) == L.KSA_ERR_INVALID
+    for t in (dq, dk, dv):
+        assert torch.all(t == 5.0)

@@ -384,18 +384,24 @@ ORACLE_API void oracle_cache_decode(oracle_cache *c, int kind, int Hq, double sc
     oracle_cache_slice(c, kind, &lo, &hi);
     const int d = c->d, Hkv = c->Hkv, G = Hq / Hkv;
     const int64_t nk = hi - lo;
-    const double **keys = (const double **)malloc(sizeof(double *) * (nk + 1));
-    const double **vals = (const double **)malloc(sizeof(double *) * (nk + 1));
-    double *scores = (double *)malloc(sizeof(double) * (nk + 1));
-    for (int h = 0; h < Hq; ++h) {
-        int hk = h / G;
-        for (int64_t t = 0; t < nk; ++t) {
-            keys[t] = c->K + ((lo + t) * Hkv + hk) * (int64_t)d;
-            vals[t] = c->V + ((lo + t) * Hkv + hk) * (int64_t)d;
+    /* the query heads are independent: one per thread, each with its own
+     * key lists and score buffer (the per-head arithmetic is unchanged) */
+    #pragma omp parallel
+    {
+        const double **keys = (const double **)malloc(sizeof(double *) * (nk + 1));
+        const double **vals = (const double **)malloc(sizeof(double *) * (nk + 1));
+        double *scores = (double *)malloc(sizeof(double) * (nk + 1));
+        #pragma omp for schedule(static)
+        for (int h = 0; h < Hq; ++h) {
+            int hk = h / G;
+            for (int64_t t = 0; t < nk; ++t) {
+                keys[t] = c->K + ((lo + t) * Hkv + hk) * (int64_t)d;
+                vals[t] = c->V + ((lo + t) * Hkv + hk) * (int64_t)d;
+            }
+            attend(d, scale, q + (int64_t)h * d, nk, keys, vals, scores, o + (int64_t)h * d, lse + h);
         }
-        attend(d, scale, q + (int64_t)h * d, nk, keys, vals, scores, o + (int64_t)h * d, lse + h);
+        free(keys); free(vals); free(scores);
     }
-    free(keys); free(vals); free(scores);
 }
 
 /* Decode over an externally held cache image laid out [S, Hkv, d] (the

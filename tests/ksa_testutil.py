@@ -29,6 +29,27 @@ def assert_close(gpu: np.ndarray, ref: np.ndarray, what: str, max_abs=MAX_ABS, r
     return ma, rf
 
 
+class RowSet:
+    """Output rows of one test compared with the oracle: max-abs on every row
+    as it is added, relative Frobenius over all added rows together (the bar
+    applies to the test's outputs as one set, so a row whose reference is
+    small does not decide it alone)."""
+
+    def __init__(self, what: str, max_abs=MAX_ABS, rel_frob=REL_FROB):
+        self.what, self.max_abs, self.rel_frob = what, max_abs, rel_frob
+        self.got, self.want = [], []
+
+    def add(self, gpu: np.ndarray, ref: np.ndarray, what: str):
+        assert_close(gpu, ref, what, max_abs=self.max_abs, rel_frob=None)
+        self.got.append(np.asarray(gpu, np.float64).ravel())
+        self.want.append(np.asarray(ref, np.float64).ravel())
+
+    def check(self):
+        assert self.got, f"{self.what}: no rows were checked"
+        return assert_close(np.concatenate(self.got), np.concatenate(self.want), self.what,
+                            max_abs=self.max_abs, rel_frob=self.rel_frob)
+
+
 def chunk_offsets(seqlens, k):
     off = [0]
     for n in seqlens:

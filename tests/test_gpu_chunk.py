@@ -17,7 +17,7 @@ import oracle
 from kv_cache_compression_ksa_b200 import _lib as L
 from kv_cache_compression_ksa_b200.api import DecodeCache
 from kv_cache_compression_ksa_b200.inputs import token_stream
-from ksa_testutil import LSE_ABS, assert_close, sample_rows, to_f64
+from ksa_testutil import LSE_ABS, RowSet, assert_close, sample_rows, to_f64
 
 pytestmark = pytest.mark.gpu
 THETA = 1e6
@@ -184,11 +184,13 @@ def test_chunk_cache_equals_one_pass_handoff(k, w, Hq, Hkv, d):
                  torch.stack([s[2][n] for s, n in zip(streams, n1s)]).cuda())
     o, lse = cache.decode(kind, torch.stack([s[0][n] for s, n in zip(streams, n1s)]).cuda(), max(n1s) + 1)
     o, lse = to_f64(o), to_f64(lse)
+    rows = RowSet("decode after chunks")
     for b, n in enumerate(n1s):
         ref = oracle.ksa_prefill([n + 1], k, w, *[to_f64(t) for t in streams[b]], THETA,
                                  text_rows=[np.array([n])], sum_rows=[np.zeros(0, np.int64)])[0]
-        assert_close(o[b], ref.text_o[0], f"decode after chunks, seq {b}", rel_frob=None)
+        rows.add(o[b], ref.text_o[0], f"decode after chunks, seq {b}")
         assert_close(lse[b], ref.text_lse[0], f"lse after chunks, seq {b}", max_abs=LSE_ABS, rel_frob=None)
+    rows.check()
 
 
 def test_chunk_state_errors():

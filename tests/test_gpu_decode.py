@@ -10,7 +10,7 @@ import oracle
 from kv_cache_compression_ksa_b200 import _lib as L
 from kv_cache_compression_ksa_b200.api import DecodeCache
 from kv_cache_compression_ksa_b200.inputs import fill_normal_, token_stream, uniform_ints
-from ksa_testutil import LSE_ABS, assert_close, to_f64
+from ksa_testutil import LSE_ABS, RowSet, assert_close, to_f64
 
 pytestmark = pytest.mark.gpu
 THETA = 1e6
@@ -109,6 +109,7 @@ def test_decode_steps_equal_prefill_rows(k, w, Hq, Hkv, d):
                 ev.append(("s", (i + 1) // k - 1))
         events.append(ev)
     steps = max(len(e) for e in events)
+    rows = RowSet(f"decode outputs k{k} w{w} G{Hq // Hkv} d{d}")
     for s in range(steps):
         kinds, kn, vn, qn = [], [], [], []
         for b in range(B):
@@ -129,11 +130,12 @@ def test_decode_steps_equal_prefill_rows(k, w, Hq, Hkv, d):
             ev = events[b][s] if s < len(events[b]) else ("skip", None)
             r = refs[b]
             if ev[0] == "t":
-                assert_close(o[b], r.text_o[ev[1]], f"text step {ev[1]}", rel_frob=None)
+                rows.add(o[b], r.text_o[ev[1]], f"text step {ev[1]}")
                 assert_close(lse[b], r.text_lse[ev[1]], f"text lse {ev[1]}", max_abs=LSE_ABS, rel_frob=None)
             elif ev[0] == "s":
-                assert_close(o[b], r.sum_o[ev[1]], f"summary step {ev[1]}", rel_frob=None)
+                rows.add(o[b], r.sum_o[ev[1]], f"summary step {ev[1]}")
                 assert_close(lse[b], r.sum_lse[ev[1]], f"summary lse {ev[1]}", max_abs=LSE_ABS, rel_frob=None)
+    rows.check()
     assert (cache.state[:, 3] == 0).all()
 
 
@@ -175,19 +177,20 @@ def test_decode_full_size_against_cache_model(B, m_chunks, nsample):
     assert np.all(st[:, 3] == 0)
     np.testing.assert_array_equal(st[:, 0], m_chunks * k + fills + 1)
     pos = st[:, 0] - 1
+    rows = RowSet(f"decode {B} x {m_chunks} summaries")
     for b in sorted(set(np.linspace(0, B - 1, nsample).astype(int).tolist())):
         Kimg, Vimg = gpu_image(cache, b)
-        # the library rotates q at position n_text-1 and keeps it in bf16
+        # the oracle rotates the bf16 input query itself, in fp64
         qr = oracle.rope(to_f64(q[b])[None], np.array([pos[b]]), THETA)[0]
-        qr = to_f64(torch.from_numpy(qr).to(torch.bfloat16))
         want_o, want_l = oracle.decode_image(k, w, cache.cap, int(st[b, 0]), int(st[b, 1]), oracle.TEXT,
                                              Kimg, Vimg, qr)
-        assert_close(o[b], want_o, f"decode seq {b}", rel_frob=None)
+        rows.add(o[b], want_o, f"decode seq {b}")
         assert_close(lse[b], want_l, f"decode lse {b}", max_abs=LSE_ABS, rel_frob=None)
         # the appended key is the rotated input, one bf16 rounding away
         kr = oracle.rope(to_f64(kn[b])[None], np.array([pos[b]]), THETA)[0]
         slot = k - fills[b]
         assert np.all(np.abs(Kimg[slot] - kr) <= 2.0 ** -8 * np.abs(kr) + 1e-5)
+    rows.check()
 
 
 def test_decode_multistep_ring_wrap_and_summaries():
@@ -203,6 +206,7 @@ def test_decode_multistep_ring_wrap_and_summaries():
     ws = cache.workspace(m0 * k + 80)
     fill = fills.copy()
     watch = [0, 11]
+    rows = RowSet("decode multistep outputs")
     for step in range(64):
         for phase in ("text", "summary"):
             if phase == "text":
@@ -224,15 +228,15 @@ def test_decode_multistep_ring_wrap_and_summaries():
                     continue
                 Kimg, Vimg = gpu_image(cache, b)
                 qr = oracle.rope(to_f64(q[b])[None], np.array([st[b, 0] - 1]), THETA)[0]
-                qr = to_f64(torch.from_numpy(qr).to(torch.bfloat16))
                 kd = oracle.TEXT if kinds[b] == TEXT else oracle.SUMMARY
                 want_o, want_l = oracle.decode_image(k, w, cache.cap, int(st[b, 0]), int(st[b, 1]), kd,
                                                      Kimg, Vimg, qr)
-                assert_close(to_f64(o[b]), want_o, f"step {step} seq {b} {phase}", rel_frob=None)
+                rows.add(to_f64(o[b]), want_o, f"step {step} seq {b} {phase}")
                 assert_close(to_f64(lse[b]), want_l, f"step {step} seq {b} lse", max_abs=LSE_ABS, rel_frob=None)
             if phase == "text":
                 fill = fill + 1
             else:
                 fill = np.where(kinds == SUMMARY, 0, fill)
+    rows.check()
     assert (cache.state[:, 3] == 0).all()
     assert (cache.state[:, 1].cpu().numpy() > m0).all()

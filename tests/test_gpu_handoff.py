@@ -11,7 +11,7 @@ import oracle
 from kv_cache_compression_ksa_b200 import _lib as L
 from kv_cache_compression_ksa_b200.api import DecodeCache
 from kv_cache_compression_ksa_b200.inputs import token_stream
-from ksa_testutil import LSE_ABS, assert_close, to_f64
+from ksa_testutil import LSE_ABS, RowSet, assert_close, to_f64
 
 pytestmark = pytest.mark.gpu
 THETA = 1e6
@@ -85,12 +85,14 @@ def test_cache_from_prefill_equals_appends(seqlens, k, w, Hq, Hkv, d):
     o, lse = cache.decode(kind, qn, max(seqlens) + 1)
     o, lse = to_f64(o), to_f64(lse)
     assert (cache.state[:, 3] == 0).all()
+    rows = RowSet("decode after hand-off")
     for b, n in enumerate(seqlens):
         s = streams[b]
         ref = oracle.ksa_prefill([n + 1], k, w, *[to_f64(t) for t in s], THETA, text_rows=[np.array([n])],
                                  sum_rows=[np.zeros(0, np.int64)])[0]
-        assert_close(o[b], ref.text_o[0], f"decode after hand-off, seq {b}", rel_frob=None)
+        rows.add(o[b], ref.text_o[0], f"decode after hand-off, seq {b}")
         assert_close(lse[b], ref.text_lse[0], f"lse after hand-off, seq {b}", max_abs=LSE_ABS, rel_frob=None)
+    rows.check()
 
 
 def test_cache_from_prefill_capacity_error():

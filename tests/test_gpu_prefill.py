@@ -201,7 +201,8 @@ def test_visible_counts_full_size(seqlens, k, w, Hq, Hkv, d):
 
 @pytest.mark.parametrize("seqlens,w,scale,seed,nsample", [
     ([32768], 8, 0.5, 1, 160),
-    ([131072, 65536, 16384, 4003], 16, 1.0, 2, 48),
+    ([131072, 65536, 16384, 4000], 16, 1.0, 2, 48),     # the long varlen batch as written
+    ([131072, 65536, 16384, 4003], 16, 1.0, 2, 48),     # with a trailing partial chunk
 ])
 def test_prefill_full_size_sampled(seqlens, w, scale, seed, nsample):
     """Full-size workloads in the benchmark's launch configuration, checked on

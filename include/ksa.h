@@ -308,18 +308,21 @@ KSA_API int ksa_decode(const ksa_params *p, const ksa_cache *cache, const int8_t
  * custom op that is handed only its inputs and outputs has no allocator to
  * take a workspace from, and a cudaMalloc of its own would break that
  * ownership and stall the device in the middle of its decode loop.
- * Arguments and results are those of ksa_decode minus the workspace; the
- * split-K partials go to a 4 MiB device array that the library keeps on
- * every GPU that loads it, until the process exits.  The first call made
- * on a device looks up that array's device address, with that device
- * current; make this first call before any stream capture.  A problem whose
- * partials (ksa_decode_workspace_size) exceed 4 MiB returns
- * KSA_ERR_CAPACITY and launches nothing.  Every call shares the one array
- * and it keeps the last call's contents (nothing in it needs to start at
- * zero); calls whose kernels can overlap on the GPU (other streams, other
- * host threads) race on it, so the caller must order them.  The report has
- * no counterpart to this call: it serves the library's callers, not the
- * method. */
+ * Arguments, argument checks and results are those of ksa_decode minus the
+ * workspace; the split-K partials go to a 4 MiB device array that the
+ * library keeps on every GPU that loads it, until the process exits.  The
+ * first call made on a device looks up that array's device address, with
+ * that device current; make this first call before any stream capture.
+ * One split of the partials takes 4 * batch * num_q_heads * (head_dim + 2)
+ * bytes; the call uses as many of ksa_decode's splits as fit in 4 MiB
+ * (fewer splits only lengthen each split's share of the slice), and returns
+ * KSA_ERR_CAPACITY, launching nothing, when a single split does not fit
+ * (batch * num_q_heads * (head_dim + 2) > 1048576).  Every call shares the
+ * one array and it keeps the last call's contents (nothing in it needs to
+ * start at zero); calls whose kernels can overlap on the GPU (other
+ * streams, other host threads) race on it, so the caller must order them.
+ * The report has no counterpart to this call: it serves the library's
+ * callers, not the method. */
 KSA_API int ksa_decode_noalloc(const ksa_params *p, const ksa_cache *cache, const int8_t *kind,
                                const void *q, void *o, float *lse, int64_t max_text, void *stream);
 
@@ -382,6 +385,23 @@ KSA_API int ksa_mla_decode(const ksa_mla_params *p, const ksa_mla_cache *cache, 
 /* Synchronise `stream`, return the device error word (KSA_OK if clear) and
  * reset it to KSA_OK.  dev_err: device int32. */
 KSA_API int ksa_get_device_error(int32_t *dev_err, void *stream);
+
+/* Self-check of the bounded-wait error path of the tensor-core pipelines
+ * (the prefill, its backward and the chunked prefill): every mbarrier wait
+ * there gives up after a bounded number of polls or sleeps, records
+ * KSA_ERR_TIMEOUT in the caller's error word, makes the CTA's other roles
+ * stop waiting, and the CTA frees its tensor memory and exits, so the
+ * context stays usable.  This call launches one CTA of 128 threads that
+ * allocates all 512 TMEM columns of its SM and waits, with those same
+ * routines, on two mbarriers that nothing ever completes: one waiter polls
+ * (at most poll_limit polls, 1 .. 2^22), one sleeps in try_wait (at most
+ * sleep_limit sleeps of up to 20 us, 1 .. 2^17).  Afterwards *dev_err holds
+ * KSA_ERR_TIMEOUT (read it with ksa_get_device_error) and the TMEM is
+ * free again.  No passage of the report corresponds to it: it checks the
+ * library's own failure handling.  dev_err: device int32, 4-byte aligned.
+ * Returns KSA_ERR_INVALID for a limit out of range or a bad error word. */
+KSA_API int ksa_selftest_wait_timeout(uint32_t poll_limit, uint32_t sleep_limit, int32_t *dev_err,
+                                      void *stream);
 
 /* Human-readable name of a status code (static storage). */
 KSA_API const char *ksa_status_string(int status);

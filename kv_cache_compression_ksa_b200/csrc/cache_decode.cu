@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeArgs a, __nv_
     }
 }
 
-static int decode_splits(const ksa_params *p, int batch, int64_t max_text)
+int decode_splits(const ksa_params *p, int batch, int64_t max_text)
 {
     int64_t max_slice = 1 + p->k + (int64_t)p->w * p->k + max_text / p->k;
     int64_t units = (int64_t)batch * p->num_kv_heads;
@@ -517,11 +517,15 @@ static int decode_splits(const ksa_params *p, int batch, int64_t max_text)
     return (int)s;
 }
 
+size_t decode_split_bytes(const ksa_params *p, int batch)
+{
+    const int G = p->num_q_heads / p->num_kv_heads;
+    return sizeof(float) * (size_t)batch * p->num_kv_heads * G * (2 + p->head_dim);
+}
+
 size_t decode_workspace_bytes(const ksa_params *p, int batch, int64_t max_text)
 {
-    int G = p->num_q_heads / p->num_kv_heads;
-    int s = decode_splits(p, batch, max_text);
-    return align_up(sizeof(float) * (size_t)batch * p->num_kv_heads * s * G * (2 + p->head_dim));
+    return align_up(decode_split_bytes(p, batch) * (size_t)decode_splits(p, batch, max_text));
 }
 
 template <int D, int G>
@@ -539,9 +543,17 @@ int launch_decode(const ksa_params *p, const ksa_cache *c, const int8_t *kind, c
 {
     if (c->batch == 0) return KSA_OK;
     if (ws_bytes < decode_workspace_bytes(p, c->batch, max_text)) return KSA_ERR_WORKSPACE;
+    return launch_decode_splits(p, c, kind, q, o, lse, decode_splits(p, c->batch, max_text), ws, st);
+}
+
+int launch_decode_splits(const ksa_params *p, const ksa_cache *c, const int8_t *kind, const void *q, void *o,
+                         float *lse, int nsplit, void *ws, cudaStream_t st)
+{
+    if (c->batch == 0) return KSA_OK;
+    if (nsplit < 1) return KSA_ERR_INVALID;
     DecodeArgs a;
     a.k = p->k; a.w = p->w; a.Hkv = p->num_kv_heads; a.Hq = p->num_q_heads;
-    a.nsplit = decode_splits(p, c->batch, max_text);
+    a.nsplit = nsplit;
     a.S = ksa_cache_slots(p, c->cap_summaries);
     float scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->head_dim);
     a.scale_log2 = scale * 1.4426950408889634f;

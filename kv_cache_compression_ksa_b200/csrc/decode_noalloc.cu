@@ -20,8 +20,12 @@
 
 namespace ksa {
 
-// 4 MiB: enough for the split-K partials of 64 sequences x 8 kv heads x 4 q
-// heads per kv head at d = 128 with several splits (about 0.5 MiB per split).
+// 4 MiB.  One split of the partials (m, l and the d-wide accumulator of
+// every q head) takes 4 B x batch x Hq x (d + 2): 1.02 MiB for 64 sequences
+// x 32 q heads at d = 128, 0.25 MiB for 16 of them.  The call keeps as many
+// of ksa_decode's splits as fit (3 and 15 for those two batches) and
+// refuses only a batch whose single split does not fit (batch x Hq x (d + 2)
+// above 1 Mi floats).
 constexpr size_t kScratchBytes = 4u << 20;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
@@ -52,16 +56,17 @@ using namespace ksa;
 extern "C" KSA_API int ksa_decode_noalloc(const ksa_params *p, const ksa_cache *cache, const int8_t *kind,
                                           const void *q, void *o, float *lse, int64_t max_text, void *stream)
 {
-    if (!p || !cache) return KSA_ERR_INVALID;
-    if (max_text < 0 || cache->batch < 0) return KSA_ERR_INVALID;
-    if (cache->batch == 0) return KSA_OK;
-    if (p->num_kv_heads < 1 || p->num_q_heads < 1 || p->head_dim < 1) return KSA_ERR_INVALID;
-    // the partials this problem needs must fit the fixed scratch
-    size_t need = ksa_decode_workspace_size(p, cache->batch, max_text);
-    if (need == 0) return KSA_ERR_INVALID;
-    if (need > kScratchBytes) return KSA_ERR_CAPACITY;
-    void *scratch = nullptr;
-    int rc = scratch_for_current_device(&scratch);
+    // the same argument checks, in the same order, as ksa_decode
+    int rc = check_decode_args(p, cache, kind, q, o, lse, max_text);
     if (rc != KSA_OK) return rc;
-    return ksa_decode(p, cache, kind, q, o, lse, max_text, scratch, kScratchBytes, stream);
+    if (cache->batch == 0) return KSA_OK;
+    // as many of ksa_decode's splits as the fixed scratch holds
+    const size_t per_split = decode_split_bytes(p, cache->batch);
+    if (per_split > kScratchBytes) return KSA_ERR_CAPACITY;
+    int nsplit = decode_splits(p, cache->batch, max_text);
+    if ((size_t)nsplit * per_split > kScratchBytes) nsplit = (int)(kScratchBytes / per_split);
+    void *scratch = nullptr;
+    rc = scratch_for_current_device(&scratch);
+    if (rc != KSA_OK) return rc;
+    return launch_decode_splits(p, cache, kind, q, o, lse, nsplit, scratch, (cudaStream_t)stream);
 }

@@ -319,17 +319,31 @@ size_t ksa_decode_workspace_size(const ksa_params *p, int32_t batch, int64_t max
     return decode_workspace_bytes(p, batch, max_text);
 }
 
-int ksa_decode(const ksa_params *p, const ksa_cache *cache, const int8_t *kind, const void *q, void *o, float *lse,
-               int64_t max_text, void *workspace, size_t workspace_bytes, void *stream)
+}  // extern "C"
+
+namespace ksa {
+int check_decode_args(const ksa_params *p, const ksa_cache *cache, const int8_t *kind, const void *q,
+                      const void *o, const float *lse, int64_t max_text)
 {
     int rc = check_cache(p, cache, kind);
     if (rc != KSA_OK) return rc;
     if (max_text < 0) return KSA_ERR_INVALID;
     if (cache->batch > 0) {
-        if (!q || !o || !workspace || !aligned16(q) || !aligned16(o) || !aligned16(workspace))
-            return KSA_ERR_INVALID;
+        if (!q || !o || !aligned16(q) || !aligned16(o)) return KSA_ERR_INVALID;
         if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return KSA_ERR_INVALID;
     }
+    return KSA_OK;
+}
+}  // namespace ksa
+
+extern "C" {
+
+int ksa_decode(const ksa_params *p, const ksa_cache *cache, const int8_t *kind, const void *q, void *o, float *lse,
+               int64_t max_text, void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_decode_args(p, cache, kind, q, o, lse, max_text);
+    if (rc != KSA_OK) return rc;
+    if (cache->batch > 0 && (!workspace || !aligned16(workspace))) return KSA_ERR_INVALID;
     return launch_decode(p, cache, kind, q, o, lse, max_text, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 

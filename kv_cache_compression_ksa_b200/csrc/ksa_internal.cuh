@@ -124,9 +124,19 @@ int launch_cache_append(const ksa_params *p, const ksa_cache *c, const int8_t *k
                         const void *k_new, const void *v_new, cudaStream_t st);
 
 size_t decode_workspace_bytes(const ksa_params *p, int batch, int64_t max_text);
+// Split-K shape of the decode: the split count it chooses for a batch and
+// max_text, and the bytes of partials (m, l, acc) one split needs.
+int decode_splits(const ksa_params *p, int batch, int64_t max_text);
+size_t decode_split_bytes(const ksa_params *p, int batch);
 int launch_decode(const ksa_params *p, const ksa_cache *c, const int8_t *kind, const void *q,
                   void *o, float *lse, int64_t max_text, void *ws, size_t ws_bytes,
                   cudaStream_t st);
+// The same decode with an explicit split count; ws holds nsplit splits.
+int launch_decode_splits(const ksa_params *p, const ksa_cache *c, const int8_t *kind, const void *q, void *o,
+                         float *lse, int nsplit, void *ws, cudaStream_t st);
+// The argument checks of ksa_decode (everything but the workspace).
+int check_decode_args(const ksa_params *p, const ksa_cache *cache, const int8_t *kind, const void *q,
+                      const void *o, const float *lse, int64_t max_text);
 
 // Number of SMs of the current device (cached per device).
 int sm_count();

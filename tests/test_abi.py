@@ -158,3 +158,40 @@ def test_window_bound(lib):
     pm = L.make_mla_params(8, 1 << 27, 16)
     assert L.ksa_mla_decode_workspace_size(pm, 4, 1000) == 0
     assert L.ksa_mla_decode_workspace_size(L.make_mla_params(8, (1 << 27) - 1, 16), 4, 1000) > 0
+
+
+def test_noalloc_decode_checks_arguments_like_decode(lib):
+    """The no-workspace decode runs the same argument checks as ksa_decode
+    and returns the same status for the same bad call (a window beyond the
+    32-bit bound, bad parameters, a missing query, an empty batch), all
+    before any launch."""
+    from kv_cache_compression_ksa_b200 import _lib as L
+    nul = ctypes.c_void_p(0)
+    good = L.make_params(8, 8, 32, 8, 128)
+    cases = [
+        (L.make_params(8, 1 << 27, 32, 8, 128), L.ksa_cache(16, 16, 16, 1, 4), 16, L.KSA_ERR_UNSUPPORTED),
+        (L.make_params(0, 8, 32, 8, 128), L.ksa_cache(16, 16, 16, 1, 4), 16, L.KSA_ERR_INVALID),
+        (L.make_params(8, 8, 32, 8, 96), L.ksa_cache(16, 16, 16, 1, 4), 16, L.KSA_ERR_UNSUPPORTED),
+        (good, L.ksa_cache(16, 16, 16, 1, 4), 0, L.KSA_ERR_INVALID),          # no query
+        (good, L.ksa_cache(16, 16, 16, -1, 4), 16, L.KSA_ERR_INVALID),        # negative batch
+        (good, L.ksa_cache(0, 0, 0, 0, 4), 0, L.KSA_OK),                      # empty batch: nothing to do
+    ]
+    for p, cache, q, want in cases:
+        rc_ws = lib.ksa_decode(ctypes.byref(p), ctypes.byref(cache), 16, q, 16, nul, 100, 16, 1 << 20, nul)
+        rc_na = lib.ksa_decode_noalloc(ctypes.byref(p), ctypes.byref(cache), 16, q, 16, nul, 100, nul)
+        assert rc_ws == want and rc_na == want, (p.k, p.w, p.head_dim, cache.batch, rc_ws, rc_na)
+
+
+def test_selftest_wait_timeout_arguments(lib):
+    """The timeout self-check launches one CTA whose waits are bounded by the
+    given limits; limits outside (0, the pipelines' own limit] and a missing
+    error word are refused before the launch."""
+    from kv_cache_compression_ksa_b200 import _lib as L
+    nul = ctypes.c_void_p(0)
+    word = ctypes.c_void_p(1 << 20)
+    assert lib.ksa_selftest_wait_timeout(16, 16, nul, nul) == L.KSA_ERR_INVALID
+    assert lib.ksa_selftest_wait_timeout(0, 16, word, nul) == L.KSA_ERR_INVALID
+    assert lib.ksa_selftest_wait_timeout(16, 0, word, nul) == L.KSA_ERR_INVALID
+    assert lib.ksa_selftest_wait_timeout((1 << 22) + 1, 16, word, nul) == L.KSA_ERR_INVALID
+    assert lib.ksa_selftest_wait_timeout(16, (1 << 17) + 1, word, nul) == L.KSA_ERR_INVALID
+    assert lib.ksa_selftest_wait_timeout(16, 16, ctypes.c_void_p((1 << 20) + 2), nul) == L.KSA_ERR_INVALID

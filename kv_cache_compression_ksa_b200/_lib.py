@@ -114,6 +114,7 @@ SYMBOLS = {
     "ksa_mla_decode": (ctypes.c_int, [ctypes.POINTER(ksa_mla_params), ctypes.POINTER(ksa_mla_cache), _P, _P, _P, _P,
                                       _I64, _P, _SZ, _P]),
     "ksa_get_device_error": (ctypes.c_int, [_P, _P]),
+    "ksa_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_uint32, _P, _P]),
     "ksa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -314,6 +315,13 @@ def ksa_mla_decode(p, cache: ksa_mla_cache, kind, q, o, lse, max_text, workspace
                                _ptr(o, BF16), _ptr(lse, F32), max_text, _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream))
     _check("ksa_mla_decode", rc)
+
+
+def ksa_selftest_wait_timeout(poll_limit: int, sleep_limit: int, dev_err, stream=None):
+    """Run the bounded-wait self-check: its waits run out and record
+    KSA_ERR_TIMEOUT in dev_err (an int32 device word)."""
+    rc = load().ksa_selftest_wait_timeout(poll_limit, sleep_limit, _ptr(dev_err, I32), _stream(stream))
+    _check("ksa_selftest_wait_timeout", rc)
 
 
 def ksa_get_device_error(dev_err, stream=None) -> int:

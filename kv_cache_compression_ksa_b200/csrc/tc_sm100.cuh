@@ -89,10 +89,10 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
 // mbar_wait_sleep suspends between checks (for producer and issuer warps,
 // which would otherwise take issue slots from the compute warps).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          int32_t *err)
+                                          int32_t *err, uint32_t limit = kSpinLimit)
 {
     if (mbar_test(bar, parity)) return true;  // non-blocking fast path
-    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+    for (uint32_t it = 0; it < limit; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
     }
@@ -102,10 +102,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, volatile int *abort,
-                                                int32_t *err)
+                                                int32_t *err, uint32_t limit = kWaitLimit)
 {
     if (mbar_test(bar, parity)) return true;
-    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+    for (uint32_t it = 0; it < limit; ++it) {
         if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*abort) return false;
     }

@@ -108,10 +108,13 @@ def test_noalloc_decode_on_a_caller_stream():
     B, m = 8, 200
     p, cache = _cache(B, m, seed=60)
     kind = torch.zeros(B, dtype=torch.int8, device="cuda")
+    kn = torch.randn(B, p.num_kv_heads, p.head_dim, device="cuda").to(torch.bfloat16)
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
+        cache.append(kind, kn, kn, stream=s)      # every sequence gets its open token
         results = _two_calls(p, cache, kind, m * p.k + p.k, seed=61, stream=s)
+    assert (cache.state[:, 3] == 0).all()
     for call, (q, o1, l1, o2, l2) in enumerate(results):
         assert_close(o2, o1, f"noalloc on a stream, call {call} O", max_abs=MAX_ABS)
         assert_close(l2, l1, f"noalloc on a stream, call {call} LSE", max_abs=LSE_ABS, rel_frob=None)

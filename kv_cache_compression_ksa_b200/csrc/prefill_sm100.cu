@@ -21,10 +21,12 @@
 //     other kind.
 //   * A query tile is 128 TMEM lanes holding the G = Hq/Hkv heads of one kv
 //     head for floor(128/(G k)) chunks of text rows (GQA packing: every K/V
-//     tile serves all G heads).  Each CTA runs two query tiles (two softmax
-//     warpgroups) against one stream of K/V tiles: S = Q K^T and O += P V
-//     are tcgen05.mma (kind::f16, bf16 in, fp32 accumulate in TMEM); P is
-//     written back into TMEM as bf16 over S and fed as the A operand.
+//     tile serves all G heads).  Each CTA runs one query tile at a time
+//     against a stream of K/V tiles, its softmax split over the two 64-key
+//     halves of every tile (eight warps, each half with its own running max
+//     and O accumulator): S = Q K^T and O += P V are tcgen05.mma (kind::f16,
+//     bf16 in, fp32 accumulate in TMEM); P is written back into TMEM as bf16
+//     over S and fed as the A operand.
 //   * The set of K/V tiles of a work unit follows from its chunk
 //     coordinates: ceil(min(m, c_last-w)/128) summary tiles plus the window
 //     tiles covering chunks c_first-w .. c_last.  Every other tile of the
@@ -36,7 +38,8 @@
 //     LSE), which runs while the softmax warps start the next work item.
 //     All mbarrier waits are bounded; on expiry the CTA records
 //     KSA_ERR_TIMEOUT, drains, frees TMEM and exits.
-//   * Summary query rows (k+1 keys each) run in a separate CUDA-core kernel.
+//   * Summary query rows (k+1 keys each) run on the CUDA cores of the
+//     epilogue warps, between the items whose chunks they close.
 #include <cuda.h>
 #include <math.h>
 
@@ -100,6 +103,7 @@ struct Params {
     Plan pl;
     int32_t *err;
     const __nv_bfloat16 *q;   // augmented query tensor (read row by row into TMEM)
+    const __nv_bfloat16 *kk, *vv;   // augmented K and V (the summary rows' keys, read by the epilogue warps)
     __nv_bfloat16 *o;
     float *lse;
     // Chunk mode (a block of new tokens against a decode cache): per-sequence
@@ -115,6 +119,7 @@ struct Params {
     const int32_t *ck_ntot;       // [B] text tokens after the block
     const int32_t *ck_qbase, *ck_kvbase;
     int sum_slot0;
+    int sum_rows;   // 1: the epilogue warps also compute the summary rows of each item's chunks
 };
 
 // ---------------------------------------------------------------------------
@@ -177,8 +182,117 @@ __host__ __device__ __forceinline__ Unit unit_of(const Params &P, int item, int 
     return U;
 }
 
-// Persistent kernel: one CTA per SM walks work items blockIdx.x,
-// blockIdx.x + gridDim.x, ... (heavy first, round robin), so the loads and
+// The work item a CTA takes in its n-th round.  Items are numbered heaviest
+// first; the rounds alternate direction over the CTAs (snake order), so each
+// CTA gets a light item for every heavy one and all CTAs finish together.
+__device__ __forceinline__ int item_of_round(int n)
+{
+    const int g = (int)gridDim.x, b = (int)blockIdx.x;
+    return n * g + ((n & 1) ? g - 1 - b : b);
+}
+
+// Summary rows (section 2.2.1 and Figure 4c): s_j attends to the k text
+// tokens of its chunk and to itself, which are exactly the k+1 consecutive
+// augmented rows of chunk j.  One warp computes q heads h0 .. h0+ng-1 of kv
+// head hkv for global chunk gc, on the CUDA cores in fp32 with an online
+// softmax over the keys; lane l holds dims [l D/32, (l+1) D/32).  The
+// epilogue warps run it between items: the rows are independent of the
+// text rows' pipeline and take ~0.05 % of the FLOPs.
+template <int D>
+__device__ __forceinline__ void summary_rows_warp(const Params &P, int64_t gc, int hkv, int h0, int ng, int lane)
+{
+    constexpr int DL = D / 32;          // dims per lane: 4 (one 8-byte load) or 2 (one 4-byte load)
+    constexpr int KB = D == 128 ? 2 : 8;   // keys loaded together (their loads are in flight at once)
+    static_assert(DL == 2 || DL == 4, "head_dim 64 or 128");
+    using Vec = typename std::conditional<DL == 4, uint2, uint32_t>::type;
+    const int k = P.k;
+    const int64_t row0 = gc * (k + 1);
+    const int64_t srow = row0 + k;
+    const float sl2 = P.scale_log2;
+    auto unpack = [](const Vec &v, float *f) {
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(&v);
+#pragma unroll
+        for (int e = 0; e < DL / 2; ++e) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+            f[2 * e] = x.x;
+            f[2 * e + 1] = x.y;
+        }
+    };
+    const Vec *Kr = reinterpret_cast<const Vec *>(P.kk + (row0 * P.Hkv + hkv) * D) + lane;
+    const Vec *Vr = reinterpret_cast<const Vec *>(P.vv + (row0 * P.Hkv + hkv) * D) + lane;
+    const int64_t rstride = (int64_t)P.Hkv * (D / DL);   // Vec per augmented row
+    for (int g0 = 0; g0 < ng; g0 += 4) {
+        const int gn = min(4, ng - g0);
+        float q[4][DL], o[4][DL], m[4], l[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            m[g] = -INFINITY;
+            l[g] = 0.f;
+#pragma unroll
+            for (int e = 0; e < DL; ++e) o[g][e] = 0.f;
+            Vec qv;
+            if (g < gn)
+                qv = reinterpret_cast<const Vec *>(P.q + (srow * P.Hq + h0 + g0 + g) * D)[lane];
+            else
+                qv = Vec{};
+            unpack(qv, q[g]);
+        }
+        for (int r0 = 0; r0 <= k; r0 += KB) {
+            Vec kv[KB], vv[KB];
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                if (r0 + u <= k) {
+                    kv[u] = Kr[(r0 + u) * rstride];
+                    vv[u] = Vr[(r0 + u) * rstride];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                if (r0 + u > k) break;
+                float kf[DL], vf[DL];
+                unpack(kv[u], kf);
+                unpack(vv[u], vf);
+                float sc[4];
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    sc[g] = 0.f;
+#pragma unroll
+                    for (int e = 0; e < DL; ++e) sc[g] = fmaf(q[g][e], kf[e], sc[g]);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], off);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const float x = sc[g] * sl2;
+                    const float mn = fmaxf(m[g], x);
+                    const float corr = ex2(m[g] - mn);   // 0 on the first key
+                    const float pr = ex2(x - mn);
+                    l[g] = l[g] * corr + pr;
+#pragma unroll
+                    for (int e = 0; e < DL; ++e) o[g][e] = fmaf(pr, vf[e], o[g][e] * corr);
+                    m[g] = mn;
+                }
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            if (g >= gn) break;
+            const int head = h0 + g0 + g;
+            const float inv = 1.f / l[g];
+            Vec ov;
+            uint32_t *w = reinterpret_cast<uint32_t *>(&ov);
+#pragma unroll
+            for (int e = 0; e < DL / 2; ++e) w[e] = pack_bf16(o[g][2 * e] * inv, o[g][2 * e + 1] * inv);
+            reinterpret_cast<Vec *>(P.o + (srow * P.Hq + head) * D)[lane] = ov;
+            if (P.lse && lane == 0) P.lse[srow * P.Hq + head] = (m[g] + log2f(l[g])) * 0.69314718055994530942f;
+        }
+    }
+}
+
+// Persistent kernel: one CTA per SM walks one work item per round (heavy
+// first, in snake order over the CTAs), so the loads and
 // first MMAs of the next item overlap the last tiles and the epilogue of
 // the current one.  Every role walks the same item list; barrier phases
 // follow a tile counter that runs on across items.
@@ -287,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             int q_issued[QSTAGES] = {0};
             bool ok = true;
             int gt = 0;
-            for (int item = blockIdx.x, n = 0; item < W && ok; item += gridDim.x, ++n) {
+            for (int n = 0, item; (item = item_of_round(n)) < W && ok; ++n) {
                 const Unit U = unit_of(P, item, n_units);
                 if (isk) {
                     // query buffer n % 2 is free once the QKs of item n - 2 are done
@@ -347,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             const uint32_t id_qk = idesc_bf16(BN, false);
             bool ok = true;
             int gt = 0;
-            for (int item = blockIdx.x, n = 0; item < W && ok; item += gridDim.x, ++n) {
+            for (int n = 0, item; (item = item_of_round(n)) < W && ok; ++n) {
                 const Unit U = unit_of(P, item, n_units);
                 const int qb = n % QSTAGES;
                 const uint32_t qa = sbase + L::kQ + qb * L::kQTile;
@@ -380,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             const uint32_t id_pv = idesc_bf16(D, true);
             bool ok = true;
             int gt = 0;
-            for (int item = blockIdx.x, n = 0; item < W && ok; item += gridDim.x, ++n) {
+            for (int n = 0, item; (item = item_of_round(n)) < W && ok; ++n) {
                 const Unit U = unit_of(P, item, n_units);
                 for (int j = 0; j < U.T && ok; ++j, ++gt) {
                     const int s = gt % VSTAGES, bf = gt % NSBUF;
@@ -420,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         // An expired wait clears ok; every warp still walks all items.
         bool ok = true;
         int gt = 0;
-        for (int item = blockIdx.x, n = 0; item < W; item += gridDim.x, ++n) {
+        for (int n = 0, item; (item = item_of_round(n)) < W; ++n) {
             const Unit U = unit_of(P, item, n_units);
             const int c = U.c0 + cl;
             const int i = c * P.k + r_slot;            // local text index
@@ -563,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const bool leader = warp == kWarpEpi && lane == 0;
         bool ok = true;
         int gt = 0;   // tiles up to and including this item
-        for (int item = blockIdx.x, n = 0; item < W; item += gridDim.x, ++n) {
+        for (int n = 0, item; (item = item_of_round(n)) < W; ++n) {
             const Unit U = unit_of(P, item, n_units);
             gt += U.T;
             const int c = U.c0 + cl;
@@ -636,6 +750,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 }
             }
+            // the summary rows of this item's complete chunks, one warp per chunk
+            if (P.sum_rows && ok)
+                for (int c2 = U.c0 + (warp - kWarpEpi); c2 < min(U.cend, U.mb); c2 += 4)
+                    summary_rows_warp<D>(P, (int64_t)U.qbase + c2, U.hkv, U.h0, P.Gp, lane);
         }
         // every store has finished reading shared memory before the CTA exits
         if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -889,10 +1007,13 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
     P.scale_log2 = scale * 1.4426950408889634f;
     P.cu = cu; P.pl = pl; P.err = err;
     P.q = (const __nv_bfloat16 *)qa;
+    P.kk = (const __nv_bfloat16 *)ka;
+    P.vv = (const __nv_bfloat16 *)va;
     P.o = (__nv_bfloat16 *)oa;
     P.lse = lse;
     P.ck_tile_off = P.ck_cbeg = P.ck_ntot = P.ck_qbase = P.ck_kvbase = nullptr;
     P.sum_slot0 = 0;
+    P.sum_rows = 1;
     bool ok = make_map(&P.tm_q, qa, D, Hq, k, chunks, P.Gp, k, P.Tc) &&
               make_map(&P.tm_ksum, ka, D, Hkv, k, chunks, 1, 1, pf::BN) &&
               make_map(&P.tm_kwin, ka, D, Hkv, k, chunks, 1, k, P.Tk) &&
@@ -915,25 +1036,6 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
     pf::prefill_kernel<D><<<(unsigned)grid, pf::kThreads, L::kAlloc, st>>>(P);
     if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
 
-    pf::SumArgs s;
-    s.k = k; s.G = G; s.Hq = Hq; s.Hkv = Hkv; s.batch = batch; s.chunks = chunks;
-    s.scale = scale; s.scale_log2 = P.scale_log2;
-    s.cu = cu; s.pl = pl; s.err = err;
-    s.q = (const __nv_bfloat16 *)qa; s.kk = (const __nv_bfloat16 *)ka; s.v = (const __nv_bfloat16 *)va;
-    s.o = (__nv_bfloat16 *)oa; s.lse = lse;
-    int64_t tasks = chunks * Hkv;
-    if (tasks > 0) {
-        const unsigned blocks = (unsigned)((tasks + pf::kSumWarps - 1) / pf::kSumWarps);
-        const unsigned thr = pf::kSumWarps * 32;
-        switch (G) {
-        case 1: pf::summary_rows_kernel<D, 1><<<blocks, thr, 0, st>>>(s); break;
-        case 2: pf::summary_rows_kernel<D, 2><<<blocks, thr, 0, st>>>(s); break;
-        case 4: pf::summary_rows_kernel<D, 4><<<blocks, thr, 0, st>>>(s); break;
-        case 8: pf::summary_rows_kernel<D, 8><<<blocks, thr, 0, st>>>(s); break;
-        default: return KSA_ERR_UNSUPPORTED;
-        }
-        if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
-    }
     return KSA_OK;
 }
 
@@ -978,8 +1080,10 @@ static int launch_prefill_cache_t(const ksa_params *p, const ksa_cache *c, const
     P.pl = Plan{nullptr, nullptr, nullptr, nullptr};
     P.err = err;
     P.q = (const __nv_bfloat16 *)t.qa;
+    P.kk = P.vv = nullptr;
     P.o = (__nv_bfloat16 *)t.oa;
     P.lse = t.lse;
+    P.sum_rows = 0;
     P.ck_tile_off = t.tile_off; P.ck_cbeg = t.cbeg; P.ck_ntot = t.ntot;
     P.ck_qbase = t.qbase; P.ck_kvbase = t.kvbase;
     P.sum_slot0 = 1 + k + p->w * k;

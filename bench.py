@@ -31,20 +31,18 @@ sys.path.insert(0, ROOT)
 
 # workloads
 PF = dict(seqlens=[32768], k=8, w=8, Hq=32, Hkv=8, d=128, scale=0.5, seed=1, theta=1e6)
-# DRAM bytes (read + write) per launch of the dominant kernels, from the ncu
-# captures summarised under profiles/ for the kernels as they now stand (to be
-# set to None whenever one of those kernels changes, until it is captured again).
-# The decode capture ran at batch 16; its traffic grows in proportion to the batch.
+# DRAM bytes (read + write) per launch of the dominant kernels, from one ncu
+# --set full capture of each kernel as it now stands (set to None whenever
+# one of these kernels changes, until it is captured again).
 TRAFFIC = {
-    # the softmax changed (three-input max, packed fp32 pairs) after the last
-    # capture (661.2 MB of the previous build, profiles/prefill_kernel_qwen3_4b_32k.md)
-    "prefill": (None, "not captured for this build; 661.2 MB for the previous one in "
-                      "profiles/prefill_kernel_qwen3_4b_32k.md (prefill_kernel<128>)"),
-    # the decode kernel gained a state check (slice within the cache's slots,
-    # no negative counts) after its capture; the capture read 1.0851 GB per
-    # 16 sequences, 1.007x the algorithmic bytes
-    "decode_per_seq": (None, "not captured for this build; 1.0851e9 B per 16 sequences for the previous one in "
-                             "profiles/decode_split_kernel_b16_m16384.md (batch 16 capture)"),
+    # prefill_kernel<128> at this workload: 453.6 MB read (q_aug, k_aug, v_aug
+    # once) + 271.6 MB written (o_aug and the LSE, part still in L2 at exit)
+    "prefill": (725.2e6, "ncu capture of prefill_kernel<128>, 1 x 32768 text tokens (Qwen3-4B layer): "
+                         "dram read 453.6 MB + write 271.6 MB per launch"),
+    # decode_split_kernel<128,4> captured at batch 16 (1.0851 GB: 1.0778 GB
+    # read, 7.3 MB written); its traffic grows in proportion to the batch
+    "decode_per_seq": (1.0851e9 / 16, "ncu capture of decode_split_kernel<128,4> at batch 16 x 16384 summaries: "
+                                      "1.0851 GB per 16 sequences, scaled by the batch"),
 }
 DC = dict(B=64, m=16384, k=8, w=8, Hq=32, Hkv=8, d=128, seed=3, theta=1e6)
 
@@ -459,7 +457,8 @@ def run_ksa(args, rank, world, local):
             "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": tc_peak, "unit": "TFLOP/s",
                          "frac": kern_tflops / tc_peak,
                          "traffic": TRAFFIC["prefill"][0], "traffic_source": TRAFFIC["prefill"][1],
-                         "kernel": "prefill_kernel<128> (text rows; time of the ksa_prefill_fwd call)",
+                         "kernel": "prefill_kernel<128> (text rows, with the summary rows on its epilogue warps; "
+                                   "time of the ksa_prefill_fwd call)",
                          "peak_source": f"{peak_src} burst bf16", "peak_sustained": tc_sus},
             "roofline_decode": {"bound": "hbm", "achieved": dec_gbs / world, "peak": hbm_peak, "unit": "GB/s",
                                 "frac": (dec_gbs / world) / hbm_peak,

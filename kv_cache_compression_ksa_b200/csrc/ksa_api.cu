@@ -95,7 +95,7 @@ int64_t ksa_aug_rows(const ksa_params *p, int32_t batch, const int32_t *seqlens_
     int64_t chunks = 0;
     for (int b = 0; b < batch; ++b) {
         if (seqlens_host[b] < 0) return -1;
-        chunks += (seqlens_host[b] + p->k - 1) / p->k;
+        chunks += ((int64_t)seqlens_host[b] + p->k - 1) / p->k;
     }
     return chunks * (p->k + 1);
 }

@@ -204,4 +204,14 @@ __host__ __device__ __forceinline__ bool decode_slice(int kind, int64_t n, int64
     return true;
 }
 
+// (j + w + 1) k clamped to n: the first text position that sees summary j,
+// which is also one past the last text query that sees the text keys of
+// chunk j.  Taken in 64 bits: on a sequence of close to 2^31 tokens the
+// 32-bit product would pass INT32_MAX (w + 1) k alone may be 2^30.
+__host__ __device__ __forceinline__ int window_end(int64_t j, int w, int k, int n)
+{
+    const int64_t e = (j + w + 1) * (int64_t)k;
+    return e < n ? (int)e : n;
+}
+
 }  // namespace ksa

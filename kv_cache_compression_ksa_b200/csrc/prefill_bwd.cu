@@ -370,10 +370,10 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
             qt_lo[x] = 1; qt_hi[x] = 0; qs_lo[x] = qs_hi[x] = 0;
         } else if (K.kind == TEXT_ROWS) {
             const int cp = ki[x] / a.k;
-            qt_lo[x] = ki[x]; qt_hi[x] = (cp + a.w + 1) * a.k - 1;
+            qt_lo[x] = ki[x]; qt_hi[x] = window_end(cp, a.w, a.k, K.n) - 1;
             qs_lo[x] = cp; qs_hi[x] = cp < K.m ? cp + 1 : cp;
         } else {
-            qt_lo[x] = (ki[x] + a.w + 1) * a.k; qt_hi[x] = INT32_MAX;
+            qt_lo[x] = window_end(ki[x], a.w, a.k, K.n); qt_hi[x] = INT32_MAX;
             qs_lo[x] = ki[x]; qs_hi[x] = ki[x] + 1;
         }
     }
@@ -386,11 +386,11 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
     if (K.kind == TEXT_ROWS) {
         const int ca = K.idx0 / a.k, cb = (K.idx0 + K.cnt - 1) / a.k;
         t_lo = K.idx0;
-        t_hi = min(K.n, (cb + a.w + 1) * a.k);
+        t_hi = window_end(cb, a.w, a.k, K.n);
         s_lo = ca;
         s_hi = min(cb + 1, K.m);
     } else {
-        t_lo = min(K.n, (K.idx0 + a.w + 1) * a.k);
+        t_lo = window_end(K.idx0, a.w, a.k, K.n);
         t_hi = K.n;
         s_lo = K.idx0;
         s_hi = K.idx0 + K.cnt;
@@ -445,8 +445,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dkv_kernel(Args a)
             bool full = Q.cnt == RB && Q.kind == TEXT_ROWS;
             if (full) {
                 const int k_last = K.idx0 + K.cnt - 1;
-                full = K.kind == SUM_ROWS ? Q.idx0 >= (k_last + a.w + 1) * a.k
-                                          : (Q.idx0 >= k_last && Q.idx0 + RB - 1 <= (K.idx0 / a.k + a.w + 1) * a.k - 1);
+                full = K.kind == SUM_ROWS ? Q.idx0 >= window_end(k_last, a.w, a.k, K.n)
+                                          : (Q.idx0 >= k_last && Q.idx0 + RB - 1 <= window_end(K.idx0 / a.k, a.w, a.k, K.n) - 1);
             }
             // two halves of 32 queries: S^T = K Q^T, dP^T = V dO^T (16 keys x 32 queries)
 #pragma unroll 1

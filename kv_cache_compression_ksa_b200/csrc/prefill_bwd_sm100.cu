@@ -124,15 +124,29 @@ __host__ __device__ __forceinline__ void key_tile(const TArgs &a, int tile, KTil
     T.c0 = a.pl.chunk_off[T.b];
     if (T.sum) {
         T.kcnt = min(BK, T.m - T.j0);
-        T.qlo = min(T.n, (T.j0 + a.w + 1) * a.k);   // first text query of summary j0
+        T.qlo = window_end(T.j0, a.w, a.k, T.n);   // first text query of summary j0
         T.qhi = T.n;
     } else {
         T.kcnt = min(BK, T.n - T.j0);
         const int cb = (T.j0 + T.kcnt - 1) / a.k;
         T.qlo = T.j0;
-        T.qhi = min(T.n, (cb + a.w + 1) * a.k);     // past the last text query of chunk cb's keys
+        T.qhi = window_end(cb, a.w, a.k, T.n);     // past the last text query of chunk cb's keys
     }
-    T.nq = T.qhi > T.qlo ? (T.qhi - T.qlo + a.nqs - 1) / a.nqs : 0;   // dk/dv steps per q head
+    T.nq = T.qhi > T.qlo ? (int)(((int64_t)T.qhi - T.qlo + a.nqs - 1) / a.nqs) : 0;   // dk/dv steps per q head
+}
+
+// The text queries [lo, hi) that see key row r of tile T (text position or
+// summary index j0 + r).  Host-callable too, for the same CPU tests.
+__host__ __device__ __forceinline__ void key_queries(const TArgs &a, const KTile &T, int r, int &lo, int &hi)
+{
+    const int key = T.j0 + r;
+    if (T.sum) {
+        lo = window_end(key, a.w, a.k, T.n);
+        hi = T.n;
+    } else {
+        lo = key;
+        hi = window_end(key / a.k, a.w, a.k, T.n);
+    }
 }
 
 // Key tiles (summary tiles of all sequences, then text tiles) and the CTA
@@ -413,6 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const bool live = r < T.kcnt;
         const int key = T.j0 + r;            // text position or summary index
+        int klo, khi;                        // the text queries that see it
+        key_queries(a, T, r, klo, khi);
         const float sl2 = a.scale_log2;
         bool ok = true;
         for (int s = 0; s < n_steps; ++s) {
@@ -421,14 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
             const int q0 = step_q0(s);
             const int qn = min(NQ, T.n - q0);
             // this row's visible columns [lo, hi) of the step, inside this half
-            int lo, hi;
-            if (T.sum) {
-                lo = (key + a.w + 1) * a.k - q0;
-                hi = qn;
-            } else {
-                lo = key - q0;
-                hi = min(qn, (key / a.k + a.w + 1) * a.k - q0);
-            }
+            int lo = klo - q0, hi = min(qn, khi - q0);
             if (!live) lo = hi = 0;
             lo = max(lo - half * HQ2, 0);
             hi = min(hi - half * HQ2, HQ2);

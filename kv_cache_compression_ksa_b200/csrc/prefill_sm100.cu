@@ -173,7 +173,7 @@ __host__ __device__ __forceinline__ Unit unit_of(const Params &P, int item, int 
         U.c0 = (u - toff[b]) * P.unit_chunks;
     }
     U.mb = U.nb / P.k;
-    U.ncb = (U.nb + P.k - 1) / P.k;
+    U.ncb = (int)(((int64_t)U.nb + P.k - 1) / P.k);
     U.cend = min(U.ncb, U.c0 + P.unit_chunks);
     const int ns = max(min(U.mb, U.cend - 1 - P.w), 0);   // summaries any row may see
     U.cw_lo = max(0, U.c0 - P.w);

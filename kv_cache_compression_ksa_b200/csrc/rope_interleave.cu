@@ -40,7 +40,7 @@ plan_kernel(int batch, const int32_t *__restrict__ cu, int k, int unit_chunks,
         int n = cu[b + 1] - cu[b];
         if (n < 0) bad = 1;
         n = max(n, 0);
-        int c = (n + k - 1) / k;
+        int c = (int)(((int64_t)n + k - 1) / k);   // n may be INT32_MAX
         ch += c;
         su += n / k;
         if (unit_chunks > 0) ti += (c + unit_chunks - 1) / unit_chunks;
@@ -59,7 +59,7 @@ plan_kernel(int batch, const int32_t *__restrict__ cu, int k, int unit_chunks,
     int64_t ch0 = t ? s_chunks[t - 1] : 0, su0 = t ? s_sums[t - 1] : 0, ti0 = t ? s_tiles[t - 1] : 0;
     for (int b = b0; b < b1; ++b) {
         int n = max(cu[b + 1] - cu[b], 0);
-        int c = (n + k - 1) / k;
+        int c = (int)(((int64_t)n + k - 1) / k);   // n may be INT32_MAX
         pl.chunk_off[b] = (int32_t)ch0;
         pl.sum_off[b] = (int32_t)su0;
         pl.tile_off[b] = (int32_t)ti0;

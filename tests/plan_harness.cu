@@ -5,7 +5,7 @@
 // functions under test are the kernels' own, marked __host__ __device__:
 //   pf::unit_of           the forward's work items and their K/V tiles
 //                         (plain prefill and chunk mode),
-//   bt::key_tile, bt::q_tile
+//   bt::key_tile, bt::key_queries, bt::q_tile
 //                         the backward's key tiles with the text query range
 //                         that sees each (dk/dv), and its query tiles with
 //                         their key tiles (dq),
@@ -33,6 +33,10 @@
 //         "ns nt nqs split max_tiles dkv_grid dq_grid dkv_ctas", then per key
 //         tile "b sum j0 kcnt n m c0 qlo qhi nq", then "ntt" and per dq CTA
 //         "b n m c0 q0 qn c_first ns n_sum t_lo n_win"
+//   bwdt  k w n t_0 .. t_{j-1}
+//         one sequence of n tokens (n up to INT32_MAX: only the listed key
+//         tiles are built); per tile "b sum j0 kcnt n m c0 qlo qhi nq", then
+//         "lo hi" of key rows 0, 1 and kcnt - 1 (bt::key_queries)
 //   slice k w kind n m
 //         "ok lo hi"
 //   keys  k w n0 m0 T
@@ -207,6 +211,37 @@ static void run_bwd(int k, int w, int Hq, int Hkv, const std::vector<int> &n)
     }
 }
 
+static void run_bwd_tiles(int k, int w, int64_t n, const std::vector<int> &tiles)
+{
+    int nqs, split;
+    bt_step_shape(k, &nqs, &split);
+    const int32_t cu[2] = {0, (int32_t)n};
+    const int32_t chunk_off[2] = {0, (int32_t)((n + k - 1) / k)};
+    const int32_t ks_off[2] = {0, (int32_t)((n / k + bt::BK - 1) / bt::BK)};
+    const int32_t kt_off[2] = {0, (int32_t)((n + bt::BK - 1) / bt::BK)};
+    bt::TArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.k = k; a.w = w; a.G = 1; a.Hq = 1; a.Hkv = 1; a.batch = 1;
+    a.cu = cu;
+    a.pl.chunk_off = const_cast<int32_t *>(chunk_off);
+    a.ks_off = ks_off;
+    a.kt_off = kt_off;
+    a.nqs = nqs;
+    a.split = split;
+    for (int t : tiles) {
+        bt::KTile T;
+        bt::key_tile(a, t, T);
+        std::printf("%d %d %d %d %d %d %d %d %d %d\n", T.b, T.sum, T.j0, T.kcnt, T.n, T.m, T.c0, T.qlo, T.qhi, T.nq);
+        const int rows[3] = {0, 1, T.kcnt - 1};
+        for (int r : rows) {
+            int lo, hi;
+            bt::key_queries(a, T, r, lo, hi);
+            std::printf("%d %d ", lo, hi);
+        }
+        std::printf("\n");
+    }
+}
+
 static void run_keys(int k, int w, int n0, int m0, int T)
 {
     constexpr int D = 64;
@@ -267,6 +302,8 @@ int main()
             run_chunk((int)v[0], (int)v[1], (int)v[2], (int)v[3], ints(5));
         } else if (m == "bwd" && v.size() >= 5 && v.size() == 5 + (size_t)v[4]) {
             run_bwd((int)v[0], (int)v[1], (int)v[2], (int)v[3], ints(5));
+        } else if (m == "bwdt" && v.size() >= 3) {
+            run_bwd_tiles((int)v[0], (int)v[1], v[2], ints(3));
         } else if (m == "keys" && v.size() == 5) {
             run_keys((int)v[0], (int)v[1], (int)v[2], (int)v[3], (int)v[4]);
         } else if (m == "slice" && v.size() == 5) {

@@ -341,6 +341,57 @@ def test_backward_launch_bounds_at_their_edges(harness, k, w, G):
         bwd_case(harness, k, w, 8 * G, 8, lens)
 
 
+def _sees(n, k, w, q, kind, key):
+    """Text query q sees key (text position or summary index) by the
+    oracle's visibility rule; queries outside [0, n) see nothing."""
+    return 0 <= q < n and oracle.visible(n, k, w, TEXT, q, kind, key)
+
+
+def _check_span(n, k, w, kind, first, last, lo, hi):
+    """[lo, hi) is exactly the span of text queries that see some key of
+    first..last.  Each key's visible queries form one interval; the first
+    key's starts earliest.  A text key's interval ends at its chunk's window
+    end, latest for the last key; a summary's runs to the end of the
+    sequence when it is seen at all, and the first summary is seen if any."""
+    if hi <= lo:
+        assert not _sees(n, k, w, n - 1, kind, first), "a key seen by the last query got an empty range"
+        return
+    end_key = last if kind == TEXT else first
+    assert 0 <= lo < hi <= n
+    assert _sees(n, k, w, lo, kind, first) and not _sees(n, k, w, lo - 1, kind, first)
+    assert _sees(n, k, w, hi - 1, kind, end_key) and not _sees(n, k, w, hi, kind, end_key)
+
+
+@pytest.mark.parametrize("w", [0, 5, (1 << 27) - 1])
+def test_backward_ranges_on_a_sequence_of_2_31_tokens(harness, w):
+    """One sequence of INT32_MAX tokens (k = 8; w up to the largest accepted
+    window): the summary tiles from j0 = 2^27 on, and the text tiles past
+    position 2^30, have a window end (j + w + 1) k beyond INT32_MAX.  Each
+    tile's query range and the ranges of its key rows are checked against
+    the oracle's visibility rule at their ends."""
+    k, n = 8, (1 << 31) - 1
+    m = n // k
+    ns, nt = -(-m // BK), -(-n // BK)
+    pick_s = [0, 1, (1 << 27) // BK - 1, (1 << 27) // BK, (1 << 27) // BK + 1, ns - 2, ns - 1]
+    pick_t = [0, (1 << 30) // BK - 1, (1 << 30) // BK, nt // 2, nt - 2, nt - 1]
+    tiles = pick_s + [ns + t for t in pick_t]
+    rows = harness("bwdt", k, w, n, *tiles)
+    assert len(rows) == 2 * len(tiles)
+    nqs = 64   # k divides 64
+    for i, t in enumerate(tiles):
+        T = dict(zip(KT, rows[2 * i]))
+        kind = SUMMARY if t < ns else TEXT
+        j0 = (t if t < ns else t - ns) * BK
+        count = m if kind == SUMMARY else n
+        kc = min(BK, count - j0)
+        assert (T["b"], T["sum"], T["j0"], T["kcnt"], T["n"], T["m"], T["c0"]) == (0, int(kind == SUMMARY), j0, kc, n, m, 0)
+        _check_span(n, k, w, kind, j0, j0 + kc - 1, T["qlo"], T["qhi"])
+        assert T["nq"] == (-(-(T["qhi"] - T["qlo"]) // nqs) if T["qhi"] > T["qlo"] else 0)
+        lohi = rows[2 * i + 1]
+        for r, (lo, hi) in zip((0, 1, kc - 1), zip(lohi[0::2], lohi[1::2])):
+            _check_span(n, k, w, kind, j0 + r, j0 + r, lo, hi)
+
+
 # ---------------------------------------------------------------------------
 # Decode slice
 # ---------------------------------------------------------------------------

@@ -90,15 +90,28 @@ struct TArgs {
     const int32_t *item_off;          // [tiles+1] first CTA of each key tile (summary tiles first)
     int max_tiles;
     int nqs, split;                   // dk/dv: query positions per step, steps per CTA
+    int bpw;                          // dk/dv: query blocks of nqs per share window, max(1, split / G)
     int32_t *err;
     const float *lse, *dsum;
     float *dk32, *dv32;
 };
 
-// A key tile and the text query range that sees it.  key_tile is
-// host-callable too, for CPU tests of the ranges against the dense mask.
+// A key tile, the text query range that sees it, and its CTA shares.
+// key_tile is host-callable too, for CPU tests of the ranges against the
+// dense mask.
+//
+// The range [qlo, qhi) is cut into nq blocks of nqs query positions.  A
+// share (one CTA) takes the blocks of one window of bpw blocks, each block
+// for all G q heads of the kv head.  A summary tile's windows are aligned
+// to the sequence's block grid, common to all its summary tiles (their qlo
+// differ by multiples of 128 k, a multiple of nqs), so that the shares of
+// neighbouring summary tiles over one window read the same Q and dO blocks
+// and, walking the window from its last block down, read them at about the
+// same time: the data is fetched from DRAM once and reused from L2.  lead
+// is the tile's first block's place in its window (0 for text tiles, whose
+// shares start at qlo), nsh the number of shares.
 struct KTile {
-    int b, sum, j0, kcnt, n, m, c0, qlo, qhi, nq;   // nq: query tiles of 128 positions
+    int b, sum, j0, kcnt, n, m, c0, qlo, qhi, nq, lead, nsh;
 };
 
 __host__ __device__ __forceinline__ int find_off(const int32_t *off, int batch, int id)
@@ -133,6 +146,15 @@ __host__ __device__ __forceinline__ void key_tile(const TArgs &a, int tile, KTil
         T.qhi = window_end(cb, a.w, a.k, T.n);     // past the last text query of chunk cb's keys
     }
     T.nq = T.qhi > T.qlo ? (int)(((int64_t)T.qhi - T.qlo + a.nqs - 1) / a.nqs) : 0;   // dk/dv steps per q head
+    T.lead = T.sum ? (T.qlo / a.nqs) % a.bpw : 0;
+    T.nsh = T.nq > 0 ? (T.nq + T.lead + a.bpw - 1) / a.bpw : 0;
+}
+
+// Blocks [r_lo, r_hi) of share sh of tile T (relative to T.qlo).
+__host__ __device__ __forceinline__ void share_blocks(const TArgs &a, const KTile &T, int sh, int &r_lo, int &r_hi)
+{
+    r_lo = max(0, sh * a.bpw - T.lead);
+    r_hi = min(T.nq, (sh + 1) * a.bpw - T.lead);
 }
 
 // The text queries [lo, hi) that see key row r of tile T (text position or
@@ -150,7 +172,7 @@ __host__ __device__ __forceinline__ void key_queries(const TArgs &a, const KTile
 }
 
 // Key tiles (summary tiles of all sequences, then text tiles) and the CTA
-// offsets of their shares of ceil(G nq / split) CTAs each.
+// offsets of their nsh shares each.
 __global__ void __launch_bounds__(1024) bt_plan_kernel(TArgs a, int32_t *ks_off, int32_t *kt_off, int32_t *item_off)
 {
     __shared__ int part[1024];
@@ -180,7 +202,7 @@ __global__ void __launch_bounds__(1024) bt_plan_kernel(TArgs a, int32_t *ks_off,
     for (int t = lo; t < hi; ++t) {
         KTile T;
         key_tile(a, t, T);
-        sum += (a.G * T.nq + a.split - 1) / a.split;
+        sum += T.nsh;
     }
     part[threadIdx.x] = sum;
     __syncthreads();
@@ -199,7 +221,7 @@ __global__ void __launch_bounds__(1024) bt_plan_kernel(TArgs a, int32_t *ks_off,
         item_off[t] = run;
         KTile T;
         key_tile(a, t, T);
-        run += (a.G * T.nq + a.split - 1) / a.split;
+        run += T.nsh;
     }
 }
 
@@ -229,8 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
     KTile T;
     key_tile(a, tile, T);
     const int g = blockIdx.y;
-    const int s_lo = (item - a.item_off[tile]) * L::kSplit;
-    const int n_steps = min(a.G * T.nq, s_lo + L::kSplit) - s_lo;
+    int r_lo, r_hi;
+    share_blocks(a, T, item - a.item_off[tile], r_lo, r_hi);
+    const int n_steps = (r_hi - r_lo) * a.G;
     if (n_steps <= 0) return;
 
     auto bar = [&](int i) { return sbase + L::kBar + 8u * (uint32_t)i; };
@@ -281,9 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1) bt_dkv_kernel(const __grid_consta
     constexpr uint32_t kTileBytes = (uint32_t)L::kTile, kQBytes = (uint32_t)L::kQTile;
     constexpr uint32_t kQHalf = (uint32_t)L::kQHalf;
 
-    // step s of the share -> (query tile, q head)
-    auto step_q0 = [&](int s) { return T.qlo + ((s_lo + s) / a.G) * NQ; };
-    auto step_h = [&](int s) { return g * a.G + (s_lo + s) % a.G; };
+    // step s of the share -> (query block, q head): the share's last block
+    // first, each block for the G q heads in turn
+    auto step_q0 = [&](int s) { return T.qlo + (r_hi - 1 - s / a.G) * NQ; };
+    auto step_h = [&](int s) { return g * a.G + s % a.G; };
 
     if (warp == kWarpTMA) {
         if (lane == 0) {
@@ -928,16 +952,21 @@ static void bt_step_shape(int k, int *nqs, int *split)
     *split = *nqs == 64 ? bt::DkvCfg<128, 64>::kSplit : bt::DkvCfg<128, 128>::kSplit;
 }
 
+// Query blocks per dk/dv share window: as many as fit split steps of G heads.
+static int bt_bpw(int G, int split) { return split / G > 1 ? split / G : 1; }
+
 // CTAs of the dk/dv launch: an upper bound on the plan's share count (CTAs
-// past it exit).  At most one CTA per key tile plus G nq / split per tile; a
-// summary tile's queries number at most total_text, a text tile's
-// 128 + (w+1) k.
+// past it exit).  A tile of nq blocks has at most nq / bpw + 2 shares (a
+// summary tile's first window may be partial), a text tile at most
+// nq / bpw + 1; a summary tile's queries number at most total_text, a text
+// tile's 128 + (w+1) k.
 static int64_t bt_dkv_grid(int64_t total_text, int batch, int k, int w, int G, int nqs, int split)
 {
+    const int64_t bpw = bt_bpw(G, split);
     const int64_t ns_tiles = (total_text / k) / bt::BK + batch, nt_tiles = total_text / bt::BK + batch;
     const int64_t q_sum = (total_text + nqs - 1) / nqs + 1;
     const int64_t q_txt = (bt::BK + (int64_t)(w + 1) * k + nqs - 1) / nqs + 1;
-    return ns_tiles * (1 + ((int64_t)G * q_sum) / split) + nt_tiles * (1 + ((int64_t)G * q_txt) / split);
+    return ns_tiles * (2 + q_sum / bpw) + nt_tiles * (1 + q_txt / bpw);
 }
 
 // CTAs of the dq launch: an upper bound on the query tiles of 128 text
@@ -993,7 +1022,7 @@ int launch_prefill_bwd_tc(const ksa_params *p, int batch, const int32_t *cu, int
     a.scale_log2 = a.scale * 1.4426950408889634f;
     a.cu = cu; a.pl = pl; a.err = err;
     a.lse = lse; a.dsum = dsum; a.dk32 = dk32; a.dv32 = dv32;
-    a.nqs = nqs; a.split = split;
+    a.nqs = nqs; a.split = split; a.bpw = bt_bpw(a.G, split);
     char *w = static_cast<char *>(ws);
     const size_t ab = align_up(sizeof(int32_t) * (size_t)(batch + 1));
     int32_t *ks_off = reinterpret_cast<int32_t *>(w), *kt_off = reinterpret_cast<int32_t *>(w + ab);

@@ -411,6 +411,66 @@ def ksa_attention_bwd_dq_rows(n, k, C, q, kk, v, do, rows, scale=None):
     return out
 
 
+def seeing_queries(n: int, k: int, C: int, a: int) -> np.ndarray:
+    """Eq. (1) indices of the queries that see the key at Eq. (1) index a:
+    the visibility rules read from the key's side.  Summary s_j is seen by
+    itself (section 2.2.1) and by every text t_i with j < c_i - C, that is
+    i >= (j + C + 1) k (Eq. (3)).  Text t_p of chunk c_p is seen by the text
+    t_i with p <= i and c_i - C <= c_p, that is p <= i < (c_p + C + 1) k
+    (Eqs. (2)-(3)), and by its chunk's summary s_{c_p} when that chunk is
+    complete (section 2.2.1)."""
+    m = n // k
+    txt = lambda i: i + i // k                       # Eq. (1) index of text i
+    if a < m * (k + 1) and a % (k + 1) == k:         # summary j
+        j = a // (k + 1)
+        return np.concatenate([[a], txt(np.arange((j + C + 1) * k, n))]).astype(np.int64)
+    p = a - min(a // (k + 1), m)                      # text token index
+    c = p // k
+    out = txt(np.arange(p, min(n, (c + C + 1) * k)))
+    if c < m:
+        out = np.concatenate([out, [c * (k + 1) + k]])
+    return out.astype(np.int64)
+
+
+def ksa_attention_bwd_dkv_keys(n, k, C, q, kk, v, do, keys, scale=None):
+    """dk and dv of the given Eq. (1) key rows only: the same formulas as
+    ksa_attention_bwd, summed over the query rows that see those keys.  Each
+    such row needs its whole softmax row (its own visible keys) for P and
+    D = rowsum(do * o); dk_a = scale sum_b dS_ba q_b and dv_a = sum_b P_ba
+    do_b, over those rows b and the q heads of a's kv head.  Returns
+    ([len(keys), Hkv, d], [len(keys), Hkv, d])."""
+    q, kk, v, do = (_f64(a) for a in (q, kk, v, do))
+    Hq, d = q.shape[1], q.shape[2]
+    Hkv = kk.shape[1]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    keys = np.asarray(keys, dtype=np.int64)
+    out_of = np.full(q.shape[0], -1, dtype=np.int64)    # Eq. (1) index -> output row, -1 if not requested
+    out_of[keys] = np.arange(len(keys))
+    assert len(np.unique(keys)) == len(keys), "keys must be distinct"
+    dk = np.zeros((len(keys), Hkv, d))
+    dv = np.zeros((len(keys), Hkv, d))
+    rows = np.unique(np.concatenate([seeing_queries(n, k, C, int(a)) for a in keys]))
+    for b in rows:
+        vis = visible_keys(n, k, C, int(b))
+        at = np.flatnonzero(out_of[vis] >= 0)         # positions in vis of requested keys
+        to = out_of[vis[at]]
+        for g in range(Hkv):
+            hs = slice(g * G, (g + 1) * G)
+            Kb, Vb = kk[vis, g], v[vis, g]            # [nvis, d]
+            S = scale * (Kb @ q[b, hs].T)             # [nvis, G]
+            P = np.exp(S - S.max(axis=0))
+            P /= P.sum(axis=0)
+            O = P.T @ Vb                              # [G, d]
+            dP = Vb @ do[b, hs].T                     # [nvis, G]
+            D = (do[b, hs] * O).sum(axis=1)           # [G]
+            dS = P * (dP - D)
+            dk[to, g] += scale * (dS[at] @ q[b, hs])
+            dv[to, g] += P[at] @ do[b, hs]
+    return dk, dv
+
+
 def interleave_rope_bwd(seqlens, k, theta, dq_aug, dk_aug, dv_aug):
     """Gradients of the text and summary projections from those of the
     augmented rows: the transpose of Eq. (1)'s interleave and of RoPE (an

@@ -5,7 +5,7 @@
 // functions under test are the kernels' own, marked __host__ __device__:
 //   pf::unit_of           the forward's work items and their K/V tiles
 //                         (plain prefill and chunk mode),
-//   bt::key_tile, bt::key_queries, bt::q_tile
+//   bt::key_tile, bt::key_queries, bt::share_blocks, bt::q_tile
 //                         the backward's key tiles with the text query range
 //                         that sees each (dk/dv), and its query tiles with
 //                         their key tiles (dq),
@@ -31,11 +31,13 @@
 //         then the work items as for fwd
 //   bwd   k w Hq Hkv B n_0 .. n_{B-1}
 //         "ns nt nqs split max_tiles dkv_grid dq_grid dkv_ctas", then per key
-//         tile "b sum j0 kcnt n m c0 qlo qhi nq", then "ntt" and per dq CTA
+//         tile "b sum j0 kcnt n m c0 qlo qhi nq lead nsh" followed by each
+//         share's query blocks "r_lo r_hi", then "ntt" and per dq CTA
 //         "b n m c0 q0 qn c_first ns n_sum t_lo n_win"
 //   bwdt  k w n t_0 .. t_{j-1}
 //         one sequence of n tokens (n up to INT32_MAX: only the listed key
-//         tiles are built); per tile "b sum j0 kcnt n m c0 qlo qhi nq", then
+//         tiles are built); per tile "b sum j0 kcnt n m c0 qlo qhi nq lead
+//         nsh", then
 //         "lo hi" of key rows 0, 1 and kcnt - 1 (bt::key_queries)
 //   slice k w kind n m
 //         "ok lo hi"
@@ -188,20 +190,29 @@ static void run_bwd(int k, int w, int Hq, int Hkv, const std::vector<int> &n)
     a.kt_off = kt_off.data();
     a.nqs = nqs;
     a.split = split;
+    a.bpw = bt_bpw(a.G, split);
     const int ns = ks_off[B], nt = kt_off[B];
     const int64_t total_text = cu[B], aug_rows = (int64_t)chunk_off[B] * (k + 1);
-    // the plan's CTA shares: ceil(G nq / split) per key tile
+    // the plan's CTA shares: nsh per key tile
     int64_t ctas = 0;
     std::vector<bt::KTile> tiles(ns + nt);
     for (int t = 0; t < ns + nt; ++t) {
         bt::key_tile(a, t, tiles[t]);
-        ctas += (a.G * tiles[t].nq + split - 1) / split;
+        ctas += tiles[t].nsh;
     }
     std::printf("%d %d %d %d %lld %lld %lld %lld\n", ns, nt, nqs, split, (long long)bt_max_tiles(B, aug_rows),
                 (long long)bt_dkv_grid(total_text, B, k, w, a.G, nqs, split), (long long)bt_dq_grid(total_text, B),
                 (long long)ctas);
-    for (const bt::KTile &T : tiles)
-        std::printf("%d %d %d %d %d %d %d %d %d %d\n", T.b, T.sum, T.j0, T.kcnt, T.n, T.m, T.c0, T.qlo, T.qhi, T.nq);
+    for (const bt::KTile &T : tiles) {
+        std::printf("%d %d %d %d %d %d %d %d %d %d %d %d", T.b, T.sum, T.j0, T.kcnt, T.n, T.m, T.c0, T.qlo, T.qhi,
+                    T.nq, T.lead, T.nsh);
+        for (int sh = 0; sh < T.nsh; ++sh) {
+            int r_lo, r_hi;
+            bt::share_blocks(a, T, sh, r_lo, r_hi);
+            std::printf(" %d %d", r_lo, r_hi);
+        }
+        std::printf("\n");
+    }
     std::printf("%d\n", nt);
     for (int cta = 0;; ++cta) {
         bt::QTile Q;
@@ -228,10 +239,12 @@ static void run_bwd_tiles(int k, int w, int64_t n, const std::vector<int> &tiles
     a.kt_off = kt_off;
     a.nqs = nqs;
     a.split = split;
+    a.bpw = bt_bpw(a.G, split);
     for (int t : tiles) {
         bt::KTile T;
         bt::key_tile(a, t, T);
-        std::printf("%d %d %d %d %d %d %d %d %d %d\n", T.b, T.sum, T.j0, T.kcnt, T.n, T.m, T.c0, T.qlo, T.qhi, T.nq);
+        std::printf("%d %d %d %d %d %d %d %d %d %d %d %d\n", T.b, T.sum, T.j0, T.kcnt, T.n, T.m, T.c0, T.qlo, T.qhi,
+                    T.nq, T.lead, T.nsh);
         const int rows[3] = {0, 1, T.kcnt - 1};
         for (int r : rows) {
             int lo, hi;

@@ -32,7 +32,7 @@ CASES = [
     ("long_summaries", [1500], 8, 4, 8, 2, 128, 15),
     ("k16_d64", [700, 333], 16, 2, 8, 4, 64, 17),
     ("k6_warp_path", [200, 50], 6, 2, 8, 2, 128, 19),          # k does not divide 128: warp-level dk/dv
-    ("summary_shares", [2600, 300], 8, 1, 8, 2, 128, 23),      # summary key tiles split over several CTAs
+    ("summary_shares", [2600, 300], 8, 1, 16, 2, 128, 23),     # 8 heads x 41 steps: summary tile 0 over two CTAs
     ("k128_steps_of_128", [700, 300], 128, 1, 4, 2, 128, 29),  # k does not divide 64: 128-query dk/dv steps
     ("k64_one_chunk_steps", [1300, 260], 64, 2, 8, 2, 128, 31),  # a dk/dv step is one chunk of 64 slots
 ]
@@ -81,12 +81,12 @@ def test_prefill_bwd_matches_oracle(name, seqlens, k, w, Hq, Hkv, d, seed):
     _check(name + " dv", to_f64(dv), want[2], live)
 
 
-def test_prefill_bwd_full_size_identities_and_sampled_rows():
+@pytest.fixture(scope="module")
+def full_size():
     """The 32768-token Qwen3-4B-layer prefill (32 q / 8 kv heads, d 128, k 8,
-    w 8): per kv head the key gradients sum to zero and the value gradients
-    sum to the output gradients of its q heads (exact for softmax attention;
-    checked to 1e-2 of the summed magnitudes); sampled dq rows against the
-    oracle's per-row backward."""
+    w 8) and its backward through the library, with fp64 host copies of the
+    tensors the oracle needs (n % k == 0: the padded layout has no padding
+    rows and equals Eq. (1) order)."""
     dev = torch.device("cuda")
     seqlens, k, w, Hq, Hkv, d = [32768], 8, 8, 32, 8, 128
     x = prefill_inputs(seqlens, k, Hq, Hkv, d, seed=1, scale=0.5, device=dev)
@@ -109,8 +109,19 @@ def test_prefill_bwd_full_size_identities_and_sampled_rows():
     L.ksa_prefill_bwd(p, x.cu_seqlens, nt, rows, qa, ka, va, oa, lse, do, dq, dk, dv, wsb)
     torch.cuda.synchronize()
     assert L.ksa_get_device_error(wsb) == 0
-    # n % k == 0: no padding rows
-    dkf, dvf, dof = dk.double(), dv.double(), do.double()
+    return dict(n=seqlens[0], k=k, w=w, Hq=Hq, Hkv=Hkv, d=d, rows=rows, do_dev=do, dk_dev=dk, dv_dev=dv,
+                q=to_f64(qa), kk=to_f64(ka), v=to_f64(va), do=to_f64(do), dq=to_f64(dq), dk=to_f64(dk),
+                dv=to_f64(dv))
+
+
+def test_prefill_bwd_full_size_identities_and_sampled_rows(full_size):
+    """Per kv head the key gradients sum to zero and the value gradients sum
+    to the output gradients of its q heads (exact for softmax attention;
+    checked to 1e-2 of the summed magnitudes); sampled dq rows against the
+    oracle's per-row backward."""
+    F = full_size
+    rows, Hq, Hkv, d = F["rows"], F["Hq"], F["Hkv"], F["d"]
+    dkf, dvf, dof = F["dk_dev"].double(), F["dv_dev"].double(), F["do_dev"].double()
     sk = dkf.sum(0)
     assert (sk.abs().sum(-1) <= 1e-2 * dkf.abs().sum(0).sum(-1)).all()
     want_v = dof.view(rows, Hkv, Hq // Hkv, d).sum((0, 2))
@@ -118,11 +129,38 @@ def test_prefill_bwd_full_size_identities_and_sampled_rows():
     # sampled dq rows (Eq. (1) order = the layout here): text rows early, mid
     # and late, and summary rows
     sample = np.array([0, 5, 80, 9 * 1000 + 3, 9 * 2047 + 8, 9 * 3000 + 4, rows - 2, rows - 1])
-    n = seqlens[0]
-    want = oracle.ksa_attention_bwd_dq_rows(n, k, w, to_f64(qa), to_f64(ka), to_f64(va), to_f64(do), sample)
-    got = to_f64(dq)[sample]
+    want = oracle.ksa_attention_bwd_dq_rows(F["n"], F["k"], F["w"], F["q"], F["kk"], F["v"], F["do"], sample)
+    got = F["dq"][sample]
     err = np.linalg.norm(got - want) / np.linalg.norm(want)
     assert err <= REL_FROB, f"sampled dq rel-Frob {err:.3e}"
+
+
+# Per kv head, the first key of one summary tile (128 summaries s_j0 ..) and
+# one text tile (128 text positions p0 ..) of the dk/dv kernel.  The summary
+# tile j0 = 3456 is seen by 5048 text queries x 4 q heads, more than one CTA
+# share of 256 steps of 64 queries, so its dk/dv is summed over two CTAs;
+# the others fit one share.  Text tiles: the sequence start (window clipped),
+# middle ones, and the end.
+KEY_TILES = [(3968, 0), (3456, 128), (3968, 12800), (3840, 20480), (3968, 8192), (3968, 24576), (3840, 29952),
+             (3968, 32640)]
+
+
+def test_prefill_bwd_full_size_sampled_key_tiles(full_size):
+    """dk and dv element by element on whole key tiles of the full-size
+    backward, one summary tile and one text tile per kv head, against the
+    oracle's per-key backward of the same kv head."""
+    F = full_size
+    k, G = F["k"], F["Hq"] // F["Hkv"]
+    for g, (j0, p0) in enumerate(KEY_TILES):
+        hs = slice(g * G, (g + 1) * G)
+        kv = slice(g, g + 1)
+        for name, keys in (("summary", np.arange(j0, j0 + 128) * (k + 1) + k),
+                           ("text", np.arange(p0, p0 + 128) + np.arange(p0, p0 + 128) // k)):
+            wk, wv = oracle.ksa_attention_bwd_dkv_keys(F["n"], k, F["w"], F["q"][:, hs], F["kk"][:, kv],
+                                                       F["v"][:, kv], F["do"][:, hs], keys)
+            live = np.ones(len(keys), bool)
+            _check(f"kv head {g} {name} tile {keys[0]} dk", F["dk"][keys, g], wk[:, 0], live)
+            _check(f"kv head {g} {name} tile {keys[0]} dv", F["dv"][keys, g], wv[:, 0], live)
 
 
 @pytest.mark.parametrize("seqlens,k,w,Hq,Hkv,d", [([100, 37, 8, 3], 8, 2, 8, 2, 128), ([150, 41], 4, 1, 4, 4, 64)])

@@ -118,6 +118,27 @@ def test_bwd_dq_rows_match_dense(n, k, C):
                                atol=1e-12)
 
 
+@pytest.mark.parametrize("n,k,C", [(40, 4, 2), (35, 8, 1), (13, 1, 0), (30, 3, 0)])
+def test_bwd_dkv_keys_match_dense(n, k, C):
+    """The per-key form (queries from the key's side of the rules) equals the
+    dense backward's dk and dv, and each key's seeing queries equal the
+    column of the dense mask."""
+    Hq, Hkv, d = 4, 2, 8
+    q, kk, v, do = _inputs(n, k, Hq, Hkv, d, seed=19)
+    _, dk, dv, _, _ = oracle.ksa_attention_bwd(n, k, C, q, kk, v, do)
+    M = oracle.dense_mask(n, k, C)
+    for a in range(q.shape[0]):
+        np.testing.assert_array_equal(np.sort(oracle.seeing_queries(n, k, C, a)), np.nonzero(M[:, a])[0])
+    keys = np.arange(q.shape[0])[::-1]   # any order
+    gk, gv = oracle.ksa_attention_bwd_dkv_keys(n, k, C, q, kk, v, do, keys)
+    np.testing.assert_allclose(gk, dk[keys], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gv, dv[keys], rtol=1e-12, atol=1e-12)
+    sub = keys[::5]   # a subset: rows that see no requested key add nothing
+    gk, gv = oracle.ksa_attention_bwd_dkv_keys(n, k, C, q, kk, v, do, sub)
+    np.testing.assert_allclose(gk, dk[sub], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gv, dv[sub], rtol=1e-12, atol=1e-12)
+
+
 def test_rope_transpose_and_inverse():
     """RoPE is a rotation: rotating by -pos undoes it, and it is its own
     transpose's inverse (<R x, g> = <x, R^T g>)."""

@@ -248,7 +248,7 @@ def test_chunk_invalid_states_get_no_work(harness):
 # ---------------------------------------------------------------------------
 # Backward key tiles
 # ---------------------------------------------------------------------------
-KT = ("b", "sum", "j0", "kcnt", "n", "m", "c0", "qlo", "qhi", "nq")
+KT = ("b", "sum", "j0", "kcnt", "n", "m", "c0", "qlo", "qhi", "nq", "lead", "nsh")
 QT = ("b", "n", "m", "c0", "q0", "qn", "c_first", "ns", "n_sum", "t_lo", "n_win")
 
 
@@ -261,7 +261,9 @@ def bwd_case(harness, k, w, Hq, Hkv, seqlens):
     # launch bounds: the plan never needs more tiles, or CTAs, than reserved
     assert ns + nt <= max_tiles and dkv_ctas <= dkv_grid and nt <= dq_grid
     tiles = [dict(zip(KT, r)) for r in rows[1:1 + ns + nt]]
+    shares = [list(zip(r[len(KT)::2], r[len(KT) + 1::2])) for r in rows[1:1 + ns + nt]]
     check_dq_tiles(rows[1 + ns + nt:], k, w, seqlens, nt)
+    check_shares(tiles, shares, G, nqs, split)
     coff = offsets([-(-n // k) for n in seqlens])
     got_s = {b: [] for b in range(len(seqlens))}
     got_t = {b: [] for b in range(len(seqlens))}
@@ -291,7 +293,38 @@ def bwd_case(harness, k, w, Hq, Hkv, seqlens):
     for b, n in enumerate(seqlens):
         assert got_s[b] == list(range(0, n // k, BK))
         assert got_t[b] == list(range(0, n, BK))
-    assert dkv_ctas == sum(-(-(G * T["nq"]) // split) for T in tiles)
+    assert dkv_ctas == sum(T["nsh"] for T in tiles)
+
+
+def check_shares(tiles, shares, G, nqs, split):
+    """dk/dv shares: each tile's shares cut its nq query blocks into
+    consecutive non-empty runs of at most split // G blocks (a CTA's steps
+    are blocks x G heads, at most split); text tiles' shares start at the
+    tile's first block; the summary tiles of one sequence cut the queries
+    at common positions (a window grid of split // G blocks), so that the
+    shares of different tiles over one window read the same Q and dO."""
+    bpw = max(1, split // G)
+    grid = {}
+    for T, sh in zip(tiles, shares):
+        assert len(sh) == T["nsh"]
+        if T["nq"] == 0:
+            assert sh == []
+            continue
+        assert sh[0][0] == 0 and sh[-1][1] == T["nq"]
+        for (a0, a1), (b0, _) in zip(sh, sh[1:]):
+            assert a1 == b0
+        assert all(1 <= r1 - r0 <= bpw for r0, r1 in sh)
+        if not T["sum"]:
+            assert T["lead"] == 0 and len(sh) == -(-T["nq"] // bpw)
+            continue
+        assert 0 <= T["lead"] < bpw
+        # the share starts after the first, and the start of the first
+        # share's window (lead blocks before qlo), all on one grid
+        cuts = {(T["qlo"] + r0 * nqs) % (bpw * nqs) for r0, _ in sh[1:]}
+        cuts.add((T["qlo"] - T["lead"] * nqs) % (bpw * nqs))
+        grid.setdefault(T["b"], set()).update(cuts)
+    for b, cuts in grid.items():
+        assert len(cuts) == 1, ("summary tiles of a sequence cut their queries on different grids", b, cuts)
 
 
 def check_dq_tiles(rows, k, w, seqlens, nt):

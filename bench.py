@@ -643,7 +643,10 @@ def run_sweep(args):
                                   "ms": ms, "slice_gb": rows * 576 * 2 / 1e9, "gbs": gbs,
                                   "frac_of_hbm_peak": gbs / hbm_peak, "tflops": tf,
                                   "frac_of_bf16_peak": tf / tc_peak,
-                                  "note": "one TEXT step over latent rows of d_c 512 + d_r 64; warp-level mma.sync"}),
+                                  "note": "one TEXT step over latent rows of d_c 512 + d_r 64; " +
+                                          ("tcgen05 on CTA pairs (latent dims split, partial scores exchanged "
+                                           "through distributed shared memory)" if H % 128 == 0
+                                           else "warp-level mma.sync")}),
                       flush=True)
                 del cache, q, o, lse_m, mws
                 torch.cuda.empty_cache()

@@ -22,31 +22,15 @@
 #include <math.h>
 
 #include "ksa_internal.cuh"
+#include "mla_common.cuh"
 #include "warp_mma.cuh"
 
 namespace ksa {
 namespace mla {
 
-constexpr int DC = 512, DR = 64, DL = DC + DR;   // latent, RoPE key, row
 constexpr int KB = 32;                           // slots per block
 constexpr int PITCH = DL + 8;                    // smem row pitch (elements)
 constexpr int PPITCH = KB + 8;                   // P tile row pitch
-
-struct Args {
-    int k, w, H, batch, splits;
-    int64_t S, per;                  // slots per sequence; slots per share (multiple of KB)
-    float scale_log2;
-    double log2_theta;
-    int rotate;
-    const int8_t *kind;
-    int32_t *state;
-    const __nv_bfloat16 *lat;        // [B, S, DL]
-    const __nv_bfloat16 *q;          // [B, H, DL], d_r part not rotated
-    float *part_o;                   // [splits, B, H, DC]
-    float *part_ml;                  // [splits, B, H, 2] (max in log2 units, sum)
-    __nv_bfloat16 *o;                // [B, H, DC]
-    float *lse;                      // [B, H] or null
-};
 
 // ---------------------------------------------------------------------------
 struct AppendArgs {
@@ -637,11 +621,51 @@ static_assert(DC == 4 * kCombineThreads, "combine: four latent dims per thread")
 struct Plan {
     int mt, groups, splits;
     int64_t per;
+    bool tc;   // the tensor-core kernel (head groups of 128)
 };
+
+// Shares for the tensor-core kernel: each share (one CTA pair) reads its
+// rows once and writes 2 x 128 x 512 fp32 partials per 128 heads that the
+// combine reads back.  Taken: the share count (at least 4 blocks a share)
+// that minimises waves x (share bytes + partial bytes), pairs per wave =
+// SMs / 2; ties to the fewer shares.
+static Plan plan_tc(const ksa_mla_params *p, int batch, int64_t lmax)
+{
+    Plan P;
+    P.mt = 0;
+    P.tc = true;
+    P.groups = p->num_heads / 128;
+    const int64_t ctas = (int64_t)batch * P.groups, pairs = sm_count() / 2 > 0 ? sm_count() / 2 : 1;
+    const int64_t most = lmax / (4 * kTcBlock) > 1 ? lmax / (4 * kTcBlock) : 1;
+    const double part = 2.0 * 128 * DC * 4;
+    int64_t best_sp = 1;
+    double best = -1.0;
+    for (int64_t sp = 1; sp <= most && sp <= 1024 && ctas > 0; ++sp) {
+        int64_t per = (lmax + sp - 1) / sp;
+        per = (per + kTcBlock - 1) / kTcBlock * kTcBlock;
+        const int64_t real = (lmax + per - 1) / per;
+        const int64_t waves = (ctas * real + pairs - 1) / pairs;
+        const double cost = (double)waves * ((double)per * DL * 2 + part);
+        if (best < 0 || cost < best * (1 - 1e-9)) { best = cost; best_sp = real; }
+    }
+    int64_t per = (lmax + best_sp - 1) / best_sp;
+    per = (per + kTcBlock - 1) / kTcBlock * kTcBlock;
+    if (per < kTcBlock) per = kTcBlock;
+    P.per = per;
+    P.splits = (int)((lmax + per - 1) / per);
+    if (P.splits < 1) P.splits = 1;
+    return P;
+}
 
 static Plan plan(const ksa_mla_params *p, int batch, int64_t max_text)
 {
     Plan P;
+    {
+        const int64_t mmax = max_text / p->k;
+        const int64_t lmax = (int64_t)p->k + 1 + (int64_t)p->w * p->k + (mmax > p->w ? mmax - p->w : 0);
+        if (p->num_heads % 128 == 0) return plan_tc(p, batch, lmax);
+    }
+    P.tc = false;
     P.mt = p->num_heads >= 64 ? 4 : p->num_heads >= 32 ? 2 : 1;
     P.groups = (p->num_heads + 16 * P.mt - 1) / (16 * P.mt);
     const int64_t mmax = max_text / p->k;
@@ -743,8 +767,10 @@ int launch_mla_decode(const ksa_mla_params *p, const ksa_mla_cache *c, const int
     a.part_ml = reinterpret_cast<float *>(static_cast<char *>(ws) + align_up(rows * mla::DC * 4));
     a.o = (__nv_bfloat16 *)o;
     a.lse = lse;
-    int rc = P.mt == 4 ? launch_mla_ws(a, P.groups, st) : P.mt == 2 ? launch_mla_t<2>(a, P.groups, st)
-                                                                     : launch_mla_t<1>(a, P.groups, st);
+    int rc = P.tc        ? mla::launch_mla_tc(a, st)
+             : P.mt == 4 ? launch_mla_ws(a, P.groups, st)
+             : P.mt == 2 ? launch_mla_t<2>(a, P.groups, st)
+                         : launch_mla_t<1>(a, P.groups, st);
     if (rc != KSA_OK) return rc;
     dim3 grid((unsigned)p->num_heads, (unsigned)c->batch);
     mla::mla_combine_kernel<<<grid, mla::kCombineThreads, 0, st>>>(a);

@@ -13,15 +13,17 @@
 // share of a sequence's slice runs on a cluster of two CTAs that split each
 // row's dims: rank 0 takes latent dims 0..255 and the RoPE dims, rank 1
 // latent dims 256..511.  TMEM per CTA: its half of O (256 columns), two S
-// buffers (64 each) and its latent half of Q (bf16, 128 columns), so that
-// shared memory holds four K/V stages.  Per block, each CTA computes its
-// partial scores S_r = Q_r K_r^T of all 128 heads.  The softmax of heads
-// 0..63 belongs to rank 0 and of heads 64..127 to rank 1 (the owner):
-//   * each CTA sends its partial scores of the other's heads (64 x 64 fp32)
+// buffers (64 each) and its latent half of Q (bf16, 128 columns), which
+// leaves shared memory room for three K/V stages.  Per block, each CTA
+// computes its partial scores S_r = Q_r K_r^T of all 128 heads.  The
+// softmax of half the heads belongs to each CTA (the owner: rank 0 owns TMEM
+// lanes 32 q + 0..15 of every lane quarter q, rank 1 lanes 32 q + 16..31):
+//   * each CTA sends its partial scores of the other's rows (64 x 64 fp32)
 //     to the owner through distributed shared memory;
-//   * the owner adds them to its own, runs the online softmax of its heads
-//     (two threads per head, 32 slots each), writes P (bf16) into its TMEM
-//     and sends P and the rows' rescale factors back;
+//   * the owner adds them to its own, runs the online softmax of its rows
+//     (16-lane TMEM accesses: a thread holds two rows of 16 slots, a row's
+//     four threads reduce by shuffles), writes P (bf16) over S in its TMEM
+//     and sends P and the rows' rescale factors back by bulk copy;
 //   * each CTA writes the received P into its TMEM, rescales its O rows of
 //     the other's heads when asked, and accumulates its half of O = P V, a
 //     128 x 256 x 64 product with P read from TMEM.
@@ -29,17 +31,16 @@
 // the 32 KB of a full exchange; distributed shared memory moves about 20
 // bytes per clock per direction on this part.
 //
-// Roles (384 threads): for the lane quarters q of the owned heads, warps
-// 4 + q and 8 + q are the softmax's two column halves; for the other
-// quarters, warp 4 + q sends the partial scores and warp 8 + q stores the
-// returned P, and two warps of those quarters issue the TMA loads and the
-// MMAs.  The online softmax works in
-// log2 units with a lazy rescale: O rows and row sums are rescaled only when
-// a block's maximum passes the one in use by more than 8 (so p <= 2^8), once
-// the previous PV product has completed.  The owner's exchanges need no
-// acknowledgement: the K/V and S buffers a block reuses are released only
-// after the product that follows the other CTA's reads (see the receive
-// buffers below).
+// Roles (512 threads): warp 0 issues the TMA loads, warp 1 the MMAs; warps
+// 4..7 own (lane quarter w % 4), 8..11 send the other rows' partial scores,
+// 12..15 store the other rows' P.  Owned rows in every quarter spread the
+// softmax over the four SM sub-partitions.  The online softmax works in log2
+// units with a lazy rescale: O rows and row sums are rescaled only when a
+// block's maximum passes the one in use by more than 8 (so p <= 2^8), once
+// the previous PV product has completed.  The exchanges need no
+// acknowledgement: an exchange buffer is refilled two blocks later, and the
+// sender's next use of it depends, through the S buffer's reuse, on the PV
+// product that follows the receiver's read.
 //
 // Every wait is bounded; a timeout records KSA_ERR_TIMEOUT in the sequence's
 // state word.  Both CTAs always meet at a final cluster barrier: a CTA must

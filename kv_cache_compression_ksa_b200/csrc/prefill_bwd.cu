@@ -149,16 +149,18 @@ using wm::frag_b_kn;
 using wm::frag_b_nk;
 
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) bwd_dot_kernel(Args a, int64_t rows, int D)
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dot_kernel(Args a, int64_t cells)
 {
-    // one thread per (row, head): D = dO . O over d
+    // D = dO . O over d for each (row, head) cell: D / 8 consecutive lanes
+    // take one cell, 16 bytes each, so that a warp's loads are contiguous
+    constexpr int L = D / 8;
     const int64_t t = (int64_t)blockIdx.x * 256 + threadIdx.x;
-    if (t >= rows * a.Hq) return;
-    const uint4 *x = reinterpret_cast<const uint4 *>(a.dout + t * D);
-    const uint4 *y = reinterpret_cast<const uint4 *>(a.o + t * D);
+    const int64_t cell = t / L;
+    const bool live = cell < cells;
     float s = 0.f;
-    for (int c = 0; c < D / 8; ++c) {
-        const uint4 u = x[c], w = y[c];
+    if (live) {
+        const uint4 u = reinterpret_cast<const uint4 *>(a.dout)[t], w = reinterpret_cast<const uint4 *>(a.o)[t];
         const uint32_t uu[4] = {u.x, u.y, u.z, u.w}, ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -166,7 +168,9 @@ __global__ void __launch_bounds__(256) bwd_dot_kernel(Args a, int64_t rows, int 
             s = fmaf(__uint_as_float(uu[i] & 0xffff0000u), __uint_as_float(ww[i] & 0xffff0000u), s);
         }
     }
-    a.dsum[t] = s;
+#pragma unroll
+    for (int off = L / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (live && (t % L) == 0) a.dsum[cell] = s;
 }
 
 // ---------------------------------------------------------------------------
@@ -659,6 +663,136 @@ __global__ void __launch_bounds__(128) bwd_sum_rows_kernel(Args a, int64_t chunk
     }
 }
 
+// The same for a compile-time G, in one pass over the chunk's rows: the
+// summary row's q and dO of the G heads stay in registers, and each row r
+// (loaded once, with its fp32 dk, dv accumulators) gives the G heads' P and
+// dS, adds their dk, dv terms and its dS K term to the summary row's dq, and
+// is written out.  The G heads' dot products reduce together (independent
+// shuffle chains), and the next row's loads are issued before this row's
+// arithmetic.
+template <int D, int G>
+__global__ void __launch_bounds__(128) bwd_sum_rows_g_kernel(Args a, int64_t chunks)
+{
+    constexpr int CPL = D / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t gc = (int64_t)blockIdx.x * 4 + warp;
+    if (*a.err != 0 || gc >= chunks) return;   // warp-uniform; only warp-level syncs below
+    const int g = blockIdx.y, K1 = a.k + 1;
+    const int b = find_seq(a.pl.chunk_off, a.batch, (int)gc);
+    const int j = (int)(gc - a.pl.chunk_off[b]);
+    const int n = a.cu[b + 1] - a.cu[b], m = n / a.k;
+    if (j * a.k >= n) return;                  // past the sequence (a padding chunk cannot occur)
+    const bool has_sum = j < m;
+    const int ntext = min(a.k, n - j * a.k);
+    const int64_t row0 = gc * K1, srow = row0 + a.k;
+    const int col0 = lane * CPL;
+    auto ld = [&](const __nv_bfloat16 *p, float *f) {
+        if constexpr (CPL == 4) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(p);
+            f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
+            f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
+        } else {
+            const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
+            f[0] = __uint_as_float(u << 16); f[1] = __uint_as_float(u & 0xffff0000u);
+        }
+    };
+    auto ld32 = [&](const float *p, float *f) {
+        if constexpr (CPL == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(p);
+            f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+        } else {
+            const float2 v = *reinterpret_cast<const float2 *>(p);
+            f[0] = v.x; f[1] = v.y;
+        }
+    };
+    auto st = [&](__nv_bfloat16 *p, const float *f) {
+        if constexpr (CPL == 4)
+            *reinterpret_cast<uint2 *>(p) = make_uint2(wm::pack2(f[0], f[1]), wm::pack2(f[2], f[3]));
+        else
+            *reinterpret_cast<uint32_t *>(p) = wm::pack2(f[0], f[1]);
+    };
+    // the summary row's q, dO, LSE (log2 units) and D of the G heads
+    float qs[G][CPL], os[G][CPL], l2[G], dd[G], dq[G][CPL];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+        const int h = g * G + hh;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) qs[hh][c] = os[hh][c] = dq[hh][c] = 0.f;
+        l2[hh] = dd[hh] = 0.f;
+        if (has_sum) {
+            ld(a.q + (srow * a.Hq + h) * D + col0, qs[hh]);
+            ld(a.dout + (srow * a.Hq + h) * D + col0, os[hh]);
+            l2[hh] = a.lse[srow * a.Hq + h] * 1.4426950408889634f;
+            dd[hh] = a.dsum[srow * a.Hq + h];
+        }
+    }
+    // rows of the chunk that exist: its text rows, then s_j
+    auto real = [&](int r) { return r < a.k ? r < ntext : has_sum; };
+    float kr[CPL], vr[CPL], dkr[CPL], dvr[CPL];
+    auto load_row = [&](int r) {
+        const int64_t off = ((row0 + r) * a.Hkv + g) * D + col0;
+        ld32(a.dk32 + off, dkr);
+        ld32(a.dv32 + off, dvr);
+        if (has_sum) {
+            ld(a.kk + off, kr);
+            ld(a.v + off, vr);
+        }
+    };
+    int r = 0;
+    while (r < K1 && !real(r)) ++r;
+    if (r < K1) load_row(r);
+    while (r < K1) {
+        float k0[CPL], v0[CPL], dk0[CPL], dv0[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) { k0[c] = kr[c]; v0[c] = vr[c]; dk0[c] = dkr[c]; dv0[c] = dvr[c]; }
+        int rn = r + 1;
+        while (rn < K1 && !real(rn)) ++rn;
+        if (rn < K1) load_row(rn);   // the next row's loads ahead of this row's arithmetic
+        if (has_sum) {
+            float sc[G], dp[G];
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) {
+                sc[hh] = dp[hh] = 0.f;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    sc[hh] = fmaf(qs[hh][c], k0[c], sc[hh]);
+                    dp[hh] = fmaf(os[hh][c], v0[c], dp[hh]);
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                for (int hh = 0; hh < G; ++hh) {
+                    sc[hh] += __shfl_xor_sync(0xffffffffu, sc[hh], off);
+                    dp[hh] += __shfl_xor_sync(0xffffffffu, dp[hh], off);
+                }
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) {
+                const float pr = wm::ex2(sc[hh] * a.scale_log2 - l2[hh]);
+                const float ds = pr * (dp[hh] - dd[hh]);
+                const float ws = ds * a.scale;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    dq[hh][c] = fmaf(ds, k0[c], dq[hh][c]);
+                    dk0[c] = fmaf(ws, qs[hh][c], dk0[c]);
+                    dv0[c] = fmaf(pr, os[hh][c], dv0[c]);
+                }
+            }
+        }
+        const int64_t off = ((row0 + r) * a.Hkv + g) * D + col0;
+        st(a.dk + off, dk0);
+        st(a.dv + off, dv0);
+        r = rn;
+    }
+    if (has_sum)
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) dq[hh][c] *= a.scale;
+            st(a.dq + (srow * a.Hq + g * G + hh) * D + col0, dq[hh]);
+        }
+}
+
 // per-sequence block counts: text blocks ceil(n/64), summary blocks ceil(m/64)
 __global__ void bwd_blocks_kernel(int batch, const int32_t *cu, int k, int32_t *tb_off, int32_t *sb_off)
 {
@@ -692,7 +826,14 @@ static int bw_sum_launch(const bw::Args &a, int64_t chunks, cudaStream_t st)
             attr = smem;
         }
     }
-    bw::bwd_sum_rows_kernel<D><<<dim3((unsigned)((chunks + 3) / 4), a.Hkv), 128, smem, st>>>(a, chunks);
+    const dim3 grid((unsigned)((chunks + 3) / 4), a.Hkv);
+    switch (a.G) {
+    case 1: bw::bwd_sum_rows_g_kernel<D, 1><<<grid, 128, 0, st>>>(a, chunks); break;
+    case 2: bw::bwd_sum_rows_g_kernel<D, 2><<<grid, 128, 0, st>>>(a, chunks); break;
+    case 4: bw::bwd_sum_rows_g_kernel<D, 4><<<grid, 128, 0, st>>>(a, chunks); break;
+    case 8: bw::bwd_sum_rows_g_kernel<D, 8><<<grid, 128, 0, st>>>(a, chunks); break;
+    default: bw::bwd_sum_rows_kernel<D><<<grid, 128, smem, st>>>(a, chunks); break;
+    }
     return KSA_OK;
 }
 
@@ -749,7 +890,10 @@ int launch_prefill_bwd(const ksa_params *p, int batch, const int32_t *cu, int64_
     bw::bwd_blocks_kernel<<<1, 32, 0, st>>>(batch, cu, p->k, const_cast<int32_t *>(a.tb_off),
                                             const_cast<int32_t *>(a.sb_off));
     const int64_t cells = aug_rows * a.Hq;
-    bw::bwd_dot_kernel<<<(unsigned)((cells + 255) / 256), 256, 0, st>>>(a, aug_rows, p->head_dim);
+    if (p->head_dim == 128)
+        bw::bwd_dot_kernel<128><<<(unsigned)((cells * 16 + 255) / 256), 256, 0, st>>>(a, cells);
+    else
+        bw::bwd_dot_kernel<64><<<(unsigned)((cells * 8 + 255) / 256), 256, 0, st>>>(a, cells);
     // upper bound of the block count; CTAs past the real count exit
     const int64_t nblk = total_text / bw::RB + (total_text / p->k) / bw::RB + 2LL * batch;
     if (nblk > 0x7fffffffLL) return KSA_ERR_UNSUPPORTED;

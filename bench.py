@@ -617,8 +617,10 @@ def run_sweep(args):
         M = SWEEP_MLA
         k, w, H = M["k"], M["w"], M["H"]
         pm = L.make_mla_params(k, w, H, 512, 64, 0.0, 1e6)
-        for B in M["batches"]:
-            for n in M["contexts"]:
+        batches = [int(x) for x in args.mla_batches.split(",")] if args.mla_batches else M["batches"]
+        contexts = [int(x) for x in args.mla_contexts.split(",")] if args.mla_contexts else M["contexts"]
+        for B in batches:
+            for n in contexts:
                 m = n // k
                 cache = api.MlaCache(pm, B, cap=m + 1, device=dev)
                 fill_normal_(cache.latent, M["seed"] + B)
@@ -767,6 +769,8 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=DC["B"])
     ap.add_argument("--sweep-parts", default="prefill,chunk,mla,bwd,decode",
                     help="comma list of the sweep's parts: prefill, chunk, mla, bwd, decode")
+    ap.add_argument("--mla-batches", default=None, help="comma list: the MLA sweep's batches (default all)")
+    ap.add_argument("--mla-contexts", default=None, help="comma list: the MLA sweep's contexts (default all)")
     ap.add_argument("--sweep", action="store_true",
                     help="time the long varlen prefill batch and the decode batch x context grid (one JSON line per point)")
     args = ap.parse_args()

@@ -1,8 +1,10 @@
 """Discrete-event models of the barrier protocols of the warp-specialised
 kernels (csrc/prefill_sm100.cu prefill_kernel, csrc/prefill_bwd_sm100.cu
-bt_dkv_kernel and bq_dq_kernel on mbarriers; csrc/mla_decode.cu
+bt_dkv_kernel and bq_dq_kernel, and the CTA pair of
+csrc/mla_decode_tc.cu mla_decode_tc_kernel, on mbarriers; csrc/mla_decode.cu
 mla_decode_ws_kernel on named barriers), checked for deadlock, parity
-aliasing and mismatched named-barrier use under many random interleavings.
+aliasing, buffers refilled before they were read, and mismatched
+named-barrier use under many random interleavings.
 
 Each role of a kernel (TMA producers, MMA issuers, elementwise and epilogue
 warps) is restated as the sequence of its waits, arrivals and MMA commits, in
@@ -34,11 +36,14 @@ class _Bar:
 
 def _simulate(bars, roles, seed, max_rounds=400000):
     """roles: name -> generator yielding ("wait", bar, phase), ("arrive", bar),
-    ("load", bar) (a TMA load completing later on bar) or ("mma", issuer) /
-    ("commit", issuer, bar).  Returns (status, stuck waits, aliasing events)."""
+    ("load", bar) (a TMA load or bulk copy completing later on bar),
+    ("mma", issuer) / ("commit", issuer, bar), or ("mark", key) / ("expect",
+    key, n) (a buffer read finished / a write that needs n reads done before
+    it: a shortfall is reported with the aliasing events).  Returns (status,
+    stuck waits, aliasing events)."""
     rng = random.Random(seed)
     B = {name: _Bar(count) for name, count in bars.items()}
-    aliasing, loads, mma = [], [], {}
+    aliasing, loads, mma, marks = [], [], {}, {}
     cur = {k: None for k in roles}
     done = set()
 
@@ -87,6 +92,11 @@ def _simulate(bars, roles, seed, max_rounds=400000):
                         mma.setdefault(a[1], []).append(None)
                     elif a[0] == "commit":
                         mma.setdefault(a[1], []).append(a[2])
+                    elif a[0] == "mark":          # a read of a buffer finished
+                        marks[a[1]] = marks.get(a[1], 0) + 1
+                    elif a[0] == "expect":        # a write needs that many reads done first
+                        if marks.get(a[1], 0) < a[2]:
+                            aliasing.append(("overwrite", a[1], a[2], marks.get(a[1], 0)))
                     cur[c] = None
                     progressed = True
         if not progressed and not loads and not any(mma.values()):
@@ -367,6 +377,142 @@ def test_engine_catches_a_parity_aliasing_bug():
             status, _, aliasing = _simulate(bars, roles, seed)
             failures += status != "ok" or bool(aliasing)
     assert failures > 0
+
+
+# ---------------------------------------------------------------- mla_decode_tc_kernel
+def _mla_tc_roles(nblk, rescale_rng, qk_runs_ahead=False):
+    """Both CTAs of a pair (ranks 0, 1), warps as roles; barrier names carry
+    the rank.  Per CTA: TMA (three K/V stages), the MMA issuer (QK(j) into S
+    buffer j % 2 once PV(j - 2) has completed, then PV(j - 1) once P(j - 1)
+    is in), four owner warps (S, then the other CTA's partial scores, the
+    softmax, a bulk copy of P to the other CTA, P in), four sender warps
+    (S, then a push of the other CTA's rows to it) and four receiver warps
+    (the other CTA's P, P in).  The receive buffers have no acknowledgement;
+    "expect" checks that each is refilled only after its previous contents
+    were read, and that P is written over S only after S was read."""
+    ST = 3
+    bars = {}
+    for r in range(2):
+        for i in range(ST):
+            bars.update({f"{r}KF{i}": 1, f"{r}KE{i}": 1})
+        for i in range(2):
+            bars.update({f"{r}S{i}": 1, f"{r}PF{i}": 8, f"{r}O{i}": 1, f"{r}RS{i}": 4, f"{r}RP{i}": 1 + 4})
+
+    def init(r):
+        for i in range(2):
+            yield ("arrive", f"{r}RP{i}")            # the receive buffers' first phases armed
+
+    def tma(r):
+        for j in range(nblk):
+            if j >= ST:
+                yield ("wait", f"{r}KE{j % ST}", j // ST - 1)
+            yield ("load", f"{r}KF{j % ST}")
+
+    def mma(r):
+        for j in range(nblk + 1):
+            if j < nblk:
+                sb = j & 1
+                yield ("wait", f"{r}KF{j % ST}", j // ST)
+                if j >= 2:
+                    yield ("wait", f"{r}O{sb}", (j - 2) >> 1)
+                yield ("expect", f"{r}Sread{sb}", 8 * (j >> 1))   # S(j - 2) read by owners and senders
+                yield ("mma", f"{r}")
+                yield ("commit", f"{r}", f"{r}S{sb}")
+            if j >= 1:
+                i = j - 1
+                yield ("wait", f"{r}PF{i & 1}", i >> 1)
+                yield ("mma", f"{r}")
+                yield ("commit", f"{r}", f"{r}O{i & 1}")
+                yield ("commit", f"{r}", f"{r}KE{i % ST}")
+
+    def owner(r, q):
+        o = 1 - r
+        for j in range(nblk):
+            sb = j & 1
+            yield ("wait", f"{r}S{sb}", j >> 1)
+            yield ("mark", f"{r}Sread{sb}")
+            yield ("wait", f"{r}RS{sb}", j >> 1)
+            yield ("mark", f"{r}RSread{sb}")
+            if j > 0 and rescale_rng.random() < 0.3:
+                yield ("wait", f"{r}O{sb ^ 1}", (j - 1) >> 1)
+            yield ("expect", f"{o}RPread{sb}", 4 * (j >> 1))   # the other CTA read P(j - 2) from buffer sb
+            yield ("load", f"{o}RP{sb}")                         # bulk copy of P and the factors
+            yield ("arrive", f"{r}PF{sb}")
+        if nblk > 0:
+            yield ("wait", f"{r}O{(nblk - 1) & 1}", (nblk - 1) >> 1)
+
+    def sender(r, q):
+        o = 1 - r
+        for j in range(nblk):
+            sb = j & 1
+            yield ("wait", f"{r}S{sb}", j >> 1)
+            yield ("mark", f"{r}Sread{sb}")
+            yield ("mark", f"{r}Ssent{q}")
+            yield ("expect", f"{o}RSread{sb}", 4 * (j >> 1))   # the other CTA read S(j - 2) from buffer sb
+            yield ("arrive", f"{o}RS{sb}")
+
+    def receiver(r, q):
+        for j in range(nblk):
+            sb = j & 1
+            yield ("wait", f"{r}RP{sb}", j >> 1)
+            if q == 0 and j + 2 < nblk:
+                yield ("arrive", f"{r}RP{sb}")                 # one thread arms buffer sb's next phase
+            yield ("mark", f"{r}RPread{sb}")
+            if j > 0 and rescale_rng.random() < 0.3:
+                yield ("wait", f"{r}O{sb ^ 1}", (j - 1) >> 1)
+            yield ("expect", f"{r}Ssent{q}", j + 1)            # P over S(j) only after the sender read it
+            yield ("arrive", f"{r}PF{sb}")
+        if nblk > 0:
+            yield ("wait", f"{r}O{(nblk - 1) & 1}", (nblk - 1) >> 1)
+
+    def qk_only(r):   # the mutation: QK issued as soon as its rows land
+        for j in range(nblk):
+            yield ("wait", f"{r}KF{j % ST}", j // ST)
+            yield ("expect", f"{r}Sread{j & 1}", 8 * (j >> 1))
+            yield ("mma", f"{r}q")
+            yield ("commit", f"{r}q", f"{r}S{j & 1}")
+
+    def pv_only(r):
+        for i in range(nblk):
+            yield ("wait", f"{r}PF{i & 1}", i >> 1)
+            yield ("mma", f"{r}p")
+            yield ("commit", f"{r}p", f"{r}O{i & 1}")
+            yield ("commit", f"{r}p", f"{r}KE{i % ST}")
+
+    roles = {}
+    for r in range(2):
+        roles[f"init{r}"] = init(r)
+        roles[f"tma{r}"] = tma(r)
+        if qk_runs_ahead:
+            roles[f"qk{r}"] = qk_only(r)
+            roles[f"pv{r}"] = pv_only(r)
+        else:
+            roles[f"mma{r}"] = mma(r)
+        for q in range(4):
+            roles[f"own{r}{q}"] = owner(r, q)
+            roles[f"snd{r}{q}"] = sender(r, q)
+            roles[f"rcv{r}{q}"] = receiver(r, q)
+    return bars, roles
+
+
+def test_mla_tc_kernel_pair_protocol():
+    for nblk in list(range(0, 9)) + [13, 20]:
+        for seed in range(30):
+            bars, roles = _mla_tc_roles(nblk, random.Random(seed + 77))
+            status, stuck, aliasing = _simulate(bars, roles, seed)
+            assert status == "ok" and not aliasing, (nblk, seed, status, stuck, aliasing)
+
+
+def test_mla_tc_model_catches_a_missing_buffer_wait():
+    """If QK ran ahead of the PV products (issued as soon as its rows land,
+    without the wait for PV(j - 2)), S(j - 2) could be overwritten before it
+    is read and the phases of its barrier alias."""
+    flagged = 0
+    for seed in range(30):
+        bars, roles = _mla_tc_roles(8, random.Random(seed), qk_runs_ahead=True)
+        status, _, aliasing = _simulate(bars, roles, seed)
+        flagged += status != "ok" or bool(aliasing)
+    assert flagged > 0
 
 
 # ---------------------------------------------------------------- mla_decode_ws_kernel

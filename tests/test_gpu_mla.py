@@ -43,6 +43,7 @@ CASES = [
     (2, 48, 16, 3, [70, 2], [16, 9], [0, 2]),                       # 48 heads (padded group), SKIP
     (2, 256, 8, 8, [300, 1200], [3, 8], [0, 0]),                    # two groups of 128 heads
     (4, 128, 4, 1, [5000, 1, 0, 700], [2, 4, 1, 0], [2, 0, 0, 1]),  # SKIP first, m < w, m = 0, SUMMARY
+    (2, 128, 4, 2, [1, 0], [4, 2], [0, 0]),                         # a 16-slot cache: one partial block
 ]
 
 

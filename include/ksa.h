@@ -376,8 +376,12 @@ KSA_API size_t ksa_mla_decode_workspace_size(const ksa_mla_params *p, int32_t ba
  * q_r NOT rotated; rotated here at position n_text - 1).  Slices and kinds
  * as for ksa_decode.  o: [batch, num_heads, d_c] bf16, the latent output;
  * lse: [batch, num_heads] fp32 (natural log) or NULL.  max_text bounds
- * n_text over the batch and must match the workspace query.  Runs on the
- * warp-level tensor-core MMA. */
+ * n_text over the batch and must match the workspace query.  When
+ * num_heads is a multiple of 128 each group of 128 heads runs on tcgen05 in
+ * clusters of two CTAs (split-K over the slice, the latent dims split
+ * between the pair); other head counts run on the warp-level MMA.  A
+ * pipeline wait that times out on the tcgen05 path records KSA_ERR_TIMEOUT
+ * in the sequence's state[3], like the other per-sequence errors. */
 KSA_API int ksa_mla_decode(const ksa_mla_params *p, const ksa_mla_cache *cache, const int8_t *kind, const void *q,
                            void *o, float *lse, int64_t max_text, void *workspace, size_t workspace_bytes,
                            void *stream);
@@ -387,7 +391,7 @@ KSA_API int ksa_mla_decode(const ksa_mla_params *p, const ksa_mla_cache *cache, 
 KSA_API int ksa_get_device_error(int32_t *dev_err, void *stream);
 
 /* Self-check of the bounded-wait error path of the tensor-core pipelines
- * (the prefill, its backward and the chunked prefill): every mbarrier wait
+ * (the prefill, its backward, the chunked prefill and the MLA decode): every mbarrier wait
  * there gives up after a bounded number of polls or sleeps, records
  * KSA_ERR_TIMEOUT in the caller's error word, makes the CTA's other roles
  * stop waiting, and the CTA frees its tensor memory and exits, so the

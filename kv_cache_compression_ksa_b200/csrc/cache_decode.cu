@@ -475,7 +475,8 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_split_kernel(DecodeArgs
     }
 }
 
-// Merge the nsplit partial states of each (sequence, kv head) and write o, lse.
+// Merge the nsplit partial states of each (sequence, kv head) and write o, lse,
+// for few splits: one thread per output element walks the splits.
 template <int D, int G>
 __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeArgs a, __nv_bfloat16 *o, float *lse)
 {
@@ -505,6 +506,87 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeArgs a, __nv_
     }
 }
 
+// The same merge for many splits (kDecWideCombine or more; a batch of one
+// long sequence takes hundreds), where a thread per element walking every
+// split in turn waits on one load at a time.  One CTA per (kv head,
+// sequence): the G heads' maxima over the splits first
+// (threads strided over the splits, then a block reduction), then warp w sums
+// splits w, w + 8, ... (each lane 32-strided over the G x D outputs, so a
+// split's row of partials is one coalesced read and every lane has
+// independent loads in flight), and the eight warps' sums are added at the end.
+template <int D, int G>
+__global__ void __launch_bounds__(256) decode_combine_wide_kernel(DecodeArgs a, __nv_bfloat16 *o, float *lse)
+{
+    constexpr int W = 8, E = G * D, EPL = E / 32;
+    __shared__ float s_red[W][E + G];   // per warp: the G x D sums, then the G row sums
+    __shared__ float s_mx[W][G];
+    const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int kind = a.kind[b];
+    if (kind == KSA_SKIP) return;
+    int64_t lo, hi;
+    if (!decode_slice(kind, a.state[4 * (int64_t)b], a.state[4 * (int64_t)b + 1], a.k, a.w, &lo, &hi) ||
+        hi > a.S)
+        return;
+    const float *part = a.part + (((int64_t)b * a.Hkv + h) * a.nsplit) * (G * (2 + D));
+    const int stride = G * (2 + D);
+    float mm[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) mm[g] = -INFINITY;
+    for (int s = t; s < a.nsplit; s += blockDim.x)
+#pragma unroll
+        for (int g = 0; g < G; ++g) mm[g] = fmaxf(mm[g], part[(int64_t)s * stride + g]);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mm[g] = fmaxf(mm[g], __shfl_xor_sync(0xffffffffu, mm[g], off));
+        if (lane == 0) s_mx[warp][g] = mm[g];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        mm[g] = s_mx[0][g];
+#pragma unroll
+        for (int w2 = 1; w2 < W; ++w2) mm[g] = fmaxf(mm[g], s_mx[w2][g]);
+    }
+    float acc[EPL], ll[G];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int g = 0; g < G; ++g) ll[g] = 0.f;
+    for (int s = warp; s < a.nsplit; s += W) {
+        const float *ps = part + (int64_t)s * stride;
+        float cf[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float ms = ps[g];
+            cf[g] = (ms == -INFINITY) ? 0.f : ex2f_approx(ms - mm[g]);
+            ll[g] += ps[G + g] * cf[g];
+        }
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) acc[i] += ps[2 * G + lane + 32 * i] * cf[(32 * i) / D];
+    }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) s_red[warp][lane + 32 * i] = acc[i];
+    if (lane == 0)
+#pragma unroll
+        for (int g = 0; g < G; ++g) s_red[warp][E + g] = ll[g];
+    __syncthreads();
+    for (int e = t; e < E; e += blockDim.x) {
+        const int g = e / D, dd = e % D;
+        float aa = 0.f, lt = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < W; ++w2) {
+            aa += s_red[w2][e];
+            lt += s_red[w2][E + g];
+        }
+        const int64_t oi = ((int64_t)b * a.Hq + (int64_t)h * G + g) * D + dd;
+        o[oi] = __float2bfloat16_rn(aa / lt);
+        if (lse && dd == 0) lse[(int64_t)b * a.Hq + (int64_t)h * G + g] = (mm[g] + log2f(lt)) * 0.69314718055994530942f;
+    }
+}
+
+constexpr int kDecWideCombine = 16;   // split count from which the wide merge is faster
+
 int decode_splits(const ksa_params *p, int batch, int64_t max_text)
 {
     int64_t max_slice = 1 + p->k + (int64_t)p->w * p->k + max_text / p->k;
@@ -533,7 +615,10 @@ static int launch_decode_t(const DecodeArgs &a, int batch, __nv_bfloat16 *o, flo
 {
     dim3 grid(a.nsplit, a.Hkv, batch);
     decode_split_kernel<D, G><<<grid, kDecThreads, 0, st>>>(a);
-    decode_combine_kernel<D, G><<<dim3(a.Hkv, batch), 256, 0, st>>>(a, o, lse);
+    if (a.nsplit >= kDecWideCombine)
+        decode_combine_wide_kernel<D, G><<<dim3(a.Hkv, batch), 256, 0, st>>>(a, o, lse);
+    else
+        decode_combine_kernel<D, G><<<dim3(a.Hkv, batch), 256, 0, st>>>(a, o, lse);
     return cudaGetLastError() == cudaSuccess ? KSA_OK : KSA_ERR_CUDA;
 }
 

@@ -591,9 +591,17 @@ int decode_splits(const ksa_params *p, int batch, int64_t max_text)
 {
     int64_t max_slice = 1 + p->k + (int64_t)p->w * p->k + max_text / p->k;
     int64_t units = (int64_t)batch * p->num_kv_heads;
-    int64_t want = (32LL * sm_count() + units - 1) / units;  // ~8 waves of 4 CTAs per SM
-    int64_t cap = (max_slice + 511) / 512;                      // >= 512 rows per split
+    // ~8 waves of 4 CTAs per SM, at least 1024 rows per split; but at least
+    // two CTAs per SM while splits keep 512 rows or more (small batches)
+    const int64_t sms = sm_count();
+    int64_t want = (32LL * sms + units - 1) / units;
+    int64_t cap = (max_slice + 1023) / 1024;
     int64_t s = want < cap ? want : cap;
+    if (s * units < 2 * sms) {
+        const int64_t fill = (2 * sms + units - 1) / units, cap512 = (max_slice + 511) / 512;
+        const int64_t s2 = fill < cap512 ? fill : cap512;
+        if (s2 > s) s = s2;
+    }
     if (s < 1) s = 1;
     if (s > 1024) s = 1024;
     return (int)s;

@@ -935,6 +935,15 @@ __global__ void __launch_bounds__(kSumWarps * 32) summary_rows_kernel(SumArgs a)
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+
+// Longest chunk whose summary rows the epilogue warps take (k + 1 keys per
+// row, one warp per chunk).  Same box, 32K tokens, whole call: with the
+// epilogue warps at every k, k = 16 / 32 / 64 took 1.05-1.09 / 1.07-1.08 /
+// 1.61-1.62 ms; with the separate kernel above k = 8, 0.87-0.91 / 0.68-0.69
+// / 0.67 ms; k = 8 unchanged (1.273-1.275 ms).
+constexpr int kEpilogueSumMaxK = 8;
+
+// ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -1013,7 +1022,11 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
     P.lse = lse;
     P.ck_tile_off = P.ck_cbeg = P.ck_ntot = P.ck_qbase = P.ck_kvbase = nullptr;
     P.sum_slot0 = 0;
-    P.sum_rows = 1;
+    // The summary rows run on the prefill kernel's epilogue warps (one warp
+    // per chunk, between items) for chunks of up to 8 tokens; longer chunks
+    // make those rows slow enough to hold up the items' O hand-off, so they
+    // take the separate warp-MMA kernel after the prefill.
+    P.sum_rows = k <= kEpilogueSumMaxK ? 1 : 0;
     bool ok = make_map(&P.tm_q, qa, D, Hq, k, chunks, P.Gp, k, P.Tc) &&
               make_map(&P.tm_ksum, ka, D, Hkv, k, chunks, 1, 1, pf::BN) &&
               make_map(&P.tm_kwin, ka, D, Hkv, k, chunks, 1, k, P.Tk) &&
@@ -1035,7 +1048,27 @@ static int launch_prefill_t(const ksa_params *p, int batch, const int32_t *cu, i
     }
     pf::prefill_kernel<D><<<(unsigned)grid, pf::kThreads, L::kAlloc, st>>>(P);
     if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
-
+    if (!P.sum_rows) {
+        pf::SumArgs s;
+        s.k = k; s.G = G; s.Hq = Hq; s.Hkv = Hkv; s.batch = batch; s.chunks = chunks;
+        s.scale = scale; s.scale_log2 = P.scale_log2;
+        s.cu = cu; s.pl = pl; s.err = err;
+        s.q = (const __nv_bfloat16 *)qa; s.kk = (const __nv_bfloat16 *)ka; s.v = (const __nv_bfloat16 *)va;
+        s.o = (__nv_bfloat16 *)oa; s.lse = lse;
+        const int64_t tasks = chunks * Hkv;
+        if (tasks > 0) {
+            const unsigned blocks = (unsigned)((tasks + pf::kSumWarps - 1) / pf::kSumWarps);
+            const unsigned thr = pf::kSumWarps * 32;
+            switch (G) {
+            case 1: pf::summary_rows_kernel<D, 1><<<blocks, thr, 0, st>>>(s); break;
+            case 2: pf::summary_rows_kernel<D, 2><<<blocks, thr, 0, st>>>(s); break;
+            case 4: pf::summary_rows_kernel<D, 4><<<blocks, thr, 0, st>>>(s); break;
+            case 8: pf::summary_rows_kernel<D, 8><<<blocks, thr, 0, st>>>(s); break;
+            default: return KSA_ERR_UNSUPPORTED;
+            }
+            if (cudaGetLastError() != cudaSuccess) return KSA_ERR_CUDA;
+        }
+    }
     return KSA_OK;
 }
 

@@ -386,9 +386,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (j < nblk) {
                     // S(j) = Q K(j)^T over this rank's dims, into S buffer j % 2
                     const int stg = j % ST, sb = j & 1;
-                    ok = mbar_wait_sleep(bar(B_KV_FULL + stg), (uint32_t)(j / ST) & 1u, abort, err);
+                    ok = mbar_wait(bar(B_KV_FULL + stg), (uint32_t)(j / ST) & 1u, abort, err);
                     // the buffer's last reader, PV(j - 2), has completed
-                    if (ok && j >= 2) ok = mbar_wait_sleep(bar(B_O_DONE + sb), (uint32_t)((j - 2) >> 1) & 1u, abort, err);
+                    if (ok && j >= 2) ok = mbar_wait(bar(B_O_DONE + sb), (uint32_t)((j - 2) >> 1) & 1u, abort, err);
                     if (!ok) break;
                     tc_fence_after();
                     const uint64_t dk = dk0 + (uint64_t)((stg * kStage) >> 4);
@@ -412,7 +412,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     // O += P(i) V(i): P from TMEM, V = the stage's four latent
                     // chunks (N = 256 dims, MN-major)
                     const int i = j - 1, stg = i % ST, sb = i & 1;
-                    if (!(ok = mbar_wait_sleep(bar(B_P_FULL + sb), (uint32_t)(i >> 1) & 1u, abort, err))) break;
+                    if (!(ok = mbar_wait(bar(B_P_FULL + sb), (uint32_t)(i >> 1) & 1u, abort, err))) break;
                     tc_fence_after();
                     const uint64_t dv = dv0 + (uint64_t)((stg * kStage) >> 4);
 #pragma unroll

@@ -598,7 +598,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t peer_bar_s = peer_addr(bar(B_RECV_S), peer);
             for (int j = 0; j < nblk; ++j) {
                 const int sb = j & 1;
-                if (!__all_sync(FULL, mbar_wait_sleep(bar(B_S_FULL + sb), (uint32_t)(j >> 1) & 1u, abort, err))) break;
+                if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + sb), (uint32_t)(j >> 1) & 1u, abort, err))) break;
                 tc_fence_after();
                 uint32_t sp[32];
                 tmem_ld16x256_x8(tmem + taddr + kSCol + sb * NB, sp);

@@ -638,7 +638,7 @@ def run_sweep(args):
                 lse_m = torch.empty(B, H, dtype=torch.float32, device=dev)
                 ms = ev_time(lambda: L.ksa_mla_decode(pm, cache.desc, kind, q, o, lse_m, max_text, mws))
                 assert (cache.state[:, 3] == 0).all()
-                rows = float((fills + min(m, w) * k + max(0, m - w)).sum())
+                rows = float(decode_slice_rows(m, k, w, fills - 1).sum())   # fills counts the step's token
                 gbs = rows * 576 * 2 / (ms * 1e-3) / 1e9
                 tf = rows * H * (576 + 512) * 2 / (ms * 1e-3) / 1e12
                 print(json.dumps({"sweep": "mla_decode", "batch": B, "context": n, "summaries": m, "heads": H,

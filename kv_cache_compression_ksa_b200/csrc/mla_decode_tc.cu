@@ -19,8 +19,7 @@
 // softmax of half the heads belongs to each CTA (the owner: rank 0 owns TMEM
 // lanes 32 q + 0..15 of every lane quarter q, rank 1 lanes 32 q + 16..31):
 //   * each CTA sends its partial scores of the other's rows (64 x 64 fp32)
-//     to the owner through distributed shared memory, staged in its own
-//     shared memory and moved by one bulk copy per lane quarter;
+//     to the owner through distributed shared memory;
 //   * the owner adds them to its own, runs the online softmax of its rows
 //     (16-lane TMEM accesses: a thread holds two rows of 16 slots, a row's
 //     four threads reduce by shuffles), writes P (bf16) over S in its TMEM
@@ -30,9 +29,7 @@
 //     128 x 256 x 64 product with P read from TMEM.
 // Per block and direction that is 16 KB of scores and 8 KB of P instead of
 // the 32 KB of a full exchange; distributed shared memory moves about 20
-// bytes per clock per direction on this part.  Each receive buffer's
-// barrier takes one local arrival with the expected bytes, armed a phase
-// ahead, and the bulk copies' completions.
+// bytes per clock per direction on this part.
 //
 // Roles (512 threads): warp 0 issues the TMA loads, warp 1 the MMAs; warps
 // 4..7 own (lane quarter w % 4), 8..11 send the other rows' partial scores,
@@ -82,10 +79,8 @@ constexpr int kRecvPBuf = 4 * 4 * 32 * 16;
 constexpr int kAlpha = kRecvP + 2 * kRecvPBuf;       // [2][4 q][16] float: their rescale factors
 constexpr int kPStage = kAlpha + 2 * HO * 4;         // [2][4 q][4][32 t] uint4: this CTA's P, sent by bulk copy
 constexpr int kAStage = kPStage + 2 * kRecvPBuf;     // [2][4 q][16] float: its rescale factors
-constexpr int kSStage = kAStage + 2 * HO * 4;        // [4 q][8][32 t] float4: its partial scores of the other's rows
 constexpr int kPBytes = 4 * 32 * 16, kABytes = 16 * 4;   // one quarter's P and factors
-constexpr int kSBytes = 8 * 32 * 16;                  // one quarter's partial scores
-constexpr int kBar = kSStage + kRecvSBuf;
+constexpr int kBar = kAStage + 2 * HO * 4;
 // kv_full[ST], kv_empty[ST], s_full[2], p_full[2], o_done[2], recv_s[2], recv_p[2], drain
 constexpr int B_KV_FULL = 0, B_KV_EMPTY = B_KV_FULL + ST, B_S_FULL = B_KV_EMPTY + ST, B_P_FULL = B_S_FULL + 2,
               B_O_DONE = B_P_FULL + 2, B_RECV_S = B_O_DONE + 2, B_RECV_P = B_RECV_S + 2, B_DRAIN = B_RECV_P + 2,
@@ -120,9 +115,22 @@ __device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank)
     return r;
 }
 
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w)
+{
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
+
 __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t x)
 {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(x) : "memory");
+}
+
+// arrive on an mbarrier of the peer, ordering this thread's earlier
+// accesses before it at cluster scope
+__device__ __forceinline__ void arrive_cluster(uint32_t addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
 
 // bounded wait on a local mbarrier whose arrivals come from the peer
@@ -153,6 +161,11 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, ui
                  "r"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
+// Bulk async-groups batch only the copies that complete through a bulk group
+// (shared -> global); a copy into the peer's shared memory completes on the
+// peer's mbarrier instead, so these group waits do not order its reads of the
+// source.  What frees a staging buffer here is the exchange's causal chain
+// (see the owner's P staging).
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
@@ -254,10 +267,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(bar(B_S_FULL + s), 1);
             mbar_init(bar(B_P_FULL + s), 256);   // this CTA's owner and receiver warps
             mbar_init(bar(B_O_DONE + s), 1);
-            // the other CTA's partial scores and P: one local arrival with the
-            // expected bytes, armed a phase ahead, and the bulk copies' completions
-            mbar_init(bar(B_RECV_S + s), 1);
-            mbar_expect_tx(bar(B_RECV_S + s), 4 * kSBytes);
+            mbar_init(bar(B_RECV_S + s), 128);   // the other CTA's sender warps
+            // the other CTA's P: one local arrival with the expected bytes, armed
+            // a phase ahead, and the bulk copies' completions
             mbar_init(bar(B_RECV_P + s), 1);
             mbar_expect_tx(bar(B_RECV_P + s), 4 * (kPBytes + kABytes));
         }
@@ -479,9 +491,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
                 ok = __all_sync(FULL, wait_cluster(bar(B_RECV_S + sb), (uint32_t)(j >> 1) & 1u, abort, err));
                 if (!ok) break;
-                // arm buffer sb's next phase (block j + 2), whose copies start only
-                // after this block's P has reached the other CTA's product
-                if (q == 0 && lane == 0 && j + 2 < nblk) mbar_expect_tx(bar(B_RECV_S + sb), 4 * kSBytes);
                 // S = own + other partial scores, in log2 units; slots past the
                 // share's end masked
                 const int cnt = (int)min((int64_t)NB, s1 - (s0 + (int64_t)j * NB));
@@ -537,7 +546,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // half of O: staged here, then one bulk copy per quarter, so that
                 // this warp does not wait on the distributed shared memory
                 {
-                    if (lane == 0 && copies >= 2) bulk_wait_read_1();   // staging buffer sb is free again
+                    // staging buffer sb was last read by the copy of P(j - 2), which
+                    // landed in the other CTA before its PV(j - 2), and so before its
+                    // QK(j) and the scores of block j that this warp has received
+                    if (lane == 0 && copies >= 2) bulk_wait_read_1();
                     __syncwarp();
                     uint4 *ps = reinterpret_cast<uint4 *>(smem + kPStage + sb * kRecvPBuf + q * kPBytes) + lane;
 #pragma unroll
@@ -563,7 +575,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(bar(B_P_FULL + sb));
             }
-            if (lane == 0) bulk_wait_read_0();   // the staging buffers stay valid until read
+            // the last copies land before the other CTA leaves its receive loop,
+            // and so before the final cluster barrier
+            if (lane == 0) bulk_wait_read_0();
             __syncwarp();
             // ---- epilogue: this CTA's half of the rows' O and the rows' (max, sum) ----
             if (ok && nblk > 0)
@@ -590,12 +604,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         } else if (role == 1) {
             // ================= sender: the other CTA's rows' partial scores =================
-            // staged in this CTA's shared memory and sent as one bulk copy per
-            // quarter: remote stores from the four warps, each thread then
-            // releasing its own, took two to three times as long in the kernel
             const uint32_t peer_recv_s = peer_addr(sbase + kRecvS, peer);
             const uint32_t peer_bar_s = peer_addr(bar(B_RECV_S), peer);
-            uint4 *ss = reinterpret_cast<uint4 *>(smem + kSStage) + q * 256 + lane;
             for (int j = 0; j < nblk; ++j) {
                 const int sb = j & 1;
                 if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + sb), (uint32_t)(j >> 1) & 1u, abort, err))) break;
@@ -604,20 +614,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tmem_ld16x256_x8(tmem + taddr + kSCol + sb * NB, sp);
                 tmem_wait_ld();
                 tc_fence_before();   // these reads precede the P that the owner's reply brings
-                if (lane == 0 && j > 0) bulk_wait_read_0();   // the previous block's copy has read the staging
-                __syncwarp();
+                const uint32_t dst = peer_recv_s + (uint32_t)(sb * kRecvSBuf + (q * 256 + lane) * 16);
 #pragma unroll
-                for (int r = 0; r < 8; ++r) ss[32 * r] = make_uint4(sp[4 * r], sp[4 * r + 1], sp[4 * r + 2], sp[4 * r + 3]);
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // for the bulk copy's reads
-                __syncwarp();
-                if (lane == 0) {
-                    bulk_copy_to_peer(peer_recv_s + (uint32_t)(sb * kRecvSBuf + q * kSBytes),
-                                      sbase + (uint32_t)(kSStage + q * kSBytes), kSBytes, peer_bar_s + 8u * (uint32_t)sb);
-                    bulk_commit();
-                }
+                for (int r = 0; r < 8; ++r)
+                    st_cluster_v4(dst + (uint32_t)(r * 32 * 16), sp[4 * r], sp[4 * r + 1], sp[4 * r + 2], sp[4 * r + 3]);
+                arrive_cluster(peer_bar_s + 8u * (uint32_t)sb);
             }
-            if (lane == 0) bulk_wait_read_0();   // the staging buffer stays valid until read
-            __syncwarp();
         } else {
             // ================= receiver: the owner's P for the other CTA's rows =================
             bool ok = true;

@@ -386,10 +386,8 @@ def _mla_tc_roles(nblk, rescale_rng, qk_runs_ahead=False):
     buffer j % 2 once PV(j - 2) has completed, then PV(j - 1) once P(j - 1)
     is in), four owner warps (S, then the other CTA's partial scores, the
     softmax, a bulk copy of P to the other CTA, P in), four sender warps
-    (S, then a bulk copy of the other CTA's rows to it) and four receiver
-    warps (the other CTA's P, P in).  Each receive buffer's barrier takes one
-    local arrival (armed a phase ahead) and the four copies; the buffers have
-    no acknowledgement;
+    (S, then a push of the other CTA's rows to it) and four receiver warps
+    (the other CTA's P, P in).  The receive buffers have no acknowledgement;
     "expect" checks that each is refilled only after its previous contents
     were read, and that P is written over S only after S was read."""
     ST = 3
@@ -398,12 +396,11 @@ def _mla_tc_roles(nblk, rescale_rng, qk_runs_ahead=False):
         for i in range(ST):
             bars.update({f"{r}KF{i}": 1, f"{r}KE{i}": 1})
         for i in range(2):
-            bars.update({f"{r}S{i}": 1, f"{r}PF{i}": 8, f"{r}O{i}": 1, f"{r}RS{i}": 1 + 4, f"{r}RP{i}": 1 + 4})
+            bars.update({f"{r}S{i}": 1, f"{r}PF{i}": 8, f"{r}O{i}": 1, f"{r}RS{i}": 4, f"{r}RP{i}": 1 + 4})
 
     def init(r):
         for i in range(2):
-            yield ("arrive", f"{r}RS{i}")            # the receive buffers' first phases armed
-            yield ("arrive", f"{r}RP{i}")
+            yield ("arrive", f"{r}RP{i}")            # the receive buffers' first phases armed
 
     def tma(r):
         for j in range(nblk):
@@ -435,8 +432,6 @@ def _mla_tc_roles(nblk, rescale_rng, qk_runs_ahead=False):
             yield ("wait", f"{r}S{sb}", j >> 1)
             yield ("mark", f"{r}Sread{sb}")
             yield ("wait", f"{r}RS{sb}", j >> 1)
-            if q == 0 and j + 2 < nblk:
-                yield ("arrive", f"{r}RS{sb}")                 # one thread arms buffer sb's next phase
             yield ("mark", f"{r}RSread{sb}")
             if j > 0 and rescale_rng.random() < 0.3:
                 yield ("wait", f"{r}O{sb ^ 1}", (j - 1) >> 1)
@@ -454,7 +449,7 @@ def _mla_tc_roles(nblk, rescale_rng, qk_runs_ahead=False):
             yield ("mark", f"{r}Sread{sb}")
             yield ("mark", f"{r}Ssent{q}")
             yield ("expect", f"{o}RSread{sb}", 4 * (j >> 1))   # the other CTA read S(j - 2) from buffer sb
-            yield ("load", f"{o}RS{sb}")                         # bulk copy of this quarter's scores
+            yield ("arrive", f"{o}RS{sb}")
 
     def receiver(r, q):
         for j in range(nblk):

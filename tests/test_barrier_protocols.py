@@ -36,7 +36,8 @@ class _Bar:
 
 def _simulate(bars, roles, seed, max_rounds=400000):
     """roles: name -> generator yielding ("wait", bar, phase), ("arrive", bar),
-    ("load", bar) (a TMA load or bulk copy completing later on bar),
+    ("load", bar[, key]) (a TMA load or bulk copy completing later on bar;
+    with a key, its completion also marks a read of its source buffer),
     ("mma", issuer) / ("commit", issuer, bar), or ("mark", key) / ("expect",
     key, n) (a buffer read finished / a write that needs n reads done before
     it: a shortfall is reported with the aliasing events).  Returns (status,
@@ -63,7 +64,10 @@ def _simulate(bars, roles, seed, max_rounds=400000):
         for c in order:
             if c == "loads":
                 if loads and rng.random() < 0.5:
-                    B[loads.pop(0)].arrive()
+                    name, key = loads.pop(0)
+                    B[name].arrive()
+                    if key is not None:
+                        marks[key] = marks.get(key, 0) + 1
                     progressed = True
             elif c.startswith("mma:"):
                 q = mma[c[4:]]
@@ -87,7 +91,7 @@ def _simulate(bars, roles, seed, max_rounds=400000):
                     elif a[0] == "arrive":
                         B[a[1]].arrive()
                     elif a[0] == "load":
-                        loads.append(a[1])
+                        loads.append((a[1], a[2] if len(a) > 2 else None))
                     elif a[0] == "mma":
                         mma.setdefault(a[1], []).append(None)
                     elif a[0] == "commit":
@@ -380,7 +384,7 @@ def test_engine_catches_a_parity_aliasing_bug():
 
 
 # ---------------------------------------------------------------- mla_decode_tc_kernel
-def _mla_tc_roles(nblk, rescale_rng, qk_runs_ahead=False):
+def _mla_tc_roles(nblk, rescale_rng, qk_runs_ahead=False, single_p_staging=False):
     """Both CTAs of a pair (ranks 0, 1), warps as roles; barrier names carry
     the rank.  Per CTA: TMA (three K/V stages), the MMA issuer (QK(j) into S
     buffer j % 2 once PV(j - 2) has completed, then PV(j - 1) once P(j - 1)
@@ -389,7 +393,10 @@ def _mla_tc_roles(nblk, rescale_rng, qk_runs_ahead=False):
     (S, then a push of the other CTA's rows to it) and four receiver warps
     (the other CTA's P, P in).  The receive buffers have no acknowledgement;
     "expect" checks that each is refilled only after its previous contents
-    were read, and that P is written over S only after S was read."""
+    were read, that P is written over S only after S was read, and that an
+    owner refills its P staging buffer only after the copy that last read
+    it has completed (the copy completes on the other CTA's barrier; no
+    bulk-group wait covers it, only the exchange's causal chain)."""
     ST = 3
     bars = {}
     for r in range(2):
@@ -436,7 +443,9 @@ def _mla_tc_roles(nblk, rescale_rng, qk_runs_ahead=False):
             if j > 0 and rescale_rng.random() < 0.3:
                 yield ("wait", f"{r}O{sb ^ 1}", (j - 1) >> 1)
             yield ("expect", f"{o}RPread{sb}", 4 * (j >> 1))   # the other CTA read P(j - 2) from buffer sb
-            yield ("load", f"{o}RP{sb}")                         # bulk copy of P and the factors
+            ps = 0 if single_p_staging else sb
+            yield ("expect", f"{r}PSread{ps}{q}", j if single_p_staging else j >> 1)   # staging free
+            yield ("load", f"{o}RP{sb}", f"{r}PSread{ps}{q}")     # bulk copy of P and the factors
             yield ("arrive", f"{r}PF{sb}")
         if nblk > 0:
             yield ("wait", f"{r}O{(nblk - 1) & 1}", (nblk - 1) >> 1)
@@ -501,6 +510,18 @@ def test_mla_tc_kernel_pair_protocol():
             bars, roles = _mla_tc_roles(nblk, random.Random(seed + 77))
             status, stuck, aliasing = _simulate(bars, roles, seed)
             assert status == "ok" and not aliasing, (nblk, seed, status, stuck, aliasing)
+
+
+def test_mla_tc_model_catches_a_single_p_staging_buffer():
+    """With one P staging buffer per owner warp instead of two, block j's
+    stores could overwrite P(j - 1) while its copy to the other CTA still
+    reads it: nothing in the exchange orders the two."""
+    flagged = 0
+    for seed in range(30):
+        bars, roles = _mla_tc_roles(8, random.Random(seed), single_p_staging=True)
+        status, _, aliasing = _simulate(bars, roles, seed)
+        flagged += status != "ok" or bool(aliasing)
+    assert flagged > 0
 
 
 def test_mla_tc_model_catches_a_missing_buffer_wait():

@@ -182,6 +182,23 @@ def test_noalloc_decode_checks_arguments_like_decode(lib):
         assert rc_ws == want and rc_na == want, (p.k, p.w, p.head_dim, cache.batch, rc_ws, rc_na)
 
 
+def test_noalloc_decode_refuses_a_batch_whose_split_does_not_fit(lib):
+    """One split of the partials takes 4 B x batch x Hq x (d + 2); above the
+    fixed 4 MiB array (253 sequences x 32 q heads at d 128: 4,209,920 B)
+    the no-workspace call refuses with KSA_ERR_CAPACITY, and ksa_decode
+    with a workspace too small for it with KSA_ERR_WORKSPACE, both before
+    any launch or device access."""
+    from kv_cache_compression_ksa_b200 import _lib as L
+    nul = ctypes.c_void_p(0)
+    p = L.make_params(8, 8, 32, 8, 128)
+    cache = L.ksa_cache(16, 16, 16, 253, 4)
+    assert 4 * 253 * 32 * (128 + 2) > 4 << 20
+    assert lib.ksa_decode_noalloc(ctypes.byref(p), ctypes.byref(cache), 16, 16, 16, nul, 100, nul) == \
+        L.KSA_ERR_CAPACITY
+    assert lib.ksa_decode(ctypes.byref(p), ctypes.byref(cache), 16, 16, 16, nul, 100, 16, 1 << 20, nul) == \
+        L.KSA_ERR_WORKSPACE
+
+
 def test_selftest_wait_timeout_arguments(lib):
     """The timeout self-check launches one CTA whose waits are bounded by the
     given limits; limits outside (0, the pipelines' own limit] and a missing
